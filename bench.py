@@ -1,0 +1,463 @@
+"""Benchmark of the BitLinear training hot path (fwd + bwd) on B200.
+
+One step = one pass of the whole hot path over one batch:
+  S1 bl_quantize_weight (2 launches) -> S2 bl_quantize_act -> S3 bl_forward
+  -> S4 bl_backward dX -> S4 bl_backward dW                    (6 launches)
+
+Default workload: the up-projection BitLinear 2560 -> 6912 at 8 x 512 tokens
+(M=4096, K=2560, N=6912; x, dY bf16 ~ N(0,1), W bf16 kaiming-uniform).
+Metric: effective TOPS = 6 M N K / step time (plus ms per step and the
+roofline fraction of the dominant kernel).
+
+Timing: W >= 3 untimed warm-up steps, then exactly K timed steps on
+resident inputs. L2 is flushed (256 MiB write) before every step, outside
+the timed events; each step is bracketed by CUDA events on the launching
+stream, with events between the C-ABI calls for per-kernel times. For N > 1
+(torchrun, one rank per GPU) every rank runs its own batch (weak scaling, no
+data-path collective); the job time is the max over ranks.
+
+`--impl reference` times the CPU oracle (the only reference this path has)
+on a bounded sample of the same workload, on the host cores.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from workloads import WORKLOADS, workload_inputs  # noqa: E402
+
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+INT8_OVER_BF16 = 2.0  # nominal dense ratio (4.5 / 2.25 PFLOP/s)
+KERNEL_SOURCES = ["ternary_weight_quantization_b200/csrc/k_quant.cu",
+                  "ternary_weight_quantization_b200/csrc/k_gemm.cu",
+                  "ternary_weight_quantization_b200/csrc/bl_device.cuh"]
+
+
+def load_peaks():
+    try:
+        with open(PEAKS_FILE) as f:
+            p = json.load(f)
+        return {k: float(p[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash():
+    import hashlib
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def load_traffic(workload):
+    """Per-launch DRAM bytes from a committed ncu capture, if it matches the
+    current kernel sources (else None)."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            t = json.load(f)
+    except Exception:
+        return {}
+    if t.get("source_hash") != kernel_source_hash():
+        return {}
+    return t.get("workloads", {}).get(workload, {})
+
+
+# ----------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons with NVML in a background thread."""
+
+    BAD = {"hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown"}
+
+    def __init__(self, device_index, period_s=0.005):
+        self.samples = []
+        self.reasons = set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._t = None
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.period = period_s
+            self.ok = True
+        except Exception:
+            self.ok = False
+
+    def _reason_names(self, mask):
+        nv = self.nv
+        table = {
+            "sw_power_cap": getattr(nv, "nvmlClocksEventReasonSwPowerCap", 0x4),
+            "hw_slowdown": getattr(nv, "nvmlClocksEventReasonHwSlowdown", 0x8),
+            "sw_thermal_slowdown": getattr(nv, "nvmlClocksEventReasonSwThermalSlowdown", 0x20),
+            "hw_thermal_slowdown": getattr(nv, "nvmlClocksEventReasonHwThermalSlowdown", 0x40),
+            "hw_power_brake_slowdown": getattr(nv, "nvmlClocksEventReasonHwPowerBrakeSlowdown", 0x80),
+        }
+        return {k for k, v in table.items() if mask & v}
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                try:
+                    mask = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                except Exception:
+                    mask = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+                self.reasons |= self._reason_names(mask)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        if self.ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+
+    def stop(self):
+        if self._t:
+            self._stop.set()
+            self._t.join()
+        s = sorted(self.samples)
+        med = s[len(s) // 2] if s else None
+        return {"sm_mhz": med, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(s), "source": "nvml" if self.ok else "unavailable"}
+
+    def rejected(self, rec):
+        return bool(self.BAD & set(rec["reasons"]))
+
+
+# ----------------------------------------------------------------- our arm
+
+STAGES = ["quantize_weight", "quantize_act", "forward", "backward_dx", "backward_dw"]
+LAUNCHES_PER_STEP = 6
+
+
+def stage_work(M, N, K, w_bytes):
+    """Algorithmic work per launch group: bytes for the HBM passes, ops for GEMMs."""
+    return {
+        "quantize_weight": {"bound": "hbm", "bytes": N * K * w_bytes + N * K // 4 + 4},
+        "quantize_act": {"bound": "hbm", "bytes": M * K * 2 + M * K + 4 * M},
+        "forward": {"bound": "tensor", "ops": 2 * M * N * K, "dtype": "int8"},
+        "backward_dx": {"bound": "tensor", "ops": 2 * M * N * K, "dtype": "bf16"},
+        "backward_dw": {"bound": "tensor", "ops": 2 * M * N * K, "dtype": "bf16"},
+    }
+
+
+def run_ours(args, rank, world, local_rank):
+    import ternary_weight_quantization_b200 as bl
+
+    bl.load_library()
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    wl = WORKLOADS[args.workload]
+    M, K, N = wl.M, wl.K, wl.N
+    x_cpu, w_cpu, dy_cpu = workload_inputs(args.workload, seed=rank)
+    x, w, dy = x_cpu.to(dev), w_cpu.to(dev), dy_cpu.to(dev)
+    bufs = bl.StepBuffers.allocate(M, N, K, torch.bfloat16, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(evs=None):
+        if evs:
+            evs[0].record(stream)
+        bl.bl_quantize_weight(w, bufs.w_packed, bufs.gamma, bufs.workspace, stream)
+        if evs:
+            evs[1].record(stream)
+        bl.bl_quantize_act(x, bufs.xq, bufs.sx, stream)
+        if evs:
+            evs[2].record(stream)
+        bl.bl_forward(bufs.xq, bufs.sx, bufs.w_packed, bufs.gamma, bufs.y, None, stream)
+        if evs:
+            evs[3].record(stream)
+        bl.bl_backward(dy, bufs.xq, bufs.sx, bufs.w_packed, bufs.gamma, bufs.dX, None, False, stream)
+        if evs:
+            evs[4].record(stream)
+        bl.bl_backward(dy, bufs.xq, bufs.sx, bufs.w_packed, bufs.gamma, None, bufs.dW, False, stream)
+        if evs:
+            evs[5].record(stream)
+
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        step()
+    torch.cuda.synchronize(dev)
+    if bl.bl_get_last_error() != 0:
+        raise RuntimeError("device error during warm-up")
+
+    def timed():
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize(dev)
+        for i in range(args.steps):
+            flush.fill_(i & 0xFF)
+            step(evs[i])
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            torch.distributed.barrier()
+        per_stage = {s: 0.0 for s in STAGES}
+        total = 0.0
+        for e in evs:
+            for j, s in enumerate(STAGES):
+                per_stage[s] += e[j].elapsed_time(e[j + 1])
+            total += e[0].elapsed_time(e[5])
+        return total, per_stage
+
+    sampler = ClockSampler(dev.index if dev.index is not None else 0)
+    sampler.start()
+    total_ms, per_stage = timed()
+    clocks = sampler.stop()
+    remeasured = False
+    if sampler.rejected(clocks):
+        sampler = ClockSampler(dev.index if dev.index is not None else 0)
+        sampler.start()
+        total_ms, per_stage = timed()
+        clocks = sampler.stop()
+        remeasured = True
+    clocks["remeasured"] = remeasured
+    if bl.bl_get_last_error() != 0:
+        raise RuntimeError("device error during the timed region")
+
+    # max over ranks of the device time
+    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    job_ms = float(t.item())
+
+    e2e = measure_e2e(bl, args, dev, stream, bufs, x_cpu, w_cpu, dy_cpu, world)
+    if rank != 0:
+        return None
+
+    ops_step = 6.0 * M * N * K
+    ms_per_step = job_ms / args.steps
+    value = ops_step * world * args.steps / (job_ms * 1e-3) / 1e12
+    peaks, peak_src = load_peaks()
+    work = stage_work(M, N, K, 2 if wl.w_dtype == torch.bfloat16 else 4)
+    traffic = load_traffic(args.workload)
+    kernels = {}
+    roof_ms = 0.0
+    for s in STAGES:
+        ms = per_stage[s] / args.steps
+        wk = work[s]
+        if wk["bound"] == "hbm":
+            ach = wk["bytes"] / (ms * 1e-3) / 1e9
+            peak = peaks["hbm_gbs"]
+            unit = "GB/s"
+            roof_ms += wk["bytes"] / (peak * 1e9) * 1e3
+        else:
+            ach = wk["ops"] / (ms * 1e-3) / 1e12
+            peak = peaks["bf16_tflops"] * (INT8_OVER_BF16 if wk["dtype"] == "int8" else 1.0)
+            unit = "TOPS" if wk["dtype"] == "int8" else "TFLOP/s"
+            roof_ms += wk["ops"] / (peak * 1e12) * 1e3
+        kernels[s] = {"ms": round(ms, 5), "achieved": round(ach, 1), "unit": unit, "peak": peak,
+                      "frac": round(ach / peak, 4), "share": round(per_stage[s] / sum(per_stage.values()), 4),
+                      "traffic": traffic.get(s)}
+    dom = max(STAGES, key=lambda s: per_stage[s])
+    dk = kernels[dom]
+    roofline = {"kernel": dom, "bound": work[dom]["bound"], "achieved": dk["achieved"], "peak": dk["peak"],
+                "unit": "GB/s" if work[dom]["bound"] == "hbm" else "TFLOP/s", "frac": dk["frac"],
+                "traffic": dk["traffic"], "peak_source": f"{peak_src} (burst bf16"
+                + (" x2 nominal int8/bf16 ratio" if work[dom].get("dtype") == "int8" else "") + ")"
+                if work[dom]["bound"] == "tensor" else f"{peak_src} hbm copy"}
+    out = {
+        "metric": "bitlinear_fwd_bwd_effective_tops", "value": round(value, 2), "unit": "TOPS",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8/bf16",
+        "data": "synthetic",
+        "config": {"workload": args.workload, "M": M, "K": K, "N": N,
+                   "x": f"bf16 [{M},{K}] N(0,1)" + (" + 1% x20 outliers" if wl.outliers else ""),
+                   "W": f"{'bf16' if wl.w_dtype == torch.bfloat16 else 'f32'} [{N},{K}] {wl.w_init}",
+                   "dY": f"bf16 [{M},{N}] N(0,1)", "global_batch_tokens": M * world,
+                   "l2": "flushed before every step (256 MiB write, outside the timed events)",
+                   "parallelism": f"dp{world} independent replicas" if world > 1 else "single GPU"},
+        "roofline": roofline,
+        "step_roofline_frac": round(roof_ms / ms_per_step, 4),
+        "kernels": kernels,
+        "e2e": e2e,
+        "gpu_launches": LAUNCHES_PER_STEP * args.steps,
+        "clocks": clocks,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(args.workload, budget_tokens=args.cpu_tokens)
+    return out
+
+
+def measure_e2e(bl, args, dev, stream, bufs, x_cpu, w_cpu, dy_cpu, world):
+    """Same metric through the C ABI with host buffers: pinned H2D of the
+    step's inputs, the six launches, D2H of y, dX and dW, all timed."""
+    xh, wh, dyh = x_cpu.pin_memory(), w_cpu.pin_memory(), dy_cpu.pin_memory()
+    yh = torch.empty(bufs.y.shape, dtype=bufs.y.dtype).pin_memory()
+    dxh = torch.empty(bufs.dX.shape, dtype=bufs.dX.dtype).pin_memory()
+    dwh = torch.empty(bufs.dW.shape, dtype=bufs.dW.dtype).pin_memory()
+    x = torch.empty_like(x_cpu, device=dev)
+    w = torch.empty_like(w_cpu, device=dev)
+    dy = torch.empty_like(dy_cpu, device=dev)
+    steps = max(3, min(args.steps, 20))
+
+    def one():
+        x.copy_(xh, non_blocking=True)
+        w.copy_(wh, non_blocking=True)
+        dy.copy_(dyh, non_blocking=True)
+        bl.bitlinear_step(x, w, dy, bufs, stream)
+        yh.copy_(bufs.y, non_blocking=True)
+        dxh.copy_(bufs.dX, non_blocking=True)
+        dwh.copy_(bufs.dW, non_blocking=True)
+
+    for _ in range(2):
+        one()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record(stream)
+    for _ in range(steps):
+        one()
+    e.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = s.elapsed_time(e)
+    t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    M, K = x_cpu.shape
+    N = w_cpu.shape[0]
+    ops = 6.0 * M * N * K * world * steps
+    h2d = sum(tt.numel() * tt.element_size() for tt in (xh, wh, dyh))
+    d2h = sum(tt.numel() * tt.element_size() for tt in (yh, dxh, dwh))
+    return {"value": round(ops / (float(t.item()) * 1e-3) / 1e12, 3), "unit": "TOPS",
+            "ms_per_step": round(float(t.item()) / steps, 4), "steps": steps,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+
+# ----------------------------------------------------------------- oracle (CPU)
+
+def _blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        n = [i.get("num_threads", 0) for i in info if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return 1
+
+
+_INPUT_CACHE = {}
+
+
+def oracle_sample(workload, m_tokens, n_rows):
+    """Run the oracle's fwd+bwd on the first m_tokens tokens and n_rows output
+    features of the workload (full K). Returns (seconds, ops)."""
+    import numpy as np
+    from oracle import bitlinear_ref as ref
+
+    if workload not in _INPUT_CACHE:
+        _INPUT_CACHE[workload] = workload_inputs(workload)
+    x, w, dy = _INPUT_CACHE[workload]
+    x = x[:m_tokens]
+    w = w[:n_rows]
+    dy = dy[:m_tokens, :n_rows].contiguous()
+
+    def b(t):
+        return t.contiguous().view(torch.int16).numpy().view(np.uint16)
+
+    w_is_bf16 = w.dtype == torch.bfloat16
+    t0 = time.perf_counter()
+    ref.bitlinear_step(b(x), b(w) if w_is_bf16 else w.numpy(), b(dy), w_is_bf16)
+    dt = time.perf_counter() - t0
+    return dt, 6.0 * x.shape[0] * w.shape[0] * x.shape[1]
+
+
+def cpu_baseline(workload, budget_tokens=512):
+    wl = WORKLOADS[workload]
+    m = min(budget_tokens, wl.M)
+    dt, ops = oracle_sample(workload, m, wl.N)
+    return {"value": round(ops / dt / 1e12, 6), "unit": "TOPS", "cores": _blas_threads(), "kind": "oracle",
+            "seconds": round(dt, 3),
+            "sample": f"first {m} of {wl.M} tokens, all {wl.N} output features, K={wl.K} "
+                      f"(S1 on the full weight); TOPS = 6*{m}*{wl.N}*{wl.K} / time"}
+
+
+def run_reference(args):
+    wl = WORKLOADS[args.workload]
+    m, n = min(64, wl.M), min(512, wl.N)
+    for _ in range(args.warmup):
+        oracle_sample(args.workload, m, n)
+    total = 0.0
+    ops = 0.0
+    for _ in range(args.steps):
+        dt, o = oracle_sample(args.workload, m, n)
+        total += dt
+        ops += o
+    value = ops / total / 1e12
+    sample = f"first {m} of {wl.M} tokens and first {n} of {wl.N} output features, K={wl.K}, per step"
+    return {
+        "impl": "reference", "metric": "bitlinear_fwd_bwd_effective_tops", "value": round(value, 6), "unit": "TOPS",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(total / args.steps * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": args.workload, "M": wl.M, "K": wl.K, "N": wl.N},
+        "cpu_baseline": {"value": round(value, 6), "unit": "TOPS", "cores": _blas_threads(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 6), "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+# ----------------------------------------------------------------- main
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=["up_proj", "down_proj", "tiny"], default="up_proj")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-tokens", type=int, default=512)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local_rank))
+    try:
+        out = run_ours(args, rank, world, local_rank)
+        if rank == 0 and out is not None:
+            print(json.dumps(out), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

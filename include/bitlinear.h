@@ -1,0 +1,179 @@
+/*
+ * bitlinear.h -- C ABI of the B200 (sm_100a) BitNet b1.58 BitLinear training
+ * hot path: absmean ternarisation with 2-bit packing, per-token absmax INT8
+ * activation quantisation, the INT32-exact forward GEMM and the
+ * straight-through backward GEMMs.
+ *
+ * Sources, cited by page title and section:
+ *   "bitnet-qat-train" (kernel card): intro bullets (fused ternarise + scale +
+ *       pack pass, INT8 tensor-core forward, saved 2-bit/INT8 state),
+ *       Semantics, Requirements (K divisible by 32, bf16 activations, bf16 or
+ *       f32 master weights), Usage (export of packed weights and scale).
+ *   "1BitTraining.md": quantisation helpers (activation_quant, weight_quant).
+ *   "bitlinear.py": ternary_quantize, activation_quant_int8, BitLinear.forward.
+ *
+ * Conventions shared by every entry point
+ *   - Every tensor argument is a DEVICE pointer unless its name starts with
+ *     host_. The caller allocates and owns every buffer; the library never
+ *     allocates device memory and keeps no state except one error word per
+ *     device.
+ *   - Tensors are dense, row-major, and 16-byte aligned at their base.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream). All work is enqueued asynchronously on it; nothing here
+ *     synchronises the host except bl_export_weights and bl_get_last_error.
+ *   - Argument errors are detected on the host before anything is enqueued
+ *     and returned as a bl_status; bl_last_error_message() then holds a
+ *     one-line description (thread-local).
+ *   - Device-side failures (a pipeline wait that exceeded its time bound) are
+ *     recorded in the device error word and reported by bl_get_last_error.
+ *     No kernel traps or asserts.
+ *   - Shapes: M = tokens, K = in_features, N = out_features.
+ *     x [M,K] bf16, W [N,K] bf16|f32, dY [M,N] bf16.
+ *   - Requires an sm_100 device (B200).
+ *
+ * Saved state between forward and backward ("bitnet-qat-train", third intro
+ * bullet): (xq, sx, w_packed, gamma). The caller keeps it.
+ */
+#ifndef BITLINEAR_H_
+#define BITLINEAR_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum bl_status {
+    BL_OK = 0,
+    BL_ERR_INVALID_ARG = 1,        /* null pointer or negative size */
+    BL_ERR_UNSUPPORTED_SHAPE = 2,  /* K % 32 != 0, K < 32, or N % 8 != 0 in backward */
+    BL_ERR_DTYPE = 3,              /* unknown bl_dtype */
+    BL_ERR_ALIGNMENT = 4,          /* a tensor base is not 16-byte aligned */
+    BL_ERR_ARCH = 5,               /* current device is not sm_100 */
+    BL_ERR_CUDA = 6,               /* a CUDA runtime/driver call failed */
+    BL_ERR_TIMEOUT = 7,            /* a device pipeline wait exceeded its bound */
+    BL_ERR_WORKSPACE = 8           /* workspace missing or too small */
+} bl_status;
+
+typedef enum bl_dtype {
+    BL_BF16 = 0,
+    BL_F32 = 1
+} bl_dtype;
+
+/* Library version, (major << 16) | minor. */
+int bl_version(void);
+
+/* Human-readable name of a status code (static string). */
+const char* bl_status_string(bl_status status);
+
+/* Description of the last host-side failure on the calling thread. */
+const char* bl_last_error_message(void);
+
+/*
+ * Bytes of device workspace bl_quantize_weight needs for an [N,K] tensor
+ * (fp64 partial sums of |W|). Returns 0 for an empty tensor.
+ */
+size_t bl_quantize_weight_workspace_size(int64_t N, int64_t K);
+
+/*
+ * S1 -- absmean ternarisation + 2-bit packing ("1BitTraining.md",
+ * weight_quant; "bitlinear.py", ternary_quantize; "bitnet-qat-train", first
+ * intro bullet: one fused ternarise + scale + pack pass, no bf16 fake-quant
+ * tensor).
+ *
+ *   gamma   = max(fp32(sum|W| / (N*K)), 1e-5)   sum in fp64, fixed order
+ *   code    = clamp(rint_half_even(fp32(W / gamma)), -1, 1)
+ *   packing : element k of row n -> byte n*K/4 + k/4, bits 2*(k%4)..+1,
+ *             field 00 = 0, 01 = +1, 11 = -1 (10 never written)
+ *
+ * W         [N,K] master weights, w_dtype = BL_BF16 or BL_F32 (read only)
+ * w_packed  [N,K/4] uint8 output
+ * gamma     one float output (device); the dequantisation multiplier
+ * workspace device scratch of at least bl_quantize_weight_workspace_size(N,K)
+ *           bytes, 16-byte aligned; contents need no initialisation and are
+ *           overwritten.
+ * Deterministic: the same W gives bit-identical outputs on every call.
+ * Errors: BL_ERR_INVALID_ARG, BL_ERR_UNSUPPORTED_SHAPE (K % 32), BL_ERR_DTYPE,
+ *         BL_ERR_ALIGNMENT, BL_ERR_WORKSPACE, BL_ERR_ARCH, BL_ERR_CUDA.
+ */
+bl_status bl_quantize_weight(const void* W, bl_dtype w_dtype, int64_t N, int64_t K,
+                             uint8_t* w_packed, float* gamma,
+                             void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * S2 -- per-token absmax INT8 quantisation ("1BitTraining.md",
+ * activation_quant; "bitlinear.py", activation_quant_int8).
+ *
+ *   a     = max(max_k |x[m,k]|, 1e-5)
+ *   xq    = clamp(rint_half_even(fp32(x * fp32(127 / a))), -127, 127)
+ *   sx[m] = fp32(a / 127)                (x_hat = xq * sx)
+ *
+ * x  [M,K] bf16 (finite values), xq [M,K] int8 output, sx [M] float output.
+ * M == 0 is a no-op. Errors: as bl_quantize_weight (no workspace).
+ */
+bl_status bl_quantize_act(const void* x, int64_t M, int64_t K,
+                          int8_t* xq, float* sx, void* stream);
+
+/*
+ * S3 -- forward ("bitnet-qat-train", Semantics):
+ *
+ *   acc[m,n] = sum_k xq[m,k] * code[n,k]            exact INT32 (tensor cores)
+ *   y[m,n]   = bf16_rn(fp32(acc) * fp32(sx[m] * gamma))
+ *
+ * xq [M,K] int8, sx [M] float, w_packed [N,K/4] uint8, gamma one float.
+ * y [M,N] bf16 output. debug_acc: NULL, or an [M,N] int32 output that
+ * receives acc (parity checking).
+ * Errors: BL_ERR_INVALID_ARG, BL_ERR_UNSUPPORTED_SHAPE (K % 32), BL_ERR_ALIGNMENT,
+ *         BL_ERR_ARCH, BL_ERR_CUDA; device timeouts via bl_get_last_error.
+ */
+bl_status bl_forward(const int8_t* xq, const float* sx, const uint8_t* w_packed,
+                     const float* gamma, int64_t M, int64_t N, int64_t K,
+                     void* y, int32_t* debug_acc, void* stream);
+
+/*
+ * S4 -- straight-through backward ("bitnet-qat-train", Semantics; the
+ * quantisers' Jacobian is taken as 1 and gamma as constant):
+ *
+ *   dX[m,k] = bf16_rn(gamma * sum_n dY[m,n] * code[n,k])          fp32 accumulate
+ *   dW[n,k] = round(sum_m dY[m,n] * x_hat[m,k] (+ dW[n,k] if accumulate_dW))
+ *   x_hat[m,k] = bf16_rn(fp32(xq[m,k]) * sx[m])
+ *
+ * Both operands are rebuilt in shared memory from the saved 2-bit / INT8
+ * state; no bf16 copy of W_hat or x_hat is written to device memory.
+ * dY [M,N] bf16. dX [M,K] bf16 output or NULL (skipped). dW [N,K] output or
+ * NULL (skipped), of dw_dtype (BL_BF16 or BL_F32); accumulate_dW != 0 adds to
+ * the existing contents instead of overwriting them.
+ * Requires N % 8 == 0 (dY rows must be 16-byte multiples for the TMA loads).
+ * Errors: as bl_forward, plus BL_ERR_DTYPE.
+ */
+bl_status bl_backward(const void* dY, const int8_t* xq, const float* sx,
+                      const uint8_t* w_packed, const float* gamma,
+                      int64_t M, int64_t N, int64_t K,
+                      void* dX, void* dW, bl_dtype dw_dtype, int accumulate_dW,
+                      void* stream);
+
+/*
+ * Export of the packed weights and their scale for inference
+ * ("bitnet-qat-train", Usage: export_inference returns w_packed, scale_wt).
+ * Copies w_packed [N,K/4] and gamma (scale_wt = gamma, the dequantisation
+ * multiplier) into HOST buffers and synchronises `stream`.
+ */
+bl_status bl_export_weights(const uint8_t* w_packed, const float* gamma,
+                            int64_t N, int64_t K,
+                            uint8_t* host_packed, float* host_gamma, void* stream);
+
+/*
+ * Synchronises the current device, then returns BL_OK or the first device
+ * failure recorded since the last bl_reset_error (BL_ERR_TIMEOUT).
+ */
+bl_status bl_get_last_error(void);
+
+/* Clears the current device's error word (synchronous). */
+bl_status bl_reset_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BITLINEAR_H_ */

@@ -1,0 +1,222 @@
+"""Thin Python binding of libbitlinear.so (argument marshalling only).
+
+Each function has the name of the C entry point it calls, takes torch CUDA
+tensors, checks dtype / shape / contiguity, passes raw device pointers and
+the current CUDA stream, and raises :class:`BitLinearError` on any status
+other than BL_OK. Every step of the computation runs in the library's CUDA
+kernels; there is no CPU or PyTorch fallback, and importing the library fails
+loudly when the shared object is missing.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libbitlinear.so")
+
+BL_BF16 = 0
+BL_F32 = 1
+
+STATUS = {
+    0: "BL_OK", 1: "BL_ERR_INVALID_ARG", 2: "BL_ERR_UNSUPPORTED_SHAPE", 3: "BL_ERR_DTYPE",
+    4: "BL_ERR_ALIGNMENT", 5: "BL_ERR_ARCH", 6: "BL_ERR_CUDA", 7: "BL_ERR_TIMEOUT", 8: "BL_ERR_WORKSPACE",
+}
+
+# (name, restype, argtypes) of every symbol include/bitlinear.h declares
+_VP, _I64, _I32, _SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
+SIGNATURES = {
+    "bl_version": (_I32, []),
+    "bl_status_string": (ctypes.c_char_p, [_I32]),
+    "bl_last_error_message": (ctypes.c_char_p, []),
+    "bl_quantize_weight_workspace_size": (_SZ, [_I64, _I64]),
+    "bl_quantize_weight": (_I32, [_VP, _I32, _I64, _I64, _VP, _VP, _VP, _SZ, _VP]),
+    "bl_quantize_act": (_I32, [_VP, _I64, _I64, _VP, _VP, _VP]),
+    "bl_forward": (_I32, [_VP, _VP, _VP, _VP, _I64, _I64, _I64, _VP, _VP, _VP]),
+    "bl_backward": (_I32, [_VP, _VP, _VP, _VP, _VP, _I64, _I64, _I64, _VP, _VP, _I32, _I32, _VP]),
+    "bl_export_weights": (_I32, [_VP, _VP, _I64, _I64, _VP, _VP, _VP]),
+    "bl_get_last_error": (_I32, []),
+    "bl_reset_error": (_I32, []),
+}
+
+
+class BitLinearError(RuntimeError):
+    def __init__(self, status: int, where: str, detail: str):
+        super().__init__(f"{where}: {STATUS.get(status, status)}: {detail}")
+        self.status = status
+
+
+_LIB = None
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libbitlinear.so and declare its C signatures (raises if absent)."""
+    global _LIB
+    if _LIB is not None:
+        return _LIB
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is missing: build it with `python -m ternary_weight_quantization_b200.build`")
+    lib = ctypes.CDLL(path)
+    for name, (res, args) in SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    _LIB = lib
+    return lib
+
+
+def _check(status: int, where: str):
+    if status != 0:
+        lib = load_library()
+        detail = lib.bl_last_error_message().decode(errors="replace")
+        raise BitLinearError(status, where, detail)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _need(t, dtype, shape, name):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+# ----------------------------------------------------------------- entry points
+
+def bl_version() -> int:
+    return load_library().bl_version()
+
+
+def bl_quantize_weight_workspace_size(N: int, K: int) -> int:
+    return load_library().bl_quantize_weight_workspace_size(N, K)
+
+
+def bl_quantize_weight(W, w_packed, gamma, workspace, stream=None):
+    """S1: W [N,K] bf16|f32 -> w_packed [N,K/4] uint8, gamma [1] f32."""
+    N, K = W.shape
+    if W.dtype not in (torch.bfloat16, torch.float32):
+        raise ValueError("W must be bf16 or f32")
+    _need(W, W.dtype, (N, K), "W")
+    _need(w_packed, torch.uint8, (N, K // 4), "w_packed")
+    _need(gamma, torch.float32, (1,), "gamma")
+    wdt = BL_F32 if W.dtype == torch.float32 else BL_BF16
+    _check(load_library().bl_quantize_weight(_ptr(W), wdt, N, K, _ptr(w_packed), _ptr(gamma), _ptr(workspace),
+                                             workspace.numel() * workspace.element_size(), _stream(stream)),
+           "bl_quantize_weight")
+
+
+def bl_quantize_act(x, xq, sx, stream=None):
+    """S2: x [M,K] bf16 -> xq [M,K] int8, sx [M] f32."""
+    M, K = x.shape
+    _need(x, torch.bfloat16, (M, K), "x")
+    _need(xq, torch.int8, (M, K), "xq")
+    _need(sx, torch.float32, (M,), "sx")
+    _check(load_library().bl_quantize_act(_ptr(x), M, K, _ptr(xq), _ptr(sx), _stream(stream)), "bl_quantize_act")
+
+
+def bl_forward(xq, sx, w_packed, gamma, y, debug_acc=None, stream=None):
+    """S3: y [M,N] bf16 = xq . codes^T * sx * gamma (debug_acc [M,N] int32 optional)."""
+    M, K = xq.shape
+    N = w_packed.shape[0]
+    _need(xq, torch.int8, (M, K), "xq")
+    _need(sx, torch.float32, (M,), "sx")
+    _need(w_packed, torch.uint8, (N, K // 4), "w_packed")
+    _need(gamma, torch.float32, (1,), "gamma")
+    _need(y, torch.bfloat16, (M, N), "y")
+    if debug_acc is not None:
+        _need(debug_acc, torch.int32, (M, N), "debug_acc")
+    _check(load_library().bl_forward(_ptr(xq), _ptr(sx), _ptr(w_packed), _ptr(gamma), M, N, K, _ptr(y),
+                                     _ptr(debug_acc), _stream(stream)), "bl_forward")
+
+
+def bl_backward(dY, xq, sx, w_packed, gamma, dX=None, dW=None, accumulate_dW=False, stream=None):
+    """S4: dX [M,K] bf16 = gamma * dY . codes; dW [N,K] (bf16|f32) = dY^T . x_hat."""
+    M, N = dY.shape
+    K = xq.shape[1]
+    _need(dY, torch.bfloat16, (M, N), "dY")
+    _need(xq, torch.int8, (M, K), "xq")
+    _need(sx, torch.float32, (M,), "sx")
+    _need(w_packed, torch.uint8, (N, K // 4), "w_packed")
+    _need(gamma, torch.float32, (1,), "gamma")
+    dwdt = BL_BF16
+    if dX is not None:
+        _need(dX, torch.bfloat16, (M, K), "dX")
+    if dW is not None:
+        if dW.dtype not in (torch.bfloat16, torch.float32):
+            raise ValueError("dW must be bf16 or f32")
+        _need(dW, dW.dtype, (N, K), "dW")
+        dwdt = BL_F32 if dW.dtype == torch.float32 else BL_BF16
+    _check(load_library().bl_backward(_ptr(dY), _ptr(xq), _ptr(sx), _ptr(w_packed), _ptr(gamma), M, N, K,
+                                      _ptr(dX), _ptr(dW), dwdt, int(bool(accumulate_dW)), _stream(stream)),
+           "bl_backward")
+
+
+def bl_export_weights(w_packed, gamma, stream=None):
+    """Copy (w_packed, gamma) to host: returns (uint8 [N,K/4] CPU tensor, float gamma)."""
+    N, Kq = w_packed.shape
+    host = torch.empty((N, Kq), dtype=torch.uint8, pin_memory=True)
+    hg = torch.empty(1, dtype=torch.float32, pin_memory=True)
+    _check(load_library().bl_export_weights(_ptr(w_packed), _ptr(gamma), N, Kq * 4, _ptr(host), _ptr(hg),
+                                            _stream(stream)), "bl_export_weights")
+    return host, float(hg[0])
+
+
+def bl_get_last_error() -> int:
+    return load_library().bl_get_last_error()
+
+
+def bl_reset_error() -> int:
+    return load_library().bl_reset_error()
+
+
+# ----------------------------------------------------------------- one whole step
+
+@dataclass
+class StepBuffers:
+    """Device buffers of one BitLinear fwd+bwd (caller-owned, reused)."""
+    w_packed: torch.Tensor
+    gamma: torch.Tensor
+    workspace: torch.Tensor
+    xq: torch.Tensor
+    sx: torch.Tensor
+    y: torch.Tensor
+    dX: torch.Tensor
+    dW: torch.Tensor
+
+    @staticmethod
+    def allocate(M, N, K, dw_dtype=torch.bfloat16, device="cuda"):
+        ws = bl_quantize_weight_workspace_size(N, K)
+        return StepBuffers(
+            w_packed=torch.empty((N, K // 4), dtype=torch.uint8, device=device),
+            gamma=torch.empty(1, dtype=torch.float32, device=device),
+            workspace=torch.empty(max(ws, 16), dtype=torch.uint8, device=device),
+            xq=torch.empty((M, K), dtype=torch.int8, device=device),
+            sx=torch.empty(M, dtype=torch.float32, device=device),
+            y=torch.empty((M, N), dtype=torch.bfloat16, device=device),
+            dX=torch.empty((M, K), dtype=torch.bfloat16, device=device),
+            dW=torch.empty((N, K), dtype=dw_dtype, device=device),
+        )
+
+
+def bitlinear_step(x, W, dY, bufs: StepBuffers, stream=None):
+    """One BitLinear forward + backward: S1 -> S2 -> S3 -> S4 (six kernel launches)."""
+    bl_quantize_weight(W, bufs.w_packed, bufs.gamma, bufs.workspace, stream)
+    bl_quantize_act(x, bufs.xq, bufs.sx, stream)
+    bl_forward(bufs.xq, bufs.sx, bufs.w_packed, bufs.gamma, bufs.y, None, stream)
+    bl_backward(dY, bufs.xq, bufs.sx, bufs.w_packed, bufs.gamma, bufs.dX, bufs.dW, False, stream)

@@ -1,0 +1,220 @@
+// C ABI of the BitLinear library: argument validation on the host, dispatch
+// to the kernels, and the per-device error word that bounded device waits
+// write on timeout. See include/bitlinear.h for the contract of each call.
+#include <cuda_runtime.h>
+
+#include <cstdarg>
+#include <cstdint>
+#include <cstdio>
+#include <mutex>
+
+#include "../../include/bitlinear.h"
+#include "bl_internal.h"
+
+namespace {
+
+__device__ int g_device_error = 0;
+
+thread_local char g_msg[256] = "";
+
+bl_status fail(bl_status s, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_msg, sizeof(g_msg), fmt, ap);
+  va_end(ap);
+  return s;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Device address of the error word, looked up once per device.
+int* device_error_ptr(int dev) {
+  static int* ptrs[64] = {};
+  static std::mutex mu;
+  if (dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!ptrs[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return nullptr;
+    ptrs[dev] = static_cast<int*>(p);
+  }
+  return ptrs[dev];
+}
+
+// Checks the current device is sm_100 and returns its error word.
+bl_status current_device(int** err) {
+  static int arch_ok[64] = {};  // 0 unknown, 1 ok, 2 bad
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return fail(BL_ERR_CUDA, "cudaGetDevice failed");
+  if (dev < 0 || dev >= 64) return fail(BL_ERR_CUDA, "device index %d out of range", dev);
+  if (arch_ok[dev] == 0) {
+    int major = 0, minor = 0;
+    cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+    arch_ok[dev] = (major == 10 && minor == 0) ? 1 : 2;
+  }
+  if (arch_ok[dev] != 1) return fail(BL_ERR_ARCH, "device %d is not sm_100", dev);
+  *err = device_error_ptr(dev);
+  if (!*err) return fail(BL_ERR_CUDA, "cannot resolve the device error word");
+  return BL_OK;
+}
+
+bl_status check_k(int64_t K) {
+  if (K < 32 || K % 32 != 0) return fail(BL_ERR_UNSUPPORTED_SHAPE, "K=%lld must be a positive multiple of 32", (long long)K);
+  if (K > (int64_t(1) << 30)) return fail(BL_ERR_UNSUPPORTED_SHAPE, "K=%lld too large", (long long)K);
+  return BL_OK;
+}
+
+bl_status cuda_status(cudaError_t e, const char* what) {
+  if (e == cudaSuccess) return BL_OK;
+  return fail(BL_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+}  // namespace
+
+extern "C" {
+
+int bl_version(void) { return (1 << 16) | 0; }
+
+const char* bl_status_string(bl_status s) {
+  switch (s) {
+    case BL_OK: return "BL_OK";
+    case BL_ERR_INVALID_ARG: return "BL_ERR_INVALID_ARG";
+    case BL_ERR_UNSUPPORTED_SHAPE: return "BL_ERR_UNSUPPORTED_SHAPE";
+    case BL_ERR_DTYPE: return "BL_ERR_DTYPE";
+    case BL_ERR_ALIGNMENT: return "BL_ERR_ALIGNMENT";
+    case BL_ERR_ARCH: return "BL_ERR_ARCH";
+    case BL_ERR_CUDA: return "BL_ERR_CUDA";
+    case BL_ERR_TIMEOUT: return "BL_ERR_TIMEOUT";
+    case BL_ERR_WORKSPACE: return "BL_ERR_WORKSPACE";
+  }
+  return "BL_ERR_UNKNOWN";
+}
+
+const char* bl_last_error_message(void) { return g_msg; }
+
+size_t bl_quantize_weight_workspace_size(int64_t N, int64_t K) {
+  if (N <= 0 || K <= 0) return 0;
+  return static_cast<size_t>(bl::weight_partials_count(N * K)) * sizeof(double);
+}
+
+bl_status bl_quantize_weight(const void* W, bl_dtype w_dtype, int64_t N, int64_t K, uint8_t* w_packed,
+                             float* gamma, void* workspace, size_t workspace_bytes, void* stream) {
+  g_msg[0] = 0;
+  if (N < 1) return fail(BL_ERR_INVALID_ARG, "N=%lld must be >= 1", (long long)N);
+  if (bl_status s = check_k(K)) return s;
+  if (w_dtype != BL_BF16 && w_dtype != BL_F32) return fail(BL_ERR_DTYPE, "w_dtype %d", (int)w_dtype);
+  if (!W || !w_packed || !gamma) return fail(BL_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(W) || !aligned16(w_packed) || !aligned16(gamma))
+    return fail(BL_ERR_ALIGNMENT, "W, w_packed and gamma must be 16-byte aligned");
+  const size_t need = bl_quantize_weight_workspace_size(N, K);
+  if (!workspace || workspace_bytes < need || !aligned16(workspace))
+    return fail(BL_ERR_WORKSPACE, "workspace needs %zu bytes, 16-byte aligned", need);
+  int* err = nullptr;
+  if (bl_status s = current_device(&err)) return s;
+  return cuda_status(bl::launch_quantize_weight(W, w_dtype == BL_F32, N, K, w_packed, gamma,
+                                                static_cast<double*>(workspace),
+                                                static_cast<cudaStream_t>(stream)),
+                     "bl_quantize_weight launch");
+}
+
+bl_status bl_quantize_act(const void* x, int64_t M, int64_t K, int8_t* xq, float* sx, void* stream) {
+  g_msg[0] = 0;
+  if (M < 0) return fail(BL_ERR_INVALID_ARG, "M=%lld must be >= 0", (long long)M);
+  if (bl_status s = check_k(K)) return s;
+  if (M == 0) return BL_OK;
+  if (!x || !xq || !sx) return fail(BL_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(x) || !aligned16(xq) || !aligned16(sx))
+    return fail(BL_ERR_ALIGNMENT, "x, xq and sx must be 16-byte aligned");
+  int* err = nullptr;
+  if (bl_status s = current_device(&err)) return s;
+  return cuda_status(bl::launch_quantize_act(x, M, K, xq, sx, static_cast<cudaStream_t>(stream)),
+                     "bl_quantize_act launch");
+}
+
+bl_status bl_forward(const int8_t* xq, const float* sx, const uint8_t* w_packed, const float* gamma, int64_t M,
+                     int64_t N, int64_t K, void* y, int32_t* debug_acc, void* stream) {
+  g_msg[0] = 0;
+  if (M < 0 || N < 1) return fail(BL_ERR_INVALID_ARG, "M=%lld, N=%lld", (long long)M, (long long)N);
+  if (bl_status s = check_k(K)) return s;
+  if (M > (int64_t(1) << 30) || N > (int64_t(1) << 30)) return fail(BL_ERR_UNSUPPORTED_SHAPE, "M or N too large");
+  if (M == 0) return BL_OK;
+  if (!xq || !sx || !w_packed || !gamma || !y) return fail(BL_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(xq) || !aligned16(sx) || !aligned16(w_packed) || !aligned16(gamma) || !aligned16(y) ||
+      (debug_acc && !aligned16(debug_acc)))
+    return fail(BL_ERR_ALIGNMENT, "tensors must be 16-byte aligned");
+  int* err = nullptr;
+  if (bl_status s = current_device(&err)) return s;
+  return cuda_status(bl::launch_forward(xq, sx, w_packed, gamma, M, N, K, y, debug_acc, err,
+                                        static_cast<cudaStream_t>(stream)),
+                     "bl_forward launch");
+}
+
+bl_status bl_backward(const void* dY, const int8_t* xq, const float* sx, const uint8_t* w_packed,
+                      const float* gamma, int64_t M, int64_t N, int64_t K, void* dX, void* dW, bl_dtype dw_dtype,
+                      int accumulate_dW, void* stream) {
+  g_msg[0] = 0;
+  if (M < 0 || N < 1) return fail(BL_ERR_INVALID_ARG, "M=%lld, N=%lld", (long long)M, (long long)N);
+  if (bl_status s = check_k(K)) return s;
+  if (N % 8 != 0) return fail(BL_ERR_UNSUPPORTED_SHAPE, "N=%lld must be a multiple of 8", (long long)N);
+  if (M > (int64_t(1) << 30) || N > (int64_t(1) << 30)) return fail(BL_ERR_UNSUPPORTED_SHAPE, "M or N too large");
+  if (dW && dw_dtype != BL_BF16 && dw_dtype != BL_F32) return fail(BL_ERR_DTYPE, "dw_dtype %d", (int)dw_dtype);
+  if (!dX && !dW) return BL_OK;
+  if (M > 0 && !dY) return fail(BL_ERR_INVALID_ARG, "null dY");
+  if (dX && (!w_packed || !gamma)) return fail(BL_ERR_INVALID_ARG, "dX needs w_packed and gamma");
+  if (dW && M > 0 && (!xq || !sx)) return fail(BL_ERR_INVALID_ARG, "dW needs xq and sx");
+  if ((dY && !aligned16(dY)) || (xq && !aligned16(xq)) || (sx && !aligned16(sx)) ||
+      (w_packed && !aligned16(w_packed)) || (gamma && !aligned16(gamma)) || (dX && !aligned16(dX)) ||
+      (dW && !aligned16(dW)))
+    return fail(BL_ERR_ALIGNMENT, "tensors must be 16-byte aligned");
+  int* err = nullptr;
+  if (bl_status s = current_device(&err)) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (dX) {
+    if (bl_status s = cuda_status(bl::launch_backward_dx(dY, w_packed, gamma, M, N, K, dX, err, st),
+                                  "bl_backward dX launch"))
+      return s;
+  }
+  if (dW) {
+    if (bl_status s = cuda_status(
+            bl::launch_backward_dw(dY, xq, sx, M, N, K, dW, dw_dtype == BL_F32, accumulate_dW != 0, err, st),
+            "bl_backward dW launch"))
+      return s;
+  }
+  return BL_OK;
+}
+
+bl_status bl_export_weights(const uint8_t* w_packed, const float* gamma, int64_t N, int64_t K,
+                            uint8_t* host_packed, float* host_gamma, void* stream) {
+  g_msg[0] = 0;
+  if (N < 1) return fail(BL_ERR_INVALID_ARG, "N=%lld must be >= 1", (long long)N);
+  if (bl_status s = check_k(K)) return s;
+  if (!w_packed || !gamma || !host_packed || !host_gamma) return fail(BL_ERR_INVALID_ARG, "null pointer");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (bl_status s = cuda_status(cudaMemcpyAsync(host_packed, w_packed, static_cast<size_t>(N * (K / 4)),
+                                                cudaMemcpyDeviceToHost, st),
+                                "export packed"))
+    return s;
+  if (bl_status s = cuda_status(cudaMemcpyAsync(host_gamma, gamma, sizeof(float), cudaMemcpyDeviceToHost, st),
+                                "export gamma"))
+    return s;
+  return cuda_status(cudaStreamSynchronize(st), "export sync");
+}
+
+bl_status bl_get_last_error(void) {
+  g_msg[0] = 0;
+  if (cudaError_t e = cudaDeviceSynchronize(); e != cudaSuccess) return cuda_status(e, "cudaDeviceSynchronize");
+  int v = 0;
+  if (cudaError_t e = cudaMemcpyFromSymbol(&v, g_device_error, sizeof(int)); e != cudaSuccess)
+    return cuda_status(e, "read device error word");
+  if (v == BL_ERR_TIMEOUT) return fail(BL_ERR_TIMEOUT, "a device pipeline wait exceeded its bound");
+  return v == 0 ? BL_OK : fail(static_cast<bl_status>(v), "device error %d", v);
+}
+
+bl_status bl_reset_error(void) {
+  g_msg[0] = 0;
+  const int zero = 0;
+  return cuda_status(cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int)), "reset device error word");
+}
+
+}  // extern "C"

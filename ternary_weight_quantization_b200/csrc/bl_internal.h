@@ -1,0 +1,38 @@
+// Host-side launchers shared between the kernel translation units and the
+// C ABI layer. Not part of the public interface.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace bl {
+
+// ---- S1: absmean ternarisation + 2-bit packing
+// Number of fp64 partial sums pass A writes for a tensor of `numel` elements
+// (a fixed function of numel, so the reduction order never depends on the GPU).
+int weight_partials_count(int64_t numel);
+
+// Pass A (|W| partial sums) + pass B (gamma, codes, packing).
+// `partials` holds weight_partials_count(N*K) doubles.
+cudaError_t launch_quantize_weight(const void* W, int w_is_f32, int64_t N, int64_t K, uint8_t* packed,
+                                   float* gamma, double* partials, cudaStream_t s);
+
+// ---- S2: per-token absmax INT8
+cudaError_t launch_quantize_act(const void* x, int64_t M, int64_t K, int8_t* xq, float* sx, cudaStream_t s);
+
+// ---- S3 / S4 GEMMs (tcgen05)
+cudaError_t launch_forward(const int8_t* xq, const float* sx, const uint8_t* w_packed, const float* gamma,
+                           int64_t M, int64_t N, int64_t K, void* y, int32_t* debug_acc, int* err,
+                           cudaStream_t s);
+
+cudaError_t launch_backward_dx(const void* dY, const uint8_t* w_packed, const float* gamma, int64_t M, int64_t N,
+                               int64_t K, void* dX, int* err, cudaStream_t s);
+
+cudaError_t launch_backward_dw(const void* dY, const int8_t* xq, const float* sx, int64_t M, int64_t N, int64_t K,
+                               void* dW, int dw_is_f32, int accumulate, int* err, cudaStream_t s);
+
+// Number of SMs of the current device (cached per device).
+int device_sm_count();
+
+}  // namespace bl

@@ -1,0 +1,740 @@
+// S3 and S4 of the BitLinear hot path on sm_100a: the INT32-exact forward GEMM
+// and the two straight-through backward GEMMs ("bitnet-qat-train", Semantics:
+// y = quant(x) . ternarize(W)^T . s_x . gamma; dX = dY . W_hat;
+// dW = dY^T . x_hat, with W_hat and x_hat rebuilt from the saved 2-bit and
+// INT8 state).
+//
+// One persistent, warp-specialised kernel template serves all three:
+//
+//   D[i][j] = sum_r A[i][r] * B[j][r]        (tcgen05.mma, accumulator in TMEM)
+//   out[j][i] = epilogue(D[i][j])            (transposed store)
+//
+//   op   A (128-row tile, REBUILT in smem)      B (256-row tile, TMA)        r
+//   Fwd  codes[n][k] int8, K-major              xq[m][k] int8, K-major        k
+//   Dx   codes^T[k][n] bf16 {-1,0,1}, MN-major  dY[m][n] bf16, K-major        n
+//   Dw   x_hat^T[k][m] bf16, MN-major           dY^T[n][m] bf16, MN-major     m
+//
+// The ternary / INT8 operand is always A: its rebuild writes a 128-row tile
+// per stage into shared memory (never to HBM), while the wider 256-row
+// operand streams in by TMA. The output tile is transposed through shared
+// memory so global stores stay row-contiguous.
+//
+// Warp roles (320 threads):
+//   warp 0    loads: TMA for B (and Dw's q/s_x), cp.async for packed codes
+//   warp 1    TMEM allocation (2 x 256 columns) and tcgen05.mma issue
+//   warps 2-5 rebuild A from the staged 2-bit / INT8 source
+//   warps 6-9 epilogue: TMEM -> registers -> smem (transpose) -> global
+// Shared-memory stages form a ring guarded by mbarriers; two TMEM
+// accumulators let the epilogue of one tile overlap the MMAs of the next.
+// Every wait is bounded: on expiry the CTA records a timeout in the device
+// error word, drains what it has in flight, frees TMEM and exits.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cstdint>
+#include <cstdio>
+#include <mutex>
+
+#include "bl_device.cuh"
+#include "bl_internal.h"
+
+namespace bl {
+namespace {
+
+constexpr int kThreads = 320;
+constexpr int kWarpLoad = 0;
+constexpr int kWarpMma = 1;
+constexpr int kWarpRebuild0 = 2;
+constexpr int kNumRebuildWarps = 4;
+constexpr int kWarpEpi0 = 6;
+constexpr int kNumEpiWarps = 4;
+
+constexpr int BM = 128;            // A rows per tile (UMMA M)
+constexpr int BN = 256;            // B rows per tile (UMMA N)
+constexpr uint32_t kTmemCols = 512;  // two BN-column accumulators
+constexpr int kEpiStageBytes = 32 * 32 * 4;  // per epilogue warp
+
+enum class Op { Fwd, Dx, Dw };
+
+template <Op op>
+struct Cfg;
+
+template <>
+struct Cfg<Op::Fwd> {
+  static constexpr int kBlockR = 128;           // reduction elements (k) per stage
+  static constexpr int kUmmaK = 32;             // kind::i8: 32 bytes of K per MMA
+  static constexpr int kABytes = BM * 128;      // 128 rows x 128 int8
+  static constexpr int kBBytes = BN * 128;      // 256 rows x 128 int8
+  static constexpr int kSrcBytes = BM * 32;     // packed codes: 128 rows x 32 bytes
+  static constexpr int kSxBytes = 0;
+  static constexpr int kStages = 4;
+  static constexpr uint32_t kIdesc = make_idesc(2 /*s32*/, 1 /*s8*/, 0, 0, BM, BN);
+  static constexpr uint32_t kTxBytes = kBBytes;
+  static constexpr uint32_t kLoadArrivals = 1 + 32;  // expect_tx + 32 cp.async lanes
+};
+
+template <>
+struct Cfg<Op::Dx> {
+  static constexpr int kBlockR = 64;            // reduction elements (n) per stage
+  static constexpr int kUmmaK = 16;
+  static constexpr int kABytes = BM * 64 * 2;   // 128 k x 64 n bf16
+  static constexpr int kBBytes = BN * 64 * 2;   // 256 m x 64 n bf16
+  static constexpr int kSrcBytes = 64 * 32;     // packed: 64 rows (n) x 32 bytes (128 k)
+  static constexpr int kSxBytes = 0;
+  static constexpr int kStages = 4;
+  static constexpr uint32_t kIdesc = make_idesc(1 /*f32*/, 1 /*bf16*/, 1 /*A MN*/, 0, BM, BN);
+  static constexpr uint32_t kTxBytes = kBBytes;
+  static constexpr uint32_t kLoadArrivals = 1 + 32;
+};
+
+template <>
+struct Cfg<Op::Dw> {
+  static constexpr int kBlockR = 64;            // reduction elements (m) per stage
+  static constexpr int kUmmaK = 16;
+  static constexpr int kABytes = BM * 64 * 2;   // 128 k x 64 m bf16
+  static constexpr int kBBytes = BN * 64 * 2;   // 256 n x 64 m bf16 (4 TMA boxes)
+  static constexpr int kSrcBytes = 64 * 128;    // q: 64 rows (m) x 128 int8 (k), swizzled
+  static constexpr int kSxBytes = 64 * 4;       // s_x for the 64 tokens
+  static constexpr int kStages = 3;
+  static constexpr uint32_t kIdesc = make_idesc(1, 1, 1 /*A MN*/, 1 /*B MN*/, BM, BN);
+  static constexpr uint32_t kTxBytes = kBBytes + kSrcBytes + kSxBytes;
+  static constexpr uint32_t kLoadArrivals = 1;
+};
+
+template <Op op>
+struct Layout {
+  using C = Cfg<op>;
+  static constexpr int kS = C::kStages;
+  static constexpr int kOffA = 0;
+  static constexpr int kOffB = kOffA + kS * C::kABytes;
+  static constexpr int kOffSrc = kOffB + kS * C::kBBytes;
+  static constexpr int kOffSx = kOffSrc + kS * C::kSrcBytes;
+  static constexpr int kOffEpi = kOffSx + kS * C::kSxBytes;
+  static constexpr int kOffBar = kOffEpi + kNumEpiWarps * kEpiStageBytes;
+  // barriers: load_full[S], a_full[S], empty[S], tmem_full[2], tmem_empty[2], done
+  static constexpr int kNumBars = 3 * kS + 5;
+  static constexpr int kOffMisc = kOffBar + kNumBars * 8;
+  static constexpr int kBytes = kOffMisc + 64;
+  static constexpr int kDynBytes = kBytes + 1024;  // slack to align the base to 1024
+  static_assert(kDynBytes <= 232448, "shared memory budget");
+  static_assert(C::kABytes % 1024 == 0 && C::kBBytes % 1024 == 0 && C::kSrcBytes % 1024 == 0, "alignment");
+};
+
+struct GemmParams {
+  int rows_a;      // extent of the A-row index i (N for Fwd, K for Dx/Dw)
+  int rows_b;      // extent of the B-row index j (M for Fwd/Dx, N for Dw)
+  int red;         // reduction length (K, N, M)
+  int tiles_a, tiles_b, num_kb, num_tiles;
+  int64_t K;                  // in_features (row length of packed codes / q)
+  const uint8_t* packed;      // Fwd, Dx
+  const float* sx;            // Fwd epilogue
+  const float* gamma;         // Fwd, Dx epilogue
+  void* out;                  // [rows_b][ldo]
+  int64_t ldo;
+  int32_t* debug_acc;         // Fwd, optional
+  int out_f32;                // Dw
+  int accumulate;             // Dw
+  int* err;
+};
+
+// ---------------------------------------------------------------- rebuild helpers
+
+// 8 two-bit fields (16 bits) -> nibble i holds field i.
+__device__ __forceinline__ uint32_t spread_fields8(uint32_t h) {
+  uint32_t x = h & 0xFFFFu;
+  x = (x | (x << 8)) & 0x00FF00FFu;
+  x = (x | (x << 4)) & 0x0F0F0F0Fu;
+  x = (x | (x << 2)) & 0x33333333u;
+  return x;
+}
+
+// 16 packed codes (one 32-bit word) -> 16 int8 codes.
+__device__ __forceinline__ uint4 codes16_to_s8(uint32_t w) {
+  constexpr uint32_t kTable = 0xFFFE0100u;  // field 0 -> 0, 1 -> +1, 2 -> -2 (unused), 3 -> -1
+  const uint32_t lo = spread_fields8(w);
+  const uint32_t hi = spread_fields8(w >> 16);
+  uint4 r;
+  r.x = __byte_perm(kTable, 0u, lo & 0xFFFFu);
+  r.y = __byte_perm(kTable, 0u, lo >> 16);
+  r.z = __byte_perm(kTable, 0u, hi & 0xFFFFu);
+  r.w = __byte_perm(kTable, 0u, hi >> 16);
+  return r;
+}
+
+// 8 packed codes (16 bits) -> 8 bf16 values in {-1, 0, +1}.
+// Field bit 0 marks a nonzero code and bit 1 a negative one, so each bf16 is
+// b0 * 0x3F80 + b1 * 0x8000; two codes are handled per 32-bit word.
+__device__ __forceinline__ uint4 codes8_to_bf16(uint32_t h) {
+  h &= 0xFFFFu;
+  const uint32_t s = h | (h << 14);  // field 2w at bits 4w.., field 2w+1 at bits 4w+16..
+  uint32_t r[4];
+#pragma unroll
+  for (int w = 0; w < 4; ++w) {
+    const uint32_t g = s >> (4 * w);
+    const uint32_t nz = g & 0x00010001u;
+    const uint32_t neg = (g << 14) & 0x80008000u;
+    r[w] = nz * 0x3F80u + neg;
+  }
+  return make_uint4(r[0], r[1], r[2], r[3]);
+}
+
+// 16 int8 (x_hat source) * s -> 16 bf16, each bf16_rn(fp32(q) * s).
+// fp32(q) uses the 2^23 shifter: bits 0x4B0000uu are 2^23 + u with
+// u = q + 128, so subtracting 2^23 + 128 is exact.
+__device__ __forceinline__ void s8x16_to_bf16(const uint4& v, float s, uint4& o0, uint4& o1) {
+  const uint32_t w[4] = {v.x ^ 0x80808080u, v.y ^ 0x80808080u, v.z ^ 0x80808080u, v.w ^ 0x80808080u};
+  uint32_t out[8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+#pragma unroll
+    for (int b = 0; b < 4; b += 2) {
+      const float f0 = __fsub_rn(__uint_as_float(__byte_perm(w[i], 0x4B000000u, 0x7440u | b)), 8388736.0f);
+      const float f1 = __fsub_rn(__uint_as_float(__byte_perm(w[i], 0x4B000000u, 0x7440u | (b + 1))), 8388736.0f);
+      const __nv_bfloat162 p = __floats2bfloat162_rn(__fmul_rn(f0, s), __fmul_rn(f1, s));
+      out[i * 2 + b / 2] = *reinterpret_cast<const uint32_t*>(&p);
+    }
+  }
+  o0 = make_uint4(out[0], out[1], out[2], out[3]);
+  o1 = make_uint4(out[4], out[5], out[6], out[7]);
+}
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, const uint4& v) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+               : "memory");
+}
+
+__device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr)
+               : "memory");
+  return v;
+}
+
+// ---------------------------------------------------------------- the kernel
+
+template <Op op>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_kernel(const __grid_constant__ CUtensorMap map_b, const __grid_constant__ CUtensorMap map_src,
+                const __grid_constant__ CUtensorMap map_sx, const GemmParams p) {
+  using C = Cfg<op>;
+  using L = Layout<op>;
+  constexpr int S = C::kStages;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kOffBar);
+  uint64_t* load_full = bars;
+  uint64_t* a_full = bars + S;
+  uint64_t* empty = bars + 2 * S;
+  uint64_t* tmem_full = bars + 3 * S;
+  uint64_t* tmem_empty = bars + 3 * S + 2;
+  uint64_t* done_bar = bars + 3 * S + 4;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::kOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kOffMisc + 4);
+  int* issued_parity = reinterpret_cast<int*>(smem + L::kOffMisc + 8);  // [S], load warp's last issue
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&load_full[s], C::kLoadArrivals);
+      mbar_init(&a_full[s], kNumRebuildWarps);
+      mbar_init(&empty[s], 1);
+      issued_parity[s] = -1;
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tmem_full[b], 1);
+      mbar_init(&tmem_empty[b], kNumEpiWarps);
+    }
+    mbar_init(done_bar, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == kWarpMma) {
+    tmem_alloc(tmem_holder, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  const int kq = static_cast<int>(p.K / 4);  // bytes per packed row
+
+  if (warp == kWarpLoad) {
+    // ------------------------------------------------------------ loads
+    if (lane == 0) {
+      prefetch_tensormap(&map_b);
+      if constexpr (op == Op::Dw) {
+        prefetch_tensormap(&map_src);
+        prefetch_tensormap(&map_sx);
+      }
+    }
+    int stage = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
+      const int a0 = (tile % p.tiles_a) * BM;
+      const int b0 = (tile / p.tiles_a) * BN;
+      for (int kb = 0; kb < p.num_kb; ++kb) {
+        if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.err)) {
+          ok = false;
+          break;
+        }
+        uint8_t* sB = smem + L::kOffB + stage * C::kBBytes;
+        uint8_t* sSrc = smem + L::kOffSrc + stage * C::kSrcBytes;
+        const int r0 = kb * C::kBlockR;
+        if (lane == 0) {
+          issued_parity[stage] = static_cast<int>(phase);
+          mbar_arrive_expect_tx(&load_full[stage], C::kTxBytes);
+          if constexpr (op == Op::Fwd) {
+            tma_load_2d(&map_b, &load_full[stage], sB, r0, b0);
+          } else if constexpr (op == Op::Dx) {
+            tma_load_2d(&map_b, &load_full[stage], sB, r0, b0);
+          } else {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) tma_load_2d(&map_b, &load_full[stage], sB + j * 8192, b0 + 64 * j, r0);
+            tma_load_2d(&map_src, &load_full[stage], sSrc, a0, r0);
+            tma_load_1d(&map_sx, &load_full[stage], smem + L::kOffSx + stage * C::kSxBytes, r0);
+          }
+        }
+        if constexpr (op == Op::Fwd) {
+          // packed rows a0..a0+127, bytes [kb*32, kb*32+32): 512 chunks of 8 bytes
+#pragma unroll
+          for (int it = 0; it < 16; ++it) {
+            const int c = lane + 32 * it;
+            const int row = c >> 2, part = c & 3;
+            const bool valid = (a0 + row < p.rows_a) && (r0 + part * 32 < p.red);
+            const uint8_t* src = valid ? p.packed + static_cast<int64_t>(a0 + row) * kq + kb * 32 + part * 8
+                                       : p.packed;
+            cp_async_8(sSrc + row * 32 + part * 8, src, valid ? 8u : 0u);
+          }
+          cp_async_mbar_arrive_noinc(&load_full[stage]);
+        } else if constexpr (op == Op::Dx) {
+          // packed rows (n) r0..r0+63, bytes covering k in [a0, a0+128): 256 chunks
+#pragma unroll
+          for (int it = 0; it < 8; ++it) {
+            const int c = lane + 32 * it;
+            const int row = c >> 2, part = c & 3;
+            const bool valid = (r0 + row < p.red) && (a0 + part * 32 < p.rows_a);
+            const uint8_t* src =
+                valid ? p.packed + static_cast<int64_t>(r0 + row) * kq + a0 / 4 + part * 8 : p.packed;
+            cp_async_8(sSrc + row * 32 + part * 8, src, valid ? 8u : 0u);
+          }
+          cp_async_mbar_arrive_noinc(&load_full[stage]);
+        }
+        if (++stage == S) {
+          stage = 0;
+          phase ^= 1;
+        }
+      }
+    }
+    __syncwarp();
+    if (!ok && lane == 0) {
+      // let every copy already issued land before the CTA exits
+      for (int s = 0; s < S; ++s)
+        if (issued_parity[s] >= 0) mbar_drain(&load_full[s], static_cast<uint32_t>(issued_parity[s]));
+    }
+  } else if (warp == kWarpMma) {
+    // ------------------------------------------------------------ MMA issue
+    int stage = 0;
+    uint32_t phase = 0;
+    int buf = 0;
+    uint32_t buf_phase = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
+      if (!mbar_wait(&tmem_empty[buf], buf_phase ^ 1, abort_flag, p.err)) break;
+      tc_fence_after();
+      const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * BN);
+      for (int kb = 0; kb < p.num_kb; ++kb) {
+        if (!mbar_wait(&load_full[stage], phase, abort_flag, p.err) ||
+            !mbar_wait(&a_full[stage], phase, abort_flag, p.err)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (lane == 0) {
+          const uint32_t sa = smem_u32(smem + L::kOffA + stage * C::kABytes);
+          const uint32_t sb = smem_u32(smem + L::kOffB + stage * C::kBBytes);
+#pragma unroll
+          for (int kk = 0; kk < C::kBlockR / C::kUmmaK; ++kk) {
+            uint64_t adesc, bdesc;
+            if constexpr (op == Op::Fwd) {
+              adesc = smem_desc_sw128(sa + kk * 32, 16, 1024);
+              bdesc = smem_desc_sw128(sb + kk * 32, 16, 1024);
+              mma_i8(d_tmem, adesc, bdesc, C::kIdesc, (kb | kk) != 0);
+            } else if constexpr (op == Op::Dx) {
+              adesc = smem_desc_sw128(sa + kk * 2048, 8192, 1024);  // MN-major
+              bdesc = smem_desc_sw128(sb + kk * 32, 16, 1024);      // K-major
+              mma_f16(d_tmem, adesc, bdesc, C::kIdesc, (kb | kk) != 0);
+            } else {
+              adesc = smem_desc_sw128(sa + kk * 2048, 8192, 1024);  // MN-major
+              bdesc = smem_desc_sw128(sb + kk * 2048, 8192, 1024);  // MN-major
+              mma_f16(d_tmem, adesc, bdesc, C::kIdesc, (kb | kk) != 0);
+            }
+          }
+          mma_commit(&empty[stage]);
+          if (kb == p.num_kb - 1) mma_commit(&tmem_full[buf]);
+        }
+        __syncwarp();
+        if (++stage == S) {
+          stage = 0;
+          phase ^= 1;
+        }
+      }
+      if (++buf == 2) {
+        buf = 0;
+        buf_phase ^= 1;
+      }
+    }
+    // every MMA issued so far has completed once done_bar flips
+    if (lane == 0) {
+      mma_commit(done_bar);
+      mbar_drain(done_bar, 0);
+    }
+    __syncwarp();
+  } else if (warp < kWarpEpi0) {
+    // ------------------------------------------------------------ rebuild A
+    const int rt = threadIdx.x - 32 * kWarpRebuild0;  // 0..127
+    int stage = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
+      for (int kb = 0; kb < p.num_kb; ++kb) {
+        if (!mbar_wait(&load_full[stage], phase, abort_flag, p.err)) {
+          ok = false;
+          break;
+        }
+        const uint32_t sA = smem_u32(smem + L::kOffA + stage * C::kABytes);
+        const uint32_t sSrc = smem_u32(smem + L::kOffSrc + stage * C::kSrcBytes);
+        if constexpr (op == Op::Fwd) {
+          // row rt: 32 packed bytes -> 128 int8 codes, K-major with 128-byte swizzle
+          const uint4 w0 = ld_shared_v4(sSrc + rt * 32);
+          const uint4 w1 = ld_shared_v4(sSrc + rt * 32 + 16);
+          const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+          const uint32_t row_base = sA + rt * 128;
+#pragma unroll
+          for (int c = 0; c < 8; ++c) st_shared_v4(row_base + ((c ^ (rt & 7)) << 4), codes16_to_s8(words[c]));
+        } else if constexpr (op == Op::Dx) {
+          // reduction row n = rt % 64, output k half = rt / 64 (64 k values)
+          const int n = rt & 63, half = rt >> 6;
+          const uint4 w = ld_shared_v4(sSrc + n * 32 + half * 16);
+          const uint32_t words[4] = {w.x, w.y, w.z, w.w};
+          const uint32_t base = sA + half * 8192 + n * 128;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const uint32_t h = words[j >> 1] >> ((j & 1) * 16);
+            st_shared_v4(base + ((j ^ (n & 7)) << 4), codes8_to_bf16(h));
+          }
+        } else {
+          // token m = rt % 64, k half = rt / 64; q staging is 128-byte swizzled
+          const int m = rt & 63, half = rt >> 6;
+          const float s = reinterpret_cast<const float*>(smem + L::kOffSx + stage * C::kSxBytes)[m];
+          const uint32_t base = sA + half * 8192 + m * 128;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int c = half * 4 + i;  // logical 16-byte chunk (16 k values)
+            const uint4 v = ld_shared_v4(sSrc + m * 128 + ((c ^ (m & 7)) << 4));
+            uint4 o0, o1;
+            s8x16_to_bf16(v, s, o0, o1);
+            const int j0 = 2 * i, j1 = 2 * i + 1;  // 8-k units within this half
+            st_shared_v4(base + ((j0 ^ (m & 7)) << 4), o0);
+            st_shared_v4(base + ((j1 ^ (m & 7)) << 4), o1);
+          }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&a_full[stage]);
+        if (++stage == S) {
+          stage = 0;
+          phase ^= 1;
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;  // TMEM lane quadrant this warp may access
+    const uint32_t stg = smem_u32(smem + L::kOffEpi + (warp - kWarpEpi0) * kEpiStageBytes);
+    const float gamma = (op == Op::Dw) ? 1.0f : __ldg(p.gamma);
+    int buf = 0;
+    uint32_t buf_phase = 0;
+    for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
+      const int a0 = (tile % p.tiles_a) * BM;
+      const int b0 = (tile / p.tiles_a) * BN;
+      if (!mbar_wait(&tmem_full[buf], buf_phase, abort_flag, p.err)) break;
+      tc_fence_after();
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * BN + c * 32, r);
+        tmem_ld_wait();
+        if (c == BN / 32 - 1) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&tmem_empty[buf]);
+        }
+        // transpose through smem: staging[j][lane] = D[row lane][column j]
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          asm volatile("st.shared.b32 [%0], %1;" ::"r"(stg + (j * 32 + lane) * 4), "r"(r[j]) : "memory");
+        __syncwarp();
+        // each lane stores 8 consecutive i of one output row j, 4 rows per pass
+        const int seg = (lane & 3) * 8;
+        const int i0 = a0 + q * 32 + seg;
+#pragma unroll
+        for (int pass = 0; pass < 4; ++pass) {
+          const int jl = pass * 8 + (lane >> 2);
+          const int j = b0 + c * 32 + jl;
+          if (j >= p.rows_b || i0 >= p.rows_a) continue;
+          const uint4 v0 = ld_shared_v4(stg + (jl * 32 + seg) * 4);
+          const uint4 v1 = ld_shared_v4(stg + (jl * 32 + seg + 4) * 4);
+          const uint32_t acc[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+          const int nvalid = min(8, p.rows_a - i0);
+          const int64_t off = static_cast<int64_t>(j) * p.ldo + i0;
+          if constexpr (op == Op::Fwd) {
+            const float scale = __fmul_rn(__ldg(p.sx + j), gamma);
+            __nv_bfloat16* y = static_cast<__nv_bfloat16*>(p.out) + off;
+            uint32_t pk[4];
+#pragma unroll
+            for (int e = 0; e < 8; e += 2) {
+              const __nv_bfloat162 b2 =
+                  __floats2bfloat162_rn(__fmul_rn(static_cast<float>(static_cast<int32_t>(acc[e])), scale),
+                                        __fmul_rn(static_cast<float>(static_cast<int32_t>(acc[e + 1])), scale));
+              pk[e / 2] = *reinterpret_cast<const uint32_t*>(&b2);
+            }
+            const bool vec = nvalid == 8 && (p.ldo % 8) == 0;
+            if (vec) {
+              *reinterpret_cast<uint4*>(y) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            } else {
+              for (int e = 0; e < nvalid; ++e)
+                reinterpret_cast<uint16_t*>(y)[e] = static_cast<uint16_t>(pk[e / 2] >> ((e & 1) * 16));
+            }
+            if (p.debug_acc) {
+              int32_t* d = p.debug_acc + off;
+              if (nvalid == 8 && (p.ldo % 4) == 0) {
+                reinterpret_cast<uint4*>(d)[0] = v0;
+                reinterpret_cast<uint4*>(d)[1] = v1;
+              } else {
+                for (int e = 0; e < nvalid; ++e) d[e] = static_cast<int32_t>(acc[e]);
+              }
+            }
+          } else if constexpr (op == Op::Dx) {
+            __nv_bfloat16* dx = static_cast<__nv_bfloat16*>(p.out) + off;
+            uint32_t pk[4];
+#pragma unroll
+            for (int e = 0; e < 8; e += 2) {
+              const __nv_bfloat162 b2 = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(acc[e]), gamma),
+                                                              __fmul_rn(__uint_as_float(acc[e + 1]), gamma));
+              pk[e / 2] = *reinterpret_cast<const uint32_t*>(&b2);
+            }
+            *reinterpret_cast<uint4*>(dx) = make_uint4(pk[0], pk[1], pk[2], pk[3]);  // K % 32 == 0
+          } else {
+            float v[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) v[e] = __uint_as_float(acc[e]);
+            if (p.out_f32) {
+              float4* dw = reinterpret_cast<float4*>(static_cast<float*>(p.out) + off);
+              if (p.accumulate) {
+                const float4 o0 = dw[0], o1 = dw[1];
+                v[0] = __fadd_rn(v[0], o0.x); v[1] = __fadd_rn(v[1], o0.y);
+                v[2] = __fadd_rn(v[2], o0.z); v[3] = __fadd_rn(v[3], o0.w);
+                v[4] = __fadd_rn(v[4], o1.x); v[5] = __fadd_rn(v[5], o1.y);
+                v[6] = __fadd_rn(v[6], o1.z); v[7] = __fadd_rn(v[7], o1.w);
+              }
+              dw[0] = make_float4(v[0], v[1], v[2], v[3]);
+              dw[1] = make_float4(v[4], v[5], v[6], v[7]);
+            } else {
+              uint4* dw = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + off);
+              if (p.accumulate) {
+                const uint4 o = *dw;
+                const uint32_t ow[4] = {o.x, o.y, o.z, o.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  v[2 * e] = __fadd_rn(v[2 * e], __uint_as_float(ow[e] << 16));
+                  v[2 * e + 1] = __fadd_rn(v[2 * e + 1], __uint_as_float(ow[e] & 0xFFFF0000u));
+                }
+              }
+              uint32_t pk[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const __nv_bfloat162 b2 = __floats2bfloat162_rn(v[2 * e], v[2 * e + 1]);
+                pk[e] = *reinterpret_cast<const uint32_t*>(&b2);
+              }
+              *dw = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            }
+          }
+        }
+        __syncwarp();
+      }
+      if (++buf == 2) {
+        buf = 0;
+        buf_phase ^= 1;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kWarpMma) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+// Degenerate reduction (M == 0 in dW): the product is all zeros.
+__global__ void zero_dw_kernel(void* out, int64_t n, int out_f32, int accumulate) {
+  if (accumulate) return;
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  if (out_f32)
+    static_cast<float*>(out)[i] = 0.0f;
+  else
+    static_cast<uint16_t*>(out)[i] = 0;
+}
+
+// ---------------------------------------------------------------- host side
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  });
+  return fn;
+}
+
+bool make_map_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64_t inner, uint64_t outer,
+                 uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle sw) {
+  auto enc = get_encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool make_map_1d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64_t n, uint32_t box) {
+  auto enc = get_encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[1] = {n};
+  const cuuint32_t boxd[1] = {box};
+  const cuuint32_t estr[1] = {1};
+  return enc(m, dt, 1, const_cast<void*>(base), dims, nullptr, boxd, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <Op op>
+cudaError_t launch_gemm(const CUtensorMap& mb, const CUtensorMap& msrc, const CUtensorMap& msx, GemmParams p,
+                        cudaStream_t s) {
+  using L = Layout<op>;
+  static int configured_device = -1;  // attribute set once per process per device id
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (configured_device != dev) {
+    cudaError_t e =
+        cudaFuncSetAttribute(gemm_kernel<op>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kDynBytes);
+    if (e != cudaSuccess) return e;
+    configured_device = dev;
+  }
+  p.tiles_a = (p.rows_a + BM - 1) / BM;
+  p.tiles_b = (p.rows_b + BN - 1) / BN;
+  p.num_kb = (p.red + Cfg<op>::kBlockR - 1) / Cfg<op>::kBlockR;
+  p.num_tiles = p.tiles_a * p.tiles_b;
+  const int grid = p.num_tiles < device_sm_count() ? p.num_tiles : device_sm_count();
+  gemm_kernel<op><<<grid, kThreads, L::kDynBytes, s>>>(mb, msrc, msx, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+int device_sm_count() {
+  static int cached[64];
+  static bool init[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) return 148;
+  if (!init[dev]) {
+    int n = 0;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    cached[dev] = n > 0 ? n : 148;
+    init[dev] = true;
+  }
+  return cached[dev];
+}
+
+cudaError_t launch_forward(const int8_t* xq, const float* sx, const uint8_t* w_packed, const float* gamma,
+                           int64_t M, int64_t N, int64_t K, void* y, int32_t* debug_acc, int* err,
+                           cudaStream_t s) {
+  if (M == 0 || N == 0) return cudaSuccess;
+  CUtensorMap mb{}, unused{};
+  if (!make_map_2d(&mb, xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, K, M, K, 128, BN, CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  GemmParams p{};
+  p.rows_a = static_cast<int>(N);
+  p.rows_b = static_cast<int>(M);
+  p.red = static_cast<int>(K);
+  p.K = K;
+  p.packed = w_packed;
+  p.sx = sx;
+  p.gamma = gamma;
+  p.out = y;
+  p.ldo = N;
+  p.debug_acc = debug_acc;
+  p.err = err;
+  return launch_gemm<Op::Fwd>(mb, unused, unused, p, s);
+}
+
+cudaError_t launch_backward_dx(const void* dY, const uint8_t* w_packed, const float* gamma, int64_t M, int64_t N,
+                               int64_t K, void* dX, int* err, cudaStream_t s) {
+  if (M == 0) return cudaSuccess;
+  CUtensorMap mb{}, unused{};
+  if (!make_map_2d(&mb, dY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, N, M, N * 2, 64, BN, CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  GemmParams p{};
+  p.rows_a = static_cast<int>(K);
+  p.rows_b = static_cast<int>(M);
+  p.red = static_cast<int>(N);
+  p.K = K;
+  p.packed = w_packed;
+  p.gamma = gamma;
+  p.out = dX;
+  p.ldo = K;
+  p.err = err;
+  return launch_gemm<Op::Dx>(mb, unused, unused, p, s);
+}
+
+cudaError_t launch_backward_dw(const void* dY, const int8_t* xq, const float* sx, int64_t M, int64_t N, int64_t K,
+                               void* dW, int dw_is_f32, int accumulate, int* err, cudaStream_t s) {
+  if (M == 0) {
+    const int64_t n = N * K;
+    zero_dw_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, s>>>(dW, n, dw_is_f32, accumulate);
+    return cudaGetLastError();
+  }
+  CUtensorMap mb{}, msrc{}, msx{};
+  if (!make_map_2d(&mb, dY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, N, M, N * 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map_2d(&msrc, xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, K, M, K, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map_1d(&msx, sx, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, M, 64))
+    return cudaErrorInvalidValue;
+  GemmParams p{};
+  p.rows_a = static_cast<int>(K);
+  p.rows_b = static_cast<int>(N);
+  p.red = static_cast<int>(M);
+  p.K = K;
+  p.out = dW;
+  p.ldo = K;
+  p.out_f32 = dw_is_f32;
+  p.accumulate = accumulate;
+  p.err = err;
+  return launch_gemm<Op::Dw>(mb, msrc, msx, p, s);
+}
+
+}  // namespace bl

@@ -1,0 +1,286 @@
+// S1 and S2 of the BitLinear hot path on sm_100a: absmean ternarisation with
+// 2-bit packing, and per-token absmax INT8 activation quantisation.
+//
+// Both are HBM-bound streaming passes: 16-byte vector loads, one pass over
+// the data per output, no intermediate tensors in device memory.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdint>
+
+#include "bl_device.cuh"
+#include "bl_internal.h"
+
+namespace bl {
+namespace {
+
+constexpr int kQuantThreads = 256;
+// Upper bound on pass-A blocks: four 256-thread blocks per SM on a 148-SM
+// B200. A fixed constant, so the fp64 reduction tree is the same on any GPU.
+constexpr int kMaxPartials = 592;
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// A "group" is 16 consecutive elements of the flattened [N,K] tensor. Its 16
+// codes pack into one 32-bit word: element i of the group sits at bits 2i..2i+1
+// (little-endian, so byte j of the word holds elements 4j..4j+3, LSB first).
+template <bool kF32>
+struct Group {
+  static constexpr int kVecs = kF32 ? 4 : 2;  // uint4 per 16 elements
+  uint4 v[kVecs];
+
+  __device__ __forceinline__ void load(const uint4* __restrict__ base, int64_t g) {
+#pragma unroll
+    for (int i = 0; i < kVecs; ++i) v[i] = __ldg(base + g * kVecs + i);
+  }
+
+  // Element i (0..15) as fp32.
+  __device__ __forceinline__ float elem(int i) const {
+    if constexpr (kF32) {
+      const uint4& q = v[i >> 2];
+      const uint32_t w = (i & 3) == 0 ? q.x : (i & 3) == 1 ? q.y : (i & 3) == 2 ? q.z : q.w;
+      return __uint_as_float(w);
+    } else {
+      const uint4& q = v[i >> 3];
+      const int j = (i & 7) >> 1;
+      const uint32_t w = j == 0 ? q.x : j == 1 ? q.y : j == 2 ? q.z : q.w;
+      return (i & 1) ? bf16_hi(w) : bf16_lo(w);
+    }
+  }
+};
+
+// ---------------------------------------------------------------- S1 pass A
+// partials[b] = sum of |w| over block b's contiguous range of groups, fp64,
+// each thread summing its groups in order, then a fixed shuffle/smem tree.
+template <bool kF32>
+__global__ void __launch_bounds__(kQuantThreads) absmean_partials_kernel(const uint4* __restrict__ W,
+                                                                         int64_t ngroups, int64_t per_block,
+                                                                         double* __restrict__ partials) {
+  const int64_t g0 = static_cast<int64_t>(blockIdx.x) * per_block;
+  const int64_t g1 = min(g0 + per_block, ngroups);
+  double acc = 0.0;
+  int64_t g = g0 + threadIdx.x;
+  for (; g + kQuantThreads < g1; g += 2 * kQuantThreads) {
+    Group<kF32> a, b;
+    a.load(W, g);
+    b.load(W, g + kQuantThreads);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) acc = __dadd_rn(acc, static_cast<double>(fabsf(a.elem(i))));
+#pragma unroll
+    for (int i = 0; i < 16; ++i) acc = __dadd_rn(acc, static_cast<double>(fabsf(b.elem(i))));
+  }
+  if (g < g1) {
+    Group<kF32> a;
+    a.load(W, g);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) acc = __dadd_rn(acc, static_cast<double>(fabsf(a.elem(i))));
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) acc = __dadd_rn(acc, __shfl_xor_sync(0xffffffffu, acc, off));
+  __shared__ double warp_sums[kQuantThreads / 32];
+  if ((threadIdx.x & 31) == 0) warp_sums[threadIdx.x >> 5] = acc;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double s = 0.0;
+#pragma unroll
+    for (int w = 0; w < kQuantThreads / 32; ++w) s = __dadd_rn(s, warp_sums[w]);
+    partials[blockIdx.x] = s;
+  }
+}
+
+// ---------------------------------------------------------------- S1 pass B
+// Every block reduces the partials in the same fixed order (so all blocks hold
+// the same gamma), then writes the codes of its range of groups.
+//
+// Code rule: code = clamp(rint_half_even(fp32(w / gamma)), -1, 1) is nonzero
+// exactly when fp32(|w| / gamma) > 0.5, i.e. when the exact quotient exceeds
+// 0.5 + 2^-25 (the midpoint between 0.5 and the next float, which rounds to
+// the even 0.5). With T = gamma * (0.5 + 2^-25) computed exactly in fp64 and
+// thr the largest float <= T, that is |w| > thr: one compare, no division.
+template <bool kF32>
+__global__ void __launch_bounds__(kQuantThreads) ternarize_pack_kernel(const uint4* __restrict__ W,
+                                                                       int64_t ngroups, int64_t per_block,
+                                                                       const double* __restrict__ partials,
+                                                                       int nparts, int64_t numel,
+                                                                       uint32_t* __restrict__ packed,
+                                                                       float* __restrict__ gamma_out) {
+  __shared__ float s_thr;
+  if (threadIdx.x < 32) {
+    double s = 0.0;
+    for (int i = threadIdx.x; i < nparts; i += 32) s = __dadd_rn(s, partials[i]);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) s = __dadd_rn(s, __shfl_xor_sync(0xffffffffu, s, off));
+    if (threadIdx.x == 0) {
+      const double mean = __ddiv_rn(s, static_cast<double>(numel));
+      const float gamma = fmaxf(__double2float_rn(mean), 1e-5f);
+      const double t = __dmul_rn(static_cast<double>(gamma), 0.5 + 0x1p-25);
+      s_thr = __double2float_rd(t);
+      if (blockIdx.x == 0) *gamma_out = gamma;
+    }
+  }
+  __syncthreads();
+  const float thr = s_thr;
+  const int64_t g0 = static_cast<int64_t>(blockIdx.x) * per_block;
+  const int64_t g1 = min(g0 + per_block, ngroups);
+  for (int64_t g = g0 + threadIdx.x; g < g1; g += kQuantThreads) {
+    Group<kF32> a;
+    a.load(W, g);
+    uint32_t word = 0;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const float w = a.elem(i);
+      const uint32_t nz = fabsf(w) > thr ? 1u : 0u;
+      const uint32_t neg = __float_as_uint(w) >> 31;
+      word |= (nz * (1u | (neg << 1))) << (2 * i);  // 00 = 0, 01 = +1, 11 = -1
+    }
+    packed[g] = word;
+  }
+}
+
+// ---------------------------------------------------------------- S2
+// One warp per token. The row stays in registers between the absmax and the
+// quantisation (VPL 16-byte vectors per lane, rows up to 256 * VPL elements).
+//
+// q = rint_half_even(fp32(x * inv)) uses the 1.5 * 2^23 shifter: adding it
+// rounds |x * inv| <= 127.0001 to an integer (ties to even), and the low byte
+// of the sum's bit pattern is that integer in two's complement. |q| <= 127
+// holds without a clamp because |x| <= a and inv = fp32(127 / a).
+__device__ __forceinline__ uint32_t quant4(float a, float b, float c, float d, float inv) {
+  const float kShift = 12582912.0f;  // 1.5 * 2^23
+  const uint32_t qa = __float_as_uint(__fadd_rn(__fmul_rn(a, inv), kShift));
+  const uint32_t qb = __float_as_uint(__fadd_rn(__fmul_rn(b, inv), kShift));
+  const uint32_t qc = __float_as_uint(__fadd_rn(__fmul_rn(c, inv), kShift));
+  const uint32_t qd = __float_as_uint(__fadd_rn(__fmul_rn(d, inv), kShift));
+  const uint32_t ab = __byte_perm(qa, qb, 0x0040);
+  const uint32_t cd = __byte_perm(qc, qd, 0x0040);
+  return __byte_perm(ab, cd, 0x5410);
+}
+
+__device__ __forceinline__ uint2 quant8(const uint4& v, float inv) {
+  uint2 r;
+  r.x = quant4(bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y), inv);
+  r.y = quant4(bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w), inv);
+  return r;
+}
+
+__device__ __forceinline__ float absmax8(const uint4& v, float m) {
+  m = fmaxf(m, fabsf(bf16_lo(v.x)));
+  m = fmaxf(m, fabsf(bf16_hi(v.x)));
+  m = fmaxf(m, fabsf(bf16_lo(v.y)));
+  m = fmaxf(m, fabsf(bf16_hi(v.y)));
+  m = fmaxf(m, fabsf(bf16_lo(v.z)));
+  m = fmaxf(m, fabsf(bf16_hi(v.z)));
+  m = fmaxf(m, fabsf(bf16_lo(v.w)));
+  m = fmaxf(m, fabsf(bf16_hi(v.w)));
+  return m;
+}
+
+__device__ __forceinline__ float warp_max(float m) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+  return m;
+}
+
+constexpr int kActRowsPerBlock = 4;
+
+template <int VPL>
+__global__ void __launch_bounds__(32 * kActRowsPerBlock) act_quant_kernel(const uint4* __restrict__ x, int64_t M,
+                                                                          int nv, int8_t* __restrict__ xq,
+                                                                          float* __restrict__ sx) {
+  const int lane = threadIdx.x & 31;
+  const int64_t m = static_cast<int64_t>(blockIdx.x) * kActRowsPerBlock + (threadIdx.x >> 5);
+  if (m >= M) return;
+  const uint4* row = x + m * nv;
+  uint4 v[VPL];
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) {
+    const int j = lane + 32 * i;
+    v[i] = j < nv ? __ldg(row + j) : make_uint4(0u, 0u, 0u, 0u);
+  }
+  float amax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) amax = absmax8(v[i], amax);
+  const float a = fmaxf(warp_max(amax), 1e-5f);
+  const float inv = __fdiv_rn(127.0f, a);
+  if (lane == 0) sx[m] = __fdiv_rn(a, 127.0f);
+  uint2* out = reinterpret_cast<uint2*>(xq + m * static_cast<int64_t>(nv) * 8);
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) {
+    const int j = lane + 32 * i;
+    if (j < nv) out[j] = quant8(v[i], inv);
+  }
+}
+
+// Rows longer than 8192 elements: absmax pass, then a second read (from L2).
+__global__ void __launch_bounds__(32 * kActRowsPerBlock) act_quant_long_kernel(const uint4* __restrict__ x,
+                                                                               int64_t M, int nv,
+                                                                               int8_t* __restrict__ xq,
+                                                                               float* __restrict__ sx) {
+  const int lane = threadIdx.x & 31;
+  const int64_t m = static_cast<int64_t>(blockIdx.x) * kActRowsPerBlock + (threadIdx.x >> 5);
+  if (m >= M) return;
+  const uint4* row = x + m * nv;
+  float amax = 0.0f;
+  for (int j = lane; j < nv; j += 32) amax = absmax8(__ldg(row + j), amax);
+  const float a = fmaxf(warp_max(amax), 1e-5f);
+  const float inv = __fdiv_rn(127.0f, a);
+  if (lane == 0) sx[m] = __fdiv_rn(a, 127.0f);
+  uint2* out = reinterpret_cast<uint2*>(xq + m * static_cast<int64_t>(nv) * 8);
+  for (int j = lane; j < nv; j += 32) out[j] = quant8(__ldg(row + j), inv);
+}
+
+}  // namespace
+
+int weight_partials_count(int64_t numel) {
+  const int64_t ngroups = numel / 16;
+  const int64_t want = (ngroups + kQuantThreads - 1) / kQuantThreads;
+  return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(kMaxPartials, want)));
+}
+
+cudaError_t launch_quantize_weight(const void* W, int w_is_f32, int64_t N, int64_t K, uint8_t* packed,
+                                   float* gamma, double* partials, cudaStream_t s) {
+  const int64_t numel = N * K;  // multiple of 32
+  const int64_t ngroups = numel / 16;
+  const int nparts = weight_partials_count(numel);
+  const int64_t per_block = (ngroups + nparts - 1) / nparts;
+  const uint4* w = static_cast<const uint4*>(W);
+  uint32_t* out = reinterpret_cast<uint32_t*>(packed);
+  if (w_is_f32) {
+    absmean_partials_kernel<true><<<nparts, kQuantThreads, 0, s>>>(w, ngroups, per_block, partials);
+    ternarize_pack_kernel<true>
+        <<<nparts, kQuantThreads, 0, s>>>(w, ngroups, per_block, partials, nparts, numel, out, gamma);
+  } else {
+    absmean_partials_kernel<false><<<nparts, kQuantThreads, 0, s>>>(w, ngroups, per_block, partials);
+    ternarize_pack_kernel<false>
+        <<<nparts, kQuantThreads, 0, s>>>(w, ngroups, per_block, partials, nparts, numel, out, gamma);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quantize_act(const void* x, int64_t M, int64_t K, int8_t* xq, float* sx, cudaStream_t s) {
+  if (M == 0) return cudaSuccess;
+  const int nv = static_cast<int>(K / 8);
+  const unsigned grid = static_cast<unsigned>((M + kActRowsPerBlock - 1) / kActRowsPerBlock);
+  const dim3 block(32 * kActRowsPerBlock);
+  const uint4* xv = static_cast<const uint4*>(x);
+  const int per_lane = (nv + 31) / 32;
+  if (per_lane <= 1)
+    act_quant_kernel<1><<<grid, block, 0, s>>>(xv, M, nv, xq, sx);
+  else if (per_lane <= 2)
+    act_quant_kernel<2><<<grid, block, 0, s>>>(xv, M, nv, xq, sx);
+  else if (per_lane <= 4)
+    act_quant_kernel<4><<<grid, block, 0, s>>>(xv, M, nv, xq, sx);
+  else if (per_lane <= 8)
+    act_quant_kernel<8><<<grid, block, 0, s>>>(xv, M, nv, xq, sx);
+  else if (per_lane <= 16)
+    act_quant_kernel<16><<<grid, block, 0, s>>>(xv, M, nv, xq, sx);
+  else if (per_lane <= 32)
+    act_quant_kernel<32><<<grid, block, 0, s>>>(xv, M, nv, xq, sx);
+  else
+    act_quant_long_kernel<<<grid, block, 0, s>>>(xv, M, nv, xq, sx);
+  return cudaGetLastError();
+}
+
+}  // namespace bl

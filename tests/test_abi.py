@@ -1,0 +1,75 @@
+"""The C ABI library loads and exports every symbol include/bitlinear.h
+declares; host-side argument validation works without a GPU."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from ternary_weight_quantization_b200 import bitlinear as b
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "bitlinear.h")
+
+
+def _declared_symbols():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(bl_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol():
+    lib = b.load_library()
+    declared = _declared_symbols()
+    assert len(declared) >= 10
+    for name in declared:
+        assert hasattr(lib, name), name
+    assert set(declared) == set(b.SIGNATURES), "binding signatures drift from the header"
+
+
+def test_version_and_status_strings():
+    lib = b.load_library()
+    assert lib.bl_version() >> 16 == 1
+    for code, name in b.STATUS.items():
+        assert lib.bl_status_string(code).decode() == name
+
+
+def test_workspace_size():
+    assert b.bl_quantize_weight_workspace_size(0, 32) == 0
+    assert b.bl_quantize_weight_workspace_size(256, 128) == 8 * 8       # 2048 groups -> 8 partials
+    assert b.bl_quantize_weight_workspace_size(6912, 2560) == 592 * 8   # capped
+
+
+FAKE = ctypes.c_void_p(0x10000)        # never dereferenced: validation fails first
+MISALIGNED = ctypes.c_void_p(0x10008)
+
+
+@pytest.mark.parametrize("call,expect", [
+    (lambda L: L.bl_quantize_act(FAKE, 4, 33, FAKE, FAKE, None), 2),          # K % 32
+    (lambda L: L.bl_quantize_act(FAKE, 4, 0, FAKE, FAKE, None), 2),
+    (lambda L: L.bl_quantize_act(None, 4, 64, FAKE, FAKE, None), 1),          # null
+    (lambda L: L.bl_quantize_act(MISALIGNED, 4, 64, FAKE, FAKE, None), 4),    # alignment
+    (lambda L: L.bl_quantize_act(FAKE, -1, 64, FAKE, FAKE, None), 1),
+    (lambda L: L.bl_quantize_weight(FAKE, 7, 8, 64, FAKE, FAKE, FAKE, 1 << 20, None), 3),  # dtype
+    (lambda L: L.bl_quantize_weight(FAKE, 0, 8, 64, FAKE, FAKE, FAKE, 0, None), 8),        # workspace
+    (lambda L: L.bl_quantize_weight(FAKE, 0, 0, 64, FAKE, FAKE, FAKE, 64, None), 1),
+    (lambda L: L.bl_forward(FAKE, FAKE, FAKE, FAKE, 4, 8, 48, FAKE, None, None), 2),
+    (lambda L: L.bl_forward(FAKE, FAKE, None, FAKE, 4, 8, 64, FAKE, None, None), 1),
+    (lambda L: L.bl_forward(FAKE, FAKE, FAKE, FAKE, 4, 8, 64, FAKE, MISALIGNED, None), 4),
+    (lambda L: L.bl_backward(FAKE, FAKE, FAKE, FAKE, FAKE, 4, 12, 64, FAKE, FAKE, 0, 0, None), 2),  # N % 8
+    (lambda L: L.bl_backward(FAKE, FAKE, FAKE, FAKE, FAKE, 4, 16, 64, FAKE, FAKE, 9, 0, None), 3),
+    (lambda L: L.bl_backward(FAKE, FAKE, FAKE, None, FAKE, 4, 16, 64, FAKE, None, 0, 0, None), 1),
+    (lambda L: L.bl_export_weights(FAKE, FAKE, 4, 64, None, FAKE, None), 1),
+])
+def test_host_validation_without_gpu(call, expect):
+    lib = b.load_library()
+    assert call(lib) == expect
+    assert lib.bl_last_error_message().decode()
+
+
+def test_empty_work_is_ok_without_gpu():
+    lib = b.load_library()
+    assert lib.bl_quantize_act(None, 0, 64, None, None, None) == 0
+    assert lib.bl_forward(None, None, None, None, 0, 8, 64, None, None, None) == 0
+    assert lib.bl_backward(None, None, None, None, None, 4, 16, 64, None, None, 0, 0, None) == 0
