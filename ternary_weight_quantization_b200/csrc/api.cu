@@ -67,7 +67,10 @@ bl_status check_k(int64_t K) {
 
 bl_status cuda_status(cudaError_t e, const char* what) {
   if (e == cudaSuccess) return BL_OK;
-  return fail(BL_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+  const char* detail = bl::launch_detail();
+  bl_status s = fail(BL_ERR_CUDA, "%s: %s%s%s", what, cudaGetErrorString(e), detail[0] ? "; " : "", detail);
+  bl::clear_launch_detail();
+  return s;
 }
 
 }  // namespace

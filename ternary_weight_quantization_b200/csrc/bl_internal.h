@@ -35,4 +35,8 @@ cudaError_t launch_backward_dw(const void* dY, const int8_t* xq, const float* sx
 // Number of SMs of the current device (cached per device).
 int device_sm_count();
 
+// Detail of the last host-side launch failure on this thread ("" if none).
+const char* launch_detail();
+void clear_launch_detail();
+
 }  // namespace bl

@@ -33,6 +33,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <cstdarg>
 #include <cstdint>
 #include <cstdio>
 #include <mutex>
@@ -298,7 +299,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int j = 0; j < 4; ++j) tma_load_2d(&map_b, &load_full[stage], sB + j * 8192, b0 + 64 * j, r0);
             tma_load_2d(&map_src, &load_full[stage], sSrc, a0, r0);
-            tma_load_1d(&map_sx, &load_full[stage], smem + L::kOffSx + stage * C::kSxBytes, r0);
+            tma_load_2d(&map_sx, &load_full[stage], smem + L::kOffSx + stage * C::kSxBytes, r0, 0);
           }
         }
         if constexpr (op == Op::Fwd) {
@@ -596,6 +597,15 @@ __global__ void zero_dw_kernel(void* out, int64_t n, int out_f32, int accumulate
 
 // ---------------------------------------------------------------- host side
 
+thread_local char g_launch_detail[160] = "";
+
+void set_launch_detail(const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_launch_detail, sizeof(g_launch_detail), fmt, ap);
+  va_end(ap);
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   static std::once_flag once;
@@ -610,26 +620,24 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
 }
 
 bool make_map_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64_t inner, uint64_t outer,
-                 uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle sw) {
+                 uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle sw,
+                 const char* what) {
   auto enc = get_encode_fn();
-  if (!enc) return false;
+  if (!enc) {
+    set_launch_detail("cuTensorMapEncodeTiled is unavailable (%s)", what);
+    return false;
+  }
   const cuuint64_t dims[2] = {inner, outer};
   const cuuint64_t strides[1] = {row_bytes};
   const cuuint32_t box[2] = {box_inner, box_outer};
   const cuuint32_t estr[2] = {1, 1};
-  return enc(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
-             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-bool make_map_1d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64_t n, uint32_t box) {
-  auto enc = get_encode_fn();
-  if (!enc) return false;
-  const cuuint64_t dims[1] = {n};
-  const cuuint32_t boxd[1] = {box};
-  const cuuint32_t estr[1] = {1};
-  return enc(m, dt, 1, const_cast<void*>(base), dims, nullptr, boxd, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-             CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  const CUresult r = enc(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    set_launch_detail("tensor map for %s rejected (CUresult %d)", what, static_cast<int>(r));
+    return false;
+  }
+  return true;
 }
 
 template <Op op>
@@ -656,6 +664,10 @@ cudaError_t launch_gemm(const CUtensorMap& mb, const CUtensorMap& msrc, const CU
 
 }  // namespace
 
+const char* launch_detail() { return g_launch_detail; }
+
+void clear_launch_detail() { g_launch_detail[0] = 0; }
+
 int device_sm_count() {
   static int cached[64];
   static bool init[64] = {};
@@ -676,7 +688,7 @@ cudaError_t launch_forward(const int8_t* xq, const float* sx, const uint8_t* w_p
                            cudaStream_t s) {
   if (M == 0 || N == 0) return cudaSuccess;
   CUtensorMap mb{}, unused{};
-  if (!make_map_2d(&mb, xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, K, M, K, 128, BN, CU_TENSOR_MAP_SWIZZLE_128B))
+  if (!make_map_2d(&mb, xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, K, M, K, 128, BN, CU_TENSOR_MAP_SWIZZLE_128B, "xq"))
     return cudaErrorInvalidValue;
   GemmParams p{};
   p.rows_a = static_cast<int>(N);
@@ -697,7 +709,8 @@ cudaError_t launch_backward_dx(const void* dY, const uint8_t* w_packed, const fl
                                int64_t K, void* dX, int* err, cudaStream_t s) {
   if (M == 0) return cudaSuccess;
   CUtensorMap mb{}, unused{};
-  if (!make_map_2d(&mb, dY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, N, M, N * 2, 64, BN, CU_TENSOR_MAP_SWIZZLE_128B))
+  if (!make_map_2d(&mb, dY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, N, M, N * 2, 64, BN, CU_TENSOR_MAP_SWIZZLE_128B,
+                   "dY (dX)"))
     return cudaErrorInvalidValue;
   GemmParams p{};
   p.rows_a = static_cast<int>(K);
@@ -720,9 +733,13 @@ cudaError_t launch_backward_dw(const void* dY, const int8_t* xq, const float* sx
     return cudaGetLastError();
   }
   CUtensorMap mb{}, msrc{}, msx{};
-  if (!make_map_2d(&mb, dY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, N, M, N * 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_map_2d(&msrc, xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, K, M, K, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_map_1d(&msx, sx, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, M, 64))
+  // s_x as a one-row 2D tensor: [1][M] floats, row pitch rounded up to 16 bytes
+  const uint64_t sx_pitch = ((static_cast<uint64_t>(M) * 4 + 15) / 16) * 16;
+  if (!make_map_2d(&mb, dY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, N, M, N * 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B,
+                   "dY (dW)") ||
+      !make_map_2d(&msrc, xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, K, M, K, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B, "xq (dW)") ||
+      !make_map_2d(&msx, sx, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, M, 1, sx_pitch, 64, 1, CU_TENSOR_MAP_SWIZZLE_NONE,
+                   "sx (dW)"))
     return cudaErrorInvalidValue;
   GemmParams p{};
   p.rows_a = static_cast<int>(K);
