@@ -16,7 +16,7 @@
  *   - Every tensor argument is a DEVICE pointer unless its name starts with
  *     host_. The caller allocates and owns every buffer; the library never
  *     allocates device memory and keeps no state except one error word per
- *     device.
+ *     device (and the fixed scratch array of bl_quantize_weight_noalloc).
  *   - Tensors are dense, row-major, and 16-byte aligned at their base.
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
  *     stream). All work is enqueued asynchronously on it; nothing here
@@ -100,6 +100,34 @@ size_t bl_quantize_weight_workspace_size(int64_t N, int64_t K);
 bl_status bl_quantize_weight(const void* W, bl_dtype w_dtype, int64_t N, int64_t K,
                              uint8_t* w_packed, float* gamma,
                              void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * bl_quantize_weight without a workspace. The pages have no counterpart to
+ * this call; it exists for callers that cannot allocate device memory --
+ * plugin hosts that hand the library only the input and output buffers they
+ * own, and runtimes whose device memory is a fixed pool reserved up front --
+ * and so cannot pass the workspace bl_quantize_weight asks for.
+ *
+ * It computes exactly what bl_quantize_weight computes (same kernels, same
+ * bit-identical outputs) and calls no allocator. Its fp64 partial sums go to
+ * a fixed array inside the library of 592 doubles (4736 bytes), enough for a
+ * tensor of any size; each GPU that loads the library keeps that array until
+ * the process exits. A request that would need more scratch than the array
+ * holds returns BL_ERR_WORKSPACE.
+ *
+ * The first call on each device looks up the array's device address (a
+ * runtime query, done with that device current) and caches it; make that
+ * first call before any stream capture. All calls share the one array and
+ * nothing in it needs to start at zero (every call overwrites the part it
+ * reads), but two calls whose kernels overlap on the GPU -- on different
+ * streams of one device without ordering between them -- race on it and may
+ * produce wrong codes: order them on one stream or with events.
+ *
+ * Arguments, outputs and errors: as bl_quantize_weight, without the
+ * workspace pair.
+ */
+bl_status bl_quantize_weight_noalloc(const void* W, bl_dtype w_dtype, int64_t N, int64_t K,
+                                     uint8_t* w_packed, float* gamma, void* stream);
 
 /*
  * S2 -- per-token absmax INT8 quantisation ("1BitTraining.md",

@@ -35,6 +35,7 @@ SIGNATURES = {
     "bl_last_error_message": (ctypes.c_char_p, []),
     "bl_quantize_weight_workspace_size": (_SZ, [_I64, _I64]),
     "bl_quantize_weight": (_I32, [_VP, _I32, _I64, _I64, _VP, _VP, _VP, _SZ, _VP]),
+    "bl_quantize_weight_noalloc": (_I32, [_VP, _I32, _I64, _I64, _VP, _VP, _VP]),
     "bl_quantize_act": (_I32, [_VP, _I64, _I64, _VP, _VP, _VP]),
     "bl_forward": (_I32, [_VP, _VP, _VP, _VP, _I64, _I64, _I64, _VP, _VP, _VP]),
     "bl_backward": (_I32, [_VP, _VP, _VP, _VP, _VP, _I64, _I64, _I64, _VP, _VP, _I32, _I32, _VP]),

@@ -121,6 +121,26 @@ bl_status bl_quantize_weight(const void* W, bl_dtype w_dtype, int64_t N, int64_t
                      "bl_quantize_weight launch");
 }
 
+bl_status bl_quantize_weight_noalloc(const void* W, bl_dtype w_dtype, int64_t N, int64_t K, uint8_t* w_packed,
+                                     float* gamma, void* stream) {
+  g_msg[0] = 0;
+  if (N < 1) return fail(BL_ERR_INVALID_ARG, "N=%lld must be >= 1", (long long)N);
+  if (bl_status s = check_k(K)) return s;
+  if (w_dtype != BL_BF16 && w_dtype != BL_F32) return fail(BL_ERR_DTYPE, "w_dtype %d", (int)w_dtype);
+  if (!W || !w_packed || !gamma) return fail(BL_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(W) || !aligned16(w_packed) || !aligned16(gamma))
+    return fail(BL_ERR_ALIGNMENT, "W, w_packed and gamma must be 16-byte aligned");
+  const size_t need = bl_quantize_weight_workspace_size(N, K);
+  if (need > bl::noalloc_scratch_bytes())
+    return fail(BL_ERR_WORKSPACE, "needs %zu bytes of scratch; the built-in scratch holds %zu", need,
+                bl::noalloc_scratch_bytes());
+  int* err = nullptr;
+  if (bl_status s = current_device(&err)) return s;
+  return cuda_status(bl::launch_quantize_weight_noalloc(W, w_dtype == BL_F32, N, K, w_packed, gamma,
+                                                        static_cast<cudaStream_t>(stream)),
+                     "bl_quantize_weight_noalloc launch");
+}
+
 bl_status bl_quantize_act(const void* x, int64_t M, int64_t K, int8_t* xq, float* sx, void* stream) {
   g_msg[0] = 0;
   if (M < 0) return fail(BL_ERR_INVALID_ARG, "M=%lld must be >= 0", (long long)M);

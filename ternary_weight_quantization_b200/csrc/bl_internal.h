@@ -18,6 +18,12 @@ int weight_partials_count(int64_t numel);
 cudaError_t launch_quantize_weight(const void* W, int w_is_f32, int64_t N, int64_t K, uint8_t* packed,
                                    float* gamma, double* partials, cudaStream_t s);
 
+// Same two passes with the partial sums in a fixed device array
+// (g_noalloc_partials in k_quant.cu) instead of a caller workspace.
+cudaError_t launch_quantize_weight_noalloc(const void* W, int w_is_f32, int64_t N, int64_t K, uint8_t* packed,
+                                           float* gamma, cudaStream_t s);
+size_t noalloc_scratch_bytes();
+
 // ---- S2: per-token absmax INT8
 cudaError_t launch_quantize_act(const void* x, int64_t M, int64_t K, int8_t* xq, float* sx, cudaStream_t s);
 

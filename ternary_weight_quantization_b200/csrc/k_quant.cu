@@ -8,6 +8,7 @@
 
 #include <algorithm>
 #include <cstdint>
+#include <mutex>
 
 #include "bl_device.cuh"
 #include "bl_internal.h"
@@ -233,6 +234,11 @@ __global__ void __launch_bounds__(32 * kActRowsPerBlock) act_quant_long_kernel(c
 
 }  // namespace
 
+// Fixed device scratch for bl_quantize_weight_noalloc: room for the largest
+// number of fp64 partial sums pass A ever writes (kMaxPartials), 4736 bytes.
+// Every GPU that loads the library holds this array until the process exits.
+static __device__ __align__(256) double g_noalloc_partials[kMaxPartials];
+
 int weight_partials_count(int64_t numel) {
   const int64_t ngroups = numel / 16;
   const int64_t want = (ngroups + kQuantThreads - 1) / kQuantThreads;
@@ -257,6 +263,39 @@ cudaError_t launch_quantize_weight(const void* W, int w_is_f32, int64_t N, int64
         <<<nparts, kQuantThreads, 0, s>>>(w, ngroups, per_block, partials, nparts, numel, out, gamma);
   }
   return cudaGetLastError();
+}
+
+size_t noalloc_scratch_bytes() { return sizeof(g_noalloc_partials); }
+
+// Device address of g_noalloc_partials on the current device. Host code only
+// holds a stand-in for the array's name, so the address is looked up once per
+// device (with that device current) and cached.
+static cudaError_t noalloc_scratch_ptr(double** out) {
+  static double* ptrs[64] = {};
+  static std::mutex mu;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!ptrs[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_partials);
+    if (e != cudaSuccess) return e;
+    ptrs[dev] = static_cast<double*>(p);
+  }
+  *out = ptrs[dev];
+  return cudaSuccess;
+}
+
+cudaError_t launch_quantize_weight_noalloc(const void* W, int w_is_f32, int64_t N, int64_t K, uint8_t* packed,
+                                           float* gamma, cudaStream_t s) {
+  if (static_cast<size_t>(weight_partials_count(N * K)) * sizeof(double) > sizeof(g_noalloc_partials))
+    return cudaErrorInvalidValue;
+  double* scratch = nullptr;
+  const cudaError_t e = noalloc_scratch_ptr(&scratch);
+  if (e != cudaSuccess) return e;
+  return launch_quantize_weight(W, w_is_f32, N, K, packed, gamma, scratch, s);
 }
 
 cudaError_t launch_quantize_act(const void* x, int64_t M, int64_t K, int8_t* xq, float* sx, cudaStream_t s) {
