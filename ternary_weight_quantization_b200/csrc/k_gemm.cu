@@ -4,30 +4,37 @@
 // dW = dY^T . x_hat, with W_hat and x_hat rebuilt from the saved 2-bit and
 // INT8 state).
 //
-// One persistent, warp-specialised kernel template serves all three:
+// One persistent, warp-specialised CTA-pair kernel template serves all three:
 //
-//   D[i][j] = sum_r A[i][r] * B[j][r]        (tcgen05.mma, accumulator in TMEM)
+//   D[i][j] = sum_r A[i][r] * B[j][r]        (tcgen05.mma cta_group::2, TMEM accumulators)
 //   out[j][i] = epilogue(D[i][j])            (transposed store)
 //
-//   op   A (128-row tile, REBUILT in smem)      B (256-row tile, TMA)        r
+//   op   A (REBUILT in smem)                    B (TMA)                       r
 //   Fwd  codes[n][k] int8, K-major              xq[m][k] int8, K-major        k
 //   Dx   codes^T[k][n] bf16 {-1,0,1}, MN-major  dY[m][n] bf16, K-major        n
 //   Dw   x_hat^T[k][m] bf16, MN-major           dY^T[n][m] bf16, MN-major     m
 //
-// The ternary / INT8 operand is always A: its rebuild writes a 128-row tile
-// per stage into shared memory (never to HBM), while the wider 256-row
-// operand streams in by TMA. The output tile is transposed through shared
-// memory so global stores stay row-contiguous.
+// A pair tile is 256 A rows x BN B rows. Each CTA of the pair rebuilds its own
+// 128 A rows from the staged 2-bit / INT8 source (never written to HBM) and
+// TMA-loads its own BN/2 B rows; the leader CTA issues one M=256 MMA that
+// reads both CTAs' shared memory and accumulates 128 rows into each CTA's
+// TMEM. Splitting both operands across the pair halves the B traffic per SM
+// compared with a single-CTA 128 x BN tile. No TMA multicast is used.
 //
-// Warp roles (320 threads):
-//   warp 0    loads: TMA for B (and Dw's q/s_x), cp.async for packed codes
-//   warp 1    TMEM allocation (2 x 256 columns) and tcgen05.mma issue
-//   warps 2-5 rebuild A from the staged 2-bit / INT8 source
+// Warp roles (320 threads per CTA):
+//   warp 0    loads: TMA for B, for Dw's q / s_x and for the packed codes
+//             (cp.async for the codes when K % 64 != 0: their rows are then not
+//             16-byte aligned, which a tensor map requires)
+//   warp 1    TMEM allocation (2 x 256 columns, pair-wide); in the leader CTA
+//             also tcgen05.mma issue
+//   warps 2-5 rebuild A from the staged source
 //   warps 6-9 epilogue: TMEM -> registers -> smem (transpose) -> global
-// Shared-memory stages form a ring guarded by mbarriers; two TMEM
-// accumulators let the epilogue of one tile overlap the MMAs of the next.
-// Every wait is bounded: on expiry the CTA records a timeout in the device
-// error word, drains what it has in flight, frees TMEM and exits.
+// Barriers: src_full (per CTA: staged source landed), load_full and a_full
+// (leader: both CTAs' B bytes landed / both CTAs' A rebuilt), empty and
+// tmem_full (both CTAs, completed by multicast tcgen05.commit), tmem_empty
+// (leader: both CTAs' epilogues drained a TMEM buffer). Every wait is
+// bounded: on expiry a CTA records a timeout in the device error word, tells
+// its peer, drains what it has in flight, frees TMEM and exits.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -36,6 +43,7 @@
 #include <cstdarg>
 #include <cstdint>
 #include <cstdio>
+#include <cstdlib>
 #include <mutex>
 
 #include "bl_device.cuh"
@@ -52,74 +60,77 @@ constexpr int kNumRebuildWarps = 4;
 constexpr int kWarpEpi0 = 6;
 constexpr int kNumEpiWarps = 4;
 
-constexpr int BM = 128;            // A rows per tile (UMMA M)
-constexpr int BN = 256;            // B rows per tile (UMMA N)
-constexpr uint32_t kTmemCols = 512;  // two BN-column accumulators
+constexpr int BM = 128;              // A rows per CTA; a pair covers 2 * BM
+constexpr uint32_t kTmemCols = 512;  // two accumulators at columns 0 and 256
 constexpr int kEpiStageBytes = 32 * 32 * 4;  // per epilogue warp
+constexpr int kSmemLimit = 232448;           // per-CTA dynamic shared memory on sm_100
 
 enum class Op { Fwd, Dx, Dw };
 
-template <Op op>
+template <Op op, int BN>
 struct Cfg;
 
-template <>
-struct Cfg<Op::Fwd> {
-  static constexpr int kBlockR = 128;           // reduction elements (k) per stage
-  static constexpr int kUmmaK = 32;             // kind::i8: 32 bytes of K per MMA
-  static constexpr int kABytes = BM * 128;      // 128 rows x 128 int8
-  static constexpr int kBBytes = BN * 128;      // 256 rows x 128 int8
-  static constexpr int kSrcBytes = BM * 32;     // packed codes: 128 rows x 32 bytes
+// Forward: reduction over k in blocks of 128 bytes; kind::i8 consumes 32 k per MMA.
+template <int BN>
+struct Cfg<Op::Fwd, BN> {
+  static constexpr int kBlockR = 128;
+  static constexpr int kUmmaK = 32;
+  static constexpr int kABytes = BM * 128;         // 128 rows x 128 int8
+  static constexpr int kBBytes = (BN / 2) * 128;   // BN/2 rows x 128 int8
+  static constexpr int kSrcBytes = BM * 32;        // packed: 128 rows x 32 bytes
   static constexpr int kSxBytes = 0;
-  static constexpr int kStages = 4;
-  static constexpr uint32_t kIdesc = make_idesc(2 /*s32*/, 1 /*s8*/, 0, 0, BM, BN);
-  static constexpr uint32_t kTxBytes = kBBytes;
-  static constexpr uint32_t kLoadArrivals = 1 + 32;  // expect_tx + 32 cp.async lanes
+  static constexpr uint32_t kSrcArrivals = 32;     // cp.async lanes (1 with the TMA source)
+  static constexpr uint32_t kIdesc = make_idesc(2 /*s32*/, 1 /*s8*/, 0, 0, 2 * BM, BN);
 };
 
-template <>
-struct Cfg<Op::Dx> {
-  static constexpr int kBlockR = 64;            // reduction elements (n) per stage
+// dX: reduction over n in blocks of 64; kind::f16 consumes 16 n per MMA.
+template <int BN>
+struct Cfg<Op::Dx, BN> {
+  static constexpr int kBlockR = 64;
   static constexpr int kUmmaK = 16;
-  static constexpr int kABytes = BM * 64 * 2;   // 128 k x 64 n bf16
-  static constexpr int kBBytes = BN * 64 * 2;   // 256 m x 64 n bf16
-  static constexpr int kSrcBytes = 64 * 32;     // packed: 64 rows (n) x 32 bytes (128 k)
+  static constexpr int kABytes = BM * 64 * 2;      // 128 k x 64 n bf16
+  static constexpr int kBBytes = (BN / 2) * 128;   // BN/2 m x 64 n bf16
+  static constexpr int kSrcBytes = 64 * 32;        // packed: 64 rows (n) x 32 bytes (128 k)
   static constexpr int kSxBytes = 0;
-  static constexpr int kStages = 4;
-  static constexpr uint32_t kIdesc = make_idesc(1 /*f32*/, 1 /*bf16*/, 1 /*A MN*/, 0, BM, BN);
-  static constexpr uint32_t kTxBytes = kBBytes;
-  static constexpr uint32_t kLoadArrivals = 1 + 32;
+  static constexpr uint32_t kSrcArrivals = 32;
+  static constexpr uint32_t kIdesc = make_idesc(1 /*f32*/, 1 /*bf16*/, 1 /*A MN*/, 0, 2 * BM, BN);
 };
 
-template <>
-struct Cfg<Op::Dw> {
-  static constexpr int kBlockR = 64;            // reduction elements (m) per stage
+// dW: reduction over m in blocks of 64. B is MN-major: BN/2 must be a
+// multiple of 64 (whole 128-byte swizzle atoms).
+template <int BN>
+struct Cfg<Op::Dw, BN> {
+  static_assert((BN / 2) % 64 == 0, "MN-major B needs whole 64-element chunks");
+  static constexpr int kBlockR = 64;
   static constexpr int kUmmaK = 16;
-  static constexpr int kABytes = BM * 64 * 2;   // 128 k x 64 m bf16
-  static constexpr int kBBytes = BN * 64 * 2;   // 256 n x 64 m bf16 (4 TMA boxes)
-  static constexpr int kSrcBytes = 64 * 128;    // q: 64 rows (m) x 128 int8 (k), swizzled
-  static constexpr int kSxBytes = 64 * 4;       // s_x for the 64 tokens
-  static constexpr int kStages = 3;
-  static constexpr uint32_t kIdesc = make_idesc(1, 1, 1 /*A MN*/, 1 /*B MN*/, BM, BN);
-  static constexpr uint32_t kTxBytes = kBBytes + kSrcBytes + kSxBytes;
-  static constexpr uint32_t kLoadArrivals = 1;
+  static constexpr int kABytes = BM * 64 * 2;      // 128 k x 64 m bf16
+  static constexpr int kBBytes = (BN / 2) * 128;   // BN/2 n x 64 m bf16 ((BN/2)/64 TMA boxes)
+  static constexpr int kSrcBytes = 64 * 128;       // q: 64 rows (m) x 128 int8 (k), swizzled
+  static constexpr int kSxBytes = 64 * 4;          // s_x of the 64 tokens
+  static constexpr uint32_t kSrcArrivals = 1;      // expect_tx
+  static constexpr uint32_t kIdesc = make_idesc(1, 1, 1 /*A MN*/, 1 /*B MN*/, 2 * BM, BN);
 };
 
-template <Op op>
+template <Op op, int BN>
 struct Layout {
-  using C = Cfg<op>;
-  static constexpr int kS = C::kStages;
+  using C = Cfg<op, BN>;
+  static constexpr int kStageBytes = C::kABytes + C::kBBytes + C::kSrcBytes + C::kSxBytes;
+  static constexpr int kReserve = 1024 /*base alignment*/ + kNumEpiWarps * kEpiStageBytes + 512;
+  static constexpr int kS0 = (kSmemLimit - kReserve) / kStageBytes;
+  static constexpr int kS = kS0 > 8 ? 8 : kS0;
   static constexpr int kOffA = 0;
   static constexpr int kOffB = kOffA + kS * C::kABytes;
   static constexpr int kOffSrc = kOffB + kS * C::kBBytes;
   static constexpr int kOffSx = kOffSrc + kS * C::kSrcBytes;
   static constexpr int kOffEpi = kOffSx + kS * C::kSxBytes;
   static constexpr int kOffBar = kOffEpi + kNumEpiWarps * kEpiStageBytes;
-  // barriers: load_full[S], a_full[S], empty[S], tmem_full[2], tmem_empty[2], done
-  static constexpr int kNumBars = 3 * kS + 5;
+  // src_full[S], load_full[S], a_full[S], empty[S], tmem_full[2], tmem_empty[2], done
+  static constexpr int kNumBars = 4 * kS + 5;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kBytes = kOffMisc + 64;
-  static constexpr int kDynBytes = kBytes + 1024;  // slack to align the base to 1024
-  static_assert(kDynBytes <= 232448, "shared memory budget");
+  static constexpr int kDynBytes = kBytes + 1024;
+  static_assert(kS >= 2, "at least two pipeline stages");
+  static_assert(kDynBytes <= kSmemLimit, "shared memory budget");
   static_assert(C::kABytes % 1024 == 0 && C::kBBytes % 1024 == 0 && C::kSrcBytes % 1024 == 0, "alignment");
 };
 
@@ -137,6 +148,7 @@ struct GemmParams {
   int32_t* debug_acc;         // Fwd, optional
   int out_f32;                // Dw
   int accumulate;             // Dw
+  int src_tma;                // Fwd/Dx: packed codes by TMA (K % 64 == 0) instead of cp.async
   int* err;
 };
 
@@ -215,53 +227,72 @@ __device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
 
 // ---------------------------------------------------------------- the kernel
 
-template <Op op>
-__global__ void __launch_bounds__(kThreads, 1)
-    gemm_kernel(const __grid_constant__ CUtensorMap map_b, const __grid_constant__ CUtensorMap map_src,
-                const __grid_constant__ CUtensorMap map_sx, const GemmParams p) {
-  using C = Cfg<op>;
-  using L = Layout<op>;
-  constexpr int S = C::kStages;
+// Staging word of element (row j, column i) of an epilogue warp's 32 x 32
+// transpose tile; flipping bit 2 of i on odd rows keeps both the row-wise
+// writes and the 16-byte reads of two adjacent rows free of bank conflicts.
+__device__ __forceinline__ uint32_t stg_word(int j, int i) { return j * 32 + (i ^ ((j & 1) << 2)); }
+
+template <Op op, int BN>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+    gemm_pair_kernel(const __grid_constant__ CUtensorMap map_b, const __grid_constant__ CUtensorMap map_src,
+                     const __grid_constant__ CUtensorMap map_sx, const GemmParams p) {
+  using C = Cfg<op, BN>;
+  using L = Layout<op, BN>;
+  constexpr int S = L::kS;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kOffBar);
-  uint64_t* load_full = bars;
-  uint64_t* a_full = bars + S;
-  uint64_t* empty = bars + 2 * S;
-  uint64_t* tmem_full = bars + 3 * S;
-  uint64_t* tmem_empty = bars + 3 * S + 2;
-  uint64_t* done_bar = bars + 3 * S + 4;
+  uint64_t* src_full = bars;
+  uint64_t* load_full = bars + S;
+  uint64_t* a_full = bars + 2 * S;
+  uint64_t* empty = bars + 3 * S;
+  uint64_t* tmem_full = bars + 4 * S;
+  uint64_t* tmem_empty = bars + 4 * S + 2;
+  uint64_t* done_bar = bars + 4 * S + 4;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kOffMisc + 4);
-  int* issued_parity = reinterpret_cast<int*>(smem + L::kOffMisc + 8);  // [S], load warp's last issue
+  int* issued_parity = reinterpret_cast<int*>(smem + L::kOffMisc + 8);  // [S]
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int pair = static_cast<int>(blockIdx.x >> 1);
+  const int npairs = static_cast<int>(gridDim.x >> 1);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
-      mbar_init(&load_full[s], C::kLoadArrivals);
-      mbar_init(&a_full[s], kNumRebuildWarps);
+      mbar_init(&src_full[s], p.src_tma ? 1u : C::kSrcArrivals);
+      mbar_init(&load_full[s], 1);
+      mbar_init(&a_full[s], 2 * kNumRebuildWarps);
       mbar_init(&empty[s], 1);
       issued_parity[s] = -1;
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tmem_full[b], 1);
-      mbar_init(&tmem_empty[b], kNumEpiWarps);
+      mbar_init(&tmem_empty[b], 2 * kNumEpiWarps);
     }
     mbar_init(done_bar, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
   if (warp == kWarpMma) {
-    tmem_alloc(tmem_holder, kTmemCols);
-    tmem_relinquish();
+    tmem_alloc_pair(tmem_holder, kTmemCols);
+    tmem_relinquish_pair();
   }
   tc_fence_before();
-  __syncthreads();
+  cluster_sync_all();  // barriers initialised and TMEM allocated in both CTAs
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
+
+  // A failed wait also stops the peer CTA's waits.
+  auto wait = [&](uint64_t* bar, uint32_t parity) -> bool {
+    if (mbar_wait(bar, parity, abort_flag, p.err)) return true;
+    st_cluster_u32(map_to_rank(smem_u32(const_cast<int*>(abort_flag)), rank ^ 1u), 1u);
+    return false;
+  };
+  auto lead = [&](uint64_t* bar) -> uint32_t { return map_to_rank(smem_u32(bar), 0); };
 
   const int kq = static_cast<int>(p.K / 4);  // bytes per packed row
 
@@ -269,19 +300,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ loads
     if (lane == 0) {
       prefetch_tensormap(&map_b);
-      if constexpr (op == Op::Dw) {
-        prefetch_tensormap(&map_src);
-        prefetch_tensormap(&map_sx);
-      }
+      if (op == Op::Dw || p.src_tma) prefetch_tensormap(&map_src);
+      if constexpr (op == Op::Dw) prefetch_tensormap(&map_sx);
     }
     int stage = 0;
     uint32_t phase = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
-      const int a0 = (tile % p.tiles_a) * BM;
-      const int b0 = (tile / p.tiles_a) * BN;
+    for (int tile = pair; ok && tile < p.num_tiles; tile += npairs) {
+      const int a0 = (tile % p.tiles_a) * (2 * BM) + static_cast<int>(rank) * BM;  // this CTA's A rows
+      const int bh = (tile / p.tiles_a) * BN + static_cast<int>(rank) * (BN / 2);  // this CTA's B rows
       for (int kb = 0; kb < p.num_kb; ++kb) {
-        if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.err)) {
+        if (!wait(&empty[stage], phase ^ 1)) {
           ok = false;
           break;
         }
@@ -290,19 +319,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int r0 = kb * C::kBlockR;
         if (lane == 0) {
           issued_parity[stage] = static_cast<int>(phase);
-          mbar_arrive_expect_tx(&load_full[stage], C::kTxBytes);
-          if constexpr (op == Op::Fwd) {
-            tma_load_2d(&map_b, &load_full[stage], sB, r0, b0);
-          } else if constexpr (op == Op::Dx) {
-            tma_load_2d(&map_b, &load_full[stage], sB, r0, b0);
-          } else {
+          if (leader) mbar_arrive_expect_tx(&load_full[stage], 2 * C::kBBytes);
+          const uint32_t lb = lead(&load_full[stage]);
+          if constexpr (op == Op::Dw) {
 #pragma unroll
-            for (int j = 0; j < 4; ++j) tma_load_2d(&map_b, &load_full[stage], sB + j * 8192, b0 + 64 * j, r0);
-            tma_load_2d(&map_src, &load_full[stage], sSrc, a0, r0);
-            tma_load_2d(&map_sx, &load_full[stage], smem + L::kOffSx + stage * C::kSxBytes, r0, 0);
+            for (int j = 0; j < (BN / 2) / 64; ++j) tma_load_2d_pair(&map_b, lb, sB + j * 8192, bh + 64 * j, r0);
+            mbar_arrive_expect_tx(&src_full[stage], C::kSrcBytes + C::kSxBytes);
+            tma_load_2d(&map_src, &src_full[stage], sSrc, a0, r0);
+            tma_load_2d(&map_sx, &src_full[stage], smem + L::kOffSx + stage * C::kSxBytes, r0, 0);
+          } else {
+            tma_load_2d_pair(&map_b, lb, sB, r0, bh);
           }
         }
-        if constexpr (op == Op::Fwd) {
+        if (op != Op::Dw && p.src_tma) {
+          // packed codes as one TMA box: Fwd rows a0..a0+127 x bytes [kb*32, +32);
+          // Dx rows (n) r0..r0+63 x bytes [a0/4, +32)
+          if (lane == 0) {
+            mbar_arrive_expect_tx(&src_full[stage], C::kSrcBytes);
+            if constexpr (op == Op::Fwd)
+              tma_load_2d(&map_src, &src_full[stage], sSrc, kb * 32, a0);
+            else
+              tma_load_2d(&map_src, &src_full[stage], sSrc, a0 / 4, r0);
+          }
+        } else if constexpr (op == Op::Fwd) {
           // packed rows a0..a0+127, bytes [kb*32, kb*32+32): 512 chunks of 8 bytes
 #pragma unroll
           for (int it = 0; it < 16; ++it) {
@@ -313,7 +352,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                        : p.packed;
             cp_async_8(sSrc + row * 32 + part * 8, src, valid ? 8u : 0u);
           }
-          cp_async_mbar_arrive_noinc(&load_full[stage]);
+          cp_async_mbar_arrive_noinc(&src_full[stage]);
         } else if constexpr (op == Op::Dx) {
           // packed rows (n) r0..r0+63, bytes covering k in [a0, a0+128): 256 chunks
 #pragma unroll
@@ -325,7 +364,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 valid ? p.packed + static_cast<int64_t>(r0 + row) * kq + a0 / 4 + part * 8 : p.packed;
             cp_async_8(sSrc + row * 32 + part * 8, src, valid ? 8u : 0u);
           }
-          cp_async_mbar_arrive_noinc(&load_full[stage]);
+          cp_async_mbar_arrive_noinc(&src_full[stage]);
         }
         if (++stage == S) {
           stage = 0;
@@ -336,85 +375,87 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
     if (!ok && lane == 0) {
       // let every copy already issued land before the CTA exits
-      for (int s = 0; s < S; ++s)
-        if (issued_parity[s] >= 0) mbar_drain(&load_full[s], static_cast<uint32_t>(issued_parity[s]));
+      for (int s = 0; s < S; ++s) {
+        if (issued_parity[s] < 0) continue;
+        mbar_drain(&src_full[s], static_cast<uint32_t>(issued_parity[s]));
+        if (leader) mbar_drain(&load_full[s], static_cast<uint32_t>(issued_parity[s]));
+      }
     }
   } else if (warp == kWarpMma) {
-    // ------------------------------------------------------------ MMA issue
-    int stage = 0;
-    uint32_t phase = 0;
-    int buf = 0;
-    uint32_t buf_phase = 0;
-    bool ok = true;
-    for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
-      if (!mbar_wait(&tmem_empty[buf], buf_phase ^ 1, abort_flag, p.err)) break;
-      tc_fence_after();
-      const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * BN);
-      for (int kb = 0; kb < p.num_kb; ++kb) {
-        if (!mbar_wait(&load_full[stage], phase, abort_flag, p.err) ||
-            !mbar_wait(&a_full[stage], phase, abort_flag, p.err)) {
-          ok = false;
-          break;
-        }
+    // ------------------------------------------------------------ MMA issue (leader CTA)
+    if (leader) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int buf = 0;
+      uint32_t buf_phase = 0;
+      bool ok = true;
+      for (int tile = pair; ok && tile < p.num_tiles; tile += npairs) {
+        if (!wait(&tmem_empty[buf], buf_phase ^ 1)) break;
         tc_fence_after();
-        if (lane == 0) {
-          const uint32_t sa = smem_u32(smem + L::kOffA + stage * C::kABytes);
-          const uint32_t sb = smem_u32(smem + L::kOffB + stage * C::kBBytes);
-#pragma unroll
-          for (int kk = 0; kk < C::kBlockR / C::kUmmaK; ++kk) {
-            uint64_t adesc, bdesc;
-            if constexpr (op == Op::Fwd) {
-              adesc = smem_desc_sw128(sa + kk * 32, 16, 1024);
-              bdesc = smem_desc_sw128(sb + kk * 32, 16, 1024);
-              mma_i8(d_tmem, adesc, bdesc, C::kIdesc, (kb | kk) != 0);
-            } else if constexpr (op == Op::Dx) {
-              adesc = smem_desc_sw128(sa + kk * 2048, 8192, 1024);  // MN-major
-              bdesc = smem_desc_sw128(sb + kk * 32, 16, 1024);      // K-major
-              mma_f16(d_tmem, adesc, bdesc, C::kIdesc, (kb | kk) != 0);
-            } else {
-              adesc = smem_desc_sw128(sa + kk * 2048, 8192, 1024);  // MN-major
-              bdesc = smem_desc_sw128(sb + kk * 2048, 8192, 1024);  // MN-major
-              mma_f16(d_tmem, adesc, bdesc, C::kIdesc, (kb | kk) != 0);
-            }
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * 256);
+        for (int kb = 0; kb < p.num_kb; ++kb) {
+          if (!wait(&load_full[stage], phase) || !wait(&a_full[stage], phase)) {
+            ok = false;
+            break;
           }
-          mma_commit(&empty[stage]);
-          if (kb == p.num_kb - 1) mma_commit(&tmem_full[buf]);
+          tc_fence_after();
+          if (lane == 0) {
+            const uint32_t sa = smem_u32(smem + L::kOffA + stage * C::kABytes);
+            const uint32_t sb = smem_u32(smem + L::kOffB + stage * C::kBBytes);
+#pragma unroll
+            for (int kk = 0; kk < C::kBlockR / C::kUmmaK; ++kk) {
+              const uint32_t acc = (kb | kk) != 0;
+              if constexpr (op == Op::Fwd) {
+                mma_i8_pair(d_tmem, smem_desc_sw128(sa + kk * 32, 16, 1024), smem_desc_sw128(sb + kk * 32, 16, 1024),
+                            C::kIdesc, acc);
+              } else if constexpr (op == Op::Dx) {
+                mma_f16_pair(d_tmem, smem_desc_sw128(sa + kk * 2048, 8192, 1024),
+                             smem_desc_sw128(sb + kk * 32, 16, 1024), C::kIdesc, acc);
+              } else {
+                mma_f16_pair(d_tmem, smem_desc_sw128(sa + kk * 2048, 8192, 1024),
+                             smem_desc_sw128(sb + kk * 2048, 8192, 1024), C::kIdesc, acc);
+              }
+            }
+            mma_commit_pair(&empty[stage], 0x3);
+            if (kb == p.num_kb - 1) mma_commit_pair(&tmem_full[buf], 0x3);
+          }
+          __syncwarp();
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1;
+          }
         }
-        __syncwarp();
-        if (++stage == S) {
-          stage = 0;
-          phase ^= 1;
+        if (++buf == 2) {
+          buf = 0;
+          buf_phase ^= 1;
         }
       }
-      if (++buf == 2) {
-        buf = 0;
-        buf_phase ^= 1;
-      }
+      // done_bar completes in both CTAs once every MMA issued so far has finished
+      if (lane == 0) mma_commit_pair(done_bar, 0x3);
     }
-    // every MMA issued so far has completed once done_bar flips
-    if (lane == 0) {
-      mma_commit(done_bar);
-      mbar_drain(done_bar, 0);
-    }
+    if (lane == 0) mbar_drain(done_bar, 0);
     __syncwarp();
   } else if (warp < kWarpEpi0) {
-    // ------------------------------------------------------------ rebuild A
+    // ------------------------------------------------------------ rebuild A (both CTAs)
     const int rt = threadIdx.x - 32 * kWarpRebuild0;  // 0..127
     int stage = 0;
     uint32_t phase = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
+    for (int tile = pair; ok && tile < p.num_tiles; tile += npairs) {
       for (int kb = 0; kb < p.num_kb; ++kb) {
-        if (!mbar_wait(&load_full[stage], phase, abort_flag, p.err)) {
+        if (!wait(&src_full[stage], phase)) {
           ok = false;
           break;
         }
         const uint32_t sA = smem_u32(smem + L::kOffA + stage * C::kABytes);
         const uint32_t sSrc = smem_u32(smem + L::kOffSrc + stage * C::kSrcBytes);
         if constexpr (op == Op::Fwd) {
-          // row rt: 32 packed bytes -> 128 int8 codes, K-major with 128-byte swizzle
-          const uint4 w0 = ld_shared_v4(sSrc + rt * 32);
-          const uint4 w1 = ld_shared_v4(sSrc + rt * 32 + 16);
+          // row rt: 32 packed bytes -> 128 int8 codes, K-major with 128-byte swizzle.
+          // Lanes 4..7 of each group of 8 read their second half first (bank spread).
+          const uint32_t h = (rt >> 2) & 1;
+          const uint4 wa = ld_shared_v4(sSrc + rt * 32 + h * 16);
+          const uint4 wb = ld_shared_v4(sSrc + rt * 32 + (h ^ 1) * 16);
+          const uint4 w0 = h ? wb : wa, w1 = h ? wa : wb;
           const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
           const uint32_t row_base = sA + rt * 128;
 #pragma unroll
@@ -427,8 +468,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t base = sA + half * 8192 + n * 128;
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
-            const uint32_t h = words[j >> 1] >> ((j & 1) * 16);
-            st_shared_v4(base + ((j ^ (n & 7)) << 4), codes8_to_bf16(h));
+            const uint32_t hw = words[j >> 1] >> ((j & 1) * 16);
+            st_shared_v4(base + ((j ^ (n & 7)) << 4), codes8_to_bf16(hw));
           }
         } else {
           // token m = rt % 64, k half = rt / 64; q staging is 128-byte swizzled
@@ -448,7 +489,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&a_full[stage]);
+        if (lane == 0) mbar_arrive_cluster(lead(&a_full[stage]));
         if (++stage == S) {
           stage = 0;
           phase ^= 1;
@@ -456,30 +497,41 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else {
-    // ------------------------------------------------------------ epilogue
+    // ------------------------------------------------------------ epilogue (both CTAs)
     const int q = warp & 3;  // TMEM lane quadrant this warp may access
     const uint32_t stg = smem_u32(smem + L::kOffEpi + (warp - kWarpEpi0) * kEpiStageBytes);
     const float gamma = (op == Op::Dw) ? 1.0f : __ldg(p.gamma);
     int buf = 0;
     uint32_t buf_phase = 0;
-    for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
-      const int a0 = (tile % p.tiles_a) * BM;
+    for (int tile = pair; tile < p.num_tiles; tile += npairs) {
+      const int a0 = (tile % p.tiles_a) * (2 * BM) + static_cast<int>(rank) * BM;
       const int b0 = (tile / p.tiles_a) * BN;
-      if (!mbar_wait(&tmem_full[buf], buf_phase, abort_flag, p.err)) break;
+      // forward: s_x[m] * gamma of the tile's BN columns, loaded before the
+      // accumulator is ready; lane l holds column 32c + l of chunk c
+      float col_scale[BN / 32];
+      if constexpr (op == Op::Fwd) {
+#pragma unroll
+        for (int c = 0; c < BN / 32; ++c) {
+          const int j = b0 + c * 32 + lane;
+          col_scale[c] = j < p.rows_b ? __fmul_rn(__ldg(p.sx + j), gamma) : 0.0f;
+        }
+      }
+      if (!wait(&tmem_full[buf], buf_phase)) break;
       tc_fence_after();
+#pragma unroll
       for (int c = 0; c < BN / 32; ++c) {
         uint32_t r[32];
-        tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * BN + c * 32, r);
+        tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * 256 + c * 32, r);
         tmem_ld_wait();
         if (c == BN / 32 - 1) {
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&tmem_empty[buf]);
+          if (lane == 0) mbar_arrive_cluster(lead(&tmem_empty[buf]));
         }
-        // transpose through smem: staging[j][lane] = D[row lane][column j]
+        // transpose through smem: staging(j, lane) = D[row lane][column j]
 #pragma unroll
         for (int j = 0; j < 32; ++j)
-          asm volatile("st.shared.b32 [%0], %1;" ::"r"(stg + (j * 32 + lane) * 4), "r"(r[j]) : "memory");
+          asm volatile("st.shared.b32 [%0], %1;" ::"r"(stg + stg_word(j, lane) * 4), "r"(r[j]) : "memory");
         __syncwarp();
         // each lane stores 8 consecutive i of one output row j, 4 rows per pass
         const int seg = (lane & 3) * 8;
@@ -488,14 +540,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int pass = 0; pass < 4; ++pass) {
           const int jl = pass * 8 + (lane >> 2);
           const int j = b0 + c * 32 + jl;
+          float row_scale = 0.0f;
+          if constexpr (op == Op::Fwd) row_scale = __shfl_sync(0xffffffffu, col_scale[c], jl);
           if (j >= p.rows_b || i0 >= p.rows_a) continue;
-          const uint4 v0 = ld_shared_v4(stg + (jl * 32 + seg) * 4);
-          const uint4 v1 = ld_shared_v4(stg + (jl * 32 + seg + 4) * 4);
-          const uint32_t acc[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+          // the two 4-word halves of this 8-word run (swapped on odd rows)
+          const int sw = (jl & 1) << 2;
+          const uint4 v0 = ld_shared_v4(stg + stg_word(jl, seg + sw) * 4);
+          const uint4 v1 = ld_shared_v4(stg + stg_word(jl, seg + (4 ^ sw)) * 4);
+          const uint4 lo = sw ? v1 : v0, hi = sw ? v0 : v1;
+          const uint32_t acc[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
           const int nvalid = min(8, p.rows_a - i0);
           const int64_t off = static_cast<int64_t>(j) * p.ldo + i0;
           if constexpr (op == Op::Fwd) {
-            const float scale = __fmul_rn(__ldg(p.sx + j), gamma);
+            const float scale = row_scale;
             __nv_bfloat16* y = static_cast<__nv_bfloat16*>(p.out) + off;
             uint32_t pk[4];
 #pragma unroll
@@ -505,8 +562,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                         __fmul_rn(static_cast<float>(static_cast<int32_t>(acc[e + 1])), scale));
               pk[e / 2] = *reinterpret_cast<const uint32_t*>(&b2);
             }
-            const bool vec = nvalid == 8 && (p.ldo % 8) == 0;
-            if (vec) {
+            if (nvalid == 8 && (p.ldo % 8) == 0) {
               *reinterpret_cast<uint4*>(y) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
             } else {
               for (int e = 0; e < nvalid; ++e)
@@ -515,8 +571,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (p.debug_acc) {
               int32_t* d = p.debug_acc + off;
               if (nvalid == 8 && (p.ldo % 4) == 0) {
-                reinterpret_cast<uint4*>(d)[0] = v0;
-                reinterpret_cast<uint4*>(d)[1] = v1;
+                reinterpret_cast<uint4*>(d)[0] = lo;
+                reinterpret_cast<uint4*>(d)[1] = hi;
               } else {
                 for (int e = 0; e < nvalid; ++e) d[e] = static_cast<int32_t>(acc[e]);
               }
@@ -577,10 +633,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   tc_fence_before();
-  __syncthreads();
+  cluster_sync_all();  // no CTA leaves while its peer may still signal it
   if (warp == kWarpMma) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, kTmemCols);
+    tmem_dealloc_pair(tmem_base, kTmemCols);
   }
 }
 
@@ -640,26 +696,81 @@ bool make_map_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint6
   return true;
 }
 
-template <Op op>
-cudaError_t launch_gemm(const CUtensorMap& mb, const CUtensorMap& msrc, const CUtensorMap& msx, GemmParams p,
-                        cudaStream_t s) {
-  using L = Layout<op>;
-  static int configured_device = -1;  // attribute set once per process per device id
+template <Op op, int BN>
+cudaError_t launch_pair(const CUtensorMap& mb, const CUtensorMap& msrc, const CUtensorMap& msx, GemmParams p,
+                        int npairs, cudaStream_t s) {
+  using L = Layout<op, BN>;
+  static int configured[64] = {};  // attribute set once per process per device
   int dev = 0;
   cudaGetDevice(&dev);
-  if (configured_device != dev) {
+  if (dev >= 0 && dev < 64 && !configured[dev]) {
     cudaError_t e =
-        cudaFuncSetAttribute(gemm_kernel<op>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kDynBytes);
+        cudaFuncSetAttribute(gemm_pair_kernel<op, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kDynBytes);
     if (e != cudaSuccess) return e;
-    configured_device = dev;
+    configured[dev] = 1;
   }
-  p.tiles_a = (p.rows_a + BM - 1) / BM;
+  p.tiles_a = (p.rows_a + 2 * BM - 1) / (2 * BM);
   p.tiles_b = (p.rows_b + BN - 1) / BN;
-  p.num_kb = (p.red + Cfg<op>::kBlockR - 1) / Cfg<op>::kBlockR;
+  p.num_kb = (p.red + Cfg<op, BN>::kBlockR - 1) / Cfg<op, BN>::kBlockR;
   p.num_tiles = p.tiles_a * p.tiles_b;
-  const int grid = p.num_tiles < device_sm_count() ? p.num_tiles : device_sm_count();
-  gemm_kernel<op><<<grid, kThreads, L::kDynBytes, s>>>(mb, msrc, msx, p);
+  const int pairs = p.num_tiles < npairs ? p.num_tiles : npairs;
+  static const bool log = std::getenv("BL_LOG") != nullptr;
+  if (log)
+    std::fprintf(stderr, "[bitlinear] gemm op=%d BN=%d stages=%d smem=%d tiles=%dx%d kb=%d pairs=%d (of %d)\n",
+                 static_cast<int>(op), BN, L::kS, L::kDynBytes, p.tiles_a, p.tiles_b, p.num_kb, pairs, npairs);
+  gemm_pair_kernel<op, BN><<<2 * pairs, kThreads, L::kDynBytes, s>>>(mb, msrc, msx, p);
   return cudaGetLastError();
+}
+
+// B rows per pair tile: the candidate with the fewest tile-rows of work per
+// pair after wave quantisation (waves x BN), ties to the larger tile.
+int choose_bn(int rows_a, int rows_b, int npairs, const int* cands, int ncands) {
+  const int tiles_a = (rows_a + 2 * BM - 1) / (2 * BM);
+  int best = cands[0];
+  long long best_cost = -1;
+  for (int i = 0; i < ncands; ++i) {
+    const int bn = cands[i];
+    const long long tiles = static_cast<long long>(tiles_a) * ((rows_b + bn - 1) / bn);
+    const long long cost = ((tiles + npairs - 1) / npairs) * bn;
+    if (best_cost < 0 || cost < best_cost) {
+      best = bn;
+      best_cost = cost;
+    }
+  }
+  return best;
+}
+
+// Number of CTA pairs of this kernel that can be resident at once (GPCs with
+// an odd number of SMs leave one SM out of pairing), capped at SMs / 2.
+template <Op op, int BN>
+int resident_pairs() {
+  static int cached[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && cached[dev]) return cached[dev];
+  using L = Layout<op, BN>;
+  int n = device_sm_count() / 2;
+  if (cudaFuncSetAttribute(gemm_pair_kernel<op, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kDynBytes) ==
+      cudaSuccess) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(2 * n);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = L::kDynBytes;
+    int clusters = 0;
+    if (cudaOccupancyMaxActiveClusters(&clusters, gemm_pair_kernel<op, BN>, &cfg) == cudaSuccess && clusters > 0 &&
+        clusters < n)
+      n = clusters;
+  }
+  cudaGetLastError();
+  if (dev >= 0 && dev < 64) cached[dev] = n;
+  return n;
+}
+
+// All candidate configurations of one op share the same pair budget; the
+// largest tile is the most constrained, so its residency is used for all.
+template <Op op>
+int pair_count() {
+  return resident_pairs<op, 256>();
 }
 
 }  // namespace
@@ -687,10 +798,19 @@ cudaError_t launch_forward(const int8_t* xq, const float* sx, const uint8_t* w_p
                            int64_t M, int64_t N, int64_t K, void* y, int32_t* debug_acc, int* err,
                            cudaStream_t s) {
   if (M == 0 || N == 0) return cudaSuccess;
-  CUtensorMap mb{}, unused{};
-  if (!make_map_2d(&mb, xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, K, M, K, 128, BN, CU_TENSOR_MAP_SWIZZLE_128B, "xq"))
+  static const int kCands[3] = {256, 192, 128};
+  const int npairs = pair_count<Op::Fwd>();
+  const int bn = choose_bn(static_cast<int>(N), static_cast<int>(M), npairs, kCands, 3);
+  CUtensorMap mb{}, msrc{}, unused{};
+  if (!make_map_2d(&mb, xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, K, M, K, 128, bn / 2, CU_TENSOR_MAP_SWIZZLE_128B, "xq"))
+    return cudaErrorInvalidValue;
+  // packed codes [N][K/4] bytes: a TMA tensor needs 16-byte row pitch (K % 64 == 0)
+  const bool src_tma = (K % 64) == 0;
+  if (src_tma && !make_map_2d(&msrc, w_packed, CU_TENSOR_MAP_DATA_TYPE_UINT8, K / 4, N, K / 4, 32, BM,
+                              CU_TENSOR_MAP_SWIZZLE_NONE, "w_packed (fwd)"))
     return cudaErrorInvalidValue;
   GemmParams p{};
+  p.src_tma = src_tma;
   p.rows_a = static_cast<int>(N);
   p.rows_b = static_cast<int>(M);
   p.red = static_cast<int>(K);
@@ -702,17 +822,27 @@ cudaError_t launch_forward(const int8_t* xq, const float* sx, const uint8_t* w_p
   p.ldo = N;
   p.debug_acc = debug_acc;
   p.err = err;
-  return launch_gemm<Op::Fwd>(mb, unused, unused, p, s);
+  if (bn == 256) return launch_pair<Op::Fwd, 256>(mb, msrc, unused, p, npairs, s);
+  if (bn == 192) return launch_pair<Op::Fwd, 192>(mb, msrc, unused, p, npairs, s);
+  return launch_pair<Op::Fwd, 128>(mb, msrc, unused, p, npairs, s);
 }
 
 cudaError_t launch_backward_dx(const void* dY, const uint8_t* w_packed, const float* gamma, int64_t M, int64_t N,
                                int64_t K, void* dX, int* err, cudaStream_t s) {
   if (M == 0) return cudaSuccess;
-  CUtensorMap mb{}, unused{};
-  if (!make_map_2d(&mb, dY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, N, M, N * 2, 64, BN, CU_TENSOR_MAP_SWIZZLE_128B,
+  static const int kCands[3] = {256, 192, 128};
+  const int npairs = pair_count<Op::Dx>();
+  const int bn = choose_bn(static_cast<int>(K), static_cast<int>(M), npairs, kCands, 3);
+  CUtensorMap mb{}, msrc{}, unused{};
+  if (!make_map_2d(&mb, dY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, N, M, N * 2, 64, bn / 2, CU_TENSOR_MAP_SWIZZLE_128B,
                    "dY (dX)"))
     return cudaErrorInvalidValue;
+  const bool src_tma = (K % 64) == 0;
+  if (src_tma && !make_map_2d(&msrc, w_packed, CU_TENSOR_MAP_DATA_TYPE_UINT8, K / 4, N, K / 4, 32, 64,
+                              CU_TENSOR_MAP_SWIZZLE_NONE, "w_packed (dX)"))
+    return cudaErrorInvalidValue;
   GemmParams p{};
+  p.src_tma = src_tma;
   p.rows_a = static_cast<int>(K);
   p.rows_b = static_cast<int>(M);
   p.red = static_cast<int>(N);
@@ -722,7 +852,9 @@ cudaError_t launch_backward_dx(const void* dY, const uint8_t* w_packed, const fl
   p.out = dX;
   p.ldo = K;
   p.err = err;
-  return launch_gemm<Op::Dx>(mb, unused, unused, p, s);
+  if (bn == 256) return launch_pair<Op::Dx, 256>(mb, msrc, unused, p, npairs, s);
+  if (bn == 192) return launch_pair<Op::Dx, 192>(mb, msrc, unused, p, npairs, s);
+  return launch_pair<Op::Dx, 128>(mb, msrc, unused, p, npairs, s);
 }
 
 cudaError_t launch_backward_dw(const void* dY, const int8_t* xq, const float* sx, int64_t M, int64_t N, int64_t K,
@@ -732,9 +864,12 @@ cudaError_t launch_backward_dw(const void* dY, const int8_t* xq, const float* sx
     zero_dw_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, s>>>(dW, n, dw_is_f32, accumulate);
     return cudaGetLastError();
   }
-  CUtensorMap mb{}, msrc{}, msx{};
+  static const int kCands[2] = {256, 128};
+  const int npairs = pair_count<Op::Dw>();
+  const int bn = choose_bn(static_cast<int>(K), static_cast<int>(N), npairs, kCands, 2);
   // s_x as a one-row 2D tensor: [1][M] floats, row pitch rounded up to 16 bytes
   const uint64_t sx_pitch = ((static_cast<uint64_t>(M) * 4 + 15) / 16) * 16;
+  CUtensorMap mb{}, msrc{}, msx{};
   if (!make_map_2d(&mb, dY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, N, M, N * 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B,
                    "dY (dW)") ||
       !make_map_2d(&msrc, xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, K, M, K, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B, "xq (dW)") ||
@@ -751,7 +886,8 @@ cudaError_t launch_backward_dw(const void* dY, const int8_t* xq, const float* sx
   p.out_f32 = dw_is_f32;
   p.accumulate = accumulate;
   p.err = err;
-  return launch_gemm<Op::Dw>(mb, msrc, msx, p, s);
+  if (bn == 256) return launch_pair<Op::Dw, 256>(mb, msrc, msx, p, npairs, s);
+  return launch_pair<Op::Dw, 128>(mb, msrc, msx, p, npairs, s);
 }
 
 }  // namespace bl

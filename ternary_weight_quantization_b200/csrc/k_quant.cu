@@ -52,31 +52,50 @@ struct Group {
   }
 };
 
+// |x| widened to fp64 exactly. Normal values are re-biased with integer
+// arithmetic (full-rate ALU instead of the conversion pipe); zero and
+// subnormals take the conversion. Inputs are finite.
+__device__ __forceinline__ double abs_to_f64(float x) {
+  const uint32_t b = __float_as_uint(x) & 0x7FFFFFFFu;
+  if (b >= 0x00800000u) return __longlong_as_double((static_cast<long long>(b) << 29) + 0x3800000000000000ll);
+  return static_cast<double>(__uint_as_float(b));
+}
+
+template <bool kF32>
+__device__ __forceinline__ double add_group(double acc, const Group<kF32>& a) {
+#pragma unroll
+  for (int i = 0; i < 16; ++i) acc = __dadd_rn(acc, abs_to_f64(a.elem(i)));
+  return acc;
+}
+
 // ---------------------------------------------------------------- S1 pass A
 // partials[b] = sum of |w| over block b's contiguous range of groups, fp64,
-// each thread summing its groups in order, then a fixed shuffle/smem tree.
+// each thread summing its groups in increasing order (four loads in flight),
+// then a fixed shuffle/smem tree.
 template <bool kF32>
 __global__ void __launch_bounds__(kQuantThreads) absmean_partials_kernel(const uint4* __restrict__ W,
                                                                          int64_t ngroups, int64_t per_block,
                                                                          double* __restrict__ partials) {
+  constexpr int T = kQuantThreads;
   const int64_t g0 = static_cast<int64_t>(blockIdx.x) * per_block;
   const int64_t g1 = min(g0 + per_block, ngroups);
   double acc = 0.0;
   int64_t g = g0 + threadIdx.x;
-  for (; g + kQuantThreads < g1; g += 2 * kQuantThreads) {
-    Group<kF32> a, b;
+  for (; g + 3 * T < g1; g += 4 * T) {
+    Group<kF32> a, b, c, d;
     a.load(W, g);
-    b.load(W, g + kQuantThreads);
-#pragma unroll
-    for (int i = 0; i < 16; ++i) acc = __dadd_rn(acc, static_cast<double>(fabsf(a.elem(i))));
-#pragma unroll
-    for (int i = 0; i < 16; ++i) acc = __dadd_rn(acc, static_cast<double>(fabsf(b.elem(i))));
+    b.load(W, g + T);
+    c.load(W, g + 2 * T);
+    d.load(W, g + 3 * T);
+    acc = add_group(acc, a);
+    acc = add_group(acc, b);
+    acc = add_group(acc, c);
+    acc = add_group(acc, d);
   }
-  if (g < g1) {
+  for (; g < g1; g += T) {
     Group<kF32> a;
     a.load(W, g);
-#pragma unroll
-    for (int i = 0; i < 16; ++i) acc = __dadd_rn(acc, static_cast<double>(fabsf(a.elem(i))));
+    acc = add_group(acc, a);
   }
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) acc = __dadd_rn(acc, __shfl_xor_sync(0xffffffffu, acc, off));
@@ -101,6 +120,19 @@ __global__ void __launch_bounds__(kQuantThreads) absmean_partials_kernel(const u
 // the even 0.5). With T = gamma * (0.5 + 2^-25) computed exactly in fp64 and
 // thr the largest float <= T, that is |w| > thr: one compare, no division.
 template <bool kF32>
+__device__ __forceinline__ uint32_t pack_group(const Group<kF32>& a, float thr) {
+  uint32_t word = 0;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const float w = a.elem(i);
+    const uint32_t nz = fabsf(w) > thr ? 1u : 0u;
+    const uint32_t neg = __float_as_uint(w) >> 31;
+    word |= (nz * (1u | (neg << 1))) << (2 * i);  // 00 = 0, 01 = +1, 11 = -1
+  }
+  return word;
+}
+
+template <bool kF32>
 __global__ void __launch_bounds__(kQuantThreads) ternarize_pack_kernel(const uint4* __restrict__ W,
                                                                        int64_t ngroups, int64_t per_block,
                                                                        const double* __restrict__ partials,
@@ -123,26 +155,27 @@ __global__ void __launch_bounds__(kQuantThreads) ternarize_pack_kernel(const uin
   }
   __syncthreads();
   const float thr = s_thr;
+  constexpr int T = kQuantThreads;
   const int64_t g0 = static_cast<int64_t>(blockIdx.x) * per_block;
   const int64_t g1 = min(g0 + per_block, ngroups);
-  for (int64_t g = g0 + threadIdx.x; g < g1; g += kQuantThreads) {
+  int64_t g = g0 + threadIdx.x;
+  for (; g + 3 * T < g1; g += 4 * T) {
+    Group<kF32> a[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) a[u].load(W, g + u * T);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) packed[g + u * T] = pack_group(a[u], thr);
+  }
+  for (; g < g1; g += T) {
     Group<kF32> a;
     a.load(W, g);
-    uint32_t word = 0;
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const float w = a.elem(i);
-      const uint32_t nz = fabsf(w) > thr ? 1u : 0u;
-      const uint32_t neg = __float_as_uint(w) >> 31;
-      word |= (nz * (1u | (neg << 1))) << (2 * i);  // 00 = 0, 01 = +1, 11 = -1
-    }
-    packed[g] = word;
+    packed[g] = pack_group(a, thr);
   }
 }
 
 // ---------------------------------------------------------------- S2
 // One warp per token. The row stays in registers between the absmax and the
-// quantisation (VPL 16-byte vectors per lane, rows up to 256 * VPL elements).
+// quantisation: VPL = ceil(K / 256) 16-byte vectors per lane (K <= 8192).
 //
 // q = rint_half_even(fp32(x * inv)) uses the 1.5 * 2^23 shifter: adding it
 // rounds |x * inv| <= 127.0001 to an integer (ties to even), and the low byte
@@ -305,20 +338,21 @@ cudaError_t launch_quantize_act(const void* x, int64_t M, int64_t K, int8_t* xq,
   const dim3 block(32 * kActRowsPerBlock);
   const uint4* xv = static_cast<const uint4*>(x);
   const int per_lane = (nv + 31) / 32;
-  if (per_lane <= 1)
-    act_quant_kernel<1><<<grid, block, 0, s>>>(xv, M, nv, xq, sx);
-  else if (per_lane <= 2)
-    act_quant_kernel<2><<<grid, block, 0, s>>>(xv, M, nv, xq, sx);
-  else if (per_lane <= 4)
-    act_quant_kernel<4><<<grid, block, 0, s>>>(xv, M, nv, xq, sx);
-  else if (per_lane <= 8)
-    act_quant_kernel<8><<<grid, block, 0, s>>>(xv, M, nv, xq, sx);
-  else if (per_lane <= 16)
-    act_quant_kernel<16><<<grid, block, 0, s>>>(xv, M, nv, xq, sx);
-  else if (per_lane <= 32)
-    act_quant_kernel<32><<<grid, block, 0, s>>>(xv, M, nv, xq, sx);
-  else
-    act_quant_long_kernel<<<grid, block, 0, s>>>(xv, M, nv, xq, sx);
+  switch (per_lane) {
+#define BL_ACT_CASE(n) \
+  case n:              \
+    act_quant_kernel<n><<<grid, block, 0, s>>>(xv, M, nv, xq, sx); \
+    break;
+    BL_ACT_CASE(1) BL_ACT_CASE(2) BL_ACT_CASE(3) BL_ACT_CASE(4) BL_ACT_CASE(5) BL_ACT_CASE(6) BL_ACT_CASE(7)
+    BL_ACT_CASE(8) BL_ACT_CASE(9) BL_ACT_CASE(10) BL_ACT_CASE(11) BL_ACT_CASE(12) BL_ACT_CASE(13)
+    BL_ACT_CASE(14) BL_ACT_CASE(15) BL_ACT_CASE(16) BL_ACT_CASE(17) BL_ACT_CASE(18) BL_ACT_CASE(19)
+    BL_ACT_CASE(20) BL_ACT_CASE(21) BL_ACT_CASE(22) BL_ACT_CASE(23) BL_ACT_CASE(24) BL_ACT_CASE(25)
+    BL_ACT_CASE(26) BL_ACT_CASE(27) BL_ACT_CASE(28) BL_ACT_CASE(29) BL_ACT_CASE(30) BL_ACT_CASE(31)
+    BL_ACT_CASE(32)
+#undef BL_ACT_CASE
+    default:
+      act_quant_long_kernel<<<grid, block, 0, s>>>(xv, M, nv, xq, sx);
+  }
   return cudaGetLastError();
 }
 
