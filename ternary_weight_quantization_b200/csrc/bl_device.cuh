@@ -96,6 +96,14 @@ __device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
   }
 }
 
+// As mbar_drain, with an absolute deadline shared by several drains.
+__device__ __forceinline__ void mbar_drain_until(uint64_t* bar, uint32_t parity, unsigned long long deadline) {
+  const uint32_t a = smem_u32(bar);
+  while (!mbar_try_wait(a, parity)) {
+    if (globaltimer_ns() > deadline) return;
+  }
+}
+
 // ---------------------------------------------------------------- clusters (CTA pairs)
 
 __device__ __forceinline__ uint32_t cluster_ctarank() {

@@ -21,18 +21,22 @@
 // TMEM. Splitting both operands across the pair halves the B traffic per SM
 // compared with a single-CTA 128 x BN tile. No TMA multicast is used.
 //
-// Warp roles (320 threads per CTA):
-//   warp 0    loads: TMA for B, for Dw's q / s_x and for the packed codes
-//             (cp.async for the codes when K % 64 != 0: their rows are then not
-//             16-byte aligned, which a tensor map requires)
-//   warp 1    TMEM allocation (2 x 256 columns, pair-wide); in the leader CTA
-//             also tcgen05.mma issue
-//   warps 2-5 rebuild A from the staged source
-//   warps 6-9 epilogue: TMEM -> registers -> smem (transpose) -> global
-// Barriers: src_full (per CTA: staged source landed), load_full and a_full
-// (leader: both CTAs' B bytes landed / both CTAs' A rebuilt), empty and
-// tmem_full (both CTAs, completed by multicast tcgen05.commit), tmem_empty
-// (leader: both CTAs' epilogues drained a TMEM buffer). Every wait is
+// Warp roles (512 threads per CTA):
+//   warp 0      loads: TMA for B, for Dw's q / s_x and for the packed codes
+//               (cp.async for the codes when K % 64 != 0: their rows are then
+//               not 16-byte aligned, which a tensor map requires)
+//   warp 1      TMEM allocation (2 x 256 columns, pair-wide); in the leader
+//               CTA one lane issues the tcgen05.mma
+//   warps 2-4, 6-8, 10-11  rebuild A from the staged source
+//   warps 5, 9  idle (keeps sub-partition 1 free for the MMA warp)
+//   warps 12-15 epilogue: TMEM -> registers -> smem (transpose) -> global
+// Barriers: src_full (per CTA: staged source landed), full (leader: both
+// CTAs' B bytes landed and both CTAs' A rebuilt -- one wait per stage for the
+// MMA lane), empty and tmem_full (both CTAs, completed by multicast
+// tcgen05.commit), tmem_empty (leader: both CTAs' epilogues drained a TMEM
+// buffer). The MMA lane's loop is kept minimal because the tensor core's
+// instruction queue is shallow: the next stage's MMAs must be issued while
+// the current stage's last MMA still executes. Every wait is
 // bounded: on expiry a CTA records a timeout in the device error word, tells
 // its peer, drains what it has in flight, frees TMEM and exits.
 #include <cuda.h>
@@ -52,13 +56,22 @@
 namespace bl {
 namespace {
 
-constexpr int kThreads = 320;
+// Warp w runs on SM sub-partition w % 4. The MMA warp (1) keeps sub-partition
+// 1 to itself apart from one epilogue warp: rebuild warps there would compete
+// with it for issue slots and delay the next MMAs.
+constexpr int kThreads = 512;
 constexpr int kWarpLoad = 0;
 constexpr int kWarpMma = 1;
-constexpr int kWarpRebuild0 = 2;
-constexpr int kNumRebuildWarps = 4;
-constexpr int kWarpEpi0 = 6;
+constexpr int kNumRebuildWarps = 8;  // warps 2, 3, 4, 6, 7, 8, 10, 11
+constexpr int kRebuildThreads = 32 * kNumRebuildWarps;
+constexpr int kWarpEpi0 = 12;        // warps 12..15 (TMEM lane quadrants 0..3)
 constexpr int kNumEpiWarps = 4;
+
+// Rebuild slot of warp w (0..7), or -1 (warps 0, 1, 5, 9 and 12..15).
+__device__ __forceinline__ int rebuild_slot(int w) {
+  if (w < 2 || w >= kWarpEpi0 || (w & 3) == 1) return -1;
+  return w - 2 - (w >= 6) - (w >= 10);
+}
 
 constexpr int BM = 128;              // A rows per CTA; a pair covers 2 * BM
 constexpr uint32_t kTmemCols = 512;  // two accumulators at columns 0 and 256
@@ -124,8 +137,8 @@ struct Layout {
   static constexpr int kOffSx = kOffSrc + kS * C::kSrcBytes;
   static constexpr int kOffEpi = kOffSx + kS * C::kSxBytes;
   static constexpr int kOffBar = kOffEpi + kNumEpiWarps * kEpiStageBytes;
-  // src_full[S], load_full[S], a_full[S], empty[S], tmem_full[2], tmem_empty[2], done
-  static constexpr int kNumBars = 4 * kS + 5;
+  // src_full[S], full[S], empty[S], tmem_full[2], tmem_empty[2], done
+  static constexpr int kNumBars = 3 * kS + 5;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kBytes = kOffMisc + 64;
   static constexpr int kDynBytes = kBytes + 1024;
@@ -244,12 +257,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kOffBar);
   uint64_t* src_full = bars;
-  uint64_t* load_full = bars + S;
-  uint64_t* a_full = bars + 2 * S;
-  uint64_t* empty = bars + 3 * S;
-  uint64_t* tmem_full = bars + 4 * S;
-  uint64_t* tmem_empty = bars + 4 * S + 2;
-  uint64_t* done_bar = bars + 4 * S + 4;
+  uint64_t* full = bars + S;
+  uint64_t* empty = bars + 2 * S;
+  uint64_t* tmem_full = bars + 3 * S;
+  uint64_t* tmem_empty = bars + 3 * S + 2;
+  uint64_t* done_bar = bars + 3 * S + 4;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kOffMisc + 4);
   int* issued_parity = reinterpret_cast<int*>(smem + L::kOffMisc + 8);  // [S]
@@ -264,8 +276,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(&src_full[s], p.src_tma ? 1u : C::kSrcArrivals);
-      mbar_init(&load_full[s], 1);
-      mbar_init(&a_full[s], 2 * kNumRebuildWarps);
+      mbar_init(&full[s], 1 + 2 * kNumRebuildWarps);  // leader's expect_tx + both CTAs' rebuild warps
       mbar_init(&empty[s], 1);
       issued_parity[s] = -1;
     }
@@ -319,8 +330,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const int r0 = kb * C::kBlockR;
         if (lane == 0) {
           issued_parity[stage] = static_cast<int>(phase);
-          if (leader) mbar_arrive_expect_tx(&load_full[stage], 2 * C::kBBytes);
-          const uint32_t lb = lead(&load_full[stage]);
+          if (leader) mbar_arrive_expect_tx(&full[stage], 2 * C::kBBytes);
+          const uint32_t lb = lead(&full[stage]);
           if constexpr (op == Op::Dw) {
 #pragma unroll
             for (int j = 0; j < (BN / 2) / 64; ++j) tma_load_2d_pair(&map_b, lb, sB + j * 8192, bh + 64 * j, r0);
@@ -374,16 +385,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
     __syncwarp();
     if (!ok && lane == 0) {
-      // let every copy already issued land before the CTA exits
+      // let every copy already issued land before the CTA exits (one time
+      // bound for all of them; `full` also counts rebuild arrivals that may
+      // never come on this path)
+      const unsigned long long deadline = globaltimer_ns() + kWaitLimitNs;
       for (int s = 0; s < S; ++s) {
         if (issued_parity[s] < 0) continue;
-        mbar_drain(&src_full[s], static_cast<uint32_t>(issued_parity[s]));
-        if (leader) mbar_drain(&load_full[s], static_cast<uint32_t>(issued_parity[s]));
+        mbar_drain_until(&src_full[s], static_cast<uint32_t>(issued_parity[s]), deadline);
+        if (leader) mbar_drain_until(&full[s], static_cast<uint32_t>(issued_parity[s]), deadline);
       }
     }
   } else if (warp == kWarpMma) {
-    // ------------------------------------------------------------ MMA issue (leader CTA)
-    if (leader) {
+    // ------------------------------------------------------------ MMA issue (leader CTA, one lane)
+    if (leader && lane == 0) {
+      // descriptors of stage 0; a stage or k step is an offset (in 16-byte
+      // units) added to the start-address field
+      constexpr uint32_t kLboA = (op == Op::Fwd) ? 16 : 8192;
+      constexpr uint32_t kLboB = (op == Op::Dw) ? 8192 : 16;
+      constexpr uint64_t kStepA = (op == Op::Fwd) ? 2 : 128;   // 32 B (K-major) or 16 rows (MN-major)
+      constexpr uint64_t kStepB = (op == Op::Dw) ? 128 : 2;
+      const uint64_t a_desc0 = smem_desc_sw128(smem_u32(smem + L::kOffA), kLboA, 1024);
+      const uint64_t b_desc0 = smem_desc_sw128(smem_u32(smem + L::kOffB), kLboB, 1024);
       int stage = 0;
       uint32_t phase = 0;
       int buf = 0;
@@ -394,32 +416,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * 256);
         for (int kb = 0; kb < p.num_kb; ++kb) {
-          if (!wait(&load_full[stage], phase) || !wait(&a_full[stage], phase)) {
+          if (!wait(&full[stage], phase)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          if (lane == 0) {
-            const uint32_t sa = smem_u32(smem + L::kOffA + stage * C::kABytes);
-            const uint32_t sb = smem_u32(smem + L::kOffB + stage * C::kBBytes);
+          const uint64_t ad = a_desc0 + static_cast<uint64_t>((stage * C::kABytes) >> 4);
+          const uint64_t bd = b_desc0 + static_cast<uint64_t>((stage * C::kBBytes) >> 4);
 #pragma unroll
-            for (int kk = 0; kk < C::kBlockR / C::kUmmaK; ++kk) {
-              const uint32_t acc = (kb | kk) != 0;
-              if constexpr (op == Op::Fwd) {
-                mma_i8_pair(d_tmem, smem_desc_sw128(sa + kk * 32, 16, 1024), smem_desc_sw128(sb + kk * 32, 16, 1024),
-                            C::kIdesc, acc);
-              } else if constexpr (op == Op::Dx) {
-                mma_f16_pair(d_tmem, smem_desc_sw128(sa + kk * 2048, 8192, 1024),
-                             smem_desc_sw128(sb + kk * 32, 16, 1024), C::kIdesc, acc);
-              } else {
-                mma_f16_pair(d_tmem, smem_desc_sw128(sa + kk * 2048, 8192, 1024),
-                             smem_desc_sw128(sb + kk * 2048, 8192, 1024), C::kIdesc, acc);
-              }
-            }
-            mma_commit_pair(&empty[stage], 0x3);
-            if (kb == p.num_kb - 1) mma_commit_pair(&tmem_full[buf], 0x3);
+          for (int kk = 0; kk < C::kBlockR / C::kUmmaK; ++kk) {
+            const uint32_t acc = (kb | kk) != 0;
+            if constexpr (op == Op::Fwd)
+              mma_i8_pair(d_tmem, ad + kk * kStepA, bd + kk * kStepB, C::kIdesc, acc);
+            else
+              mma_f16_pair(d_tmem, ad + kk * kStepA, bd + kk * kStepB, C::kIdesc, acc);
           }
-          __syncwarp();
+          mma_commit_pair(&empty[stage], 0x3);
+          if (kb == p.num_kb - 1) mma_commit_pair(&tmem_full[buf], 0x3);
           if (++stage == S) {
             stage = 0;
             phase ^= 1;
@@ -431,13 +444,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
       }
       // done_bar completes in both CTAs once every MMA issued so far has finished
-      if (lane == 0) mma_commit_pair(done_bar, 0x3);
+      mma_commit_pair(done_bar, 0x3);
     }
     if (lane == 0) mbar_drain(done_bar, 0);
     __syncwarp();
-  } else if (warp < kWarpEpi0) {
+  } else if (rebuild_slot(warp) >= 0) {
     // ------------------------------------------------------------ rebuild A (both CTAs)
-    const int rt = threadIdx.x - 32 * kWarpRebuild0;  // 0..127
+    const int rt = rebuild_slot(warp) * 32 + lane;  // 0 .. kRebuildThreads-1
+    static_assert(kRebuildThreads == 256, "rebuild mappings assume 256 threads");
     int stage = 0;
     uint32_t phase = 0;
     bool ok = true;
@@ -450,53 +464,56 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const uint32_t sA = smem_u32(smem + L::kOffA + stage * C::kABytes);
         const uint32_t sSrc = smem_u32(smem + L::kOffSrc + stage * C::kSrcBytes);
         if constexpr (op == Op::Fwd) {
-          // row rt: 32 packed bytes -> 128 int8 codes, K-major with 128-byte swizzle.
-          // Lanes 4..7 of each group of 8 read their second half first (bank spread).
-          const uint32_t h = (rt >> 2) & 1;
-          const uint4 wa = ld_shared_v4(sSrc + rt * 32 + h * 16);
-          const uint4 wb = ld_shared_v4(sSrc + rt * 32 + (h ^ 1) * 16);
-          const uint4 w0 = h ? wb : wa, w1 = h ? wa : wb;
-          const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-          const uint32_t row_base = sA + rt * 128;
-#pragma unroll
-          for (int c = 0; c < 8; ++c) st_shared_v4(row_base + ((c ^ (rt & 7)) << 4), codes16_to_s8(words[c]));
-        } else if constexpr (op == Op::Dx) {
-          // reduction row n = rt % 64, output k half = rt / 64 (64 k values)
-          const int n = rt & 63, half = rt >> 6;
-          const uint4 w = ld_shared_v4(sSrc + n * 32 + half * 16);
+          // row = rt % 128: its 32 packed bytes -> 128 int8 codes, K-major with
+          // 128-byte swizzle; this thread does half rt / 128 (four 16-code chunks)
+          const int row = rt & 127, half = rt >> 7;
+          const uint4 w = ld_shared_v4(sSrc + row * 32 + half * 16);
           const uint32_t words[4] = {w.x, w.y, w.z, w.w};
-          const uint32_t base = sA + half * 8192 + n * 128;
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const uint32_t hw = words[j >> 1] >> ((j & 1) * 16);
-            st_shared_v4(base + ((j ^ (n & 7)) << 4), codes8_to_bf16(hw));
-          }
-        } else {
-          // token m = rt % 64, k half = rt / 64; q staging is 128-byte swizzled
-          const int m = rt & 63, half = rt >> 6;
-          const float s = reinterpret_cast<const float*>(smem + L::kOffSx + stage * C::kSxBytes)[m];
-          const uint32_t base = sA + half * 8192 + m * 128;
+          const uint32_t row_base = sA + row * 128;
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
-            const int c = half * 4 + i;  // logical 16-byte chunk (16 k values)
+            const int c = half * 4 + i;
+            st_shared_v4(row_base + ((c ^ (row & 7)) << 4), codes16_to_s8(words[i]));
+          }
+        } else if constexpr (op == Op::Dx) {
+          // reduction row n = rt % 64; output k range [32 q, 32 q + 32), q = rt / 64
+          const int n = rt & 63, qr = rt >> 6;
+          uint32_t w0, w1;
+          asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];" : "=r"(w0), "=r"(w1) : "r"(sSrc + n * 32 + qr * 8));
+          const uint32_t base = sA + (qr >> 1) * 8192 + n * 128;
+#pragma unroll
+          for (int jj = 0; jj < 4; ++jj) {
+            const uint32_t hw = (jj < 2 ? w0 : w1) >> ((jj & 1) * 16);
+            const int col = (qr & 1) * 4 + jj;
+            st_shared_v4(base + ((col ^ (n & 7)) << 4), codes8_to_bf16(hw));
+          }
+        } else {
+          // token m = rt % 64; k range [32 q, 32 q + 32), q = rt / 64; q staging
+          // is 128-byte swizzled
+          const int m = rt & 63, qr = rt >> 6;
+          const float s = reinterpret_cast<const float*>(smem + L::kOffSx + stage * C::kSxBytes)[m];
+          const uint32_t base = sA + (qr >> 1) * 8192 + m * 128;
+#pragma unroll
+          for (int i = 0; i < 2; ++i) {
+            const int c = qr * 2 + i;  // logical 16-byte chunk (16 k values)
             const uint4 v = ld_shared_v4(sSrc + m * 128 + ((c ^ (m & 7)) << 4));
             uint4 o0, o1;
             s8x16_to_bf16(v, s, o0, o1);
-            const int j0 = 2 * i, j1 = 2 * i + 1;  // 8-k units within this half
-            st_shared_v4(base + ((j0 ^ (m & 7)) << 4), o0);
-            st_shared_v4(base + ((j1 ^ (m & 7)) << 4), o1);
+            const int col0 = (qr & 1) * 4 + 2 * i;  // 8-k units within this 64-k chunk
+            st_shared_v4(base + ((col0 ^ (m & 7)) << 4), o0);
+            st_shared_v4(base + (((col0 + 1) ^ (m & 7)) << 4), o1);
           }
         }
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(lead(&a_full[stage]));
+        if (lane == 0) mbar_arrive_cluster(lead(&full[stage]));
         if (++stage == S) {
           stage = 0;
           phase ^= 1;
         }
       }
     }
-  } else {
+  } else if (warp >= kWarpEpi0) {
     // ------------------------------------------------------------ epilogue (both CTAs)
     const int q = warp & 3;  // TMEM lane quadrant this warp may access
     const uint32_t stg = smem_u32(smem + L::kOffEpi + (warp - kWarpEpi0) * kEpiStageBytes);
