@@ -52,55 +52,73 @@ struct Group {
   }
 };
 
-// |x| widened to fp64 exactly. Normal values are re-biased with integer
-// arithmetic (full-rate ALU instead of the conversion pipe); zero and
-// subnormals take the conversion. Inputs are finite.
-__device__ __forceinline__ double abs_to_f64(float x) {
-  const uint32_t b = __float_as_uint(x) & 0x7FFFFFFFu;
-  if (b >= 0x00800000u) return __longlong_as_double((static_cast<long long>(b) << 29) + 0x3800000000000000ll);
-  return static_cast<double>(__uint_as_float(b));
+// |w| widened to fp64 exactly from its bit pattern with the sign cleared.
+// Zero and normal values take integer arithmetic only (a bf16's fp64 high
+// word is b * 2^13 + 0x38000000: exponent re-bias 127 -> 1023; an fp32's is
+// (b >> 3) + 0x38000000 with low word b << 29), leaving the conversion pipe
+// free. Subnormals (nonzero with a zero exponent field) are converted with
+// the conversion instruction on a separate, rarely taken path. Inputs are
+// finite.
+__device__ __forceinline__ uint32_t abs_bits(float x) { return __float_as_uint(x) & 0x7FFFFFFFu; }
+
+__device__ __forceinline__ double normal_abs_to_f64(uint32_t b32) {
+  if (b32 == 0) return 0.0;
+  return __hiloint2double(static_cast<int>((b32 >> 3) + 0x38000000u), static_cast<int>(b32 << 29));
 }
 
+__device__ __forceinline__ bool is_subnormal(uint32_t b32) { return b32 - 1u < 0x007FFFFFu; }
+
+// acc + sum of |element| over one group, in element order.
 template <bool kF32>
 __device__ __forceinline__ double add_group(double acc, const Group<kF32>& a) {
+  bool sub = false;
 #pragma unroll
-  for (int i = 0; i < 16; ++i) acc = __dadd_rn(acc, abs_to_f64(a.elem(i)));
+  for (int i = 0; i < 16; ++i) sub |= is_subnormal(abs_bits(a.elem(i)));
+  if (sub) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) acc = __dadd_rn(acc, static_cast<double>(__uint_as_float(abs_bits(a.elem(i)))));
+  } else {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) acc = __dadd_rn(acc, normal_abs_to_f64(abs_bits(a.elem(i))));
+  }
   return acc;
 }
 
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait_primary() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // ---------------------------------------------------------------- S1 pass A
-// partials[b] = sum of |w| over block b's contiguous range of groups, fp64,
-// each thread summing its groups in increasing order (four loads in flight),
-// then a fixed shuffle/smem tree.
+// partials[b] = sum of |w| over block b's contiguous range of groups, fp64.
+// Each thread keeps four accumulators (group u of every four goes to
+// accumulator u; leftover groups to accumulator 0), adds them as
+// (a0 + a1) + (a2 + a3), then a fixed shuffle/smem tree.
 template <bool kF32>
 __global__ void __launch_bounds__(kQuantThreads) absmean_partials_kernel(const uint4* __restrict__ W,
                                                                          int64_t ngroups, int64_t per_block,
                                                                          double* __restrict__ partials) {
+  pdl_launch_dependents();  // the code pass may start loading W while this pass finishes
   constexpr int T = kQuantThreads;
   const int64_t g0 = static_cast<int64_t>(blockIdx.x) * per_block;
   const int64_t g1 = min(g0 + per_block, ngroups);
-  double acc = 0.0;
+  double acc[4] = {0.0, 0.0, 0.0, 0.0};
   int64_t g = g0 + threadIdx.x;
   for (; g + 3 * T < g1; g += 4 * T) {
-    Group<kF32> a, b, c, d;
-    a.load(W, g);
-    b.load(W, g + T);
-    c.load(W, g + 2 * T);
-    d.load(W, g + 3 * T);
-    acc = add_group(acc, a);
-    acc = add_group(acc, b);
-    acc = add_group(acc, c);
-    acc = add_group(acc, d);
+    Group<kF32> a[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) a[u].load(W, g + u * T);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) acc[u] = add_group(acc[u], a[u]);
   }
   for (; g < g1; g += T) {
     Group<kF32> a;
     a.load(W, g);
-    acc = add_group(acc, a);
+    acc[0] = add_group(acc[0], a);
   }
+  double t = __dadd_rn(__dadd_rn(acc[0], acc[1]), __dadd_rn(acc[2], acc[3]));
 #pragma unroll
-  for (int off = 16; off > 0; off >>= 1) acc = __dadd_rn(acc, __shfl_xor_sync(0xffffffffu, acc, off));
+  for (int off = 16; off > 0; off >>= 1) t = __dadd_rn(t, __shfl_xor_sync(0xffffffffu, t, off));
   __shared__ double warp_sums[kQuantThreads / 32];
-  if ((threadIdx.x & 31) == 0) warp_sums[threadIdx.x >> 5] = acc;
+  if ((threadIdx.x & 31) == 0) warp_sums[threadIdx.x >> 5] = t;
   __syncthreads();
   if (threadIdx.x == 0) {
     double s = 0.0;
@@ -111,8 +129,10 @@ __global__ void __launch_bounds__(kQuantThreads) absmean_partials_kernel(const u
 }
 
 // ---------------------------------------------------------------- S1 pass B
-// Every block reduces the partials in the same fixed order (so all blocks hold
-// the same gamma), then writes the codes of its range of groups.
+// Launched as a programmatic dependent of pass A: each thread first loads its
+// first groups of W (inputs pass A does not write), then waits for pass A,
+// then every block reduces the partials in the same fixed order (so all
+// blocks hold the same gamma) and writes the codes of its range of groups.
 //
 // Code rule: code = clamp(rint_half_even(fp32(w / gamma)), -1, 1) is nonzero
 // exactly when fp32(|w| / gamma) > 0.5, i.e. when the exact quotient exceeds
@@ -139,26 +159,41 @@ __global__ void __launch_bounds__(kQuantThreads) ternarize_pack_kernel(const uin
                                                                        int nparts, int64_t numel,
                                                                        uint32_t* __restrict__ packed,
                                                                        float* __restrict__ gamma_out) {
-  __shared__ float s_thr;
-  if (threadIdx.x < 32) {
-    double s = 0.0;
-    for (int i = threadIdx.x; i < nparts; i += 32) s = __dadd_rn(s, partials[i]);
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) s = __dadd_rn(s, __shfl_xor_sync(0xffffffffu, s, off));
-    if (threadIdx.x == 0) {
-      const double mean = __ddiv_rn(s, static_cast<double>(numel));
-      const float gamma = fmaxf(__double2float_rn(mean), 1e-5f);
-      const double t = __dmul_rn(static_cast<double>(gamma), 0.5 + 0x1p-25);
-      s_thr = __double2float_rd(t);
-      if (blockIdx.x == 0) *gamma_out = gamma;
-    }
-  }
-  __syncthreads();
-  const float thr = s_thr;
   constexpr int T = kQuantThreads;
   const int64_t g0 = static_cast<int64_t>(blockIdx.x) * per_block;
   const int64_t g1 = min(g0 + per_block, ngroups);
-  int64_t g = g0 + threadIdx.x;
+  const int64_t gf = g0 + threadIdx.x;
+  Group<kF32> first[4];
+#pragma unroll
+  for (int u = 0; u < 4; ++u)
+    if (gf + u * T < g1) first[u].load(W, gf + u * T);
+
+  pdl_wait_primary();  // pass A has finished and its partial sums are visible
+
+  __shared__ double red[kQuantThreads / 32];
+  __shared__ float s_thr;
+  double t = 0.0;
+  for (int i = threadIdx.x; i < nparts; i += T) t = __dadd_rn(t, partials[i]);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) t = __dadd_rn(t, __shfl_xor_sync(0xffffffffu, t, off));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = t;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double sum = 0.0;
+#pragma unroll
+    for (int w = 0; w < kQuantThreads / 32; ++w) sum = __dadd_rn(sum, red[w]);
+    const double mean = __ddiv_rn(sum, static_cast<double>(numel));
+    const float gamma = fmaxf(__double2float_rn(mean), 1e-5f);
+    s_thr = __double2float_rd(__dmul_rn(static_cast<double>(gamma), 0.5 + 0x1p-25));
+    if (blockIdx.x == 0) *gamma_out = gamma;
+  }
+  __syncthreads();
+  const float thr = s_thr;
+
+#pragma unroll
+  for (int u = 0; u < 4; ++u)
+    if (gf + u * T < g1) packed[gf + u * T] = pack_group(first[u], thr);
+  int64_t g = gf + 4 * T;
   for (; g + 3 * T < g1; g += 4 * T) {
     Group<kF32> a[4];
 #pragma unroll
@@ -220,19 +255,17 @@ __device__ __forceinline__ float warp_max(float m) {
 constexpr int kActRowsPerBlock = 4;
 
 template <int VPL>
-__global__ void __launch_bounds__(32 * kActRowsPerBlock) act_quant_kernel(const uint4* __restrict__ x, int64_t M,
-                                                                          int nv, int8_t* __restrict__ xq,
-                                                                          float* __restrict__ sx) {
-  const int lane = threadIdx.x & 31;
-  const int64_t m = static_cast<int64_t>(blockIdx.x) * kActRowsPerBlock + (threadIdx.x >> 5);
-  if (m >= M) return;
-  const uint4* row = x + m * nv;
-  uint4 v[VPL];
+__device__ __forceinline__ void load_row(const uint4* __restrict__ row, int nv, int lane, uint4 (&v)[VPL]) {
 #pragma unroll
   for (int i = 0; i < VPL; ++i) {
     const int j = lane + 32 * i;
     v[i] = j < nv ? __ldg(row + j) : make_uint4(0u, 0u, 0u, 0u);
   }
+}
+
+template <int VPL>
+__device__ __forceinline__ void quant_row(const uint4 (&v)[VPL], int nv, int lane, int64_t m,
+                                          int8_t* __restrict__ xq, float* __restrict__ sx) {
   float amax = 0.0f;
 #pragma unroll
   for (int i = 0; i < VPL; ++i) amax = absmax8(v[i], amax);
@@ -244,6 +277,36 @@ __global__ void __launch_bounds__(32 * kActRowsPerBlock) act_quant_kernel(const 
   for (int i = 0; i < VPL; ++i) {
     const int j = lane + 32 * i;
     if (j < nv) out[j] = quant8(v[i], inv);
+  }
+}
+
+// Warps stride over rows; with short rows (kPrefetch) the next row's loads
+// are issued before the current row is quantised.
+template <int VPL, bool kPrefetch>
+__global__ void __launch_bounds__(32 * kActRowsPerBlock) act_quant_kernel(const uint4* __restrict__ x, int64_t M,
+                                                                          int nv, int8_t* __restrict__ xq,
+                                                                          float* __restrict__ sx) {
+  const int lane = threadIdx.x & 31;
+  const int64_t nwarps = static_cast<int64_t>(gridDim.x) * kActRowsPerBlock;
+  int64_t m = static_cast<int64_t>(blockIdx.x) * kActRowsPerBlock + (threadIdx.x >> 5);
+  if (m >= M) return;
+  uint4 v[VPL];
+  load_row<VPL>(x + m * nv, nv, lane, v);
+  while (true) {
+    const int64_t mn = m + nwarps;
+    if constexpr (kPrefetch) {
+      uint4 vn[VPL];
+      if (mn < M) load_row<VPL>(x + mn * nv, nv, lane, vn);
+      quant_row<VPL>(v, nv, lane, m, xq, sx);
+      if (mn >= M) break;
+#pragma unroll
+      for (int i = 0; i < VPL; ++i) v[i] = vn[i];
+    } else {
+      quant_row<VPL>(v, nv, lane, m, xq, sx);
+      if (mn >= M) break;
+      load_row<VPL>(x + mn * nv, nv, lane, v);
+    }
+    m = mn;
   }
 }
 
@@ -278,6 +341,23 @@ int weight_partials_count(int64_t numel) {
   return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(kMaxPartials, want)));
 }
 
+template <bool kF32>
+static cudaError_t launch_weight_passes(const uint4* w, int64_t ngroups, int64_t per_block, int nparts, int64_t numel,
+                                        uint32_t* out, float* gamma, double* partials, cudaStream_t s) {
+  absmean_partials_kernel<kF32><<<nparts, kQuantThreads, 0, s>>>(w, ngroups, per_block, partials);
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(nparts);
+  cfg.blockDim = dim3(kQuantThreads);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, ternarize_pack_kernel<kF32>, w, ngroups, per_block,
+                            static_cast<const double*>(partials), nparts, numel, out, gamma);
+}
+
 cudaError_t launch_quantize_weight(const void* W, int w_is_f32, int64_t N, int64_t K, uint8_t* packed,
                                    float* gamma, double* partials, cudaStream_t s) {
   const int64_t numel = N * K;  // multiple of 32
@@ -286,15 +366,9 @@ cudaError_t launch_quantize_weight(const void* W, int w_is_f32, int64_t N, int64
   const int64_t per_block = (ngroups + nparts - 1) / nparts;
   const uint4* w = static_cast<const uint4*>(W);
   uint32_t* out = reinterpret_cast<uint32_t*>(packed);
-  if (w_is_f32) {
-    absmean_partials_kernel<true><<<nparts, kQuantThreads, 0, s>>>(w, ngroups, per_block, partials);
-    ternarize_pack_kernel<true>
-        <<<nparts, kQuantThreads, 0, s>>>(w, ngroups, per_block, partials, nparts, numel, out, gamma);
-  } else {
-    absmean_partials_kernel<false><<<nparts, kQuantThreads, 0, s>>>(w, ngroups, per_block, partials);
-    ternarize_pack_kernel<false>
-        <<<nparts, kQuantThreads, 0, s>>>(w, ngroups, per_block, partials, nparts, numel, out, gamma);
-  }
+  cudaError_t e = w_is_f32 ? launch_weight_passes<true>(w, ngroups, per_block, nparts, numel, out, gamma, partials, s)
+                           : launch_weight_passes<false>(w, ngroups, per_block, nparts, numel, out, gamma, partials, s);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
@@ -331,17 +405,35 @@ cudaError_t launch_quantize_weight_noalloc(const void* W, int w_is_f32, int64_t 
   return launch_quantize_weight(W, w_is_f32, N, K, packed, gamma, scratch, s);
 }
 
+template <int VPL>
+static void launch_act(const uint4* xv, int64_t M, int nv, int8_t* xq, float* sx, cudaStream_t s) {
+  constexpr bool kPrefetch = VPL <= 12;
+  static int per_sm[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  int occ = (dev >= 0 && dev < 64) ? per_sm[dev] : 0;
+  if (!occ) {
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, act_quant_kernel<VPL, kPrefetch>,
+                                                      32 * kActRowsPerBlock, 0) != cudaSuccess || occ < 1)
+      occ = 1;
+    cudaGetLastError();
+    if (dev >= 0 && dev < 64) per_sm[dev] = occ;
+  }
+  const int64_t want = (M + kActRowsPerBlock - 1) / kActRowsPerBlock;
+  const int64_t cap = static_cast<int64_t>(occ) * device_sm_count();
+  const unsigned grid = static_cast<unsigned>(want < cap ? want : cap);
+  act_quant_kernel<VPL, kPrefetch><<<grid, 32 * kActRowsPerBlock, 0, s>>>(xv, M, nv, xq, sx);
+}
+
 cudaError_t launch_quantize_act(const void* x, int64_t M, int64_t K, int8_t* xq, float* sx, cudaStream_t s) {
   if (M == 0) return cudaSuccess;
   const int nv = static_cast<int>(K / 8);
-  const unsigned grid = static_cast<unsigned>((M + kActRowsPerBlock - 1) / kActRowsPerBlock);
-  const dim3 block(32 * kActRowsPerBlock);
   const uint4* xv = static_cast<const uint4*>(x);
   const int per_lane = (nv + 31) / 32;
   switch (per_lane) {
 #define BL_ACT_CASE(n) \
   case n:              \
-    act_quant_kernel<n><<<grid, block, 0, s>>>(xv, M, nv, xq, sx); \
+    launch_act<n>(xv, M, nv, xq, sx, s); \
     break;
     BL_ACT_CASE(1) BL_ACT_CASE(2) BL_ACT_CASE(3) BL_ACT_CASE(4) BL_ACT_CASE(5) BL_ACT_CASE(6) BL_ACT_CASE(7)
     BL_ACT_CASE(8) BL_ACT_CASE(9) BL_ACT_CASE(10) BL_ACT_CASE(11) BL_ACT_CASE(12) BL_ACT_CASE(13)
@@ -350,8 +442,10 @@ cudaError_t launch_quantize_act(const void* x, int64_t M, int64_t K, int8_t* xq,
     BL_ACT_CASE(26) BL_ACT_CASE(27) BL_ACT_CASE(28) BL_ACT_CASE(29) BL_ACT_CASE(30) BL_ACT_CASE(31)
     BL_ACT_CASE(32)
 #undef BL_ACT_CASE
-    default:
-      act_quant_long_kernel<<<grid, block, 0, s>>>(xv, M, nv, xq, sx);
+    default: {
+      const unsigned grid = static_cast<unsigned>((M + kActRowsPerBlock - 1) / kActRowsPerBlock);
+      act_quant_long_kernel<<<grid, 32 * kActRowsPerBlock, 0, s>>>(xv, M, nv, xq, sx);
+    }
   }
   return cudaGetLastError();
 }

@@ -286,3 +286,19 @@ def test_full_size_parity_sampled(name):
     xh = ref.bf16_bits_to_f32(ref.round_to_bf16_bits(ref.dequantize_activations(q, sx)))
     dw_o = ref.round_to_bf16_bits(ref.backward_dw(dyf[:, nrows], xh))
     assert_close(ref.bf16_bits_to_f32(bits(bufs.dW)[nrows]), ref.bf16_bits_to_f32(dw_o), "dW")
+
+
+@pytest.mark.parametrize("w_dtype", [torch.float32, torch.bfloat16])
+def test_weight_subnormals_and_zeros(w_dtype):
+    """Masters holding zeros and subnormals (the exact widening's rare path)
+    next to ordinary values: gamma and codes stay bit-exact."""
+    M, N, K = 16, 64, 256
+    x, w, dy = make_inputs(M, K, N, w_dtype=torch.float32, w_init="normal0.02", seed=17)
+    g = torch.Generator().manual_seed(5)
+    pick = torch.rand(N, K, generator=g)
+    tiny = torch.full((N, K), 3e-39 if w_dtype == torch.bfloat16 else 7e-42)
+    w = torch.where(pick < 0.05, tiny * torch.sign(torch.randn(N, K, generator=g)), w)
+    w = torch.where((pick >= 0.05) & (pick < 0.1), torch.zeros_like(w), w)
+    w = w.to(w_dtype)
+    assert (w.float().abs() < 1.17e-38).any() and (w.float() != 0).any()
+    check_all(run_step(x, w, dy), oracle_step(x, w, dy), N)
