@@ -147,6 +147,22 @@ class ClockSampler:
         return bool(self.BAD & set(rec["reasons"]))
 
 
+# ----------------------------------------------------------------- multi-rank aggregation
+
+def job_time_ms(local_ms: float, world: int, device=None) -> float:
+    """Device time of the whole job: the max over ranks (all ranks call)."""
+    if world <= 1:
+        return float(local_ms)
+    t = torch.tensor([float(local_ms)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tops(ops_per_rank_step: float, world: int, steps: int, job_ms: float) -> float:
+    """Whole-job throughput: every rank's work divided by the job time."""
+    return ops_per_rank_step * world * steps / (job_ms * 1e-3) / 1e12
+
+
 # ----------------------------------------------------------------- our arm
 
 STAGES = ["quantize_weight", "quantize_act", "forward", "backward_dx", "backward_dw"]
@@ -238,11 +254,7 @@ def run_ours(args, rank, world, local_rank):
     if bl.bl_get_last_error() != 0:
         raise RuntimeError("device error during the timed region")
 
-    # max over ranks of the device time
-    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-    job_ms = float(t.item())
+    job_ms = job_time_ms(total_ms, world, dev)
 
     e2e = measure_e2e(bl, args, dev, stream, bufs, x_cpu, w_cpu, dy_cpu, world)
     if rank != 0:
@@ -250,7 +262,7 @@ def run_ours(args, rank, world, local_rank):
 
     ops_step = 6.0 * M * N * K
     ms_per_step = job_ms / args.steps
-    value = ops_step * world * args.steps / (job_ms * 1e-3) / 1e12
+    value = job_tops(ops_step, world, args.steps, job_ms)
     peaks, peak_src = load_peaks()
     work = stage_work(M, N, K, 2 if wl.w_dtype == torch.bfloat16 else 4)
     traffic = load_traffic(args.workload)
@@ -334,17 +346,13 @@ def measure_e2e(bl, args, dev, stream, bufs, x_cpu, w_cpu, dy_cpu, world):
         one()
     e.record(stream)
     torch.cuda.synchronize(dev)
-    ms = s.elapsed_time(e)
-    t = torch.tensor([ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    ms = job_time_ms(s.elapsed_time(e), world, dev)
     M, K = x_cpu.shape
     N = w_cpu.shape[0]
-    ops = 6.0 * M * N * K * world * steps
     h2d = sum(tt.numel() * tt.element_size() for tt in (xh, wh, dyh))
     d2h = sum(tt.numel() * tt.element_size() for tt in (yh, dxh, dwh))
-    return {"value": round(ops / (float(t.item()) * 1e-3) / 1e12, 3), "unit": "TOPS",
-            "ms_per_step": round(float(t.item()) / steps, 4), "steps": steps,
+    return {"value": round(job_tops(6.0 * M * N * K, world, steps, ms), 3), "unit": "TOPS",
+            "ms_per_step": round(ms / steps, 4), "steps": steps,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
 

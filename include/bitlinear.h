@@ -200,6 +200,16 @@ bl_status bl_get_last_error(void);
 /* Clears the current device's error word (synchronous). */
 bl_status bl_reset_error(void);
 
+/*
+ * Failure-detection self-test: enqueues one warp that waits on a pipeline
+ * barrier nothing ever completes, with the same bounded wait (2 s) every
+ * pipeline kernel uses. The wait gives up, records BL_ERR_TIMEOUT in the
+ * device error word and the kernel returns; bl_get_last_error then reports
+ * BL_ERR_TIMEOUT and the CUDA context stays usable. Clear it with
+ * bl_reset_error. Returns the launch status.
+ */
+bl_status bl_selftest_timeout(void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -42,6 +42,7 @@ SIGNATURES = {
     "bl_export_weights": (_I32, [_VP, _VP, _I64, _I64, _VP, _VP, _VP]),
     "bl_get_last_error": (_I32, []),
     "bl_reset_error": (_I32, []),
+    "bl_selftest_timeout": (_I32, [_VP]),
 }
 
 

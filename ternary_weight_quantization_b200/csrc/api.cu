@@ -224,6 +224,13 @@ bl_status bl_export_weights(const uint8_t* w_packed, const float* gamma, int64_t
   return cuda_status(cudaStreamSynchronize(st), "export sync");
 }
 
+bl_status bl_selftest_timeout(void* stream) {
+  g_msg[0] = 0;
+  int* err = nullptr;
+  if (bl_status s = current_device(&err)) return s;
+  return cuda_status(bl::launch_selftest_timeout(err, static_cast<cudaStream_t>(stream)), "bl_selftest_timeout");
+}
+
 bl_status bl_get_last_error(void) {
   g_msg[0] = 0;
   if (cudaError_t e = cudaDeviceSynchronize(); e != cudaSuccess) return cuda_status(e, "cudaDeviceSynchronize");

@@ -38,6 +38,9 @@ cudaError_t launch_backward_dx(const void* dY, const uint8_t* w_packed, const fl
 cudaError_t launch_backward_dw(const void* dY, const int8_t* xq, const float* sx, int64_t M, int64_t N, int64_t K,
                                void* dW, int dw_is_f32, int accumulate, int* err, cudaStream_t s);
 
+// One warp waiting on an mbarrier that is never completed (bounded wait test).
+cudaError_t launch_selftest_timeout(int* err, cudaStream_t s);
+
 // Number of SMs of the current device (cached per device).
 int device_sm_count();
 
