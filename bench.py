@@ -2,7 +2,7 @@
 
 One step = one pass of the whole hot path over one batch:
   S1 bl_quantize_weight (2 launches) -> S2 bl_quantize_act -> S3 bl_forward
-  -> S4 bl_backward dX -> S4 bl_backward dW                    (6 launches)
+  -> S4 bl_backward (dX and dW in one launch)                  (5 launches)
 
 Default workload: the up-projection BitLinear 2560 -> 6912 at 8 x 512 tokens
 (M=4096, K=2560, N=6912; x, dY bf16 ~ N(0,1), W bf16 kaiming-uniform).
@@ -165,8 +165,8 @@ def job_tops(ops_per_rank_step: float, world: int, steps: int, job_ms: float) ->
 
 # ----------------------------------------------------------------- our arm
 
-STAGES = ["quantize_weight", "quantize_act", "forward", "backward_dx", "backward_dw"]
-LAUNCHES_PER_STEP = 6
+STAGES = ["quantize_weight", "quantize_act", "forward", "backward"]
+LAUNCHES_PER_STEP = 5  # S1 two passes, S2, S3, S4 (dX and dW in one launch)
 
 
 def stage_work(M, N, K, w_bytes):
@@ -175,8 +175,7 @@ def stage_work(M, N, K, w_bytes):
         "quantize_weight": {"bound": "hbm", "bytes": N * K * w_bytes + N * K // 4 + 4},
         "quantize_act": {"bound": "hbm", "bytes": M * K * 2 + M * K + 4 * M},
         "forward": {"bound": "tensor", "ops": 2 * M * N * K, "dtype": "int8"},
-        "backward_dx": {"bound": "tensor", "ops": 2 * M * N * K, "dtype": "bf16"},
-        "backward_dw": {"bound": "tensor", "ops": 2 * M * N * K, "dtype": "bf16"},
+        "backward": {"bound": "tensor", "ops": 4 * M * N * K, "dtype": "bf16"},
     }
 
 
@@ -206,12 +205,9 @@ def run_ours(args, rank, world, local_rank):
         bl.bl_forward(bufs.xq, bufs.sx, bufs.w_packed, bufs.gamma, bufs.y, None, stream)
         if evs:
             evs[3].record(stream)
-        bl.bl_backward(dy, bufs.xq, bufs.sx, bufs.w_packed, bufs.gamma, bufs.dX, None, False, stream)
+        bl.bl_backward(dy, bufs.xq, bufs.sx, bufs.w_packed, bufs.gamma, bufs.dX, bufs.dW, False, stream)
         if evs:
             evs[4].record(stream)
-        bl.bl_backward(dy, bufs.xq, bufs.sx, bufs.w_packed, bufs.gamma, None, bufs.dW, False, stream)
-        if evs:
-            evs[5].record(stream)
 
     for _ in range(args.warmup):
         flush.fill_(1)
@@ -221,7 +217,7 @@ def run_ours(args, rank, world, local_rank):
         raise RuntimeError("device error during warm-up")
 
     def timed():
-        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(STAGES) + 1)] for _ in range(args.steps)]
         if world > 1:
             torch.distributed.barrier()
         torch.cuda.synchronize(dev)
@@ -236,7 +232,7 @@ def run_ours(args, rank, world, local_rank):
         for e in evs:
             for j, s in enumerate(STAGES):
                 per_stage[s] += e[j].elapsed_time(e[j + 1])
-            total += e[0].elapsed_time(e[5])
+            total += e[0].elapsed_time(e[len(STAGES)])
         return total, per_stage
 
     sampler = ClockSampler(dev.index if dev.index is not None else 0)

@@ -217,7 +217,7 @@ class StepBuffers:
 
 
 def bitlinear_step(x, W, dY, bufs: StepBuffers, stream=None):
-    """One BitLinear forward + backward: S1 -> S2 -> S3 -> S4 (six kernel launches)."""
+    """One BitLinear forward + backward: S1 -> S2 -> S3 -> S4 (five kernel launches)."""
     bl_quantize_weight(W, bufs.w_packed, bufs.gamma, bufs.workspace, stream)
     bl_quantize_act(x, bufs.xq, bufs.sx, stream)
     bl_forward(bufs.xq, bufs.sx, bufs.w_packed, bufs.gamma, bufs.y, None, stream)

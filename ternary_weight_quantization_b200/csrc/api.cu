@@ -192,19 +192,9 @@ bl_status bl_backward(const void* dY, const int8_t* xq, const float* sx, const u
     return fail(BL_ERR_ALIGNMENT, "tensors must be 16-byte aligned");
   int* err = nullptr;
   if (bl_status s = current_device(&err)) return s;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (dX) {
-    if (bl_status s = cuda_status(bl::launch_backward_dx(dY, w_packed, gamma, M, N, K, dX, err, st),
-                                  "bl_backward dX launch"))
-      return s;
-  }
-  if (dW) {
-    if (bl_status s = cuda_status(
-            bl::launch_backward_dw(dY, xq, sx, M, N, K, dW, dw_dtype == BL_F32, accumulate_dW != 0, err, st),
-            "bl_backward dW launch"))
-      return s;
-  }
-  return BL_OK;
+  return cuda_status(bl::launch_backward(dY, xq, sx, w_packed, gamma, M, N, K, dX, dW, dw_dtype == BL_F32,
+                                         accumulate_dW != 0, err, static_cast<cudaStream_t>(stream)),
+                     "bl_backward launch");
 }
 
 bl_status bl_export_weights(const uint8_t* w_packed, const float* gamma, int64_t N, int64_t K,

@@ -178,10 +178,11 @@ __device__ __forceinline__ void cp_async_8(void* dst, const void* src, uint32_t 
                : "memory");
 }
 
-// The barrier receives one arrival once all of this thread's earlier
-// cp.async copies have landed (counts toward the barrier's expected count).
-__device__ __forceinline__ void cp_async_mbar_arrive_noinc(uint64_t* bar) {
-  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+// Holds the barrier's current phase open until all of this thread's earlier
+// cp.async copies have landed (the pending count is raised now and lowered
+// when they complete, so it is not one of the expected arrivals).
+__device__ __forceinline__ void cp_async_mbar_arrive(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
 // ---------------------------------------------------------------- tcgen05

@@ -32,11 +32,10 @@ cudaError_t launch_forward(const int8_t* xq, const float* sx, const uint8_t* w_p
                            int64_t M, int64_t N, int64_t K, void* y, int32_t* debug_acc, int* err,
                            cudaStream_t s);
 
-cudaError_t launch_backward_dx(const void* dY, const uint8_t* w_packed, const float* gamma, int64_t M, int64_t N,
-                               int64_t K, void* dX, int* err, cudaStream_t s);
-
-cudaError_t launch_backward_dw(const void* dY, const int8_t* xq, const float* sx, int64_t M, int64_t N, int64_t K,
-                               void* dW, int dw_is_f32, int accumulate, int* err, cudaStream_t s);
+// dX and/or dW (either output may be null) in one launch.
+cudaError_t launch_backward(const void* dY, const int8_t* xq, const float* sx, const uint8_t* w_packed,
+                            const float* gamma, int64_t M, int64_t N, int64_t K, void* dX, void* dW, int dw_is_f32,
+                            int accumulate, int* err, cudaStream_t s);
 
 // One warp waiting on an mbarrier that is never completed (bounded wait test).
 cudaError_t launch_selftest_timeout(int* err, cudaStream_t s);

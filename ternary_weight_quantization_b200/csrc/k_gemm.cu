@@ -18,17 +18,23 @@
 // 128 A rows from the staged 2-bit / INT8 source (never written to HBM) and
 // TMA-loads its own BN/2 B rows; the leader CTA issues one M=256 MMA that
 // reads both CTAs' shared memory and accumulates 128 rows into each CTA's
-// TMEM. Splitting both operands across the pair halves the B traffic per SM
-// compared with a single-CTA 128 x BN tile. No TMA multicast is used.
+// TMEM. No TMA multicast is used.
 //
-// Warp roles (512 threads per CTA):
+// The forward family runs one GEMM per launch. The backward family runs dX
+// and dW in ONE launch: the two GEMMs' tiles (different lengths: N/64 and M/64
+// k-blocks) are spread over the CTA pairs by a longest-processing-time
+// schedule computed on the host and passed in the kernel parameters, so the
+// pairs finish together instead of idling through a partly filled last wave.
+//
+// Warp w runs on SM sub-partition w % 4. Roles (512 threads per CTA):
 //   warp 0      loads: TMA for B, for Dw's q / s_x and for the packed codes
 //               (cp.async for the codes when K % 64 != 0: their rows are then
 //               not 16-byte aligned, which a tensor map requires)
 //   warp 1      TMEM allocation (2 x 256 columns, pair-wide); in the leader
 //               CTA one lane issues the tcgen05.mma
 //   warps 2-4, 6-8, 10-11  rebuild A from the staged source
-//   warps 5, 9  idle (keeps sub-partition 1 free for the MMA warp)
+//   warps 5, 9  idle (keeps sub-partition 1 to the MMA warp: rebuild warps
+//               there would compete with it for issue slots)
 //   warps 12-15 epilogue: TMEM -> registers -> smem (transpose) -> global
 // Barriers: src_full (per CTA: staged source landed), full (leader: both
 // CTAs' B bytes landed and both CTAs' A rebuilt -- one wait per stage for the
@@ -36,19 +42,23 @@
 // tcgen05.commit), tmem_empty (leader: both CTAs' epilogues drained a TMEM
 // buffer). The MMA lane's loop is kept minimal because the tensor core's
 // instruction queue is shallow: the next stage's MMAs must be issued while
-// the current stage's last MMA still executes. Every wait is
-// bounded: on expiry a CTA records a timeout in the device error word, tells
-// its peer, drains what it has in flight, frees TMEM and exits.
+// the current stage's last MMA still executes. Every wait is bounded: on
+// expiry a CTA records a timeout in the device error word, tells its peer,
+// drains what it has in flight, frees TMEM and exits.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <cstdarg>
+#include <cstddef>
 #include <cstdint>
 #include <cstdio>
 #include <cstdlib>
+#include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "bl_device.cuh"
 #include "bl_internal.h"
@@ -56,9 +66,6 @@
 namespace bl {
 namespace {
 
-// Warp w runs on SM sub-partition w % 4. The MMA warp (1) keeps sub-partition
-// 1 to itself apart from one epilogue warp: rebuild warps there would compete
-// with it for issue slots and delay the next MMAs.
 constexpr int kThreads = 512;
 constexpr int kWarpLoad = 0;
 constexpr int kWarpMma = 1;
@@ -77,65 +84,75 @@ constexpr int BM = 128;              // A rows per CTA; a pair covers 2 * BM
 constexpr uint32_t kTmemCols = 512;  // two accumulators at columns 0 and 256
 constexpr int kEpiStageBytes = 32 * 32 * 4;  // per epilogue warp
 constexpr int kSmemLimit = 232448;           // per-CTA dynamic shared memory on sm_100
+constexpr int kMaxPairs = 128;
+constexpr int kMaxSchedTiles = 2048;
 
 enum class Op { Fwd, Dx, Dw };
+enum class Family { Fwd, Bwd };
 
-template <Op op, int BN>
-struct Cfg;
+// Stage geometry of a family. Every op issues four MMAs per stage.
+template <Family F, int BN>
+struct Geo;
 
 // Forward: reduction over k in blocks of 128 bytes; kind::i8 consumes 32 k per MMA.
 template <int BN>
-struct Cfg<Op::Fwd, BN> {
+struct Geo<Family::Fwd, BN> {
   static constexpr int kBlockR = 128;
-  static constexpr int kUmmaK = 32;
   static constexpr int kABytes = BM * 128;         // 128 rows x 128 int8
   static constexpr int kBBytes = (BN / 2) * 128;   // BN/2 rows x 128 int8
   static constexpr int kSrcBytes = BM * 32;        // packed: 128 rows x 32 bytes
   static constexpr int kSxBytes = 0;
-  static constexpr uint32_t kSrcArrivals = 32;     // cp.async lanes (1 with the TMA source)
-  static constexpr uint32_t kIdesc = make_idesc(2 /*s32*/, 1 /*s8*/, 0, 0, 2 * BM, BN);
 };
 
-// dX: reduction over n in blocks of 64; kind::f16 consumes 16 n per MMA.
-template <int BN>
-struct Cfg<Op::Dx, BN> {
-  static constexpr int kBlockR = 64;
-  static constexpr int kUmmaK = 16;
-  static constexpr int kABytes = BM * 64 * 2;      // 128 k x 64 n bf16
-  static constexpr int kBBytes = (BN / 2) * 128;   // BN/2 m x 64 n bf16
-  static constexpr int kSrcBytes = 64 * 32;        // packed: 64 rows (n) x 32 bytes (128 k)
-  static constexpr int kSxBytes = 0;
-  static constexpr uint32_t kSrcArrivals = 32;
-  static constexpr uint32_t kIdesc = make_idesc(1 /*f32*/, 1 /*bf16*/, 1 /*A MN*/, 0, 2 * BM, BN);
-};
-
-// dW: reduction over m in blocks of 64. B is MN-major: BN/2 must be a
+// Backward: reduction blocks of 64 (n for dX, m for dW); kind::f16 consumes
+// 16 per MMA. The source slot fits dW's q tile (64 x 128 int8, swizzled) and
+// dX's packed tile (64 rows x 32 bytes). dW's B is MN-major: BN/2 must be a
 // multiple of 64 (whole 128-byte swizzle atoms).
 template <int BN>
-struct Cfg<Op::Dw, BN> {
+struct Geo<Family::Bwd, BN> {
   static_assert((BN / 2) % 64 == 0, "MN-major B needs whole 64-element chunks");
   static constexpr int kBlockR = 64;
-  static constexpr int kUmmaK = 16;
-  static constexpr int kABytes = BM * 64 * 2;      // 128 k x 64 m bf16
-  static constexpr int kBBytes = (BN / 2) * 128;   // BN/2 n x 64 m bf16 ((BN/2)/64 TMA boxes)
-  static constexpr int kSrcBytes = 64 * 128;       // q: 64 rows (m) x 128 int8 (k), swizzled
-  static constexpr int kSxBytes = 64 * 4;          // s_x of the 64 tokens
-  static constexpr uint32_t kSrcArrivals = 1;      // expect_tx
-  static constexpr uint32_t kIdesc = make_idesc(1, 1, 1 /*A MN*/, 1 /*B MN*/, 2 * BM, BN);
+  static constexpr int kABytes = BM * 64 * 2;      // 128 x 64 bf16
+  static constexpr int kBBytes = (BN / 2) * 128;   // BN/2 x 64 bf16
+  static constexpr int kSrcBytes = 64 * 128;
+  static constexpr int kSxBytes = 64 * 4;
 };
 
+// Per-op MMA operand formats: instruction descriptor, descriptor leading byte
+// offsets and the per-MMA step of each operand's start address (16-byte units).
 template <Op op, int BN>
+struct MmaCfg;
+template <int BN>
+struct MmaCfg<Op::Fwd, BN> {
+  static constexpr uint32_t kIdesc = make_idesc(2 /*s32*/, 1 /*s8*/, 0, 0, 2 * BM, BN);
+  static constexpr uint32_t kLboA = 16, kLboB = 16;
+  static constexpr uint64_t kStepA = 2, kStepB = 2;  // 32 bytes of K (K-major)
+};
+template <int BN>
+struct MmaCfg<Op::Dx, BN> {
+  static constexpr uint32_t kIdesc = make_idesc(1 /*f32*/, 1 /*bf16*/, 1 /*A MN*/, 0, 2 * BM, BN);
+  static constexpr uint32_t kLboA = 8192, kLboB = 16;
+  static constexpr uint64_t kStepA = 128, kStepB = 2;  // 16 rows (MN-major) / 32 bytes (K-major)
+};
+template <int BN>
+struct MmaCfg<Op::Dw, BN> {
+  static constexpr uint32_t kIdesc = make_idesc(1, 1, 1 /*A MN*/, 1 /*B MN*/, 2 * BM, BN);
+  static constexpr uint32_t kLboA = 8192, kLboB = 8192;
+  static constexpr uint64_t kStepA = 128, kStepB = 128;
+};
+
+template <Family F, int BN>
 struct Layout {
-  using C = Cfg<op, BN>;
-  static constexpr int kStageBytes = C::kABytes + C::kBBytes + C::kSrcBytes + C::kSxBytes;
+  using G = Geo<F, BN>;
+  static constexpr int kStageBytes = G::kABytes + G::kBBytes + G::kSrcBytes + G::kSxBytes;
   static constexpr int kReserve = 1024 /*base alignment*/ + kNumEpiWarps * kEpiStageBytes + 512;
   static constexpr int kS0 = (kSmemLimit - kReserve) / kStageBytes;
   static constexpr int kS = kS0 > 8 ? 8 : kS0;
   static constexpr int kOffA = 0;
-  static constexpr int kOffB = kOffA + kS * C::kABytes;
-  static constexpr int kOffSrc = kOffB + kS * C::kBBytes;
-  static constexpr int kOffSx = kOffSrc + kS * C::kSrcBytes;
-  static constexpr int kOffEpi = kOffSx + kS * C::kSxBytes;
+  static constexpr int kOffB = kOffA + kS * G::kABytes;
+  static constexpr int kOffSrc = kOffB + kS * G::kBBytes;
+  static constexpr int kOffSx = kOffSrc + kS * G::kSrcBytes;
+  static constexpr int kOffEpi = kOffSx + kS * G::kSxBytes;
   static constexpr int kOffBar = kOffEpi + kNumEpiWarps * kEpiStageBytes;
   // src_full[S], full[S], empty[S], tmem_full[2], tmem_empty[2], done
   static constexpr int kNumBars = 3 * kS + 5;
@@ -144,26 +161,65 @@ struct Layout {
   static constexpr int kDynBytes = kBytes + 1024;
   static_assert(kS >= 2, "at least two pipeline stages");
   static_assert(kDynBytes <= kSmemLimit, "shared memory budget");
-  static_assert(C::kABytes % 1024 == 0 && C::kBBytes % 1024 == 0 && C::kSrcBytes % 1024 == 0, "alignment");
+  static_assert(G::kABytes % 1024 == 0 && G::kBBytes % 1024 == 0 && G::kSrcBytes % 1024 == 0, "alignment");
+};
+
+// One GEMM of a launch.
+struct OpParams {
+  int rows_a;     // extent of the A-row index i (N for Fwd, K for Dx/Dw)
+  int rows_b;     // extent of the B-row index j (M for Fwd/Dx, N for Dw)
+  int red;        // reduction length (K, N, M)
+  int tiles_a, num_kb, ntiles;
+  void* out;      // [rows_b][ldo]
+  int64_t ldo;
+  int out_f32;    // Dw
+  int accumulate; // Dw
+  int src_tma;    // Fwd/Dx: packed codes by TMA (K % 64 == 0) instead of cp.async
 };
 
 struct GemmParams {
-  int rows_a;      // extent of the A-row index i (N for Fwd, K for Dx/Dw)
-  int rows_b;      // extent of the B-row index j (M for Fwd/Dx, N for Dw)
-  int red;         // reduction length (K, N, M)
-  int tiles_a, tiles_b, num_kb, num_tiles;
-  int64_t K;                  // in_features (row length of packed codes / q)
-  const uint8_t* packed;      // Fwd, Dx
-  const float* sx;            // Fwd epilogue
-  const float* gamma;         // Fwd, Dx epilogue
-  void* out;                  // [rows_b][ldo]
-  int64_t ldo;
-  int32_t* debug_acc;         // Fwd, optional
-  int out_f32;                // Dw
-  int accumulate;             // Dw
-  int src_tma;                // Fwd/Dx: packed codes by TMA (K % 64 == 0) instead of cp.async
+  OpParams op[2];         // Fwd: op[0]; Bwd: op[0] = dX, op[1] = dW (either may have 0 tiles)
+  int ntiles;             // op[0].ntiles + op[1].ntiles
+  int64_t K;              // in_features (row length of packed codes / q)
+  const uint8_t* packed;  // Fwd, Dx
+  const float* sx;        // Fwd epilogue
+  const float* gamma;     // Fwd, Dx epilogue
+  int32_t* debug_acc;     // Fwd, optional
   int* err;
+  int use_sched;          // 1: pair p runs sched_tile[sched_start[p] .. sched_start[p+1])
+                          // 0: pair p runs tiles p, p + npairs, ...
+  uint16_t sched_start[kMaxPairs + 1];
+  uint16_t sched_tile[kMaxSchedTiles];
 };
+
+struct TileInfo {
+  int opi;  // index into GemmParams::op
+  int a0;   // first A row of this CTA
+  int bp;   // first B row of the pair tile
+};
+
+__device__ __forceinline__ bool next_tile(const GemmParams& p, int pair, int npairs, int i, int& tile) {
+  if (p.use_sched) {
+    const int idx = p.sched_start[pair] + i;
+    if (idx >= p.sched_start[pair + 1]) return false;
+    tile = p.sched_tile[idx];
+  } else {
+    tile = pair + i * npairs;
+    if (tile >= p.ntiles) return false;
+  }
+  return true;
+}
+
+template <int BN>
+__device__ __forceinline__ TileInfo decode_tile(const GemmParams& p, int tile, uint32_t rank) {
+  TileInfo t;
+  t.opi = tile >= p.op[0].ntiles ? 1 : 0;
+  const int u = tile - (t.opi ? p.op[0].ntiles : 0);
+  const OpParams& P = p.op[t.opi];
+  t.a0 = (u % P.tiles_a) * (2 * BM) + static_cast<int>(rank) * BM;
+  t.bp = (u / P.tiles_a) * BN;
+  return t;
+}
 
 // ---------------------------------------------------------------- rebuild helpers
 
@@ -238,20 +294,284 @@ __device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
   return v;
 }
 
-// ---------------------------------------------------------------- the kernel
+// ---------------------------------------------------------------- per-op stage work
 
 // Staging word of element (row j, column i) of an epilogue warp's 32 x 32
 // transpose tile; flipping bit 2 of i on odd rows keeps both the row-wise
 // writes and the 16-byte reads of two adjacent rows free of bank conflicts.
 __device__ __forceinline__ uint32_t stg_word(int j, int i) { return j * 32 + (i ^ ((j & 1) << 2)); }
 
+struct Maps {
+  const CUtensorMap* b;
+  const CUtensorMap* src;
+  const CUtensorMap* sx;
+};
+
+// Load warp, one stage: this CTA's B rows (pair TMA, counted on the leader's
+// `full`), and the source of its A rows (counted on the local `src_full`,
+// which expects one arrival).
+template <Op op, Family F, int BN>
+__device__ __forceinline__ void load_stage(const GemmParams& p, const OpParams& P, const Maps& m, bool leader,
+                                           int lane, int a0, int bh, int kb, uint64_t* full, uint32_t full_lead,
+                                           uint64_t* src_full, uint8_t* sB, uint8_t* sSrc, uint8_t* sSx) {
+  using G = Geo<F, BN>;
+  const int r0 = kb * G::kBlockR;
+  const int kq = static_cast<int>(p.K / 4);
+  if (lane == 0) {
+    if (leader) mbar_arrive_expect_tx(full, 2 * G::kBBytes);
+    if constexpr (op == Op::Dw) {
+#pragma unroll
+      for (int j = 0; j < (BN / 2) / 64; ++j) tma_load_2d_pair(m.b, full_lead, sB + j * 8192, bh + 64 * j, r0);
+      mbar_arrive_expect_tx(src_full, 64 * 128 + 64 * 4);
+      tma_load_2d(m.src, src_full, sSrc, a0, r0);
+      tma_load_2d(m.sx, src_full, sSx, r0, 0);
+    } else {
+      tma_load_2d_pair(m.b, full_lead, sB, r0, bh);
+      if (P.src_tma) {
+        // packed codes as one TMA box: Fwd rows a0..a0+127 x bytes [kb*32, +32);
+        // Dx rows (n) r0..r0+63 x bytes [a0/4, +32)
+        if constexpr (op == Op::Fwd) {
+          mbar_arrive_expect_tx(src_full, BM * 32);
+          tma_load_2d(m.src, src_full, sSrc, kb * 32, a0);
+        } else {
+          mbar_arrive_expect_tx(src_full, 64 * 32);
+          tma_load_2d(m.src, src_full, sSrc, a0 / 4, r0);
+        }
+      }
+    }
+  }
+  if constexpr (op != Op::Dw) {
+    if (!P.src_tma) {
+      // packed codes by 8-byte cp.async (rows not 16-byte aligned); every lane's
+      // copies hold the phase open until they land, lane 0 gives the one arrival
+      constexpr int kChunks = (op == Op::Fwd) ? 16 : 8;  // per lane
+#pragma unroll
+      for (int it = 0; it < kChunks; ++it) {
+        const int c = lane + 32 * it;
+        const int row = c >> 2, part = c & 3;
+        bool valid;
+        const uint8_t* src;
+        if constexpr (op == Op::Fwd) {
+          // packed rows a0..a0+127, bytes [kb*32, kb*32+32)
+          valid = (a0 + row < P.rows_a) && (r0 + part * 32 < P.red);
+          src = p.packed + static_cast<int64_t>(a0 + row) * kq + kb * 32 + part * 8;
+        } else {
+          // packed rows (n) r0..r0+63, bytes covering k in [a0, a0+128)
+          valid = (r0 + row < P.red) && (a0 + part * 32 < P.rows_a);
+          src = p.packed + static_cast<int64_t>(r0 + row) * kq + a0 / 4 + part * 8;
+        }
+        cp_async_8(sSrc + row * 32 + part * 8, valid ? src : p.packed, valid ? 8u : 0u);
+      }
+      cp_async_mbar_arrive(src_full);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(src_full);
+    }
+  }
+}
+
+// Rebuild warps, one stage: A rows of this CTA from the staged source.
+template <Op op, Family F, int BN>
+__device__ __forceinline__ void rebuild_stage(int rt, uint32_t sA, uint32_t sSrc, const float* sSx) {
+  if constexpr (op == Op::Fwd) {
+    // row = rt % 128: its 32 packed bytes -> 128 int8 codes, K-major with
+    // 128-byte swizzle; this thread does half rt / 128 (four 16-code chunks)
+    const int row = rt & 127, half = rt >> 7;
+    const uint4 w = ld_shared_v4(sSrc + row * 32 + half * 16);
+    const uint32_t words[4] = {w.x, w.y, w.z, w.w};
+    const uint32_t row_base = sA + row * 128;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int c = half * 4 + i;
+      st_shared_v4(row_base + ((c ^ (row & 7)) << 4), codes16_to_s8(words[i]));
+    }
+  } else if constexpr (op == Op::Dx) {
+    // reduction row n = rt % 64; output k range [32 q, 32 q + 32), q = rt / 64
+    const int n = rt & 63, qr = rt >> 6;
+    uint32_t w0, w1;
+    asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];" : "=r"(w0), "=r"(w1) : "r"(sSrc + n * 32 + qr * 8));
+    const uint32_t base = sA + (qr >> 1) * 8192 + n * 128;
+#pragma unroll
+    for (int jj = 0; jj < 4; ++jj) {
+      const uint32_t hw = (jj < 2 ? w0 : w1) >> ((jj & 1) * 16);
+      const int col = (qr & 1) * 4 + jj;
+      st_shared_v4(base + ((col ^ (n & 7)) << 4), codes8_to_bf16(hw));
+    }
+  } else {
+    // token m = rt % 64; k range [32 q, 32 q + 32), q = rt / 64; q staging is
+    // 128-byte swizzled
+    const int m = rt & 63, qr = rt >> 6;
+    const float s = sSx[m];
+    const uint32_t base = sA + (qr >> 1) * 8192 + m * 128;
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const int c = qr * 2 + i;  // logical 16-byte chunk (16 k values)
+      const uint4 v = ld_shared_v4(sSrc + m * 128 + ((c ^ (m & 7)) << 4));
+      uint4 o0, o1;
+      s8x16_to_bf16(v, s, o0, o1);
+      const int col0 = (qr & 1) * 4 + 2 * i;  // 8-k units within this 64-k chunk
+      st_shared_v4(base + ((col0 ^ (m & 7)) << 4), o0);
+      st_shared_v4(base + (((col0 + 1) ^ (m & 7)) << 4), o1);
+    }
+  }
+}
+
+// MMA lane, one stage: four pair MMAs.
 template <Op op, int BN>
+__device__ __forceinline__ void mma_stage(uint32_t d_tmem, uint32_t sa, uint32_t sb, int kb) {
+  using M = MmaCfg<op, BN>;
+  const uint64_t ad = smem_desc_sw128(sa, M::kLboA, 1024);
+  const uint64_t bd = smem_desc_sw128(sb, M::kLboB, 1024);
+#pragma unroll
+  for (int kk = 0; kk < 4; ++kk) {
+    const uint32_t acc = (kb | kk) != 0;
+    if constexpr (op == Op::Fwd)
+      mma_i8_pair(d_tmem, ad + kk * M::kStepA, bd + kk * M::kStepB, M::kIdesc, acc);
+    else
+      mma_f16_pair(d_tmem, ad + kk * M::kStepA, bd + kk * M::kStepB, M::kIdesc, acc);
+  }
+}
+
+// Epilogue, one 32-column chunk already transposed into staging: each lane
+// stores 8 consecutive i of one output row j, 4 rows per pass.
+template <Op op>
+__device__ __forceinline__ void store_chunk(const GemmParams& p, const OpParams& P, uint32_t stg, int lane, int q,
+                                            int a0, int jbase, float gamma, float col_scale) {
+  const int seg = (lane & 3) * 8;
+  const int i0 = a0 + q * 32 + seg;
+#pragma unroll
+  for (int pass = 0; pass < 4; ++pass) {
+    const int jl = pass * 8 + (lane >> 2);
+    const int j = jbase + jl;
+    float row_scale = 0.0f;
+    if constexpr (op == Op::Fwd) row_scale = __shfl_sync(0xffffffffu, col_scale, jl);
+    if (j >= P.rows_b || i0 >= P.rows_a) continue;
+    // the two 4-word halves of this 8-word run (swapped on odd rows)
+    const int sw = (jl & 1) << 2;
+    const uint4 v0 = ld_shared_v4(stg + stg_word(jl, seg + sw) * 4);
+    const uint4 v1 = ld_shared_v4(stg + stg_word(jl, seg + (4 ^ sw)) * 4);
+    const uint4 lo = sw ? v1 : v0, hi = sw ? v0 : v1;
+    const uint32_t acc[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+    const int nvalid = min(8, P.rows_a - i0);
+    const int64_t off = static_cast<int64_t>(j) * P.ldo + i0;
+    if constexpr (op == Op::Fwd) {
+      __nv_bfloat16* y = static_cast<__nv_bfloat16*>(P.out) + off;
+      uint32_t pk[4];
+#pragma unroll
+      for (int e = 0; e < 8; e += 2) {
+        const __nv_bfloat162 b2 =
+            __floats2bfloat162_rn(__fmul_rn(static_cast<float>(static_cast<int32_t>(acc[e])), row_scale),
+                                  __fmul_rn(static_cast<float>(static_cast<int32_t>(acc[e + 1])), row_scale));
+        pk[e / 2] = *reinterpret_cast<const uint32_t*>(&b2);
+      }
+      if (nvalid == 8 && (P.ldo % 8) == 0) {
+        *reinterpret_cast<uint4*>(y) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      } else {
+        for (int e = 0; e < nvalid; ++e)
+          reinterpret_cast<uint16_t*>(y)[e] = static_cast<uint16_t>(pk[e / 2] >> ((e & 1) * 16));
+      }
+      if (p.debug_acc) {
+        int32_t* d = p.debug_acc + off;
+        if (nvalid == 8 && (P.ldo % 4) == 0) {
+          reinterpret_cast<uint4*>(d)[0] = lo;
+          reinterpret_cast<uint4*>(d)[1] = hi;
+        } else {
+          for (int e = 0; e < nvalid; ++e) d[e] = static_cast<int32_t>(acc[e]);
+        }
+      }
+    } else if constexpr (op == Op::Dx) {
+      __nv_bfloat16* dx = static_cast<__nv_bfloat16*>(P.out) + off;
+      uint32_t pk[4];
+#pragma unroll
+      for (int e = 0; e < 8; e += 2) {
+        const __nv_bfloat162 b2 = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(acc[e]), gamma),
+                                                        __fmul_rn(__uint_as_float(acc[e + 1]), gamma));
+        pk[e / 2] = *reinterpret_cast<const uint32_t*>(&b2);
+      }
+      *reinterpret_cast<uint4*>(dx) = make_uint4(pk[0], pk[1], pk[2], pk[3]);  // K % 32 == 0
+    } else {
+      float v[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) v[e] = __uint_as_float(acc[e]);
+      if (P.out_f32) {
+        float4* dw = reinterpret_cast<float4*>(static_cast<float*>(P.out) + off);
+        if (P.accumulate) {
+          const float4 o0 = dw[0], o1 = dw[1];
+          v[0] = __fadd_rn(v[0], o0.x); v[1] = __fadd_rn(v[1], o0.y);
+          v[2] = __fadd_rn(v[2], o0.z); v[3] = __fadd_rn(v[3], o0.w);
+          v[4] = __fadd_rn(v[4], o1.x); v[5] = __fadd_rn(v[5], o1.y);
+          v[6] = __fadd_rn(v[6], o1.z); v[7] = __fadd_rn(v[7], o1.w);
+        }
+        dw[0] = make_float4(v[0], v[1], v[2], v[3]);
+        dw[1] = make_float4(v[4], v[5], v[6], v[7]);
+      } else {
+        uint4* dw = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(P.out) + off);
+        if (P.accumulate) {
+          const uint4 o = *dw;
+          const uint32_t ow[4] = {o.x, o.y, o.z, o.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            v[2 * e] = __fadd_rn(v[2 * e], __uint_as_float(ow[e] << 16));
+            v[2 * e + 1] = __fadd_rn(v[2 * e + 1], __uint_as_float(ow[e] & 0xFFFF0000u));
+          }
+        }
+        uint32_t pk[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const __nv_bfloat162 b2 = __floats2bfloat162_rn(v[2 * e], v[2 * e + 1]);
+          pk[e] = *reinterpret_cast<const uint32_t*>(&b2);
+        }
+        *dw = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      }
+    }
+  }
+}
+
+// Epilogue, one tile: drain the TMEM accumulator chunk by chunk.
+template <Op op, int BN>
+__device__ __forceinline__ void epilogue_tile(const GemmParams& p, const OpParams& P, uint32_t tmem_base, int buf,
+                                              uint32_t stg, int lane, int q, int a0, int bp, float gamma,
+                                              uint32_t tmem_empty_lead) {
+  // forward: s_x[m] * gamma of the tile's BN columns; lane l holds column 32c + l
+  float col_scale[BN / 32];
+#pragma unroll
+  for (int c = 0; c < BN / 32; ++c) {
+    col_scale[c] = 0.0f;
+    if constexpr (op == Op::Fwd) {
+      const int j = bp + c * 32 + lane;
+      col_scale[c] = j < P.rows_b ? __fmul_rn(__ldg(p.sx + j), gamma) : 0.0f;
+    }
+  }
+#pragma unroll
+  for (int c = 0; c < BN / 32; ++c) {
+    uint32_t r[32];
+    tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * 256 + c * 32, r);
+    tmem_ld_wait();
+    if (c == BN / 32 - 1) {
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(tmem_empty_lead);
+    }
+    // transpose through smem: staging(j, lane) = D[row lane][column j]
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+      asm volatile("st.shared.b32 [%0], %1;" ::"r"(stg + stg_word(j, lane) * 4), "r"(r[j]) : "memory");
+    __syncwarp();
+    store_chunk<op>(p, P, stg, lane, q, a0, bp + c * 32, gamma, col_scale[c]);
+    __syncwarp();
+  }
+}
+
+// ---------------------------------------------------------------- the kernel
+
+template <Family F, int BN>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
-    gemm_pair_kernel(const __grid_constant__ CUtensorMap map_b, const __grid_constant__ CUtensorMap map_src,
-                     const __grid_constant__ CUtensorMap map_sx, const GemmParams p) {
-  using C = Cfg<op, BN>;
-  using L = Layout<op, BN>;
+    gemm_pair_kernel(const __grid_constant__ CUtensorMap map_b0, const __grid_constant__ CUtensorMap map_src0,
+                     const __grid_constant__ CUtensorMap map_b1, const __grid_constant__ CUtensorMap map_src1,
+                     const __grid_constant__ CUtensorMap map_sx, const __grid_constant__ GemmParams p) {
+  using G = Geo<F, BN>;
+  using L = Layout<F, BN>;
   constexpr int S = L::kS;
+  constexpr Op kOp0 = (F == Family::Fwd) ? Op::Fwd : Op::Dx;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -275,7 +595,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
-      mbar_init(&src_full[s], p.src_tma ? 1u : C::kSrcArrivals);
+      mbar_init(&src_full[s], 1);
       mbar_init(&full[s], 1 + 2 * kNumRebuildWarps);  // leader's expect_tx + both CTAs' rebuild warps
       mbar_init(&empty[s], 1);
       issued_parity[s] = -1;
@@ -304,79 +624,45 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     return false;
   };
   auto lead = [&](uint64_t* bar) -> uint32_t { return map_to_rank(smem_u32(bar), 0); };
-
-  const int kq = static_cast<int>(p.K / 4);  // bytes per packed row
+  const Maps maps0{&map_b0, &map_src0, &map_sx};
+  const Maps maps1{&map_b1, &map_src1, &map_sx};
 
   if (warp == kWarpLoad) {
     // ------------------------------------------------------------ loads
     if (lane == 0) {
-      prefetch_tensormap(&map_b);
-      if (op == Op::Dw || p.src_tma) prefetch_tensormap(&map_src);
-      if constexpr (op == Op::Dw) prefetch_tensormap(&map_sx);
+      if (p.op[0].ntiles) {
+        prefetch_tensormap(&map_b0);
+        if (p.op[0].src_tma) prefetch_tensormap(&map_src0);
+      }
+      if (F == Family::Bwd && p.op[1].ntiles) {
+        prefetch_tensormap(&map_b1);
+        prefetch_tensormap(&map_src1);
+        prefetch_tensormap(&map_sx);
+      }
     }
     int stage = 0;
     uint32_t phase = 0;
     bool ok = true;
-    for (int tile = pair; ok && tile < p.num_tiles; tile += npairs) {
-      const int a0 = (tile % p.tiles_a) * (2 * BM) + static_cast<int>(rank) * BM;  // this CTA's A rows
-      const int bh = (tile / p.tiles_a) * BN + static_cast<int>(rank) * (BN / 2);  // this CTA's B rows
-      for (int kb = 0; kb < p.num_kb; ++kb) {
+    int tile;
+    for (int i = 0; ok && next_tile(p, pair, npairs, i, tile); ++i) {
+      const TileInfo t = decode_tile<BN>(p, tile, rank);
+      const OpParams& P = p.op[t.opi];
+      const int bh = t.bp + static_cast<int>(rank) * (BN / 2);  // this CTA's B rows
+      for (int kb = 0; kb < P.num_kb; ++kb) {
         if (!wait(&empty[stage], phase ^ 1)) {
           ok = false;
           break;
         }
-        uint8_t* sB = smem + L::kOffB + stage * C::kBBytes;
-        uint8_t* sSrc = smem + L::kOffSrc + stage * C::kSrcBytes;
-        const int r0 = kb * C::kBlockR;
-        if (lane == 0) {
-          issued_parity[stage] = static_cast<int>(phase);
-          if (leader) mbar_arrive_expect_tx(&full[stage], 2 * C::kBBytes);
-          const uint32_t lb = lead(&full[stage]);
-          if constexpr (op == Op::Dw) {
-#pragma unroll
-            for (int j = 0; j < (BN / 2) / 64; ++j) tma_load_2d_pair(&map_b, lb, sB + j * 8192, bh + 64 * j, r0);
-            mbar_arrive_expect_tx(&src_full[stage], C::kSrcBytes + C::kSxBytes);
-            tma_load_2d(&map_src, &src_full[stage], sSrc, a0, r0);
-            tma_load_2d(&map_sx, &src_full[stage], smem + L::kOffSx + stage * C::kSxBytes, r0, 0);
-          } else {
-            tma_load_2d_pair(&map_b, lb, sB, r0, bh);
-          }
-        }
-        if (op != Op::Dw && p.src_tma) {
-          // packed codes as one TMA box: Fwd rows a0..a0+127 x bytes [kb*32, +32);
-          // Dx rows (n) r0..r0+63 x bytes [a0/4, +32)
-          if (lane == 0) {
-            mbar_arrive_expect_tx(&src_full[stage], C::kSrcBytes);
-            if constexpr (op == Op::Fwd)
-              tma_load_2d(&map_src, &src_full[stage], sSrc, kb * 32, a0);
-            else
-              tma_load_2d(&map_src, &src_full[stage], sSrc, a0 / 4, r0);
-          }
-        } else if constexpr (op == Op::Fwd) {
-          // packed rows a0..a0+127, bytes [kb*32, kb*32+32): 512 chunks of 8 bytes
-#pragma unroll
-          for (int it = 0; it < 16; ++it) {
-            const int c = lane + 32 * it;
-            const int row = c >> 2, part = c & 3;
-            const bool valid = (a0 + row < p.rows_a) && (r0 + part * 32 < p.red);
-            const uint8_t* src = valid ? p.packed + static_cast<int64_t>(a0 + row) * kq + kb * 32 + part * 8
-                                       : p.packed;
-            cp_async_8(sSrc + row * 32 + part * 8, src, valid ? 8u : 0u);
-          }
-          cp_async_mbar_arrive_noinc(&src_full[stage]);
-        } else if constexpr (op == Op::Dx) {
-          // packed rows (n) r0..r0+63, bytes covering k in [a0, a0+128): 256 chunks
-#pragma unroll
-          for (int it = 0; it < 8; ++it) {
-            const int c = lane + 32 * it;
-            const int row = c >> 2, part = c & 3;
-            const bool valid = (r0 + row < p.red) && (a0 + part * 32 < p.rows_a);
-            const uint8_t* src =
-                valid ? p.packed + static_cast<int64_t>(r0 + row) * kq + a0 / 4 + part * 8 : p.packed;
-            cp_async_8(sSrc + row * 32 + part * 8, src, valid ? 8u : 0u);
-          }
-          cp_async_mbar_arrive_noinc(&src_full[stage]);
-        }
+        if (lane == 0) issued_parity[stage] = static_cast<int>(phase);
+        uint8_t* sB = smem + L::kOffB + stage * G::kBBytes;
+        uint8_t* sSrc = smem + L::kOffSrc + stage * G::kSrcBytes;
+        uint8_t* sSx = smem + L::kOffSx + stage * G::kSxBytes;
+        if (t.opi == 0)
+          load_stage<kOp0, F, BN>(p, P, maps0, leader, lane, t.a0, bh, kb, &full[stage], lead(&full[stage]),
+                                  &src_full[stage], sB, sSrc, sSx);
+        else if constexpr (F == Family::Bwd)
+          load_stage<Op::Dw, F, BN>(p, P, maps1, leader, lane, t.a0, bh, kb, &full[stage], lead(&full[stage]),
+                                    &src_full[stage], sB, sSrc, sSx);
         if (++stage == S) {
           stage = 0;
           phase ^= 1;
@@ -398,41 +684,32 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   } else if (warp == kWarpMma) {
     // ------------------------------------------------------------ MMA issue (leader CTA, one lane)
     if (leader && lane == 0) {
-      // descriptors of stage 0; a stage or k step is an offset (in 16-byte
-      // units) added to the start-address field
-      constexpr uint32_t kLboA = (op == Op::Fwd) ? 16 : 8192;
-      constexpr uint32_t kLboB = (op == Op::Dw) ? 8192 : 16;
-      constexpr uint64_t kStepA = (op == Op::Fwd) ? 2 : 128;   // 32 B (K-major) or 16 rows (MN-major)
-      constexpr uint64_t kStepB = (op == Op::Dw) ? 128 : 2;
-      const uint64_t a_desc0 = smem_desc_sw128(smem_u32(smem + L::kOffA), kLboA, 1024);
-      const uint64_t b_desc0 = smem_desc_sw128(smem_u32(smem + L::kOffB), kLboB, 1024);
+      const uint32_t sa0 = smem_u32(smem + L::kOffA), sb0 = smem_u32(smem + L::kOffB);
       int stage = 0;
       uint32_t phase = 0;
       int buf = 0;
       uint32_t buf_phase = 0;
       bool ok = true;
-      for (int tile = pair; ok && tile < p.num_tiles; tile += npairs) {
+      int tile;
+      for (int i = 0; ok && next_tile(p, pair, npairs, i, tile); ++i) {
+        const int opi = tile >= p.op[0].ntiles ? 1 : 0;
+        const int num_kb = p.op[opi].num_kb;
         if (!wait(&tmem_empty[buf], buf_phase ^ 1)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * 256);
-        for (int kb = 0; kb < p.num_kb; ++kb) {
+        for (int kb = 0; kb < num_kb; ++kb) {
           if (!wait(&full[stage], phase)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint64_t ad = a_desc0 + static_cast<uint64_t>((stage * C::kABytes) >> 4);
-          const uint64_t bd = b_desc0 + static_cast<uint64_t>((stage * C::kBBytes) >> 4);
-#pragma unroll
-          for (int kk = 0; kk < C::kBlockR / C::kUmmaK; ++kk) {
-            const uint32_t acc = (kb | kk) != 0;
-            if constexpr (op == Op::Fwd)
-              mma_i8_pair(d_tmem, ad + kk * kStepA, bd + kk * kStepB, C::kIdesc, acc);
-            else
-              mma_f16_pair(d_tmem, ad + kk * kStepA, bd + kk * kStepB, C::kIdesc, acc);
-          }
+          const uint32_t sa = sa0 + stage * G::kABytes, sb = sb0 + stage * G::kBBytes;
+          if (opi == 0)
+            mma_stage<kOp0, BN>(d_tmem, sa, sb, kb);
+          else if constexpr (F == Family::Bwd)
+            mma_stage<Op::Dw, BN>(d_tmem, sa, sb, kb);
           mma_commit_pair(&empty[stage], 0x3);
-          if (kb == p.num_kb - 1) mma_commit_pair(&tmem_full[buf], 0x3);
+          if (kb == num_kb - 1) mma_commit_pair(&tmem_full[buf], 0x3);
           if (++stage == S) {
             stage = 0;
             phase ^= 1;
@@ -450,60 +727,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else if (rebuild_slot(warp) >= 0) {
     // ------------------------------------------------------------ rebuild A (both CTAs)
-    const int rt = rebuild_slot(warp) * 32 + lane;  // 0 .. kRebuildThreads-1
     static_assert(kRebuildThreads == 256, "rebuild mappings assume 256 threads");
+    const int rt = rebuild_slot(warp) * 32 + lane;
     int stage = 0;
     uint32_t phase = 0;
     bool ok = true;
-    for (int tile = pair; ok && tile < p.num_tiles; tile += npairs) {
-      for (int kb = 0; kb < p.num_kb; ++kb) {
+    int tile;
+    for (int i = 0; ok && next_tile(p, pair, npairs, i, tile); ++i) {
+      const int opi = tile >= p.op[0].ntiles ? 1 : 0;
+      const int num_kb = p.op[opi].num_kb;
+      for (int kb = 0; kb < num_kb; ++kb) {
         if (!wait(&src_full[stage], phase)) {
           ok = false;
           break;
         }
-        const uint32_t sA = smem_u32(smem + L::kOffA + stage * C::kABytes);
-        const uint32_t sSrc = smem_u32(smem + L::kOffSrc + stage * C::kSrcBytes);
-        if constexpr (op == Op::Fwd) {
-          // row = rt % 128: its 32 packed bytes -> 128 int8 codes, K-major with
-          // 128-byte swizzle; this thread does half rt / 128 (four 16-code chunks)
-          const int row = rt & 127, half = rt >> 7;
-          const uint4 w = ld_shared_v4(sSrc + row * 32 + half * 16);
-          const uint32_t words[4] = {w.x, w.y, w.z, w.w};
-          const uint32_t row_base = sA + row * 128;
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int c = half * 4 + i;
-            st_shared_v4(row_base + ((c ^ (row & 7)) << 4), codes16_to_s8(words[i]));
-          }
-        } else if constexpr (op == Op::Dx) {
-          // reduction row n = rt % 64; output k range [32 q, 32 q + 32), q = rt / 64
-          const int n = rt & 63, qr = rt >> 6;
-          uint32_t w0, w1;
-          asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];" : "=r"(w0), "=r"(w1) : "r"(sSrc + n * 32 + qr * 8));
-          const uint32_t base = sA + (qr >> 1) * 8192 + n * 128;
-#pragma unroll
-          for (int jj = 0; jj < 4; ++jj) {
-            const uint32_t hw = (jj < 2 ? w0 : w1) >> ((jj & 1) * 16);
-            const int col = (qr & 1) * 4 + jj;
-            st_shared_v4(base + ((col ^ (n & 7)) << 4), codes8_to_bf16(hw));
-          }
-        } else {
-          // token m = rt % 64; k range [32 q, 32 q + 32), q = rt / 64; q staging
-          // is 128-byte swizzled
-          const int m = rt & 63, qr = rt >> 6;
-          const float s = reinterpret_cast<const float*>(smem + L::kOffSx + stage * C::kSxBytes)[m];
-          const uint32_t base = sA + (qr >> 1) * 8192 + m * 128;
-#pragma unroll
-          for (int i = 0; i < 2; ++i) {
-            const int c = qr * 2 + i;  // logical 16-byte chunk (16 k values)
-            const uint4 v = ld_shared_v4(sSrc + m * 128 + ((c ^ (m & 7)) << 4));
-            uint4 o0, o1;
-            s8x16_to_bf16(v, s, o0, o1);
-            const int col0 = (qr & 1) * 4 + 2 * i;  // 8-k units within this 64-k chunk
-            st_shared_v4(base + ((col0 ^ (m & 7)) << 4), o0);
-            st_shared_v4(base + (((col0 + 1) ^ (m & 7)) << 4), o1);
-          }
-        }
+        const uint32_t sA = smem_u32(smem + L::kOffA + stage * G::kABytes);
+        const uint32_t sSrc = smem_u32(smem + L::kOffSrc + stage * G::kSrcBytes);
+        const float* sSx = reinterpret_cast<const float*>(smem + L::kOffSx + stage * G::kSxBytes);
+        if (opi == 0)
+          rebuild_stage<kOp0, F, BN>(rt, sA, sSrc, sSx);
+        else if constexpr (F == Family::Bwd)
+          rebuild_stage<Op::Dw, F, BN>(rt, sA, sSrc, sSx);
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster(lead(&full[stage]));
@@ -517,131 +761,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ epilogue (both CTAs)
     const int q = warp & 3;  // TMEM lane quadrant this warp may access
     const uint32_t stg = smem_u32(smem + L::kOffEpi + (warp - kWarpEpi0) * kEpiStageBytes);
-    const float gamma = (op == Op::Dw) ? 1.0f : __ldg(p.gamma);
+    const float gamma = p.gamma ? __ldg(p.gamma) : 1.0f;
     int buf = 0;
     uint32_t buf_phase = 0;
-    for (int tile = pair; tile < p.num_tiles; tile += npairs) {
-      const int a0 = (tile % p.tiles_a) * (2 * BM) + static_cast<int>(rank) * BM;
-      const int b0 = (tile / p.tiles_a) * BN;
-      // forward: s_x[m] * gamma of the tile's BN columns, loaded before the
-      // accumulator is ready; lane l holds column 32c + l of chunk c
-      float col_scale[BN / 32];
-      if constexpr (op == Op::Fwd) {
-#pragma unroll
-        for (int c = 0; c < BN / 32; ++c) {
-          const int j = b0 + c * 32 + lane;
-          col_scale[c] = j < p.rows_b ? __fmul_rn(__ldg(p.sx + j), gamma) : 0.0f;
-        }
-      }
+    int tile;
+    for (int i = 0; next_tile(p, pair, npairs, i, tile); ++i) {
+      const TileInfo t = decode_tile<BN>(p, tile, rank);
+      const OpParams& P = p.op[t.opi];
       if (!wait(&tmem_full[buf], buf_phase)) break;
       tc_fence_after();
-#pragma unroll
-      for (int c = 0; c < BN / 32; ++c) {
-        uint32_t r[32];
-        tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * 256 + c * 32, r);
-        tmem_ld_wait();
-        if (c == BN / 32 - 1) {
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive_cluster(lead(&tmem_empty[buf]));
-        }
-        // transpose through smem: staging(j, lane) = D[row lane][column j]
-#pragma unroll
-        for (int j = 0; j < 32; ++j)
-          asm volatile("st.shared.b32 [%0], %1;" ::"r"(stg + stg_word(j, lane) * 4), "r"(r[j]) : "memory");
-        __syncwarp();
-        // each lane stores 8 consecutive i of one output row j, 4 rows per pass
-        const int seg = (lane & 3) * 8;
-        const int i0 = a0 + q * 32 + seg;
-#pragma unroll
-        for (int pass = 0; pass < 4; ++pass) {
-          const int jl = pass * 8 + (lane >> 2);
-          const int j = b0 + c * 32 + jl;
-          float row_scale = 0.0f;
-          if constexpr (op == Op::Fwd) row_scale = __shfl_sync(0xffffffffu, col_scale[c], jl);
-          if (j >= p.rows_b || i0 >= p.rows_a) continue;
-          // the two 4-word halves of this 8-word run (swapped on odd rows)
-          const int sw = (jl & 1) << 2;
-          const uint4 v0 = ld_shared_v4(stg + stg_word(jl, seg + sw) * 4);
-          const uint4 v1 = ld_shared_v4(stg + stg_word(jl, seg + (4 ^ sw)) * 4);
-          const uint4 lo = sw ? v1 : v0, hi = sw ? v0 : v1;
-          const uint32_t acc[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
-          const int nvalid = min(8, p.rows_a - i0);
-          const int64_t off = static_cast<int64_t>(j) * p.ldo + i0;
-          if constexpr (op == Op::Fwd) {
-            const float scale = row_scale;
-            __nv_bfloat16* y = static_cast<__nv_bfloat16*>(p.out) + off;
-            uint32_t pk[4];
-#pragma unroll
-            for (int e = 0; e < 8; e += 2) {
-              const __nv_bfloat162 b2 =
-                  __floats2bfloat162_rn(__fmul_rn(static_cast<float>(static_cast<int32_t>(acc[e])), scale),
-                                        __fmul_rn(static_cast<float>(static_cast<int32_t>(acc[e + 1])), scale));
-              pk[e / 2] = *reinterpret_cast<const uint32_t*>(&b2);
-            }
-            if (nvalid == 8 && (p.ldo % 8) == 0) {
-              *reinterpret_cast<uint4*>(y) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-            } else {
-              for (int e = 0; e < nvalid; ++e)
-                reinterpret_cast<uint16_t*>(y)[e] = static_cast<uint16_t>(pk[e / 2] >> ((e & 1) * 16));
-            }
-            if (p.debug_acc) {
-              int32_t* d = p.debug_acc + off;
-              if (nvalid == 8 && (p.ldo % 4) == 0) {
-                reinterpret_cast<uint4*>(d)[0] = lo;
-                reinterpret_cast<uint4*>(d)[1] = hi;
-              } else {
-                for (int e = 0; e < nvalid; ++e) d[e] = static_cast<int32_t>(acc[e]);
-              }
-            }
-          } else if constexpr (op == Op::Dx) {
-            __nv_bfloat16* dx = static_cast<__nv_bfloat16*>(p.out) + off;
-            uint32_t pk[4];
-#pragma unroll
-            for (int e = 0; e < 8; e += 2) {
-              const __nv_bfloat162 b2 = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(acc[e]), gamma),
-                                                              __fmul_rn(__uint_as_float(acc[e + 1]), gamma));
-              pk[e / 2] = *reinterpret_cast<const uint32_t*>(&b2);
-            }
-            *reinterpret_cast<uint4*>(dx) = make_uint4(pk[0], pk[1], pk[2], pk[3]);  // K % 32 == 0
-          } else {
-            float v[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) v[e] = __uint_as_float(acc[e]);
-            if (p.out_f32) {
-              float4* dw = reinterpret_cast<float4*>(static_cast<float*>(p.out) + off);
-              if (p.accumulate) {
-                const float4 o0 = dw[0], o1 = dw[1];
-                v[0] = __fadd_rn(v[0], o0.x); v[1] = __fadd_rn(v[1], o0.y);
-                v[2] = __fadd_rn(v[2], o0.z); v[3] = __fadd_rn(v[3], o0.w);
-                v[4] = __fadd_rn(v[4], o1.x); v[5] = __fadd_rn(v[5], o1.y);
-                v[6] = __fadd_rn(v[6], o1.z); v[7] = __fadd_rn(v[7], o1.w);
-              }
-              dw[0] = make_float4(v[0], v[1], v[2], v[3]);
-              dw[1] = make_float4(v[4], v[5], v[6], v[7]);
-            } else {
-              uint4* dw = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + off);
-              if (p.accumulate) {
-                const uint4 o = *dw;
-                const uint32_t ow[4] = {o.x, o.y, o.z, o.w};
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                  v[2 * e] = __fadd_rn(v[2 * e], __uint_as_float(ow[e] << 16));
-                  v[2 * e + 1] = __fadd_rn(v[2 * e + 1], __uint_as_float(ow[e] & 0xFFFF0000u));
-                }
-              }
-              uint32_t pk[4];
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const __nv_bfloat162 b2 = __floats2bfloat162_rn(v[2 * e], v[2 * e + 1]);
-                pk[e] = *reinterpret_cast<const uint32_t*>(&b2);
-              }
-              *dw = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-            }
-          }
-        }
-        __syncwarp();
-      }
+      if (t.opi == 0)
+        epilogue_tile<kOp0, BN>(p, P, tmem_base, buf, stg, lane, q, t.a0, t.bp, gamma, lead(&tmem_empty[buf]));
+      else if constexpr (F == Family::Bwd)
+        epilogue_tile<Op::Dw, BN>(p, P, tmem_base, buf, stg, lane, q, t.a0, t.bp, gamma, lead(&tmem_empty[buf]));
       if (++buf == 2) {
         buf = 0;
         buf_phase ^= 1;
@@ -713,34 +845,113 @@ bool make_map_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint6
   return true;
 }
 
-template <Op op, int BN>
-cudaError_t launch_pair(const CUtensorMap& mb, const CUtensorMap& msrc, const CUtensorMap& msx, GemmParams p,
-                        int npairs, cudaStream_t s) {
-  using L = Layout<op, BN>;
+// Number of CTA pairs of this kernel that can be resident at once (GPCs with
+// an odd number of SMs leave one SM out of pairing), capped at SMs / 2.
+template <Family F, int BN>
+int resident_pairs() {
+  static int cached[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && cached[dev]) return cached[dev];
+  using L = Layout<F, BN>;
+  int n = device_sm_count() / 2;
+  if (cudaFuncSetAttribute(gemm_pair_kernel<F, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kDynBytes) ==
+      cudaSuccess) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(2 * n);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = L::kDynBytes;
+    int clusters = 0;
+    if (cudaOccupancyMaxActiveClusters(&clusters, gemm_pair_kernel<F, BN>, &cfg) == cudaSuccess && clusters > 0 &&
+        clusters < n)
+      n = clusters;
+  }
+  cudaGetLastError();
+  if (n > kMaxPairs) n = kMaxPairs;
+  if (dev >= 0 && dev < 64) cached[dev] = n;
+  return n;
+}
+
+void fill_op(OpParams& P, int rows_a, int rows_b, int red, int block_r, int bn) {
+  P.rows_a = rows_a;
+  P.rows_b = rows_b;
+  P.red = red;
+  P.tiles_a = (rows_a + 2 * BM - 1) / (2 * BM);
+  P.num_kb = (red + block_r - 1) / block_r;
+  P.ntiles = rows_a > 0 && rows_b > 0 ? P.tiles_a * ((rows_b + bn - 1) / bn) : 0;
+}
+
+// Longest-processing-time schedule of the launch's tiles over the pairs:
+// tiles in decreasing cost (k-blocks plus a per-tile overhead), each to the
+// least-loaded pair. Falls back to round robin beyond the parameter capacity.
+// The last schedule is cached (thread-local) by its inputs.
+void build_schedule(GemmParams& p, int npairs) {
+  p.use_sched = 0;
+  if (p.ntiles > kMaxSchedTiles || npairs > kMaxPairs || p.ntiles <= npairs) return;
+  struct Key {
+    int n0, n1, kb0, kb1, np;
+  };
+  thread_local Key key{-1, -1, -1, -1, -1};
+  thread_local std::vector<uint16_t> start, tiles;
+  const Key k{p.op[0].ntiles, p.op[1].ntiles, p.op[0].num_kb, p.op[1].num_kb, npairs};
+  if (std::memcmp(&k, &key, sizeof(Key)) != 0) {
+    constexpr int kTileOverhead = 4;  // k-block equivalents per tile (epilogue, pipeline ramp)
+    const int cost[2] = {k.kb0 + kTileOverhead, k.kb1 + kTileOverhead};
+    std::vector<int> order(p.ntiles);
+    for (int t = 0; t < p.ntiles; ++t) order[t] = t;
+    auto tcost = [&](int t) { return cost[t >= k.n0 ? 1 : 0]; };
+    std::stable_sort(order.begin(), order.end(), [&](int a, int b) { return tcost(a) > tcost(b); });
+    std::vector<long long> load(npairs, 0);
+    std::vector<std::vector<uint16_t>> lists(npairs);
+    for (int t : order) {
+      int best = 0;
+      for (int q = 1; q < npairs; ++q)
+        if (load[q] < load[best]) best = q;
+      load[best] += tcost(t);
+      lists[best].push_back(static_cast<uint16_t>(t));
+    }
+    start.assign(npairs + 1, 0);
+    tiles.clear();
+    for (int q = 0; q < npairs; ++q) {
+      start[q] = static_cast<uint16_t>(tiles.size());
+      tiles.insert(tiles.end(), lists[q].begin(), lists[q].end());
+    }
+    start[npairs] = static_cast<uint16_t>(tiles.size());
+    key = k;
+  }
+  std::memcpy(p.sched_start, start.data(), start.size() * sizeof(uint16_t));
+  std::memcpy(p.sched_tile, tiles.data(), tiles.size() * sizeof(uint16_t));
+  p.use_sched = 1;
+}
+
+template <Family F, int BN>
+cudaError_t launch_pair(const CUtensorMap* maps, GemmParams& p, int npairs, cudaStream_t s) {
+  using L = Layout<F, BN>;
   static int configured[64] = {};  // attribute set once per process per device
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !configured[dev]) {
     cudaError_t e =
-        cudaFuncSetAttribute(gemm_pair_kernel<op, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kDynBytes);
+        cudaFuncSetAttribute(gemm_pair_kernel<F, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kDynBytes);
     if (e != cudaSuccess) return e;
     configured[dev] = 1;
   }
-  p.tiles_a = (p.rows_a + 2 * BM - 1) / (2 * BM);
-  p.tiles_b = (p.rows_b + BN - 1) / BN;
-  p.num_kb = (p.red + Cfg<op, BN>::kBlockR - 1) / Cfg<op, BN>::kBlockR;
-  p.num_tiles = p.tiles_a * p.tiles_b;
-  const int pairs = p.num_tiles < npairs ? p.num_tiles : npairs;
+  p.ntiles = p.op[0].ntiles + p.op[1].ntiles;
+  if (p.ntiles == 0) return cudaSuccess;
+  const int pairs = p.ntiles < npairs ? p.ntiles : npairs;
+  build_schedule(p, pairs);
   static const bool log = std::getenv("BL_LOG") != nullptr;
   if (log)
-    std::fprintf(stderr, "[bitlinear] gemm op=%d BN=%d stages=%d smem=%d tiles=%dx%d kb=%d pairs=%d (of %d)\n",
-                 static_cast<int>(op), BN, L::kS, L::kDynBytes, p.tiles_a, p.tiles_b, p.num_kb, pairs, npairs);
-  gemm_pair_kernel<op, BN><<<2 * pairs, kThreads, L::kDynBytes, s>>>(mb, msrc, msx, p);
+    std::fprintf(stderr, "[bitlinear] gemm family=%d BN=%d stages=%d smem=%d tiles=%d+%d kb=%d/%d pairs=%d sched=%d\n",
+                 static_cast<int>(F), BN, L::kS, L::kDynBytes, p.op[0].ntiles, p.op[1].ntiles, p.op[0].num_kb,
+                 p.op[1].num_kb, pairs, p.use_sched);
+  gemm_pair_kernel<F, BN><<<2 * pairs, kThreads, L::kDynBytes, s>>>(maps[0], maps[1], maps[2], maps[3], maps[4], p);
   return cudaGetLastError();
 }
 
-// B rows per pair tile: the candidate with the fewest tile-rows of work per
-// pair after wave quantisation (waves x BN), ties to the larger tile.
+// B rows per pair tile for the forward: the candidate with the fewest
+// tile-rows of work per pair after wave quantisation (waves x BN), ties to
+// the larger tile.
 int choose_bn(int rows_a, int rows_b, int npairs, const int* cands, int ncands) {
   const int tiles_a = (rows_a + 2 * BM - 1) / (2 * BM);
   int best = cands[0];
@@ -755,39 +966,6 @@ int choose_bn(int rows_a, int rows_b, int npairs, const int* cands, int ncands) 
     }
   }
   return best;
-}
-
-// Number of CTA pairs of this kernel that can be resident at once (GPCs with
-// an odd number of SMs leave one SM out of pairing), capped at SMs / 2.
-template <Op op, int BN>
-int resident_pairs() {
-  static int cached[64] = {};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && cached[dev]) return cached[dev];
-  using L = Layout<op, BN>;
-  int n = device_sm_count() / 2;
-  if (cudaFuncSetAttribute(gemm_pair_kernel<op, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kDynBytes) ==
-      cudaSuccess) {
-    cudaLaunchConfig_t cfg{};
-    cfg.gridDim = dim3(2 * n);
-    cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = L::kDynBytes;
-    int clusters = 0;
-    if (cudaOccupancyMaxActiveClusters(&clusters, gemm_pair_kernel<op, BN>, &cfg) == cudaSuccess && clusters > 0 &&
-        clusters < n)
-      n = clusters;
-  }
-  cudaGetLastError();
-  if (dev >= 0 && dev < 64) cached[dev] = n;
-  return n;
-}
-
-// All candidate configurations of one op share the same pair budget; the
-// largest tile is the most constrained, so its residency is used for all.
-template <Op op>
-int pair_count() {
-  return resident_pairs<op, 256>();
 }
 
 }  // namespace
@@ -816,95 +994,88 @@ cudaError_t launch_forward(const int8_t* xq, const float* sx, const uint8_t* w_p
                            cudaStream_t s) {
   if (M == 0 || N == 0) return cudaSuccess;
   static const int kCands[3] = {256, 192, 128};
-  const int npairs = pair_count<Op::Fwd>();
+  const int npairs = resident_pairs<Family::Fwd, 256>();
   const int bn = choose_bn(static_cast<int>(N), static_cast<int>(M), npairs, kCands, 3);
-  CUtensorMap mb{}, msrc{}, unused{};
-  if (!make_map_2d(&mb, xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, K, M, K, 128, bn / 2, CU_TENSOR_MAP_SWIZZLE_128B, "xq"))
+  CUtensorMap maps[5] = {};
+  if (!make_map_2d(&maps[0], xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, K, M, K, 128, bn / 2, CU_TENSOR_MAP_SWIZZLE_128B,
+                   "xq"))
     return cudaErrorInvalidValue;
-  // packed codes [N][K/4] bytes: a TMA tensor needs 16-byte row pitch (K % 64 == 0)
+  // packed codes [N][K/4] bytes: a TMA tensor needs a 16-byte row pitch (K % 64 == 0)
   const bool src_tma = (K % 64) == 0;
-  if (src_tma && !make_map_2d(&msrc, w_packed, CU_TENSOR_MAP_DATA_TYPE_UINT8, K / 4, N, K / 4, 32, BM,
+  if (src_tma && !make_map_2d(&maps[1], w_packed, CU_TENSOR_MAP_DATA_TYPE_UINT8, K / 4, N, K / 4, 32, BM,
                               CU_TENSOR_MAP_SWIZZLE_NONE, "w_packed (fwd)"))
     return cudaErrorInvalidValue;
-  GemmParams p{};
-  p.src_tma = src_tma;
-  p.rows_a = static_cast<int>(N);
-  p.rows_b = static_cast<int>(M);
-  p.red = static_cast<int>(K);
+  static thread_local GemmParams p;
+  std::memset(&p, 0, offsetof(GemmParams, sched_start));
+  fill_op(p.op[0], static_cast<int>(N), static_cast<int>(M), static_cast<int>(K), 128, bn);
+  p.op[0].out = y;
+  p.op[0].ldo = N;
+  p.op[0].src_tma = src_tma;
   p.K = K;
   p.packed = w_packed;
   p.sx = sx;
   p.gamma = gamma;
-  p.out = y;
-  p.ldo = N;
   p.debug_acc = debug_acc;
   p.err = err;
-  if (bn == 256) return launch_pair<Op::Fwd, 256>(mb, msrc, unused, p, npairs, s);
-  if (bn == 192) return launch_pair<Op::Fwd, 192>(mb, msrc, unused, p, npairs, s);
-  return launch_pair<Op::Fwd, 128>(mb, msrc, unused, p, npairs, s);
+  if (bn == 256) return launch_pair<Family::Fwd, 256>(maps, p, npairs, s);
+  if (bn == 192) return launch_pair<Family::Fwd, 192>(maps, p, npairs, s);
+  return launch_pair<Family::Fwd, 128>(maps, p, npairs, s);
 }
 
-cudaError_t launch_backward_dx(const void* dY, const uint8_t* w_packed, const float* gamma, int64_t M, int64_t N,
-                               int64_t K, void* dX, int* err, cudaStream_t s) {
-  if (M == 0) return cudaSuccess;
-  static const int kCands[3] = {256, 192, 128};
-  const int npairs = pair_count<Op::Dx>();
-  const int bn = choose_bn(static_cast<int>(K), static_cast<int>(M), npairs, kCands, 3);
-  CUtensorMap mb{}, msrc{}, unused{};
-  if (!make_map_2d(&mb, dY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, N, M, N * 2, 64, bn / 2, CU_TENSOR_MAP_SWIZZLE_128B,
-                   "dY (dX)"))
-    return cudaErrorInvalidValue;
-  const bool src_tma = (K % 64) == 0;
-  if (src_tma && !make_map_2d(&msrc, w_packed, CU_TENSOR_MAP_DATA_TYPE_UINT8, K / 4, N, K / 4, 32, 64,
-                              CU_TENSOR_MAP_SWIZZLE_NONE, "w_packed (dX)"))
-    return cudaErrorInvalidValue;
-  GemmParams p{};
-  p.src_tma = src_tma;
-  p.rows_a = static_cast<int>(K);
-  p.rows_b = static_cast<int>(M);
-  p.red = static_cast<int>(N);
-  p.K = K;
-  p.packed = w_packed;
-  p.gamma = gamma;
-  p.out = dX;
-  p.ldo = K;
-  p.err = err;
-  if (bn == 256) return launch_pair<Op::Dx, 256>(mb, msrc, unused, p, npairs, s);
-  if (bn == 192) return launch_pair<Op::Dx, 192>(mb, msrc, unused, p, npairs, s);
-  return launch_pair<Op::Dx, 128>(mb, msrc, unused, p, npairs, s);
-}
-
-cudaError_t launch_backward_dw(const void* dY, const int8_t* xq, const float* sx, int64_t M, int64_t N, int64_t K,
-                               void* dW, int dw_is_f32, int accumulate, int* err, cudaStream_t s) {
-  if (M == 0) {
+// dX and/or dW in one launch (either output may be null).
+cudaError_t launch_backward(const void* dY, const int8_t* xq, const float* sx, const uint8_t* w_packed,
+                            const float* gamma, int64_t M, int64_t N, int64_t K, void* dX, void* dW, int dw_is_f32,
+                            int accumulate, int* err, cudaStream_t s) {
+  if (dW && M == 0) {
     const int64_t n = N * K;
     zero_dw_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, s>>>(dW, n, dw_is_f32, accumulate);
-    return cudaGetLastError();
+    if (cudaError_t e = cudaGetLastError(); e != cudaSuccess) return e;
   }
-  static const int kCands[2] = {256, 128};
-  const int npairs = pair_count<Op::Dw>();
-  const int bn = choose_bn(static_cast<int>(K), static_cast<int>(N), npairs, kCands, 2);
-  // s_x as a one-row 2D tensor: [1][M] floats, row pitch rounded up to 16 bytes
-  const uint64_t sx_pitch = ((static_cast<uint64_t>(M) * 4 + 15) / 16) * 16;
-  CUtensorMap mb{}, msrc{}, msx{};
-  if (!make_map_2d(&mb, dY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, N, M, N * 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B,
-                   "dY (dW)") ||
-      !make_map_2d(&msrc, xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, K, M, K, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B, "xq (dW)") ||
-      !make_map_2d(&msx, sx, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, M, 1, sx_pitch, 64, 1, CU_TENSOR_MAP_SWIZZLE_NONE,
-                   "sx (dW)"))
-    return cudaErrorInvalidValue;
-  GemmParams p{};
-  p.rows_a = static_cast<int>(K);
-  p.rows_b = static_cast<int>(N);
-  p.red = static_cast<int>(M);
+  if (M == 0) return cudaSuccess;
+  constexpr int BN = 256;
+  const int npairs = resident_pairs<Family::Bwd, BN>();
+  CUtensorMap maps[5] = {};
+  const bool src_tma = (K % 64) == 0;
+  if (dX) {
+    if (!make_map_2d(&maps[0], dY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, N, M, N * 2, 64, BN / 2,
+                     CU_TENSOR_MAP_SWIZZLE_128B, "dY (dX)"))
+      return cudaErrorInvalidValue;
+    if (src_tma && !make_map_2d(&maps[1], w_packed, CU_TENSOR_MAP_DATA_TYPE_UINT8, K / 4, N, K / 4, 32, 64,
+                                CU_TENSOR_MAP_SWIZZLE_NONE, "w_packed (dX)"))
+      return cudaErrorInvalidValue;
+  }
+  if (dW) {
+    // s_x as a one-row 2D tensor: [1][M] floats, row pitch rounded up to 16 bytes
+    const uint64_t sx_pitch = ((static_cast<uint64_t>(M) * 4 + 15) / 16) * 16;
+    if (!make_map_2d(&maps[2], dY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, N, M, N * 2, 64, 64,
+                     CU_TENSOR_MAP_SWIZZLE_128B, "dY (dW)") ||
+        !make_map_2d(&maps[3], xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, K, M, K, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B,
+                     "xq (dW)") ||
+        !make_map_2d(&maps[4], sx, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, M, 1, sx_pitch, 64, 1, CU_TENSOR_MAP_SWIZZLE_NONE,
+                     "sx (dW)"))
+      return cudaErrorInvalidValue;
+  }
+  static thread_local GemmParams p;
+  std::memset(&p, 0, offsetof(GemmParams, sched_start));
+  if (dX) {
+    fill_op(p.op[0], static_cast<int>(K), static_cast<int>(M), static_cast<int>(N), 64, BN);
+    p.op[0].out = dX;
+    p.op[0].ldo = K;
+    p.op[0].src_tma = src_tma;
+  }
+  if (dW) {
+    fill_op(p.op[1], static_cast<int>(K), static_cast<int>(N), static_cast<int>(M), 64, BN);
+    p.op[1].out = dW;
+    p.op[1].ldo = K;
+    p.op[1].out_f32 = dw_is_f32;
+    p.op[1].accumulate = accumulate;
+  }
   p.K = K;
-  p.out = dW;
-  p.ldo = K;
-  p.out_f32 = dw_is_f32;
-  p.accumulate = accumulate;
+  p.packed = w_packed;
+  p.sx = sx;
+  p.gamma = dX ? gamma : nullptr;
   p.err = err;
-  if (bn == 256) return launch_pair<Op::Dw, 256>(mb, msrc, msx, p, npairs, s);
-  return launch_pair<Op::Dw, 128>(mb, msrc, msx, p, npairs, s);
+  return launch_pair<Family::Bwd, BN>(maps, p, npairs, s);
 }
 
 }  // namespace bl

@@ -302,3 +302,28 @@ def test_weight_subnormals_and_zeros(w_dtype):
     w = w.to(w_dtype)
     assert (w.float().abs() < 1.17e-38).any() and (w.float() != 0).any()
     check_all(run_step(x, w, dy), oracle_step(x, w, dy), N)
+
+
+def test_dx_only_launch():
+    """bl_backward with dW = NULL: a launch holding only dX tiles."""
+    bl = _bl()
+    M, N, K = 300, 264, 352
+    x, w, dy = make_inputs(M, K, N, seed=29)
+    bufs = bl.StepBuffers.allocate(M, N, K)
+    bl.bl_quantize_weight(w.cuda(), bufs.w_packed, bufs.gamma, bufs.workspace)
+    bl.bl_quantize_act(x.cuda(), bufs.xq, bufs.sx)
+    bl.bl_backward(dy.cuda(), bufs.xq, bufs.sx, bufs.w_packed, bufs.gamma, bufs.dX, None)
+    torch.cuda.synchronize()
+    o = oracle_step(x, w, dy)
+    assert_close(ref.bf16_bits_to_f32(bits(bufs.dX)), ref.bf16_bits_to_f32(o["dx_bits"]), "dX")
+
+
+def test_backward_scheduled_tiles_full_compare():
+    """Enough dX + dW tiles (64 + 64) that the launch spreads them over the
+    pairs by its precomputed schedule; every output element compared."""
+    M = N = K = 2048
+    x, w, dy = make_inputs(M, K, N, seed=31)
+    g = run_step(x, w, dy, debug_acc=False)
+    o = oracle_step(x, w, dy)
+    g["acc"] = None
+    check_all(g, o, N)
