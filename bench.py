@@ -12,7 +12,9 @@ roofline fraction of the dominant kernel).
 Timing: W >= 3 untimed warm-up steps, then exactly K timed steps on
 resident inputs. L2 is flushed (256 MiB write) before every step, outside
 the timed events; each step is bracketed by CUDA events on the launching
-stream, with events between the C-ABI calls for per-kernel times. For N > 1
+stream (the headline); a second pass of K steps puts events between the C-ABI
+calls for the per-kernel times (events between kernels can cost the overlap
+of programmatically dependent launches, so that pass is not the headline). For N > 1
 (torchrun, one rank per GPU) every rank runs its own batch (weak scaling, no
 data-path collective); the job time is the max over ranks.
 
@@ -216,36 +218,47 @@ def run_ours(args, rank, world, local_rank):
     if bl.bl_get_last_error() != 0:
         raise RuntimeError("device error during warm-up")
 
-    def timed():
-        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(STAGES) + 1)] for _ in range(args.steps)]
+    def timed(per_stage):
+        """K steps, L2 flushed before each. per_stage: events between the C-ABI
+        calls (kernel breakdown); otherwise events only around each step, so
+        consecutive kernels keep their programmatic-launch overlap."""
+        n_ev = len(STAGES) + 1 if per_stage else 2
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
         if world > 1:
             torch.distributed.barrier()
         torch.cuda.synchronize(dev)
         for i in range(args.steps):
             flush.fill_(i & 0xFF)
-            step(evs[i])
+            if per_stage:
+                step(evs[i])
+            else:
+                evs[i][0].record(stream)
+                step()
+                evs[i][1].record(stream)
         torch.cuda.synchronize(dev)
         if world > 1:
             torch.distributed.barrier()
-        per_stage = {s: 0.0 for s in STAGES}
+        per = {s: 0.0 for s in STAGES}
         total = 0.0
         for e in evs:
-            for j, s in enumerate(STAGES):
-                per_stage[s] += e[j].elapsed_time(e[j + 1])
-            total += e[0].elapsed_time(e[len(STAGES)])
-        return total, per_stage
+            if per_stage:
+                for j, st in enumerate(STAGES):
+                    per[st] += e[j].elapsed_time(e[j + 1])
+            total += e[0].elapsed_time(e[-1])
+        return total, per
 
     sampler = ClockSampler(dev.index if dev.index is not None else 0)
     sampler.start()
-    total_ms, per_stage = timed()
+    total_ms, _ = timed(False)
     clocks = sampler.stop()
     remeasured = False
     if sampler.rejected(clocks):
         sampler = ClockSampler(dev.index if dev.index is not None else 0)
         sampler.start()
-        total_ms, per_stage = timed()
+        total_ms, _ = timed(False)
         clocks = sampler.stop()
         remeasured = True
+    breakdown_ms, per_stage = timed(True)
     clocks["remeasured"] = remeasured
     if bl.bl_get_last_error() != 0:
         raise RuntimeError("device error during the timed region")
@@ -300,6 +313,7 @@ def run_ours(args, rank, world, local_rank):
                    "parallelism": f"dp{world} independent replicas" if world > 1 else "single GPU"},
         "roofline": roofline,
         "step_roofline_frac": round(roof_ms / ms_per_step, 4),
+        "kernel_breakdown_ms_per_step": round(breakdown_ms / args.steps, 5),
         "kernels": kernels,
         "e2e": e2e,
         "gpu_launches": LAUNCHES_PER_STEP * args.steps,

@@ -185,6 +185,17 @@ __device__ __forceinline__ void cp_async_mbar_arrive(uint64_t* bar) {
   asm volatile("cp.async.mbarrier.arrive.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
+// ---------------------------------------------------------------- programmatic dependent launch
+// Kernels of this library are launched as programmatic dependents of the
+// previous kernel in the stream. Each one waits for that kernel to finish
+// (and its writes to be visible) before reading any input, and only then lets
+// its own dependents launch, so every kernel still starts its reads after all
+// earlier work in the stream has completed.
+__device__ __forceinline__ void pdl_wait_primary() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- tcgen05
 
 __device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {

@@ -8,6 +8,24 @@
 
 namespace bl {
 
+// Launches `kernel` as a programmatic dependent of the previous kernel in
+// `stream` (the kernel itself waits for it before reading its inputs).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 // ---- S1: absmean ternarisation + 2-bit packing
 // Number of fp64 partial sums pass A writes for a tensor of `numel` elements
 // (a fixed function of numel, so the reduction order never depends on the GPU).

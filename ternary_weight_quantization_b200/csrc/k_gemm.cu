@@ -616,6 +616,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   cluster_sync_all();  // barriers initialised and TMEM allocated in both CTAs
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
+  // inputs come from earlier kernels in the stream: the set-up above overlaps
+  // their tail, the first read waits for them
+  pdl_wait_primary();
+  pdl_launch_dependents();
 
   // A failed wait also stops the peer CTA's waits.
   auto wait = [&](uint64_t* bar, uint32_t parity) -> bool {
@@ -945,7 +949,9 @@ cudaError_t launch_pair(const CUtensorMap* maps, GemmParams& p, int npairs, cuda
     std::fprintf(stderr, "[bitlinear] gemm family=%d BN=%d stages=%d smem=%d tiles=%d+%d kb=%d/%d pairs=%d sched=%d\n",
                  static_cast<int>(F), BN, L::kS, L::kDynBytes, p.op[0].ntiles, p.op[1].ntiles, p.op[0].num_kb,
                  p.op[1].num_kb, pairs, p.use_sched);
-  gemm_pair_kernel<F, BN><<<2 * pairs, kThreads, L::kDynBytes, s>>>(maps[0], maps[1], maps[2], maps[3], maps[4], p);
+  cudaError_t e = launch_pdl(gemm_pair_kernel<F, BN>, dim3(2 * pairs), dim3(kThreads), L::kDynBytes, s, maps[0],
+                             maps[1], maps[2], maps[3], maps[4], p);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

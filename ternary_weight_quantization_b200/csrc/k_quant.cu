@@ -84,8 +84,6 @@ __device__ __forceinline__ double add_group(double acc, const Group<kF32>& a) {
   return acc;
 }
 
-__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
-__device__ __forceinline__ void pdl_wait_primary() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
 // ---------------------------------------------------------------- S1 pass A
 // partials[b] = sum of |w| over block b's contiguous range of groups, fp64.
@@ -96,6 +94,7 @@ template <bool kF32>
 __global__ void __launch_bounds__(kQuantThreads) absmean_partials_kernel(const uint4* __restrict__ W,
                                                                          int64_t ngroups, int64_t per_block,
                                                                          double* __restrict__ partials) {
+  pdl_wait_primary();       // W may come from the previous kernel (e.g. an optimizer step)
   pdl_launch_dependents();  // the code pass may start loading W while this pass finishes
   constexpr int T = kQuantThreads;
   const int64_t g0 = static_cast<int64_t>(blockIdx.x) * per_block;
@@ -130,7 +129,8 @@ __global__ void __launch_bounds__(kQuantThreads) absmean_partials_kernel(const u
 
 // ---------------------------------------------------------------- S1 pass B
 // Launched as a programmatic dependent of pass A: each thread first loads its
-// first groups of W (inputs pass A does not write), then waits for pass A,
+// first groups of W (pass A only started after W's producer finished, and it
+// does not write W), then waits for pass A,
 // then every block reduces the partials in the same fixed order (so all
 // blocks hold the same gamma) and writes the codes of its range of groups.
 //
@@ -169,6 +169,7 @@ __global__ void __launch_bounds__(kQuantThreads) ternarize_pack_kernel(const uin
     if (gf + u * T < g1) first[u].load(W, gf + u * T);
 
   pdl_wait_primary();  // pass A has finished and its partial sums are visible
+  pdl_launch_dependents();
 
   __shared__ double red[kQuantThreads / 32];
   __shared__ float s_thr;
@@ -286,6 +287,8 @@ template <int VPL, bool kPrefetch>
 __global__ void __launch_bounds__(32 * kActRowsPerBlock) act_quant_kernel(const uint4* __restrict__ x, int64_t M,
                                                                           int nv, int8_t* __restrict__ xq,
                                                                           float* __restrict__ sx) {
+  pdl_wait_primary();
+  pdl_launch_dependents();
   const int lane = threadIdx.x & 31;
   const int64_t nwarps = static_cast<int64_t>(gridDim.x) * kActRowsPerBlock;
   int64_t m = static_cast<int64_t>(blockIdx.x) * kActRowsPerBlock + (threadIdx.x >> 5);
@@ -315,6 +318,8 @@ __global__ void __launch_bounds__(32 * kActRowsPerBlock) act_quant_long_kernel(c
                                                                                int64_t M, int nv,
                                                                                int8_t* __restrict__ xq,
                                                                                float* __restrict__ sx) {
+  pdl_wait_primary();
+  pdl_launch_dependents();
   const int lane = threadIdx.x & 31;
   const int64_t m = static_cast<int64_t>(blockIdx.x) * kActRowsPerBlock + (threadIdx.x >> 5);
   if (m >= M) return;
@@ -344,18 +349,11 @@ int weight_partials_count(int64_t numel) {
 template <bool kF32>
 static cudaError_t launch_weight_passes(const uint4* w, int64_t ngroups, int64_t per_block, int nparts, int64_t numel,
                                         uint32_t* out, float* gamma, double* partials, cudaStream_t s) {
-  absmean_partials_kernel<kF32><<<nparts, kQuantThreads, 0, s>>>(w, ngroups, per_block, partials);
-  cudaLaunchConfig_t cfg{};
-  cfg.gridDim = dim3(nparts);
-  cfg.blockDim = dim3(kQuantThreads);
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, ternarize_pack_kernel<kF32>, w, ngroups, per_block,
-                            static_cast<const double*>(partials), nparts, numel, out, gamma);
+  cudaError_t e = launch_pdl(absmean_partials_kernel<kF32>, dim3(nparts), dim3(kQuantThreads), 0, s, w, ngroups,
+                             per_block, partials);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(ternarize_pack_kernel<kF32>, dim3(nparts), dim3(kQuantThreads), 0, s, w, ngroups, per_block,
+                    static_cast<const double*>(partials), nparts, numel, out, gamma);
 }
 
 cudaError_t launch_quantize_weight(const void* W, int w_is_f32, int64_t N, int64_t K, uint8_t* packed,
@@ -422,7 +420,7 @@ static void launch_act(const uint4* xv, int64_t M, int nv, int8_t* xq, float* sx
   const int64_t want = (M + kActRowsPerBlock - 1) / kActRowsPerBlock;
   const int64_t cap = static_cast<int64_t>(occ) * device_sm_count();
   const unsigned grid = static_cast<unsigned>(want < cap ? want : cap);
-  act_quant_kernel<VPL, kPrefetch><<<grid, 32 * kActRowsPerBlock, 0, s>>>(xv, M, nv, xq, sx);
+  launch_pdl(act_quant_kernel<VPL, kPrefetch>, dim3(grid), dim3(32 * kActRowsPerBlock), 0, s, xv, M, nv, xq, sx);
 }
 
 cudaError_t launch_quantize_act(const void* x, int64_t M, int64_t K, int8_t* xq, float* sx, cudaStream_t s) {
@@ -444,7 +442,7 @@ cudaError_t launch_quantize_act(const void* x, int64_t M, int64_t K, int8_t* xq,
 #undef BL_ACT_CASE
     default: {
       const unsigned grid = static_cast<unsigned>((M + kActRowsPerBlock - 1) / kActRowsPerBlock);
-      act_quant_long_kernel<<<grid, 32 * kActRowsPerBlock, 0, s>>>(xv, M, nv, xq, sx);
+      launch_pdl(act_quant_long_kernel, dim3(grid), dim3(32 * kActRowsPerBlock), 0, s, xv, M, nv, xq, sx);
     }
   }
   return cudaGetLastError();
