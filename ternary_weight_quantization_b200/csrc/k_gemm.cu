@@ -32,7 +32,8 @@
 //               not 16-byte aligned, which a tensor map requires)
 //   warp 1      TMEM allocation (2 x 256 columns, pair-wide); in the leader
 //               CTA one lane issues the tcgen05.mma
-//   warps 2-4, 6-8, 10-11  rebuild A from the staged source
+//   warps 2-4, 6-8, 10-11  rebuild A from the staged source, in two groups
+//               of four taking alternate stages
 //   warps 5, 9  idle (keeps sub-partition 1 to the MMA warp: rebuild warps
 //               there would compete with it for issue slots)
 //   warps 12-15 epilogue: TMEM -> registers -> smem (transpose) -> global
@@ -70,7 +71,11 @@ constexpr int kThreads = 512;
 constexpr int kWarpLoad = 0;
 constexpr int kWarpMma = 1;
 constexpr int kNumRebuildWarps = 8;  // warps 2, 3, 4, 6, 7, 8, 10, 11
-constexpr int kRebuildThreads = 32 * kNumRebuildWarps;
+// The rebuild warps form two groups of four that take alternate pipeline
+// stages, so one group's fixed per-stage latency (shared loads, proxy fence,
+// barrier arrival) overlaps the other's work.
+constexpr int kRebuildGroups = 2;
+constexpr int kRebuildThreads = 32 * kNumRebuildWarps / kRebuildGroups;  // threads per stage
 constexpr int kWarpEpi0 = 12;        // warps 12..15 (TMEM lane quadrants 0..3)
 constexpr int kNumEpiWarps = 4;
 
@@ -264,18 +269,40 @@ __device__ __forceinline__ uint4 codes8_to_bf16(uint32_t h) {
 
 // 16 int8 (x_hat source) * s -> 16 bf16, each bf16_rn(fp32(q) * s).
 // fp32(q) uses the 2^23 shifter: bits 0x4B0000uu are 2^23 + u with
-// u = q + 128, so subtracting 2^23 + 128 is exact.
+// u = q + 128, so subtracting 2^23 + 128 is exact. The subtraction and the
+// product by s run on pairs (packed fp32x2, each lane rounded like the scalar
+// instruction).
+__device__ __forceinline__ uint64_t f32x2_sub(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
+__device__ __forceinline__ uint64_t f32x2_mul(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
+__device__ __forceinline__ uint32_t f32x2_to_bf16x2(uint64_t v) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "r"(static_cast<uint32_t>(v >> 32)), "r"(static_cast<uint32_t>(v)));
+  return r;
+}
+
 __device__ __forceinline__ void s8x16_to_bf16(const uint4& v, float s, uint4& o0, uint4& o1) {
   const uint32_t w[4] = {v.x ^ 0x80808080u, v.y ^ 0x80808080u, v.z ^ 0x80808080u, v.w ^ 0x80808080u};
+  constexpr uint64_t kShift2 = 0x4B0000804B000080ull;  // {2^23 + 128, 2^23 + 128}
+  const uint64_t s2 = (static_cast<uint64_t>(__float_as_uint(s)) << 32) | __float_as_uint(s);
   uint32_t out[8];
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
 #pragma unroll
     for (int b = 0; b < 4; b += 2) {
-      const float f0 = __fsub_rn(__uint_as_float(__byte_perm(w[i], 0x4B000000u, 0x7440u | b)), 8388736.0f);
-      const float f1 = __fsub_rn(__uint_as_float(__byte_perm(w[i], 0x4B000000u, 0x7440u | (b + 1))), 8388736.0f);
-      const __nv_bfloat162 p = __floats2bfloat162_rn(__fmul_rn(f0, s), __fmul_rn(f1, s));
-      out[i * 2 + b / 2] = *reinterpret_cast<const uint32_t*>(&p);
+      const uint32_t lo = __byte_perm(w[i], 0x4B000000u, 0x7440u | b);
+      const uint32_t hi = __byte_perm(w[i], 0x4B000000u, 0x7440u | (b + 1));
+      const uint64_t q2 = f32x2_sub((static_cast<uint64_t>(hi) << 32) | lo, kShift2);
+      out[i * 2 + b / 2] = f32x2_to_bf16x2(f32x2_mul(q2, s2));
     }
   }
   o0 = make_uint4(out[0], out[1], out[2], out[3]);
@@ -369,48 +396,45 @@ __device__ __forceinline__ void load_stage(const GemmParams& p, const OpParams& 
   }
 }
 
-// Rebuild warps, one stage: A rows of this CTA from the staged source.
+// Rebuild group (128 threads), one stage: A rows of this CTA from the staged source.
 template <Op op, Family F, int BN>
 __device__ __forceinline__ void rebuild_stage(int rt, uint32_t sA, uint32_t sSrc, const float* sSx) {
   if constexpr (op == Op::Fwd) {
-    // row = rt % 128: its 32 packed bytes -> 128 int8 codes, K-major with
-    // 128-byte swizzle; this thread does half rt / 128 (four 16-code chunks)
-    const int row = rt & 127, half = rt >> 7;
-    const uint4 w = ld_shared_v4(sSrc + row * 32 + half * 16);
-    const uint32_t words[4] = {w.x, w.y, w.z, w.w};
-    const uint32_t row_base = sA + row * 128;
+    // row rt: 32 packed bytes -> 128 int8 codes, K-major with 128-byte swizzle.
+    // Lanes 4..7 of each group of 8 read their second half first (bank spread).
+    const uint32_t h = (rt >> 2) & 1;
+    const uint4 wa = ld_shared_v4(sSrc + rt * 32 + h * 16);
+    const uint4 wb = ld_shared_v4(sSrc + rt * 32 + (h ^ 1) * 16);
+    const uint4 w0 = h ? wb : wa, w1 = h ? wa : wb;
+    const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+    const uint32_t row_base = sA + rt * 128;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int c = half * 4 + i;
-      st_shared_v4(row_base + ((c ^ (row & 7)) << 4), codes16_to_s8(words[i]));
-    }
+    for (int c = 0; c < 8; ++c) st_shared_v4(row_base + ((c ^ (rt & 7)) << 4), codes16_to_s8(words[c]));
   } else if constexpr (op == Op::Dx) {
-    // reduction row n = rt % 64; output k range [32 q, 32 q + 32), q = rt / 64
-    const int n = rt & 63, qr = rt >> 6;
-    uint32_t w0, w1;
-    asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];" : "=r"(w0), "=r"(w1) : "r"(sSrc + n * 32 + qr * 8));
-    const uint32_t base = sA + (qr >> 1) * 8192 + n * 128;
+    // reduction row n = rt % 64, output k half = rt / 64 (64 k values)
+    const int n = rt & 63, half = rt >> 6;
+    const uint4 w = ld_shared_v4(sSrc + n * 32 + half * 16);
+    const uint32_t words[4] = {w.x, w.y, w.z, w.w};
+    const uint32_t base = sA + half * 8192 + n * 128;
 #pragma unroll
-    for (int jj = 0; jj < 4; ++jj) {
-      const uint32_t hw = (jj < 2 ? w0 : w1) >> ((jj & 1) * 16);
-      const int col = (qr & 1) * 4 + jj;
-      st_shared_v4(base + ((col ^ (n & 7)) << 4), codes8_to_bf16(hw));
+    for (int j = 0; j < 8; ++j) {
+      const uint32_t hw = words[j >> 1] >> ((j & 1) * 16);
+      st_shared_v4(base + ((j ^ (n & 7)) << 4), codes8_to_bf16(hw));
     }
   } else {
-    // token m = rt % 64; k range [32 q, 32 q + 32), q = rt / 64; q staging is
-    // 128-byte swizzled
-    const int m = rt & 63, qr = rt >> 6;
+    // token m = rt % 64, k half = rt / 64; q staging is 128-byte swizzled
+    const int m = rt & 63, half = rt >> 6;
     const float s = sSx[m];
-    const uint32_t base = sA + (qr >> 1) * 8192 + m * 128;
+    const uint32_t base = sA + half * 8192 + m * 128;
 #pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      const int c = qr * 2 + i;  // logical 16-byte chunk (16 k values)
+    for (int i = 0; i < 4; ++i) {
+      const int c = half * 4 + i;  // logical 16-byte chunk (16 k values)
       const uint4 v = ld_shared_v4(sSrc + m * 128 + ((c ^ (m & 7)) << 4));
       uint4 o0, o1;
       s8x16_to_bf16(v, s, o0, o1);
-      const int col0 = (qr & 1) * 4 + 2 * i;  // 8-k units within this 64-k chunk
-      st_shared_v4(base + ((col0 ^ (m & 7)) << 4), o0);
-      st_shared_v4(base + (((col0 + 1) ^ (m & 7)) << 4), o1);
+      const int j0 = 2 * i, j1 = 2 * i + 1;  // 8-k units within this half
+      st_shared_v4(base + ((j0 ^ (m & 7)) << 4), o0);
+      st_shared_v4(base + ((j1 ^ (m & 7)) << 4), o1);
     }
   }
 }
@@ -596,7 +620,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(&src_full[s], 1);
-      mbar_init(&full[s], 1 + 2 * kNumRebuildWarps);  // leader's expect_tx + both CTAs' rebuild warps
+      mbar_init(&full[s], 1 + 2 * (kNumRebuildWarps / kRebuildGroups));  // expect_tx + both CTAs' rebuilding warps
       mbar_init(&empty[s], 1);
       issued_parity[s] = -1;
     }
@@ -731,30 +755,35 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else if (rebuild_slot(warp) >= 0) {
     // ------------------------------------------------------------ rebuild A (both CTAs)
-    static_assert(kRebuildThreads == 256, "rebuild mappings assume 256 threads");
-    const int rt = rebuild_slot(warp) * 32 + lane;
+    static_assert(kRebuildThreads == 128, "rebuild mappings assume 128 threads per stage");
+    const int slot = rebuild_slot(warp);
+    const int group = slot >> 2;                    // 0 or 1: even or odd stage sequence numbers
+    const int rt = (slot & 3) * 32 + lane;          // 0..127 within the group
     int stage = 0;
     uint32_t phase = 0;
+    int seq = 0;                                    // stage sequence number across tiles
     bool ok = true;
     int tile;
     for (int i = 0; ok && next_tile(p, pair, npairs, i, tile); ++i) {
       const int opi = tile >= p.op[0].ntiles ? 1 : 0;
       const int num_kb = p.op[opi].num_kb;
-      for (int kb = 0; kb < num_kb; ++kb) {
-        if (!wait(&src_full[stage], phase)) {
-          ok = false;
-          break;
+      for (int kb = 0; kb < num_kb; ++kb, ++seq) {
+        if ((seq & 1) == group) {
+          if (!wait(&src_full[stage], phase)) {
+            ok = false;
+            break;
+          }
+          const uint32_t sA = smem_u32(smem + L::kOffA + stage * G::kABytes);
+          const uint32_t sSrc = smem_u32(smem + L::kOffSrc + stage * G::kSrcBytes);
+          const float* sSx = reinterpret_cast<const float*>(smem + L::kOffSx + stage * G::kSxBytes);
+          if (opi == 0)
+            rebuild_stage<kOp0, F, BN>(rt, sA, sSrc, sSx);
+          else if constexpr (F == Family::Bwd)
+            rebuild_stage<Op::Dw, F, BN>(rt, sA, sSrc, sSx);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive_cluster(lead(&full[stage]));
         }
-        const uint32_t sA = smem_u32(smem + L::kOffA + stage * G::kABytes);
-        const uint32_t sSrc = smem_u32(smem + L::kOffSrc + stage * G::kSrcBytes);
-        const float* sSx = reinterpret_cast<const float*>(smem + L::kOffSx + stage * G::kSxBytes);
-        if (opi == 0)
-          rebuild_stage<kOp0, F, BN>(rt, sA, sSrc, sSx);
-        else if constexpr (F == Family::Bwd)
-          rebuild_stage<Op::Dw, F, BN>(rt, sA, sSrc, sSx);
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(lead(&full[stage]));
         if (++stage == S) {
           stage = 0;
           phase ^= 1;
