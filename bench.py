@@ -10,8 +10,8 @@ Metric: effective TOPS = 6 M N K / step time (plus ms per step and the
 roofline fraction of the dominant kernel).
 
 Timing: W >= 3 untimed warm-up steps, then exactly K timed steps on
-resident inputs. L2 is flushed (256 MiB write) before every step, outside
-the timed events; each step is bracketed by CUDA events on the launching
+resident inputs. L2 is flushed (256 MiB written, then read back, so that no
+dirty line is left) before every step, outside the timed events; each step is bracketed by CUDA events on the launching
 stream (the headline); a second pass of K steps puts events between the C-ABI
 calls for the per-kernel times (events between kernels can cost the overlap
 of programmatically dependent launches, so that pass is not the headline). For N > 1
@@ -195,6 +195,13 @@ def run_ours(args, rank, world, local_rank):
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
+    def flush_l2(i):
+        # Write a buffer twice the size of L2, then read it back: no workload
+        # data stays in L2 and no dirty line is left for the timed kernels to
+        # write back.
+        flush.fill_(i & 0xFF)
+        flush.view(torch.int64).max()
+
     def step(evs=None):
         if evs:
             evs[0].record(stream)
@@ -211,8 +218,8 @@ def run_ours(args, rank, world, local_rank):
         if evs:
             evs[4].record(stream)
 
-    for _ in range(args.warmup):
-        flush.fill_(1)
+    for i in range(args.warmup):
+        flush_l2(i)
         step()
     torch.cuda.synchronize(dev)
     if bl.bl_get_last_error() != 0:
@@ -228,7 +235,7 @@ def run_ours(args, rank, world, local_rank):
             torch.distributed.barrier()
         torch.cuda.synchronize(dev)
         for i in range(args.steps):
-            flush.fill_(i & 0xFF)
+            flush_l2(i)
             if per_stage:
                 step(evs[i])
             else:
@@ -309,7 +316,7 @@ def run_ours(args, rank, world, local_rank):
                    "x": f"bf16 [{M},{K}] N(0,1)" + (" + 1% x20 outliers" if wl.outliers else ""),
                    "W": f"{'bf16' if wl.w_dtype == torch.bfloat16 else 'f32'} [{N},{K}] {wl.w_init}",
                    "dY": f"bf16 [{M},{N}] N(0,1)", "global_batch_tokens": M * world,
-                   "l2": "flushed before every step (256 MiB write, outside the timed events)",
+                   "l2": "flushed before every step (256 MiB write then read, outside the timed events)",
                    "parallelism": f"dp{world} independent replicas" if world > 1 else "single GPU"},
         "roofline": roofline,
         "step_roofline_frac": round(roof_ms / ms_per_step, 4),
