@@ -7,7 +7,7 @@
 // One persistent, warp-specialised CTA-pair kernel template serves all three:
 //
 //   D[i][j] = sum_r A[i][r] * B[j][r]        (tcgen05.mma cta_group::2, TMEM accumulators)
-//   out[j][i] = epilogue(D[i][j])            (transposed store)
+//   out[j][i] = epilogue(D[i][j])            (i contiguous in the output)
 //
 //   op   A (REBUILT in smem)                    B (TMA)                       r
 //   Fwd  codes[n][k] int8, K-major              xq[m][k] int8, K-major        k
@@ -36,7 +36,7 @@
 //               of four taking alternate stages
 //   warps 5, 9  idle (keeps sub-partition 1 to the MMA warp: rebuild warps
 //               there would compete with it for issue slots)
-//   warps 12-15 epilogue: TMEM -> registers -> smem (transpose) -> global
+//   warps 12-15 epilogue: TMEM -> registers -> bf16/f32 box in smem -> TMA store
 // Barriers: src_full (per CTA: staged source landed), full (leader: both
 // CTAs' B bytes landed and both CTAs' A rebuilt -- one wait per stage for the
 // MMA lane), empty and tmem_full (both CTAs, completed by multicast
@@ -180,6 +180,7 @@ struct OpParams {
   int out_f32;    // Dw
   int accumulate; // Dw
   int src_tma;    // Fwd/Dx: packed codes by TMA (K % 64 == 0) instead of cp.async
+  int tma_store;  // output through the TMA store map of this op
 };
 
 struct GemmParams {
@@ -323,11 +324,6 @@ __device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
 
 // ---------------------------------------------------------------- per-op stage work
 
-// Staging word of element (row j, column i) of an epilogue warp's 32 x 32
-// transpose tile; flipping bit 2 of i on odd rows keeps both the row-wise
-// writes and the 16-byte reads of two adjacent rows free of bank conflicts.
-__device__ __forceinline__ uint32_t stg_word(int j, int i) { return j * 32 + (i ^ ((j & 1) << 2)); }
-
 struct Maps {
   const CUtensorMap* b;
   const CUtensorMap* src;
@@ -455,106 +451,99 @@ __device__ __forceinline__ void mma_stage(uint32_t d_tmem, uint32_t sa, uint32_t
   }
 }
 
-// Epilogue, one 32-column chunk already transposed into staging: each lane
-// stores 8 consecutive i of one output row j, 4 rows per pass.
+// Epilogue value of accumulator word `a`: the forward scales the exact INT32
+// sum by s_x[m] * gamma, dX by gamma; dW is the fp32 sum.
 template <Op op>
-__device__ __forceinline__ void store_chunk(const GemmParams& p, const OpParams& P, uint32_t stg, int lane, int q,
-                                            int a0, int jbase, float gamma, float col_scale) {
-  const int seg = (lane & 3) * 8;
-  const int i0 = a0 + q * 32 + seg;
+__device__ __forceinline__ float epi_value(uint32_t a, float scale) {
+  if constexpr (op == Op::Fwd) return __fmul_rn(static_cast<float>(static_cast<int32_t>(a)), scale);
+  else if constexpr (op == Op::Dx) return __fmul_rn(__uint_as_float(a), scale);
+  else return __uint_as_float(a);
+}
+
+__device__ __forceinline__ void st_shared_b16(uint32_t addr, uint16_t v) {
+  asm volatile("st.shared.b16 [%0], %1;" ::"r"(addr), "h"(v) : "memory");
+}
+
+__device__ __forceinline__ void st_shared_b32(uint32_t addr, uint32_t v) {
+  asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+
+// Epilogue, one 32 x 32 chunk in registers: lane = output column i (A row),
+// r[jj] = output row j0 + jj. Written as one TMA store box from a staging
+// slot in shared memory (bf16: two 2 KB slots per warp, used in turn; f32:
+// the warp's whole 4 KB), or stored directly when the output is accumulated
+// into, for the debug output, and for row pitches a tensor map cannot take.
+// `seq` counts the warp's stored chunks (slot choice and reuse waits).
+template <Op op>
+__device__ __forceinline__ void epilogue_chunk(const GemmParams& p, const OpParams& P, const CUtensorMap* out_map,
+                                               const uint32_t (&r)[32], uint32_t stg, int lane, int i0, int j0,
+                                               float col_scale, float gamma, uint32_t& seq) {
+  if (i0 >= P.rows_a || j0 >= P.rows_b) return;
+  if (P.tma_store) {
+    uint32_t slot;
+    if (P.out_f32) {
+      slot = stg;
+      if (lane == 0) bulk_wait_group_read<0>();  // the previous box has been read
+      __syncwarp();
 #pragma unroll
-  for (int pass = 0; pass < 4; ++pass) {
-    const int jl = pass * 8 + (lane >> 2);
-    const int j = jbase + jl;
-    float row_scale = 0.0f;
-    if constexpr (op == Op::Fwd) row_scale = __shfl_sync(0xffffffffu, col_scale, jl);
-    if (j >= P.rows_b || i0 >= P.rows_a) continue;
-    // the two 4-word halves of this 8-word run (swapped on odd rows)
-    const int sw = (jl & 1) << 2;
-    const uint4 v0 = ld_shared_v4(stg + stg_word(jl, seg + sw) * 4);
-    const uint4 v1 = ld_shared_v4(stg + stg_word(jl, seg + (4 ^ sw)) * 4);
-    const uint4 lo = sw ? v1 : v0, hi = sw ? v0 : v1;
-    const uint32_t acc[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
-    const int nvalid = min(8, P.rows_a - i0);
-    const int64_t off = static_cast<int64_t>(j) * P.ldo + i0;
-    if constexpr (op == Op::Fwd) {
-      __nv_bfloat16* y = static_cast<__nv_bfloat16*>(P.out) + off;
-      uint32_t pk[4];
-#pragma unroll
-      for (int e = 0; e < 8; e += 2) {
-        const __nv_bfloat162 b2 =
-            __floats2bfloat162_rn(__fmul_rn(static_cast<float>(static_cast<int32_t>(acc[e])), row_scale),
-                                  __fmul_rn(static_cast<float>(static_cast<int32_t>(acc[e + 1])), row_scale));
-        pk[e / 2] = *reinterpret_cast<const uint32_t*>(&b2);
-      }
-      if (nvalid == 8 && (P.ldo % 8) == 0) {
-        *reinterpret_cast<uint4*>(y) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-      } else {
-        for (int e = 0; e < nvalid; ++e)
-          reinterpret_cast<uint16_t*>(y)[e] = static_cast<uint16_t>(pk[e / 2] >> ((e & 1) * 16));
-      }
-      if (p.debug_acc) {
-        int32_t* d = p.debug_acc + off;
-        if (nvalid == 8 && (P.ldo % 4) == 0) {
-          reinterpret_cast<uint4*>(d)[0] = lo;
-          reinterpret_cast<uint4*>(d)[1] = hi;
-        } else {
-          for (int e = 0; e < nvalid; ++e) d[e] = static_cast<int32_t>(acc[e]);
-        }
-      }
-    } else if constexpr (op == Op::Dx) {
-      __nv_bfloat16* dx = static_cast<__nv_bfloat16*>(P.out) + off;
-      uint32_t pk[4];
-#pragma unroll
-      for (int e = 0; e < 8; e += 2) {
-        const __nv_bfloat162 b2 = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(acc[e]), gamma),
-                                                        __fmul_rn(__uint_as_float(acc[e + 1]), gamma));
-        pk[e / 2] = *reinterpret_cast<const uint32_t*>(&b2);
-      }
-      *reinterpret_cast<uint4*>(dx) = make_uint4(pk[0], pk[1], pk[2], pk[3]);  // K % 32 == 0
+      for (int jj = 0; jj < 32; ++jj)
+        st_shared_b32(slot + jj * 128 + lane * 4, __float_as_uint(epi_value<op>(r[jj], 0.0f)));
     } else {
-      float v[8];
+      slot = stg + (seq & 1u) * 2048u;
+      if (lane == 0) bulk_wait_group_read<1>();  // the box stored from this slot two chunks ago has been read
+      __syncwarp();
 #pragma unroll
-      for (int e = 0; e < 8; ++e) v[e] = __uint_as_float(acc[e]);
-      if (P.out_f32) {
-        float4* dw = reinterpret_cast<float4*>(static_cast<float*>(P.out) + off);
-        if (P.accumulate) {
-          const float4 o0 = dw[0], o1 = dw[1];
-          v[0] = __fadd_rn(v[0], o0.x); v[1] = __fadd_rn(v[1], o0.y);
-          v[2] = __fadd_rn(v[2], o0.z); v[3] = __fadd_rn(v[3], o0.w);
-          v[4] = __fadd_rn(v[4], o1.x); v[5] = __fadd_rn(v[5], o1.y);
-          v[6] = __fadd_rn(v[6], o1.z); v[7] = __fadd_rn(v[7], o1.w);
-        }
-        dw[0] = make_float4(v[0], v[1], v[2], v[3]);
-        dw[1] = make_float4(v[4], v[5], v[6], v[7]);
-      } else {
-        uint4* dw = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(P.out) + off);
-        if (P.accumulate) {
-          const uint4 o = *dw;
-          const uint32_t ow[4] = {o.x, o.y, o.z, o.w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            v[2 * e] = __fadd_rn(v[2 * e], __uint_as_float(ow[e] << 16));
-            v[2 * e + 1] = __fadd_rn(v[2 * e + 1], __uint_as_float(ow[e] & 0xFFFF0000u));
-          }
-        }
-        uint32_t pk[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const __nv_bfloat162 b2 = __floats2bfloat162_rn(v[2 * e], v[2 * e + 1]);
-          pk[e] = *reinterpret_cast<const uint32_t*>(&b2);
-        }
-        *dw = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      for (int jj = 0; jj < 32; ++jj) {
+        float scale = 0.0f;
+        if constexpr (op == Op::Fwd) scale = __shfl_sync(0xffffffffu, col_scale, jj);
+        else if constexpr (op == Op::Dx) scale = gamma;
+        const __nv_bfloat16 b = __float2bfloat16_rn(epi_value<op>(r[jj], scale));
+        st_shared_b16(slot + jj * 64 + lane * 2, *reinterpret_cast<const uint16_t*>(&b));
       }
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      tma_store_2d(out_map, slot, i0, j0);
+      bulk_commit_group();
+    }
+    ++seq;
+    return;
+  }
+  // direct stores: lane i writes column i of each row j (the warp's 32 lanes
+  // write contiguous elements of one row)
+  const int i = i0 + lane;
+#pragma unroll
+  for (int jj = 0; jj < 32; ++jj) {
+    float scale = 0.0f;
+    if constexpr (op == Op::Fwd) scale = __shfl_sync(0xffffffffu, col_scale, jj);
+    else if constexpr (op == Op::Dx) scale = gamma;
+    const int j = j0 + jj;
+    if (i >= P.rows_a || j >= P.rows_b) continue;
+    const int64_t off = static_cast<int64_t>(j) * P.ldo + i;
+    float v = epi_value<op>(r[jj], scale);
+    if constexpr (op == Op::Fwd) {
+      if (p.debug_acc) p.debug_acc[off] = static_cast<int32_t>(r[jj]);
+    }
+    if (P.out_f32) {
+      float* o = static_cast<float*>(P.out) + off;
+      if (P.accumulate) v = __fadd_rn(v, *o);
+      *o = v;
+    } else {
+      __nv_bfloat16* o = static_cast<__nv_bfloat16*>(P.out) + off;
+      if (P.accumulate) v = __fadd_rn(v, __bfloat162float(*o));
+      *o = __float2bfloat16_rn(v);
     }
   }
 }
 
-// Epilogue, one tile: drain the TMEM accumulator chunk by chunk.
+// Epilogue, one tile: drain the TMEM accumulator chunk by chunk (the next
+// chunk's TMEM load overlaps this chunk's conversion and store); the buffer is
+// handed back once its last load has landed.
 template <Op op, int BN>
-__device__ __forceinline__ void epilogue_tile(const GemmParams& p, const OpParams& P, uint32_t tmem_base, int buf,
-                                              uint32_t stg, int lane, int q, int a0, int bp, float gamma,
-                                              uint32_t tmem_empty_lead) {
+__device__ __forceinline__ void epilogue_tile(const GemmParams& p, const OpParams& P, const CUtensorMap* out_map,
+                                              uint32_t tmem_base, int buf, uint32_t stg, int lane, int q, int a0,
+                                              int bp, float gamma, uint32_t tmem_empty_lead, uint32_t& seq) {
   // forward: s_x[m] * gamma of the tile's BN columns; lane l holds column 32c + l
   float col_scale[BN / 32];
 #pragma unroll
@@ -565,23 +554,25 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams& p, const OpParam
       col_scale[c] = j < P.rows_b ? __fmul_rn(__ldg(p.sx + j), gamma) : 0.0f;
     }
   }
+  const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * 256;
+  const int i0 = a0 + q * 32;
+  uint32_t ra[32], rb[32];
+  tmem_ld_32x32b_x32(tbase, ra);
+  tmem_ld_wait();
 #pragma unroll
   for (int c = 0; c < BN / 32; ++c) {
-    uint32_t r[32];
-    tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * 256 + c * 32, r);
-    tmem_ld_wait();
-    if (c == BN / 32 - 1) {
+    uint32_t(&cur)[32] = (c & 1) ? rb : ra;
+    uint32_t(&nxt)[32] = (c & 1) ? ra : rb;
+    if (c + 1 < BN / 32) {
+      tmem_ld_32x32b_x32(tbase + 32 * (c + 1), nxt);
+    } else {
+      // every TMEM load of this buffer has landed: hand it back
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(tmem_empty_lead);
     }
-    // transpose through smem: staging(j, lane) = D[row lane][column j]
-#pragma unroll
-    for (int j = 0; j < 32; ++j)
-      asm volatile("st.shared.b32 [%0], %1;" ::"r"(stg + stg_word(j, lane) * 4), "r"(r[j]) : "memory");
-    __syncwarp();
-    store_chunk<op>(p, P, stg, lane, q, a0, bp + c * 32, gamma, col_scale[c]);
-    __syncwarp();
+    epilogue_chunk<op>(p, P, out_map, cur, stg, lane, i0, bp + c * 32, col_scale[c], gamma, seq);
+    if (c + 1 < BN / 32) tmem_ld_wait();
   }
 }
 
@@ -590,7 +581,8 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams& p, const OpParam
 template <Family F, int BN>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap map_b0, const __grid_constant__ CUtensorMap map_src0,
-                     const __grid_constant__ CUtensorMap map_b1, const __grid_constant__ CUtensorMap map_src1,
+                     const __grid_constant__ CUtensorMap map_out0, const __grid_constant__ CUtensorMap map_b1,
+                     const __grid_constant__ CUtensorMap map_src1, const __grid_constant__ CUtensorMap map_out1,
                      const __grid_constant__ CUtensorMap map_sx, const __grid_constant__ GemmParams p) {
   using G = Geo<F, BN>;
   using L = Layout<F, BN>;
@@ -797,6 +789,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const float gamma = p.gamma ? __ldg(p.gamma) : 1.0f;
     int buf = 0;
     uint32_t buf_phase = 0;
+    uint32_t seq = 0;
     int tile;
     for (int i = 0; next_tile(p, pair, npairs, i, tile); ++i) {
       const TileInfo t = decode_tile<BN>(p, tile, rank);
@@ -804,14 +797,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       if (!wait(&tmem_full[buf], buf_phase)) break;
       tc_fence_after();
       if (t.opi == 0)
-        epilogue_tile<kOp0, BN>(p, P, tmem_base, buf, stg, lane, q, t.a0, t.bp, gamma, lead(&tmem_empty[buf]));
+        epilogue_tile<kOp0, BN>(p, P, &map_out0, tmem_base, buf, stg, lane, q, t.a0, t.bp, gamma,
+                                lead(&tmem_empty[buf]), seq);
       else if constexpr (F == Family::Bwd)
-        epilogue_tile<Op::Dw, BN>(p, P, tmem_base, buf, stg, lane, q, t.a0, t.bp, gamma, lead(&tmem_empty[buf]));
+        epilogue_tile<Op::Dw, BN>(p, P, &map_out1, tmem_base, buf, stg, lane, q, t.a0, t.bp, gamma,
+                                  lead(&tmem_empty[buf]), seq);
       if (++buf == 2) {
         buf = 0;
         buf_phase ^= 1;
       }
     }
+    if (lane == 0) bulk_wait_group_all();  // output writes complete before the CTA exits
+    __syncwarp();
   }
 
   tc_fence_before();
@@ -979,9 +976,16 @@ cudaError_t launch_pair(const CUtensorMap* maps, GemmParams& p, int npairs, cuda
                  static_cast<int>(F), BN, L::kS, L::kDynBytes, p.op[0].ntiles, p.op[1].ntiles, p.op[0].num_kb,
                  p.op[1].num_kb, pairs, p.use_sched);
   cudaError_t e = launch_pdl(gemm_pair_kernel<F, BN>, dim3(2 * pairs), dim3(kThreads), L::kDynBytes, s, maps[0],
-                             maps[1], maps[2], maps[3], maps[4], p);
+                             maps[1], maps[2], maps[3], maps[4], maps[5], maps[6], p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
+}
+
+// Output tensor map for TMA stores: [rows][cols] of 2- or 4-byte elements,
+// 32 x 32 boxes. TMA needs a 16-byte row pitch.
+bool make_out_map(CUtensorMap* m, void* base, bool f32, int64_t rows, int64_t cols, const char* what) {
+  return make_map_2d(m, base, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, cols, rows,
+                     cols * (f32 ? 4 : 2), 32, 32, CU_TENSOR_MAP_SWIZZLE_NONE, what);
 }
 
 // B rows per pair tile for the forward: the candidate with the fewest
@@ -1031,10 +1035,13 @@ cudaError_t launch_forward(const int8_t* xq, const float* sx, const uint8_t* w_p
   static const int kCands[3] = {256, 192, 128};
   const int npairs = resident_pairs<Family::Fwd, 256>();
   const int bn = choose_bn(static_cast<int>(N), static_cast<int>(M), npairs, kCands, 3);
-  CUtensorMap maps[5] = {};
+  CUtensorMap maps[7] = {};  // b0, src0, out0, b1, src1, out1, sx
   if (!make_map_2d(&maps[0], xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, K, M, K, 128, bn / 2, CU_TENSOR_MAP_SWIZZLE_128B,
                    "xq"))
     return cudaErrorInvalidValue;
+  // y [M][N] bf16 by TMA stores when its rows are 16-byte multiples
+  const bool tma_store = (N % 8) == 0 && debug_acc == nullptr;
+  if (tma_store && !make_out_map(&maps[2], y, false, M, N, "y")) return cudaErrorInvalidValue;
   // packed codes [N][K/4] bytes: a TMA tensor needs a 16-byte row pitch (K % 64 == 0)
   const bool src_tma = (K % 64) == 0;
   if (src_tma && !make_map_2d(&maps[1], w_packed, CU_TENSOR_MAP_DATA_TYPE_UINT8, K / 4, N, K / 4, 32, BM,
@@ -1046,6 +1053,7 @@ cudaError_t launch_forward(const int8_t* xq, const float* sx, const uint8_t* w_p
   p.op[0].out = y;
   p.op[0].ldo = N;
   p.op[0].src_tma = src_tma;
+  p.op[0].tma_store = tma_store;
   p.K = K;
   p.packed = w_packed;
   p.sx = sx;
@@ -1069,9 +1077,10 @@ cudaError_t launch_backward(const void* dY, const int8_t* xq, const float* sx, c
   if (M == 0) return cudaSuccess;
   constexpr int BN = 256;
   const int npairs = resident_pairs<Family::Bwd, BN>();
-  CUtensorMap maps[5] = {};
+  CUtensorMap maps[7] = {};  // b0, src0, out0, b1, src1, out1, sx
   const bool src_tma = (K % 64) == 0;
   if (dX) {
+    if (!make_out_map(&maps[2], dX, false, M, K, "dX")) return cudaErrorInvalidValue;
     if (!make_map_2d(&maps[0], dY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, N, M, N * 2, 64, BN / 2,
                      CU_TENSOR_MAP_SWIZZLE_128B, "dY (dX)"))
       return cudaErrorInvalidValue;
@@ -1082,13 +1091,14 @@ cudaError_t launch_backward(const void* dY, const int8_t* xq, const float* sx, c
   if (dW) {
     // s_x as a one-row 2D tensor: [1][M] floats, row pitch rounded up to 16 bytes
     const uint64_t sx_pitch = ((static_cast<uint64_t>(M) * 4 + 15) / 16) * 16;
-    if (!make_map_2d(&maps[2], dY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, N, M, N * 2, 64, 64,
+    if (!make_map_2d(&maps[3], dY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, N, M, N * 2, 64, 64,
                      CU_TENSOR_MAP_SWIZZLE_128B, "dY (dW)") ||
-        !make_map_2d(&maps[3], xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, K, M, K, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B,
+        !make_map_2d(&maps[4], xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, K, M, K, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B,
                      "xq (dW)") ||
-        !make_map_2d(&maps[4], sx, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, M, 1, sx_pitch, 64, 1, CU_TENSOR_MAP_SWIZZLE_NONE,
+        !make_map_2d(&maps[6], sx, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, M, 1, sx_pitch, 64, 1, CU_TENSOR_MAP_SWIZZLE_NONE,
                      "sx (dW)"))
       return cudaErrorInvalidValue;
+    if (!accumulate && !make_out_map(&maps[5], dW, dw_is_f32 != 0, N, K, "dW")) return cudaErrorInvalidValue;
   }
   static thread_local GemmParams p;
   std::memset(&p, 0, offsetof(GemmParams, sched_start));
@@ -1097,6 +1107,7 @@ cudaError_t launch_backward(const void* dY, const int8_t* xq, const float* sx, c
     p.op[0].out = dX;
     p.op[0].ldo = K;
     p.op[0].src_tma = src_tma;
+    p.op[0].tma_store = 1;
   }
   if (dW) {
     fill_op(p.op[1], static_cast<int>(K), static_cast<int>(N), static_cast<int>(M), 64, BN);
@@ -1104,6 +1115,7 @@ cudaError_t launch_backward(const void* dY, const int8_t* xq, const float* sx, c
     p.op[1].ldo = K;
     p.op[1].out_f32 = dw_is_f32;
     p.op[1].accumulate = accumulate;
+    p.op[1].tma_store = !accumulate;
   }
   p.K = K;
   p.packed = w_packed;
