@@ -468,52 +468,30 @@ __device__ __forceinline__ void st_shared_b32(uint32_t addr, uint32_t v) {
   asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
 }
 
-// Epilogue, one 32 x 32 chunk in registers: lane = output column i (A row),
-// r[jj] = output row j0 + jj. Written as one TMA store box from a staging
-// slot in shared memory (bf16: two 2 KB slots per warp, used in turn; f32:
-// the warp's whole 4 KB), or stored directly when the output is accumulated
-// into, for the debug output, and for row pitches a tensor map cannot take.
-// `seq` counts the warp's stored chunks (slot choice and reuse waits).
+// Epilogue paths taken for f32 output, accumulation, the debug output and
+// row pitches a tensor map cannot take: kept out of line so that the common
+// bf16 path stays small in the instruction caches.
+// f32 box through the warp's whole 4 KB staging slot.
 template <Op op>
-__device__ __forceinline__ void epilogue_chunk(const GemmParams& p, const OpParams& P, const CUtensorMap* out_map,
-                                               const uint32_t (&r)[32], uint32_t stg, int lane, int i0, int j0,
-                                               float col_scale, float gamma, uint32_t& seq) {
-  if (i0 >= P.rows_a || j0 >= P.rows_b) return;
-  if (P.tma_store) {
-    uint32_t slot;
-    if (P.out_f32) {
-      slot = stg;
-      if (lane == 0) bulk_wait_group_read<0>();  // the previous box has been read
-      __syncwarp();
-#pragma unroll
-      for (int jj = 0; jj < 32; ++jj)
-        st_shared_b32(slot + jj * 128 + lane * 4, __float_as_uint(epi_value<op>(r[jj], 0.0f)));
-    } else {
-      slot = stg + (seq & 1u) * 2048u;
-      if (lane == 0) bulk_wait_group_read<1>();  // the box stored from this slot two chunks ago has been read
-      __syncwarp();
-#pragma unroll
-      for (int jj = 0; jj < 32; ++jj) {
-        float scale = 0.0f;
-        if constexpr (op == Op::Fwd) scale = __shfl_sync(0xffffffffu, col_scale, jj);
-        else if constexpr (op == Op::Dx) scale = gamma;
-        const __nv_bfloat16 b = __float2bfloat16_rn(epi_value<op>(r[jj], scale));
-        st_shared_b16(slot + jj * 64 + lane * 2, *reinterpret_cast<const uint16_t*>(&b));
-      }
-    }
-    fence_proxy_async_smem();
-    __syncwarp();
-    if (lane == 0) {
-      tma_store_2d(out_map, slot, i0, j0);
-      bulk_commit_group();
-    }
-    ++seq;
-    return;
+__device__ __noinline__ void epilogue_chunk_f32(const CUtensorMap* out_map, const uint32_t* r, uint32_t stg, int lane,
+                                                int i0, int j0) {
+  if (lane == 0) bulk_wait_group_read<0>();  // the previous box has been read
+  __syncwarp();
+  for (int jj = 0; jj < 32; ++jj) st_shared_b32(stg + jj * 128 + lane * 4, __float_as_uint(epi_value<op>(r[jj], 0.0f)));
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (lane == 0) {
+    tma_store_2d(out_map, stg, i0, j0);
+    bulk_commit_group();
   }
-  // direct stores: lane i writes column i of each row j (the warp's 32 lanes
-  // write contiguous elements of one row)
+}
+
+// Direct stores: lane i writes column i of each row j (the warp's 32 lanes
+// write contiguous elements of one row).
+template <Op op>
+__device__ __noinline__ void epilogue_chunk_direct(const GemmParams& p, const OpParams& P, const uint32_t* r, int lane,
+                                                   int i0, int j0, float col_scale, float gamma) {
   const int i = i0 + lane;
-#pragma unroll
   for (int jj = 0; jj < 32; ++jj) {
     float scale = 0.0f;
     if constexpr (op == Op::Fwd) scale = __shfl_sync(0xffffffffu, col_scale, jj);
@@ -537,42 +515,82 @@ __device__ __forceinline__ void epilogue_chunk(const GemmParams& p, const OpPara
   }
 }
 
-// Epilogue, one tile: drain the TMEM accumulator chunk by chunk (the next
-// chunk's TMEM load overlaps this chunk's conversion and store); the buffer is
-// handed back once its last load has landed.
+// Epilogue, one 32 x 32 chunk in registers: lane = output column i (A row),
+// r[jj] = output row j0 + jj. The common case is a bf16 box converted into
+// one of the warp's two 2 KB staging slots (used in turn) and written by one
+// TMA store. `seq` counts the warp's bf16 boxes.
+template <Op op>
+__device__ __forceinline__ void epilogue_chunk(const GemmParams& p, const OpParams& P, const CUtensorMap* out_map,
+                                               uint32_t (&r)[32], uint32_t stg, int lane, int i0, int j0,
+                                               float col_scale, float gamma, uint32_t& seq) {
+  if (i0 >= P.rows_a || j0 >= P.rows_b) return;
+  if (!P.tma_store || P.out_f32) {
+    // the out-of-line paths take a copy, so that r itself stays in registers
+    uint32_t t[32];
+#pragma unroll
+    for (int jj = 0; jj < 32; ++jj) t[jj] = r[jj];
+    if (!P.tma_store)
+      epilogue_chunk_direct<op>(p, P, t, lane, i0, j0, col_scale, gamma);
+    else
+      epilogue_chunk_f32<op>(out_map, t, stg, lane, i0, j0);
+    return;
+  }
+  const uint32_t slot = stg + (seq & 1u) * 2048u;
+  if (lane == 0) bulk_wait_group_read<1>();  // the box stored from this slot two chunks ago has been read
+  __syncwarp();
+#pragma unroll
+  for (int jj = 0; jj < 32; ++jj) {
+    float scale = 0.0f;
+    if constexpr (op == Op::Fwd) scale = __shfl_sync(0xffffffffu, col_scale, jj);
+    else if constexpr (op == Op::Dx) scale = gamma;
+    const __nv_bfloat16 b = __float2bfloat16_rn(epi_value<op>(r[jj], scale));
+    st_shared_b16(slot + jj * 64 + lane * 2, *reinterpret_cast<const uint16_t*>(&b));
+  }
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (lane == 0) {
+    tma_store_2d(out_map, slot, i0, j0);
+    bulk_commit_group();
+  }
+  ++seq;
+}
+
+// Epilogue, one tile: drain the TMEM accumulator two 32-column chunks per
+// (rolled) iteration; each chunk's TMEM load overlaps the previous chunk's
+// conversion and store, and the buffer is handed back once the last load has
+// landed.
 template <Op op, int BN>
 __device__ __forceinline__ void epilogue_tile(const GemmParams& p, const OpParams& P, const CUtensorMap* out_map,
                                               uint32_t tmem_base, int buf, uint32_t stg, int lane, int q, int a0,
                                               int bp, float gamma, uint32_t tmem_empty_lead, uint32_t& seq) {
-  // forward: s_x[m] * gamma of the tile's BN columns; lane l holds column 32c + l
-  float col_scale[BN / 32];
-#pragma unroll
-  for (int c = 0; c < BN / 32; ++c) {
-    col_scale[c] = 0.0f;
-    if constexpr (op == Op::Fwd) {
-      const int j = bp + c * 32 + lane;
-      col_scale[c] = j < P.rows_b ? __fmul_rn(__ldg(p.sx + j), gamma) : 0.0f;
-    }
-  }
+  static_assert(BN % 64 == 0, "chunks are drained in pairs");
   const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * 256;
   const int i0 = a0 + q * 32;
   uint32_t ra[32], rb[32];
   tmem_ld_32x32b_x32(tbase, ra);
   tmem_ld_wait();
-#pragma unroll
-  for (int c = 0; c < BN / 32; ++c) {
-    uint32_t(&cur)[32] = (c & 1) ? rb : ra;
-    uint32_t(&nxt)[32] = (c & 1) ? ra : rb;
-    if (c + 1 < BN / 32) {
-      tmem_ld_32x32b_x32(tbase + 32 * (c + 1), nxt);
+#pragma unroll 1
+  for (int c = 0; c < BN / 32; c += 2) {
+    // forward: s_x[m] * gamma of the two chunks' columns (lane l: column 32c + l)
+    float s0 = 0.0f, s1 = 0.0f;
+    if constexpr (op == Op::Fwd) {
+      const int j = bp + c * 32 + lane;
+      s0 = j < P.rows_b ? __fmul_rn(__ldg(p.sx + j), gamma) : 0.0f;
+      s1 = j + 32 < P.rows_b ? __fmul_rn(__ldg(p.sx + j + 32), gamma) : 0.0f;
+    }
+    tmem_ld_32x32b_x32(tbase + 32 * (c + 1), rb);
+    epilogue_chunk<op>(p, P, out_map, ra, stg, lane, i0, bp + c * 32, s0, gamma, seq);
+    tmem_ld_wait();
+    if (c + 2 < BN / 32) {
+      tmem_ld_32x32b_x32(tbase + 32 * (c + 2), ra);
     } else {
       // every TMEM load of this buffer has landed: hand it back
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(tmem_empty_lead);
     }
-    epilogue_chunk<op>(p, P, out_map, cur, stg, lane, i0, bp + c * 32, col_scale[c], gamma, seq);
-    if (c + 1 < BN / 32) tmem_ld_wait();
+    epilogue_chunk<op>(p, P, out_map, rb, stg, lane, i0, bp + (c + 1) * 32, s1, gamma, seq);
+    if (c + 2 < BN / 32) tmem_ld_wait();
   }
 }
 
