@@ -1,8 +1,9 @@
 """Benchmark of the BitLinear training hot path (fwd + bwd) on B200.
 
 One step = one pass of the whole hot path over one batch:
-  S1 bl_quantize_weight (2 launches) -> S2 bl_quantize_act -> S3 bl_forward
-  -> S4 bl_backward (dX and dW in one launch)                  (5 launches)
+  S1 + S2 bl_quantize (2 launches: |W| partial sums together with the
+  token quantisation, then the code pass) -> S3 bl_forward
+  -> S4 bl_backward (dX and dW in one launch)                  (4 launches)
 
 Default workload: the up-projection BitLinear 2560 -> 6912 at 8 x 512 tokens
 (M=4096, K=2560, N=6912; x, dY bf16 ~ N(0,1), W bf16 kaiming-uniform).
@@ -167,15 +168,14 @@ def job_tops(ops_per_rank_step: float, world: int, steps: int, job_ms: float) ->
 
 # ----------------------------------------------------------------- our arm
 
-STAGES = ["quantize_weight", "quantize_act", "forward", "backward"]
-LAUNCHES_PER_STEP = 5  # S1 two passes, S2, S3, S4 (dX and dW in one launch)
+STAGES = ["quantize", "forward", "backward"]
+LAUNCHES_PER_STEP = 4  # S1 pass A with S2, S1 pass B, S3, S4 (dX and dW in one launch)
 
 
 def stage_work(M, N, K, w_bytes):
     """Algorithmic work per launch group: bytes for the HBM passes, ops for GEMMs."""
     return {
-        "quantize_weight": {"bound": "hbm", "bytes": N * K * w_bytes + N * K // 4 + 4},
-        "quantize_act": {"bound": "hbm", "bytes": M * K * 2 + M * K + 4 * M},
+        "quantize": {"bound": "hbm", "bytes": N * K * w_bytes + N * K // 4 + 4 + M * K * 2 + M * K + 4 * M},
         "forward": {"bound": "tensor", "ops": 2 * M * N * K, "dtype": "int8"},
         "backward": {"bound": "tensor", "ops": 4 * M * N * K, "dtype": "bf16"},
     }
@@ -205,18 +205,15 @@ def run_ours(args, rank, world, local_rank):
     def step(evs=None):
         if evs:
             evs[0].record(stream)
-        bl.bl_quantize_weight(w, bufs.w_packed, bufs.gamma, bufs.workspace, stream)
+        bl.bl_quantize(w, x, bufs.w_packed, bufs.gamma, bufs.xq, bufs.sx, bufs.workspace, stream)
         if evs:
             evs[1].record(stream)
-        bl.bl_quantize_act(x, bufs.xq, bufs.sx, stream)
-        if evs:
-            evs[2].record(stream)
         bl.bl_forward(bufs.xq, bufs.sx, bufs.w_packed, bufs.gamma, bufs.y, None, stream)
         if evs:
-            evs[3].record(stream)
+            evs[2].record(stream)
         bl.bl_backward(dy, bufs.xq, bufs.sx, bufs.w_packed, bufs.gamma, bufs.dX, bufs.dW, False, stream)
         if evs:
-            evs[4].record(stream)
+            evs[3].record(stream)
 
     for i in range(args.warmup):
         flush_l2(i)

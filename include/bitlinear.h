@@ -110,7 +110,7 @@ bl_status bl_quantize_weight(const void* W, bl_dtype w_dtype, int64_t N, int64_t
  *
  * It computes exactly what bl_quantize_weight computes (same kernels, same
  * bit-identical outputs) and calls no allocator. Its fp64 partial sums go to
- * a fixed array inside the library of 592 doubles (4736 bytes), enough for a
+ * a fixed array inside the library of 296 doubles (2368 bytes), enough for a
  * tensor of any size; each GPU that loads the library keeps that array until
  * the process exits. A request that would need more scratch than the array
  * holds returns BL_ERR_WORKSPACE.
@@ -142,6 +142,22 @@ bl_status bl_quantize_weight_noalloc(const void* W, bl_dtype w_dtype, int64_t N,
  */
 bl_status bl_quantize_act(const void* x, int64_t M, int64_t K,
                           int8_t* xq, float* sx, void* stream);
+
+/*
+ * S1 + S2 in one call: the same outputs as bl_quantize_weight(W, ...) followed
+ * by bl_quantize_act(x, ...), bit for bit. The two steps are independent, so
+ * the |W| partial sums of S1 and the whole of S2 run in one launch and their
+ * memory traffic overlaps; S1's code pass follows. (The pages run the two
+ * quantisers one after the other; this is a scheduling choice only.)
+ *
+ * Arguments: those of bl_quantize_weight and bl_quantize_act. M == 0 skips
+ * S2 (x, xq, sx may then be NULL). Errors: as bl_quantize_weight, plus those
+ * of bl_quantize_act's arguments.
+ */
+bl_status bl_quantize(const void* W, bl_dtype w_dtype, int64_t N, int64_t K,
+                      const void* x, int64_t M,
+                      uint8_t* w_packed, float* gamma, int8_t* xq, float* sx,
+                      void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * S3 -- forward ("bitnet-qat-train", Semantics):

@@ -37,6 +37,7 @@ SIGNATURES = {
     "bl_quantize_weight": (_I32, [_VP, _I32, _I64, _I64, _VP, _VP, _VP, _SZ, _VP]),
     "bl_quantize_weight_noalloc": (_I32, [_VP, _I32, _I64, _I64, _VP, _VP, _VP]),
     "bl_quantize_act": (_I32, [_VP, _I64, _I64, _VP, _VP, _VP]),
+    "bl_quantize": (_I32, [_VP, _I32, _I64, _I64, _VP, _I64, _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
     "bl_forward": (_I32, [_VP, _VP, _VP, _VP, _I64, _I64, _I64, _VP, _VP, _VP]),
     "bl_backward": (_I32, [_VP, _VP, _VP, _VP, _VP, _I64, _I64, _I64, _VP, _VP, _I32, _I32, _VP]),
     "bl_export_weights": (_I32, [_VP, _VP, _I64, _I64, _VP, _VP, _VP]),
@@ -132,6 +133,25 @@ def bl_quantize_act(x, xq, sx, stream=None):
     _check(load_library().bl_quantize_act(_ptr(x), M, K, _ptr(xq), _ptr(sx), _stream(stream)), "bl_quantize_act")
 
 
+def bl_quantize(W, x, w_packed, gamma, xq, sx, workspace, stream=None):
+    """S1 + S2 in one call (same outputs as bl_quantize_weight then bl_quantize_act)."""
+    N, K = W.shape
+    M = x.shape[0]
+    if W.dtype not in (torch.bfloat16, torch.float32):
+        raise ValueError("W must be bf16 or f32")
+    _need(W, W.dtype, (N, K), "W")
+    _need(x, torch.bfloat16, (M, K), "x")
+    _need(w_packed, torch.uint8, (N, K // 4), "w_packed")
+    _need(gamma, torch.float32, (1,), "gamma")
+    _need(xq, torch.int8, (M, K), "xq")
+    _need(sx, torch.float32, (M,), "sx")
+    wdt = BL_F32 if W.dtype == torch.float32 else BL_BF16
+    _check(load_library().bl_quantize(_ptr(W), wdt, N, K, _ptr(x), M, _ptr(w_packed), _ptr(gamma), _ptr(xq),
+                                      _ptr(sx), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                      _stream(stream)),
+           "bl_quantize")
+
+
 def bl_forward(xq, sx, w_packed, gamma, y, debug_acc=None, stream=None):
     """S3: y [M,N] bf16 = xq . codes^T * sx * gamma (debug_acc [M,N] int32 optional)."""
     M, K = xq.shape
@@ -217,8 +237,7 @@ class StepBuffers:
 
 
 def bitlinear_step(x, W, dY, bufs: StepBuffers, stream=None):
-    """One BitLinear forward + backward: S1 -> S2 -> S3 -> S4 (five kernel launches)."""
-    bl_quantize_weight(W, bufs.w_packed, bufs.gamma, bufs.workspace, stream)
-    bl_quantize_act(x, bufs.xq, bufs.sx, stream)
+    """One BitLinear forward + backward: S1 + S2 (bl_quantize) -> S3 -> S4 (four kernel launches)."""
+    bl_quantize(W, x, bufs.w_packed, bufs.gamma, bufs.xq, bufs.sx, bufs.workspace, stream)
     bl_forward(bufs.xq, bufs.sx, bufs.w_packed, bufs.gamma, bufs.y, None, stream)
     bl_backward(dY, bufs.xq, bufs.sx, bufs.w_packed, bufs.gamma, bufs.dX, bufs.dW, False, stream)

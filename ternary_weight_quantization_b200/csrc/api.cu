@@ -155,6 +155,29 @@ bl_status bl_quantize_act(const void* x, int64_t M, int64_t K, int8_t* xq, float
                      "bl_quantize_act launch");
 }
 
+bl_status bl_quantize(const void* W, bl_dtype w_dtype, int64_t N, int64_t K, const void* x, int64_t M,
+                      uint8_t* w_packed, float* gamma, int8_t* xq, float* sx, void* workspace,
+                      size_t workspace_bytes, void* stream) {
+  g_msg[0] = 0;
+  if (N < 1) return fail(BL_ERR_INVALID_ARG, "N=%lld must be >= 1", (long long)N);
+  if (M < 0) return fail(BL_ERR_INVALID_ARG, "M=%lld must be >= 0", (long long)M);
+  if (bl_status s = check_k(K)) return s;
+  if (w_dtype != BL_BF16 && w_dtype != BL_F32) return fail(BL_ERR_DTYPE, "w_dtype %d", (int)w_dtype);
+  if (!W || !w_packed || !gamma) return fail(BL_ERR_INVALID_ARG, "null pointer");
+  if (M > 0 && (!x || !xq || !sx)) return fail(BL_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(W) || !aligned16(w_packed) || !aligned16(gamma) || (x && !aligned16(x)) ||
+      (xq && !aligned16(xq)) || (sx && !aligned16(sx)))
+    return fail(BL_ERR_ALIGNMENT, "tensors must be 16-byte aligned");
+  const size_t need = bl_quantize_weight_workspace_size(N, K);
+  if (!workspace || workspace_bytes < need || !aligned16(workspace))
+    return fail(BL_ERR_WORKSPACE, "workspace needs %zu bytes, 16-byte aligned", need);
+  int* err = nullptr;
+  if (bl_status s = current_device(&err)) return s;
+  return cuda_status(bl::launch_quantize(W, w_dtype == BL_F32, N, K, x, M, w_packed, gamma,
+                                         static_cast<double*>(workspace), xq, sx, static_cast<cudaStream_t>(stream)),
+                     "bl_quantize launch");
+}
+
 bl_status bl_forward(const int8_t* xq, const float* sx, const uint8_t* w_packed, const float* gamma, int64_t M,
                      int64_t N, int64_t K, void* y, int32_t* debug_acc, void* stream) {
   g_msg[0] = 0;

@@ -45,6 +45,11 @@ size_t noalloc_scratch_bytes();
 // ---- S2: per-token absmax INT8
 cudaError_t launch_quantize_act(const void* x, int64_t M, int64_t K, int8_t* xq, float* sx, cudaStream_t s);
 
+// ---- S1 + S2 together (bl_quantize): pass A and the activation quantisation
+// in one launch, then pass B. `partials` as for launch_quantize_weight.
+cudaError_t launch_quantize(const void* W, int w_is_f32, int64_t N, int64_t K, const void* x, int64_t M,
+                            uint8_t* packed, float* gamma, double* partials, int8_t* xq, float* sx, cudaStream_t s);
+
 // ---- S3 / S4 GEMMs (tcgen05)
 cudaError_t launch_forward(const int8_t* xq, const float* sx, const uint8_t* w_packed, const float* gamma,
                            int64_t M, int64_t N, int64_t K, void* y, int32_t* debug_acc, int* err,

@@ -17,9 +17,9 @@ namespace bl {
 namespace {
 
 constexpr int kQuantThreads = 256;
-// Upper bound on pass-A blocks: four 256-thread blocks per SM on a 148-SM
+// Upper bound on pass-A blocks: two 256-thread blocks per SM on a 148-SM
 // B200. A fixed constant, so the fp64 reduction tree is the same on any GPU.
-constexpr int kMaxPartials = 592;
+constexpr int kMaxPartials = 296;
 
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
@@ -89,26 +89,50 @@ __device__ __forceinline__ double add_group(double acc, const Group<kF32>& a) {
 // partials[b] = sum of |w| over block b's contiguous range of groups, fp64.
 // Each thread keeps four accumulators (group u of every four goes to
 // accumulator u; leftover groups to accumulator 0), adds them as
-// (a0 + a1) + (a2 + a3), then a fixed shuffle/smem tree.
-template <bool kF32>
-__global__ void __launch_bounds__(kQuantThreads) absmean_partials_kernel(const uint4* __restrict__ W,
-                                                                         int64_t ngroups, int64_t per_block,
-                                                                         double* __restrict__ partials) {
-  pdl_wait_primary();       // W may come from the previous kernel (e.g. an optimizer step)
-  pdl_launch_dependents();  // the code pass may start loading W while this pass finishes
+// (a0 + a1) + (a2 + a3), then a fixed shuffle/smem tree. The groups are
+// loaded kLoad at a time (4 or 2), the next batch while the current one is
+// summed; the order of the additions does not depend on kLoad.
+template <bool kF32, int kLoad>
+__device__ __forceinline__ void absmean_block(const uint4* __restrict__ W, int64_t ngroups, int64_t per_block,
+                                              int64_t block, double* __restrict__ partials) {
+  static_assert(kLoad == 2 || kLoad == 4, "batches split a quad of groups");
   constexpr int T = kQuantThreads;
-  const int64_t g0 = static_cast<int64_t>(blockIdx.x) * per_block;
+  constexpr int kPerQuad = 4 / kLoad;
+  const int64_t g0 = block * per_block;
   const int64_t g1 = min(g0 + per_block, ngroups);
   double acc[4] = {0.0, 0.0, 0.0, 0.0};
-  int64_t g = g0 + threadIdx.x;
-  for (; g + 3 * T < g1; g += 4 * T) {
-    Group<kF32> a[4];
+  const int64_t gt = g0 + threadIdx.x;
+  // full quads of this thread: groups gt + (4q + u) T, u = 0..3, all < g1
+  const int64_t nquads = gt + 3 * T < g1 ? (g1 - 1 - 3 * T - gt) / (4 * T) + 1 : 0;
+  const int64_t nbatch = nquads * kPerQuad;
+  if (nbatch > 0) {
+    Group<kF32> a[kLoad];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) a[u].load(W, g + u * T);
+    for (int v = 0; v < kLoad; ++v) a[v].load(W, gt + v * T);
+    for (int64_t b = 0; b < nbatch; ++b) {
+      const int64_t bn = b + 1;
+      Group<kF32> nxt[kLoad];
+      if (bn < nbatch) {
+        const int64_t base = gt + (bn / kPerQuad) * 4 * T + (bn % kPerQuad) * kLoad * T;
 #pragma unroll
-    for (int u = 0; u < 4; ++u) acc[u] = add_group(acc[u], a[u]);
+        for (int v = 0; v < kLoad; ++v) nxt[v].load(W, base + v * T);
+      }
+      const int u0 = static_cast<int>(b % kPerQuad) * kLoad;
+#pragma unroll
+      for (int v = 0; v < kLoad; ++v) {
+        if constexpr (kLoad == 4) {
+          acc[v] = add_group(acc[v], a[v]);
+        } else {
+          // accumulator u0 + v (u0 is 0 or 2)
+          if (u0 == 0) acc[v] = add_group(acc[v], a[v]);
+          else acc[2 + v] = add_group(acc[2 + v], a[v]);
+        }
+      }
+#pragma unroll
+      for (int v = 0; v < kLoad; ++v) a[v] = nxt[v];
+    }
   }
-  for (; g < g1; g += T) {
+  for (int64_t g = gt + nquads * 4 * T; g < g1; g += T) {
     Group<kF32> a;
     a.load(W, g);
     acc[0] = add_group(acc[0], a);
@@ -120,11 +144,20 @@ __global__ void __launch_bounds__(kQuantThreads) absmean_partials_kernel(const u
   if ((threadIdx.x & 31) == 0) warp_sums[threadIdx.x >> 5] = t;
   __syncthreads();
   if (threadIdx.x == 0) {
-    double s = 0.0;
+    double sum = 0.0;
 #pragma unroll
-    for (int w = 0; w < kQuantThreads / 32; ++w) s = __dadd_rn(s, warp_sums[w]);
-    partials[blockIdx.x] = s;
+    for (int w = 0; w < kQuantThreads / 32; ++w) sum = __dadd_rn(sum, warp_sums[w]);
+    partials[block] = sum;
   }
+}
+
+template <bool kF32>
+__global__ void __launch_bounds__(kQuantThreads) absmean_partials_kernel(const uint4* __restrict__ W,
+                                                                         int64_t ngroups, int64_t per_block,
+                                                                         double* __restrict__ partials) {
+  pdl_wait_primary();       // W may come from the previous kernel (e.g. an optimizer step)
+  pdl_launch_dependents();  // the code pass may start loading W while this pass finishes
+  absmean_block<kF32, 4>(W, ngroups, per_block, blockIdx.x, partials);
 }
 
 // ---------------------------------------------------------------- S1 pass B
@@ -153,20 +186,21 @@ __device__ __forceinline__ uint32_t pack_group(const Group<kF32>& a, float thr) 
 }
 
 template <bool kF32>
-__global__ void __launch_bounds__(kQuantThreads) ternarize_pack_kernel(const uint4* __restrict__ W,
-                                                                       int64_t ngroups, int64_t per_block,
-                                                                       const double* __restrict__ partials,
-                                                                       int nparts, int64_t numel,
-                                                                       uint32_t* __restrict__ packed,
-                                                                       float* __restrict__ gamma_out) {
-  constexpr int T = kQuantThreads;
-  const int64_t g0 = static_cast<int64_t>(blockIdx.x) * per_block;
-  const int64_t g1 = min(g0 + per_block, ngroups);
-  const int64_t gf = g0 + threadIdx.x;
-  Group<kF32> first[4];
+__global__ void __launch_bounds__(kQuantThreads, kF32 ? 2 : 4) ternarize_pack_kernel(const uint4* __restrict__ W,
+                                                                          int64_t ngroups,
+                                                                          const double* __restrict__ partials,
+                                                                          int nparts, int64_t numel,
+                                                                          uint32_t* __restrict__ packed,
+                                                                          float* __restrict__ gamma_out) {
+  // Threads stride over the groups (consecutive threads, consecutive groups),
+  // two groups per batch, the next batch loaded while the current one is
+  // packed; the first batch is loaded before the wait.
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * kQuantThreads;
+  int64_t g = static_cast<int64_t>(blockIdx.x) * kQuantThreads + threadIdx.x;
+  Group<kF32> a[2];
 #pragma unroll
-  for (int u = 0; u < 4; ++u)
-    if (gf + u * T < g1) first[u].load(W, gf + u * T);
+  for (int u = 0; u < 2; ++u)
+    if (g + u * stride < ngroups) a[u].load(W, g + u * stride);
 
   pdl_wait_primary();  // pass A has finished and its partial sums are visible
   pdl_launch_dependents();
@@ -174,7 +208,7 @@ __global__ void __launch_bounds__(kQuantThreads) ternarize_pack_kernel(const uin
   __shared__ double red[kQuantThreads / 32];
   __shared__ float s_thr;
   double t = 0.0;
-  for (int i = threadIdx.x; i < nparts; i += T) t = __dadd_rn(t, partials[i]);
+  for (int i = threadIdx.x; i < nparts; i += kQuantThreads) t = __dadd_rn(t, partials[i]);
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) t = __dadd_rn(t, __shfl_xor_sync(0xffffffffu, t, off));
   if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = t;
@@ -191,21 +225,17 @@ __global__ void __launch_bounds__(kQuantThreads) ternarize_pack_kernel(const uin
   __syncthreads();
   const float thr = s_thr;
 
+  for (; g < ngroups; g += 2 * stride) {
+    const int64_t gn = g + 2 * stride;
+    Group<kF32> b[2];
 #pragma unroll
-  for (int u = 0; u < 4; ++u)
-    if (gf + u * T < g1) packed[gf + u * T] = pack_group(first[u], thr);
-  int64_t g = gf + 4 * T;
-  for (; g + 3 * T < g1; g += 4 * T) {
-    Group<kF32> a[4];
+    for (int u = 0; u < 2; ++u)
+      if (gn + u * stride < ngroups) b[u].load(W, gn + u * stride);
 #pragma unroll
-    for (int u = 0; u < 4; ++u) a[u].load(W, g + u * T);
+    for (int u = 0; u < 2; ++u)
+      if (g + u * stride < ngroups) packed[g + u * stride] = pack_group(a[u], thr);
 #pragma unroll
-    for (int u = 0; u < 4; ++u) packed[g + u * T] = pack_group(a[u], thr);
-  }
-  for (; g < g1; g += T) {
-    Group<kF32> a;
-    a.load(W, g);
-    packed[g] = pack_group(a, thr);
+    for (int u = 0; u < 2; ++u) a[u] = b[u];
   }
 }
 
@@ -281,22 +311,18 @@ __device__ __forceinline__ void quant_row(const uint4 (&v)[VPL], int nv, int lan
   }
 }
 
-// Warps stride over rows; with short rows (kPrefetch) the next row's loads
-// are issued before the current row is quantised.
+// Warps stride over rows (first row m, then m + stride, ...); with short rows
+// (kPrefetch) the next row's loads are issued before the current row is
+// quantised.
 template <int VPL, bool kPrefetch>
-__global__ void __launch_bounds__(32 * kActRowsPerBlock) act_quant_kernel(const uint4* __restrict__ x, int64_t M,
-                                                                          int nv, int8_t* __restrict__ xq,
-                                                                          float* __restrict__ sx) {
-  pdl_wait_primary();
-  pdl_launch_dependents();
+__device__ __forceinline__ void act_rows(const uint4* __restrict__ x, int64_t M, int nv, int8_t* __restrict__ xq,
+                                         float* __restrict__ sx, int64_t m, int64_t stride) {
   const int lane = threadIdx.x & 31;
-  const int64_t nwarps = static_cast<int64_t>(gridDim.x) * kActRowsPerBlock;
-  int64_t m = static_cast<int64_t>(blockIdx.x) * kActRowsPerBlock + (threadIdx.x >> 5);
   if (m >= M) return;
   uint4 v[VPL];
   load_row<VPL>(x + m * nv, nv, lane, v);
   while (true) {
-    const int64_t mn = m + nwarps;
+    const int64_t mn = m + stride;
     if constexpr (kPrefetch) {
       uint4 vn[VPL];
       if (mn < M) load_row<VPL>(x + mn * nv, nv, lane, vn);
@@ -311,6 +337,66 @@ __global__ void __launch_bounds__(32 * kActRowsPerBlock) act_quant_kernel(const 
     }
     m = mn;
   }
+}
+
+template <int VPL, bool kPrefetch>
+__global__ void __launch_bounds__(32 * kActRowsPerBlock) act_quant_kernel(const uint4* __restrict__ x, int64_t M,
+                                                                          int nv, int8_t* __restrict__ xq,
+                                                                          float* __restrict__ sx) {
+  pdl_wait_primary();
+  pdl_launch_dependents();
+  act_rows<VPL, kPrefetch>(x, M, nv, xq, sx,
+                           static_cast<int64_t>(blockIdx.x) * kActRowsPerBlock + (threadIdx.x >> 5),
+                           static_cast<int64_t>(gridDim.x) * kActRowsPerBlock);
+}
+
+// One row per warp, read twice: absmax, then quantisation (the second read
+// mostly hits L1/L2).
+__device__ __forceinline__ void act_rows_two_pass(const uint4* __restrict__ x, int64_t M, int nv,
+                                                  int8_t* __restrict__ xq, float* __restrict__ sx, int64_t m,
+                                                  int64_t stride) {
+  const int lane = threadIdx.x & 31;
+  for (; m < M; m += stride) {
+    const uint4* row = x + m * nv;
+    float amax = 0.0f;
+    for (int j = lane; j < nv; j += 32) amax = absmax8(__ldg(row + j), amax);
+    const float a = fmaxf(warp_max(amax), 1e-5f);
+    const float inv = __fdiv_rn(127.0f, a);
+    if (lane == 0) sx[m] = __fdiv_rn(a, 127.0f);
+    uint2* out = reinterpret_cast<uint2*>(xq + m * static_cast<int64_t>(nv) * 8);
+    for (int j = lane; j < nv; j += 32) out[j] = quant8(__ldg(row + j), inv);
+  }
+}
+
+// S1 pass A and S2 in one launch (bl_quantize): blocks 0 .. nparts-1 sum |W|
+// over their ranges (the same partial sums absmean_partials_kernel writes);
+// the other blocks' warps quantise tokens. The two kinds of work are
+// independent, so their memory traffic and arithmetic overlap. Four blocks
+// fit on an SM with bf16 weights (64 registers; two with f32 weights): rows of
+// up to 1024 elements stay in registers (VPL <= 4), longer ones are read
+// twice (VPL = 0).
+constexpr int kFusedMaxVpl = 4;
+
+template <bool kF32, int VPL>
+__global__ void __launch_bounds__(kQuantThreads, kF32 ? 2 : 4) quant_phase1_kernel(const uint4* __restrict__ W,
+                                                                        int64_t ngroups, int64_t per_block,
+                                                                        int nparts, double* __restrict__ partials,
+                                                                        const uint4* __restrict__ x, int64_t M,
+                                                                        int nv, int8_t* __restrict__ xq,
+                                                                        float* __restrict__ sx) {
+  pdl_wait_primary();
+  pdl_launch_dependents();
+  if (static_cast<int>(blockIdx.x) < nparts) {
+    absmean_block<kF32, 2>(W, ngroups, per_block, blockIdx.x, partials);
+    return;
+  }
+  constexpr int kWarps = kQuantThreads / 32;
+  const int64_t m = static_cast<int64_t>(blockIdx.x - nparts) * kWarps + (threadIdx.x >> 5);
+  const int64_t stride = static_cast<int64_t>(gridDim.x - nparts) * kWarps;
+  if constexpr (VPL > 0)
+    act_rows<VPL, false>(x, M, nv, xq, sx, m, stride);
+  else
+    act_rows_two_pass(x, M, nv, xq, sx, m, stride);
 }
 
 // Rows longer than 8192 elements: absmax pass, then a second read (from L2).
@@ -336,9 +422,16 @@ __global__ void __launch_bounds__(32 * kActRowsPerBlock) act_quant_long_kernel(c
 }  // namespace
 
 // Fixed device scratch for bl_quantize_weight_noalloc: room for the largest
-// number of fp64 partial sums pass A ever writes (kMaxPartials), 4736 bytes.
+// number of fp64 partial sums pass A ever writes (kMaxPartials), 2368 bytes.
 // Every GPU that loads the library holds this array until the process exits.
 static __device__ __align__(256) double g_noalloc_partials[kMaxPartials];
+
+// Blocks of the code pass: four per SM, fewer for small tensors.
+static unsigned code_pass_blocks(int64_t ngroups) {
+  const int64_t want = (ngroups + kQuantThreads - 1) / kQuantThreads;
+  const int64_t cap = static_cast<int64_t>(4) * device_sm_count();
+  return static_cast<unsigned>(want < cap ? want : cap);
+}
 
 int weight_partials_count(int64_t numel) {
   const int64_t ngroups = numel / 16;
@@ -352,8 +445,8 @@ static cudaError_t launch_weight_passes(const uint4* w, int64_t ngroups, int64_t
   cudaError_t e = launch_pdl(absmean_partials_kernel<kF32>, dim3(nparts), dim3(kQuantThreads), 0, s, w, ngroups,
                              per_block, partials);
   if (e != cudaSuccess) return e;
-  return launch_pdl(ternarize_pack_kernel<kF32>, dim3(nparts), dim3(kQuantThreads), 0, s, w, ngroups, per_block,
-                    static_cast<const double*>(partials), nparts, numel, out, gamma);
+  return launch_pdl(ternarize_pack_kernel<kF32>, dim3(code_pass_blocks(ngroups)), dim3(kQuantThreads), 0, s, w,
+                    ngroups, static_cast<const double*>(partials), nparts, numel, out, gamma);
 }
 
 cudaError_t launch_quantize_weight(const void* W, int w_is_f32, int64_t N, int64_t K, uint8_t* packed,
@@ -423,6 +516,43 @@ static void launch_act(const uint4* xv, int64_t M, int nv, int8_t* xq, float* sx
   launch_pdl(act_quant_kernel<VPL, kPrefetch>, dim3(grid), dim3(32 * kActRowsPerBlock), 0, s, xv, M, nv, xq, sx);
 }
 
+// bl_quantize: S1 pass A and S2 in one launch (quant_phase1_kernel), then the
+// code pass. Rows longer than 8192 elements take the separate launches.
+template <bool kF32, int VPL>
+static cudaError_t launch_quantize_fused(const uint4* w, int64_t N, int64_t K, const uint4* xv, int64_t M,
+                                         uint32_t* packed, float* gamma, double* partials, int8_t* xq, float* sx,
+                                         cudaStream_t s) {
+  static int per_sm[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const bool dev_ok = dev >= 0 && dev < 64;
+  int occ = dev_ok ? per_sm[dev] : 0;
+  if (!occ) {
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, quant_phase1_kernel<kF32, VPL>, kQuantThreads, 0) !=
+            cudaSuccess ||
+        occ < 1)
+      occ = 1;
+    cudaGetLastError();
+    if (dev_ok) per_sm[dev] = occ;
+  }
+  const int64_t numel = N * K;
+  const int64_t ngroups = numel / 16;
+  const int nparts = weight_partials_count(numel);
+  const int64_t per_block = (ngroups + nparts - 1) / nparts;
+  // token blocks: the resident capacity left beside the |W| blocks (at least
+  // one block per two SMs), no more than the rows need
+  const int64_t rows_blocks = (M + kQuantThreads / 32 - 1) / (kQuantThreads / 32);
+  int64_t act_blocks = static_cast<int64_t>(occ) * device_sm_count() - nparts;
+  act_blocks = std::max<int64_t>(act_blocks, device_sm_count() / 2);
+  act_blocks = std::min<int64_t>(act_blocks, rows_blocks);
+  const int nv = static_cast<int>(K / 8);
+  cudaError_t e = launch_pdl(quant_phase1_kernel<kF32, VPL>, dim3(static_cast<unsigned>(nparts + act_blocks)),
+                             dim3(kQuantThreads), 0, s, w, ngroups, per_block, nparts, partials, xv, M, nv, xq, sx);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(ternarize_pack_kernel<kF32>, dim3(code_pass_blocks(ngroups)), dim3(kQuantThreads), 0, s, w,
+                    ngroups, static_cast<const double*>(partials), nparts, numel, packed, gamma);
+}
+
 cudaError_t launch_quantize_act(const void* x, int64_t M, int64_t K, int8_t* xq, float* sx, cudaStream_t s) {
   if (M == 0) return cudaSuccess;
   const int nv = static_cast<int>(K / 8);
@@ -445,6 +575,34 @@ cudaError_t launch_quantize_act(const void* x, int64_t M, int64_t K, int8_t* xq,
       launch_pdl(act_quant_long_kernel, dim3(grid), dim3(32 * kActRowsPerBlock), 0, s, xv, M, nv, xq, sx);
     }
   }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quantize(const void* W, int w_is_f32, int64_t N, int64_t K, const void* x, int64_t M,
+                            uint8_t* packed, float* gamma, double* partials, int8_t* xq, float* sx, cudaStream_t s) {
+  const int nv = static_cast<int>(K / 8);
+  const int per_lane = (nv + 31) / 32;
+  if (M == 0 || per_lane > 32) {
+    cudaError_t e = launch_quantize_weight(W, w_is_f32, N, K, packed, gamma, partials, s);
+    if (e != cudaSuccess) return e;
+    return launch_quantize_act(x, M, K, xq, sx, s);
+  }
+  const uint4* w = static_cast<const uint4*>(W);
+  const uint4* xv = static_cast<const uint4*>(x);
+  uint32_t* out = reinterpret_cast<uint32_t*>(packed);
+  cudaError_t e = cudaSuccess;
+  switch (per_lane <= kFusedMaxVpl ? per_lane : 0) {
+#define BL_Q_CASE(n)                                                                                  \
+  case n:                                                                                             \
+    e = w_is_f32 ? launch_quantize_fused<true, n>(w, N, K, xv, M, out, gamma, partials, xq, sx, s)    \
+                 : launch_quantize_fused<false, n>(w, N, K, xv, M, out, gamma, partials, xq, sx, s); \
+    break;
+    BL_Q_CASE(0) BL_Q_CASE(1) BL_Q_CASE(2) BL_Q_CASE(3) BL_Q_CASE(4)
+#undef BL_Q_CASE
+    default:
+      break;
+  }
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

@@ -38,7 +38,7 @@ def test_version_and_status_strings():
 def test_workspace_size():
     assert b.bl_quantize_weight_workspace_size(0, 32) == 0
     assert b.bl_quantize_weight_workspace_size(256, 128) == 8 * 8       # 2048 groups -> 8 partials
-    assert b.bl_quantize_weight_workspace_size(6912, 2560) == 592 * 8   # capped
+    assert b.bl_quantize_weight_workspace_size(6912, 2560) == 296 * 8   # capped
 
 
 FAKE = ctypes.c_void_p(0x10000)        # never dereferenced: validation fails first

@@ -327,3 +327,44 @@ def test_backward_scheduled_tiles_full_compare():
     o = oracle_step(x, w, dy)
     g["acc"] = None
     check_all(g, o, N)
+
+
+@pytest.mark.parametrize("M,N,K,w_dtype", [
+    (4096, 6912, 2560, torch.bfloat16),   # rows read twice in the fused launch
+    (300, 520, 320, torch.bfloat16),      # rows in registers
+    (64, 264, 1024, torch.float32),
+    (17, 136, 96, torch.bfloat16),
+    (40, 64, 8448, torch.bfloat16),       # rows past 8192: separate launches
+    (0, 128, 256, torch.bfloat16),        # no tokens: S1 only
+])
+def test_quantize_fused_matches_separate(M, N, K, w_dtype):
+    """bl_quantize gives bit for bit what bl_quantize_weight + bl_quantize_act give."""
+    bl = _bl()
+    x, w, _ = make_inputs(max(M, 1), K, N, w_dtype=w_dtype, seed=M + N)
+    x = x[:M]
+    xd, wd = x.cuda(), w.cuda()
+    ws = torch.empty(max(bl.bl_quantize_weight_workspace_size(N, K), 16), dtype=torch.uint8, device="cuda")
+    outs = []
+    for fused in (False, True):
+        packed = torch.full((N, K // 4), 0xAA, dtype=torch.uint8, device="cuda")
+        gamma = torch.full((1,), -1.0, dtype=torch.float32, device="cuda")
+        xq = torch.full((M, K), 99, dtype=torch.int8, device="cuda")
+        sx = torch.full((M,), -1.0, dtype=torch.float32, device="cuda")
+        if fused:
+            bl.bl_quantize(wd, xd, packed, gamma, xq, sx, ws)
+        else:
+            bl.bl_quantize_weight(wd, packed, gamma, ws)
+            if M:
+                bl.bl_quantize_act(xd, xq, sx)
+        torch.cuda.synchronize()
+        assert bl.bl_get_last_error() == 0
+        outs.append([t.cpu() for t in (packed, gamma, xq, sx)])
+    for a, b in zip(*outs):
+        assert torch.equal(a, b)
+    codes, g = ref.ternarize(ref.bf16_bits_to_f32(bits(w)) if w_dtype == torch.bfloat16 else w.numpy())
+    assert outs[1][1].numpy()[0].tobytes() == np.float32(g).tobytes()
+    np.testing.assert_array_equal(outs[1][0].numpy(), ref.pack_ternary(codes))
+    if M:
+        q, s = ref.quantize_activations(ref.bf16_bits_to_f32(bits(x)))
+        np.testing.assert_array_equal(outs[1][2].numpy(), q)
+        np.testing.assert_array_equal(outs[1][3].numpy().view(np.uint32), s.view(np.uint32))
