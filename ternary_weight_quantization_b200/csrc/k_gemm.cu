@@ -87,7 +87,6 @@ __device__ __forceinline__ int rebuild_slot(int w) {
 
 constexpr int BM = 128;              // A rows per CTA; a pair covers 2 * BM
 constexpr uint32_t kTmemCols = 512;  // two accumulators at columns 0 and 256
-constexpr int kEpiStageBytes = 32 * 32 * 4;  // per epilogue warp
 constexpr int kSmemLimit = 232448;           // per-CTA dynamic shared memory on sm_100
 constexpr int kMaxPairs = 128;
 constexpr int kMaxSchedTiles = 2048;
@@ -99,9 +98,13 @@ enum class Family { Fwd, Bwd };
 template <Family F, int BN>
 struct Geo;
 
+// Epilogue staging per warp: kEpiSlots boxes of 32 x 32 bf16 (2 KB each);
+// an f32 box takes two slots.
 // Forward: reduction over k in blocks of 128 bytes; kind::i8 consumes 32 k per MMA.
 template <int BN>
 struct Geo<Family::Fwd, BN> {
+  static constexpr int kEpiSlots = 4;
+  static constexpr int kEpiScaleBytes = 256 * 4;  // s_x[m] * gamma of the tile's columns
   static constexpr int kBlockR = 128;
   static constexpr int kABytes = BM * 128;         // 128 rows x 128 int8
   static constexpr int kBBytes = (BN / 2) * 128;   // BN/2 rows x 128 int8
@@ -116,6 +119,8 @@ struct Geo<Family::Fwd, BN> {
 template <int BN>
 struct Geo<Family::Bwd, BN> {
   static_assert((BN / 2) % 64 == 0, "MN-major B needs whole 64-element chunks");
+  static constexpr int kEpiSlots = 2;
+  static constexpr int kEpiScaleBytes = 0;
   static constexpr int kBlockR = 64;
   static constexpr int kABytes = BM * 64 * 2;      // 128 x 64 bf16
   static constexpr int kBBytes = (BN / 2) * 128;   // BN/2 x 64 bf16
@@ -150,6 +155,7 @@ template <Family F, int BN>
 struct Layout {
   using G = Geo<F, BN>;
   static constexpr int kStageBytes = G::kABytes + G::kBBytes + G::kSrcBytes + G::kSxBytes;
+  static constexpr int kEpiStageBytes = G::kEpiSlots * 2048 + G::kEpiScaleBytes;  // per epilogue warp
   static constexpr int kReserve = 1024 /*base alignment*/ + kNumEpiWarps * kEpiStageBytes + 512;
   static constexpr int kS0 = (kSmemLimit - kReserve) / kStageBytes;
   static constexpr int kS = kS0 > 8 ? 8 : kS0;
@@ -460,6 +466,24 @@ __device__ __forceinline__ float epi_value(uint32_t a, float scale) {
   else return __uint_as_float(a);
 }
 
+// Largest K for which every forward accumulator (|acc| <= 127 K) is below
+// 2^22, the range of the exact 1.5 * 2^23 int -> float shifter.
+constexpr int kShifterMaxK = 33024;
+
+// {hi, lo} -> bf16x2 (round to nearest even), lo in the low half.
+__device__ __forceinline__ uint32_t cvt_bf16x2(float hi, float lo) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+__device__ __forceinline__ float4 ld_shared_f4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr)
+               : "memory");
+  return v;
+}
+
 __device__ __forceinline__ void st_shared_b16(uint32_t addr, uint16_t v) {
   asm volatile("st.shared.b16 [%0], %1;" ::"r"(addr), "h"(v) : "memory");
 }
@@ -517,12 +541,12 @@ __device__ __noinline__ void epilogue_chunk_direct(const GemmParams& p, const Op
 
 // Epilogue, one 32 x 32 chunk in registers: lane = output column i (A row),
 // r[jj] = output row j0 + jj. The common case is a bf16 box converted into
-// one of the warp's two 2 KB staging slots (used in turn) and written by one
-// TMA store. `seq` counts the warp's bf16 boxes.
-template <Op op>
+// one of the warp's kSlots 2 KB staging slots (used in turn) and written by
+// one TMA store. `seq` counts the warp's bf16 boxes.
+template <Op op, int kSlots>
 __device__ __forceinline__ void epilogue_chunk(const GemmParams& p, const OpParams& P, const CUtensorMap* out_map,
-                                               uint32_t (&r)[32], uint32_t stg, int lane, int i0, int j0,
-                                               float col_scale, float gamma, uint32_t& seq) {
+                                               uint32_t (&r)[32], uint32_t stg, uint32_t scales, int lane, int i0,
+                                               int j0, int c, float col_scale, float gamma, uint32_t& seq) {
   if (i0 >= P.rows_a || j0 >= P.rows_b) return;
   if (!P.tma_store || P.out_f32) {
     // the out-of-line paths take a copy, so that r itself stays in registers
@@ -535,16 +559,43 @@ __device__ __forceinline__ void epilogue_chunk(const GemmParams& p, const OpPara
       epilogue_chunk_f32<op>(out_map, t, stg, lane, i0, j0);
     return;
   }
-  const uint32_t slot = stg + (seq & 1u) * 2048u;
-  if (lane == 0) bulk_wait_group_read<1>();  // the box stored from this slot two chunks ago has been read
+  const uint32_t slot = stg + (seq % kSlots) * 2048u;
+  if (lane == 0) bulk_wait_group_read<kSlots - 1>();  // the box last stored from this slot has been read
   __syncwarp();
+  // values of this lane's column for the chunk's 32 rows
+  float v[32];
+  if constexpr (op == Op::Fwd) {
+    // exact int32 -> fp32 through the 1.5 * 2^23 shifter (|acc| <= 127 K < 2^22)
+    // when K allows, else the conversion instruction; then one rounding by
+    // the row's scale, read from the warp's table (broadcast loads)
+    const bool shifter = P.red <= kShifterMaxK;
 #pragma unroll
-  for (int jj = 0; jj < 32; ++jj) {
-    float scale = 0.0f;
-    if constexpr (op == Op::Fwd) scale = __shfl_sync(0xffffffffu, col_scale, jj);
-    else if constexpr (op == Op::Dx) scale = gamma;
-    const __nv_bfloat16 b = __float2bfloat16_rn(epi_value<op>(r[jj], scale));
-    st_shared_b16(slot + jj * 64 + lane * 2, *reinterpret_cast<const uint16_t*>(&b));
+    for (int u = 0; u < 8; ++u) {
+      const float4 sc = ld_shared_f4(scales + (c * 32 + 4 * u) * 4);
+      const float sv[4] = {sc.x, sc.y, sc.z, sc.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const uint32_t a = r[4 * u + e];
+        const float f = shifter ? __fsub_rn(__int_as_float(static_cast<int>(a) + 0x4B400000), 12582912.0f)
+                                : static_cast<float>(static_cast<int32_t>(a));
+        v[4 * u + e] = __fmul_rn(f, sv[e]);
+      }
+    }
+  } else {
+#pragma unroll
+    for (int jj = 0; jj < 32; ++jj) v[jj] = epi_value<op>(r[jj], gamma);
+  }
+  // lanes 2k and 2k+1 swap one value per pair of rows, so that each holds two
+  // adjacent columns of one row: one bf16x2 conversion and one 32-bit store
+  const bool odd = lane & 1;
+  const uint32_t col_bytes = static_cast<uint32_t>(lane & ~1) * 2;
+#pragma unroll
+  for (int pr = 0; pr < 16; ++pr) {
+    const float send = odd ? v[2 * pr] : v[2 * pr + 1];
+    const float recv = __shfl_xor_sync(0xffffffffu, send, 1);
+    const float lo = odd ? recv : v[2 * pr];
+    const float hi = odd ? v[2 * pr + 1] : recv;
+    st_shared_b32(slot + (2 * pr + (odd ? 1 : 0)) * 64 + col_bytes, cvt_bf16x2(hi, lo));
   }
   fence_proxy_async_smem();
   __syncwarp();
@@ -559,13 +610,24 @@ __device__ __forceinline__ void epilogue_chunk(const GemmParams& p, const OpPara
 // (rolled) iteration; each chunk's TMEM load overlaps the previous chunk's
 // conversion and store, and the buffer is handed back once the last load has
 // landed.
-template <Op op, int BN>
+template <Op op, int BN, int kSlots>
 __device__ __forceinline__ void epilogue_tile(const GemmParams& p, const OpParams& P, const CUtensorMap* out_map,
                                               uint32_t tmem_base, int buf, uint32_t stg, int lane, int q, int a0,
                                               int bp, float gamma, uint32_t tmem_empty_lead, uint32_t& seq) {
   static_assert(BN % 64 == 0, "chunks are drained in pairs");
   const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * 256;
   const int i0 = a0 + q * 32;
+  // forward: the warp's table of the tile's column scales s_x[m] * gamma
+  const uint32_t scales = stg + kSlots * 2048u;
+  if constexpr (op == Op::Fwd) {
+#pragma unroll
+    for (int c = 0; c < BN / 32; ++c) {
+      const int j = bp + c * 32 + lane;
+      st_shared_b32(scales + (c * 32 + lane) * 4, __float_as_uint(j < P.rows_b ? __fmul_rn(__ldg(p.sx + j), gamma)
+                                                                               : 0.0f));
+    }
+    __syncwarp();
+  }
   uint32_t ra[32], rb[32];
   tmem_ld_32x32b_x32(tbase, ra);
   tmem_ld_wait();
@@ -579,7 +641,7 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams& p, const OpParam
       s1 = j + 32 < P.rows_b ? __fmul_rn(__ldg(p.sx + j + 32), gamma) : 0.0f;
     }
     tmem_ld_32x32b_x32(tbase + 32 * (c + 1), rb);
-    epilogue_chunk<op>(p, P, out_map, ra, stg, lane, i0, bp + c * 32, s0, gamma, seq);
+    epilogue_chunk<op, kSlots>(p, P, out_map, ra, stg, scales, lane, i0, bp + c * 32, c, s0, gamma, seq);
     tmem_ld_wait();
     if (c + 2 < BN / 32) {
       tmem_ld_32x32b_x32(tbase + 32 * (c + 2), ra);
@@ -589,7 +651,7 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams& p, const OpParam
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(tmem_empty_lead);
     }
-    epilogue_chunk<op>(p, P, out_map, rb, stg, lane, i0, bp + (c + 1) * 32, s1, gamma, seq);
+    epilogue_chunk<op, kSlots>(p, P, out_map, rb, stg, scales, lane, i0, bp + (c + 1) * 32, c + 1, s1, gamma, seq);
     if (c + 2 < BN / 32) tmem_ld_wait();
   }
 }
@@ -803,7 +865,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   } else if (warp >= kWarpEpi0) {
     // ------------------------------------------------------------ epilogue (both CTAs)
     const int q = warp & 3;  // TMEM lane quadrant this warp may access
-    const uint32_t stg = smem_u32(smem + L::kOffEpi + (warp - kWarpEpi0) * kEpiStageBytes);
+    const uint32_t stg = smem_u32(smem + L::kOffEpi + (warp - kWarpEpi0) * L::kEpiStageBytes);
     const float gamma = p.gamma ? __ldg(p.gamma) : 1.0f;
     int buf = 0;
     uint32_t buf_phase = 0;
@@ -815,10 +877,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       if (!wait(&tmem_full[buf], buf_phase)) break;
       tc_fence_after();
       if (t.opi == 0)
-        epilogue_tile<kOp0, BN>(p, P, &map_out0, tmem_base, buf, stg, lane, q, t.a0, t.bp, gamma,
+        epilogue_tile<kOp0, BN, G::kEpiSlots>(p, P, &map_out0, tmem_base, buf, stg, lane, q, t.a0, t.bp, gamma,
                                 lead(&tmem_empty[buf]), seq);
       else if constexpr (F == Family::Bwd)
-        epilogue_tile<Op::Dw, BN>(p, P, &map_out1, tmem_base, buf, stg, lane, q, t.a0, t.bp, gamma,
+        epilogue_tile<Op::Dw, BN, G::kEpiSlots>(p, P, &map_out1, tmem_base, buf, stg, lane, q, t.a0, t.bp, gamma,
                                   lead(&tmem_empty[buf]), seq);
       if (++buf == 2) {
         buf = 0;

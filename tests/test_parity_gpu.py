@@ -116,9 +116,10 @@ def test_tiny_workload_parity():
     check_all(g, oracle_step(x, w, dy), 256, dw_f32=True)
 
 
-@pytest.mark.parametrize("M,N,K", [(33, 130, 64), (5, 7, 32), (200, 301, 256)])
+@pytest.mark.parametrize("M,N,K", [(33, 130, 64), (5, 7, 32), (200, 301, 256), (8, 64, 33056)])
 def test_forward_ragged_n(M, N, K):
-    """Forward with N not a multiple of 8 (scalar epilogue stores)."""
+    """Forward with N not a multiple of 8 (scalar epilogue stores), and with
+    K past the range of the int32 -> fp32 shifter (conversion instruction)."""
     x, w, dy = make_inputs(M, K, N, seed=7)
     check_all(run_step(x, w, dy), oracle_step(x, w, dy), N)
 
