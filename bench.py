@@ -453,7 +453,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=["up_proj", "down_proj", "tiny"], default="up_proj")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-tokens", type=int, default=512)
+    ap.add_argument("--cpu-tokens", type=int, default=4096)
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
