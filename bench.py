@@ -445,6 +445,81 @@ def run_reference(args):
 
 # ----------------------------------------------------------------- main
 
+def run_stack(args, rank, world, local_rank):
+    """Layer-stack mode: SURVEY config 4 (8 BitLinear layers alternating
+    2560 -> 6912 -> 2560, 2048 tokens). One step = the forward of every layer
+    (bl_quantize + bl_forward, only the 2-bit / INT8 state kept) and the
+    backward of every layer in reverse (bl_backward, dX feeding the layer
+    below). Reports the step time, effective TOPS and the peak device memory."""
+    import ternary_weight_quantization_b200 as bl
+    from ternary_weight_quantization_b200.stack import BitLinearStack
+    from workloads import STACKS, stack_inputs
+
+    bl.load_library()
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    M, dims = STACKS[args.stack]
+    x_cpu, ws_cpu, dy_cpu = stack_inputs(M, dims, seed=rank)
+    torch.cuda.reset_peak_memory_stats(dev)
+    base = torch.cuda.memory_allocated(dev)
+    x, dy = x_cpu.to(dev), dy_cpu.to(dev)
+    ws = [w.to(dev) for w in ws_cpu]
+    st = BitLinearStack.allocate(M, dims, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        st.forward(x, ws, stream)
+        st.backward(dy, True, stream)
+
+    for i in range(args.warmup):
+        flush.fill_(i & 0xFF)
+        flush.view(torch.int64).max()
+        step()
+    torch.cuda.synchronize(dev)
+    if bl.bl_get_last_error() != 0:
+        raise RuntimeError("device error during warm-up")
+    peak_mb = (torch.cuda.max_memory_allocated(dev) - base - flush.numel()) / 1e6
+    sampler = ClockSampler(dev.index if dev.index is not None else 0)
+    sampler.start()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        flush.view(torch.int64).max()
+        evs[i][0].record(stream)
+        step()
+        evs[i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
+    clocks = sampler.stop()
+    if bl.bl_get_last_error() != 0:
+        raise RuntimeError("device error during the timed region")
+    total = sum(e[0].elapsed_time(e[1]) for e in evs)
+    job_ms = job_time_ms(total, world, dev)
+    if rank != 0:
+        return None
+    ops_step = 6.0 * M * sum(k * n for k, n in zip(dims[:-1], dims[1:]))
+    saved = sum(L.xq.numel() + 4 * L.sx.numel() + L.w_packed.numel() + 4 for L in st.layers)
+    return {
+        "metric": "bitlinear_stack_fwd_bwd_effective_tops", "value": round(job_tops(ops_step, world, args.steps,
+                                                                                     job_ms), 2),
+        "unit": "TOPS", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(job_ms / args.steps, 5), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "int8/bf16", "data": "synthetic",
+        "config": {"workload": args.stack, "M": M, "dims": dims, "layers": len(dims) - 1,
+                   "l2": "flushed before every step (256 MiB written, then read back)",
+                   "parallelism": f"dp{world} independent replicas" if world > 1 else "single GPU"},
+        "peak_device_memory_mb": round(peak_mb, 1),
+        "saved_state_mb": round(saved / 1e6, 2),
+        "gpu_launches": 4 * (len(dims) - 1) * args.steps,
+        "clocks": clocks,
+    }
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -454,6 +529,8 @@ def main():
     ap.add_argument("--workload", choices=["up_proj", "down_proj", "tiny"], default="up_proj")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-tokens", type=int, default=4096)
+    ap.add_argument("--stack", choices=["stack8"], default=None,
+                    help="layer-stack mode (prints its own line instead of the single-layer one)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -473,7 +550,7 @@ def main():
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=torch.device("cuda", local_rank))
     try:
-        out = run_ours(args, rank, world, local_rank)
+        out = run_stack(args, rank, world, local_rank) if args.stack else run_ours(args, rank, world, local_rank)
         if rank == 0 and out is not None:
             print(json.dumps(out), flush=True)
     finally:

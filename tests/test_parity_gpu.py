@@ -369,3 +369,30 @@ def test_quantize_fused_matches_separate(M, N, K, w_dtype):
         q, s = ref.quantize_activations(ref.bf16_bits_to_f32(bits(x)))
         np.testing.assert_array_equal(outs[1][2].numpy(), q)
         np.testing.assert_array_equal(outs[1][3].numpy().view(np.uint32), s.view(np.uint32))
+
+
+@pytest.mark.parametrize("M", [1, 2, 3, 5, 8, 9, 16])
+def test_forward_few_tokens(M):
+    """Forward with few tokens on the up-projection weight (M <= 8: the
+    code-bandwidth kernel, every token-slot count; above: the tile kernel):
+    INT32 sums and y bit-exact."""
+    bl = _bl()
+    N, K = 6912, 2560
+    x, w, _ = make_inputs(M, K, 8, seed=40 + M)
+    _, w, _ = make_inputs(8, K, N, seed=41)
+    bufs = bl.StepBuffers.allocate(M, N, K)
+    acc = torch.empty((M, N), dtype=torch.int32, device="cuda")
+    bl.bl_quantize_weight(w.cuda(), bufs.w_packed, bufs.gamma, bufs.workspace)
+    bl.bl_quantize_act(x.cuda(), bufs.xq, bufs.sx)
+    bl.bl_forward(bufs.xq, bufs.sx, bufs.w_packed, bufs.gamma, bufs.y, acc)
+    y2 = torch.empty_like(bufs.y)
+    bl.bl_forward(bufs.xq, bufs.sx, bufs.w_packed, bufs.gamma, y2)  # without the debug output
+    torch.cuda.synchronize()
+    assert bl.bl_get_last_error() == 0
+    codes, gamma = ref.ternarize(ref.bf16_bits_to_f32(bits(w)))
+    q, sx = ref.quantize_activations(ref.bf16_bits_to_f32(bits(x)))
+    acc_o = ref.forward_accumulate(q, codes)
+    np.testing.assert_array_equal(acc.cpu().numpy(), acc_o)
+    y_o = ref.round_to_bf16_bits(ref.forward_output(acc_o, sx, gamma))
+    np.testing.assert_array_equal(bits(bufs.y), y_o)
+    np.testing.assert_array_equal(bits(y2), y_o)

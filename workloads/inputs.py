@@ -22,7 +22,7 @@ from dataclasses import dataclass
 
 import torch
 
-__all__ = ["Workload", "WORKLOADS", "make_inputs", "kaiming_uniform_bound"]
+__all__ = ["Workload", "WORKLOADS", "STACKS", "make_inputs", "stack_inputs", "kaiming_uniform_bound"]
 
 
 @dataclass(frozen=True)
@@ -40,6 +40,13 @@ WORKLOADS = {
     "tiny": Workload("tiny", 32, 128, 256, torch.float32, "normal0.02"),
     "up_proj": Workload("up_proj", 4096, 2560, 6912, torch.bfloat16, "kaiming"),
     "down_proj": Workload("down_proj", 2048, 6912, 2560, torch.bfloat16, "kaiming", True),
+}
+
+
+# Layer stacks (SURVEY config 4): 8 BitLinear layers alternating
+# 2560 -> 6912 -> 2560 ... over x [4, 512, 2560].
+STACKS = {
+    "stack8": (2048, [2560, 6912] * 4 + [2560]),
 }
 
 
@@ -83,3 +90,16 @@ def workload_inputs(name: str, seed: int = 0):
 
 
 __all__.append("workload_inputs")
+
+
+def stack_inputs(M: int, dims, seed: int = 0):
+    """(x [M, dims[0]] bf16, [W_l [dims[l+1], dims[l]] bf16 kaiming-uniform],
+    dY [M, dims[-1]] bf16) on the CPU; W_l from seed + 100 + l."""
+    x = torch.randn(M, dims[0], generator=_gen(seed), dtype=torch.float32)
+    ws = []
+    for l, (K, N) in enumerate(zip(dims[:-1], dims[1:])):
+        b = kaiming_uniform_bound(K)
+        w = (torch.rand(N, K, generator=_gen(seed + 100 + l), dtype=torch.float32) * 2.0 - 1.0) * b
+        ws.append(w.to(torch.bfloat16).contiguous())
+    dy = torch.randn(M, dims[-1], generator=_gen(seed + 1), dtype=torch.float32)
+    return x.to(torch.bfloat16).contiguous(), ws, dy.to(torch.bfloat16).contiguous()
