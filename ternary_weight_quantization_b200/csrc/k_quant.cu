@@ -359,11 +359,13 @@ __device__ __forceinline__ void act_rows_two_pass(const uint4* __restrict__ x, i
   for (; m < M; m += stride) {
     const uint4* row = x + m * nv;
     float amax = 0.0f;
+#pragma unroll 4
     for (int j = lane; j < nv; j += 32) amax = absmax8(__ldg(row + j), amax);
     const float a = fmaxf(warp_max(amax), 1e-5f);
     const float inv = __fdiv_rn(127.0f, a);
     if (lane == 0) sx[m] = __fdiv_rn(a, 127.0f);
     uint2* out = reinterpret_cast<uint2*>(xq + m * static_cast<int64_t>(nv) * 8);
+#pragma unroll 4
     for (int j = lane; j < nv; j += 32) out[j] = quant8(__ldg(row + j), inv);
   }
 }
