@@ -174,15 +174,41 @@ __global__ void __launch_bounds__(kQuantThreads) absmean_partials_kernel(const u
 // thr the largest float <= T, that is |w| > thr: one compare, no division.
 template <bool kF32>
 __device__ __forceinline__ uint32_t pack_group(const Group<kF32>& a, float thr) {
-  uint32_t word = 0;
+  if constexpr (!kF32) {
+    // bf16: for a 15-bit magnitude b (the bf16 bits with the sign cleared)
+    // and thr > 0, |w| > thr <=> (b << 16) > bits(thr) <=> b > bits(thr) >> 16,
+    // so both halves of a word are compared with one subtraction: per half,
+    // 0x8000 + tb - b keeps bit 15 clear exactly when b > tb (no borrow
+    // crosses the halves since b <= 0x7FFF). Field bit 0 = nonzero, bit 1 =
+    // nonzero and negative.
+    const uint32_t tb = __float_as_uint(thr) >> 16;
+    const uint32_t bias = (tb | (tb << 16)) + 0x80008000u;
+    const uint32_t w[8] = {a.v[0].x, a.v[0].y, a.v[0].z, a.v[0].w, a.v[1].x, a.v[1].y, a.v[1].z, a.v[1].w};
+    uint32_t acc[2] = {0u, 0u};
 #pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    const float w = a.elem(i);
-    const uint32_t nz = fabsf(w) > thr ? 1u : 0u;
-    const uint32_t neg = __float_as_uint(w) >> 31;
-    word |= (nz * (1u | (neg << 1))) << (2 * i);  // 00 = 0, 01 = +1, 11 = -1
+    for (int j = 0; j < 8; ++j) {
+      const uint32_t nz = ~(bias - (w[j] & 0x7FFF7FFFu)) & 0x80008000u;  // bits 15, 31
+      const uint32_t nn = nz & w[j];
+      // word j of a four-word half: low element's field to bits 4j', 4j'+1,
+      // high element's to 16 + 4j', 17 + 4j' (j' = j % 4)
+      const int sh = 4 * (j & 3);
+      acc[j >> 2] |= (nz >> (15 - sh)) | (nn >> (14 - sh));
+    }
+    // high elements' fields from bits 16.. down to 4j' + 2
+    const uint32_t lo = (acc[0] & 0x3333u) | ((acc[0] >> 14) & 0xCCCCu);
+    const uint32_t hi = (acc[1] & 0x3333u) | ((acc[1] >> 14) & 0xCCCCu);
+    return lo | (hi << 16);
+  } else {
+    uint32_t word = 0;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const float w = a.elem(i);
+      const uint32_t nz = fabsf(w) > thr ? 1u : 0u;
+      const uint32_t neg = __float_as_uint(w) >> 31;
+      word |= (nz * (1u | (neg << 1))) << (2 * i);  // 00 = 0, 01 = +1, 11 = -1
+    }
+    return word;
   }
-  return word;
 }
 
 template <bool kF32>
