@@ -1,6 +1,7 @@
-// Device primitives for sm_100a: mbarriers with bounded waits, TMA and
-// cp.async loads, and the tcgen05 (5th-generation tensor core) instructions
-// used by the GEMM kernels. Inline PTX only; no library kernels.
+// Device primitives for sm_100a: mbarriers with bounded waits, TMA loads and
+// stores, cp.async loads, programmatic-launch control, and the tcgen05
+// (5th-generation tensor core) instructions used by the GEMM kernels. Inline
+// PTX only; no library kernels.
 #pragma once
 
 #include <cstdint>

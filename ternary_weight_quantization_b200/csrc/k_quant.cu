@@ -1,8 +1,13 @@
 // S1 and S2 of the BitLinear hot path on sm_100a: absmean ternarisation with
 // 2-bit packing, and per-token absmax INT8 activation quantisation.
 //
-// Both are HBM-bound streaming passes: 16-byte vector loads, one pass over
-// the data per output, no intermediate tensors in device memory.
+// Both are HBM-bound streaming passes with 16-byte vector loads and no
+// intermediate tensors in device memory. S1 needs gamma before any code, so
+// it is two passes over W: pass A (fp64 partial sums of |W|) and the code
+// pass (gamma from the partials, codes packed 4 per byte). bl_quantize runs
+// pass A and S2 in one launch (quant_phase1_kernel: the two are independent)
+// and then the code pass; bl_quantize_weight and bl_quantize_act launch the
+// same arithmetic separately.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
