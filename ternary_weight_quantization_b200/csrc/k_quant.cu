@@ -216,18 +216,17 @@ __device__ __forceinline__ uint32_t pack_group(const Group<kF32>& a, float thr) 
   }
 }
 
+// Code-pass block `block` of `nblocks`: threads stride over the groups
+// (consecutive threads, consecutive groups), two groups per batch, the next
+// batch loaded while the current one is packed; the first batch is loaded
+// before the wait for pass A.
 template <bool kF32>
-__global__ void __launch_bounds__(kQuantThreads, kF32 ? 2 : 4) ternarize_pack_kernel(const uint4* __restrict__ W,
-                                                                          int64_t ngroups,
-                                                                          const double* __restrict__ partials,
-                                                                          int nparts, int64_t numel,
-                                                                          uint32_t* __restrict__ packed,
-                                                                          float* __restrict__ gamma_out) {
-  // Threads stride over the groups (consecutive threads, consecutive groups),
-  // two groups per batch, the next batch loaded while the current one is
-  // packed; the first batch is loaded before the wait.
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * kQuantThreads;
-  int64_t g = static_cast<int64_t>(blockIdx.x) * kQuantThreads + threadIdx.x;
+__device__ __forceinline__ void code_pass_block(const uint4* __restrict__ W, int64_t ngroups,
+                                                const double* __restrict__ partials, int nparts, int64_t numel,
+                                                uint32_t* __restrict__ packed, float* __restrict__ gamma_out,
+                                                int64_t block, int64_t nblocks) {
+  const int64_t stride = nblocks * kQuantThreads;
+  int64_t g = block * kQuantThreads + threadIdx.x;
   Group<kF32> a[2];
 #pragma unroll
   for (int u = 0; u < 2; ++u)
@@ -251,7 +250,7 @@ __global__ void __launch_bounds__(kQuantThreads, kF32 ? 2 : 4) ternarize_pack_ke
     const double mean = __ddiv_rn(sum, static_cast<double>(numel));
     const float gamma = fmaxf(__double2float_rn(mean), 1e-5f);
     s_thr = __double2float_rd(__dmul_rn(static_cast<double>(gamma), 0.5 + 0x1p-25));
-    if (blockIdx.x == 0) *gamma_out = gamma;
+    if (block == 0) *gamma_out = gamma;
   }
   __syncthreads();
   const float thr = s_thr;
@@ -268,6 +267,16 @@ __global__ void __launch_bounds__(kQuantThreads, kF32 ? 2 : 4) ternarize_pack_ke
 #pragma unroll
     for (int u = 0; u < 2; ++u) a[u] = b[u];
   }
+}
+
+template <bool kF32>
+__global__ void __launch_bounds__(kQuantThreads, kF32 ? 2 : 4) ternarize_pack_kernel(const uint4* __restrict__ W,
+                                                                          int64_t ngroups,
+                                                                          const double* __restrict__ partials,
+                                                                          int nparts, int64_t numel,
+                                                                          uint32_t* __restrict__ packed,
+                                                                          float* __restrict__ gamma_out) {
+  code_pass_block<kF32>(W, ngroups, partials, nparts, numel, packed, gamma_out, blockIdx.x, gridDim.x);
 }
 
 // ---------------------------------------------------------------- S2
@@ -401,35 +410,45 @@ __device__ __forceinline__ void act_rows_two_pass(const uint4* __restrict__ x, i
   }
 }
 
-// S1 pass A and S2 in one launch (bl_quantize): blocks 0 .. nparts-1 sum |W|
-// over their ranges (the same partial sums absmean_partials_kernel writes);
-// the other blocks' warps quantise tokens. The two kinds of work are
-// independent, so their memory traffic and arithmetic overlap. Four blocks
-// fit on an SM with bf16 weights (64 registers; two with f32 weights): rows of
-// up to 1024 elements stay in registers (VPL <= 4), longer ones are read
-// twice (VPL = 0).
+// bl_quantize, launch 1: pass A alone (two groups loaded per batch, so that
+// it fits beside two more 256-thread blocks on an SM).
+template <bool kF32>
+__global__ void __launch_bounds__(kQuantThreads, kF32 ? 2 : 4) quant_pass_a_kernel(const uint4* __restrict__ W,
+                                                                        int64_t ngroups, int64_t per_block,
+                                                                        double* __restrict__ partials) {
+  pdl_wait_primary();
+  pdl_launch_dependents();  // launch 2 may start beside this pass
+  absmean_block<kF32, 2>(W, ngroups, per_block, blockIdx.x, partials);
+}
+
+// bl_quantize, launch 2 (a programmatic dependent of launch 1): blocks
+// 0 .. act_blocks-1 quantise tokens (S2); the rest run the code pass. The token
+// blocks do not wait for launch 1: x was complete before launch 1 passed its
+// own dependency wait (and launch 2 only starts after that point), and launch
+// 1 neither reads xq / s_x nor writes x. So they run beside pass A, and the
+// code-pass blocks -- which do wait -- follow; since they wait, this grid
+// still completes only after launch 1 has. Rows of up to 1024 elements stay
+// in registers (VPL <= 4), longer ones are read twice (VPL = 0).
 constexpr int kFusedMaxVpl = 4;
 
 template <bool kF32, int VPL>
-__global__ void __launch_bounds__(kQuantThreads, kF32 ? 2 : 4) quant_phase1_kernel(const uint4* __restrict__ W,
-                                                                        int64_t ngroups, int64_t per_block,
-                                                                        int nparts, double* __restrict__ partials,
-                                                                        const uint4* __restrict__ x, int64_t M,
-                                                                        int nv, int8_t* __restrict__ xq,
-                                                                        float* __restrict__ sx) {
-  pdl_wait_primary();
-  pdl_launch_dependents();
-  if (static_cast<int>(blockIdx.x) < nparts) {
-    absmean_block<kF32, 2>(W, ngroups, per_block, blockIdx.x, partials);
+__global__ void __launch_bounds__(kQuantThreads, kF32 ? 2 : 4) quant_phase2_kernel(
+    const uint4* __restrict__ W, int64_t ngroups, const double* __restrict__ partials, int nparts, int64_t numel,
+    uint32_t* __restrict__ packed, float* __restrict__ gamma_out, const uint4* __restrict__ x, int64_t M, int nv,
+    int8_t* __restrict__ xq, float* __restrict__ sx, int act_blocks) {
+  if (static_cast<int>(blockIdx.x) < act_blocks) {
+    pdl_launch_dependents();
+    constexpr int kWarps = kQuantThreads / 32;
+    const int64_t m = static_cast<int64_t>(blockIdx.x) * kWarps + (threadIdx.x >> 5);
+    const int64_t stride = static_cast<int64_t>(act_blocks) * kWarps;
+    if constexpr (VPL > 0)
+      act_rows<VPL, false>(x, M, nv, xq, sx, m, stride);
+    else
+      act_rows_two_pass(x, M, nv, xq, sx, m, stride);
     return;
   }
-  constexpr int kWarps = kQuantThreads / 32;
-  const int64_t m = static_cast<int64_t>(blockIdx.x - nparts) * kWarps + (threadIdx.x >> 5);
-  const int64_t stride = static_cast<int64_t>(gridDim.x - nparts) * kWarps;
-  if constexpr (VPL > 0)
-    act_rows<VPL, false>(x, M, nv, xq, sx, m, stride);
-  else
-    act_rows_two_pass(x, M, nv, xq, sx, m, stride);
+  code_pass_block<kF32>(W, ngroups, partials, nparts, numel, packed, gamma_out, blockIdx.x - act_blocks,
+                        gridDim.x - act_blocks);
 }
 
 // Rows longer than 8192 elements: absmax pass, then a second read (from L2).
@@ -549,41 +568,28 @@ static void launch_act(const uint4* xv, int64_t M, int nv, int8_t* xq, float* sx
   launch_pdl(act_quant_kernel<VPL, kPrefetch>, dim3(grid), dim3(32 * kActRowsPerBlock), 0, s, xv, M, nv, xq, sx);
 }
 
-// bl_quantize: S1 pass A and S2 in one launch (quant_phase1_kernel), then the
-// code pass. Rows longer than 8192 elements take the separate launches.
+// bl_quantize: pass A (quant_pass_a_kernel), then the token blocks and the
+// code pass in one grid (quant_phase2_kernel). Rows longer than 8192
+// elements take the separate launches.
 template <bool kF32, int VPL>
 static cudaError_t launch_quantize_fused(const uint4* w, int64_t N, int64_t K, const uint4* xv, int64_t M,
                                          uint32_t* packed, float* gamma, double* partials, int8_t* xq, float* sx,
                                          cudaStream_t s) {
-  static int per_sm[64] = {};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  const bool dev_ok = dev >= 0 && dev < 64;
-  int occ = dev_ok ? per_sm[dev] : 0;
-  if (!occ) {
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, quant_phase1_kernel<kF32, VPL>, kQuantThreads, 0) !=
-            cudaSuccess ||
-        occ < 1)
-      occ = 1;
-    cudaGetLastError();
-    if (dev_ok) per_sm[dev] = occ;
-  }
   const int64_t numel = N * K;
   const int64_t ngroups = numel / 16;
   const int nparts = weight_partials_count(numel);
   const int64_t per_block = (ngroups + nparts - 1) / nparts;
-  // token blocks: the resident capacity left beside the |W| blocks (at least
-  // one block per two SMs), no more than the rows need
+  // token blocks: two per SM beside pass A, no more than the rows need
   const int64_t rows_blocks = (M + kQuantThreads / 32 - 1) / (kQuantThreads / 32);
-  int64_t act_blocks = static_cast<int64_t>(occ) * device_sm_count() - nparts;
-  act_blocks = std::max<int64_t>(act_blocks, device_sm_count() / 2);
-  act_blocks = std::min<int64_t>(act_blocks, rows_blocks);
+  const int64_t act_blocks = std::min<int64_t>(static_cast<int64_t>(2) * device_sm_count(), rows_blocks);
+  const int64_t code_blocks = code_pass_blocks(ngroups);
   const int nv = static_cast<int>(K / 8);
-  cudaError_t e = launch_pdl(quant_phase1_kernel<kF32, VPL>, dim3(static_cast<unsigned>(nparts + act_blocks)),
-                             dim3(kQuantThreads), 0, s, w, ngroups, per_block, nparts, partials, xv, M, nv, xq, sx);
+  cudaError_t e = launch_pdl(quant_pass_a_kernel<kF32>, dim3(static_cast<unsigned>(nparts)), dim3(kQuantThreads), 0,
+                             s, w, ngroups, per_block, partials);
   if (e != cudaSuccess) return e;
-  return launch_pdl(ternarize_pack_kernel<kF32>, dim3(code_pass_blocks(ngroups)), dim3(kQuantThreads), 0, s, w,
-                    ngroups, static_cast<const double*>(partials), nparts, numel, packed, gamma);
+  return launch_pdl(quant_phase2_kernel<kF32, VPL>, dim3(static_cast<unsigned>(act_blocks + code_blocks)),
+                    dim3(kQuantThreads), 0, s, w, ngroups, static_cast<const double*>(partials), nparts, numel, packed,
+                    gamma, xv, M, nv, xq, sx, static_cast<int>(act_blocks));
 }
 
 cudaError_t launch_quantize_act(const void* x, int64_t M, int64_t K, int8_t* xq, float* sx, cudaStream_t s) {
