@@ -525,6 +525,60 @@ def run_stack(args, rank, world, local_rank):
     }
 
 
+def run_few_tokens(args, rank, world, local_rank):
+    """Few-token mode: the forward alone at M in --few-tokens on the
+    up-projection weight (N 6912, K 2560). With a handful of tokens it is
+    bound by reading the packed codes once, so the line reports achieved
+    HBM GB/s (codes + q + s_x read, y written) against the measured copy
+    bandwidth, per M."""
+    import ternary_weight_quantization_b200 as bl
+    from workloads import make_inputs
+
+    bl.load_library()
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    N, K = 6912, 2560
+    _, w, _ = make_inputs(8, K, N, seed=rank)
+    packed = torch.empty((N, K // 4), dtype=torch.uint8, device=dev)
+    gamma = torch.empty(1, dtype=torch.float32, device=dev)
+    ws = torch.empty(max(bl.bl_quantize_weight_workspace_size(N, K), 16), dtype=torch.uint8, device=dev)
+    bl.bl_quantize_weight(w.to(dev), packed, gamma, ws)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    peaks, peak_src = load_peaks()
+    rows = {}
+    for M in [int(v) for v in args.few_tokens.split(",")]:
+        x, _, _ = make_inputs(M, K, 8, seed=rank + M)
+        xq = torch.empty((M, K), dtype=torch.int8, device=dev)
+        sx = torch.empty(M, dtype=torch.float32, device=dev)
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        bl.bl_quantize_act(x.to(dev), xq, sx)
+        times = []
+        for i in range(args.warmup + args.steps):
+            flush.fill_(i & 0xFF)
+            flush.view(torch.int64).max()
+            s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s.record()
+            bl.bl_forward(xq, sx, packed, gamma, y)
+            e.record()
+            torch.cuda.synchronize(dev)
+            if i >= args.warmup:
+                times.append(s.elapsed_time(e))
+        ms = sum(times) / len(times)
+        nbytes = N * K // 4 + M * K + 4 * M + 4 + M * N * 2
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        rows[str(M)] = {"ms": round(ms, 5), "bytes": nbytes, "achieved_gbs": round(gbs, 1),
+                        "frac": round(gbs / peaks["hbm_gbs"], 4)}
+    if bl.bl_get_last_error() != 0:
+        raise RuntimeError("device error")
+    if rank != 0:
+        return None
+    return {"metric": "bitlinear_forward_few_tokens_gbs", "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "higher_is_better": True, "dtype": "int8", "data": "synthetic",
+            "config": {"workload": "up_proj weight, forward only", "N": N, "K": K,
+                       "l2": "flushed before every launch (256 MiB written, then read back)"},
+            "peak_gbs": peaks["hbm_gbs"], "peak_source": f"{peak_src} hbm copy", "by_tokens": rows}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -536,6 +590,8 @@ def main():
     ap.add_argument("--cpu-tokens", type=int, default=4096)
     ap.add_argument("--stack", choices=["stack8"], default=None,
                     help="layer-stack mode (prints its own line instead of the single-layer one)")
+    ap.add_argument("--few-tokens", default=None,
+                    help="forward-only mode at these token counts, e.g. 1,8,16 (prints its own line)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -555,7 +611,12 @@ def main():
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=torch.device("cuda", local_rank))
     try:
-        out = run_stack(args, rank, world, local_rank) if args.stack else run_ours(args, rank, world, local_rank)
+        if args.stack:
+            out = run_stack(args, rank, world, local_rank)
+        elif args.few_tokens:
+            out = run_few_tokens(args, rank, world, local_rank)
+        else:
+            out = run_ours(args, rank, world, local_rank)
         if rank == 0 and out is not None:
             print(json.dumps(out), flush=True)
     finally:
