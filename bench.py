@@ -174,7 +174,7 @@ def job_tops(ops_per_rank_step: float, world: int, steps: int, job_ms: float) ->
 # ----------------------------------------------------------------- our arm
 
 STAGES = ["quantize", "forward", "backward"]
-LAUNCHES_PER_STEP = 4  # S1 pass A with S2, S1 pass B, S3, S4 (dX and dW in one launch)
+LAUNCHES_PER_STEP = 4  # S1 pass A; S2 with the S1 code pass; S3; S4 (dX and dW in one launch)
 
 
 def stage_work(M, N, K, w_bytes):

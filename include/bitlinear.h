@@ -146,8 +146,8 @@ bl_status bl_quantize_act(const void* x, int64_t M, int64_t K,
 /*
  * S1 + S2 in one call: the same outputs as bl_quantize_weight(W, ...) followed
  * by bl_quantize_act(x, ...), bit for bit. The two steps are independent, so
- * the |W| partial sums of S1 and the whole of S2 run in one launch and their
- * memory traffic overlaps; S1's code pass follows. (The pages run the two
+ * S2 runs beside the |W| partial sums of S1 and their memory traffic
+ * overlaps; S1's code pass follows in S2's launch. (The pages run the two
  * quantisers one after the other; this is a scheduling choice only.)
  *
  * Arguments: those of bl_quantize_weight and bl_quantize_act. M == 0 skips

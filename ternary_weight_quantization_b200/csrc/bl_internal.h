@@ -31,7 +31,7 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 // (a fixed function of numel, so the reduction order never depends on the GPU).
 int weight_partials_count(int64_t numel);
 
-// Pass A (|W| partial sums) + pass B (gamma, codes, packing).
+// Pass A (|W| partial sums) + the code pass (gamma, codes, packing).
 // `partials` holds weight_partials_count(N*K) doubles.
 cudaError_t launch_quantize_weight(const void* W, int w_is_f32, int64_t N, int64_t K, uint8_t* packed,
                                    float* gamma, double* partials, cudaStream_t s);
@@ -45,8 +45,9 @@ size_t noalloc_scratch_bytes();
 // ---- S2: per-token absmax INT8
 cudaError_t launch_quantize_act(const void* x, int64_t M, int64_t K, int8_t* xq, float* sx, cudaStream_t s);
 
-// ---- S1 + S2 together (bl_quantize): pass A and the activation quantisation
-// in one launch, then pass B. `partials` as for launch_quantize_weight.
+// ---- S1 + S2 together (bl_quantize): pass A, then one grid holding the
+// activation quantisation (started beside pass A) and the code pass.
+// `partials` as for launch_quantize_weight.
 cudaError_t launch_quantize(const void* W, int w_is_f32, int64_t N, int64_t K, const void* x, int64_t M,
                             uint8_t* packed, float* gamma, double* partials, int8_t* xq, float* sx, cudaStream_t s);
 

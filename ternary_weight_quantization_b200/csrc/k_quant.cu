@@ -165,7 +165,7 @@ __global__ void __launch_bounds__(kQuantThreads) absmean_partials_kernel(const u
   absmean_block<kF32, 4>(W, ngroups, per_block, blockIdx.x, partials);
 }
 
-// ---------------------------------------------------------------- S1 pass B
+// ---------------------------------------------------------------- S1 code pass
 // Launched as a programmatic dependent of pass A: each thread first loads its
 // first groups of W (pass A only started after W's producer finished, and it
 // does not write W), then waits for pass A,
