@@ -235,20 +235,23 @@ __device__ __forceinline__ TileInfo decode_tile(const GemmParams& p, int tile, u
 
 // ---------------------------------------------------------------- rebuild helpers
 
-// 8 two-bit fields (16 bits) -> nibble i holds field i.
-__device__ __forceinline__ uint32_t spread_fields8(uint32_t h) {
-  uint32_t x = h & 0xFFFFu;
-  x = (x | (x << 8)) & 0x00FF00FFu;
+// Two bytes of four 2-bit fields each, already placed in bytes 0 and 2 of x
+// -> nibble i holds field i.
+__device__ __forceinline__ uint32_t spread_fields8(uint32_t x) {
   x = (x | (x << 4)) & 0x0F0F0F0Fu;
   x = (x | (x << 2)) & 0x33333333u;
   return x;
 }
 
-// 16 packed codes (one 32-bit word) -> 16 int8 codes.
+// 16 packed codes (one 32-bit word) -> 16 int8 codes. One byte permutation
+// places each byte pair of w in bytes 0 and 2 (the first spreading step),
+// two shift/mask steps spread the fields to nibbles, and a byte permutation
+// per four codes looks each nibble up in a 4-entry table. The rebuild of the
+// forward operand is ALU-bound on its SM sub-partitions, so every step counts.
 __device__ __forceinline__ uint4 codes16_to_s8(uint32_t w) {
   constexpr uint32_t kTable = 0xFFFE0100u;  // field 0 -> 0, 1 -> +1, 2 -> -2 (unused), 3 -> -1
-  const uint32_t lo = spread_fields8(w);
-  const uint32_t hi = spread_fields8(w >> 16);
+  const uint32_t lo = spread_fields8(__byte_perm(w, 0u, 0x4140));  // bytes 0, 1 of w
+  const uint32_t hi = spread_fields8(__byte_perm(w, 0u, 0x4342));  // bytes 2, 3 of w
   uint4 r;
   r.x = __byte_perm(kTable, 0u, lo & 0xFFFFu);
   r.y = __byte_perm(kTable, 0u, lo >> 16);
@@ -482,10 +485,6 @@ __device__ __forceinline__ float4 ld_shared_f4(uint32_t addr) {
   asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr)
                : "memory");
   return v;
-}
-
-__device__ __forceinline__ void st_shared_b16(uint32_t addr, uint16_t v) {
-  asm volatile("st.shared.b16 [%0], %1;" ::"r"(addr), "h"(v) : "memory");
 }
 
 __device__ __forceinline__ void st_shared_b32(uint32_t addr, uint32_t v) {

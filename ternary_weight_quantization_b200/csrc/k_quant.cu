@@ -74,8 +74,31 @@ __device__ __forceinline__ double normal_abs_to_f64(uint32_t b32) {
 __device__ __forceinline__ bool is_subnormal(uint32_t b32) { return b32 - 1u < 0x007FFFFFu; }
 
 // acc + sum of |element| over one group, in element order.
+// bf16 groups whose 16 magnitudes all have a nonzero exponent field (no zero,
+// no subnormal) take a short path: one packed 16-bit minimum per word finds
+// them, and each fp64 high word is the 15-bit magnitude shifted into place
+// plus the re-biased exponent offset. Other groups, and fp32 groups, take the
+// per-element path below. Both give the same fp64 values in the same order.
 template <bool kF32>
 __device__ __forceinline__ double add_group(double acc, const Group<kF32>& a) {
+  if constexpr (!kF32) {
+    const uint32_t w[8] = {a.v[0].x, a.v[0].y, a.v[0].z, a.v[0].w, a.v[1].x, a.v[1].y, a.v[1].z, a.v[1].w};
+    uint32_t mn = 0xFFFFFFFFu;  // per half: smallest 15-bit magnitude
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const uint32_t m = w[j] & 0x7FFF7FFFu;
+      asm("min.u16x2 %0, %0, %1;" : "+r"(mn) : "r"(m));
+    }
+    if (min(mn << 16, mn & 0xFFFF0000u) >= 0x00800000u) {
+      // element 2j is the low half of word j, element 2j + 1 the high half
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        acc = __dadd_rn(acc, __hiloint2double(static_cast<int>(((w[j] & 0x7FFFu) << 13) + 0x38000000u), 0));
+        acc = __dadd_rn(acc, __hiloint2double(static_cast<int>(((w[j] & 0x7FFF0000u) >> 3) + 0x38000000u), 0));
+      }
+      return acc;
+    }
+  }
   bool sub = false;
 #pragma unroll
   for (int i = 0; i < 16; ++i) sub |= is_subnormal(abs_bits(a.elem(i)));
@@ -305,17 +328,25 @@ __device__ __forceinline__ uint2 quant8(const uint4& v, float inv) {
   return r;
 }
 
-__device__ __forceinline__ float absmax8(const uint4& v, float m) {
-  m = fmaxf(m, fabsf(bf16_lo(v.x)));
-  m = fmaxf(m, fabsf(bf16_hi(v.x)));
-  m = fmaxf(m, fabsf(bf16_lo(v.y)));
-  m = fmaxf(m, fabsf(bf16_hi(v.y)));
-  m = fmaxf(m, fabsf(bf16_lo(v.z)));
-  m = fmaxf(m, fabsf(bf16_hi(v.z)));
-  m = fmaxf(m, fabsf(bf16_lo(v.w)));
-  m = fmaxf(m, fabsf(bf16_hi(v.w)));
+// Running maximum of the 15-bit magnitudes of 8 bf16 values, per 16-bit
+// half of `m`. For finite values the magnitude bit patterns order like the
+// magnitudes, so this is |x|'s maximum without unpacking to fp32 (which also
+// keeps a row's unpacked values from staying live until the quantisation).
+__device__ __forceinline__ uint32_t max_mag_u16x2(uint32_t m, uint32_t w) {
+  asm("max.u16x2 %0, %0, %1;" : "+r"(m) : "r"(w & 0x7FFF7FFFu));
   return m;
 }
+
+__device__ __forceinline__ uint32_t absmax8(const uint4& v, uint32_t m) {
+  m = max_mag_u16x2(m, v.x);
+  m = max_mag_u16x2(m, v.y);
+  m = max_mag_u16x2(m, v.z);
+  m = max_mag_u16x2(m, v.w);
+  return m;
+}
+
+// The larger of the two halves as an fp32 value.
+__device__ __forceinline__ float absmax_value(uint32_t m) { return __uint_as_float(max(m & 0xFFFFu, m >> 16) << 16); }
 
 __device__ __forceinline__ float warp_max(float m) {
 #pragma unroll
@@ -325,30 +356,28 @@ __device__ __forceinline__ float warp_max(float m) {
 
 constexpr int kActRowsPerBlock = 4;
 
+// VPL = ceil(nv / 32), so only the last vector of a lane can lie past the row.
 template <int VPL>
 __device__ __forceinline__ void load_row(const uint4* __restrict__ row, int nv, int lane, uint4 (&v)[VPL]) {
+  const uint4* p = row + lane;
 #pragma unroll
-  for (int i = 0; i < VPL; ++i) {
-    const int j = lane + 32 * i;
-    v[i] = j < nv ? __ldg(row + j) : make_uint4(0u, 0u, 0u, 0u);
-  }
+  for (int i = 0; i < VPL; ++i)
+    v[i] = (i < VPL - 1 || lane + 32 * i < nv) ? __ldg(p + 32 * i) : make_uint4(0u, 0u, 0u, 0u);
 }
 
 template <int VPL>
 __device__ __forceinline__ void quant_row(const uint4 (&v)[VPL], int nv, int lane, int64_t m,
                                           int8_t* __restrict__ xq, float* __restrict__ sx) {
-  float amax = 0.0f;
+  uint32_t mx = 0u;
 #pragma unroll
-  for (int i = 0; i < VPL; ++i) amax = absmax8(v[i], amax);
-  const float a = fmaxf(warp_max(amax), 1e-5f);
+  for (int i = 0; i < VPL; ++i) mx = absmax8(v[i], mx);
+  const float a = fmaxf(warp_max(absmax_value(mx)), 1e-5f);
   const float inv = __fdiv_rn(127.0f, a);
   if (lane == 0) sx[m] = __fdiv_rn(a, 127.0f);
-  uint2* out = reinterpret_cast<uint2*>(xq + m * static_cast<int64_t>(nv) * 8);
+  uint2* out = reinterpret_cast<uint2*>(xq + m * static_cast<int64_t>(nv) * 8) + lane;
 #pragma unroll
-  for (int i = 0; i < VPL; ++i) {
-    const int j = lane + 32 * i;
-    if (j < nv) out[j] = quant8(v[i], inv);
-  }
+  for (int i = 0; i < VPL; ++i)
+    if (i < VPL - 1 || lane + 32 * i < nv) out[32 * i] = quant8(v[i], inv);
 }
 
 // Warps stride over rows (first row m, then m + stride, ...); with short rows
@@ -398,10 +427,10 @@ __device__ __forceinline__ void act_rows_two_pass(const uint4* __restrict__ x, i
   const int lane = threadIdx.x & 31;
   for (; m < M; m += stride) {
     const uint4* row = x + m * nv;
-    float amax = 0.0f;
+    uint32_t mx = 0u;
 #pragma unroll 4
-    for (int j = lane; j < nv; j += 32) amax = absmax8(__ldg(row + j), amax);
-    const float a = fmaxf(warp_max(amax), 1e-5f);
+    for (int j = lane; j < nv; j += 32) mx = absmax8(__ldg(row + j), mx);
+    const float a = fmaxf(warp_max(absmax_value(mx)), 1e-5f);
     const float inv = __fdiv_rn(127.0f, a);
     if (lane == 0) sx[m] = __fdiv_rn(a, 127.0f);
     uint2* out = reinterpret_cast<uint2*>(xq + m * static_cast<int64_t>(nv) * 8);
@@ -427,9 +456,10 @@ __global__ void __launch_bounds__(kQuantThreads, kF32 ? 2 : 4) quant_pass_a_kern
 // own dependency wait (and launch 2 only starts after that point), and launch
 // 1 neither reads xq / s_x nor writes x. So they run beside pass A, and the
 // code-pass blocks -- which do wait -- follow; since they wait, this grid
-// still completes only after launch 1 has. Rows of up to 1024 elements stay
-// in registers (VPL <= 4), longer ones are read twice (VPL = 0).
-constexpr int kFusedMaxVpl = 4;
+// still completes only after launch 1 has. Rows of up to 2560 elements stay
+// in registers (VPL <= 10, the most that fits the 64 registers a thread has at
+// four blocks per SM), longer ones are read twice (VPL = 0).
+constexpr int kFusedMaxVpl = 10;
 
 template <bool kF32, int VPL>
 __global__ void __launch_bounds__(kQuantThreads, kF32 ? 2 : 4) quant_phase2_kernel(
@@ -462,9 +492,9 @@ __global__ void __launch_bounds__(32 * kActRowsPerBlock) act_quant_long_kernel(c
   const int64_t m = static_cast<int64_t>(blockIdx.x) * kActRowsPerBlock + (threadIdx.x >> 5);
   if (m >= M) return;
   const uint4* row = x + m * nv;
-  float amax = 0.0f;
-  for (int j = lane; j < nv; j += 32) amax = absmax8(__ldg(row + j), amax);
-  const float a = fmaxf(warp_max(amax), 1e-5f);
+  uint32_t mx = 0u;
+  for (int j = lane; j < nv; j += 32) mx = absmax8(__ldg(row + j), mx);
+  const float a = fmaxf(warp_max(absmax_value(mx)), 1e-5f);
   const float inv = __fdiv_rn(127.0f, a);
   if (lane == 0) sx[m] = __fdiv_rn(a, 127.0f);
   uint2* out = reinterpret_cast<uint2*>(xq + m * static_cast<int64_t>(nv) * 8);
@@ -636,7 +666,8 @@ cudaError_t launch_quantize(const void* W, int w_is_f32, int64_t N, int64_t K, c
     e = w_is_f32 ? launch_quantize_fused<true, n>(w, N, K, xv, M, out, gamma, partials, xq, sx, s)    \
                  : launch_quantize_fused<false, n>(w, N, K, xv, M, out, gamma, partials, xq, sx, s); \
     break;
-    BL_Q_CASE(0) BL_Q_CASE(1) BL_Q_CASE(2) BL_Q_CASE(3) BL_Q_CASE(4)
+    BL_Q_CASE(0) BL_Q_CASE(1) BL_Q_CASE(2) BL_Q_CASE(3) BL_Q_CASE(4) BL_Q_CASE(5) BL_Q_CASE(6)
+    BL_Q_CASE(7) BL_Q_CASE(8) BL_Q_CASE(9) BL_Q_CASE(10)
 #undef BL_Q_CASE
     default:
       break;
