@@ -374,8 +374,9 @@ __device__ __forceinline__ void load_stage(const GemmParams& p, const OpParams& 
   }
   if constexpr (op != Op::Dw) {
     if (!P.src_tma) {
-      // packed codes by 8-byte cp.async (rows not 16-byte aligned); every lane's
-      // copies hold the phase open until they land, lane 0 gives the one arrival
+      // packed codes by 8-byte cp.async (rows not 16-byte aligned), placed in
+      // the 32-byte-swizzled layout the TMA path produces; every lane's copies
+      // hold the phase open until they land, lane 0 gives the one arrival
       constexpr int kChunks = (op == Op::Fwd) ? 16 : 8;  // per lane
 #pragma unroll
       for (int it = 0; it < kChunks; ++it) {
@@ -392,7 +393,8 @@ __device__ __forceinline__ void load_stage(const GemmParams& p, const OpParams& 
           valid = (r0 + row < P.red) && (a0 + part * 32 < P.rows_a);
           src = p.packed + static_cast<int64_t>(r0 + row) * kq + a0 / 4 + part * 8;
         }
-        cp_async_8(sSrc + row * 32 + part * 8, valid ? src : p.packed, valid ? 8u : 0u);
+        const int dst = row * 32 + ((((part >> 1) ^ (row >> 2)) & 1) << 4) + ((part & 1) << 3);
+        cp_async_8(sSrc + dst, valid ? src : p.packed, valid ? 8u : 0u);
       }
       cp_async_mbar_arrive(src_full);
       __syncwarp();
@@ -406,19 +408,20 @@ template <Op op, Family F, int BN>
 __device__ __forceinline__ void rebuild_stage(int rt, uint32_t sA, uint32_t sSrc, const float* sSx) {
   if constexpr (op == Op::Fwd) {
     // row rt: 32 packed bytes -> 128 int8 codes, K-major with 128-byte swizzle.
-    // Lanes 4..7 of each group of 8 read their second half first (bank spread).
+    // The staged rows are 32-byte swizzled (16-byte half c of row r at c ^ bit
+    // 2 of r), so lanes 0..3 and 4..7 of each group of 8 read different banks.
     const uint32_t h = (rt >> 2) & 1;
-    const uint4 wa = ld_shared_v4(sSrc + rt * 32 + h * 16);
-    const uint4 wb = ld_shared_v4(sSrc + rt * 32 + (h ^ 1) * 16);
-    const uint4 w0 = h ? wb : wa, w1 = h ? wa : wb;
+    const uint4 w0 = ld_shared_v4(sSrc + rt * 32 + h * 16);        // codes 0..63
+    const uint4 w1 = ld_shared_v4(sSrc + rt * 32 + (h ^ 1) * 16);  // codes 64..127
     const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
     const uint32_t row_base = sA + rt * 128;
 #pragma unroll
     for (int c = 0; c < 8; ++c) st_shared_v4(row_base + ((c ^ (rt & 7)) << 4), codes16_to_s8(words[c]));
   } else if constexpr (op == Op::Dx) {
-    // reduction row n = rt % 64, output k half = rt / 64 (64 k values)
+    // reduction row n = rt % 64, output k half = rt / 64 (64 k values); the
+    // staged rows are 32-byte swizzled like the forward's
     const int n = rt & 63, half = rt >> 6;
-    const uint4 w = ld_shared_v4(sSrc + n * 32 + half * 16);
+    const uint4 w = ld_shared_v4(sSrc + n * 32 + ((half ^ ((n >> 2) & 1)) << 4));
     const uint32_t words[4] = {w.x, w.y, w.z, w.w};
     const uint32_t base = sA + half * 8192 + n * 128;
 #pragma unroll
@@ -1267,7 +1270,7 @@ cudaError_t launch_forward(const int8_t* xq, const float* sx, const uint8_t* w_p
   // packed codes [N][K/4] bytes: a TMA tensor needs a 16-byte row pitch (K % 64 == 0)
   const bool src_tma = (K % 64) == 0;
   if (src_tma && !make_map_2d(&maps[1], w_packed, CU_TENSOR_MAP_DATA_TYPE_UINT8, K / 4, N, K / 4, 32, BM,
-                              CU_TENSOR_MAP_SWIZZLE_NONE, "w_packed (fwd)"))
+                              CU_TENSOR_MAP_SWIZZLE_32B, "w_packed (fwd)"))
     return cudaErrorInvalidValue;
   static thread_local GemmParams p;
   std::memset(&p, 0, offsetof(GemmParams, sched_start));
@@ -1307,7 +1310,7 @@ cudaError_t launch_backward(const void* dY, const int8_t* xq, const float* sx, c
                      CU_TENSOR_MAP_SWIZZLE_128B, "dY (dX)"))
       return cudaErrorInvalidValue;
     if (src_tma && !make_map_2d(&maps[1], w_packed, CU_TENSOR_MAP_DATA_TYPE_UINT8, K / 4, N, K / 4, 32, 64,
-                                CU_TENSOR_MAP_SWIZZLE_NONE, "w_packed (dX)"))
+                                CU_TENSOR_MAP_SWIZZLE_32B, "w_packed (dX)"))
       return cudaErrorInvalidValue;
   }
   if (dW) {
