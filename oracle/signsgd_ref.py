@@ -28,10 +28,12 @@ Readings where the pages leave a step open:
   * the update runs in fp32 and is stored in the master dtype:
     W' = dtype_rn(fp32(fp32(W) - lr * d)); with d in {-1, 0, +1} the product
     lr * d is exact, so fp32 rounds once and bf16 masters round once more.
+    Where d = 0 the step is +0: the weight is left bit for bit.
 
-Pinning: tests/test_oracle_pins.py checks these against np.signbit written
-out element by element, brute-force vote counts, closed forms of the update
-and the sign-equality identity of the same page.
+Pinning: tests/test_oracle_signsgd_pins.py checks these against a
+hand-written bit pattern, an element-by-element math.copysign loop,
+brute-force vote counts with Python integers and closed forms of the fp32
+and bf16 update.
 """
 
 from __future__ import annotations
@@ -83,5 +85,8 @@ def signsgd_update(w: np.ndarray, direction: np.ndarray, lr, w_is_bf16: bool) ->
     bits with ``bitlinear_ref.round_to_bf16_bits`` (the second rounding).
     """
     wf = np.asarray(w, dtype=np.float32)
-    step = np.float32(lr) * np.asarray(direction, dtype=np.float32)  # exact: d in {-1, 0, 1}
+    d = np.asarray(direction)
+    # lr * d is exact for d = +-1; where d = 0 the step is +0, so W is left
+    # bit for bit (also -0, and whatever the sign of lr)
+    step = np.where(d == 0, np.float32(0.0), np.float32(lr) * d.astype(np.float32)).astype(np.float32)
     return (wf - step).astype(np.float32)

@@ -113,6 +113,9 @@ def test_signsgd_update_closed_forms_f32():
     # d = 0 leaves every value bit for bit, whatever lr
     r = np.random.default_rng(7).standard_normal(64).astype(np.float32)
     assert np.array_equal(sg.signsgd_update(r, np.zeros(64, np.int8), 123.0, False).view(np.uint32), r.view(np.uint32))
+    # ... also with a negative lr, on -0
+    mz = np.array([-0.0], dtype=np.float32)
+    assert sg.signsgd_update(mz, np.array([0], np.int8), -1.0, False).view(np.uint32)[0] == 0x80000000
 
 
 def test_signsgd_update_bf16_second_rounding():
