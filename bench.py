@@ -579,6 +579,111 @@ def run_few_tokens(args, rank, world, local_rank):
             "peak_gbs": peaks["hbm_gbs"], "peak_source": f"{peak_src} hbm copy", "by_tokens": rows}
 
 
+def run_signsgd(args, rank, world, local_rank):
+    """Sign-gradient data-parallel mode at up_proj: every rank quantises its
+    tokens, runs forward and backward with the 2-bit codes it holds, packs the
+    signs of its dW and sends them to rank 0, which alone holds the master W,
+    votes, updates W, re-ternarises and broadcasts the new codes. The line
+    reports the whole step (6 M N K per rank over the max-over-ranks time) and,
+    per sign-gradient kernel, achieved HBM GB/s against the measured copy
+    bandwidth."""
+    import ternary_weight_quantization_b200 as bl
+    from ternary_weight_quantization_b200.signsgd import SignBuffers, signsgd_dp_step
+    from workloads import workload_inputs
+
+    bl.load_library()
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    x_cpu, w_cpu, dy_cpu = workload_inputs("up_proj", seed=rank)
+    M, K = x_cpu.shape
+    N = w_cpu.shape[0]
+    holder = rank == 0
+    x, dy = x_cpu.to(dev), dy_cpu.to(dev)
+    master = w_cpu.to(dev) if holder else None
+    packed = torch.empty((N, K // 4), dtype=torch.uint8, device=dev)
+    gamma = torch.empty(1, dtype=torch.float32, device=dev)
+    ws = torch.empty(max(bl.bl_quantize_weight_workspace_size(N, K), 16), dtype=torch.uint8, device=dev)
+    xq = torch.empty((M, K), dtype=torch.int8, device=dev)
+    sx = torch.empty(M, dtype=torch.float32, device=dev)
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    dX = torch.empty((M, K), dtype=torch.bfloat16, device=dev)
+    dW = torch.empty((N, K), dtype=torch.bfloat16, device=dev)
+    buf = SignBuffers.allocate(N, K, world, holder, dev)
+    lr = 2.0 ** -12
+    if holder:
+        bl.bl_quantize_weight(master, packed, gamma, ws)
+    if world > 1:
+        torch.distributed.broadcast(packed, src=0)
+        torch.distributed.broadcast(gamma, src=0)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def step():
+        bl.bl_quantize_act(x, xq, sx)
+        bl.bl_forward(xq, sx, packed, gamma, y)
+        bl.bl_backward(dy, xq, sx, packed, gamma, dX, dW)
+        signsgd_dp_step(dW, packed, gamma, lr, master_W=master, workspace=ws if holder else None, buffers=buf)
+
+    times = []
+    for i in range(args.warmup + args.steps):
+        flush.fill_(i & 0xFF)
+        flush.view(torch.int64).max()
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize(dev)
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record(stream)
+        step()
+        e.record(stream)
+        torch.cuda.synchronize(dev)
+        if i >= args.warmup:
+            times.append(s.elapsed_time(e))
+    local_ms = sum(times) / len(times)
+    job_ms = job_time_ms(local_ms, world, dev)
+
+    # breakdown of the holder's sign-gradient kernels (events between the calls)
+    peaks, peak_src = load_peaks()
+    kern = {}
+    if holder:
+        words = buf.gathered[0] if world == 1 else buf.words
+        calls = {
+            "sign_pack": (lambda: bl.bl_sign_pack(dW, words), N * K * 2 + N * K // 8),
+            "sign_vote": (lambda: bl.bl_sign_vote(buf.gathered, buf.direction), world * N * K // 8 + N * K // 4),
+            "signsgd_update": (lambda: bl.bl_signsgd_update(master, buf.direction, 0.0),
+                               2 * N * K * 2 + N * K // 4),
+            "quantize_weight": (lambda: bl.bl_quantize_weight(master, packed, gamma, ws), N * K * 2 + N * K // 4),
+        }
+        for name, (fn, nbytes) in calls.items():
+            ts = []
+            for i in range(args.warmup + min(args.steps, 50)):
+                flush.fill_(i & 0xFF)
+                flush.view(torch.int64).max()
+                s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                s.record(stream)
+                fn()
+                e.record(stream)
+                torch.cuda.synchronize(dev)
+                if i >= args.warmup:
+                    ts.append(s.elapsed_time(e))
+            ms = sum(ts) / len(ts)
+            gbs = nbytes / (ms * 1e-3) / 1e9
+            kern[name] = {"ms": round(ms, 5), "bytes": nbytes, "achieved_gbs": round(gbs, 1),
+                          "frac": round(gbs / peaks["hbm_gbs"], 4)}
+    if bl.bl_get_last_error() != 0:
+        raise RuntimeError("device error")
+    if rank != 0:
+        return None
+    ops = 6.0 * M * N * K
+    return {"metric": "bitlinear_signsgd_dp_step_tops", "value": round(job_tops(ops, world, 1, job_ms), 2),
+            "unit": "TOPS", "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(job_ms, 5),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8/bf16",
+            "data": "synthetic",
+            "config": {"workload": "up_proj, sign-gradient data-parallel step", "M": M, "K": K, "N": N,
+                       "ranks": world, "lr": lr, "masters": "bf16 on rank 0 only",
+                       "l2": "flushed before every step (256 MiB written, then read back)"},
+            "peak_gbs": peaks["hbm_gbs"], "peak_source": f"{peak_src} hbm copy", "kernels": kern}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -590,6 +695,8 @@ def main():
     ap.add_argument("--cpu-tokens", type=int, default=4096)
     ap.add_argument("--stack", choices=["stack8"], default=None,
                     help="layer-stack mode (prints its own line instead of the single-layer one)")
+    ap.add_argument("--signsgd", action="store_true",
+                    help="sign-gradient data-parallel step mode (prints its own line)")
     ap.add_argument("--few-tokens", default=None,
                     help="forward-only mode at these token counts, e.g. 1,8,16 (prints its own line)")
     args = ap.parse_args()
@@ -615,6 +722,8 @@ def main():
             out = run_stack(args, rank, world, local_rank)
         elif args.few_tokens:
             out = run_few_tokens(args, rank, world, local_rank)
+        elif args.signsgd:
+            out = run_signsgd(args, rank, world, local_rank)
         else:
             out = run_ours(args, rank, world, local_rank)
         if rank == 0 and out is not None:

@@ -208,6 +208,53 @@ bl_status bl_export_weights(const uint8_t* w_packed, const float* gamma,
                             uint8_t* host_packed, float* host_gamma, void* stream);
 
 /*
+ * Master-free sign-gradient training, data parallel ("1BitTraining.md", "Why
+ * this always holds", closing paragraph on implications: the straight-through
+ * gradient and the gradient of the quantised weight have the same sign, so a
+ * sign-based optimiser needs only the 2-bit weights on each device and one
+ * bit of gradient per weight, sent to one place that accumulates them).
+ * One step over R data-parallel ranks:
+ *   every rank   bl_backward -> dW, bl_sign_pack -> its sign words
+ *   exchange     the R ranks' sign words are gathered (N*K/8 bytes a rank)
+ *   holder of W  bl_sign_vote -> direction, bl_signsgd_update on W, then
+ *                bl_quantize_weight -> the next codes and gamma, which go
+ *                back to the ranks.
+ */
+
+/*
+ * G1: the 1-bit gradient. sign_words [N*K/32] (uint32) receives the IEEE sign
+ * bit of every element of dW [N,K] (dw_dtype BL_BF16 or BL_F32): element
+ * 32*w + j of the flattened tensor is bit j of word w (1 = negative; -0.0
+ * counts as negative). Reads N*K*(2|4) bytes, writes N*K/8.
+ * Errors: BL_ERR_INVALID_ARG (null, N < 1), BL_ERR_UNSUPPORTED_SHAPE (K),
+ *         BL_ERR_DTYPE, BL_ERR_ALIGNMENT, BL_ERR_ARCH, BL_ERR_CUDA.
+ */
+bl_status bl_sign_pack(const void* dW, bl_dtype dw_dtype, int64_t N, int64_t K,
+                       uint32_t* sign_words, void* stream);
+
+/*
+ * G2: the accumulation. sign_words holds `ranks` arrays of N*K/32 words back
+ * to back (rank r at sign_words + r*N*K/32), 1 <= ranks <= 127. direction
+ * [N,K/4] receives, per weight, +1 where more ranks have a positive (sign bit
+ * 0) gradient, -1 where more have a negative one, 0 on a tie, in the 2-bit
+ * packing of w_packed (00 = 0, 01 = +1, 11 = -1).
+ * Errors: as bl_sign_pack (BL_ERR_INVALID_ARG also for ranks out of range).
+ */
+bl_status bl_sign_vote(const uint32_t* sign_words, int ranks, int64_t N, int64_t K,
+                       uint8_t* direction, void* stream);
+
+/*
+ * G3: the sign-gradient step where the master weights are held. In place on
+ * W [N,K] (w_dtype BL_BF16 or BL_F32): W = dtype_rn(fp32(W) - lr * d) with d
+ * the direction of bl_sign_vote; the fp32 subtraction rounds once (lr * d is
+ * exact), bf16 masters round once more. Where d = 0 (or the unused field 10)
+ * the weight is left bit for bit. lr must be finite.
+ * Errors: as bl_sign_pack (BL_ERR_INVALID_ARG also for a non-finite lr).
+ */
+bl_status bl_signsgd_update(void* W, bl_dtype w_dtype, int64_t N, int64_t K,
+                            const uint8_t* direction, float lr, void* stream);
+
+/*
  * Synchronises the current device, then returns BL_OK or the first device
  * failure recorded since the last bl_reset_error (BL_ERR_TIMEOUT).
  */

@@ -44,6 +44,9 @@ SIGNATURES = {
     "bl_get_last_error": (_I32, []),
     "bl_reset_error": (_I32, []),
     "bl_selftest_timeout": (_I32, [_VP]),
+    "bl_sign_pack": (_I32, [_VP, _I32, _I64, _I64, _VP, _VP]),
+    "bl_sign_vote": (_I32, [_VP, _I32, _I64, _I64, _VP, _VP]),
+    "bl_signsgd_update": (_I32, [_VP, _I32, _I64, _I64, _VP, ctypes.c_float, _VP]),
 }
 
 
@@ -187,6 +190,38 @@ def bl_backward(dY, xq, sx, w_packed, gamma, dX=None, dW=None, accumulate_dW=Fal
     _check(load_library().bl_backward(_ptr(dY), _ptr(xq), _ptr(sx), _ptr(w_packed), _ptr(gamma), M, N, K,
                                       _ptr(dX), _ptr(dW), dwdt, int(bool(accumulate_dW)), _stream(stream)),
            "bl_backward")
+
+
+def bl_sign_pack(dW, sign_words, stream=None):
+    """G1: sign_words [N, K/32] int32 (bit patterns) <- sign bits of dW [N, K] (bf16|f32)."""
+    N, K = dW.shape
+    if dW.dtype not in (torch.bfloat16, torch.float32):
+        raise ValueError("dW must be bf16 or f32")
+    _need(dW, dW.dtype, (N, K), "dW")
+    _need(sign_words, torch.int32, (N, K // 32), "sign_words")
+    dt = BL_F32 if dW.dtype == torch.float32 else BL_BF16
+    _check(load_library().bl_sign_pack(_ptr(dW), dt, N, K, _ptr(sign_words), _stream(stream)), "bl_sign_pack")
+
+
+def bl_sign_vote(sign_words, direction, stream=None):
+    """G2: direction [N, K/4] uint8 (2-bit packed) <- majority of sign_words [R, N, K/32] int32."""
+    R, N, KW = sign_words.shape
+    _need(sign_words, torch.int32, (R, N, KW), "sign_words")
+    _need(direction, torch.uint8, (N, KW * 8), "direction")
+    _check(load_library().bl_sign_vote(_ptr(sign_words), R, N, KW * 32, _ptr(direction), _stream(stream)),
+           "bl_sign_vote")
+
+
+def bl_signsgd_update(W, direction, lr, stream=None):
+    """G3: W [N, K] (bf16|f32) <- dtype_rn(fp32(W) - lr * direction), in place."""
+    N, K = W.shape
+    if W.dtype not in (torch.bfloat16, torch.float32):
+        raise ValueError("W must be bf16 or f32")
+    _need(W, W.dtype, (N, K), "W")
+    _need(direction, torch.uint8, (N, K // 4), "direction")
+    dt = BL_F32 if W.dtype == torch.float32 else BL_BF16
+    _check(load_library().bl_signsgd_update(_ptr(W), dt, N, K, _ptr(direction), float(lr), _stream(stream)),
+           "bl_signsgd_update")
 
 
 def bl_export_weights(w_packed, gamma, stream=None):

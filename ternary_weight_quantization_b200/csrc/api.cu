@@ -237,6 +237,50 @@ bl_status bl_export_weights(const uint8_t* w_packed, const float* gamma, int64_t
   return cuda_status(cudaStreamSynchronize(st), "export sync");
 }
 
+bl_status bl_sign_pack(const void* dW, bl_dtype dw_dtype, int64_t N, int64_t K, uint32_t* sign_words, void* stream) {
+  g_msg[0] = 0;
+  if (N < 1) return fail(BL_ERR_INVALID_ARG, "N=%lld must be >= 1", (long long)N);
+  if (bl_status s = check_k(K)) return s;
+  if (dw_dtype != BL_BF16 && dw_dtype != BL_F32) return fail(BL_ERR_DTYPE, "dw_dtype %d", (int)dw_dtype);
+  if (!dW || !sign_words) return fail(BL_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(dW) || !aligned16(sign_words)) return fail(BL_ERR_ALIGNMENT, "dW and sign_words must be 16-byte aligned");
+  int* err = nullptr;
+  if (bl_status s = current_device(&err)) return s;
+  return cuda_status(bl::launch_sign_pack(dW, dw_dtype == BL_F32, N, K, sign_words, static_cast<cudaStream_t>(stream)),
+                     "bl_sign_pack");
+}
+
+bl_status bl_sign_vote(const uint32_t* sign_words, int ranks, int64_t N, int64_t K, uint8_t* direction,
+                       void* stream) {
+  g_msg[0] = 0;
+  if (N < 1) return fail(BL_ERR_INVALID_ARG, "N=%lld must be >= 1", (long long)N);
+  if (bl_status s = check_k(K)) return s;
+  if (ranks < 1 || ranks > 127) return fail(BL_ERR_INVALID_ARG, "ranks=%d must be in 1..127", ranks);
+  if (!sign_words || !direction) return fail(BL_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(sign_words) || !aligned16(direction))
+    return fail(BL_ERR_ALIGNMENT, "sign_words and direction must be 16-byte aligned");
+  int* err = nullptr;
+  if (bl_status s = current_device(&err)) return s;
+  return cuda_status(bl::launch_sign_vote(sign_words, ranks, N, K, direction, static_cast<cudaStream_t>(stream)),
+                     "bl_sign_vote");
+}
+
+bl_status bl_signsgd_update(void* W, bl_dtype w_dtype, int64_t N, int64_t K, const uint8_t* direction, float lr,
+                            void* stream) {
+  g_msg[0] = 0;
+  if (N < 1) return fail(BL_ERR_INVALID_ARG, "N=%lld must be >= 1", (long long)N);
+  if (bl_status s = check_k(K)) return s;
+  if (w_dtype != BL_BF16 && w_dtype != BL_F32) return fail(BL_ERR_DTYPE, "w_dtype %d", (int)w_dtype);
+  if (!(lr - lr == 0.0f)) return fail(BL_ERR_INVALID_ARG, "lr must be finite");
+  if (!W || !direction) return fail(BL_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(W) || !aligned16(direction)) return fail(BL_ERR_ALIGNMENT, "W and direction must be 16-byte aligned");
+  int* err = nullptr;
+  if (bl_status s = current_device(&err)) return s;
+  return cuda_status(bl::launch_signsgd_update(W, w_dtype == BL_F32, N, K, direction, lr,
+                                               static_cast<cudaStream_t>(stream)),
+                     "bl_signsgd_update");
+}
+
 bl_status bl_selftest_timeout(void* stream) {
   g_msg[0] = 0;
   int* err = nullptr;

@@ -61,6 +61,17 @@ cudaError_t launch_backward(const void* dY, const int8_t* xq, const float* sx, c
                             const float* gamma, int64_t M, int64_t N, int64_t K, void* dX, void* dW, int dw_is_f32,
                             int accumulate, int* err, cudaStream_t s);
 
+// ---- Master-free sign-gradient update (k_signsgd.cu)
+// Sign bits of dW [N,K] (bf16 or f32): out [N*K/32] words, element 32w+j -> bit j.
+cudaError_t launch_sign_pack(const void* dW, int dw_is_f32, int64_t N, int64_t K, uint32_t* out, cudaStream_t s);
+// Majority vote of `ranks` sign-word arrays (rank r at words + r*N*K/32) ->
+// 2-bit packed direction [N, K/4].
+cudaError_t launch_sign_vote(const uint32_t* words, int ranks, int64_t N, int64_t K, uint8_t* direction,
+                             cudaStream_t s);
+// W [N,K] (bf16 or f32) <- dtype_rn(fp32(W) - lr * direction), in place.
+cudaError_t launch_signsgd_update(void* W, int w_is_f32, int64_t N, int64_t K, const uint8_t* direction, float lr,
+                                  cudaStream_t s);
+
 // One warp waiting on an mbarrier that is never completed (bounded wait test).
 cudaError_t launch_selftest_timeout(int* err, cudaStream_t s);
 

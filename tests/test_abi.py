@@ -61,6 +61,16 @@ MISALIGNED = ctypes.c_void_p(0x10008)
     (lambda L: L.bl_backward(FAKE, FAKE, FAKE, FAKE, FAKE, 4, 16, 64, FAKE, FAKE, 9, 0, None), 3),
     (lambda L: L.bl_backward(FAKE, FAKE, FAKE, None, FAKE, 4, 16, 64, FAKE, None, 0, 0, None), 1),
     (lambda L: L.bl_export_weights(FAKE, FAKE, 4, 64, None, FAKE, None), 1),
+    (lambda L: L.bl_sign_pack(FAKE, 0, 4, 48, FAKE, None), 2),               # K % 32
+    (lambda L: L.bl_sign_pack(FAKE, 5, 4, 64, FAKE, None), 3),
+    (lambda L: L.bl_sign_pack(FAKE, 0, 4, 64, MISALIGNED, None), 4),
+    (lambda L: L.bl_sign_vote(FAKE, 0, 4, 64, FAKE, None), 1),               # ranks
+    (lambda L: L.bl_sign_vote(FAKE, 128, 4, 64, FAKE, None), 1),
+    (lambda L: L.bl_sign_vote(FAKE, 2, 4, 64, None, None), 1),
+    (lambda L: L.bl_signsgd_update(FAKE, 0, 4, 64, FAKE, float("inf"), None), 1),  # lr
+    (lambda L: L.bl_signsgd_update(FAKE, 0, 4, 64, FAKE, float("nan"), None), 1),
+    (lambda L: L.bl_signsgd_update(FAKE, 2, 4, 64, FAKE, 0.1, None), 3),
+    (lambda L: L.bl_signsgd_update(FAKE, 0, 0, 64, FAKE, 0.1, None), 1),
 ])
 def test_host_validation_without_gpu(call, expect):
     lib = b.load_library()

@@ -1,0 +1,136 @@
+"""GPU parity of the sign-gradient kernels against the CPU oracle.
+
+Bar: every output is integer or a once-rounded value the oracle forms in the
+same precision, so all comparisons are bit-exact:
+  G1  sign words                       bit-exact
+  G2  2-bit vote direction             bit-exact
+  G3  updated masters (bf16 / f32)     bit-exact
+  the whole single-rank step (G1 -> G2 -> G3 -> S1): codes and gamma bit-exact
+"""
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import bitlinear_ref as ref
+from oracle import signsgd_ref as sg
+
+pytestmark = pytest.mark.gpu
+
+
+def _bl():
+    import ternary_weight_quantization_b200 as bl
+    bl.load_library()
+    return bl
+
+
+def _u16(t):
+    return t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def _grad(shape, dtype, seed):
+    g = torch.Generator().manual_seed(seed)
+    d = torch.randn(shape, generator=g)
+    r = torch.rand(shape, generator=g)
+    d[r < 0.05] = 0.0
+    d[(r >= 0.05) & (r < 0.08)] = -0.0
+    d[(r >= 0.08) & (r < 0.09)] = -1e-40  # a subnormal in both dtypes
+    return d.to(dtype)
+
+
+def _as_f32(t):
+    return t.float().cpu().numpy()
+
+
+@pytest.mark.parametrize("shape", [(1, 32), (3, 96), (7, 160), (33, 2560), (6912, 2560)])
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_sign_pack_matches_oracle(shape, dtype):
+    bl = _bl()
+    if dtype == torch.float32 and shape[0] * shape[1] > 1 << 22:
+        pytest.skip("f32 covered on the smaller shapes")
+    d = _grad(shape, dtype, seed=shape[0])
+    words = torch.empty((shape[0], shape[1] // 32), dtype=torch.int32, device="cuda")
+    bl.bl_sign_pack(d.cuda(), words)
+    torch.cuda.synchronize()
+    expect = sg.sign_bits(_as_f32(d))  # float() keeps every sign bit
+    assert np.array_equal(words.cpu().numpy().view(np.uint32), expect)
+
+
+@pytest.mark.parametrize("ranks,shape", [(1, (4, 64)), (2, (5, 96)), (3, (8, 128)), (4, (2, 32)),
+                                         (7, (16, 256)), (8, (9, 160)), (127, (3, 64)), (2, (6912, 2560))])
+def test_sign_vote_matches_oracle(ranks, shape):
+    bl = _bl()
+    n, k = shape
+    g = torch.Generator().manual_seed(1000 + ranks)
+    words = torch.randint(-2 ** 31, 2 ** 31, (ranks, n, k // 32), generator=g, dtype=torch.int64).to(torch.int32)
+    direction = torch.empty((n, k // 4), dtype=torch.uint8, device="cuda")
+    bl.bl_sign_vote(words.cuda(), direction)
+    torch.cuda.synchronize()
+    expect = ref.pack_ternary(sg.majority_direction([w.numpy().view(np.uint32) for w in words]))
+    assert np.array_equal(direction.cpu().numpy(), expect)
+
+
+def _direction(shape, seed):
+    n, k = shape
+    g = torch.Generator().manual_seed(seed)
+    codes = torch.randint(-1, 2, (n, k), generator=g, dtype=torch.int8).numpy()
+    return codes, ref.pack_ternary(codes)
+
+
+@pytest.mark.parametrize("shape", [(2, 32), (5, 96), (64, 2560), (6912, 2560)])
+@pytest.mark.parametrize("lr", [2.0 ** -6, 1e-3, -0.5])
+def test_signsgd_update_bf16_matches_oracle(shape, lr):
+    bl = _bl()
+    g = torch.Generator().manual_seed(shape[0])
+    w = (torch.randn(shape, generator=g) * 0.02).to(torch.bfloat16)
+    w[0, :4] = torch.tensor([-0.0, 0.0, 1.0, -1.0], dtype=torch.bfloat16)
+    codes, packed = _direction(shape, seed=shape[1])
+    wd = w.cuda()
+    bl.bl_signsgd_update(wd, torch.from_numpy(packed).cuda(), lr)
+    torch.cuda.synchronize()
+    expect = ref.round_to_bf16_bits(sg.signsgd_update(_as_f32(w), codes, lr, w_is_bf16=True))
+    assert np.array_equal(_u16(wd), expect)
+
+
+@pytest.mark.parametrize("shape", [(2, 32), (7, 160), (128, 2560)])
+@pytest.mark.parametrize("lr", [2.0 ** -6, 3e-4])
+def test_signsgd_update_f32_matches_oracle(shape, lr):
+    bl = _bl()
+    g = torch.Generator().manual_seed(7 + shape[0])
+    w = torch.randn(shape, generator=g) * 0.02
+    w[0, 0] = -0.0
+    codes, packed = _direction(shape, seed=3 + shape[1])
+    wd = w.cuda()
+    bl.bl_signsgd_update(wd, torch.from_numpy(packed).cuda(), lr)
+    torch.cuda.synchronize()
+    expect = sg.signsgd_update(w.numpy(), codes, lr, w_is_bf16=False)
+    assert np.array_equal(wd.cpu().numpy().view(np.uint32), expect.view(np.uint32))
+
+
+@pytest.mark.parametrize("shape,w_dtype", [((6912, 2560), torch.bfloat16), ((96, 320), torch.float32)])
+def test_single_rank_step_matches_oracle_chain(shape, w_dtype):
+    bl = _bl()
+    from ternary_weight_quantization_b200.signsgd import signsgd_dp_step
+    n, k = shape
+    g = torch.Generator().manual_seed(11)
+    master = (torch.randn(shape, generator=g) * 0.02).to(w_dtype)
+    dW = _grad(shape, torch.bfloat16, seed=12)
+    lr = 2.0 ** -8
+    wd = master.cuda()
+    w_packed = torch.empty((n, k // 4), dtype=torch.uint8, device="cuda")
+    gamma = torch.empty(1, dtype=torch.float32, device="cuda")
+    ws = torch.empty(max(bl.bl_quantize_weight_workspace_size(n, k), 16), dtype=torch.uint8, device="cuda")
+    signsgd_dp_step(dW.cuda(), w_packed, gamma, lr, master_W=wd, workspace=ws)
+    torch.cuda.synchronize()
+
+    d = sg.majority_direction([sg.sign_bits(_as_f32(dW))])
+    w_new = sg.signsgd_update(_as_f32(master), d, lr, w_is_bf16=w_dtype == torch.bfloat16)
+    if w_dtype == torch.bfloat16:
+        w_new_bits = ref.round_to_bf16_bits(w_new)
+        assert np.array_equal(_u16(wd), w_new_bits)
+        w_new = ref.bf16_bits_to_f32(w_new_bits)
+    else:
+        assert np.array_equal(wd.cpu().numpy().view(np.uint32), w_new.view(np.uint32))
+    codes, gm = ref.ternarize(w_new)
+    assert float(gamma.item()) == float(gm)
+    assert np.array_equal(w_packed.cpu().numpy(), ref.pack_ternary(codes))
