@@ -451,7 +451,7 @@ def run_reference(args):
 # ----------------------------------------------------------------- main
 
 def run_stack(args, rank, world, local_rank):
-    """Layer-stack mode: SURVEY config 4 (8 BitLinear layers alternating
+    """Layer-stack mode: the 8-layer stack workload (8 BitLinear layers alternating
     2560 -> 6912 -> 2560, 2048 tokens). One step = the forward of every layer
     (bl_quantize + bl_forward, only the 2-bit / INT8 state kept) and the
     backward of every layer in reverse (bl_backward, dX feeding the layer

@@ -43,7 +43,7 @@ WORKLOADS = {
 }
 
 
-# Layer stacks (SURVEY config 4): 8 BitLinear layers alternating
+# Layer stacks: 8 BitLinear layers alternating
 # 2560 -> 6912 -> 2560 ... over x [4, 512, 2560].
 STACKS = {
     "stack8": (2048, [2560, 6912] * 4 + [2560]),
