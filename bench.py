@@ -684,6 +684,40 @@ def run_signsgd(args, rank, world, local_rank):
             "peak_gbs": peaks["hbm_gbs"], "peak_source": f"{peak_src} hbm copy", "kernels": kern}
 
 
+def run_lm(args, rank, world, local_rank):
+    """Decoder-LM mode: the 4-layer LM of workloads/lm.py trained through the
+    library (every projection a BitLinear call; the rest plain PyTorch) for
+    its 50 steps on each rank (independent replicas). Reports tokens per
+    second (batch x sequence per step over the mean device time of a step,
+    the first step excluded) and the largest |loss - oracle loss| over the
+    steps against the stored oracle curve."""
+    from ternary_weight_quantization_b200.lm import train_lm
+    from workloads.lm import LM_CONFIG, lm_batches, lm_init
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    cfg = LM_CONFIG
+    losses, ms = train_lm(lm_init(cfg, seed=0), lm_batches(cfg, seed=0), cfg, dev, timing=True)
+    job_ms = job_time_ms(ms, world, dev)
+    worst = None
+    gold_path = os.path.join(ROOT, "tests", "golden", "lm_oracle_losses.json")
+    if os.path.exists(gold_path):
+        with open(gold_path) as f:
+            gold = json.load(f)["losses"]
+        worst = max(abs(a - b) for a, b in zip(losses, gold))
+    if rank != 0:
+        return None
+    tokens = cfg.batch * cfg.seq
+    return {"metric": "bitlinear_lm_train_tokens_per_s", "value": round(tokens * world / (job_ms * 1e-3), 1),
+            "unit": "tokens/s", "n_gpus": world, "steps": cfg.steps, "warmup": 1, "ms_per_step": round(job_ms, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8/bf16 BitLinear, fp32 rest",
+            "data": "synthetic",
+            "config": {"workload": "4-layer decoder LM", "layers": cfg.layers, "d": cfg.d, "heads": cfg.heads,
+                       "ffn": cfg.ffn, "vocab": cfg.vocab, "seq": cfg.seq, "batch": cfg.batch, "lr": cfg.lr},
+            "loss_first": round(losses[0], 6), "loss_last": round(losses[-1], 6),
+            "max_abs_dloss_vs_oracle": None if worst is None else round(worst, 6)}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -695,6 +729,8 @@ def main():
     ap.add_argument("--cpu-tokens", type=int, default=4096)
     ap.add_argument("--stack", choices=["stack8"], default=None,
                     help="layer-stack mode (prints its own line instead of the single-layer one)")
+    ap.add_argument("--lm", action="store_true",
+                    help="decoder-LM training mode (prints its own line)")
     ap.add_argument("--signsgd", action="store_true",
                     help="sign-gradient data-parallel step mode (prints its own line)")
     ap.add_argument("--few-tokens", default=None,
@@ -724,6 +760,8 @@ def main():
             out = run_few_tokens(args, rank, world, local_rank)
         elif args.signsgd:
             out = run_signsgd(args, rank, world, local_rank)
+        elif args.lm:
+            out = run_lm(args, rank, world, local_rank)
         else:
             out = run_ours(args, rank, world, local_rank)
         if rank == 0 and out is not None:
