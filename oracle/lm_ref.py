@@ -60,7 +60,7 @@ class BitLinearRef(torch.autograd.Function):
         q, sx = ref.quantize_activations(x32)
         y32 = ref.forward_output(ref.forward_accumulate(q, codes), sx, gamma)
         ctx.state = (codes, gamma, q, sx)
-        return torch.from_numpy(_bf16(y32))
+        return torch.from_numpy(_bf16(y32)).to(x.dtype)
 
     @staticmethod
     def backward(ctx, gy):
@@ -69,7 +69,7 @@ class BitLinearRef(torch.autograd.Function):
         x_hat = ref.bf16_bits_to_f32(ref.round_to_bf16_bits(ref.dequantize_activations(q, sx)))
         dx = _bf16(ref.backward_dx(dy, codes, gamma))
         dw = ref.backward_dw(dy, x_hat).astype(np.float32).astype(np.float64)
-        return torch.from_numpy(dx), torch.from_numpy(dw)
+        return torch.from_numpy(dx).to(gy.dtype), torch.from_numpy(dw).to(gy.dtype)
 
 
 def _linear(x2d, w, quantize: bool):
@@ -125,9 +125,15 @@ def adamw_step(params: dict, grads: dict, state: dict, step: int, cfg):
             p.sub_(cfg.lr * (m / bc1) / (torch.sqrt(v / bc2) + cfg.eps))
 
 
-def train(init: dict, batches: torch.Tensor, cfg, steps: int | None = None, quantize: bool = True):
-    """Losses of `steps` AdamW steps from `init` (fp32 tensors) on `batches`."""
-    params = {n: t.detach().to(torch.float64).clone().requires_grad_(True) for n, t in init.items()}
+def train(init: dict, batches: torch.Tensor, cfg, steps: int | None = None, quantize: bool = True,
+          dtype=torch.float64):
+    """Losses of `steps` AdamW steps from `init` (fp32 tensors) on `batches`.
+
+    ``dtype`` is the precision of everything outside the BitLinear oracle
+    (parameters, AdamW state, the other layers): fp64 by default; fp32 gives
+    a run in the precision a GPU fp32 model keeps, to measure how far two
+    precisions alone drift apart over the steps."""
+    params = {n: t.detach().to(dtype).clone().requires_grad_(True) for n, t in init.items()}
     state: dict = {}
     losses = []
     for t in range(steps if steps is not None else batches.shape[0]):
