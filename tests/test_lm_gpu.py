@@ -42,11 +42,13 @@ def test_lm_first_loss_is_ln_vocab():
 
 # Measured on a B200: max |dloss| 0.0117 at step 45 of 50 (0.0027 at the last
 # step). The GPU model runs its non-BitLinear layers, its masters and AdamW in
-# fp32 and the oracle in fp64; the likely cause (not verified) is ternary
-# codes whose masters sit at a threshold flipping at different steps, so the
-# two trajectories drift apart by more than the 0.01 gate late in the run.
-@pytest.mark.xfail(strict=False, reason="max |dloss| 0.0117 at step 45 of 50 exceeds the 0.01 gate (fp32 model vs "
-                                        "fp64 oracle)")
+# fp32 and the oracle in fp64. The oracle itself run in fp32 around the same
+# BitLinear steps (tests/golden/lm_oracle_losses_fp32.json) drifts from its
+# fp64 curve by up to 0.0135 (step 46; above 0.01 at steps 45 and 46, mean
+# 0.0033): precision alone moves this curve past the 0.01 gate late in the run,
+# so the gate is kept and this case recorded as an expected failure.
+@pytest.mark.xfail(strict=False, reason="max |dloss| 0.0117 at step 45 of 50 exceeds the 0.01 gate; the oracle's "
+                                        "own fp32 run drifts from its fp64 curve by up to 0.0135")
 def test_lm_tracks_stored_oracle_curve():
     from ternary_weight_quantization_b200.lm import train_lm
     with open(os.path.join(GOLDEN, "lm_oracle_losses.json")) as f:
