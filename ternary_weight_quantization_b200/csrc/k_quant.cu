@@ -5,9 +5,10 @@
 // intermediate tensors in device memory. S1 needs gamma before any code, so
 // it is two passes over W: pass A (fp64 partial sums of |W|) and the code
 // pass (gamma from the partials, codes packed 4 per byte). bl_quantize runs
-// pass A and S2 in one launch (quant_phase1_kernel: the two are independent)
-// and then the code pass; bl_quantize_weight and bl_quantize_act launch the
-// same arithmetic separately.
+// pass A (quant_pass_a_kernel), then one grid (quant_phase2_kernel) whose
+// token blocks -- S2, independent of S1 -- start beside pass A and whose
+// code-pass blocks wait for it; bl_quantize_weight and bl_quantize_act launch
+// the same arithmetic separately.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
