@@ -115,9 +115,11 @@ bl_status bl_quantize_weight(const void* W, bl_dtype w_dtype, int64_t N, int64_t
  * the process exits. A request that would need more scratch than the array
  * holds returns BL_ERR_WORKSPACE.
  *
- * The first call on each device looks up the array's device address (a
- * runtime query, done with that device current) and caches it; make that
- * first call before any stream capture. All calls share the one array and
+ * Each call looks up the array's device address on the current device (a
+ * runtime query; the first one on a device loads the library's device code
+ * there, so make the first call on each device before any stream capture).
+ * The address is not cached, so a call after the caller reset the device
+ * finds the array where the reloaded device code put it. All calls share the one array and
  * nothing in it needs to start at zero (every call overwrites the part it
  * reads), but two calls whose kernels overlap on the GPU -- on different
  * streams of one device without ordering between them -- race on it and may

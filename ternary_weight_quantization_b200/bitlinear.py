@@ -89,7 +89,20 @@ def _ptr(t):
 def _stream(stream):
     if stream is None:
         stream = torch.cuda.current_stream()
+    elif stream.device.index != torch.cuda.current_device():
+        raise ValueError(f"stream of {stream.device} but the current CUDA device is cuda:{torch.cuda.current_device()}")
     return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _on_current_device(*tensors):
+    """Every tensor argument must live on the current CUDA device: the library
+    launches on the current device (and the stream passed is that device's),
+    so a tensor of another GPU would hand its kernels foreign pointers."""
+    cur = torch.cuda.current_device()
+    for t in tensors:
+        if t is not None and t.device.index != cur:
+            raise ValueError(f"tensor on {t.device} but the current CUDA device is cuda:{cur}; "
+                             "call under torch.cuda.device(...) of the tensors' device")
 
 
 def _need(t, dtype, shape, name):
@@ -121,6 +134,7 @@ def bl_quantize_weight(W, w_packed, gamma, workspace, stream=None):
     _need(W, W.dtype, (N, K), "W")
     _need(w_packed, torch.uint8, (N, K // 4), "w_packed")
     _need(gamma, torch.float32, (1,), "gamma")
+    _on_current_device(W, w_packed, gamma, workspace)
     wdt = BL_F32 if W.dtype == torch.float32 else BL_BF16
     _check(load_library().bl_quantize_weight(_ptr(W), wdt, N, K, _ptr(w_packed), _ptr(gamma), _ptr(workspace),
                                              workspace.numel() * workspace.element_size(), _stream(stream)),
@@ -133,6 +147,7 @@ def bl_quantize_act(x, xq, sx, stream=None):
     _need(x, torch.bfloat16, (M, K), "x")
     _need(xq, torch.int8, (M, K), "xq")
     _need(sx, torch.float32, (M,), "sx")
+    _on_current_device(x, xq, sx)
     _check(load_library().bl_quantize_act(_ptr(x), M, K, _ptr(xq), _ptr(sx), _stream(stream)), "bl_quantize_act")
 
 
@@ -148,6 +163,7 @@ def bl_quantize(W, x, w_packed, gamma, xq, sx, workspace, stream=None):
     _need(gamma, torch.float32, (1,), "gamma")
     _need(xq, torch.int8, (M, K), "xq")
     _need(sx, torch.float32, (M,), "sx")
+    _on_current_device(W, x, w_packed, gamma, xq, sx, workspace)
     wdt = BL_F32 if W.dtype == torch.float32 else BL_BF16
     _check(load_library().bl_quantize(_ptr(W), wdt, N, K, _ptr(x), M, _ptr(w_packed), _ptr(gamma), _ptr(xq),
                                       _ptr(sx), _ptr(workspace), workspace.numel() * workspace.element_size(),
@@ -166,6 +182,7 @@ def bl_forward(xq, sx, w_packed, gamma, y, debug_acc=None, stream=None):
     _need(y, torch.bfloat16, (M, N), "y")
     if debug_acc is not None:
         _need(debug_acc, torch.int32, (M, N), "debug_acc")
+    _on_current_device(xq, sx, w_packed, gamma, y, debug_acc)
     _check(load_library().bl_forward(_ptr(xq), _ptr(sx), _ptr(w_packed), _ptr(gamma), M, N, K, _ptr(y),
                                      _ptr(debug_acc), _stream(stream)), "bl_forward")
 
@@ -187,6 +204,7 @@ def bl_backward(dY, xq, sx, w_packed, gamma, dX=None, dW=None, accumulate_dW=Fal
             raise ValueError("dW must be bf16 or f32")
         _need(dW, dW.dtype, (N, K), "dW")
         dwdt = BL_F32 if dW.dtype == torch.float32 else BL_BF16
+    _on_current_device(dY, xq, sx, w_packed, gamma, dX, dW)
     _check(load_library().bl_backward(_ptr(dY), _ptr(xq), _ptr(sx), _ptr(w_packed), _ptr(gamma), M, N, K,
                                       _ptr(dX), _ptr(dW), dwdt, int(bool(accumulate_dW)), _stream(stream)),
            "bl_backward")
@@ -199,6 +217,7 @@ def bl_sign_pack(dW, sign_words, stream=None):
         raise ValueError("dW must be bf16 or f32")
     _need(dW, dW.dtype, (N, K), "dW")
     _need(sign_words, torch.int32, (N, K // 32), "sign_words")
+    _on_current_device(dW, sign_words)
     dt = BL_F32 if dW.dtype == torch.float32 else BL_BF16
     _check(load_library().bl_sign_pack(_ptr(dW), dt, N, K, _ptr(sign_words), _stream(stream)), "bl_sign_pack")
 
@@ -208,6 +227,7 @@ def bl_sign_vote(sign_words, direction, stream=None):
     R, N, KW = sign_words.shape
     _need(sign_words, torch.int32, (R, N, KW), "sign_words")
     _need(direction, torch.uint8, (N, KW * 8), "direction")
+    _on_current_device(sign_words, direction)
     _check(load_library().bl_sign_vote(_ptr(sign_words), R, N, KW * 32, _ptr(direction), _stream(stream)),
            "bl_sign_vote")
 
@@ -219,6 +239,7 @@ def bl_signsgd_update(W, direction, lr, stream=None):
         raise ValueError("W must be bf16 or f32")
     _need(W, W.dtype, (N, K), "W")
     _need(direction, torch.uint8, (N, K // 4), "direction")
+    _on_current_device(W, direction)
     dt = BL_F32 if W.dtype == torch.float32 else BL_BF16
     _check(load_library().bl_signsgd_update(_ptr(W), dt, N, K, _ptr(direction), float(lr), _stream(stream)),
            "bl_signsgd_update")

@@ -6,7 +6,6 @@
 #include <cstdarg>
 #include <cstdint>
 #include <cstdio>
-#include <mutex>
 
 #include "../../include/bitlinear.h"
 #include "bl_internal.h"
@@ -27,18 +26,14 @@ bl_status fail(bl_status s, const char* fmt, ...) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-// Device address of the error word, looked up once per device.
-int* device_error_ptr(int dev) {
-  static int* ptrs[64] = {};
-  static std::mutex mu;
-  if (dev < 0 || dev >= 64) return nullptr;
-  std::lock_guard<std::mutex> lock(mu);
-  if (!ptrs[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return nullptr;
-    ptrs[dev] = static_cast<int*>(p);
-  }
-  return ptrs[dev];
+// Device address of the error word on the current device. Looked up on every
+// call (a host-side table lookup once the module is loaded): a cached address
+// would go stale if the caller reset the device and the module were loaded
+// again at another address.
+int* device_error_ptr() {
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return nullptr;
+  return static_cast<int*>(p);
 }
 
 // Checks the current device is sm_100 and returns its error word.
@@ -54,7 +49,7 @@ bl_status current_device(int** err) {
     arch_ok[dev] = (major == 10 && minor == 0) ? 1 : 2;
   }
   if (arch_ok[dev] != 1) return fail(BL_ERR_ARCH, "device %d is not sm_100", dev);
-  *err = device_error_ptr(dev);
+  *err = device_error_ptr();
   if (!*err) return fail(BL_ERR_CUDA, "cannot resolve the device error word");
   return BL_OK;
 }

@@ -14,7 +14,6 @@
 
 #include <algorithm>
 #include <cstdint>
-#include <mutex>
 
 #include "bl_device.cuh"
 #include "bl_internal.h"
@@ -549,23 +548,16 @@ cudaError_t launch_quantize_weight(const void* W, int w_is_f32, int64_t N, int64
 size_t noalloc_scratch_bytes() { return sizeof(g_noalloc_partials); }
 
 // Device address of g_noalloc_partials on the current device. Host code only
-// holds a stand-in for the array's name, so the address is looked up once per
-// device (with that device current) and cached.
+// holds a stand-in for the array's name, so the address is looked up with the
+// device current, on every call: a cached address would go stale if the
+// caller reset the device and the module were loaded again elsewhere. The
+// first lookup on a device loads the module there (so it belongs before any
+// stream capture); later ones are host-side table lookups.
 static cudaError_t noalloc_scratch_ptr(double** out) {
-  static double* ptrs[64] = {};
-  static std::mutex mu;
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
+  void* p = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_partials);
   if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  std::lock_guard<std::mutex> lock(mu);
-  if (!ptrs[dev]) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_noalloc_partials);
-    if (e != cudaSuccess) return e;
-    ptrs[dev] = static_cast<double*>(p);
-  }
-  *out = ptrs[dev];
+  *out = static_cast<double*>(p);
   return cudaSuccess;
 }
 

@@ -59,25 +59,42 @@ class BitLinearStack:
         s.grad = [torch.empty(big, dtype=torch.bfloat16, device=device) for _ in range(2)]
         return s
 
-    def forward(self, x, weights, stream=None):
+    def forward(self, x, weights, stream=None, on_layer=None):
         """x [M, dims[0]] bf16, weights[l] [dims[l+1], dims[l]]: returns the last
-        layer's output (a view of an internal buffer)."""
+        layer's output (a view of an internal buffer). ``on_layer(l, y)``, if
+        given, is called after layer l with its output (a view that the next
+        layer but one overwrites)."""
         h = x
         for i, (L, W) in enumerate(zip(self.layers, weights)):
             y = self.act[i % 2][: self.M * L.N].view(self.M, L.N)
             b.bl_quantize(W, h, L.w_packed, L.gamma, L.xq, L.sx, L.workspace, stream)
             b.bl_forward(L.xq, L.sx, L.w_packed, L.gamma, y, None, stream)
+            if on_layer is not None:
+                on_layer(i, y)
             h = y
         return h
 
-    def backward(self, dY, input_grad=True, stream=None):
+    def backward(self, dY, input_grad=True, stream=None, on_layer=None):
         """dY [M, dims[-1]] bf16: fills every layer's dW; returns dX of the first
-        layer (a view of an internal buffer) or None when input_grad is False."""
+        layer (a view of an internal buffer) or None when input_grad is False.
+        ``on_layer(l, dy, dx)``, if given, is called after layer l with the
+        output gradient it was given and its input gradient (views of internal
+        buffers, or None for the first layer's dx when it is not wanted)."""
         g = dY
         for i in range(len(self.layers) - 1, -1, -1):
             L = self.layers[i]
             want_dx = input_grad or i > 0
             dX = self.grad[i % 2][: self.M * L.K].view(self.M, L.K) if want_dx else None
             b.bl_backward(g, L.xq, L.sx, L.w_packed, L.gamma, dX, L.dW, False, stream)
+            if on_layer is not None:
+                on_layer(i, g, dX)
             g = dX
         return g
+
+    @staticmethod
+    def check():
+        """Synchronises the device and raises if a kernel recorded a device
+        failure (a bounded pipeline wait that gave up) since the last reset."""
+        status = b.bl_get_last_error()
+        if status != 0:
+            raise b.BitLinearError(status, "BitLinearStack", "device error word set")

@@ -40,3 +40,22 @@ def test_adamw_steps_agree():
         lm_ref.adamw_step(p2, grads, s2, step, cfg)
     for k in p1:
         assert torch.allclose(p1[k], p2[k], rtol=1e-14, atol=1e-15)
+
+
+def test_single_rounding_to_bf16_matches_oracle():
+    """The LM's fp64 -> bf16 cast (one rounding) against the oracle's."""
+    import numpy as np
+    from oracle import bitlinear_ref as ref
+    from ternary_weight_quantization_b200.lm import to_bf16_rn
+    rng = np.random.default_rng(11)
+    vals = [rng.standard_normal(20000) * 10.0 ** rng.integers(-30, 30, 20000),
+            rng.standard_normal(2000) * 1e-39, rng.standard_normal(2000) * 1e-44]
+    # values just above and below bf16 ties, where rounding through fp32 first
+    # would land on the tie and round to even instead of away
+    base = (rng.integers(0x0080, 0x7F00, 4000).astype(np.uint32) << 16) | 0x8000   # finite fp32 bf16 ties
+    ties = base.view(np.float32).astype(np.float64)
+    vals += [ties * (1 + 2.0 ** -30), ties * (1 - 2.0 ** -30), ties, -ties * (1 + 2.0 ** -30)]
+    vals.append(np.array([0.0, -0.0, 1.0 + 2.0 ** -8 + 2.0 ** -30, 2.0 ** -126, -2.0 ** -127, 2.0 ** -133 * 1.5]))
+    x = np.concatenate(vals)
+    got = to_bf16_rn(torch.from_numpy(x)).view(torch.int16).numpy().view(np.uint16)
+    np.testing.assert_array_equal(got, ref.round_to_bf16_bits(x))

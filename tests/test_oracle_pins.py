@@ -354,6 +354,106 @@ def test_worked_example_sign_equality():
         assert same == (printed[f"layer{i + 1}_sign_equality"][0] == "True")
 
 
+def _page_listing_net(W, x0, target):
+    """The 3-layer net of "1BitTraining.md" as its listing computes it,
+    restated here: its quantisers return the dequantised values (activations
+    scaled by 127 / max(max|x|, 1e-5) along the last axis, rounded, clipped
+    to [-128, 127] and scaled back; weights multiplied by 1 / max(mean|w|,
+    1e-5), rounded, clipped to [-1, 1] and scaled back), the forward uses only
+    quantised weights and activations with no quantiser on the output, the
+    loss is half the squared error, and the backward takes the quantisers'
+    derivative as 1. Returns (loss, deltas, grads, codes, int8 codes), layer
+    by layer from the input."""
+    def act(x):
+        s = 127.0 / np.maximum(np.abs(x).max(axis=-1, keepdims=True), 1e-5)
+        r = np.clip(np.round(x * s), -128, 127)
+        return r / s, r
+
+    def wq(w):
+        s = 1.0 / max(float(np.mean(np.abs(w))), 1e-5)
+        r = np.clip(np.round(w * s), -1, 1)
+        return r / s, r
+
+    Qs, codes = zip(*(wq(w) for w in W))
+    acts, ints = [], []
+    h = x0
+    for Q in Qs:
+        a, r = act(h)
+        acts.append(a)
+        ints.append(r)
+        h = a @ Q.T
+    delta = h - target
+    loss = 0.5 * float(np.sum(delta * delta))
+    deltas, grads = [None] * 3, [None] * 3
+    for i in (2, 1, 0):
+        deltas[i] = delta
+        grads[i] = delta.T @ acts[i]
+        delta = delta @ Qs[i]
+    return loss, deltas, grads, codes, ints
+
+
+def test_worked_example_matches_page_listing():
+    """The oracle-built 3-layer net against the page's own arithmetic: its
+    quantisers (reciprocal weight scale, -128 clip) give the same codes, and
+    the loss, every delta and every grad_Q agree to 1e-12 relative."""
+    rs = np.random.RandomState(0)
+    W = [rs.randn(6, 7), rs.randn(5, 6), rs.randn(4, 5)]
+    x0 = rs.randn(2, 7)
+    target = rs.randn(2, 4)
+    p_loss, p_deltas, p_grads, p_codes, p_ints = _page_listing_net(W, x0, target)
+
+    h = x0
+    saved = []
+    for i, w in enumerate(W):
+        codes, gamma = ref.ternarize(w, np.float64)
+        q, sx = ref.quantize_activations(h, np.float64)
+        np.testing.assert_array_equal(codes, p_codes[i])
+        np.testing.assert_array_equal(q, p_ints[i])
+        saved.append((codes, gamma, ref.dequantize_activations(q, sx, np.float64)))
+        h = ref.forward_output(ref.forward_accumulate(q, codes), sx, gamma, np.float64)
+    delta = h - target
+    assert math.isclose(0.5 * float(np.sum(delta * delta)), p_loss, rel_tol=1e-12)
+    for i in (2, 1, 0):
+        codes, gamma, xh = saved[i]
+        np.testing.assert_allclose(delta, p_deltas[i], rtol=1e-12, atol=1e-14)
+        np.testing.assert_allclose(ref.backward_dw(delta, xh), p_grads[i], rtol=1e-12, atol=1e-14)
+        delta = ref.backward_dx(delta, codes, gamma)
+
+
+def test_dw_accumulation_hand_derived():
+    """bitlinear_step with dw_prev: dW = dw_prev + dY^T x_hat on the dyadic
+    fixture, sums written out by hand (every term exact)."""
+    g = _load_dyadic()
+    x_bits = ref.round_to_bf16_bits(np.array(g["x"], np.float32))
+    dy_bits = ref.round_to_bf16_bits(np.array(g["dY"], np.float32))
+    prev = np.array([[0.25, 3.0, -4.5, -0.5, 1.0, 2.0, -5.0, 0.125],
+                     [-11.875, -246.0, 0.75, 0.0, -0.125, 1.5, 0.5, -1.0]], np.float32)
+    out = ref.bitlinear_step(x_bits, np.array(g["W"], np.float32), dy_bits, w_is_bf16=False, dw_prev=prev)
+    expected = np.array([[34.0, -140.0, 0.0, 0.0, 1.25, 2.0, 0.0, 0.125],
+                         [0.0, 0.0, -7.0, 0.25, 0.0, 1.5, 3.0, -1.0]])
+    np.testing.assert_array_equal(out["dw_f64"], expected)
+    np.testing.assert_array_equal(out["dw_f32"], expected.astype(np.float32))
+    without = ref.bitlinear_step(x_bits, np.array(g["W"], np.float32), dy_bits, w_is_bf16=False)
+    np.testing.assert_array_equal(without["dw_f64"], np.array(g["dW"]))
+
+
+def test_dw_accumulation_loop():
+    """dW[n, k] = dw_prev[n, k] + sum_m dY[m, n] x_hat[m, k], element by element."""
+    rng = np.random.default_rng(12)
+    M, K, N = 6, 32, 5
+    x_bits = ref.round_to_bf16_bits(rng.standard_normal((M, K)))
+    dy_bits = ref.round_to_bf16_bits(rng.standard_normal((M, N)))
+    w = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+    prev = rng.standard_normal((N, K)).astype(np.float32)
+    out = ref.bitlinear_step(x_bits, w, dy_bits, w_is_bf16=False, dw_prev=prev)
+    dy = ref.bf16_bits_to_f32(dy_bits)
+    xh = out["x_hat"]
+    for n in range(N):
+        for k in range(K):
+            s = math.fsum([float(prev[n, k])] + [float(dy[m, n]) * float(xh[m, k]) for m in range(M)])
+            assert math.isclose(out["dw_f64"][n, k], s, rel_tol=1e-12, abs_tol=1e-12)
+
+
 # --------------------------------------------------------------------------
 # the whole step with the product's roundings
 # --------------------------------------------------------------------------
