@@ -16,8 +16,10 @@ dirty line is left) before every step, outside the timed events; each step is br
 stream (the headline); a second pass of K steps puts events between the C-ABI
 calls for the per-kernel times (events between kernels can cost the overlap
 of programmatically dependent launches, so that pass is not the headline). For N > 1
-(torchrun, one rank per GPU) every rank runs its own batch (weak scaling, no
-data-path collective); the job time is the max over ranks.
+(torchrun, one rank per GPU) the step is the data-parallel one: every rank
+runs the path on its own tokens (weak scaling) with the same W, and the
+partial dW are summed over the ranks by an NCCL all-reduce inside the timed
+step (the path's one exchange); the job time is the max over ranks.
 
 `--impl reference` times the CPU oracle (the only reference this path has)
 on a bounded sample of the same workload, on the host cores.
@@ -188,13 +190,17 @@ def stage_work(M, N, K, w_bytes):
 
 def run_ours(args, rank, world, local_rank):
     import ternary_weight_quantization_b200 as bl
+    from ternary_weight_quantization_b200.dp import dp_step
 
     bl.load_library()
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     wl = WORKLOADS[args.workload]
     M, K, N = wl.M, wl.K, wl.N
+    # every rank: its own tokens and output gradients, the same W
     x_cpu, w_cpu, dy_cpu = workload_inputs(args.workload, seed=rank)
+    if rank != 0:
+        w_cpu = workload_inputs(args.workload, seed=0)[1]
     x, w, dy = x_cpu.to(dev), w_cpu.to(dev), dy_cpu.to(dev)
     bufs = bl.StepBuffers.allocate(M, N, K, torch.bfloat16, device=dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
@@ -208,17 +214,20 @@ def run_ours(args, rank, world, local_rank):
         flush.view(torch.int64).max()
 
     def step(evs=None):
-        if evs:
-            evs[0].record(stream)
+        if not evs:
+            dp_step(x, w, dy, bufs, stream=stream)  # world 1: no exchange
+            return
+        evs[0].record(stream)
         bl.bl_quantize(w, x, bufs.w_packed, bufs.gamma, bufs.xq, bufs.sx, bufs.workspace, stream)
-        if evs:
-            evs[1].record(stream)
+        evs[1].record(stream)
         bl.bl_forward(bufs.xq, bufs.sx, bufs.w_packed, bufs.gamma, bufs.y, None, stream)
-        if evs:
-            evs[2].record(stream)
+        evs[2].record(stream)
         bl.bl_backward(dy, bufs.xq, bufs.sx, bufs.w_packed, bufs.gamma, bufs.dX, bufs.dW, False, stream)
-        if evs:
-            evs[3].record(stream)
+        evs[3].record(stream)
+        if world > 1:
+            with torch.cuda.stream(stream):
+                torch.distributed.all_reduce(bufs.dW)
+            evs[4].record(stream)
 
     for i in range(args.warmup):
         flush_l2(i)
@@ -231,7 +240,7 @@ def run_ours(args, rank, world, local_rank):
         """K steps, L2 flushed before each. per_stage: events between the C-ABI
         calls (kernel breakdown); otherwise events only around each step, so
         consecutive kernels keep their programmatic-launch overlap."""
-        n_ev = len(STAGES) + 1 if per_stage else 2
+        n_ev = len(STAGES) + 1 + (world > 1) if per_stage else 2
         evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
         if world > 1:
             torch.distributed.barrier()
@@ -247,11 +256,12 @@ def run_ours(args, rank, world, local_rank):
         torch.cuda.synchronize(dev)
         if world > 1:
             torch.distributed.barrier()
-        per = {s: 0.0 for s in STAGES}
+        names = STAGES + (["allreduce"] if world > 1 else [])
+        per = {s: 0.0 for s in names}
         total = 0.0
         for e in evs:
             if per_stage:
-                for j, st in enumerate(STAGES):
+                for j, st in enumerate(names):
                     per[st] += e[j].elapsed_time(e[j + 1])
             total += e[0].elapsed_time(e[-1])
         return total, per
@@ -300,7 +310,7 @@ def run_ours(args, rank, world, local_rank):
             unit = "TOPS" if wk["dtype"] == "int8" else "TFLOP/s"
             roof_ms += wk["ops"] / (peak * 1e12) * 1e3
         kernels[s] = {"ms": round(ms, 5), "achieved": round(ach, 1), "unit": unit, "peak": peak,
-                      "frac": round(ach / peak, 4), "share": round(per_stage[s] / sum(per_stage.values()), 4),
+                      "frac": round(ach / peak, 4), "share": round(per_stage[s] / sum(per_stage[t] for t in STAGES), 4),
                       "traffic": traffic.get(s)}
     dom = max(STAGES, key=lambda s: per_stage[s])
     dk = kernels[dom]
@@ -319,11 +329,14 @@ def run_ours(args, rank, world, local_rank):
                    "W": f"{'bf16' if wl.w_dtype == torch.bfloat16 else 'f32'} [{N},{K}] {wl.w_init}",
                    "dY": f"bf16 [{M},{N}] N(0,1)", "global_batch_tokens": M * world,
                    "l2": "flushed before every step (256 MiB write then read, outside the timed events)",
-                   "parallelism": f"dp{world} independent replicas" if world > 1 else "single GPU"},
+                   "parallelism": f"dp{world}: token shards, dW all-reduce (NCCL) in the step"
+                   if world > 1 else "single GPU"},
         "roofline": roofline,
         "step_roofline_frac": round(roof_ms / ms_per_step, 4),
         "kernel_breakdown_ms_per_step": round(breakdown_ms / args.steps, 5),
         "kernels": kernels,
+        **({"allreduce_ms_per_step": round(per_stage["allreduce"] / args.steps, 5),
+            "allreduce_bytes": bufs.dW.numel() * bufs.dW.element_size()} if world > 1 else {}),
         "e2e": e2e,
         "gpu_launches": LAUNCHES_PER_STEP * args.steps,
         "clocks": clocks,
@@ -345,11 +358,13 @@ def measure_e2e(bl, args, dev, stream, bufs, x_cpu, w_cpu, dy_cpu, world):
     dy = torch.empty_like(dy_cpu, device=dev)
     steps = max(3, min(args.steps, 20))
 
+    from ternary_weight_quantization_b200.dp import dp_step
+
     def one():
         x.copy_(xh, non_blocking=True)
         w.copy_(wh, non_blocking=True)
         dy.copy_(dyh, non_blocking=True)
-        bl.bitlinear_step(x, w, dy, bufs, stream)
+        dp_step(x, w, dy, bufs, stream=stream)
         yh.copy_(bufs.y, non_blocking=True)
         dxh.copy_(bufs.dX, non_blocking=True)
         dwh.copy_(bufs.dW, non_blocking=True)
@@ -686,7 +701,8 @@ def run_signsgd(args, rank, world, local_rank):
 
 def run_lm(args, rank, world, local_rank):
     """Decoder-LM mode: the 4-layer LM of workloads/lm.py trained through the
-    library (every projection a BitLinear call; the rest plain PyTorch) for
+    library (every projection a BitLinear call; the rest plain PyTorch in
+    fp64, the precision the LM oracle keeps it in) for
     its 50 steps on each rank (independent replicas). Reports tokens per
     second (batch x sequence per step over the mean device time of a step,
     the first step excluded) and the largest |loss - oracle loss| over the
@@ -710,7 +726,7 @@ def run_lm(args, rank, world, local_rank):
     tokens = cfg.batch * cfg.seq
     return {"metric": "bitlinear_lm_train_tokens_per_s", "value": round(tokens * world / (job_ms * 1e-3), 1),
             "unit": "tokens/s", "n_gpus": world, "steps": cfg.steps, "warmup": 1, "ms_per_step": round(job_ms, 4),
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8/bf16 BitLinear, fp32 rest",
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8/bf16 BitLinear, fp64 rest",
             "data": "synthetic",
             "config": {"workload": "4-layer decoder LM", "layers": cfg.layers, "d": cfg.d, "heads": cfg.heads,
                        "ffn": cfg.ffn, "vocab": cfg.vocab, "seq": cfg.seq, "batch": cfg.batch, "lr": cfg.lr},
