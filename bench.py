@@ -734,6 +734,43 @@ def run_lm(args, rank, world, local_rank):
             "max_abs_dloss_vs_oracle": None if worst is None else round(worst, 6)}
 
 
+def run_extras(args, local_rank):
+    """The other workloads' lines in short form, measured in the same run on
+    the same GPU (N = 1 only): the down-projection step, the 8-layer stack
+    (step time and peak memory), the few-token forward, the sign-gradient
+    step and the decoder LM (throughput and its largest loss gap to the
+    stored oracle curve). Each keeps its own mode's timing rules with fewer
+    steps; the headline line above is unaffected."""
+    import copy
+    short = copy.copy(args)
+    short.steps, short.warmup = min(args.steps, 20), max(3, min(args.warmup, 5))
+    extras = {}
+
+    def keep(line, keys):
+        return {k: line[k] for k in keys if k in line}
+
+    down = copy.copy(short)
+    down.workload, down.no_cpu_baseline = "down_proj", True
+    line = run_ours(down, 0, 1, local_rank)
+    extras["down_proj"] = keep(line, ["value", "unit", "ms_per_step", "roofline", "kernels", "clocks"])
+    st = copy.copy(short)
+    st.stack = "stack8"
+    line = run_stack(st, 0, 1, local_rank)
+    extras["stack8"] = keep(line, ["value", "unit", "ms_per_step", "peak_device_memory_mb", "saved_state_mb",
+                                   "config", "clocks"])
+    ft = copy.copy(short)
+    ft.few_tokens = "1,2,4,8,16"
+    line = run_few_tokens(ft, 0, 1, local_rank)
+    extras["few_tokens"] = keep(line, ["by_tokens", "peak_gbs", "config"])
+    line = run_signsgd(copy.copy(short), 0, 1, local_rank)
+    extras["signsgd"] = keep(line, ["value", "unit", "ms_per_step", "kernels"])
+    line = run_lm(copy.copy(short), 0, 1, local_rank)
+    extras["lm"] = keep(line, ["value", "unit", "ms_per_step", "loss_first", "loss_last", "max_abs_dloss_vs_oracle",
+                               "dtype"])
+    torch.cuda.empty_cache()
+    return extras
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -751,6 +788,8 @@ def main():
                     help="sign-gradient data-parallel step mode (prints its own line)")
     ap.add_argument("--few-tokens", default=None,
                     help="forward-only mode at these token counts, e.g. 1,8,16 (prints its own line)")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the other workloads' short measurements after the headline (N = 1)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -780,6 +819,8 @@ def main():
             out = run_lm(args, rank, world, local_rank)
         else:
             out = run_ours(args, rank, world, local_rank)
+            if world == 1 and not args.no_extras and out is not None:
+                out["other_workloads"] = run_extras(args, local_rank)
         if rank == 0 and out is not None:
             print(json.dumps(out), flush=True)
     finally:

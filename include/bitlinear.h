@@ -71,8 +71,10 @@ const char* bl_status_string(bl_status status);
 const char* bl_last_error_message(void);
 
 /*
- * Bytes of device workspace bl_quantize_weight needs for an [N,K] tensor
- * (fp64 partial sums of |W|). Returns 0 for an empty tensor.
+ * Bytes of device workspace bl_quantize_weight and bl_quantize need for an
+ * [N,K] tensor: two arrival counters, one fp64 partial sum of |W| per CTA and
+ * 256 exact-sum bins, 10304 bytes for every non-empty tensor. Returns 0 for
+ * an empty tensor.
  */
 size_t bl_quantize_weight_workspace_size(int64_t N, int64_t K);
 
@@ -82,7 +84,7 @@ size_t bl_quantize_weight_workspace_size(int64_t N, int64_t K);
  * intro bullet: one fused ternarise + scale + pack pass, no bf16 fake-quant
  * tensor).
  *
- *   gamma   = max(fp32(sum|W| / (N*K)), 1e-5)   sum in fp64, fixed order
+ *   gamma   = max(fp32(fp64(S / (N*K))), 1e-5)  S = sum|W| rounded once to fp64
  *   code    = clamp(rint_half_even(fp32(W / gamma)), -1, 1)
  *   packing : element k of row n -> byte n*K/4 + k/4, bits 2*(k%4)..+1,
  *             field 00 = 0, 01 = +1, 11 = -1 (10 never written)
@@ -93,7 +95,17 @@ size_t bl_quantize_weight_workspace_size(int64_t N, int64_t K);
  * workspace device scratch of at least bl_quantize_weight_workspace_size(N,K)
  *           bytes, 16-byte aligned; contents need no initialisation and are
  *           overwritten.
- * Deterministic: the same W gives bit-identical outputs on every call.
+ * gamma is exact: the fp64 sum of |W| is taken in a fixed tree and carries a
+ * bounded rounding error; gamma is formed at both ends of that enclosure of
+ * the exact sum, and where the two differ (about one tensor in 10^5) the
+ * library sums |W| exactly in integers and rounds once. gamma therefore never
+ * depends on the summation order or on the GPU, and the same W gives
+ * bit-identical outputs on every call.
+ * Launches: a one-CTA launch that clears the workspace's counters, then one
+ * persistent launch (at most one CTA per SM, all resident at once; they meet
+ * at a grid-wide barrier whose wait is bounded: a barrier that cannot
+ * complete -- e.g. SMs held by other work for seconds -- records
+ * BL_ERR_TIMEOUT in the device error word).
  * Errors: BL_ERR_INVALID_ARG, BL_ERR_UNSUPPORTED_SHAPE (K % 32), BL_ERR_DTYPE,
  *         BL_ERR_ALIGNMENT, BL_ERR_WORKSPACE, BL_ERR_ARCH, BL_ERR_CUDA.
  */
@@ -109,21 +121,22 @@ bl_status bl_quantize_weight(const void* W, bl_dtype w_dtype, int64_t N, int64_t
  * and so cannot pass the workspace bl_quantize_weight asks for.
  *
  * It computes exactly what bl_quantize_weight computes (same kernels, same
- * bit-identical outputs) and calls no allocator. Its fp64 partial sums go to
- * a fixed array inside the library of 296 doubles (2368 bytes), enough for a
- * tensor of any size; each GPU that loads the library keeps that array until
- * the process exits. A request that would need more scratch than the array
- * holds returns BL_ERR_WORKSPACE.
+ * bit-identical outputs) and calls no allocator. Its scratch -- the arrival
+ * counters, partial sums and exact-sum bins that bl_quantize_weight keeps in
+ * the caller's workspace -- is a fixed array inside the library of 10304
+ * bytes, enough for a tensor of any size; each GPU that loads the library
+ * keeps that array until the process exits.
  *
  * Each call looks up the array's device address on the current device (a
  * runtime query; the first one on a device loads the library's device code
  * there, so make the first call on each device before any stream capture).
  * The address is not cached, so a call after the caller reset the device
- * finds the array where the reloaded device code put it. All calls share the one array and
- * nothing in it needs to start at zero (every call overwrites the part it
- * reads), but two calls whose kernels overlap on the GPU -- on different
- * streams of one device without ordering between them -- race on it and may
- * produce wrong codes: order them on one stream or with events.
+ * finds the array where the reloaded device code put it. All calls share the
+ * one array and nothing in it needs to start at zero (each call clears its
+ * counters and bins before use and overwrites the rest), but two calls whose
+ * kernels overlap on the GPU -- on different streams of one device without
+ * ordering between them -- race on it and may produce wrong codes or a
+ * barrier timeout: order them on one stream or with events.
  *
  * Arguments, outputs and errors: as bl_quantize_weight, without the
  * workspace pair.
@@ -148,9 +161,9 @@ bl_status bl_quantize_act(const void* x, int64_t M, int64_t K,
 /*
  * S1 + S2 in one call: the same outputs as bl_quantize_weight(W, ...) followed
  * by bl_quantize_act(x, ...), bit for bit. The two steps are independent, so
- * S2 runs beside the |W| partial sums of S1 and their memory traffic
- * overlaps; S1's code pass follows in S2's launch. (The pages run the two
- * quantisers one after the other; this is a scheduling choice only.)
+ * S2 runs in the same persistent launch as S1, on other warps, while W is
+ * copied into shared memory and summed. (The pages run the two quantisers
+ * one after the other; this is a scheduling choice only.)
  *
  * Arguments: those of bl_quantize_weight and bl_quantize_act. M == 0 skips
  * S2 (x, xq, sx may then be NULL). Errors: as bl_quantize_weight, plus those

@@ -93,7 +93,7 @@ const char* bl_last_error_message(void) { return g_msg; }
 
 size_t bl_quantize_weight_workspace_size(int64_t N, int64_t K) {
   if (N <= 0 || K <= 0) return 0;
-  return static_cast<size_t>(bl::weight_partials_count(N * K)) * sizeof(double);
+  return bl::quantize_workspace_bytes();
 }
 
 bl_status bl_quantize_weight(const void* W, bl_dtype w_dtype, int64_t N, int64_t K, uint8_t* w_packed,
@@ -110,8 +110,7 @@ bl_status bl_quantize_weight(const void* W, bl_dtype w_dtype, int64_t N, int64_t
     return fail(BL_ERR_WORKSPACE, "workspace needs %zu bytes, 16-byte aligned", need);
   int* err = nullptr;
   if (bl_status s = current_device(&err)) return s;
-  return cuda_status(bl::launch_quantize_weight(W, w_dtype == BL_F32, N, K, w_packed, gamma,
-                                                static_cast<double*>(workspace),
+  return cuda_status(bl::launch_quantize_weight(W, w_dtype == BL_F32, N, K, w_packed, gamma, workspace, err,
                                                 static_cast<cudaStream_t>(stream)),
                      "bl_quantize_weight launch");
 }
@@ -125,13 +124,9 @@ bl_status bl_quantize_weight_noalloc(const void* W, bl_dtype w_dtype, int64_t N,
   if (!W || !w_packed || !gamma) return fail(BL_ERR_INVALID_ARG, "null pointer");
   if (!aligned16(W) || !aligned16(w_packed) || !aligned16(gamma))
     return fail(BL_ERR_ALIGNMENT, "W, w_packed and gamma must be 16-byte aligned");
-  const size_t need = bl_quantize_weight_workspace_size(N, K);
-  if (need > bl::noalloc_scratch_bytes())
-    return fail(BL_ERR_WORKSPACE, "needs %zu bytes of scratch; the built-in scratch holds %zu", need,
-                bl::noalloc_scratch_bytes());
   int* err = nullptr;
   if (bl_status s = current_device(&err)) return s;
-  return cuda_status(bl::launch_quantize_weight_noalloc(W, w_dtype == BL_F32, N, K, w_packed, gamma,
+  return cuda_status(bl::launch_quantize_weight_noalloc(W, w_dtype == BL_F32, N, K, w_packed, gamma, err,
                                                         static_cast<cudaStream_t>(stream)),
                      "bl_quantize_weight_noalloc launch");
 }
@@ -168,8 +163,8 @@ bl_status bl_quantize(const void* W, bl_dtype w_dtype, int64_t N, int64_t K, con
     return fail(BL_ERR_WORKSPACE, "workspace needs %zu bytes, 16-byte aligned", need);
   int* err = nullptr;
   if (bl_status s = current_device(&err)) return s;
-  return cuda_status(bl::launch_quantize(W, w_dtype == BL_F32, N, K, x, M, w_packed, gamma,
-                                         static_cast<double*>(workspace), xq, sx, static_cast<cudaStream_t>(stream)),
+  return cuda_status(bl::launch_quantize(W, w_dtype == BL_F32, N, K, x, M, w_packed, gamma, workspace, xq, sx, err,
+                                         static_cast<cudaStream_t>(stream)),
                      "bl_quantize launch");
 }
 

@@ -26,30 +26,32 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
   return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
 }
 
-// ---- S1: absmean ternarisation + 2-bit packing
-// Number of fp64 partial sums pass A writes for a tensor of `numel` elements
-// (a fixed function of numel, so the reduction order never depends on the GPU).
-int weight_partials_count(int64_t numel);
+// ---- S1: absmean ternarisation + 2-bit packing (with S2 in the same launch)
+// Most CTAs of one quantisation launch (one per SM at most; they meet at a
+// grid-wide barrier, so all must be resident together).
+constexpr int kMaxQuantCtas = 1024;
 
-// Pass A (|W| partial sums) + the code pass (gamma, codes, packing).
-// `partials` holds weight_partials_count(N*K) doubles.
-cudaError_t launch_quantize_weight(const void* W, int w_is_f32, int64_t N, int64_t K, uint8_t* packed,
-                                   float* gamma, double* partials, cudaStream_t s);
+// Bytes of the S1 workspace (arrival counters, one fp64 partial sum per CTA,
+// exact-sum bins); the same for every tensor size. Needs no initialisation.
+size_t quantize_workspace_bytes();
 
-// Same two passes with the partial sums in a fixed device array
-// (g_noalloc_partials in k_quant.cu) instead of a caller workspace.
-cudaError_t launch_quantize_weight_noalloc(const void* W, int w_is_f32, int64_t N, int64_t K, uint8_t* packed,
-                                           float* gamma, cudaStream_t s);
-size_t noalloc_scratch_bytes();
-
-// ---- S2: per-token absmax INT8
-cudaError_t launch_quantize_act(const void* x, int64_t M, int64_t K, int8_t* xq, float* sx, cudaStream_t s);
-
-// ---- S1 + S2 together (bl_quantize): pass A, then one grid holding the
-// activation quantisation (started beside pass A) and the code pass.
-// `partials` as for launch_quantize_weight.
+// S1 on W [N,K] and, when M > 0, S2 on x [M,K] in one launch (after a one-CTA
+// launch that clears the workspace's counters). `err` is the device error
+// word (a barrier wait that gave up records a timeout there).
 cudaError_t launch_quantize(const void* W, int w_is_f32, int64_t N, int64_t K, const void* x, int64_t M,
-                            uint8_t* packed, float* gamma, double* partials, int8_t* xq, float* sx, cudaStream_t s);
+                            uint8_t* packed, float* gamma, void* workspace, int8_t* xq, float* sx, int* err,
+                            cudaStream_t s);
+
+// S1 alone (launch_quantize with M = 0).
+cudaError_t launch_quantize_weight(const void* W, int w_is_f32, int64_t N, int64_t K, uint8_t* packed,
+                                   float* gamma, void* workspace, int* err, cudaStream_t s);
+
+// S1 with the workspace in a fixed device array (g_noalloc_ws in k_quant.cu).
+cudaError_t launch_quantize_weight_noalloc(const void* W, int w_is_f32, int64_t N, int64_t K, uint8_t* packed,
+                                           float* gamma, int* err, cudaStream_t s);
+
+// ---- S2 alone: per-token absmax INT8
+cudaError_t launch_quantize_act(const void* x, int64_t M, int64_t K, int8_t* xq, float* sx, cudaStream_t s);
 
 // ---- S3 / S4 GEMMs (tcgen05)
 cudaError_t launch_forward(const int8_t* xq, const float* sx, const uint8_t* w_packed, const float* gamma,

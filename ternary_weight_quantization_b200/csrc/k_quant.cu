@@ -1,18 +1,34 @@
 // S1 and S2 of the BitLinear hot path on sm_100a: absmean ternarisation with
 // 2-bit packing, and per-token absmax INT8 activation quantisation.
 //
-// Both are HBM-bound streaming passes with 16-byte vector loads and no
-// intermediate tensors in device memory. S1 needs gamma before any code, so
-// it is two passes over W: pass A (fp64 partial sums of |W|) and the code
-// pass (gamma from the partials, codes packed 4 per byte). bl_quantize runs
-// pass A (quant_pass_a_kernel), then one grid (quant_phase2_kernel) whose
-// token blocks -- S2, independent of S1 -- start beside pass A and whose
-// code-pass blocks wait for it; bl_quantize_weight and bl_quantize_act launch
-// the same arithmetic separately.
+// S1 needs the mean |W| of the whole tensor before any code can be written,
+// and S2 is independent of it. One persistent launch does both with W read
+// from HBM once: each CTA (at most one per SM, all resident together) copies
+// its contiguous slice of W into shared memory with bulk asynchronous copies
+// (TMA, issued all at once at entry), sums |W| of the slice in fp64 as the
+// copies land, publishes the partial sum and meets the other CTAs at a
+// grid-wide barrier (a counter in the workspace, bounded wait); then every
+// CTA forms gamma from all partial sums in one fixed order and writes the
+// codes of its slice from shared memory. The part of a slice that does not
+// fit in shared memory is summed from registers and read again (from L2) for
+// its codes. Other warps of the same CTAs quantise the tokens (S2) while the
+// slice copies are in flight. A one-thread launch before it clears the
+// workspace's counters, so the caller's workspace needs no initialisation.
+//
+// gamma = max(fp32(fp64(fp64(S) / numel)), 1e-5) with S = sum |W| (exactly
+// rounded to fp64, "1BitTraining.md" weight_quant / "bitlinear.py"
+// ternary_quantize with the fp64 accumulation the reading fixes). The fp64
+// tree sum carries a bounded rounding error, so gamma is formed at both ends
+// of an enclosure of S; as the chain of roundings is monotone, when the two
+// agree that value is the exact gamma (all but about one tensor in 10^5).
+// Otherwise the CTAs compute S exactly -- integer sums of the significands
+// per exponent field, combined as one wide integer and rounded once -- so
+// gamma never depends on the reduction order or on the GPU's SM count.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <cmath>
 #include <cstdint>
 
 #include "bl_device.cuh"
@@ -21,290 +37,248 @@
 namespace bl {
 namespace {
 
-constexpr int kQuantThreads = 256;
-// Upper bound on pass-A blocks: two 256-thread blocks per SM on a 148-SM
-// B200. A fixed constant, so the fp64 reduction tree is the same on any GPU.
-constexpr int kMaxPartials = 296;
-
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
-// A "group" is 16 consecutive elements of the flattened [N,K] tensor. Its 16
-// codes pack into one 32-bit word: element i of the group sits at bits 2i..2i+1
-// (little-endian, so byte j of the word holds elements 4j..4j+3, LSB first).
-template <bool kF32>
-struct Group {
-  static constexpr int kVecs = kF32 ? 4 : 2;  // uint4 per 16 elements
-  uint4 v[kVecs];
+// ---------------------------------------------------------------- S1 geometry
+constexpr int kQThreads = 512;                 // 16 warps per CTA
+constexpr int kQWarps = kQThreads / 32;
+constexpr int kTokenWarp0 = 8;                 // with tokens: warps 8..15 run S2
+constexpr int kChunkBytes = 16384;             // one bulk copy of the slice
+constexpr int kMaxOnchipBytes = 220 * 1024;    // slice bytes held in shared memory
+constexpr int kMaxChunks = kMaxOnchipBytes / kChunkBytes + 1;
+constexpr int kBarWarpsNamed = 1;              // named barrier id of the slice warps
 
-  __device__ __forceinline__ void load(const uint4* __restrict__ base, int64_t g) {
-#pragma unroll
-    for (int i = 0; i < kVecs; ++i) v[i] = __ldg(base + g * kVecs + i);
-  }
+// Workspace: [0, 8) two arrival counters; [64, 64 + 8 kMaxCtas) fp64 partial
+// sums, one per CTA; then 256 uint64 exact-sum bins (one per exponent field).
+constexpr size_t kWsPartials = 64;
+constexpr size_t kWsBins = kWsPartials + 8 * static_cast<size_t>(kMaxQuantCtas);
+constexpr size_t kWsBytes = kWsBins + 8 * 256;
 
-  // Element i (0..15) as fp32.
-  __device__ __forceinline__ float elem(int i) const {
-    if constexpr (kF32) {
-      const uint4& q = v[i >> 2];
-      const uint32_t w = (i & 3) == 0 ? q.x : (i & 3) == 1 ? q.y : (i & 3) == 2 ? q.z : q.w;
-      return __uint_as_float(w);
-    } else {
-      const uint4& q = v[i >> 3];
-      const int j = (i & 7) >> 1;
-      const uint32_t w = j == 0 ? q.x : j == 1 ? q.y : j == 2 ? q.z : q.w;
-      return (i & 1) ? bf16_hi(w) : bf16_lo(w);
-    }
-  }
-};
-
+// ---------------------------------------------------------------- |W| in fp64
 // |w| widened to fp64 exactly from its bit pattern with the sign cleared.
-// Zero and normal values take integer arithmetic only (a bf16's fp64 high
-// word is b * 2^13 + 0x38000000: exponent re-bias 127 -> 1023; an fp32's is
-// (b >> 3) + 0x38000000 with low word b << 29), leaving the conversion pipe
-// free. Subnormals (nonzero with a zero exponent field) are converted with
-// the conversion instruction on a separate, rarely taken path. Inputs are
-// finite.
-__device__ __forceinline__ uint32_t abs_bits(float x) { return __float_as_uint(x) & 0x7FFFFFFFu; }
-
-__device__ __forceinline__ double normal_abs_to_f64(uint32_t b32) {
-  if (b32 == 0) return 0.0;
-  return __hiloint2double(static_cast<int>((b32 >> 3) + 0x38000000u), static_cast<int>(b32 << 29));
-}
-
-__device__ __forceinline__ bool is_subnormal(uint32_t b32) { return b32 - 1u < 0x007FFFFFu; }
-
-// acc + sum of |element| over one group, in element order.
-// bf16 groups whose 16 magnitudes all have a nonzero exponent field (no zero,
-// no subnormal) take a short path: one packed 16-bit minimum per word finds
-// them, and each fp64 high word is the 15-bit magnitude shifted into place
-// plus the re-biased exponent offset. Other groups, and fp32 groups, take the
-// per-element path below. Both give the same fp64 values in the same order.
-template <bool kF32>
-__device__ __forceinline__ double add_group(double acc, const Group<kF32>& a) {
-  if constexpr (!kF32) {
-    const uint32_t w[8] = {a.v[0].x, a.v[0].y, a.v[0].z, a.v[0].w, a.v[1].x, a.v[1].y, a.v[1].z, a.v[1].w};
-    uint32_t mn = 0xFFFFFFFFu;  // per half: smallest 15-bit magnitude
+// Normal values take integer arithmetic only (a bf16's fp64 high word is
+// b * 2^13 + 0x38000000: exponent re-bias 127 -> 1023; an fp32's is
+// (b >> 3) + 0x38000000 with low word b << 29); zeros and subnormals (zero
+// exponent field) take a separate, rarely taken path. Inputs are finite.
+//
+// 8 bf16 magnitudes of one 16-byte vector, added to acc in element order.
+__device__ __forceinline__ double add_abs8_bf16(double acc, const uint4& v) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  uint32_t mn = 0xFFFFFFFFu;  // per half: smallest 15-bit magnitude
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const uint32_t m = w[j] & 0x7FFF7FFFu;
-      asm("min.u16x2 %0, %0, %1;" : "+r"(mn) : "r"(m));
-    }
-    if (min(mn << 16, mn & 0xFFFF0000u) >= 0x00800000u) {
-      // element 2j is the low half of word j, element 2j + 1 the high half
+  for (int j = 0; j < 4; ++j) asm("min.u16x2 %0, %0, %1;" : "+r"(mn) : "r"(w[j] & 0x7FFF7FFFu));
+  if (min(mn << 16, mn & 0xFFFF0000u) >= 0x00800000u) {
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        acc = __dadd_rn(acc, __hiloint2double(static_cast<int>(((w[j] & 0x7FFFu) << 13) + 0x38000000u), 0));
-        acc = __dadd_rn(acc, __hiloint2double(static_cast<int>(((w[j] & 0x7FFF0000u) >> 3) + 0x38000000u), 0));
-      }
-      return acc;
+    for (int j = 0; j < 4; ++j) {
+      acc = __dadd_rn(acc, __hiloint2double(static_cast<int>(((w[j] & 0x7FFFu) << 13) + 0x38000000u), 0));
+      acc = __dadd_rn(acc, __hiloint2double(static_cast<int>(((w[j] & 0x7FFF0000u) >> 3) + 0x38000000u), 0));
     }
+    return acc;
   }
-  bool sub = false;
 #pragma unroll
-  for (int i = 0; i < 16; ++i) sub |= is_subnormal(abs_bits(a.elem(i)));
-  if (sub) {
-#pragma unroll
-    for (int i = 0; i < 16; ++i) acc = __dadd_rn(acc, static_cast<double>(__uint_as_float(abs_bits(a.elem(i)))));
-  } else {
-#pragma unroll
-    for (int i = 0; i < 16; ++i) acc = __dadd_rn(acc, normal_abs_to_f64(abs_bits(a.elem(i))));
+  for (int j = 0; j < 4; ++j) {
+    acc = __dadd_rn(acc, static_cast<double>(fabsf(bf16_lo(w[j]))));
+    acc = __dadd_rn(acc, static_cast<double>(fabsf(bf16_hi(w[j]))));
   }
   return acc;
 }
 
-
-// ---------------------------------------------------------------- S1 pass A
-// partials[b] = sum of |w| over block b's contiguous range of groups, fp64.
-// Each thread keeps four accumulators (group u of every four goes to
-// accumulator u; leftover groups to accumulator 0), adds them as
-// (a0 + a1) + (a2 + a3), then a fixed shuffle/smem tree. The groups are
-// loaded kLoad at a time (4 or 2), the next batch while the current one is
-// summed; the order of the additions does not depend on kLoad.
-template <bool kF32, int kLoad>
-__device__ __forceinline__ void absmean_block(const uint4* __restrict__ W, int64_t ngroups, int64_t per_block,
-                                              int64_t block, double* __restrict__ partials) {
-  static_assert(kLoad == 2 || kLoad == 4, "batches split a quad of groups");
-  constexpr int T = kQuantThreads;
-  constexpr int kPerQuad = 4 / kLoad;
-  const int64_t g0 = block * per_block;
-  const int64_t g1 = min(g0 + per_block, ngroups);
-  double acc[4] = {0.0, 0.0, 0.0, 0.0};
-  const int64_t gt = g0 + threadIdx.x;
-  // full quads of this thread: groups gt + (4q + u) T, u = 0..3, all < g1
-  const int64_t nquads = gt + 3 * T < g1 ? (g1 - 1 - 3 * T - gt) / (4 * T) + 1 : 0;
-  const int64_t nbatch = nquads * kPerQuad;
-  if (nbatch > 0) {
-    Group<kF32> a[kLoad];
+// 4 fp32 magnitudes of one 16-byte vector, added to acc in element order.
+__device__ __forceinline__ double add_abs4_f32(double acc, const uint4& v) {
+  const uint32_t w[4] = {v.x & 0x7FFFFFFFu, v.y & 0x7FFFFFFFu, v.z & 0x7FFFFFFFu, v.w & 0x7FFFFFFFu};
+  if (min(min(w[0], w[1]), min(w[2], w[3])) >= 0x00800000u) {
 #pragma unroll
-    for (int v = 0; v < kLoad; ++v) a[v].load(W, gt + v * T);
-    for (int64_t b = 0; b < nbatch; ++b) {
-      const int64_t bn = b + 1;
-      Group<kF32> nxt[kLoad];
-      if (bn < nbatch) {
-        const int64_t base = gt + (bn / kPerQuad) * 4 * T + (bn % kPerQuad) * kLoad * T;
-#pragma unroll
-        for (int v = 0; v < kLoad; ++v) nxt[v].load(W, base + v * T);
-      }
-      const int u0 = static_cast<int>(b % kPerQuad) * kLoad;
-#pragma unroll
-      for (int v = 0; v < kLoad; ++v) {
-        if constexpr (kLoad == 4) {
-          acc[v] = add_group(acc[v], a[v]);
-        } else {
-          // accumulator u0 + v (u0 is 0 or 2)
-          if (u0 == 0) acc[v] = add_group(acc[v], a[v]);
-          else acc[2 + v] = add_group(acc[2 + v], a[v]);
-        }
-      }
-#pragma unroll
-      for (int v = 0; v < kLoad; ++v) a[v] = nxt[v];
-    }
+    for (int j = 0; j < 4; ++j)
+      acc = __dadd_rn(acc, __hiloint2double(static_cast<int>((w[j] >> 3) + 0x38000000u), static_cast<int>(w[j] << 29)));
+    return acc;
   }
-  for (int64_t g = gt + nquads * 4 * T; g < g1; g += T) {
-    Group<kF32> a;
-    a.load(W, g);
-    acc[0] = add_group(acc[0], a);
-  }
-  double t = __dadd_rn(__dadd_rn(acc[0], acc[1]), __dadd_rn(acc[2], acc[3]));
 #pragma unroll
-  for (int off = 16; off > 0; off >>= 1) t = __dadd_rn(t, __shfl_xor_sync(0xffffffffu, t, off));
-  __shared__ double warp_sums[kQuantThreads / 32];
-  if ((threadIdx.x & 31) == 0) warp_sums[threadIdx.x >> 5] = t;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    double sum = 0.0;
-#pragma unroll
-    for (int w = 0; w < kQuantThreads / 32; ++w) sum = __dadd_rn(sum, warp_sums[w]);
-    partials[block] = sum;
-  }
+  for (int j = 0; j < 4; ++j) acc = __dadd_rn(acc, static_cast<double>(__uint_as_float(w[j])));
+  return acc;
 }
 
 template <bool kF32>
-__global__ void __launch_bounds__(kQuantThreads) absmean_partials_kernel(const uint4* __restrict__ W,
-                                                                         int64_t ngroups, int64_t per_block,
-                                                                         double* __restrict__ partials) {
-  pdl_wait_primary();       // W may come from the previous kernel (e.g. an optimizer step)
-  pdl_launch_dependents();  // the code pass may start loading W while this pass finishes
-  absmean_block<kF32, 4>(W, ngroups, per_block, blockIdx.x, partials);
+__device__ __forceinline__ double add_abs(double acc, const uint4& v) {
+  if constexpr (kF32) return add_abs4_f32(acc, v);
+  else return add_abs8_bf16(acc, v);
 }
 
-// ---------------------------------------------------------------- S1 code pass
-// Launched as a programmatic dependent of pass A: each thread first loads its
-// first groups of W (pass A only started after W's producer finished, and it
-// does not write W), then waits for pass A,
-// then every block reduces the partials in the same fixed order (so all
-// blocks hold the same gamma) and writes the codes of its range of groups.
-//
+// Exact-sum bins: bin e collects the integer significands (hidden bit
+// included; none for e = 0) of the elements whose exponent field is e, so
+// that sum |W| = sum_e bin[e] * 2^(max(e, 1) - 127 - p), p = 7 (bf16) or 23.
+template <bool kF32>
+__device__ __forceinline__ void bin_abs(unsigned long long* bins, const uint4& v) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    if constexpr (kF32) {
+      const uint32_t b = w[j] & 0x7FFFFFFFu, e = b >> 23, m = (b & 0x7FFFFFu) | (e ? 0x800000u : 0u);
+      if (m) atomicAdd(&bins[e], static_cast<unsigned long long>(m));
+    } else {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const uint32_t b = (w[j] >> (16 * h)) & 0x7FFFu, e = b >> 7, m = (b & 0x7Fu) | (e ? 0x80u : 0u);
+        if (m) atomicAdd(&bins[e], static_cast<unsigned long long>(m));
+      }
+    }
+  }
+}
+
+// S = sum_e bins[e] * 2^(max(e, 1) - 127 - p), rounded once to fp64 (to
+// nearest, ties to even). The bins are added as one unsigned integer of six
+// 64-bit limbs, V = sum_e bins[e] << (max(e, 1) - 1), so S = V * 2^(-126 - p);
+// V's top 53 bits are then rounded with the round and sticky bits below.
+__device__ double exact_sum_from_bins(const unsigned long long* bins, int p) {
+  unsigned long long limb[6] = {0, 0, 0, 0, 0, 0};
+  for (int e = 0; e < 255; ++e) {
+    const unsigned long long v = __ldcg(bins + e);
+    if (!v) continue;
+    const int sh = (e > 0 ? e : 1) - 1, q = sh >> 6, r = sh & 63;
+    const unsigned long long add[2] = {v << r, r ? (v >> (64 - r)) : 0ull};
+    unsigned long long carry = 0;
+    for (int i = q; i < 6; ++i) {
+      const unsigned long long a = (i - q) < 2 ? add[i - q] : 0ull;
+      const unsigned long long s1 = limb[i] + a;
+      const unsigned long long c1 = s1 < a ? 1ull : 0ull;
+      const unsigned long long s2 = s1 + carry;
+      const unsigned long long c2 = s2 < carry ? 1ull : 0ull;
+      limb[i] = s2;
+      carry = c1 + c2;
+      if (i - q >= 1 && !carry) break;
+    }
+  }
+  int top = -1;
+  for (int i = 5; i >= 0 && top < 0; --i)
+    if (limb[i]) top = 64 * i + 63 - __clzll(static_cast<long long>(limb[i]));
+  if (top < 0) return 0.0;
+  auto bit = [&](int pos) -> unsigned long long { return pos < 0 ? 0ull : (limb[pos >> 6] >> (pos & 63)) & 1ull; };
+  unsigned long long m = 0;
+  int exp2 = -126 - p;  // S = m * 2^exp2 after the loop below
+  if (top <= 52) {
+    m = limb[0];
+  } else {
+    const int lo = top - 52;
+    for (int pos = top; pos >= lo; --pos) m = (m << 1) | bit(pos);
+    const unsigned long long round = bit(lo - 1);
+    bool sticky = false;
+    for (int pos = lo - 2; pos >= 0 && !sticky; --pos) sticky = bit(pos) != 0;
+    if (round && (sticky || (m & 1ull))) {
+      ++m;
+      if (m >> 53) {
+        m >>= 1;
+        exp2 += 1;
+      }
+    }
+    exp2 += lo;
+  }
+  // m < 2^53 converts exactly; the power of two is a normal fp64 (exp2 in
+  // [-201, 200]), so the product is exact
+  return __dmul_rn(static_cast<double>(m), __hiloint2double((exp2 + 1023) << 20, 0));
+}
+
+// gamma from S: max(fp32(fp64(S / numel)), 1e-5), rounding to nearest even.
+__device__ __forceinline__ float gamma_of_sum(double S, double numel) {
+  return fmaxf(__double2float_rn(__ddiv_rn(S, numel)), 1e-5f);
+}
+
+// ---------------------------------------------------------------- codes
 // Code rule: code = clamp(rint_half_even(fp32(w / gamma)), -1, 1) is nonzero
 // exactly when fp32(|w| / gamma) > 0.5, i.e. when the exact quotient exceeds
 // 0.5 + 2^-25 (the midpoint between 0.5 and the next float, which rounds to
 // the even 0.5). With T = gamma * (0.5 + 2^-25) computed exactly in fp64 and
 // thr the largest float <= T, that is |w| > thr: one compare, no division.
+//
+// 8 bf16 of one vector -> 16 bits of codes (element i at bits 2i, 2i + 1;
+// field 00 = 0, 01 = +1, 11 = -1). For a 15-bit magnitude b and thr > 0,
+// |w| > thr <=> b > bits(thr) >> 16, so both halves of a word are compared by
+// one subtraction: 0x8000 + tb - b keeps bit 15 clear exactly when b > tb (no
+// borrow crosses the halves, b <= 0x7FFF).
+__device__ __forceinline__ uint32_t codes8_bf16(const uint4& v, uint32_t bias) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  uint32_t r = 0;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const uint32_t nz = ~(bias - (w[j] & 0x7FFF7FFFu)) & 0x80008000u;  // bits 15, 31
+    const uint32_t nn = nz & w[j];                                     // and negative
+    r |= ((nz >> 15) & 1u) << (4 * j) | ((nn >> 15) & 1u) << (4 * j + 1) | (nz >> 31) << (4 * j + 2) |
+         (nn >> 31) << (4 * j + 3);
+  }
+  return r;
+}
+
+// 4 fp32 of one vector -> 8 bits of codes.
+__device__ __forceinline__ uint32_t codes4_f32(const uint4& v, float thr) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  uint32_t r = 0;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const uint32_t nz = fabsf(__uint_as_float(w[j])) > thr ? 1u : 0u;
+    r |= (nz | ((nz & (w[j] >> 31)) << 1)) << (2 * j);
+  }
+  return r;
+}
+
+// Code bits of one 16-byte vector (16 bits for bf16, 8 for fp32). `key` is
+// the bf16 compare bias or the fp32 threshold's bit pattern.
 template <bool kF32>
-__device__ __forceinline__ uint32_t pack_group(const Group<kF32>& a, float thr) {
-  if constexpr (!kF32) {
-    // bf16: for a 15-bit magnitude b (the bf16 bits with the sign cleared)
-    // and thr > 0, |w| > thr <=> (b << 16) > bits(thr) <=> b > bits(thr) >> 16,
-    // so both halves of a word are compared with one subtraction: per half,
-    // 0x8000 + tb - b keeps bit 15 clear exactly when b > tb (no borrow
-    // crosses the halves since b <= 0x7FFF). Field bit 0 = nonzero, bit 1 =
-    // nonzero and negative.
-    const uint32_t tb = __float_as_uint(thr) >> 16;
-    const uint32_t bias = (tb | (tb << 16)) + 0x80008000u;
-    const uint32_t w[8] = {a.v[0].x, a.v[0].y, a.v[0].z, a.v[0].w, a.v[1].x, a.v[1].y, a.v[1].z, a.v[1].w};
-    uint32_t acc[2] = {0u, 0u};
+__device__ __forceinline__ uint32_t vec_codes(const uint4& v, uint32_t key) {
+  if constexpr (kF32) return codes4_f32(v, __uint_as_float(key));
+  else return codes8_bf16(v, key);
+}
+
+// The vectors of a warp's 32 consecutive 16-byte vectors, one per lane, are
+// V = 2 (bf16) or 4 (fp32) per group: the lanes of a group OR their code bits
+// together and its first lane writes the group's 32-bit word.
+template <bool kF32>
+__device__ __forceinline__ uint32_t gather_group_word(uint32_t bits, int lane) {
+  constexpr int V = kF32 ? 4 : 2;
+  constexpr int kBits = 32 / V;
+  uint32_t word = bits << (kBits * (lane & (V - 1)));
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const uint32_t nz = ~(bias - (w[j] & 0x7FFF7FFFu)) & 0x80008000u;  // bits 15, 31
-      const uint32_t nn = nz & w[j];
-      // word j of a four-word half: low element's field to bits 4j', 4j'+1,
-      // high element's to 16 + 4j', 17 + 4j' (j' = j % 4)
-      const int sh = 4 * (j & 3);
-      acc[j >> 2] |= (nz >> (15 - sh)) | (nn >> (14 - sh));
+  for (int off = 1; off < V; off <<= 1) word |= __shfl_down_sync(0xffffffffu, word, off);
+  return word;
+}
+
+// ---------------------------------------------------------------- grid barrier
+__device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// One thread per CTA: arrive on `ctr` and wait until all `expected` CTAs have
+// (the caller's stores before this call are released to the other CTAs, and
+// theirs acquired). Gives up after the pipeline wait bound and records a
+// timeout. Returns false on timeout.
+__device__ __forceinline__ bool grid_arrive_wait(uint32_t* ctr, uint32_t expected, int* err) {
+  __threadfence();
+  atomicAdd(ctr, 1u);
+  if (ld_acquire_u32(ctr) >= expected) return true;
+  const unsigned long long t0 = globaltimer_ns();
+  for (uint32_t i = 1;; ++i) {
+    if (ld_acquire_u32(ctr) >= expected) return true;
+    if ((i & 15) == 0 && globaltimer_ns() - t0 > kWaitLimitNs) {
+      record_error(err, kDevTimeout);
+      return false;
     }
-    // high elements' fields from bits 16.. down to 4j' + 2
-    const uint32_t lo = (acc[0] & 0x3333u) | ((acc[0] >> 14) & 0xCCCCu);
-    const uint32_t hi = (acc[1] & 0x3333u) | ((acc[1] >> 14) & 0xCCCCu);
-    return lo | (hi << 16);
-  } else {
-    uint32_t word = 0;
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const float w = a.elem(i);
-      const uint32_t nz = fabsf(w) > thr ? 1u : 0u;
-      const uint32_t neg = __float_as_uint(w) >> 31;
-      word |= (nz * (1u | (neg << 1))) << (2 * i);  // 00 = 0, 01 = +1, 11 = -1
-    }
-    return word;
   }
 }
 
-// Code-pass block `block` of `nblocks`: threads stride over the groups
-// (consecutive threads, consecutive groups), two groups per batch, the next
-// batch loaded while the current one is packed; the first batch is loaded
-// before the wait for pass A.
-template <bool kF32>
-__device__ __forceinline__ void code_pass_block(const uint4* __restrict__ W, int64_t ngroups,
-                                                const double* __restrict__ partials, int nparts, int64_t numel,
-                                                uint32_t* __restrict__ packed, float* __restrict__ gamma_out,
-                                                int64_t block, int64_t nblocks) {
-  const int64_t stride = nblocks * kQuantThreads;
-  int64_t g = block * kQuantThreads + threadIdx.x;
-  Group<kF32> a[2];
-#pragma unroll
-  for (int u = 0; u < 2; ++u)
-    if (g + u * stride < ngroups) a[u].load(W, g + u * stride);
-
-  pdl_wait_primary();  // pass A has finished and its partial sums are visible
-  pdl_launch_dependents();
-
-  __shared__ double red[kQuantThreads / 32];
-  __shared__ float s_thr;
-  double t = 0.0;
-  for (int i = threadIdx.x; i < nparts; i += kQuantThreads) t = __dadd_rn(t, partials[i]);
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) t = __dadd_rn(t, __shfl_xor_sync(0xffffffffu, t, off));
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = t;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    double sum = 0.0;
-#pragma unroll
-    for (int w = 0; w < kQuantThreads / 32; ++w) sum = __dadd_rn(sum, red[w]);
-    const double mean = __ddiv_rn(sum, static_cast<double>(numel));
-    const float gamma = fmaxf(__double2float_rn(mean), 1e-5f);
-    s_thr = __double2float_rd(__dmul_rn(static_cast<double>(gamma), 0.5 + 0x1p-25));
-    if (block == 0) *gamma_out = gamma;
-  }
-  __syncthreads();
-  const float thr = s_thr;
-
-  for (; g < ngroups; g += 2 * stride) {
-    const int64_t gn = g + 2 * stride;
-    Group<kF32> b[2];
-#pragma unroll
-    for (int u = 0; u < 2; ++u)
-      if (gn + u * stride < ngroups) b[u].load(W, gn + u * stride);
-#pragma unroll
-    for (int u = 0; u < 2; ++u)
-      if (g + u * stride < ngroups) packed[g + u * stride] = pack_group(a[u], thr);
-#pragma unroll
-    for (int u = 0; u < 2; ++u) a[u] = b[u];
-  }
+__device__ __forceinline__ void named_barrier_sync(int id, int threads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
-template <bool kF32>
-__global__ void __launch_bounds__(kQuantThreads, kF32 ? 2 : 4) ternarize_pack_kernel(const uint4* __restrict__ W,
-                                                                          int64_t ngroups,
-                                                                          const double* __restrict__ partials,
-                                                                          int nparts, int64_t numel,
-                                                                          uint32_t* __restrict__ packed,
-                                                                          float* __restrict__ gamma_out) {
-  code_pass_block<kF32>(W, ngroups, partials, nparts, numel, packed, gamma_out, blockIdx.x, gridDim.x);
+__device__ __forceinline__ void bulk_copy_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   smem_u32(dst)),
+               "l"(src), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
 }
 
 // ---------------------------------------------------------------- S2
 // One warp per token. The row stays in registers between the absmax and the
-// quantisation: VPL = ceil(K / 256) 16-byte vectors per lane (K <= 8192).
+// quantisation: VPL = ceil(K / 256) 16-byte vectors per lane.
 //
 // q = rint_half_even(fp32(x * inv)) uses the 1.5 * 2^23 shifter: adding it
 // rounds |x * inv| <= 127.0001 to an integer (ties to even), and the low byte
@@ -439,48 +413,6 @@ __device__ __forceinline__ void act_rows_two_pass(const uint4* __restrict__ x, i
   }
 }
 
-// bl_quantize, launch 1: pass A alone (two groups loaded per batch, so that
-// it fits beside two more 256-thread blocks on an SM).
-template <bool kF32>
-__global__ void __launch_bounds__(kQuantThreads, kF32 ? 2 : 4) quant_pass_a_kernel(const uint4* __restrict__ W,
-                                                                        int64_t ngroups, int64_t per_block,
-                                                                        double* __restrict__ partials) {
-  pdl_wait_primary();
-  pdl_launch_dependents();  // launch 2 may start beside this pass
-  absmean_block<kF32, 2>(W, ngroups, per_block, blockIdx.x, partials);
-}
-
-// bl_quantize, launch 2 (a programmatic dependent of launch 1): blocks
-// 0 .. act_blocks-1 quantise tokens (S2); the rest run the code pass. The token
-// blocks do not wait for launch 1: x was complete before launch 1 passed its
-// own dependency wait (and launch 2 only starts after that point), and launch
-// 1 neither reads xq / s_x nor writes x. So they run beside pass A, and the
-// code-pass blocks -- which do wait -- follow; since they wait, this grid
-// still completes only after launch 1 has. Rows of up to 2560 elements stay
-// in registers (VPL <= 10, the most that fits the 64 registers a thread has at
-// four blocks per SM), longer ones are read twice (VPL = 0).
-constexpr int kFusedMaxVpl = 10;
-
-template <bool kF32, int VPL>
-__global__ void __launch_bounds__(kQuantThreads, kF32 ? 2 : 4) quant_phase2_kernel(
-    const uint4* __restrict__ W, int64_t ngroups, const double* __restrict__ partials, int nparts, int64_t numel,
-    uint32_t* __restrict__ packed, float* __restrict__ gamma_out, const uint4* __restrict__ x, int64_t M, int nv,
-    int8_t* __restrict__ xq, float* __restrict__ sx, int act_blocks) {
-  if (static_cast<int>(blockIdx.x) < act_blocks) {
-    pdl_launch_dependents();
-    constexpr int kWarps = kQuantThreads / 32;
-    const int64_t m = static_cast<int64_t>(blockIdx.x) * kWarps + (threadIdx.x >> 5);
-    const int64_t stride = static_cast<int64_t>(act_blocks) * kWarps;
-    if constexpr (VPL > 0)
-      act_rows<VPL, false>(x, M, nv, xq, sx, m, stride);
-    else
-      act_rows_two_pass(x, M, nv, xq, sx, m, stride);
-    return;
-  }
-  code_pass_block<kF32>(W, ngroups, partials, nparts, numel, packed, gamma_out, blockIdx.x - act_blocks,
-                        gridDim.x - act_blocks);
-}
-
 // Rows longer than 8192 elements: absmax pass, then a second read (from L2).
 __global__ void __launch_bounds__(32 * kActRowsPerBlock) act_quant_long_kernel(const uint4* __restrict__ x,
                                                                                int64_t M, int nv,
@@ -488,91 +420,305 @@ __global__ void __launch_bounds__(32 * kActRowsPerBlock) act_quant_long_kernel(c
                                                                                float* __restrict__ sx) {
   pdl_wait_primary();
   pdl_launch_dependents();
-  const int lane = threadIdx.x & 31;
-  const int64_t m = static_cast<int64_t>(blockIdx.x) * kActRowsPerBlock + (threadIdx.x >> 5);
-  if (m >= M) return;
-  const uint4* row = x + m * nv;
-  uint32_t mx = 0u;
-  for (int j = lane; j < nv; j += 32) mx = absmax8(__ldg(row + j), mx);
-  const float a = fmaxf(warp_max(absmax_value(mx)), 1e-5f);
-  const float inv = __fdiv_rn(127.0f, a);
-  if (lane == 0) sx[m] = __fdiv_rn(a, 127.0f);
-  uint2* out = reinterpret_cast<uint2*>(xq + m * static_cast<int64_t>(nv) * 8);
-  for (int j = lane; j < nv; j += 32) out[j] = quant8(__ldg(row + j), inv);
+  act_rows_two_pass(x, M, nv, xq, sx, static_cast<int64_t>(blockIdx.x) * kActRowsPerBlock + (threadIdx.x >> 5),
+                    static_cast<int64_t>(gridDim.x) * kActRowsPerBlock);
+}
+
+// ---------------------------------------------------------------- S1 (+ S2): the launches
+// Launch 1: clears the workspace's two arrival counters and its exact-sum
+// bins. It waits for the kernel before it in the stream (whose work may
+// still read them), and only then lets the quantisation launch start; so the
+// quantisation may read W and x and write its outputs from its first
+// instruction, and waits for this launch itself only before its first use of
+// the counters.
+__global__ void __launch_bounds__(256) quant_reset_kernel(uint8_t* __restrict__ ws) {
+  pdl_wait_primary();
+  pdl_launch_dependents();
+  if (threadIdx.x < 2) reinterpret_cast<uint32_t*>(ws)[threadIdx.x] = 0u;
+  reinterpret_cast<unsigned long long*>(ws + kWsBins)[threadIdx.x] = 0ull;
+}
+
+struct QuantArgs {
+  const uint4* W;       // [N, K] as 16-byte vectors
+  int64_t ngroups;      // N K / 16: a group's 16 codes are one 32-bit word
+  int64_t per;          // groups per CTA slice (the last slices may be shorter or empty)
+  int onchip_cap;       // groups of a slice held in shared memory
+  double numel;
+  double enc_lo, enc_hi;  // S lies in [fp64 sum * enc_lo, fp64 sum * enc_hi]
+  uint32_t* packed;
+  float* gamma_out;
+  uint8_t* ws;
+  int* err;
+  const uint4* x;       // S2: x [M, K] as 16-byte vectors (M = 0: no tokens)
+  int64_t M;
+  int nv;               // K / 8
+  int8_t* xq;
+  float* sx;
+};
+
+// Launch 2. Warps 0..7 (all 16 without tokens) work on the CTA's W slice;
+// warps 8..15 quantise tokens m = 8 b + w - 8 + 8 G i. Rows of up to 2560
+// elements (VPL <= 10) stay in registers; longer ones (VPL = 0) are read twice.
+template <bool kF32, int VPL>
+__global__ void __launch_bounds__(kQThreads, 1) quant_fused_kernel(const __grid_constant__ QuantArgs a) {
+  constexpr int V = kF32 ? 4 : 2;  // 16-byte vectors per group
+  constexpr int kGroupBytes = 16 * V;
+  constexpr int kChunkGroups = kChunkBytes / kGroupBytes;
+  constexpr int kTailRegs = 4;
+  extern __shared__ __align__(128) uint4 s_w[];
+  __shared__ __align__(8) uint64_t s_bar[kMaxChunks];
+  __shared__ unsigned long long s_bins[256];
+  __shared__ double s_red[kQWarps];
+  __shared__ float s_gamma;
+  __shared__ int s_mode;   // after the partial sums: 0 codes, 1 exact sum first
+  __shared__ int s_abort;  // a wait of this CTA gave up
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const bool tokens = a.M > 0;
+  const int nww = tokens ? kTokenWarp0 : kQWarps;
+  const int nthr = 32 * nww;
+  const int64_t b = blockIdx.x;
+  const uint32_t G = gridDim.x;
+  const int64_t g0 = b * a.per;
+  const int64_t rest = a.ngroups - g0;
+  const int64_t len = rest <= 0 ? 0 : (rest < a.per ? rest : a.per);
+  const int on = static_cast<int>(len < a.onchip_cap ? len : a.onchip_cap);
+  const int nch = (on + kChunkGroups - 1) / kChunkGroups;
+  uint32_t* ctr = reinterpret_cast<uint32_t*>(a.ws);
+  double* partials = reinterpret_cast<double*>(a.ws + kWsPartials);
+  unsigned long long* gbins = reinterpret_cast<unsigned long long*>(a.ws + kWsBins);
+
+  if (threadIdx.x == 0) {
+    s_abort = 0;
+    for (int c = 0; c < nch; ++c) mbar_init(&s_bar[c], 1);
+    fence_mbar_init();
+    fence_proxy_async_smem();
+    // the whole on-chip slice in flight at once, before any token load
+    for (int c = 0; c < nch; ++c) {
+      const int cg0 = c * kChunkGroups;
+      const int cgn = min(kChunkGroups, on - cg0);
+      mbar_arrive_expect_tx(&s_bar[c], static_cast<uint32_t>(cgn * kGroupBytes));
+      bulk_copy_g2s(s_w + static_cast<int64_t>(cg0) * V, a.W + (g0 + cg0) * V, static_cast<uint32_t>(cgn * kGroupBytes),
+                    &s_bar[c]);
+    }
+  }
+  __syncthreads();
+
+  if (warp >= nww) {
+    // ------------------------------------------------ S2 tokens
+    constexpr int kTokWarps = kQWarps - kTokenWarp0;
+    const int64_t m = b * kTokWarps + (warp - kTokenWarp0);
+    const int64_t stride = static_cast<int64_t>(G) * kTokWarps;
+    if constexpr (VPL > 0)
+      act_rows<VPL, false>(a.x, a.M, a.nv, a.xq, a.sx, m, stride);
+    else
+      act_rows_two_pass(a.x, a.M, a.nv, a.xq, a.sx, m, stride);
+    return;
+  }
+
+  // -------------------------------------------------- S1 slice warps
+  const int t = threadIdx.x;
+  const int64_t tail_v0 = (g0 + on) * V, tail_v1 = (g0 + len) * V;
+  // first vectors of the off-chip tail, loaded before the chunks are summed
+  uint4 tr[kTailRegs];
+#pragma unroll
+  for (int u = 0; u < kTailRegs; ++u) {
+    const int64_t i = tail_v0 + t + static_cast<int64_t>(u) * nthr;
+    tr[u] = i < tail_v1 ? __ldg(a.W + i) : make_uint4(0u, 0u, 0u, 0u);
+  }
+  double acc[4] = {0.0, 0.0, 0.0, 0.0};
+  for (int c = 0; c < nch; ++c) {
+    if (!mbar_wait(&s_bar[c], 0, &s_abort, a.err)) {
+      s_abort = 1;
+      break;
+    }
+    const int v1 = min((c + 1) * kChunkGroups, on) * V;
+    int i = c * kChunkGroups * V + t;
+    for (; i + 3 * nthr < v1; i += 4 * nthr) {
+      acc[0] = add_abs<kF32>(acc[0], s_w[i]);
+      acc[1] = add_abs<kF32>(acc[1], s_w[i + nthr]);
+      acc[2] = add_abs<kF32>(acc[2], s_w[i + 2 * nthr]);
+      acc[3] = add_abs<kF32>(acc[3], s_w[i + 3 * nthr]);
+    }
+    if (i < v1) acc[0] = add_abs<kF32>(acc[0], s_w[i]);
+    if (i + nthr < v1) acc[1] = add_abs<kF32>(acc[1], s_w[i + nthr]);
+    if (i + 2 * nthr < v1) acc[2] = add_abs<kF32>(acc[2], s_w[i + 2 * nthr]);
+  }
+  {
+    // the tail: the vectors already in registers, then the rest four at a time
+#pragma unroll
+    for (int u = 0; u < kTailRegs; ++u)
+      if (tail_v0 + t + static_cast<int64_t>(u) * nthr < tail_v1) acc[u] = add_abs<kF32>(acc[u], tr[u]);
+    for (int64_t i = tail_v0 + t + static_cast<int64_t>(kTailRegs) * nthr; i < tail_v1; i += 4 * nthr) {
+      uint4 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) v[u] = i + u * nthr < tail_v1 ? __ldg(a.W + i + u * nthr) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (i + u * nthr < tail_v1) acc[u] = add_abs<kF32>(acc[u], v[u]);
+    }
+  }
+  double ts = __dadd_rn(__dadd_rn(acc[0], acc[1]), __dadd_rn(acc[2], acc[3]));
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) ts = __dadd_rn(ts, __shfl_xor_sync(0xffffffffu, ts, off));
+  if (lane == 0) s_red[warp] = ts;
+  named_barrier_sync(kBarWarpsNamed, nthr);
+
+  if (t == 0) {
+    double part = 0.0;
+    for (int w = 0; w < nww; ++w) part = __dadd_rn(part, s_red[w]);
+    partials[b] = part;
+    pdl_wait_primary();  // launch 1 has cleared the counters
+    if (!grid_arrive_wait(&ctr[0], G, a.err)) s_abort = 1;
+  }
+  named_barrier_sync(kBarWarpsNamed, nthr);
+  pdl_launch_dependents();  // every CTA is resident (all arrived): the next launch may be scheduled
+
+  if (warp == 0 && !s_abort) {
+    // the partial sums in one fixed order: lane l adds l, l + 32, ..., then a
+    // fixed shuffle tree
+    double s = 0.0;
+    for (uint32_t j = lane; j < G; j += 32) s = __dadd_rn(s, __ldcg(partials + j));
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) s = __dadd_rn(s, __shfl_xor_sync(0xffffffffu, s, off));
+    if (lane == 0) {
+      const float glo = gamma_of_sum(__dmul_rd(s, a.enc_lo), a.numel);
+      const float ghi = gamma_of_sum(__dmul_ru(s, a.enc_hi), a.numel);
+      s_gamma = glo;
+      s_mode = __float_as_uint(glo) == __float_as_uint(ghi) ? 0 : 1;
+    }
+  }
+  named_barrier_sync(kBarWarpsNamed, nthr);
+
+  if (!s_abort && s_mode == 1) {
+    // ------------------------------------------------ exact sum (rare)
+    for (int e = t; e < 256; e += nthr) s_bins[e] = 0ull;
+    named_barrier_sync(kBarWarpsNamed, nthr);
+    for (int i = t; i < on * V; i += nthr) bin_abs<kF32>(s_bins, s_w[i]);
+    for (int64_t i = tail_v0 + t; i < tail_v1; i += nthr) bin_abs<kF32>(s_bins, __ldg(a.W + i));
+    named_barrier_sync(kBarWarpsNamed, nthr);
+    for (int e = t; e < 256; e += nthr)
+      if (s_bins[e]) atomicAdd(gbins + e, s_bins[e]);
+    named_barrier_sync(kBarWarpsNamed, nthr);
+    if (t == 0) {
+      if (!grid_arrive_wait(&ctr[1], G, a.err)) {
+        s_abort = 1;
+      } else {
+        s_gamma = gamma_of_sum(exact_sum_from_bins(gbins, kF32 ? 23 : 7), a.numel);
+      }
+    }
+    named_barrier_sync(kBarWarpsNamed, nthr);
+  }
+
+  if (s_abort) {
+    // let every copy already issued land before the CTA exits (one bound)
+    if (t == 0) {
+      const unsigned long long deadline = globaltimer_ns() + kWaitLimitNs;
+      for (int c = 0; c < nch; ++c) mbar_drain_until(&s_bar[c], 0, deadline);
+    }
+    return;
+  }
+
+  // -------------------------------------------------- codes
+  const float gamma = s_gamma;
+  if (b == 0 && t == 0) *a.gamma_out = gamma;
+  const float thr = __double2float_rd(__dmul_rn(static_cast<double>(gamma), 0.5 + 0x1p-25));
+  uint32_t key;
+  if constexpr (kF32) {
+    key = __float_as_uint(thr);
+  } else {
+    const uint32_t tb = __float_as_uint(thr) >> 16;
+    key = (tb | (tb << 16)) + 0x80008000u;
+  }
+  // lanes take consecutive 16-byte vectors (conflict-free shared loads); a
+  // group's V lanes combine their bits and its first lane stores the word
+  uint32_t* out = a.packed + g0;
+  for (int base = 32 * warp; base < on * V; base += 32 * nww) {
+    const int i = base + lane;
+    const bool valid = i < on * V;
+    const uint32_t word = gather_group_word<kF32>(valid ? vec_codes<kF32>(s_w[i], key) : 0u, lane);
+    if (valid && (lane & (V - 1)) == 0) out[i / V] = word;
+  }
+  for (int64_t base = tail_v0 + 32 * warp; base < tail_v1; base += 32 * nww) {
+    const int64_t i = base + lane;
+    const bool valid = i < tail_v1;
+    const uint32_t word = gather_group_word<kF32>(valid ? vec_codes<kF32>(__ldg(a.W + i), key) : 0u, lane);
+    if (valid && (lane & (V - 1)) == 0) a.packed[i / V] = word;
+  }
 }
 
 }  // namespace
 
-// Fixed device scratch for bl_quantize_weight_noalloc: room for the largest
-// number of fp64 partial sums pass A ever writes (kMaxPartials), 2368 bytes.
-// Every GPU that loads the library holds this array until the process exits.
-static __device__ __align__(256) double g_noalloc_partials[kMaxPartials];
+// Fixed device scratch for bl_quantize_weight_noalloc: the workspace of one
+// call (arrival counters, one fp64 partial sum per CTA, exact-sum bins),
+// 10304 bytes. Every GPU that loads the library holds this array until the
+// process exits.
+static __device__ __align__(256) uint8_t g_noalloc_ws[kWsBytes];
 
-// Blocks of the code pass: four per SM, fewer for small tensors.
-static unsigned code_pass_blocks(int64_t ngroups) {
-  const int64_t want = (ngroups + kQuantThreads - 1) / kQuantThreads;
-  const int64_t cap = static_cast<int64_t>(4) * device_sm_count();
-  return static_cast<unsigned>(want < cap ? want : cap);
-}
+size_t quantize_workspace_bytes() { return kWsBytes; }
 
-int weight_partials_count(int64_t numel) {
-  const int64_t ngroups = numel / 16;
-  const int64_t want = (ngroups + kQuantThreads - 1) / kQuantThreads;
-  return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(kMaxPartials, want)));
-}
+namespace {
+
+// Geometry of one S1 (+ S2) launch.
+struct QuantGeometry {
+  unsigned ctas;
+  size_t smem;
+};
 
 template <bool kF32>
-static cudaError_t launch_weight_passes(const uint4* w, int64_t ngroups, int64_t per_block, int nparts, int64_t numel,
-                                        uint32_t* out, float* gamma, double* partials, cudaStream_t s) {
-  cudaError_t e = launch_pdl(absmean_partials_kernel<kF32>, dim3(nparts), dim3(kQuantThreads), 0, s, w, ngroups,
-                             per_block, partials);
-  if (e != cudaSuccess) return e;
-  return launch_pdl(ternarize_pack_kernel<kF32>, dim3(code_pass_blocks(ngroups)), dim3(kQuantThreads), 0, s, w,
-                    ngroups, static_cast<const double*>(partials), nparts, numel, out, gamma);
+QuantGeometry quant_geometry(int64_t ngroups, int64_t M, QuantArgs& a) {
+  constexpr int V = kF32 ? 4 : 2;
+  constexpr int kGroupBytes = 16 * V;
+  constexpr int kChunkGroups = kChunkBytes / kGroupBytes;
+  constexpr int kElems = kF32 ? 4 : 8;  // elements per 16-byte vector
+  // enough CTAs to spread the slice (>= 256 groups each) and the tokens (>= 16
+  // rows each), at most one per SM so that all of them are resident together
+  const int64_t want = std::max<int64_t>((ngroups + 255) / 256, (M + 15) / 16);
+  const int64_t cap = std::min<int64_t>(device_sm_count(), kMaxQuantCtas);
+  const int64_t G = std::max<int64_t>(1, std::min(want, cap));
+  a.ngroups = ngroups;
+  a.per = (ngroups + G - 1) / G;
+  a.onchip_cap = kMaxOnchipBytes / kGroupBytes;
+  const int64_t on_max = std::min<int64_t>(a.per, a.onchip_cap);
+  // Enclosure of S around the fp64 tree sum: every leaf passes through at most
+  // d roundings (its accumulator's sequential adds, the four accumulators, the
+  // warp shuffle tree, the sequential warp sums, the lane sums of the
+  // partials, their shuffle tree), each off by at most 2^-53 of a partial sum
+  // that is at most S (1 + 2^-30) with all terms >= 0, so |fp64 sum - S| <=
+  // d 2^-53 (1 + 2^-30) S; e = d 2^-52 covers S on both sides.
+  const int64_t nch_max = (on_max + kChunkGroups - 1) / kChunkGroups;
+  const double per_acc = static_cast<double>(a.per) * V / (4.0 * 32 * kTokenWarp0) + static_cast<double>(nch_max) + 3.0;
+  const double d = kElems * per_acc + 2 + 5 + kQWarps + std::ceil(static_cast<double>(G) / 32.0) + 5 + 8;
+  const double e = std::ldexp(d, -52);
+  a.enc_lo = 1.0 - e;
+  a.enc_hi = 1.0 + e;
+  return {static_cast<unsigned>(G), static_cast<size_t>(on_max) * kGroupBytes};
 }
 
-cudaError_t launch_quantize_weight(const void* W, int w_is_f32, int64_t N, int64_t K, uint8_t* packed,
-                                   float* gamma, double* partials, cudaStream_t s) {
-  const int64_t numel = N * K;  // multiple of 32
-  const int64_t ngroups = numel / 16;
-  const int nparts = weight_partials_count(numel);
-  const int64_t per_block = (ngroups + nparts - 1) / nparts;
-  const uint4* w = static_cast<const uint4*>(W);
-  uint32_t* out = reinterpret_cast<uint32_t*>(packed);
-  cudaError_t e = w_is_f32 ? launch_weight_passes<true>(w, ngroups, per_block, nparts, numel, out, gamma, partials, s)
-                           : launch_weight_passes<false>(w, ngroups, per_block, nparts, numel, out, gamma, partials, s);
+template <bool kF32, int VPL>
+cudaError_t launch_fused(QuantArgs& a, cudaStream_t s) {
+  static bool configured[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && !configured[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(quant_fused_kernel<kF32, VPL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         kMaxOnchipBytes);
+    if (e != cudaSuccess) return e;
+    configured[dev] = true;
+  }
+  const QuantGeometry geo = quant_geometry<kF32>(a.ngroups, a.M, a);
+  cudaError_t e = launch_pdl(quant_reset_kernel, dim3(1), dim3(256), 0, s, a.ws);
   if (e != cudaSuccess) return e;
-  return cudaGetLastError();
-}
-
-size_t noalloc_scratch_bytes() { return sizeof(g_noalloc_partials); }
-
-// Device address of g_noalloc_partials on the current device. Host code only
-// holds a stand-in for the array's name, so the address is looked up with the
-// device current, on every call: a cached address would go stale if the
-// caller reset the device and the module were loaded again elsewhere. The
-// first lookup on a device loads the module there (so it belongs before any
-// stream capture); later ones are host-side table lookups.
-static cudaError_t noalloc_scratch_ptr(double** out) {
-  void* p = nullptr;
-  const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_partials);
-  if (e != cudaSuccess) return e;
-  *out = static_cast<double*>(p);
-  return cudaSuccess;
-}
-
-cudaError_t launch_quantize_weight_noalloc(const void* W, int w_is_f32, int64_t N, int64_t K, uint8_t* packed,
-                                           float* gamma, cudaStream_t s) {
-  if (static_cast<size_t>(weight_partials_count(N * K)) * sizeof(double) > sizeof(g_noalloc_partials))
-    return cudaErrorInvalidValue;
-  double* scratch = nullptr;
-  const cudaError_t e = noalloc_scratch_ptr(&scratch);
-  if (e != cudaSuccess) return e;
-  return launch_quantize_weight(W, w_is_f32, N, K, packed, gamma, scratch, s);
+  return launch_pdl(quant_fused_kernel<kF32, VPL>, dim3(geo.ctas), dim3(kQThreads), geo.smem, s, a);
 }
 
 template <int VPL>
-static void launch_act(const uint4* xv, int64_t M, int nv, int8_t* xq, float* sx, cudaStream_t s) {
+cudaError_t launch_fused_dtype(bool f32, QuantArgs& a, cudaStream_t s) {
+  return f32 ? launch_fused<true, VPL>(a, s) : launch_fused<false, VPL>(a, s);
+}
+
+template <int VPL>
+void launch_act(const uint4* xv, int64_t M, int nv, int8_t* xq, float* sx, cudaStream_t s) {
   constexpr bool kPrefetch = VPL <= 12;
   static int per_sm[64] = {};
   int dev = 0;
@@ -591,28 +737,59 @@ static void launch_act(const uint4* xv, int64_t M, int nv, int8_t* xq, float* sx
   launch_pdl(act_quant_kernel<VPL, kPrefetch>, dim3(grid), dim3(32 * kActRowsPerBlock), 0, s, xv, M, nv, xq, sx);
 }
 
-// bl_quantize: pass A (quant_pass_a_kernel), then the token blocks and the
-// code pass in one grid (quant_phase2_kernel). Rows longer than 8192
-// elements take the separate launches.
-template <bool kF32, int VPL>
-static cudaError_t launch_quantize_fused(const uint4* w, int64_t N, int64_t K, const uint4* xv, int64_t M,
-                                         uint32_t* packed, float* gamma, double* partials, int8_t* xq, float* sx,
-                                         cudaStream_t s) {
-  const int64_t numel = N * K;
-  const int64_t ngroups = numel / 16;
-  const int nparts = weight_partials_count(numel);
-  const int64_t per_block = (ngroups + nparts - 1) / nparts;
-  // token blocks: two per SM beside pass A, no more than the rows need
-  const int64_t rows_blocks = (M + kQuantThreads / 32 - 1) / (kQuantThreads / 32);
-  const int64_t act_blocks = std::min<int64_t>(static_cast<int64_t>(2) * device_sm_count(), rows_blocks);
-  const int64_t code_blocks = code_pass_blocks(ngroups);
-  const int nv = static_cast<int>(K / 8);
-  cudaError_t e = launch_pdl(quant_pass_a_kernel<kF32>, dim3(static_cast<unsigned>(nparts)), dim3(kQuantThreads), 0,
-                             s, w, ngroups, per_block, partials);
+}  // namespace
+
+cudaError_t launch_quantize(const void* W, int w_is_f32, int64_t N, int64_t K, const void* x, int64_t M,
+                            uint8_t* packed, float* gamma, void* workspace, int8_t* xq, float* sx, int* err,
+                            cudaStream_t s) {
+  QuantArgs a{};
+  a.W = static_cast<const uint4*>(W);
+  a.ngroups = N * K / 16;  // K % 32 == 0
+  a.numel = static_cast<double>(N * K);
+  a.packed = reinterpret_cast<uint32_t*>(packed);
+  a.gamma_out = gamma;
+  a.ws = static_cast<uint8_t*>(workspace);
+  a.err = err;
+  a.x = static_cast<const uint4*>(x);
+  a.M = M;
+  a.nv = static_cast<int>(K / 8);
+  a.xq = xq;
+  a.sx = sx;
+  const int per_lane = (a.nv + 31) / 32;
+  const bool f32 = w_is_f32 != 0;
+  cudaError_t e = cudaSuccess;
+  switch (M > 0 && per_lane <= 10 ? per_lane : 0) {
+#define BL_Q_CASE(n)                          \
+  case n:                                     \
+    e = launch_fused_dtype<n>(f32, a, s);     \
+    break;
+    BL_Q_CASE(0) BL_Q_CASE(1) BL_Q_CASE(2) BL_Q_CASE(3) BL_Q_CASE(4) BL_Q_CASE(5) BL_Q_CASE(6)
+    BL_Q_CASE(7) BL_Q_CASE(8) BL_Q_CASE(9) BL_Q_CASE(10)
+#undef BL_Q_CASE
+    default:
+      break;
+  }
   if (e != cudaSuccess) return e;
-  return launch_pdl(quant_phase2_kernel<kF32, VPL>, dim3(static_cast<unsigned>(act_blocks + code_blocks)),
-                    dim3(kQuantThreads), 0, s, w, ngroups, static_cast<const double*>(partials), nparts, numel, packed,
-                    gamma, xv, M, nv, xq, sx, static_cast<int>(act_blocks));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quantize_weight(const void* W, int w_is_f32, int64_t N, int64_t K, uint8_t* packed,
+                                   float* gamma, void* workspace, int* err, cudaStream_t s) {
+  return launch_quantize(W, w_is_f32, N, K, nullptr, 0, packed, gamma, workspace, nullptr, nullptr, err, s);
+}
+
+// Device address of g_noalloc_ws on the current device. Host code only holds
+// a stand-in for the array's name, so the address is looked up with the
+// device current, on every call: a cached address would go stale if the
+// caller reset the device and the module were loaded again elsewhere. The
+// first lookup on a device loads the module there (so it belongs before any
+// stream capture); later ones are host-side table lookups.
+cudaError_t launch_quantize_weight_noalloc(const void* W, int w_is_f32, int64_t N, int64_t K, uint8_t* packed,
+                                           float* gamma, int* err, cudaStream_t s) {
+  void* scratch = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&scratch, g_noalloc_ws);
+  if (e != cudaSuccess) return e;
+  return launch_quantize_weight(W, w_is_f32, N, K, packed, gamma, scratch, err, s);
 }
 
 cudaError_t launch_quantize_act(const void* x, int64_t M, int64_t K, int8_t* xq, float* sx, cudaStream_t s) {
@@ -637,35 +814,6 @@ cudaError_t launch_quantize_act(const void* x, int64_t M, int64_t K, int8_t* xq,
       launch_pdl(act_quant_long_kernel, dim3(grid), dim3(32 * kActRowsPerBlock), 0, s, xv, M, nv, xq, sx);
     }
   }
-  return cudaGetLastError();
-}
-
-cudaError_t launch_quantize(const void* W, int w_is_f32, int64_t N, int64_t K, const void* x, int64_t M,
-                            uint8_t* packed, float* gamma, double* partials, int8_t* xq, float* sx, cudaStream_t s) {
-  const int nv = static_cast<int>(K / 8);
-  const int per_lane = (nv + 31) / 32;
-  if (M == 0 || per_lane > 32) {
-    cudaError_t e = launch_quantize_weight(W, w_is_f32, N, K, packed, gamma, partials, s);
-    if (e != cudaSuccess) return e;
-    return launch_quantize_act(x, M, K, xq, sx, s);
-  }
-  const uint4* w = static_cast<const uint4*>(W);
-  const uint4* xv = static_cast<const uint4*>(x);
-  uint32_t* out = reinterpret_cast<uint32_t*>(packed);
-  cudaError_t e = cudaSuccess;
-  switch (per_lane <= kFusedMaxVpl ? per_lane : 0) {
-#define BL_Q_CASE(n)                                                                                  \
-  case n:                                                                                             \
-    e = w_is_f32 ? launch_quantize_fused<true, n>(w, N, K, xv, M, out, gamma, partials, xq, sx, s)    \
-                 : launch_quantize_fused<false, n>(w, N, K, xv, M, out, gamma, partials, xq, sx, s); \
-    break;
-    BL_Q_CASE(0) BL_Q_CASE(1) BL_Q_CASE(2) BL_Q_CASE(3) BL_Q_CASE(4) BL_Q_CASE(5) BL_Q_CASE(6)
-    BL_Q_CASE(7) BL_Q_CASE(8) BL_Q_CASE(9) BL_Q_CASE(10)
-#undef BL_Q_CASE
-    default:
-      break;
-  }
-  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

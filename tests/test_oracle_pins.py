@@ -137,6 +137,23 @@ def test_gamma_uses_exact_mean():
     assert ref.absmean_gamma(w.reshape(256, 256)) == expected
 
 
+@pytest.mark.parametrize("case,expected", [("tie", 1.0), ("above", 1.0 + 2.0 ** -23), ("below", 1.0)])
+@pytest.mark.parametrize("w_dtype", ["bf16", "f32"])
+def test_gamma_at_an_fp32_midpoint(case, expected, w_dtype):
+    """Tensors whose mean |W| is 1 + 2^-24 (the midpoint between the fp32
+    neighbours 1 and 1 + 2^-23) exactly, or 2^-44 above or below it: the
+    exactly rounded mean gives the closed forms (the tie to the even 1.0).
+    Every magnitude >= 1 gets code +-1 with its sign, every smaller one 0."""
+    from workloads import gamma_midpoint_weights
+    w = gamma_midpoint_weights(case, torch.bfloat16 if w_dtype == "bf16" else torch.float32)
+    wf = w.float().numpy()
+    codes, gamma = ref.ternarize(wf)
+    assert gamma == np.float32(expected)
+    big = np.abs(wf) >= 1.0
+    np.testing.assert_array_equal(codes[big], np.sign(wf[big]).astype(np.int8))
+    assert not codes[~big].any()
+
+
 # --------------------------------------------------------------------------
 # S2: activation quantisation
 # --------------------------------------------------------------------------

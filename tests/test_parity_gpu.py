@@ -195,6 +195,49 @@ def test_quantize_weight_deterministic():
         assert torch.equal(p, outs[0][0]) and torch.equal(g, outs[0][1])
 
 
+@pytest.mark.parametrize("case,expected", [("tie", 1.0), ("above", 1.0 + 2.0 ** -23), ("below", 1.0)])
+@pytest.mark.parametrize("w_dtype", [torch.bfloat16, torch.float32])
+def test_gamma_at_an_fp32_midpoint(case, expected, w_dtype):
+    """Mean |W| on, 2^-44 above or 2^-44 below the fp32 midpoint 1 + 2^-24
+    (the fp64 tree sum's error bound straddles it, so gamma comes from the
+    exact integer sum): gamma and the codes bit-exact to the oracle through
+    bl_quantize_weight, bl_quantize and bl_quantize_weight_noalloc, twice."""
+    from workloads import gamma_midpoint_weights
+    bl = _bl()
+    w = gamma_midpoint_weights(case, w_dtype)
+    N, K = w.shape
+    codes, g = ref.ternarize(w.float().numpy())
+    assert g == np.float32(expected)
+    expect = ref.pack_ternary(codes)
+    wd = w.cuda()
+    x, _, _ = make_inputs(64, K, 8, seed=3)
+    xd = x.cuda()
+    ws = torch.empty(bl.bl_quantize_weight_workspace_size(N, K), dtype=torch.uint8, device="cuda")
+    lib = bl.load_library()
+    for rep in range(2):
+        for how in ("weight", "fused", "noalloc"):
+            packed = torch.full((N, K // 4), 0xAA, dtype=torch.uint8, device="cuda")
+            gamma = torch.full((1,), -1.0, dtype=torch.float32, device="cuda")
+            if how == "weight":
+                bl.bl_quantize_weight(wd, packed, gamma, ws)
+            elif how == "fused":
+                xq = torch.empty((64, K), dtype=torch.int8, device="cuda")
+                sx = torch.empty(64, dtype=torch.float32, device="cuda")
+                bl.bl_quantize(wd, xd, packed, gamma, xq, sx, ws)
+            else:
+                wdt = bl.BL_F32 if w_dtype == torch.float32 else bl.BL_BF16
+                import ctypes
+                rc = lib.bl_quantize_weight_noalloc(ctypes.c_void_p(wd.data_ptr()), wdt, N, K,
+                                                    ctypes.c_void_p(packed.data_ptr()),
+                                                    ctypes.c_void_p(gamma.data_ptr()),
+                                                    ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+                assert rc == 0
+            torch.cuda.synchronize()
+            assert bl.bl_get_last_error() == 0
+            assert gamma.cpu().numpy()[0].tobytes() == np.float32(expected).tobytes(), (how, rep)
+            np.testing.assert_array_equal(packed.cpu().numpy(), expect, err_msg=f"{how} {rep}")
+
+
 @pytest.mark.parametrize("dw_dtype", [torch.float32, torch.bfloat16])
 def test_dw_accumulate(dw_dtype):
     bl = _bl()
@@ -335,7 +378,9 @@ def test_backward_scheduled_tiles_full_compare():
     (300, 520, 320, torch.bfloat16),      # rows in registers
     (64, 264, 1024, torch.float32),
     (17, 136, 96, torch.bfloat16),
-    (40, 64, 8448, torch.bfloat16),       # rows past 8192: separate launches
+    (40, 64, 8448, torch.bfloat16),       # rows past 8192 (read twice)
+    (300, 6912, 2560, torch.bfloat16),    # slices past shared memory: a tail read again
+    (2048, 2560, 6912, torch.bfloat16),   # the down-projection shape
     (0, 128, 256, torch.bfloat16),        # no tokens: S1 only
 ])
 def test_quantize_fused_matches_separate(M, N, K, w_dtype):

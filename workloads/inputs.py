@@ -103,3 +103,41 @@ def stack_inputs(M: int, dims, seed: int = 0):
         ws.append(w.to(torch.bfloat16).contiguous())
     dy = torch.randn(M, dims[-1], generator=_gen(seed + 1), dtype=torch.float32)
     return x.to(torch.bfloat16).contiguous(), ws, dy.to(torch.bfloat16).contiguous()
+
+
+def gamma_midpoint_weights(case: str, w_dtype=torch.bfloat16, seed: int = 0):
+    """W [2048, 1024] (2^21 elements) whose mean |W| lies on, just above or
+    just below the midpoint 1 + 2^-24 between the fp32 neighbours 1 and
+    1 + 2^-23. Every magnitude is a bf16 value; signs and positions are
+    shuffled with ``seed``:
+
+      2^20 ones and 2^19 twos (sum 2^21), then in the remaining 2^19 slots
+      "tie":   one 2^-3                         sum = 2^21 + 2^-3
+      "above": one 2^-3 and 2^18 of 2^-41       sum = 2^21 + 2^-3 + 2^-23
+      "below": 2^-3 - 2^-11, 2^-11 - 2^-19 and 2^-19 - 2^-23
+                                                sum = 2^21 + 2^-3 - 2^-23
+      and zeros in the slots left.
+    """
+    n, k = 1 << 21, 1 << 19
+    vals = torch.zeros(n, dtype=torch.float64)
+    vals[: n - 2 * k] = 1.0
+    vals[n - 2 * k: n - k] = 2.0
+    rest = n - k
+    if case in ("tie", "above"):
+        vals[rest] = 2.0 ** -3
+        if case == "above":
+            vals[rest + 1: rest + 1 + (1 << 18)] = 2.0 ** -41
+    elif case == "below":
+        vals[rest] = 2.0 ** -3 - 2.0 ** -11
+        vals[rest + 1] = 2.0 ** -11 - 2.0 ** -19
+        vals[rest + 2] = 2.0 ** -19 - 2.0 ** -23
+    else:
+        raise ValueError(case)
+    g = _gen(seed)
+    perm = torch.randperm(n, generator=g)
+    signs = torch.where(torch.rand(n, generator=g) < 0.5, -1.0, 1.0).to(torch.float64)
+    w = (vals[perm] * signs).reshape(2048, 1024)
+    return w.to(w_dtype).contiguous()
+
+
+__all__.append("gamma_midpoint_weights")
