@@ -73,7 +73,7 @@ const char* bl_last_error_message(void);
 /*
  * Bytes of device workspace bl_quantize_weight and bl_quantize need for an
  * [N,K] tensor: two arrival counters, one fp64 partial sum of |W| per CTA and
- * 256 exact-sum bins, 10304 bytes for every non-empty tensor. Returns 0 for
+ * 256 exact-sum bins, 10752 bytes for every non-empty tensor. Returns 0 for
  * an empty tensor.
  */
 size_t bl_quantize_weight_workspace_size(int64_t N, int64_t K);
@@ -123,7 +123,7 @@ bl_status bl_quantize_weight(const void* W, bl_dtype w_dtype, int64_t N, int64_t
  * It computes exactly what bl_quantize_weight computes (same kernels, same
  * bit-identical outputs) and calls no allocator. Its scratch -- the arrival
  * counters, partial sums and exact-sum bins that bl_quantize_weight keeps in
- * the caller's workspace -- is a fixed array inside the library of 10304
+ * the caller's workspace -- is a fixed array inside the library of 10752
  * bytes, enough for a tensor of any size; each GPU that loads the library
  * keeps that array until the process exits.
  *

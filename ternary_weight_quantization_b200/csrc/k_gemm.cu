@@ -171,6 +171,7 @@ struct Layout {
   static constexpr int kBytes = kOffMisc + 64;
   static constexpr int kDynBytes = kBytes + 1024;
   static_assert(kS >= 2, "at least two pipeline stages");
+  static_assert(12 * kEpiStageBytes <= kOffEpi, "warps 0..11 stage the last tile's epilogue in the operand stages");
   static_assert(kDynBytes <= kSmemLimit, "shared memory budget");
   static_assert(G::kABytes % 1024 == 0 && G::kBBytes % 1024 == 0 && G::kSrcBytes % 1024 == 0, "alignment");
 };
@@ -610,13 +611,18 @@ __device__ __forceinline__ void epilogue_chunk(const GemmParams& p, const OpPara
 
 // Epilogue, one tile: drain the TMEM accumulator two 32-column chunks per
 // (rolled) iteration; each chunk's TMEM load overlaps the previous chunk's
-// conversion and store, and the buffer is handed back once the last load has
-// landed.
+// conversion and store. The warp takes the chunk pairs pb, pb + ps, ... of
+// its lane quadrant (all of them for a tile whose buffer is handed back
+// afterwards; for a pair's last tile all 16 warps share the pairs). With
+// `release`, the buffer is handed back once the last load has landed.
 template <Op op, int BN, int kSlots>
 __device__ __forceinline__ void epilogue_tile(const GemmParams& p, const OpParams& P, const CUtensorMap* out_map,
                                               uint32_t tmem_base, int buf, uint32_t stg, int lane, int q, int a0,
-                                              int bp, float gamma, uint32_t tmem_empty_lead, uint32_t& seq) {
+                                              int bp, float gamma, int pb, int ps, bool release,
+                                              uint32_t tmem_empty_lead, uint32_t& seq) {
   static_assert(BN % 64 == 0, "chunks are drained in pairs");
+  constexpr int kPairs = BN / 64;
+  if (pb >= kPairs) return;
   const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * 256;
   const int i0 = a0 + q * 32;
   // forward: the warp's table of the tile's column scales s_x[m] * gamma
@@ -631,10 +637,12 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams& p, const OpParam
     __syncwarp();
   }
   uint32_t ra[32], rb[32];
-  tmem_ld_32x32b_x32(tbase, ra);
+  tmem_ld_32x32b_x32(tbase + 64 * pb, ra);
   tmem_ld_wait();
 #pragma unroll 1
-  for (int c = 0; c < BN / 32; c += 2) {
+  for (int pr = pb; pr < kPairs; pr += ps) {
+    const int c = 2 * pr;
+    const bool more = pr + ps < kPairs;
     // forward: s_x[m] * gamma of the two chunks' columns (lane l: column 32c + l)
     float s0 = 0.0f, s1 = 0.0f;
     if constexpr (op == Op::Fwd) {
@@ -645,16 +653,16 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams& p, const OpParam
     tmem_ld_32x32b_x32(tbase + 32 * (c + 1), rb);
     epilogue_chunk<op, kSlots>(p, P, out_map, ra, stg, scales, lane, i0, bp + c * 32, c, s0, gamma, seq);
     tmem_ld_wait();
-    if (c + 2 < BN / 32) {
-      tmem_ld_32x32b_x32(tbase + 32 * (c + 2), ra);
-    } else {
+    if (more) {
+      tmem_ld_32x32b_x32(tbase + 64 * (pr + ps), ra);
+    } else if (release) {
       // every TMEM load of this buffer has landed: hand it back
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(tmem_empty_lead);
     }
     epilogue_chunk<op, kSlots>(p, P, out_map, rb, stg, scales, lane, i0, bp + (c + 1) * 32, c + 1, s1, gamma, seq);
-    if (c + 2 < BN / 32) tmem_ld_wait();
+    if (more) tmem_ld_wait();
   }
 }
 
@@ -864,26 +872,40 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
       }
     }
-  } else if (warp >= kWarpEpi0) {
+  }
+
+  {
     // ------------------------------------------------------------ epilogue (both CTAs)
+    // Warps 12..15 drain every tile's accumulator. A pair's last tile is
+    // shared by all 16 warps: once its MMAs have completed (tmem_full), no
+    // operand stage is read or loaded any more, so the warps that fed the
+    // pipeline join after their own loops and take chunk pairs warp / 4,
+    // + 4, ... of lane quadrant warp % 4, staging in the operand stage area.
+    const bool epi_warp = warp >= kWarpEpi0;
     const int q = warp & 3;  // TMEM lane quadrant this warp may access
-    const uint32_t stg = smem_u32(smem + L::kOffEpi + (warp - kWarpEpi0) * L::kEpiStageBytes);
+    const uint32_t stg = epi_warp ? smem_u32(smem + L::kOffEpi + (warp - kWarpEpi0) * L::kEpiStageBytes)
+                                  : smem_u32(smem + L::kOffA + warp * L::kEpiStageBytes);
     const float gamma = p.gamma ? __ldg(p.gamma) : 1.0f;
     int buf = 0;
     uint32_t buf_phase = 0;
     uint32_t seq = 0;
     int tile;
     for (int i = 0; next_tile(p, pair, npairs, i, tile); ++i) {
-      const TileInfo t = decode_tile<BN>(p, tile, rank);
-      const OpParams& P = p.op[t.opi];
-      if (!wait(&tmem_full[buf], buf_phase)) break;
-      tc_fence_after();
-      if (t.opi == 0)
-        epilogue_tile<kOp0, BN, G::kEpiSlots>(p, P, &map_out0, tmem_base, buf, stg, lane, q, t.a0, t.bp, gamma,
-                                lead(&tmem_empty[buf]), seq);
-      else if constexpr (F == Family::Bwd)
-        epilogue_tile<Op::Dw, BN, G::kEpiSlots>(p, P, &map_out1, tmem_base, buf, stg, lane, q, t.a0, t.bp, gamma,
-                                  lead(&tmem_empty[buf]), seq);
+      int after;
+      const bool last = !next_tile(p, pair, npairs, i + 1, after);
+      if (epi_warp || last) {
+        const TileInfo t = decode_tile<BN>(p, tile, rank);
+        const OpParams& P = p.op[t.opi];
+        if (!wait(&tmem_full[buf], buf_phase)) break;
+        tc_fence_after();
+        const int pb = last ? warp >> 2 : 0, ps = last ? 4 : 1;
+        if (t.opi == 0)
+          epilogue_tile<kOp0, BN, G::kEpiSlots>(p, P, &map_out0, tmem_base, buf, stg, lane, q, t.a0, t.bp, gamma,
+                                                pb, ps, !last, lead(&tmem_empty[buf]), seq);
+        else if constexpr (F == Family::Bwd)
+          epilogue_tile<Op::Dw, BN, G::kEpiSlots>(p, P, &map_out1, tmem_base, buf, stg, lane, q, t.a0, t.bp, gamma,
+                                                  pb, ps, !last, lead(&tmem_empty[buf]), seq);
+      }
       if (++buf == 2) {
         buf = 0;
         buf_phase ^= 1;
@@ -948,7 +970,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_forward_kernel(const __gri
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bar + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bar + 2);
 
-  const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+  const int t = threadIdx.x, warp = t >> 5;
   const uint32_t rank = cluster_ctarank();
   const uint32_t S = gridDim.x;  // the cluster spans the grid's x dimension
   const int n0 = blockIdx.y * kDecRows;

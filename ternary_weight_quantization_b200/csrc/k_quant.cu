@@ -43,15 +43,19 @@ __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w 
 // ---------------------------------------------------------------- S1 geometry
 constexpr int kQThreads = 512;                 // 16 warps per CTA
 constexpr int kQWarps = kQThreads / 32;
-constexpr int kTokenWarp0 = 8;                 // with tokens: warps 8..15 run S2
 constexpr int kChunkBytes = 16384;             // one bulk copy of the slice
 constexpr int kMaxOnchipBytes = 220 * 1024;    // slice bytes held in shared memory
 constexpr int kMaxChunks = kMaxOnchipBytes / kChunkBytes + 1;
-constexpr int kBarWarpsNamed = 1;              // named barrier id of the slice warps
 
-// Workspace: [0, 8) two arrival counters; [64, 64 + 8 kMaxCtas) fp64 partial
-// sums, one per CTA; then 256 uint64 exact-sum bins (one per exponent field).
-constexpr size_t kWsPartials = 64;
+// Workspace (each part on its own 128-byte lines): at 0 the arrivals at the
+// partial-sum and at the exact-sum barrier (u32 each); at 128 the gamma flag
+// (1: gamma published, 2: the exact sum is needed) and gamma's bits; at 256
+// the next token row to claim; at 512 one fp64 partial sum per CTA; then 256
+// uint64 exact-sum bins (one per exponent field).
+constexpr size_t kWsArrive = 0;
+constexpr size_t kWsFlag = 128;
+constexpr size_t kWsRows = 256;
+constexpr size_t kWsPartials = 512;
 constexpr size_t kWsBins = kWsPartials + 8 * static_cast<size_t>(kMaxQuantCtas);
 constexpr size_t kWsBytes = kWsBins + 8 * 256;
 
@@ -193,18 +197,20 @@ __device__ __forceinline__ float gamma_of_sum(double S, double numel) {
 // field 00 = 0, 01 = +1, 11 = -1). For a 15-bit magnitude b and thr > 0,
 // |w| > thr <=> b > bits(thr) >> 16, so both halves of a word are compared by
 // one subtraction: 0x8000 + tb - b keeps bit 15 clear exactly when b > tb (no
-// borrow crosses the halves, b <= 0x7FFF).
+// borrow crosses the halves, b <= 0x7FFF). The low elements' fields collect at
+// bits 4j, 4j + 1 and the high elements' at 16 + 4j, 17 + 4j of one word, then
+// one fold moves the high ones to 4j + 2, 4j + 3 (about four operations per
+// element).
 __device__ __forceinline__ uint32_t codes8_bf16(const uint4& v, uint32_t bias) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-  uint32_t r = 0;
+  uint32_t acc = 0;
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
-    const uint32_t nz = ~(bias - (w[j] & 0x7FFF7FFFu)) & 0x80008000u;  // bits 15, 31
+    const uint32_t nz = ~(bias - (w[j] & 0x7FFF7FFFu)) & 0x80008000u;  // bits 15, 31: nonzero code
     const uint32_t nn = nz & w[j];                                     // and negative
-    r |= ((nz >> 15) & 1u) << (4 * j) | ((nn >> 15) & 1u) << (4 * j + 1) | (nz >> 31) << (4 * j + 2) |
-         (nn >> 31) << (4 * j + 3);
+    acc |= (nz >> (15 - 4 * j)) | (nn >> (14 - 4 * j));
   }
-  return r;
+  return (acc & 0x3333u) | ((acc >> 14) & 0xCCCCu);
 }
 
 // 4 fp32 of one vector -> 8 bits of codes.
@@ -263,10 +269,6 @@ __device__ __forceinline__ bool grid_arrive_wait(uint32_t* ctr, uint32_t expecte
       return false;
     }
   }
-}
-
-__device__ __forceinline__ void named_barrier_sync(int id, int threads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
 __device__ __forceinline__ void bulk_copy_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
@@ -425,16 +427,21 @@ __global__ void __launch_bounds__(32 * kActRowsPerBlock) act_quant_long_kernel(c
 }
 
 // ---------------------------------------------------------------- S1 (+ S2): the launches
-// Launch 1: clears the workspace's two arrival counters and its exact-sum
-// bins. It waits for the kernel before it in the stream (whose work may
-// still read them), and only then lets the quantisation launch start; so the
+// Launch 1: clears the workspace's counters, flag and exact-sum bins. It
+// waits for the kernel before it in the stream (whose work may still use
+// them), and only then lets the quantisation launch start; so the
 // quantisation may read W and x and write its outputs from its first
 // instruction, and waits for this launch itself only before its first use of
-// the counters.
+// the workspace.
 __global__ void __launch_bounds__(256) quant_reset_kernel(uint8_t* __restrict__ ws) {
   pdl_wait_primary();
   pdl_launch_dependents();
-  if (threadIdx.x < 2) reinterpret_cast<uint32_t*>(ws)[threadIdx.x] = 0u;
+  if (threadIdx.x == 0) {
+    reinterpret_cast<uint32_t*>(ws + kWsArrive)[0] = 0u;
+    reinterpret_cast<uint32_t*>(ws + kWsArrive)[1] = 0u;
+    reinterpret_cast<uint32_t*>(ws + kWsFlag)[0] = 0u;
+    reinterpret_cast<uint32_t*>(ws + kWsRows)[0] = 0u;
+  }
   reinterpret_cast<unsigned long long*>(ws + kWsBins)[threadIdx.x] = 0ull;
 }
 
@@ -456,27 +463,86 @@ struct QuantArgs {
   float* sx;
 };
 
-// Launch 2. Warps 0..7 (all 16 without tokens) work on the CTA's W slice;
-// warps 8..15 quantise tokens m = 8 b + w - 8 + 8 G i. Rows of up to 2560
-// elements (VPL <= 10) stay in registers; longer ones (VPL = 0) are read twice.
+__device__ __forceinline__ void st_release_u32(uint32_t* p, uint32_t v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Lane 0 claims `n` consecutive items of a counter, the warp gets the first.
+__device__ __forceinline__ uint32_t warp_claim(uint32_t* ctr, uint32_t n) {
+  uint32_t m = 0;
+  if ((threadIdx.x & 31) == 0) m = atomicAdd(ctr, n);
+  return __shfl_sync(0xffffffffu, m, 0);
+}
+
+// Token rows m0, m0 + 1 (those below M): both rows' loads are issued before
+// either is quantised. Rows longer than 2560 elements (VPL = 0) are read twice
+// (absmax, then quantisation from L1/L2).
+template <int VPL>
+__device__ __forceinline__ void token_pair(const QuantArgs& a, int64_t m0) {
+  const int lane = threadIdx.x & 31;
+  if constexpr (VPL > 0) {
+    uint4 v0[VPL], v1[VPL];
+    load_row<VPL>(a.x + m0 * a.nv, a.nv, lane, v0);
+    const bool two = m0 + 1 < a.M;
+    if (two) load_row<VPL>(a.x + (m0 + 1) * a.nv, a.nv, lane, v1);
+    quant_row<VPL>(v0, a.nv, lane, m0, a.xq, a.sx);
+    if (two) quant_row<VPL>(v1, a.nv, lane, m0 + 1, a.xq, a.sx);
+  } else {
+    act_rows_two_pass(a.x, m0 + 2 < a.M ? m0 + 2 : a.M, a.nv, a.xq, a.sx, m0, 1);
+  }
+}
+
+// Codes of 128 consecutive 16-byte vectors of W from shared memory (kShared)
+// or global memory: lane l takes vectors l, l + 32, l + 64, l + 96 (all loads
+// first, conflict-free shared loads); a group's V lanes combine their bits and
+// its first lane stores the group's word.
+template <bool kF32, bool kShared>
+__device__ __forceinline__ void code_round(const uint4* src, int64_t base, int64_t nvec, uint32_t* out, uint32_t key,
+                                           int lane) {
+  constexpr int V = kF32 ? 4 : 2;
+  uint4 v[4];
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int64_t i = base + lane + 32 * u;
+    v[u] = make_uint4(0u, 0u, 0u, 0u);
+    if (i < nvec) v[u] = kShared ? src[i] : __ldg(src + i);
+  }
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int64_t i = base + lane + 32 * u;
+    const uint32_t word = gather_group_word<kF32>(vec_codes<kF32>(v[u], key), lane);
+    if (i < nvec && (lane & (V - 1)) == 0) out[i / V] = word;
+  }
+}
+
+// Launch 2, 512 threads. Every warp first sums |W| of the CTA's slice as its
+// bulk copies land (W, which gates every code, is read before any token);
+// thread 0 then publishes the CTA's partial sum and arrives. Warp 0 becomes the
+// control warp: the last CTA to arrive forms gamma from all partial sums (in
+// one fixed order) and publishes it; the others wait for it. Meanwhile the
+// other warps quantise token rows claimed from a counter shared by the grid;
+// once gamma is known every warp takes rounds of 128 code vectors from a
+// counter of the CTA, and then token rows again until none is left. If the
+// enclosure of S straddles a rounding boundary of gamma (rare), every warp
+// first bins its share of the slice for the exact sum.
 template <bool kF32, int VPL>
 __global__ void __launch_bounds__(kQThreads, 1) quant_fused_kernel(const __grid_constant__ QuantArgs a) {
   constexpr int V = kF32 ? 4 : 2;  // 16-byte vectors per group
   constexpr int kGroupBytes = 16 * V;
   constexpr int kChunkGroups = kChunkBytes / kGroupBytes;
-  constexpr int kTailRegs = 4;
+  constexpr int kTailRegs = 2;
   extern __shared__ __align__(128) uint4 s_w[];
   __shared__ __align__(8) uint64_t s_bar[kMaxChunks];
   __shared__ unsigned long long s_bins[256];
   __shared__ double s_red[kQWarps];
   __shared__ float s_gamma;
-  __shared__ int s_mode;   // after the partial sums: 0 codes, 1 exact sum first
-  __shared__ int s_abort;  // a wait of this CTA gave up
+  __shared__ uint32_t s_key;
+  __shared__ int s_state;   // 0: gamma not known, 1: known, 2: bin for the exact sum, -1: abort
+  __shared__ int s_round;   // next code round of this CTA
+  __shared__ int s_binned;  // warps done binning
+  __shared__ int s_abort;   // a wait of this CTA gave up
 
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const bool tokens = a.M > 0;
-  const int nww = tokens ? kTokenWarp0 : kQWarps;
-  const int nthr = 32 * nww;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, t = threadIdx.x;
   const int64_t b = blockIdx.x;
   const uint32_t G = gridDim.x;
   const int64_t g0 = b * a.per;
@@ -484,16 +550,23 @@ __global__ void __launch_bounds__(kQThreads, 1) quant_fused_kernel(const __grid_
   const int64_t len = rest <= 0 ? 0 : (rest < a.per ? rest : a.per);
   const int on = static_cast<int>(len < a.onchip_cap ? len : a.onchip_cap);
   const int nch = (on + kChunkGroups - 1) / kChunkGroups;
-  uint32_t* ctr = reinterpret_cast<uint32_t*>(a.ws);
+  const int64_t onv = static_cast<int64_t>(on) * V;
+  const int64_t tail_v0 = (g0 + on) * V, tail_v1 = (g0 + len) * V;
+  uint32_t* arrive = reinterpret_cast<uint32_t*>(a.ws + kWsArrive);  // [0] partial sums, [1] exact sum
+  uint32_t* flag = reinterpret_cast<uint32_t*>(a.ws + kWsFlag);      // [0] 1 gamma / 2 exact, [1] gamma bits
+  uint32_t* rows = reinterpret_cast<uint32_t*>(a.ws + kWsRows);
   double* partials = reinterpret_cast<double*>(a.ws + kWsPartials);
   unsigned long long* gbins = reinterpret_cast<unsigned long long*>(a.ws + kWsBins);
 
-  if (threadIdx.x == 0) {
+  if (t == 0) {
     s_abort = 0;
+    s_state = 0;
+    s_round = 0;
+    s_binned = 0;
     for (int c = 0; c < nch; ++c) mbar_init(&s_bar[c], 1);
     fence_mbar_init();
     fence_proxy_async_smem();
-    // the whole on-chip slice in flight at once, before any token load
+    // the whole on-chip slice in flight at once
     for (int c = 0; c < nch; ++c) {
       const int cg0 = c * kChunkGroups;
       const int cgn = min(kChunkGroups, on - cg0);
@@ -504,26 +577,12 @@ __global__ void __launch_bounds__(kQThreads, 1) quant_fused_kernel(const __grid_
   }
   __syncthreads();
 
-  if (warp >= nww) {
-    // ------------------------------------------------ S2 tokens
-    constexpr int kTokWarps = kQWarps - kTokenWarp0;
-    const int64_t m = b * kTokWarps + (warp - kTokenWarp0);
-    const int64_t stride = static_cast<int64_t>(G) * kTokWarps;
-    if constexpr (VPL > 0)
-      act_rows<VPL, false>(a.x, a.M, a.nv, a.xq, a.sx, m, stride);
-    else
-      act_rows_two_pass(a.x, a.M, a.nv, a.xq, a.sx, m, stride);
-    return;
-  }
-
-  // -------------------------------------------------- S1 slice warps
-  const int t = threadIdx.x;
-  const int64_t tail_v0 = (g0 + on) * V, tail_v1 = (g0 + len) * V;
-  // first vectors of the off-chip tail, loaded before the chunks are summed
+  // -------------------------------------------------- |W| of the slice, all warps
+  // thread t takes vectors t, t + 512, ... of each chunk, then of the tail
   uint4 tr[kTailRegs];
 #pragma unroll
   for (int u = 0; u < kTailRegs; ++u) {
-    const int64_t i = tail_v0 + t + static_cast<int64_t>(u) * nthr;
+    const int64_t i = tail_v0 + t + static_cast<int64_t>(u) * kQThreads;
     tr[u] = i < tail_v1 ? __ldg(a.W + i) : make_uint4(0u, 0u, 0u, 0u);
   }
   double acc[4] = {0.0, 0.0, 0.0, 0.0};
@@ -534,116 +593,194 @@ __global__ void __launch_bounds__(kQThreads, 1) quant_fused_kernel(const __grid_
     }
     const int v1 = min((c + 1) * kChunkGroups, on) * V;
     int i = c * kChunkGroups * V + t;
-    for (; i + 3 * nthr < v1; i += 4 * nthr) {
-      acc[0] = add_abs<kF32>(acc[0], s_w[i]);
-      acc[1] = add_abs<kF32>(acc[1], s_w[i + nthr]);
-      acc[2] = add_abs<kF32>(acc[2], s_w[i + 2 * nthr]);
-      acc[3] = add_abs<kF32>(acc[3], s_w[i + 3 * nthr]);
-    }
-    if (i < v1) acc[0] = add_abs<kF32>(acc[0], s_w[i]);
-    if (i + nthr < v1) acc[1] = add_abs<kF32>(acc[1], s_w[i + nthr]);
-    if (i + 2 * nthr < v1) acc[2] = add_abs<kF32>(acc[2], s_w[i + 2 * nthr]);
-  }
-  {
-    // the tail: the vectors already in registers, then the rest four at a time
-#pragma unroll
-    for (int u = 0; u < kTailRegs; ++u)
-      if (tail_v0 + t + static_cast<int64_t>(u) * nthr < tail_v1) acc[u] = add_abs<kF32>(acc[u], tr[u]);
-    for (int64_t i = tail_v0 + t + static_cast<int64_t>(kTailRegs) * nthr; i < tail_v1; i += 4 * nthr) {
+    for (; i + 3 * kQThreads < v1; i += 4 * kQThreads) {
       uint4 v[4];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) v[u] = i + u * nthr < tail_v1 ? __ldg(a.W + i + u * nthr) : make_uint4(0u, 0u, 0u, 0u);
+      for (int u = 0; u < 4; ++u) v[u] = s_w[i + u * kQThreads];
 #pragma unroll
-      for (int u = 0; u < 4; ++u)
-        if (i + u * nthr < tail_v1) acc[u] = add_abs<kF32>(acc[u], v[u]);
+      for (int u = 0; u < 4; ++u) acc[u] = add_abs<kF32>(acc[u], v[u]);
     }
+    if (i < v1) acc[0] = add_abs<kF32>(acc[0], s_w[i]);
+    if (i + kQThreads < v1) acc[1] = add_abs<kF32>(acc[1], s_w[i + kQThreads]);
+    if (i + 2 * kQThreads < v1) acc[2] = add_abs<kF32>(acc[2], s_w[i + 2 * kQThreads]);
+  }
+#pragma unroll
+  for (int u = 0; u < kTailRegs; ++u)
+    if (tail_v0 + t + static_cast<int64_t>(u) * kQThreads < tail_v1) acc[u] = add_abs<kF32>(acc[u], tr[u]);
+  for (int64_t i = tail_v0 + t + static_cast<int64_t>(kTailRegs) * kQThreads; i < tail_v1; i += 4 * kQThreads) {
+    uint4 v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) v[u] = i + u * kQThreads < tail_v1 ? __ldg(a.W + i + u * kQThreads) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      if (i + u * kQThreads < tail_v1) acc[u] = add_abs<kF32>(acc[u], v[u]);
   }
   double ts = __dadd_rn(__dadd_rn(acc[0], acc[1]), __dadd_rn(acc[2], acc[3]));
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) ts = __dadd_rn(ts, __shfl_xor_sync(0xffffffffu, ts, off));
   if (lane == 0) s_red[warp] = ts;
-  named_barrier_sync(kBarWarpsNamed, nthr);
+  __syncthreads();
+  // the next launch may be scheduled once every CTA of this grid has come
+  // this far (so all of them are resident)
+  pdl_launch_dependents();
 
-  if (t == 0) {
-    double part = 0.0;
-    for (int w = 0; w < nww; ++w) part = __dadd_rn(part, s_red[w]);
-    partials[b] = part;
-    pdl_wait_primary();  // launch 1 has cleared the counters
-    if (!grid_arrive_wait(&ctr[0], G, a.err)) s_abort = 1;
-  }
-  named_barrier_sync(kBarWarpsNamed, nthr);
-  pdl_launch_dependents();  // every CTA is resident (all arrived): the next launch may be scheduled
-
-  if (warp == 0 && !s_abort) {
-    // the partial sums in one fixed order: lane l adds l, l + 32, ..., then a
-    // fixed shuffle tree
-    double s = 0.0;
-    for (uint32_t j = lane; j < G; j += 32) s = __dadd_rn(s, __ldcg(partials + j));
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) s = __dadd_rn(s, __shfl_xor_sync(0xffffffffu, s, off));
+  if (warp == 0) {
+    // ------------------------------------------------ control warp: gamma
+    uint32_t last = 0;
     if (lane == 0) {
+      double part = 0.0;
+      for (int w = 0; w < kQWarps; ++w) part = __dadd_rn(part, s_red[w]);
+      partials[b] = part;
+      pdl_wait_primary();  // launch 1 has cleared the workspace
+      __threadfence();
+      last = atomicAdd(&arrive[0], 1u) == G - 1;
+      __threadfence();  // with the atomic: acquires the other CTAs' partial sums
+    }
+    last = __shfl_sync(0xffffffffu, last, 0);
+    int mode = 0;
+    float gamma = 0.0f;
+    if (last) {
+      // the partial sums in one fixed order: lane l adds l, l + 32, ..., then a
+      // fixed shuffle tree (the same sum whichever CTA forms it)
+      double s = 0.0;
+      for (uint32_t j = lane; j < G; j += 32) s = __dadd_rn(s, __ldcg(partials + j));
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) s = __dadd_rn(s, __shfl_xor_sync(0xffffffffu, s, off));
       const float glo = gamma_of_sum(__dmul_rd(s, a.enc_lo), a.numel);
       const float ghi = gamma_of_sum(__dmul_ru(s, a.enc_hi), a.numel);
-      s_gamma = glo;
-      s_mode = __float_as_uint(glo) == __float_as_uint(ghi) ? 0 : 1;
+      mode = __float_as_uint(glo) == __float_as_uint(ghi) ? 1 : 2;
+      gamma = glo;
+      if (lane == 0) {
+        flag[1] = __float_as_uint(glo);
+        st_release_u32(&flag[0], static_cast<uint32_t>(mode));
+      }
+    } else {
+      if (lane == 0) {
+        // wait for the last CTA's gamma (bounded; polled every ~0.1 us)
+        uint32_t f = ld_acquire_u32(&flag[0]);
+        const unsigned long long t0 = globaltimer_ns();
+        while (f == 0) {
+          __nanosleep(100);
+          f = ld_acquire_u32(&flag[0]);
+          if (f == 0 && globaltimer_ns() - t0 > kWaitLimitNs) {
+            record_error(a.err, kDevTimeout);
+            break;
+          }
+        }
+        mode = static_cast<int>(f);
+        gamma = __uint_as_float(__ldcg(&flag[1]));
+      }
+      mode = __shfl_sync(0xffffffffu, mode, 0);
+      gamma = __shfl_sync(0xffffffffu, gamma, 0);
     }
-  }
-  named_barrier_sync(kBarWarpsNamed, nthr);
-
-  if (!s_abort && s_mode == 1) {
-    // ------------------------------------------------ exact sum (rare)
-    for (int e = t; e < 256; e += nthr) s_bins[e] = 0ull;
-    named_barrier_sync(kBarWarpsNamed, nthr);
-    for (int i = t; i < on * V; i += nthr) bin_abs<kF32>(s_bins, s_w[i]);
-    for (int64_t i = tail_v0 + t; i < tail_v1; i += nthr) bin_abs<kF32>(s_bins, __ldg(a.W + i));
-    named_barrier_sync(kBarWarpsNamed, nthr);
-    for (int e = t; e < 256; e += nthr)
-      if (s_bins[e]) atomicAdd(gbins + e, s_bins[e]);
-    named_barrier_sync(kBarWarpsNamed, nthr);
-    if (t == 0) {
-      if (!grid_arrive_wait(&ctr[1], G, a.err)) {
-        s_abort = 1;
-      } else {
-        s_gamma = gamma_of_sum(exact_sum_from_bins(gbins, kF32 ? 23 : 7), a.numel);
+    if (mode == 0 || s_abort) {
+      if (lane == 0) s_state = -1;
+    } else {
+      if (mode == 2) {
+        // exact sum: every warp bins its share of the slice (the work loop
+        // below); then one arrival per CTA and the exact gamma
+        for (int e = lane; e < 256; e += 32) s_bins[e] = 0ull;
+        __syncwarp();
+        if (lane == 0) {
+          __threadfence_block();
+          s_state = 2;
+        }
+        bool ok = true;
+        if (lane == 0) {
+          const unsigned long long t0 = globaltimer_ns();
+          while (*reinterpret_cast<volatile int*>(&s_binned) < kQWarps - 1) {
+            __nanosleep(100);
+            if (globaltimer_ns() - t0 > kWaitLimitNs) {
+              record_error(a.err, kDevTimeout);
+              ok = false;
+              break;
+            }
+          }
+        }
+        // warp 0's own share
+        for (int64_t i = lane; i < onv; i += 32 * kQWarps) bin_abs<kF32>(s_bins, s_w[i]);
+        for (int64_t i = tail_v0 + lane; i < tail_v1; i += 32 * kQWarps) bin_abs<kF32>(s_bins, __ldg(a.W + i));
+        __syncwarp();
+        __threadfence_block();
+        for (int e = lane; e < 256; e += 32)
+          if (s_bins[e]) atomicAdd(gbins + e, s_bins[e]);
+        __syncwarp();  // every lane's bins are added before lane 0 arrives
+        if (lane == 0 && ok) {
+          ok = grid_arrive_wait(&arrive[1], G, a.err);
+          if (ok) gamma = gamma_of_sum(exact_sum_from_bins(gbins, kF32 ? 23 : 7), a.numel);
+        }
+        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        gamma = __shfl_sync(0xffffffffu, gamma, 0);
+        if (!ok) mode = 0;
+      }
+      if (lane == 0) {
+        if (mode == 0) {
+          s_state = -1;
+        } else {
+          if (b == 0) *a.gamma_out = gamma;
+          const float thr = __double2float_rd(__dmul_rn(static_cast<double>(gamma), 0.5 + 0x1p-25));
+          uint32_t key;
+          if constexpr (kF32) {
+            key = __float_as_uint(thr);
+          } else {
+            const uint32_t tb = __float_as_uint(thr) >> 16;
+            key = (tb | (tb << 16)) + 0x80008000u;
+          }
+          s_key = key;
+          s_gamma = gamma;
+          __threadfence_block();
+          s_state = 1;
+        }
       }
     }
-    named_barrier_sync(kBarWarpsNamed, nthr);
+    __syncwarp();
   }
 
-  if (s_abort) {
-    // let every copy already issued land before the CTA exits (one bound)
-    if (t == 0) {
-      const unsigned long long deadline = globaltimer_ns() + kWaitLimitNs;
-      for (int c = 0; c < nch; ++c) mbar_drain_until(&s_bar[c], 0, deadline);
+  // -------------------------------------------------- work loop, all warps
+  const int64_t on_rounds = (onv + 127) / 128;
+  const int64_t n_rounds = on_rounds + (tail_v1 - tail_v0 + 127) / 128;
+  bool rows_left = a.M > 0;
+  bool binned = warp == 0;  // warp 0 bins inside the control block
+  if (rows_left) pdl_wait_primary();  // launch 1 has cleared the row counter
+  volatile int* state = &s_state;
+  const unsigned long long t_idle = globaltimer_ns();
+  for (;;) {
+    const int st = *state;
+    if (st < 0) break;
+    if (st == 2 && !binned) {
+      for (int64_t i = lane + 32 * warp; i < onv; i += 32 * kQWarps) bin_abs<kF32>(s_bins, s_w[i]);
+      for (int64_t i = tail_v0 + lane + 32 * warp; i < tail_v1; i += 32 * kQWarps) bin_abs<kF32>(s_bins, __ldg(a.W + i));
+      __syncwarp();
+      __threadfence_block();
+      if (lane == 0) atomicAdd(&s_binned, 1);
+      binned = true;
+      continue;
     }
-    return;
-  }
-
-  // -------------------------------------------------- codes
-  const float gamma = s_gamma;
-  if (b == 0 && t == 0) *a.gamma_out = gamma;
-  const float thr = __double2float_rd(__dmul_rn(static_cast<double>(gamma), 0.5 + 0x1p-25));
-  uint32_t key;
-  if constexpr (kF32) {
-    key = __float_as_uint(thr);
-  } else {
-    const uint32_t tb = __float_as_uint(thr) >> 16;
-    key = (tb | (tb << 16)) + 0x80008000u;
-  }
-  // lanes take consecutive 16-byte vectors (conflict-free shared loads); a
-  // group's V lanes combine their bits and its first lane stores the word
-  uint32_t* out = a.packed + g0;
-  for (int base = 32 * warp; base < on * V; base += 32 * nww) {
-    const int i = base + lane;
-    const bool valid = i < on * V;
-    const uint32_t word = gather_group_word<kF32>(valid ? vec_codes<kF32>(s_w[i], key) : 0u, lane);
-    if (valid && (lane & (V - 1)) == 0) out[i / V] = word;
-  }
-  for (int64_t base = tail_v0 + 32 * warp; base < tail_v1; base += 32 * nww) {
-    const int64_t i = base + lane;
-    const bool valid = i < tail_v1;
-    const uint32_t word = gather_group_word<kF32>(valid ? vec_codes<kF32>(__ldg(a.W + i), key) : 0u, lane);
-    if (valid && (lane & (V - 1)) == 0) a.packed[i / V] = word;
+    if (st == 1) {
+      uint32_t r = 0;
+      if (lane == 0) r = static_cast<uint32_t>(atomicAdd(&s_round, 1));
+      r = __shfl_sync(0xffffffffu, r, 0);
+      if (r < n_rounds) {
+        const uint32_t key = s_key;
+        if (r < on_rounds)
+          code_round<kF32, true>(s_w, 128 * static_cast<int64_t>(r), onv, a.packed + g0, key, lane);
+        else
+          code_round<kF32, false>(a.W + tail_v0, 128 * (r - on_rounds), tail_v1 - tail_v0, a.packed + g0 + on, key,
+                                  lane);
+        continue;
+      }
+    }
+    if (rows_left) {
+      const int64_t m0 = warp_claim(rows, 2u);
+      if (m0 < a.M) {
+        token_pair<VPL>(a, m0);
+        continue;
+      }
+      rows_left = false;
+    }
+    if (st == 1) break;  // codes all claimed, no rows left
+    __nanosleep(200);    // waiting for gamma
+    if (globaltimer_ns() - t_idle > 2 * kWaitLimitNs) break;  // the control warp gave up
   }
 }
 
@@ -651,7 +788,7 @@ __global__ void __launch_bounds__(kQThreads, 1) quant_fused_kernel(const __grid_
 
 // Fixed device scratch for bl_quantize_weight_noalloc: the workspace of one
 // call (arrival counters, one fp64 partial sum per CTA, exact-sum bins),
-// 10304 bytes. Every GPU that loads the library holds this array until the
+// 10752 bytes. Every GPU that loads the library holds this array until the
 // process exits.
 static __device__ __align__(256) uint8_t g_noalloc_ws[kWsBytes];
 
@@ -687,7 +824,7 @@ QuantGeometry quant_geometry(int64_t ngroups, int64_t M, QuantArgs& a) {
   // that is at most S (1 + 2^-30) with all terms >= 0, so |fp64 sum - S| <=
   // d 2^-53 (1 + 2^-30) S; e = d 2^-52 covers S on both sides.
   const int64_t nch_max = (on_max + kChunkGroups - 1) / kChunkGroups;
-  const double per_acc = static_cast<double>(a.per) * V / (4.0 * 32 * kTokenWarp0) + static_cast<double>(nch_max) + 3.0;
+  const double per_acc = static_cast<double>(a.per) * V / (4.0 * kQThreads) + static_cast<double>(nch_max) + 3.0;
   const double d = kElems * per_acc + 2 + 5 + kQWarps + std::ceil(static_cast<double>(G) / 32.0) + 5 + 8;
   const double e = std::ldexp(d, -52);
   a.enc_lo = 1.0 - e;
