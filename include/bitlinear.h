@@ -72,9 +72,9 @@ const char* bl_last_error_message(void);
 
 /*
  * Bytes of device workspace bl_quantize_weight and bl_quantize need for an
- * [N,K] tensor: two arrival counters, one fp64 partial sum of |W| per CTA and
- * 256 exact-sum bins, 10752 bytes for every non-empty tensor. Returns 0 for
- * an empty tensor.
+ * [N,K] tensor: an arrival counter and 256 exact-sum bins, and one fp64
+ * partial sum of |W| per CTA of the summing launch (at most 1024), 10496
+ * bytes for every non-empty tensor. Returns 0 for an empty tensor.
  */
 size_t bl_quantize_weight_workspace_size(int64_t N, int64_t K);
 
@@ -95,17 +95,21 @@ size_t bl_quantize_weight_workspace_size(int64_t N, int64_t K);
  * workspace device scratch of at least bl_quantize_weight_workspace_size(N,K)
  *           bytes, 16-byte aligned; contents need no initialisation and are
  *           overwritten.
- * gamma is exact: the fp64 sum of |W| is taken in a fixed tree and carries a
- * bounded rounding error; gamma is formed at both ends of that enclosure of
- * the exact sum, and where the two differ (about one tensor in 10^5) the
- * library sums |W| exactly in integers and rounds once. gamma therefore never
- * depends on the summation order or on the GPU, and the same W gives
- * bit-identical outputs on every call.
- * Launches: a one-CTA launch that clears the workspace's counters, then one
- * persistent launch (at most one CTA per SM, all resident at once; they meet
- * at a grid-wide barrier whose wait is bounded: a barrier that cannot
- * complete -- e.g. SMs held by other work for seconds -- records
- * BL_ERR_TIMEOUT in the device error word).
+ * gamma is exact: the fp64 sum of |W| (per-CTA trees, then the CTAs' sums in
+ * a fixed order) carries a bounded rounding error; gamma is formed at both
+ * ends of that enclosure of the exact sum, and
+ * where the two differ (about one tensor in 10^5) the library sums |W|
+ * exactly in integers and rounds once. gamma therefore never depends on the
+ * summation order or on the GPU, and the same W gives bit-identical outputs
+ * on every call.
+ * Launches: a summing launch (each CTA stores the fp64 sum of |W| over its
+ * slice of W; nothing waits) and a coding launch that starts once the first
+ * has completed (every CTA forms gamma from the partial sums and writes the
+ * codes of its share, reading W again, mostly from L2). Only in the rare
+ * exact-sum case do the coding CTAs (never more than can be resident at
+ * once) meet at a grid-wide barrier; its wait is bounded: a barrier that
+ * cannot complete -- e.g. SMs held by other work for seconds -- records
+ * BL_ERR_TIMEOUT in the device error word.
  * Errors: BL_ERR_INVALID_ARG, BL_ERR_UNSUPPORTED_SHAPE (K % 32), BL_ERR_DTYPE,
  *         BL_ERR_ALIGNMENT, BL_ERR_WORKSPACE, BL_ERR_ARCH, BL_ERR_CUDA.
  */
@@ -122,9 +126,9 @@ bl_status bl_quantize_weight(const void* W, bl_dtype w_dtype, int64_t N, int64_t
  *
  * It computes exactly what bl_quantize_weight computes (same kernels, same
  * bit-identical outputs) and calls no allocator. Its scratch -- the arrival
- * counters, partial sums and exact-sum bins that bl_quantize_weight keeps in
- * the caller's workspace -- is a fixed array inside the library of 10752
- * bytes, enough for a tensor of any size; each GPU that loads the library
+ * counter, the exact-sum bins and the partial sums that bl_quantize_weight
+ * keeps in the caller's workspace -- is a fixed array inside the library of
+ * 10496 bytes, enough for a tensor of any size; each GPU that loads the library
  * keeps that array until the process exits.
  *
  * Each call looks up the array's device address on the current device (a
@@ -133,10 +137,10 @@ bl_status bl_quantize_weight(const void* W, bl_dtype w_dtype, int64_t N, int64_t
  * The address is not cached, so a call after the caller reset the device
  * finds the array where the reloaded device code put it. All calls share the
  * one array and nothing in it needs to start at zero (each call clears its
- * counters and bins before use and overwrites the rest), but two calls whose
+ * counter and bins before use and overwrites the rest), but two calls whose
  * kernels overlap on the GPU -- on different streams of one device without
- * ordering between them -- race on it and may produce wrong codes or a
- * barrier timeout: order them on one stream or with events.
+ * ordering between them -- race on it and may produce a wrong gamma and
+ * codes or a barrier timeout: order them on one stream or with events.
  *
  * Arguments, outputs and errors: as bl_quantize_weight, without the
  * workspace pair.
@@ -161,9 +165,10 @@ bl_status bl_quantize_act(const void* x, int64_t M, int64_t K,
 /*
  * S1 + S2 in one call: the same outputs as bl_quantize_weight(W, ...) followed
  * by bl_quantize_act(x, ...), bit for bit. The two steps are independent, so
- * S2 runs in the same persistent launch as S1, on other warps, while W is
- * copied into shared memory and summed. (The pages run the two quantisers
- * one after the other; this is a scheduling choice only.)
+ * S2 runs in S1's summing launch: each CTA quantises its share of the token
+ * rows, then sums its slice of W, so that both streams share HBM in one
+ * pass. (The pages run the two quantisers one after the other; this is a
+ * scheduling choice only.)
  *
  * Arguments: those of bl_quantize_weight and bl_quantize_act. M == 0 skips
  * S2 (x, xq, sx may then be NULL). Errors: as bl_quantize_weight, plus those

@@ -26,18 +26,19 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
   return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
 }
 
-// ---- S1: absmean ternarisation + 2-bit packing (with S2 in the same launch)
-// Most CTAs of one quantisation launch (one per SM at most; they meet at a
-// grid-wide barrier, so all must be resident together).
+// ---- S1: absmean ternarisation + 2-bit packing (with S2 in the same launches)
+// Most CTAs of the sum launch of S1 (one fp64 partial sum each).
 constexpr int kMaxQuantCtas = 1024;
 
-// Bytes of the S1 workspace (arrival counters, one fp64 partial sum per CTA,
-// exact-sum bins); the same for every tensor size. Needs no initialisation.
+// Bytes of the S1 workspace (exact-sum arrival counter and bins, one fp64
+// partial sum per CTA of the sum launch); the same for every tensor size.
+// Needs no initialisation.
 size_t quantize_workspace_bytes();
 
-// S1 on W [N,K] and, when M > 0, S2 on x [M,K] in one launch (after a one-CTA
-// launch that clears the workspace's counters). `err` is the device error
-// word (a barrier wait that gave up records a timeout there).
+// S1 on W [N,K] and, when M > 0, S2 on x [M,K]: a sum launch (|W| partial
+// sums and the token rows) and a code launch (gamma and the codes). `err` is
+// the device error word (an exact-sum barrier wait that gave up records a
+// timeout there).
 cudaError_t launch_quantize(const void* W, int w_is_f32, int64_t N, int64_t K, const void* x, int64_t M,
                             uint8_t* packed, float* gamma, void* workspace, int8_t* xq, float* sx, int* err,
                             cudaStream_t s);

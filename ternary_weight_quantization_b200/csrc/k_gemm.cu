@@ -876,28 +876,36 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 
   {
     // ------------------------------------------------------------ epilogue (both CTAs)
-    // Warps 12..15 drain every tile's accumulator. A pair's last tile is
-    // shared by all 16 warps: once its MMAs have completed (tmem_full), no
-    // operand stage is read or loaded any more, so the warps that fed the
-    // pipeline join after their own loops and take chunk pairs warp / 4,
-    // + 4, ... of lane quadrant warp % 4, staging in the operand stage area.
+    // Warps 12..15 drain every tile's accumulator, waiting on tmem_full tile
+    // by tile (they hand each buffer back, so they are never two phases
+    // behind it). A pair's last tile is shared by all 16 warps: warps 0..11
+    // join after their own loops, once done_bar (committed after the pair's
+    // last MMA, used once, so its phase cannot be mistaken) shows that every
+    // MMA has completed; no operand stage is then read or loaded any more, so
+    // they stage their output boxes in the operand stage area. Warp w takes
+    // chunk pairs w / 4, + 4, ... of lane quadrant w % 4.
     const bool epi_warp = warp >= kWarpEpi0;
     const int q = warp & 3;  // TMEM lane quadrant this warp may access
     const uint32_t stg = epi_warp ? smem_u32(smem + L::kOffEpi + (warp - kWarpEpi0) * L::kEpiStageBytes)
                                   : smem_u32(smem + L::kOffA + warp * L::kEpiStageBytes);
     const float gamma = p.gamma ? __ldg(p.gamma) : 1.0f;
+    int n = 0, tile = 0;
+    while (next_tile(p, pair, npairs, n, tile)) ++n;
+    bool ready = epi_warp || (n > 0 && wait(done_bar, 0));
+    if (ready && !epi_warp) tc_fence_after();
     int buf = 0;
     uint32_t buf_phase = 0;
     uint32_t seq = 0;
-    int tile;
-    for (int i = 0; next_tile(p, pair, npairs, i, tile); ++i) {
-      int after;
-      const bool last = !next_tile(p, pair, npairs, i + 1, after);
+    for (int i = 0; ready && i < n; ++i) {
+      next_tile(p, pair, npairs, i, tile);
+      const bool last = i == n - 1;
       if (epi_warp || last) {
         const TileInfo t = decode_tile<BN>(p, tile, rank);
         const OpParams& P = p.op[t.opi];
-        if (!wait(&tmem_full[buf], buf_phase)) break;
-        tc_fence_after();
+        if (epi_warp) {
+          if (!wait(&tmem_full[buf], buf_phase)) break;
+          tc_fence_after();
+        }
         const int pb = last ? warp >> 2 : 0, ps = last ? 4 : 1;
         if (t.opi == 0)
           epilogue_tile<kOp0, BN, G::kEpiSlots>(p, P, &map_out0, tmem_base, buf, stg, lane, q, t.a0, t.bp, gamma,
@@ -924,208 +932,129 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 }
 
 // ---------------------------------------------------------------- forward for few tokens
-// With up to 16 tokens the forward is bound by reading the packed codes once
-// (N K / 4 bytes), and the CTA-pair tiles (256 code rows x >= 128 tokens)
-// would leave most SMs idle. Here a cluster of S CTAs takes 128 code rows
-// (output features n) and splits K between its CTAs; each CTA loads its
-// codes with coalesced 8-byte loads (all of them in flight at once), expands
-// them to int8 in shared memory (the GEMM's 128-byte-swizzled K-major layout),
-// stages the tokens' INT8 rows (padded with zero rows to 16) and runs
-// tcgen05.mma kind::i8 with M = 128, N = 16 into a 16-column TMEM
-// accumulator. The S partial INT32 sums are exact and are added through
-// distributed shared memory: after a cluster barrier, CTA r reads every CTA's
-// partials of tokens r, r + S, ... and writes y = bf16_rn(fp32(acc) *
-// fp32(s_x[m] * gamma)) (the GEMM epilogue's formula) for its tokens.
-constexpr int kDecThreads = 128;
-constexpr int kDecRows = 128;     // code rows per cluster
-constexpr int kDecMaxM = 16;      // tokens (the MMA's N)
-constexpr int kDecMaxKb = 8;      // k-blocks of 128 per CTA
-constexpr int kDecMaxCluster = 8;
+// With a handful of tokens the forward is bound by reading the packed codes
+// once (N K / 4 bytes), not by arithmetic, and the tensor-core tiles would
+// leave most SMs idle. Used for M <= 8, where it measured faster than the
+// tile kernel (at the up-projection weight: 10.2 us at M = 1 and 16.4 us at
+// M = 8 against 19.5 us; beyond M = 8 the tile kernel wins). A CTA takes 32 output features (lane = feature n) and all M
+// tokens; its 8 warps split K into contiguous runs of 32-code groups. The tokens'
+// INT8 rows sit in shared memory (read with broadcast loads), the codes are
+// expanded to int8 with the same bit arithmetic as the GEMM rebuild, and
+// __dp4a keeps the sums exact in INT32. The warps' partial sums are added in
+// a fixed order, and y = bf16_rn(fp32(acc) * fp32(s_x[m] * gamma)) as in the
+// GEMM epilogue.
+constexpr int kDecodeWarps = 8;
+constexpr int kDecodeMaxM = 8;
 
-struct DecodeParams {
-  const int8_t* xq;
-  const float* sx;
-  const uint8_t* packed;
-  const float* gamma;
-  int M, N, K;
-  int nkb_total;  // ceil(K / 128)
-  int kb_per;     // k-blocks per CTA of a cluster (the last CTA may have fewer)
-  __nv_bfloat16* y;
-  int32_t* debug_acc;
-  int* err;
-};
-
-__host__ __device__ constexpr int dec_smem_bytes(int kb_per) {
-  return kb_per * (kDecRows * 128 + kDecMaxM * 128) + kDecRows * kDecMaxM * 4 + 64 + 1024;
-}
-
-__global__ void __launch_bounds__(kDecThreads) decode_forward_kernel(const __grid_constant__ DecodeParams p) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const int kb_per = p.kb_per;
-  uint8_t* sA = smem;                                  // [kb][128 rows][128 B]
-  uint8_t* sB = sA + kb_per * kDecRows * 128;          // [kb][16 rows][128 B]
-  int32_t* sP = reinterpret_cast<int32_t*>(sB + kb_per * kDecMaxM * 128);  // [128 rows][16]
-  uint64_t* bar = reinterpret_cast<uint64_t*>(sP + kDecRows * kDecMaxM);
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bar + 1);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bar + 2);
-
-  const int t = threadIdx.x, warp = t >> 5;
-  const uint32_t rank = cluster_ctarank();
-  const uint32_t S = gridDim.x;  // the cluster spans the grid's x dimension
-  const int n0 = blockIdx.y * kDecRows;
-  const int kb0 = static_cast<int>(rank) * kb_per;
-  const int nkb = max(0, min(kb_per, p.nkb_total - kb0));
-  const int K = p.K, M = p.M;
-  const int64_t kq = K / 4;  // packed bytes per row
-
-  if (warp == 0) {
-    tmem_alloc_1(tmem_holder, 32);
-    tmem_relinquish_1();
-  }
-  if (t == 0) {
-    mbar_init(bar, 1);
-    *abort_flag = 0;
-    fence_mbar_init();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_holder;
+template <int kMaxM>
+__global__ void __launch_bounds__(32 * kDecodeWarps) decode_forward_kernel(
+    const int8_t* __restrict__ xq, const float* __restrict__ sx, const uint8_t* __restrict__ packed,
+    const float* __restrict__ gamma_ptr, int M, int N, int K, __nv_bfloat16* __restrict__ y,
+    int32_t* __restrict__ debug_acc) {
+  extern __shared__ __align__(16) uint8_t s_q[];  // [kMaxM][K] int8, then the warps' partial sums
   pdl_wait_primary();
   pdl_launch_dependents();
-
-  // codes: 8-byte pieces (32 codes) of rows n0.., k-blocks kb0..; consecutive
-  // threads take consecutive pieces of a row, every load issued first
-  {
-    const int per_row = nkb * 4;
-    const int total = kDecRows * per_row;
-    constexpr int kBatch = 8;
-    for (int c0 = t; c0 < total; c0 += kBatch * kDecThreads) {
-      uint2 v[kBatch];
-#pragma unroll
-      for (int j = 0; j < kBatch; ++j) {
-        const int c = c0 + j * kDecThreads;
-        v[j] = make_uint2(0u, 0u);
-        if (c < total) {
-          const int row = c / per_row, q = c % per_row;
-          const int k = (kb0 + q / 4) * 128 + (q % 4) * 32;
-          if (n0 + row < p.N && k < K)
-            v[j] = __ldg(reinterpret_cast<const uint2*>(p.packed + static_cast<int64_t>(n0 + row) * kq + k / 4));
-        }
-      }
-#pragma unroll
-      for (int j = 0; j < kBatch; ++j) {
-        const int c = c0 + j * kDecThreads;
-        if (c >= total) break;
-        const int row = c / per_row, q = c % per_row;
-        const uint32_t base = smem_u32(sA) + (q / 4) * (kDecRows * 128) + row * 128;
-        const int c16 = (q % 4) * 2;  // 16-byte chunk of the row's 128 codes
-        st_shared_v4(base + ((c16 ^ (row & 7)) << 4), codes16_to_s8(v[j].x));
-        st_shared_v4(base + (((c16 + 1) ^ (row & 7)) << 4), codes16_to_s8(v[j].y));
-      }
-    }
-  }
-  // tokens: 16-byte pieces of xq rows (rows M..15 and k past K are zero)
-  for (int c = t; c < nkb * kDecMaxM * 8; c += kDecThreads) {
-    const int kb = c / (kDecMaxM * 8), rem = c % (kDecMaxM * 8), m = rem / 8, c16 = rem % 8;
-    const int k = (kb0 + kb) * 128 + c16 * 16;
-    uint4 v = make_uint4(0u, 0u, 0u, 0u);
-    if (m < M && k < K) v = __ldg(reinterpret_cast<const uint4*>(p.xq + static_cast<int64_t>(m) * K + k));
-    st_shared_v4(smem_u32(sB) + kb * (kDecMaxM * 128) + m * 128 + ((c16 ^ (m & 7)) << 4), v);
-  }
-  fence_proxy_async_smem();
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  // tokens' codes into shared memory (rows of K bytes, K % 32 == 0); rows
+  // M .. kMaxM-1 are zero, so every token slot is summed without a branch
+  const int qvec = M * K / 16, qall = kMaxM * K / 16;
+  for (int i = threadIdx.x; i < qall; i += blockDim.x)
+    reinterpret_cast<uint4*>(s_q)[i] =
+        i < qvec ? __ldg(reinterpret_cast<const uint4*>(xq) + i) : make_uint4(0u, 0u, 0u, 0u);
   __syncthreads();
 
-  if (t == 0 && nkb > 0) {
-    tc_fence_after();
-    constexpr uint32_t kIdesc = make_idesc(2 /*s32*/, 1 /*s8*/, 0, 0, kDecRows, kDecMaxM);
-    for (int kb = 0; kb < nkb; ++kb) {
-      const uint64_t ad = smem_desc_sw128(smem_u32(sA) + kb * (kDecRows * 128), 16, 1024);
-      const uint64_t bd = smem_desc_sw128(smem_u32(sB) + kb * (kDecMaxM * 128), 16, 1024);
+  const int n = blockIdx.x * 32 + lane;
+  const bool row_ok = n < N;
+  const uint2* row = reinterpret_cast<const uint2*>(packed + static_cast<int64_t>(row_ok ? n : 0) * (K / 4));
+  int32_t acc[kMaxM];
 #pragma unroll
-      for (int kk = 0; kk < 4; ++kk) mma_i8_1(tmem, ad + 2 * kk, bd + 2 * kk, kIdesc, (kb | kk) != 0);
+  for (int m = 0; m < kMaxM; ++m) acc[m] = 0;
+  // each warp takes a contiguous run of 32-code groups (8 bytes each) and
+  // each lane loads its row's groups kBatch at a time, the next batch while
+  // the current one is summed
+  constexpr int kBatch = 8;
+  const int groups = K / 32;
+  const int gpw = (groups + kDecodeWarps - 1) / kDecodeWarps;
+  const int g_begin = warp * gpw;
+  const int g_end = min(g_begin + gpw, groups);
+  uint2 cur[kBatch];
+#pragma unroll
+  for (int b = 0; b < kBatch; ++b)
+    cur[b] = (row_ok && g_begin + b < g_end) ? __ldg(row + g_begin + b) : make_uint2(0u, 0u);
+  for (int g = g_begin; g < g_end; g += kBatch) {
+    uint2 nxt[kBatch];
+#pragma unroll
+    for (int b = 0; b < kBatch; ++b)
+      nxt[b] = (row_ok && g + kBatch + b < g_end) ? __ldg(row + g + kBatch + b) : make_uint2(0u, 0u);
+#pragma unroll
+    for (int b = 0; b < kBatch; ++b) {
+      if (g + b >= g_end) break;
+      const uint4 c0 = codes16_to_s8(cur[b].x), c1 = codes16_to_s8(cur[b].y);
+      const int32_t c[8] = {static_cast<int32_t>(c0.x), static_cast<int32_t>(c0.y), static_cast<int32_t>(c0.z),
+                            static_cast<int32_t>(c0.w), static_cast<int32_t>(c1.x), static_cast<int32_t>(c1.y),
+                            static_cast<int32_t>(c1.z), static_cast<int32_t>(c1.w)};
+      const uint32_t qbase = smem_u32(s_q) + (g + b) * 32;
+#pragma unroll
+      for (int m = 0; m < kMaxM; ++m) {
+        const uint4 qa = ld_shared_v4(qbase + m * K);
+        const uint4 qb = ld_shared_v4(qbase + m * K + 16);
+        // two independent chains, added at the end (integer sums are exact)
+        int32_t a = __dp4a(c[0], static_cast<int32_t>(qa.x), 0);
+        int32_t b = __dp4a(c[4], static_cast<int32_t>(qb.x), 0);
+        a = __dp4a(c[1], static_cast<int32_t>(qa.y), a);
+        b = __dp4a(c[5], static_cast<int32_t>(qb.y), b);
+        a = __dp4a(c[2], static_cast<int32_t>(qa.z), a);
+        b = __dp4a(c[6], static_cast<int32_t>(qb.z), b);
+        a = __dp4a(c[3], static_cast<int32_t>(qa.w), a);
+        b = __dp4a(c[7], static_cast<int32_t>(qb.w), b);
+        acc[m] += a + b;
+      }
     }
-    mma_commit_1(bar);
-  }
-  // this CTA's partial sums of its 128 rows: TMEM lane quadrant = warp
-  uint32_t r[16];
-  if (nkb > 0 && mbar_wait(bar, 0, abort_flag, p.err)) {
-    tc_fence_after();
-    tmem_ld_32x32b_x16(tmem + (static_cast<uint32_t>(warp * 32) << 16), r);
-    tmem_ld_wait();
-  } else {
 #pragma unroll
-    for (int j = 0; j < 16; ++j) r[j] = 0u;
+    for (int b = 0; b < kBatch; ++b) cur[b] = nxt[b];
   }
-  const uint32_t prow = smem_u32(sP) + t * (kDecMaxM * 4);
+  // fixed-order sum over the warps: warps 1.. park their sums, warp 0 adds
+  int32_t* red = reinterpret_cast<int32_t*>(s_q + kMaxM * K);  // [warp-1][m][32]
+  if (warp > 0) {
 #pragma unroll
-  for (int j = 0; j < 16; j += 4) st_shared_v4(prow + j * 4, make_uint4(r[j], r[j + 1], r[j + 2], r[j + 3]));
-  tc_fence_before();
-  cluster_sync_all();  // every CTA's partials are written
-
-  // tokens m = rank, rank + S, ...: sum the S partials of row t in rank order
-  const int n = n0 + t;
-  const float gamma = __ldg(p.gamma);
-  for (int m = static_cast<int>(rank); m < M; m += static_cast<int>(S)) {
-    int32_t acc = 0;
-    for (uint32_t q = 0; q < S; ++q) acc += static_cast<int32_t>(ld_cluster_u32(map_to_rank(prow + m * 4, q)));
-    if (n < p.N) {
-      const int64_t off = static_cast<int64_t>(m) * p.N + n;
-      p.y[off] = __float2bfloat16_rn(__fmul_rn(static_cast<float>(acc), __fmul_rn(__ldg(p.sx + m), gamma)));
-      if (p.debug_acc) p.debug_acc[off] = acc;
+    for (int m = 0; m < kMaxM; ++m)
+      if (m < M) red[((warp - 1) * kMaxM + m) * 32 + lane] = acc[m];
+  }
+  __syncthreads();
+  if (warp != 0) return;
+  const float gamma = __ldg(gamma_ptr);
+#pragma unroll
+  for (int m = 0; m < kMaxM; ++m) {
+    if (m < M) {
+      int32_t a = acc[m];
+      for (int w = 1; w < kDecodeWarps; ++w) a += red[((w - 1) * kMaxM + m) * 32 + lane];
+      if (row_ok) {
+        const int64_t off = static_cast<int64_t>(m) * N + n;
+        y[off] = __float2bfloat16_rn(__fmul_rn(static_cast<float>(a), __fmul_rn(__ldg(sx + m), gamma)));
+        if (debug_acc) debug_acc[off] = a;
+      }
     }
-  }
-  cluster_sync_all();  // no CTA leaves while a peer may still read its partials
-  if (warp == 0) {
-    tc_fence_after();
-    tmem_dealloc_1(tmem, 32);
   }
 }
 
-// Cluster geometry: about two CTAs per SM in all, at most 8 k-blocks of 128
-// per CTA and at most 8 CTAs per cluster; returns false when K is too long.
-bool decode_geometry(int N, int K, int& S, int& kb_per) {
-  const int nkb = (K + 127) / 128;
-  const int nblocks = (N + kDecRows - 1) / kDecRows;
-  const int target = std::max(1, (2 * device_sm_count() + nblocks / 2) / nblocks);
-  kb_per = std::min(kDecMaxKb, std::max(1, (nkb + target - 1) / target));
-  S = (nkb + kb_per - 1) / kb_per;
-  if (S > kDecMaxCluster) {
-    kb_per = (nkb + kDecMaxCluster - 1) / kDecMaxCluster;
-    S = (nkb + kb_per - 1) / kb_per;
-  }
-  return kb_per <= kDecMaxKb && S <= kDecMaxCluster;
-}
-
+template <int kMaxM>
 cudaError_t launch_decode(const int8_t* xq, const float* sx, const uint8_t* packed, const float* gamma, int M, int N,
-                          int K, void* y, int32_t* debug_acc, int* err, int S, int kb_per, cudaStream_t s) {
+                          int K, void* y, int32_t* debug_acc, cudaStream_t s) {
+  const size_t smem = static_cast<size_t>(kMaxM) * K + static_cast<size_t>(kDecodeWarps - 1) * kMaxM * 32 * 4;
   static int configured[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
+  const int max_smem = kSmemLimit;
   if (dev >= 0 && dev < 64 && !configured[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(decode_forward_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         dec_smem_bytes(kDecMaxKb));
+    cudaError_t e =
+        cudaFuncSetAttribute(decode_forward_kernel<kMaxM>, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem);
     if (e != cudaSuccess) return e;
     configured[dev] = 1;
   }
-  DecodeParams p{xq, sx, packed, gamma, M, N, K, (K + 127) / 128, kb_per,
-                 static_cast<__nv_bfloat16*>(y), debug_acc, err};
-  cudaLaunchConfig_t cfg{};
-  cfg.gridDim = dim3(static_cast<unsigned>(S), static_cast<unsigned>((N + kDecRows - 1) / kDecRows));
-  cfg.blockDim = dim3(kDecThreads);
-  cfg.dynamicSmemBytes = dec_smem_bytes(kb_per);
-  cfg.stream = s;
-  cudaLaunchAttribute attr[2];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = static_cast<unsigned>(S);
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[1].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 2;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, decode_forward_kernel, p);
+  const unsigned grid = static_cast<unsigned>((N + 31) / 32);
+  cudaError_t e = launch_pdl(decode_forward_kernel<kMaxM>, dim3(grid), dim3(32 * kDecodeWarps), smem, s, xq, sx,
+                             packed, gamma, M, N, K, static_cast<__nv_bfloat16*>(y), debug_acc);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
@@ -1343,13 +1272,20 @@ cudaError_t launch_forward(const int8_t* xq, const float* sx, const uint8_t* w_p
                            int64_t M, int64_t N, int64_t K, void* y, int32_t* debug_acc, int* err,
                            cudaStream_t s) {
   if (M == 0 || N == 0) return cudaSuccess;
-  // few tokens: the packed codes' bandwidth, not the tile GEMM's tensor-core
-  // rate, bounds the forward
-  if (M <= kDecMaxM) {
-    int S = 0, kb_per = 0;
-    if (decode_geometry(static_cast<int>(N), static_cast<int>(K), S, kb_per))
-      return launch_decode(xq, sx, w_packed, gamma, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), y,
-                           debug_acc, err, S, kb_per, s);
+  // few tokens: the packed codes' bandwidth, not the tensor cores, bounds the
+  // forward (the tokens' codes must fit in shared memory)
+  if (M <= kDecodeMaxM) {
+    int slots = 1;
+    while (slots < M) slots *= 2;
+    if (static_cast<size_t>(slots) * K + static_cast<size_t>(kDecodeWarps - 1) * slots * 32 * 4 <= kSmemLimit) {
+      const int m = static_cast<int>(M), nn = static_cast<int>(N), kk = static_cast<int>(K);
+      switch (slots) {
+        case 1: return launch_decode<1>(xq, sx, w_packed, gamma, m, nn, kk, y, debug_acc, s);
+        case 2: return launch_decode<2>(xq, sx, w_packed, gamma, m, nn, kk, y, debug_acc, s);
+        case 4: return launch_decode<4>(xq, sx, w_packed, gamma, m, nn, kk, y, debug_acc, s);
+        default: return launch_decode<8>(xq, sx, w_packed, gamma, m, nn, kk, y, debug_acc, s);
+      }
+    }
   }
   static const int kCands[3] = {256, 192, 128};
   const int npairs = resident_pairs<Family::Fwd, 256>();

@@ -2,18 +2,17 @@
 // 2-bit packing, and per-token absmax INT8 activation quantisation.
 //
 // S1 needs the mean |W| of the whole tensor before any code can be written,
-// and S2 is independent of it. One persistent launch does both with W read
-// from HBM once: each CTA (at most one per SM, all resident together) copies
-// its contiguous slice of W into shared memory with bulk asynchronous copies
-// (TMA, issued all at once at entry), sums |W| of the slice in fp64 as the
-// copies land, publishes the partial sum and meets the other CTAs at a
-// grid-wide barrier (a counter in the workspace, bounded wait); then every
-// CTA forms gamma from all partial sums in one fixed order and writes the
-// codes of its slice from shared memory. The part of a slice that does not
-// fit in shared memory is summed from registers and read again (from L2) for
-// its codes. Other warps of the same CTAs quantise the tokens (S2) while the
-// slice copies are in flight. A one-thread launch before it clears the
-// workspace's counters, so the caller's workspace needs no initialisation.
+// and S2 is independent of it. bl_quantize is two launches:
+//
+//   sum launch   every CTA sums |W| of its contiguous slice of W in fp64 and
+//                stores the partial sum in its own workspace slot (no atomics,
+//                no waits); the same warps quantise token rows (S2). This is
+//                the pass that streams W and x from HBM.
+//   code launch  (a programmatic dependent: its CTAs wait for the sum launch
+//                to complete) every CTA reduces the partial sums in one fixed
+//                order, forms gamma and writes the codes of its share of W,
+//                which it reads again (the sum launch has just left W in L2;
+//                its own loads are issued before gamma is known).
 //
 // gamma = max(fp32(fp64(fp64(S) / numel)), 1e-5) with S = sum |W| (exactly
 // rounded to fp64, "1BitTraining.md" weight_quant / "bitlinear.py"
@@ -21,9 +20,10 @@
 // tree sum carries a bounded rounding error, so gamma is formed at both ends
 // of an enclosure of S; as the chain of roundings is monotone, when the two
 // agree that value is the exact gamma (all but about one tensor in 10^5).
-// Otherwise the CTAs compute S exactly -- integer sums of the significands
-// per exponent field, combined as one wide integer and rounded once -- so
-// gamma never depends on the reduction order or on the GPU's SM count.
+// Otherwise the code launch computes S exactly -- integer sums of the
+// significands per exponent field, combined as one wide integer and rounded
+// once -- behind a grid-wide barrier with a bounded wait, so gamma never
+// depends on the reduction order or on the GPU's SM count.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -41,23 +41,21 @@ __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w 
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
 // ---------------------------------------------------------------- S1 geometry
-constexpr int kQThreads = 512;                 // 16 warps per CTA
-constexpr int kQWarps = kQThreads / 32;
-constexpr int kChunkBytes = 16384;             // one bulk copy of the slice
-constexpr int kMaxOnchipBytes = 220 * 1024;    // slice bytes held in shared memory
-constexpr int kMaxChunks = kMaxOnchipBytes / kChunkBytes + 1;
+constexpr int kSumThreads = 256;  // sum launch: 8 warps per CTA
+constexpr int kSumWarps = kSumThreads / 32;
+constexpr int kSumUnroll = 8;     // 16-byte loads in flight per thread
+constexpr int kCodeThreads = 512; // code launch: 16 warps per CTA
+constexpr int kCodeWarps = kCodeThreads / 32;
 
 // Workspace (each part on its own 128-byte lines): at 0 the arrivals at the
-// partial-sum and at the exact-sum barrier (u32 each); at 128 the gamma flag
-// (1: gamma published, 2: the exact sum is needed) and gamma's bits; at 256
-// the next token row to claim; at 512 one fp64 partial sum per CTA; then 256
-// uint64 exact-sum bins (one per exponent field).
+// exact-sum barrier (u32); at 128 256 uint64 exact-sum bins (one per exponent
+// field); at 2304 one fp64 partial sum per CTA of the sum launch. The sum
+// launch clears the first two parts and fills the third on every call, so the
+// caller's workspace needs no initialisation.
 constexpr size_t kWsArrive = 0;
-constexpr size_t kWsFlag = 128;
-constexpr size_t kWsRows = 256;
-constexpr size_t kWsPartials = 512;
-constexpr size_t kWsBins = kWsPartials + 8 * static_cast<size_t>(kMaxQuantCtas);
-constexpr size_t kWsBytes = kWsBins + 8 * 256;
+constexpr size_t kWsBins = 128;
+constexpr size_t kWsParts = kWsBins + 8 * 256 + 128;
+constexpr size_t kWsBytes = kWsParts + 8 * static_cast<size_t>(kMaxQuantCtas);
 
 // ---------------------------------------------------------------- |W| in fp64
 // |w| widened to fp64 exactly from its bit pattern with the sign cleared.
@@ -197,20 +195,25 @@ __device__ __forceinline__ float gamma_of_sum(double S, double numel) {
 // field 00 = 0, 01 = +1, 11 = -1). For a 15-bit magnitude b and thr > 0,
 // |w| > thr <=> b > bits(thr) >> 16, so both halves of a word are compared by
 // one subtraction: 0x8000 + tb - b keeps bit 15 clear exactly when b > tb (no
-// borrow crosses the halves, b <= 0x7FFF). The low elements' fields collect at
-// bits 4j, 4j + 1 and the high elements' at 16 + 4j, 17 + 4j of one word, then
-// one fold moves the high ones to 4j + 2, 4j + 3 (about four operations per
-// element).
+// borrow crosses the halves, b <= 0x7FFF). One byte permutation per word pair
+// gathers the four compare bits (and, of the weights, the four sign bits) as
+// the top bits of four bytes; a high multiply by 2^25 + 2^19 + 2^13 + 2^7
+// (2^26 + ... for the signs) moves bits 7, 15, 23, 31 to bits 0, 2, 4, 6 (1,
+// 3, 5, 7) of its high word -- every partial product lands on its own bit, so
+// nothing carries -- and one logic operation merges the two. The integer
+// logic unit, which bounds this pass, does about 1.75 operations per element;
+// the multiplies run on the multiply-add pipe.
 __device__ __forceinline__ uint32_t codes8_bf16(const uint4& v, uint32_t bias) {
-  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-  uint32_t acc = 0;
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const uint32_t nz = ~(bias - (w[j] & 0x7FFF7FFFu)) & 0x80008000u;  // bits 15, 31: nonzero code
-    const uint32_t nn = nz & w[j];                                     // and negative
-    acc |= (nz >> (15 - 4 * j)) | (nn >> (14 - 4 * j));
-  }
-  return (acc & 0x3333u) | ((acc >> 14) & 0xCCCCu);
+  constexpr uint32_t kSpread = (1u << 25) | (1u << 19) | (1u << 13) | (1u << 7);
+  const uint32_t d0 = bias - (v.x & 0x7FFF7FFFu), d1 = bias - (v.y & 0x7FFF7FFFu);
+  const uint32_t d2 = bias - (v.z & 0x7FFF7FFFu), d3 = bias - (v.w & 0x7FFF7FFFu);
+  const uint32_t nzl = ~__byte_perm(d0, d1, 0x7531) & 0x80808080u;  // elements 0..3 nonzero
+  const uint32_t nzh = ~__byte_perm(d2, d3, 0x7531) & 0x80808080u;  // elements 4..7
+  const uint32_t ngl = nzl & __byte_perm(v.x, v.y, 0x7531);          // and negative
+  const uint32_t ngh = nzh & __byte_perm(v.z, v.w, 0x7531);
+  const uint32_t lo = (__umulhi(nzl, kSpread) & 0x55u) | (__umulhi(ngl, 2 * kSpread) & 0xAAu);
+  const uint32_t hi = (__umulhi(nzh, kSpread) & 0x55u) | (__umulhi(ngh, 2 * kSpread) & 0xAAu);
+  return hi * 256u + lo;
 }
 
 // 4 fp32 of one vector -> 8 bits of codes.
@@ -269,13 +272,6 @@ __device__ __forceinline__ bool grid_arrive_wait(uint32_t* ctr, uint32_t expecte
       return false;
     }
   }
-}
-
-__device__ __forceinline__ void bulk_copy_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
-  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-                   smem_u32(dst)),
-               "l"(src), "r"(bytes), "r"(smem_u32(bar))
-               : "memory");
 }
 
 // ---------------------------------------------------------------- S2
@@ -427,86 +423,99 @@ __global__ void __launch_bounds__(32 * kActRowsPerBlock) act_quant_long_kernel(c
 }
 
 // ---------------------------------------------------------------- S1 (+ S2): the launches
-// Launch 1: clears the workspace's counters, flag and exact-sum bins. It
-// waits for the kernel before it in the stream (whose work may still use
-// them), and only then lets the quantisation launch start; so the
-// quantisation may read W and x and write its outputs from its first
-// instruction, and waits for this launch itself only before its first use of
-// the workspace.
-__global__ void __launch_bounds__(256) quant_reset_kernel(uint8_t* __restrict__ ws) {
-  pdl_wait_primary();
+struct SumArgs {
+  const uint4* W;  // [N, K] as 16-byte vectors
+  int64_t nvec;    // vectors of W
+  int64_t per;     // vectors per CTA slice (the last slices may be shorter or empty)
+  double* parts;   // one partial sum per CTA
+  uint8_t* ws;     // exact-sum counter and bins, cleared here for the code launch
+  const uint4* x;  // S2: x [M, K] as 16-byte vectors (M = 0: no tokens)
+  int64_t M;
+  int nv;          // K / 8
+  int8_t* xq;
+  float* sx;
+};
+
+// Sum launch, kSumThreads threads per CTA, several CTAs per SM. Nothing in it
+// waits on another CTA. CTA b first quantises token rows [b M / G, (b + 1) M /
+// G) (warp w: rows w, w + 8, ... of them), then sums |W| of its slice, so
+// that W is the most recent data in L2 when the code launch reads it again.
+// Thread t adds vectors t, t + 256, ... of the slice, the j-th of them into
+// accumulator j mod 4 (in order, elements of a vector in order); the CTA's
+// partial sum is the four accumulators added pairwise, then a butterfly over
+// the warp's lanes (the same value in every lane), then the warps' sums in
+// warp order. Every step is a fixed sequence of fp64 additions, so the
+// partial sums do not depend on scheduling.
+template <bool kF32, int VPL>
+__global__ void __launch_bounds__(kSumThreads, 4) quant_sum_kernel(const __grid_constant__ SumArgs a) {
+  __shared__ double s_red[kSumWarps];
+  pdl_wait_primary();  // W and x may be written by earlier work of the stream
   pdl_launch_dependents();
-  if (threadIdx.x == 0) {
-    reinterpret_cast<uint32_t*>(ws + kWsArrive)[0] = 0u;
-    reinterpret_cast<uint32_t*>(ws + kWsArrive)[1] = 0u;
-    reinterpret_cast<uint32_t*>(ws + kWsFlag)[0] = 0u;
-    reinterpret_cast<uint32_t*>(ws + kWsRows)[0] = 0u;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, t = threadIdx.x;
+  const int64_t b = blockIdx.x, G = gridDim.x;
+  if (b == 0) {
+    unsigned long long* bins = reinterpret_cast<unsigned long long*>(a.ws + kWsBins);
+    for (int e = t; e < 256; e += kSumThreads) bins[e] = 0ull;
+    if (t == 0) *reinterpret_cast<uint32_t*>(a.ws + kWsArrive) = 0u;
   }
-  reinterpret_cast<unsigned long long*>(ws + kWsBins)[threadIdx.x] = 0ull;
+  if (a.M > 0) {
+    const int64_t r0 = b * a.M / G, r1 = (b + 1) * a.M / G;
+    if constexpr (VPL > 0) act_rows<VPL, false>(a.x, r1, a.nv, a.xq, a.sx, r0 + warp, kSumWarps);
+    else act_rows_two_pass(a.x, r1, a.nv, a.xq, a.sx, r0 + warp, kSumWarps);
+  }
+  const int64_t v0 = b * a.per;
+  const int64_t v1 = v0 + a.per < a.nvec ? v0 + a.per : a.nvec;
+  double acc[4] = {0.0, 0.0, 0.0, 0.0};
+  int64_t i = v0 + t;
+  for (; i + (kSumUnroll - 1) * kSumThreads < v1; i += kSumUnroll * kSumThreads) {
+    uint4 v[kSumUnroll];
+#pragma unroll
+    for (int u = 0; u < kSumUnroll; ++u) v[u] = __ldg(a.W + i + u * kSumThreads);
+#pragma unroll
+    for (int u = 0; u < kSumUnroll; ++u) acc[u & 3] = add_abs<kF32>(acc[u & 3], v[u]);
+  }
+  if (i < v1) {  // fewer than kSumUnroll vectors left for this thread
+    uint4 v[kSumUnroll];
+#pragma unroll
+    for (int u = 0; u < kSumUnroll; ++u)
+      v[u] = i + u * kSumThreads < v1 ? __ldg(a.W + i + u * kSumThreads) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+    for (int u = 0; u < kSumUnroll; ++u)
+      if (i + u * kSumThreads < v1) acc[u & 3] = add_abs<kF32>(acc[u & 3], v[u]);
+  }
+  double ts = __dadd_rn(__dadd_rn(acc[0], acc[1]), __dadd_rn(acc[2], acc[3]));
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) ts = __dadd_rn(ts, __shfl_xor_sync(0xffffffffu, ts, off));
+  if (lane == 0) s_red[warp] = ts;
+  __syncthreads();
+  if (t == 0) {
+    double p = 0.0;
+#pragma unroll
+    for (int w = 0; w < kSumWarps; ++w) p = __dadd_rn(p, s_red[w]);
+    a.parts[b] = p;
+  }
 }
 
-struct QuantArgs {
-  const uint4* W;       // [N, K] as 16-byte vectors
-  int64_t ngroups;      // N K / 16: a group's 16 codes are one 32-bit word
-  int64_t per;          // groups per CTA slice (the last slices may be shorter or empty)
-  int onchip_cap;       // groups of a slice held in shared memory
+struct CodeArgs {
+  const uint4* W;
+  int64_t nvec;
+  const double* parts;  // the sum launch's partial sums
+  int nparts;
   double numel;
   double enc_lo, enc_hi;  // S lies in [fp64 sum * enc_lo, fp64 sum * enc_hi]
   uint32_t* packed;
   float* gamma_out;
   uint8_t* ws;
   int* err;
-  const uint4* x;       // S2: x [M, K] as 16-byte vectors (M = 0: no tokens)
-  int64_t M;
-  int nv;               // K / 8
-  int8_t* xq;
-  float* sx;
 };
 
-__device__ __forceinline__ void st_release_u32(uint32_t* p, uint32_t v) {
-  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-
-// Lane 0 claims `n` consecutive items of a counter, the warp gets the first.
-__device__ __forceinline__ uint32_t warp_claim(uint32_t* ctr, uint32_t n) {
-  uint32_t m = 0;
-  if ((threadIdx.x & 31) == 0) m = atomicAdd(ctr, n);
-  return __shfl_sync(0xffffffffu, m, 0);
-}
-
-// Token rows m0, m0 + 1 (those below M): both rows' loads are issued before
-// either is quantised. Rows longer than 2560 elements (VPL = 0) are read twice
-// (absmax, then quantisation from L1/L2).
-template <int VPL>
-__device__ __forceinline__ void token_pair(const QuantArgs& a, int64_t m0) {
-  const int lane = threadIdx.x & 31;
-  if constexpr (VPL > 0) {
-    uint4 v0[VPL], v1[VPL];
-    load_row<VPL>(a.x + m0 * a.nv, a.nv, lane, v0);
-    const bool two = m0 + 1 < a.M;
-    if (two) load_row<VPL>(a.x + (m0 + 1) * a.nv, a.nv, lane, v1);
-    quant_row<VPL>(v0, a.nv, lane, m0, a.xq, a.sx);
-    if (two) quant_row<VPL>(v1, a.nv, lane, m0 + 1, a.xq, a.sx);
-  } else {
-    act_rows_two_pass(a.x, m0 + 2 < a.M ? m0 + 2 : a.M, a.nv, a.xq, a.sx, m0, 1);
-  }
-}
-
-// Codes of 128 consecutive 16-byte vectors of W from shared memory (kShared)
-// or global memory: lane l takes vectors l, l + 32, l + 64, l + 96 (all loads
-// first, conflict-free shared loads); a group's V lanes combine their bits and
+// Codes of 128 consecutive 16-byte vectors of W from base (lane l holds
+// vectors l, l + 32, l + 64, l + 96): a group's V lanes combine their bits and
 // its first lane stores the group's word.
-template <bool kF32, bool kShared>
-__device__ __forceinline__ void code_round(const uint4* src, int64_t base, int64_t nvec, uint32_t* out, uint32_t key,
-                                           int lane) {
+template <bool kF32>
+__device__ __forceinline__ void store_codes(const uint4 (&v)[4], int64_t base, int64_t nvec, uint32_t* out,
+                                            uint32_t key, int lane) {
   constexpr int V = kF32 ? 4 : 2;
-  uint4 v[4];
-#pragma unroll
-  for (int u = 0; u < 4; ++u) {
-    const int64_t i = base + lane + 32 * u;
-    v[u] = make_uint4(0u, 0u, 0u, 0u);
-    if (i < nvec) v[u] = kShared ? src[i] : __ldg(src + i);
-  }
 #pragma unroll
   for (int u = 0; u < 4; ++u) {
     const int64_t i = base + lane + 32 * u;
@@ -515,359 +524,199 @@ __device__ __forceinline__ void code_round(const uint4* src, int64_t base, int64
   }
 }
 
-// Launch 2, 512 threads. Every warp first sums |W| of the CTA's slice as its
-// bulk copies land (W, which gates every code, is read before any token);
-// thread 0 then publishes the CTA's partial sum and arrives. Warp 0 becomes the
-// control warp: the last CTA to arrive forms gamma from all partial sums (in
-// one fixed order) and publishes it; the others wait for it. Meanwhile the
-// other warps quantise token rows claimed from a counter shared by the grid;
-// once gamma is known every warp takes rounds of 128 code vectors from a
-// counter of the CTA, and then token rows again until none is left. If the
+// Round q of W: 128 consecutive 16-byte vectors, lane l holding vectors
+// 128 q + l + 32 u (u = 0..3); vectors past W (or q past the last round) are
+// zero.
+__device__ __forceinline__ void load_round(const uint4* W, int64_t q, int64_t nrounds, int64_t nvec, int lane,
+                                           uint4 (&v)[4]) {
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int64_t i = 128 * q + lane + 32 * u;
+    v[u] = (q < nrounds && i < nvec) ? __ldg(W + i) : make_uint4(0u, 0u, 0u, 0u);
+  }
+}
+
+// The compare key of the code rule for gamma: the fp32 threshold's bit
+// pattern, or for bf16 the two-halves subtraction bias of codes8_bf16.
+template <bool kF32>
+__device__ __forceinline__ uint32_t code_key(float gamma) {
+  const float thr = __double2float_rd(__dmul_rn(static_cast<double>(gamma), 0.5 + 0x1p-25));
+  if constexpr (kF32) return __float_as_uint(thr);
+  const uint32_t tb = __float_as_uint(thr) >> 16;
+  return (tb | (tb << 16)) + 0x80008000u;
+}
+
+// Code launch, kCodeThreads threads per CTA, all CTAs resident together (the
+// exact-sum path meets at a grid-wide barrier). Warp g of the grid codes
+// rounds g, g + (warps of the grid), ...; its first round is loaded before
+// gamma is known, every later one while the previous is coded. Warp 0 of
+// every CTA adds the partial sums (lane l: partial sums l, l + 32, ... in
+// order, then a butterfly), so every CTA forms the same gamma. If the
 // enclosure of S straddles a rounding boundary of gamma (rare), every warp
-// first bins its share of the slice for the exact sum.
-template <bool kF32, int VPL>
-__global__ void __launch_bounds__(kQThreads, 1) quant_fused_kernel(const __grid_constant__ QuantArgs a) {
-  constexpr int V = kF32 ? 4 : 2;  // 16-byte vectors per group
-  constexpr int kGroupBytes = 16 * V;
-  constexpr int kChunkGroups = kChunkBytes / kGroupBytes;
-  constexpr int kTailRegs = 2;
-  extern __shared__ __align__(128) uint4 s_w[];
-  __shared__ __align__(8) uint64_t s_bar[kMaxChunks];
+// bins the vectors of its rounds for the exact sum, the CTAs add their bins
+// to the grid's and meet at the barrier, and every CTA forms the exact gamma.
+template <bool kF32>
+__global__ void __launch_bounds__(kCodeThreads) quant_code_kernel(const __grid_constant__ CodeArgs a) {
   __shared__ unsigned long long s_bins[256];
-  __shared__ double s_red[kQWarps];
+  __shared__ double s_parts[kMaxQuantCtas];
   __shared__ float s_gamma;
-  __shared__ uint32_t s_key;
-  __shared__ int s_state;   // 0: gamma not known, 1: known, 2: bin for the exact sum, -1: abort
-  __shared__ int s_round;   // next code round of this CTA
-  __shared__ int s_binned;  // warps done binning
-  __shared__ int s_abort;   // a wait of this CTA gave up
-
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, t = threadIdx.x;
-  const int64_t b = blockIdx.x;
-  const uint32_t G = gridDim.x;
-  const int64_t g0 = b * a.per;
-  const int64_t rest = a.ngroups - g0;
-  const int64_t len = rest <= 0 ? 0 : (rest < a.per ? rest : a.per);
-  const int on = static_cast<int>(len < a.onchip_cap ? len : a.onchip_cap);
-  const int nch = (on + kChunkGroups - 1) / kChunkGroups;
-  const int64_t onv = static_cast<int64_t>(on) * V;
-  const int64_t tail_v0 = (g0 + on) * V, tail_v1 = (g0 + len) * V;
-  uint32_t* arrive = reinterpret_cast<uint32_t*>(a.ws + kWsArrive);  // [0] partial sums, [1] exact sum
-  uint32_t* flag = reinterpret_cast<uint32_t*>(a.ws + kWsFlag);      // [0] 1 gamma / 2 exact, [1] gamma bits
-  uint32_t* rows = reinterpret_cast<uint32_t*>(a.ws + kWsRows);
-  double* partials = reinterpret_cast<double*>(a.ws + kWsPartials);
-  unsigned long long* gbins = reinterpret_cast<unsigned long long*>(a.ws + kWsBins);
-
-  if (t == 0) {
-    s_abort = 0;
-    s_state = 0;
-    s_round = 0;
-    s_binned = 0;
-    for (int c = 0; c < nch; ++c) mbar_init(&s_bar[c], 1);
-    fence_mbar_init();
-    fence_proxy_async_smem();
-    // the whole on-chip slice in flight at once
-    for (int c = 0; c < nch; ++c) {
-      const int cg0 = c * kChunkGroups;
-      const int cgn = min(kChunkGroups, on - cg0);
-      mbar_arrive_expect_tx(&s_bar[c], static_cast<uint32_t>(cgn * kGroupBytes));
-      bulk_copy_g2s(s_w + static_cast<int64_t>(cg0) * V, a.W + (g0 + cg0) * V, static_cast<uint32_t>(cgn * kGroupBytes),
-                    &s_bar[c]);
-    }
-  }
-  __syncthreads();
-
-  // -------------------------------------------------- |W| of the slice, all warps
-  // thread t takes vectors t, t + 512, ... of each chunk, then of the tail
-  uint4 tr[kTailRegs];
-#pragma unroll
-  for (int u = 0; u < kTailRegs; ++u) {
-    const int64_t i = tail_v0 + t + static_cast<int64_t>(u) * kQThreads;
-    tr[u] = i < tail_v1 ? __ldg(a.W + i) : make_uint4(0u, 0u, 0u, 0u);
-  }
-  double acc[4] = {0.0, 0.0, 0.0, 0.0};
-  for (int c = 0; c < nch; ++c) {
-    if (!mbar_wait(&s_bar[c], 0, &s_abort, a.err)) {
-      s_abort = 1;
-      break;
-    }
-    const int v1 = min((c + 1) * kChunkGroups, on) * V;
-    int i = c * kChunkGroups * V + t;
-    for (; i + 3 * kQThreads < v1; i += 4 * kQThreads) {
-      uint4 v[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) v[u] = s_w[i + u * kQThreads];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) acc[u] = add_abs<kF32>(acc[u], v[u]);
-    }
-    if (i < v1) acc[0] = add_abs<kF32>(acc[0], s_w[i]);
-    if (i + kQThreads < v1) acc[1] = add_abs<kF32>(acc[1], s_w[i + kQThreads]);
-    if (i + 2 * kQThreads < v1) acc[2] = add_abs<kF32>(acc[2], s_w[i + 2 * kQThreads]);
-  }
-#pragma unroll
-  for (int u = 0; u < kTailRegs; ++u)
-    if (tail_v0 + t + static_cast<int64_t>(u) * kQThreads < tail_v1) acc[u] = add_abs<kF32>(acc[u], tr[u]);
-  for (int64_t i = tail_v0 + t + static_cast<int64_t>(kTailRegs) * kQThreads; i < tail_v1; i += 4 * kQThreads) {
-    uint4 v[4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) v[u] = i + u * kQThreads < tail_v1 ? __ldg(a.W + i + u * kQThreads) : make_uint4(0u, 0u, 0u, 0u);
-#pragma unroll
-    for (int u = 0; u < 4; ++u)
-      if (i + u * kQThreads < tail_v1) acc[u] = add_abs<kF32>(acc[u], v[u]);
-  }
-  double ts = __dadd_rn(__dadd_rn(acc[0], acc[1]), __dadd_rn(acc[2], acc[3]));
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) ts = __dadd_rn(ts, __shfl_xor_sync(0xffffffffu, ts, off));
-  if (lane == 0) s_red[warp] = ts;
-  __syncthreads();
-  // the next launch may be scheduled once every CTA of this grid has come
-  // this far (so all of them are resident)
+  __shared__ int s_mode;  // 1: gamma known, 2: exact sum needed, -1: gave up
+  pdl_wait_primary();     // the sum launch has completed
   pdl_launch_dependents();
-
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t nw = static_cast<int64_t>(gridDim.x) * kCodeWarps;
+  const int64_t nrounds = (a.nvec + 127) / 128;
+  int64_t r = static_cast<int64_t>(blockIdx.x) * kCodeWarps + warp;
+  uint4 v[4];
+  load_round(a.W, r, nrounds, a.nvec, lane, v);
+  // the partial sums into shared memory, all loads of the CTA at once
+  for (int p = threadIdx.x; p < a.nparts; p += kCodeThreads) s_parts[p] = __ldcg(a.parts + p);
+  __syncthreads();
   if (warp == 0) {
-    // ------------------------------------------------ control warp: gamma
-    uint32_t last = 0;
-    if (lane == 0) {
-      double part = 0.0;
-      for (int w = 0; w < kQWarps; ++w) part = __dadd_rn(part, s_red[w]);
-      partials[b] = part;
-      pdl_wait_primary();  // launch 1 has cleared the workspace
-      __threadfence();
-      last = atomicAdd(&arrive[0], 1u) == G - 1;
-      __threadfence();  // with the atomic: acquires the other CTAs' partial sums
-    }
-    last = __shfl_sync(0xffffffffu, last, 0);
-    int mode = 0;
-    float gamma = 0.0f;
-    if (last) {
-      // the partial sums in one fixed order: lane l adds l, l + 32, ..., then a
-      // fixed shuffle tree (the same sum whichever CTA forms it)
-      double s = 0.0;
-      for (uint32_t j = lane; j < G; j += 32) s = __dadd_rn(s, __ldcg(partials + j));
+    double s = 0.0;
+    for (int p = lane; p < a.nparts; p += 32) s = __dadd_rn(s, s_parts[p]);
 #pragma unroll
-      for (int off = 16; off > 0; off >>= 1) s = __dadd_rn(s, __shfl_xor_sync(0xffffffffu, s, off));
+    for (int off = 16; off > 0; off >>= 1) s = __dadd_rn(s, __shfl_xor_sync(0xffffffffu, s, off));
+    if (lane == 0) {
       const float glo = gamma_of_sum(__dmul_rd(s, a.enc_lo), a.numel);
       const float ghi = gamma_of_sum(__dmul_ru(s, a.enc_hi), a.numel);
-      mode = __float_as_uint(glo) == __float_as_uint(ghi) ? 1 : 2;
-      gamma = glo;
-      if (lane == 0) {
-        flag[1] = __float_as_uint(glo);
-        st_release_u32(&flag[0], static_cast<uint32_t>(mode));
-      }
-    } else {
-      if (lane == 0) {
-        // wait for the last CTA's gamma (bounded; polled every ~0.1 us)
-        uint32_t f = ld_acquire_u32(&flag[0]);
-        const unsigned long long t0 = globaltimer_ns();
-        while (f == 0) {
-          __nanosleep(100);
-          f = ld_acquire_u32(&flag[0]);
-          if (f == 0 && globaltimer_ns() - t0 > kWaitLimitNs) {
-            record_error(a.err, kDevTimeout);
-            break;
-          }
-        }
-        mode = static_cast<int>(f);
-        gamma = __uint_as_float(__ldcg(&flag[1]));
-      }
-      mode = __shfl_sync(0xffffffffu, mode, 0);
-      gamma = __shfl_sync(0xffffffffu, gamma, 0);
+      s_gamma = glo;
+      s_mode = __float_as_uint(glo) == __float_as_uint(ghi) ? 1 : 2;
     }
-    if (mode == 0 || s_abort) {
-      if (lane == 0) s_state = -1;
-    } else {
-      if (mode == 2) {
-        // exact sum: every warp bins its share of the slice (the work loop
-        // below); then one arrival per CTA and the exact gamma
-        for (int e = lane; e < 256; e += 32) s_bins[e] = 0ull;
-        __syncwarp();
-        if (lane == 0) {
-          __threadfence_block();
-          s_state = 2;
-        }
-        bool ok = true;
-        if (lane == 0) {
-          const unsigned long long t0 = globaltimer_ns();
-          while (*reinterpret_cast<volatile int*>(&s_binned) < kQWarps - 1) {
-            __nanosleep(100);
-            if (globaltimer_ns() - t0 > kWaitLimitNs) {
-              record_error(a.err, kDevTimeout);
-              ok = false;
-              break;
-            }
-          }
-        }
-        // warp 0's own share
-        for (int64_t i = lane; i < onv; i += 32 * kQWarps) bin_abs<kF32>(s_bins, s_w[i]);
-        for (int64_t i = tail_v0 + lane; i < tail_v1; i += 32 * kQWarps) bin_abs<kF32>(s_bins, __ldg(a.W + i));
-        __syncwarp();
-        __threadfence_block();
-        for (int e = lane; e < 256; e += 32)
-          if (s_bins[e]) atomicAdd(gbins + e, s_bins[e]);
-        __syncwarp();  // every lane's bins are added before lane 0 arrives
-        if (lane == 0 && ok) {
-          ok = grid_arrive_wait(&arrive[1], G, a.err);
-          if (ok) gamma = gamma_of_sum(exact_sum_from_bins(gbins, kF32 ? 23 : 7), a.numel);
-        }
-        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-        gamma = __shfl_sync(0xffffffffu, gamma, 0);
-        if (!ok) mode = 0;
-      }
-      if (lane == 0) {
-        if (mode == 0) {
-          s_state = -1;
-        } else {
-          if (b == 0) *a.gamma_out = gamma;
-          const float thr = __double2float_rd(__dmul_rn(static_cast<double>(gamma), 0.5 + 0x1p-25));
-          uint32_t key;
-          if constexpr (kF32) {
-            key = __float_as_uint(thr);
-          } else {
-            const uint32_t tb = __float_as_uint(thr) >> 16;
-            key = (tb | (tb << 16)) + 0x80008000u;
-          }
-          s_key = key;
-          s_gamma = gamma;
-          __threadfence_block();
-          s_state = 1;
-        }
-      }
-    }
-    __syncwarp();
+    for (int e = lane; e < 256; e += 32) s_bins[e] = 0ull;
   }
-
-  // -------------------------------------------------- work loop, all warps
-  const int64_t on_rounds = (onv + 127) / 128;
-  const int64_t n_rounds = on_rounds + (tail_v1 - tail_v0 + 127) / 128;
-  bool rows_left = a.M > 0;
-  bool binned = warp == 0;  // warp 0 bins inside the control block
-  if (rows_left) pdl_wait_primary();  // launch 1 has cleared the row counter
-  volatile int* state = &s_state;
-  const unsigned long long t_idle = globaltimer_ns();
-  for (;;) {
-    const int st = *state;
-    if (st < 0) break;
-    if (st == 2 && !binned) {
-      for (int64_t i = lane + 32 * warp; i < onv; i += 32 * kQWarps) bin_abs<kF32>(s_bins, s_w[i]);
-      for (int64_t i = tail_v0 + lane + 32 * warp; i < tail_v1; i += 32 * kQWarps) bin_abs<kF32>(s_bins, __ldg(a.W + i));
-      __syncwarp();
-      __threadfence_block();
-      if (lane == 0) atomicAdd(&s_binned, 1);
-      binned = true;
-      continue;
+  __syncthreads();
+  if (s_mode == 2) {
+    for (int64_t q = r; q < nrounds; q += nw) {
+      uint4 w[4];
+      load_round(a.W, q, nrounds, a.nvec, lane, w);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) bin_abs<kF32>(s_bins, w[u]);
     }
-    if (st == 1) {
-      uint32_t r = 0;
-      if (lane == 0) r = static_cast<uint32_t>(atomicAdd(&s_round, 1));
-      r = __shfl_sync(0xffffffffu, r, 0);
-      if (r < n_rounds) {
-        const uint32_t key = s_key;
-        if (r < on_rounds)
-          code_round<kF32, true>(s_w, 128 * static_cast<int64_t>(r), onv, a.packed + g0, key, lane);
-        else
-          code_round<kF32, false>(a.W + tail_v0, 128 * (r - on_rounds), tail_v1 - tail_v0, a.packed + g0 + on, key,
-                                  lane);
-        continue;
+    __syncthreads();
+    if (warp == 0) {
+      unsigned long long* gbins = reinterpret_cast<unsigned long long*>(a.ws + kWsBins);
+      for (int e = lane; e < 256; e += 32)
+        if (s_bins[e]) atomicAdd(gbins + e, s_bins[e]);
+      __syncwarp();  // every lane's bins are added before lane 0 arrives
+      if (lane == 0) {
+        if (grid_arrive_wait(reinterpret_cast<uint32_t*>(a.ws + kWsArrive), gridDim.x, a.err)) {
+          s_gamma = gamma_of_sum(exact_sum_from_bins(gbins, kF32 ? 23 : 7), a.numel);
+          s_mode = 1;
+        } else {
+          s_mode = -1;
+        }
       }
     }
-    if (rows_left) {
-      const int64_t m0 = warp_claim(rows, 2u);
-      if (m0 < a.M) {
-        token_pair<VPL>(a, m0);
-        continue;
-      }
-      rows_left = false;
-    }
-    if (st == 1) break;  // codes all claimed, no rows left
-    __nanosleep(200);    // waiting for gamma
-    if (globaltimer_ns() - t_idle > 2 * kWaitLimitNs) break;  // the control warp gave up
+    __syncthreads();
+    if (s_mode < 0) return;
+  }
+  const float gamma = s_gamma;
+  if (blockIdx.x == 0 && threadIdx.x == 0) *a.gamma_out = gamma;
+  const uint32_t key = code_key<kF32>(gamma);
+  for (; r < nrounds; r += nw) {
+    uint4 nx[4];
+    load_round(a.W, r + nw, nrounds, a.nvec, lane, nx);
+    store_codes<kF32>(v, 128 * r, a.nvec, a.packed, key, lane);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) v[u] = nx[u];
   }
 }
 
 }  // namespace
 
 // Fixed device scratch for bl_quantize_weight_noalloc: the workspace of one
-// call (arrival counters, one fp64 partial sum per CTA, exact-sum bins),
-// 10752 bytes. Every GPU that loads the library holds this array until the
-// process exits.
+// call (the exact-sum arrival counter and bins, and one fp64 partial sum per
+// CTA of the sum launch). Every GPU that loads the library holds this array
+// until the process exits.
 static __device__ __align__(256) uint8_t g_noalloc_ws[kWsBytes];
 
 size_t quantize_workspace_bytes() { return kWsBytes; }
 
 namespace {
 
-// Geometry of one S1 (+ S2) launch.
-struct QuantGeometry {
-  unsigned ctas;
-  size_t smem;
-};
-
-template <bool kF32>
-QuantGeometry quant_geometry(int64_t ngroups, int64_t M, QuantArgs& a) {
-  constexpr int V = kF32 ? 4 : 2;
-  constexpr int kGroupBytes = 16 * V;
-  constexpr int kChunkGroups = kChunkBytes / kGroupBytes;
-  constexpr int kElems = kF32 ? 4 : 8;  // elements per 16-byte vector
-  // enough CTAs to spread the slice (>= 256 groups each) and the tokens (>= 16
-  // rows each), at most one per SM so that all of them are resident together
-  const int64_t want = std::max<int64_t>((ngroups + 255) / 256, (M + 15) / 16);
-  const int64_t cap = std::min<int64_t>(device_sm_count(), kMaxQuantCtas);
-  const int64_t G = std::max<int64_t>(1, std::min(want, cap));
-  a.ngroups = ngroups;
-  a.per = (ngroups + G - 1) / G;
-  a.onchip_cap = kMaxOnchipBytes / kGroupBytes;
-  const int64_t on_max = std::min<int64_t>(a.per, a.onchip_cap);
-  // Enclosure of S around the fp64 tree sum: every leaf passes through at most
-  // d roundings (its accumulator's sequential adds, the four accumulators, the
-  // warp shuffle tree, the sequential warp sums, the lane sums of the
-  // partials, their shuffle tree), each off by at most 2^-53 of a partial sum
-  // that is at most S (1 + 2^-30) with all terms >= 0, so |fp64 sum - S| <=
-  // d 2^-53 (1 + 2^-30) S; e = d 2^-52 covers S on both sides.
-  const int64_t nch_max = (on_max + kChunkGroups - 1) / kChunkGroups;
-  const double per_acc = static_cast<double>(a.per) * V / (4.0 * kQThreads) + static_cast<double>(nch_max) + 3.0;
-  const double d = kElems * per_acc + 2 + 5 + kQWarps + std::ceil(static_cast<double>(G) / 32.0) + 5 + 8;
-  const double e = std::ldexp(d, -52);
-  a.enc_lo = 1.0 - e;
-  a.enc_hi = 1.0 + e;
-  return {static_cast<unsigned>(G), static_cast<size_t>(on_max) * kGroupBytes};
-}
-
-template <bool kF32, int VPL>
-cudaError_t launch_fused(QuantArgs& a, cudaStream_t s) {
-  static bool configured[64] = {};
+// Resident CTAs per SM of `kernel` at `threads` threads (cached per device in
+// the caller's table).
+template <typename Kernel>
+int blocks_per_sm(Kernel kernel, int threads, int (&cache)[64]) {
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && !configured[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(quant_fused_kernel<kF32, VPL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         kMaxOnchipBytes);
-    if (e != cudaSuccess) return e;
-    configured[dev] = true;
-  }
-  const QuantGeometry geo = quant_geometry<kF32>(a.ngroups, a.M, a);
-  cudaError_t e = launch_pdl(quant_reset_kernel, dim3(1), dim3(256), 0, s, a.ws);
-  if (e != cudaSuccess) return e;
-  return launch_pdl(quant_fused_kernel<kF32, VPL>, dim3(geo.ctas), dim3(kQThreads), geo.smem, s, a);
+  if (dev >= 0 && dev < 64 && cache[dev]) return cache[dev];
+  int occ = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kernel, threads, 0) != cudaSuccess || occ < 1) occ = 1;
+  cudaGetLastError();
+  if (dev >= 0 && dev < 64) cache[dev] = occ;
+  return occ;
 }
 
-template <int VPL>
-cudaError_t launch_fused_dtype(bool f32, QuantArgs& a, cudaStream_t s) {
-  return f32 ? launch_fused<true, VPL>(a, s) : launch_fused<false, VPL>(a, s);
+// The two launches of S1 (+ S2 when M > 0).
+template <bool kF32, int VPL>
+cudaError_t launch_s1(const void* W, int64_t N, int64_t K, const void* x, int64_t M, uint8_t* packed, float* gamma,
+                      uint8_t* ws, int8_t* xq, float* sx, int* err, cudaStream_t s) {
+  constexpr int kElems = kF32 ? 4 : 8;  // elements per 16-byte vector
+  static int occ_sum[64] = {}, occ_code[64] = {};
+  const int64_t sms = device_sm_count();
+  SumArgs sa{};
+  sa.W = static_cast<const uint4*>(W);
+  sa.nvec = N * K / kElems;
+  sa.ws = ws;
+  sa.parts = reinterpret_cast<double*>(ws + kWsParts);
+  sa.x = static_cast<const uint4*>(x);
+  sa.M = M;
+  sa.nv = static_cast<int>(K / 8);
+  sa.xq = xq;
+  sa.sx = sx;
+  // sum launch: every SM filled (at most kMaxQuantCtas partial sums), fewer
+  // CTAs only when W has fewer than 2048 vectors per CTA and the tokens fewer
+  // than one row per warp
+  const int64_t cap1 =
+      std::min<int64_t>(sms * blocks_per_sm(quant_sum_kernel<kF32, VPL>, kSumThreads, occ_sum), kMaxQuantCtas);
+  const int64_t want1 = std::max<int64_t>((sa.nvec + kSumThreads * kSumUnroll - 1) / (kSumThreads * kSumUnroll),
+                                          (M + kSumWarps - 1) / kSumWarps);
+  const int64_t G1 = std::max<int64_t>(1, std::min(want1, cap1));
+  sa.per = (sa.nvec + G1 - 1) / G1;
+
+  CodeArgs ca{};
+  ca.W = sa.W;
+  ca.nvec = sa.nvec;
+  ca.parts = sa.parts;
+  ca.nparts = static_cast<int>(G1);
+  ca.numel = static_cast<double>(N * K);
+  ca.packed = reinterpret_cast<uint32_t*>(packed);
+  ca.gamma_out = gamma;
+  ca.ws = ws;
+  ca.err = err;
+  // code launch: no more CTAs than can be resident at once (the exact-sum
+  // barrier), and no more warps than rounds of 128 vectors
+  const int64_t nrounds = (sa.nvec + 127) / 128;
+  const int64_t cap2 = sms * blocks_per_sm(quant_code_kernel<kF32>, kCodeThreads, occ_code);
+  const int64_t G2 = std::max<int64_t>(1, std::min<int64_t>(cap2, (nrounds + kCodeWarps - 1) / kCodeWarps));
+  // Enclosure of S around the fp64 sum. Every |w| passes through at most d
+  // roundings: its accumulator's sequential adds (kElems per vector, at most
+  // ceil(nj / 4) vectors of the thread's nj), the two levels joining the four
+  // accumulators, the 5 butterfly levels, the kSumWarps sequential warp sums,
+  // the ceil(G1 / 32) sequential partial sums of a lane and the 5 butterfly
+  // levels of the code launch. Each rounding is off by at most 2^-53 of a
+  // partial sum, and with all terms >= 0 every partial sum is at most
+  // S (1 + 2^-30), so |fp64 sum - S| <= d 2^-53 (1 + 2^-30) S; e = d 2^-52
+  // (8 roundings to spare) covers S on both sides.
+  const int64_t nj = (sa.per + kSumThreads - 1) / kSumThreads;
+  const double d = static_cast<double>(kElems) * static_cast<double>((nj + 3) / 4) + 2 + 5 + kSumWarps +
+                   static_cast<double>((G1 + 31) / 32) + 5 + 8;
+  const double e = std::ldexp(d, -52);
+  ca.enc_lo = 1.0 - e;
+  ca.enc_hi = 1.0 + e;
+
+  cudaError_t st = launch_pdl(quant_sum_kernel<kF32, VPL>, dim3(static_cast<unsigned>(G1)), dim3(kSumThreads), 0, s, sa);
+  if (st != cudaSuccess) return st;
+  return launch_pdl(quant_code_kernel<kF32>, dim3(static_cast<unsigned>(G2)), dim3(kCodeThreads), 0, s, ca);
 }
 
 template <int VPL>
 void launch_act(const uint4* xv, int64_t M, int nv, int8_t* xq, float* sx, cudaStream_t s) {
   constexpr bool kPrefetch = VPL <= 12;
   static int per_sm[64] = {};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  int occ = (dev >= 0 && dev < 64) ? per_sm[dev] : 0;
-  if (!occ) {
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, act_quant_kernel<VPL, kPrefetch>,
-                                                      32 * kActRowsPerBlock, 0) != cudaSuccess || occ < 1)
-      occ = 1;
-    cudaGetLastError();
-    if (dev >= 0 && dev < 64) per_sm[dev] = occ;
-  }
+  const int occ = blocks_per_sm(act_quant_kernel<VPL, kPrefetch>, 32 * kActRowsPerBlock, per_sm);
   const int64_t want = (M + kActRowsPerBlock - 1) / kActRowsPerBlock;
   const int64_t cap = static_cast<int64_t>(occ) * device_sm_count();
   const unsigned grid = static_cast<unsigned>(want < cap ? want : cap);
@@ -879,26 +728,15 @@ void launch_act(const uint4* xv, int64_t M, int nv, int8_t* xq, float* sx, cudaS
 cudaError_t launch_quantize(const void* W, int w_is_f32, int64_t N, int64_t K, const void* x, int64_t M,
                             uint8_t* packed, float* gamma, void* workspace, int8_t* xq, float* sx, int* err,
                             cudaStream_t s) {
-  QuantArgs a{};
-  a.W = static_cast<const uint4*>(W);
-  a.ngroups = N * K / 16;  // K % 32 == 0
-  a.numel = static_cast<double>(N * K);
-  a.packed = reinterpret_cast<uint32_t*>(packed);
-  a.gamma_out = gamma;
-  a.ws = static_cast<uint8_t*>(workspace);
-  a.err = err;
-  a.x = static_cast<const uint4*>(x);
-  a.M = M;
-  a.nv = static_cast<int>(K / 8);
-  a.xq = xq;
-  a.sx = sx;
-  const int per_lane = (a.nv + 31) / 32;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const int per_lane = (static_cast<int>(K / 8) + 31) / 32;
   const bool f32 = w_is_f32 != 0;
   cudaError_t e = cudaSuccess;
   switch (M > 0 && per_lane <= 10 ? per_lane : 0) {
-#define BL_Q_CASE(n)                          \
-  case n:                                     \
-    e = launch_fused_dtype<n>(f32, a, s);     \
+#define BL_Q_CASE(n)                                                                     \
+  case n:                                                                                \
+    e = f32 ? launch_s1<true, n>(W, N, K, x, M, packed, gamma, ws, xq, sx, err, s)      \
+            : launch_s1<false, n>(W, N, K, x, M, packed, gamma, ws, xq, sx, err, s);    \
     break;
     BL_Q_CASE(0) BL_Q_CASE(1) BL_Q_CASE(2) BL_Q_CASE(3) BL_Q_CASE(4) BL_Q_CASE(5) BL_Q_CASE(6)
     BL_Q_CASE(7) BL_Q_CASE(8) BL_Q_CASE(9) BL_Q_CASE(10)

@@ -36,11 +36,12 @@ def test_version_and_status_strings():
 
 
 def test_workspace_size():
-    # counters and flags (512 bytes), a partial sum per CTA (up to 1024 CTAs)
-    # and 256 exact-sum bins: the same for every tensor
+    # the exact-sum arrival counter (128-byte line), 256 exact-sum bins, a
+    # spacer line and one fp64 partial sum per summing CTA (at most 1024): the
+    # same for every tensor
     assert b.bl_quantize_weight_workspace_size(0, 32) == 0
-    assert b.bl_quantize_weight_workspace_size(256, 128) == 512 + 8 * 1024 + 8 * 256
-    assert b.bl_quantize_weight_workspace_size(6912, 2560) == 512 + 8 * 1024 + 8 * 256
+    assert b.bl_quantize_weight_workspace_size(256, 128) == 128 + 8 * 256 + 128 + 8 * 1024
+    assert b.bl_quantize_weight_workspace_size(6912, 2560) == 128 + 8 * 256 + 128 + 8 * 1024
 
 
 FAKE = ctypes.c_void_p(0x10000)        # never dereferenced: validation fails first
