@@ -1,8 +1,8 @@
 """Benchmark of the BitLinear training hot path (fwd + bwd) on B200.
 
 One step = one pass of the whole hot path over one batch:
-  S1 + S2 bl_quantize (2 launches: |W| partial sums together with the
-  token quantisation, then the code pass) -> S3 bl_forward
+  S1 + S2 bl_quantize (2 launches: |W| partial sums with part of the token
+  rows, then gamma and the codes with the other rows) -> S3 bl_forward
   -> S4 bl_backward (dX and dW in one launch)                  (4 launches)
 
 Default workload: the up-projection BitLinear 2560 -> 6912 at 8 x 512 tokens
@@ -14,8 +14,11 @@ Timing: W >= 3 untimed warm-up steps, then exactly K timed steps on
 resident inputs. L2 is flushed (256 MiB written, then read back, so that no
 dirty line is left) before every step, outside the timed events; each step is bracketed by CUDA events on the launching
 stream (the headline); a second pass of K steps puts events between the C-ABI
-calls for the per-kernel times (events between kernels can cost the overlap
-of programmatically dependent launches, so that pass is not the headline). For N > 1
+calls (`ms_isolated` per kernel: one launch after a flush, with the launch
+latency an event in front of it costs). The per-kernel times the roofline
+fractions use come from CUDA graphs of 16 back-to-back calls of one stage over
+4 rotating sets of inputs and outputs (more than L2 between reuses), replayed
+between two events: each launch's average duration in a stream. For N > 1
 (torchrun, one rank per GPU) the step is the data-parallel one: every rank
 runs the path on its own tokens (weak scaling) with the same W, and the
 partial dW are summed over the ranks by an NCCL all-reduce inside the timed
@@ -176,7 +179,7 @@ def job_tops(ops_per_rank_step: float, world: int, steps: int, job_ms: float) ->
 # ----------------------------------------------------------------- our arm
 
 STAGES = ["quantize", "forward", "backward"]
-LAUNCHES_PER_STEP = 4  # S1 pass A; S2 with the S1 code pass; S3; S4 (dX and dW in one launch)
+LAUNCHES_PER_STEP = 4  # S1 sums (+ S2 rows); S1 codes (+ S2 rows); S3; S4 (dX and dW in one launch)
 
 
 def stage_work(M, N, K, w_bytes):
@@ -186,6 +189,60 @@ def stage_work(M, N, K, w_bytes):
         "forward": {"bound": "tensor", "ops": 2 * M * N * K, "dtype": "int8"},
         "backward": {"bound": "tensor", "ops": 4 * M * N * K, "dtype": "bf16"},
     }
+
+
+def stage_graph_ms(bl, x, w, dy, M, N, K, dev, n_sets=4, calls=16, reps=5):
+    """Per-call device time of each stage: `calls` back-to-back C-ABI calls of
+    the stage, over n_sets rotating copies of its inputs and outputs (between
+    two uses of one set the other sets move well over the 126 MB of L2),
+    captured in one CUDA graph and replayed between two events after an L2
+    flush; the median over `reps` replays, divided by `calls`. This is each
+    launch's average duration inside a stream of launches, without host launch
+    gaps or the cost of an event around every launch."""
+    sets = []
+    for _ in range(n_sets):
+        b = bl.StepBuffers.allocate(M, N, K, torch.bfloat16, device=dev)
+        xs, ws_, dys = x.clone(), w.clone(), dy.clone()
+        bl.bl_quantize(ws_, xs, b.w_packed, b.gamma, b.xq, b.sx, b.workspace)
+        sets.append((xs, ws_, dys, b))
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    calls_of = {
+        "quantize": lambda t: bl.bl_quantize(t[1], t[0], t[3].w_packed, t[3].gamma, t[3].xq, t[3].sx, t[3].workspace),
+        "forward": lambda t: bl.bl_forward(t[3].xq, t[3].sx, t[3].w_packed, t[3].gamma, t[3].y, None),
+        "backward": lambda t: bl.bl_backward(t[2], t[3].xq, t[3].sx, t[3].w_packed, t[3].gamma, t[3].dX, t[3].dW,
+                                             False),
+    }
+    out = {}
+    for name, call in calls_of.items():
+        side = torch.cuda.Stream(dev)
+        side.wait_stream(torch.cuda.current_stream(dev))
+        with torch.cuda.stream(side):
+            for i in range(n_sets):
+                call(sets[i])
+        torch.cuda.current_stream(dev).wait_stream(side)
+        torch.cuda.synchronize(dev)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for i in range(calls):
+                call(sets[i % n_sets])
+        ts = []
+        for r in range(reps + 1):
+            flush.fill_(r & 0xFF)
+            flush.view(torch.int64).max()
+            s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s.record()
+            g.replay()
+            e.record()
+            torch.cuda.synchronize(dev)
+            if r > 0:
+                ts.append(s.elapsed_time(e) / calls)
+        del g
+        out[name] = sorted(ts)[len(ts) // 2]
+    if bl.bl_get_last_error() != 0:
+        raise RuntimeError("device error during the per-stage graph timing")
+    del sets, flush
+    torch.cuda.empty_cache()
+    return out
 
 
 def run_ours(args, rank, world, local_rank):
@@ -279,6 +336,7 @@ def run_ours(args, rank, world, local_rank):
         remeasured = True
     breakdown_ms, per_stage = timed(True)
     clocks["remeasured"] = remeasured
+    graph_ms = stage_graph_ms(bl, x, w, dy, M, N, K, dev)
     if bl.bl_get_last_error() != 0:
         raise RuntimeError("device error during the timed region")
 
@@ -297,7 +355,7 @@ def run_ours(args, rank, world, local_rank):
     kernels = {}
     roof_ms = 0.0
     for s in STAGES:
-        ms = per_stage[s] / args.steps
+        ms = graph_ms[s]
         wk = work[s]
         if wk["bound"] == "hbm":
             ach = wk["bytes"] / (ms * 1e-3) / 1e9
@@ -310,9 +368,9 @@ def run_ours(args, rank, world, local_rank):
             unit = "TOPS" if wk["dtype"] == "int8" else "TFLOP/s"
             roof_ms += wk["ops"] / (peak * 1e12) * 1e3
         kernels[s] = {"ms": round(ms, 5), "achieved": round(ach, 1), "unit": unit, "peak": peak,
-                      "frac": round(ach / peak, 4), "share": round(per_stage[s] / sum(per_stage[t] for t in STAGES), 4),
-                      "traffic": traffic.get(s)}
-    dom = max(STAGES, key=lambda s: per_stage[s])
+                      "frac": round(ach / peak, 4), "share": round(graph_ms[s] / sum(graph_ms[t] for t in STAGES), 4),
+                      "ms_isolated": round(per_stage[s] / args.steps, 5), "traffic": traffic.get(s)}
+    dom = max(STAGES, key=lambda s: graph_ms[s])
     dk = kernels[dom]
     roofline = {"kernel": dom, "bound": work[dom]["bound"], "achieved": dk["achieved"], "peak": dk["peak"],
                 "unit": "GB/s" if work[dom]["bound"] == "hbm" else "TFLOP/s", "frac": dk["frac"],

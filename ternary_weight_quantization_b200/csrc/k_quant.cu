@@ -41,11 +41,13 @@ __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w 
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
 // ---------------------------------------------------------------- S1 geometry
-constexpr int kSumThreads = 256;  // sum launch: 8 warps per CTA
+constexpr int kSumThreads = 1024; // sum launch: 32 warps per CTA
 constexpr int kSumWarps = kSumThreads / 32;
 constexpr int kSumUnroll = 8;     // 16-byte loads in flight per thread
+constexpr bool kSumInterleave = false;  // W in blocks dealt to the CTAs in turn (else contiguous slices)
 constexpr int kCodeThreads = 512; // code launch: 16 warps per CTA
 constexpr int kCodeWarps = kCodeThreads / 32;
+constexpr int kCodeRowsPerCta = 10;// token rows a code-launch CTA quantises (< kCodeWarps)
 
 // Workspace (each part on its own 128-byte lines): at 0 the arrivals at the
 // exact-sum barrier (u32); at 128 256 uint64 exact-sum bins (one per exponent
@@ -192,28 +194,40 @@ __device__ __forceinline__ float gamma_of_sum(double S, double numel) {
 // thr the largest float <= T, that is |w| > thr: one compare, no division.
 //
 // 8 bf16 of one vector -> 16 bits of codes (element i at bits 2i, 2i + 1;
-// field 00 = 0, 01 = +1, 11 = -1). For a 15-bit magnitude b and thr > 0,
-// |w| > thr <=> b > bits(thr) >> 16, so both halves of a word are compared by
-// one subtraction: 0x8000 + tb - b keeps bit 15 clear exactly when b > tb (no
-// borrow crosses the halves, b <= 0x7FFF). One byte permutation per word pair
-// gathers the four compare bits (and, of the weights, the four sign bits) as
-// the top bits of four bytes; a high multiply by 2^25 + 2^19 + 2^13 + 2^7
-// (2^26 + ... for the signs) moves bits 7, 15, 23, 31 to bits 0, 2, 4, 6 (1,
-// 3, 5, 7) of its high word -- every partial product lands on its own bit, so
-// nothing carries -- and one logic operation merges the two. The integer
-// logic unit, which bounds this pass, does about 1.75 operations per element;
-// the multiplies run on the multiply-add pipe.
-__device__ __forceinline__ uint32_t codes8_bf16(const uint4& v, uint32_t bias) {
+// field 00 = 0, 01 = +1, 11 = -1). For a bf16 w and thr > 0, |w| > thr <=>
+// w > tb or w < -tb with tb = thr truncated to bf16 (the largest bf16 <= thr),
+// so two bf16x2 compares per word (on the multiply-add pipe) give both the
+// nonzero and the sign information: each half of a result is 1.0 (0x3F80)
+// where the compare holds, else 0. One byte permutation per word pair
+// gathers the low bytes of the halves (0x80 or 0) of four elements; a high
+// multiply by S = 2^25 + 2^19 + 2^13 + 2^7 moves bits 7, 15, 23, 31 to bits
+// 0, 2, 4, 6 of its high word (+1 fields), one by 3 S to bits 0-1, 2-3, 4-5,
+// 6-7 (-1 fields); every partial product lands on bits of its own, so nothing
+// carries into the low byte, and the two (exclusive) results are added by the
+// second multiply. Bits 16..31 of the result are not zero.
+__device__ __forceinline__ uint32_t bf16x2_gt(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("set.gt.bf16x2.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+__device__ __forceinline__ uint32_t bf16x2_lt(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("set.lt.bf16x2.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+// thr2: tb in both halves.
+__device__ __forceinline__ uint32_t codes8_bf16(const uint4& v, uint32_t thr2) {
   constexpr uint32_t kSpread = (1u << 25) | (1u << 19) | (1u << 13) | (1u << 7);
-  const uint32_t d0 = bias - (v.x & 0x7FFF7FFFu), d1 = bias - (v.y & 0x7FFF7FFFu);
-  const uint32_t d2 = bias - (v.z & 0x7FFF7FFFu), d3 = bias - (v.w & 0x7FFF7FFFu);
-  const uint32_t nzl = ~__byte_perm(d0, d1, 0x7531) & 0x80808080u;  // elements 0..3 nonzero
-  const uint32_t nzh = ~__byte_perm(d2, d3, 0x7531) & 0x80808080u;  // elements 4..7
-  const uint32_t ngl = nzl & __byte_perm(v.x, v.y, 0x7531);          // and negative
-  const uint32_t ngh = nzh & __byte_perm(v.z, v.w, 0x7531);
-  const uint32_t lo = (__umulhi(nzl, kSpread) & 0x55u) | (__umulhi(ngl, 2 * kSpread) & 0xAAu);
-  const uint32_t hi = (__umulhi(nzh, kSpread) & 0x55u) | (__umulhi(ngh, 2 * kSpread) & 0xAAu);
-  return hi * 256u + lo;
+  const uint32_t nthr2 = thr2 | 0x80008000u;
+  const uint32_t pl = __byte_perm(bf16x2_gt(v.x, thr2), bf16x2_gt(v.y, thr2), 0x6420);  // +1, elements 0..3
+  const uint32_t ph = __byte_perm(bf16x2_gt(v.z, thr2), bf16x2_gt(v.w, thr2), 0x6420);  // +1, elements 4..7
+  const uint32_t nl = __byte_perm(bf16x2_lt(v.x, nthr2), bf16x2_lt(v.y, nthr2), 0x6420);  // -1
+  const uint32_t nh = __byte_perm(bf16x2_lt(v.z, nthr2), bf16x2_lt(v.w, nthr2), 0x6420);
+  const uint32_t lo = __umulhi(nl, 3u * kSpread) + __umulhi(pl, kSpread);
+  const uint32_t hi = __umulhi(nh, 3u * kSpread) + __umulhi(ph, kSpread);
+  return __byte_perm(lo, hi, 0x0040);
 }
 
 // 4 fp32 of one vector -> 8 bits of codes.
@@ -229,7 +243,7 @@ __device__ __forceinline__ uint32_t codes4_f32(const uint4& v, float thr) {
 }
 
 // Code bits of one 16-byte vector (16 bits for bf16, 8 for fp32). `key` is
-// the bf16 compare bias or the fp32 threshold's bit pattern.
+// the bf16 threshold in both halves or the fp32 threshold's bit pattern.
 template <bool kF32>
 __device__ __forceinline__ uint32_t vec_codes(const uint4& v, uint32_t key) {
   if constexpr (kF32) return codes4_f32(v, __uint_as_float(key));
@@ -237,16 +251,19 @@ __device__ __forceinline__ uint32_t vec_codes(const uint4& v, uint32_t key) {
 }
 
 // The vectors of a warp's 32 consecutive 16-byte vectors, one per lane, are
-// V = 2 (bf16) or 4 (fp32) per group: the lanes of a group OR their code bits
-// together and its first lane writes the group's 32-bit word.
+// V = 2 (bf16) or 4 (fp32) per group: the lanes of a group combine their code
+// bits and its first lane gets the group's 32-bit word (bf16: the low halves
+// of the two lanes' results; fp32: the four 8-bit results).
 template <bool kF32>
 __device__ __forceinline__ uint32_t gather_group_word(uint32_t bits, int lane) {
-  constexpr int V = kF32 ? 4 : 2;
-  constexpr int kBits = 32 / V;
-  uint32_t word = bits << (kBits * (lane & (V - 1)));
+  if constexpr (kF32) {
+    uint32_t word = bits << (8 * (lane & 3));
 #pragma unroll
-  for (int off = 1; off < V; off <<= 1) word |= __shfl_down_sync(0xffffffffu, word, off);
-  return word;
+    for (int off = 1; off < 4; off <<= 1) word |= __shfl_down_sync(0xffffffffu, word, off);
+    return word;
+  } else {
+    return __byte_perm(bits, __shfl_down_sync(0xffffffffu, bits, 1), 0x5410);
+  }
 }
 
 // ---------------------------------------------------------------- grid barrier
@@ -436,18 +453,19 @@ struct SumArgs {
   float* sx;
 };
 
-// Sum launch, kSumThreads threads per CTA, several CTAs per SM. Nothing in it
-// waits on another CTA. CTA b first quantises token rows [b M / G, (b + 1) M /
-// G) (warp w: rows w, w + 8, ... of them), then sums |W| of its slice, so
-// that W is the most recent data in L2 when the code launch reads it again.
-// Thread t adds vectors t, t + 256, ... of the slice, the j-th of them into
-// accumulator j mod 4 (in order, elements of a vector in order); the CTA's
+// Sum launch, kSumThreads threads per CTA. Nothing in it waits on another
+// CTA. CTA b first quantises token rows [b M / G, (b + 1) M / G) (warp w:
+// rows w, w + kSumWarps, ... of them), then sums |W| over its share, so that
+// W is the most recent data in L2 when the code launch reads it again. Thread
+// t adds its vectors (the j-th at a fixed index: in the CTA's contiguous
+// slice, or in the j-th block of kSumThreads vectors dealt to the CTA) into
+// accumulator j mod 4, in order, the elements of a vector in order; the CTA's
 // partial sum is the four accumulators added pairwise, then a butterfly over
 // the warp's lanes (the same value in every lane), then the warps' sums in
 // warp order. Every step is a fixed sequence of fp64 additions, so the
 // partial sums do not depend on scheduling.
 template <bool kF32, int VPL>
-__global__ void __launch_bounds__(kSumThreads, 4) quant_sum_kernel(const __grid_constant__ SumArgs a) {
+__global__ void __launch_bounds__(kSumThreads, 1024 / kSumThreads) quant_sum_kernel(const __grid_constant__ SumArgs a) {
   __shared__ double s_red[kSumWarps];
   pdl_wait_primary();  // W and x may be written by earlier work of the stream
   pdl_launch_dependents();
@@ -463,25 +481,31 @@ __global__ void __launch_bounds__(kSumThreads, 4) quant_sum_kernel(const __grid_
     if constexpr (VPL > 0) act_rows<VPL, false>(a.x, r1, a.nv, a.xq, a.sx, r0 + warp, kSumWarps);
     else act_rows_two_pass(a.x, r1, a.nv, a.xq, a.sx, r0 + warp, kSumWarps);
   }
+  // the thread's j-th vector of W: in its CTA's contiguous slice, or in
+  // blocks of kSumThreads vectors dealt to the CTAs in turn
   const int64_t v0 = b * a.per;
-  const int64_t v1 = v0 + a.per < a.nvec ? v0 + a.per : a.nvec;
+  const int64_t vend = kSumInterleave ? a.nvec : (v0 + a.per < a.nvec ? v0 + a.per : a.nvec);
+  auto vec_index = [&](int64_t j) -> int64_t {
+    if constexpr (kSumInterleave) return (b + G * j) * kSumThreads + t;
+    else return v0 + t + kSumThreads * j;
+  };
   double acc[4] = {0.0, 0.0, 0.0, 0.0};
-  int64_t i = v0 + t;
-  for (; i + (kSumUnroll - 1) * kSumThreads < v1; i += kSumUnroll * kSumThreads) {
+  int64_t j = 0;
+  for (; vec_index(j + kSumUnroll - 1) < vend; j += kSumUnroll) {
     uint4 v[kSumUnroll];
 #pragma unroll
-    for (int u = 0; u < kSumUnroll; ++u) v[u] = __ldg(a.W + i + u * kSumThreads);
+    for (int u = 0; u < kSumUnroll; ++u) v[u] = __ldg(a.W + vec_index(j + u));
 #pragma unroll
     for (int u = 0; u < kSumUnroll; ++u) acc[u & 3] = add_abs<kF32>(acc[u & 3], v[u]);
   }
-  if (i < v1) {  // fewer than kSumUnroll vectors left for this thread
+  if (vec_index(j) < vend) {  // fewer than kSumUnroll vectors left for this thread
     uint4 v[kSumUnroll];
 #pragma unroll
     for (int u = 0; u < kSumUnroll; ++u)
-      v[u] = i + u * kSumThreads < v1 ? __ldg(a.W + i + u * kSumThreads) : make_uint4(0u, 0u, 0u, 0u);
+      v[u] = vec_index(j + u) < vend ? __ldg(a.W + vec_index(j + u)) : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
     for (int u = 0; u < kSumUnroll; ++u)
-      if (i + u * kSumThreads < v1) acc[u & 3] = add_abs<kF32>(acc[u & 3], v[u]);
+      if (vec_index(j + u) < vend) acc[u & 3] = add_abs<kF32>(acc[u & 3], v[u]);
   }
   double ts = __dadd_rn(__dadd_rn(acc[0], acc[1]), __dadd_rn(acc[2], acc[3]));
 #pragma unroll
@@ -507,89 +531,167 @@ struct CodeArgs {
   float* gamma_out;
   uint8_t* ws;
   int* err;
+  const uint4* x;   // S2 rows [m_begin, m_begin + M2) of x (M2 = 0: none)
+  int64_t m_begin, M2;
+  int nv;           // K / 8
+  int8_t* xq;
+  float* sx;
 };
 
-// Codes of 128 consecutive 16-byte vectors of W from base (lane l holds
-// vectors l, l + 32, l + 64, l + 96): a group's V lanes combine their bits and
-// its first lane stores the group's word.
-template <bool kF32>
-__device__ __forceinline__ void store_codes(const uint4 (&v)[4], int64_t base, int64_t nvec, uint32_t* out,
-                                            uint32_t key, int lane) {
-  constexpr int V = kF32 ? 4 : 2;
-#pragma unroll
-  for (int u = 0; u < 4; ++u) {
-    const int64_t i = base + lane + 32 * u;
-    const uint32_t word = gather_group_word<kF32>(vec_codes<kF32>(v[u], key), lane);
-    if (i < nvec && (lane & (V - 1)) == 0) out[i / V] = word;
-  }
-}
-
 // Round q of W: 128 consecutive 16-byte vectors, lane l holding vectors
-// 128 q + l + 32 u (u = 0..3); vectors past W (or q past the last round) are
-// zero.
-__device__ __forceinline__ void load_round(const uint4* W, int64_t q, int64_t nrounds, int64_t nvec, int lane,
-                                           uint4 (&v)[4]) {
+// 128 q + l + 32 u (u = 0..3); vectors past W (or q >= q_end) are zero.
+// Rounds below q_full (all 128 vectors inside W) take one address.
+__device__ __forceinline__ void load_round(const uint4* W, int64_t q, int64_t q_end, int64_t q_full, int64_t nvec,
+                                           int lane, uint4 (&v)[4]) {
+  if (q < q_full) {
+    const uint4* p = W + 128 * q + lane;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) v[u] = __ldg(p + 32 * u);
+    return;
+  }
 #pragma unroll
   for (int u = 0; u < 4; ++u) {
     const int64_t i = 128 * q + lane + 32 * u;
-    v[u] = (q < nrounds && i < nvec) ? __ldg(W + i) : make_uint4(0u, 0u, 0u, 0u);
+    v[u] = (q < q_end && i < nvec) ? __ldg(W + i) : make_uint4(0u, 0u, 0u, 0u);
+  }
+}
+
+// Codes of round q (as load_round holds it): a group's V lanes combine their
+// bits and its first lane stores the group's word.
+template <bool kF32>
+__device__ __forceinline__ void store_round(const uint4 (&v)[4], int64_t q, int64_t q_full, int64_t nvec,
+                                            uint32_t* out, uint32_t key, int lane) {
+  constexpr int V = kF32 ? 4 : 2;
+  uint32_t word[4];
+#pragma unroll
+  for (int u = 0; u < 4; ++u) word[u] = gather_group_word<kF32>(vec_codes<kF32>(v[u], key), lane);
+  if ((lane & (V - 1)) != 0) return;
+  if (q < q_full) {
+    uint32_t* p = out + (128 * q + lane) / V;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) p[32 / V * u] = word[u];
+    return;
+  }
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int64_t i = 128 * q + lane + 32 * u;
+    if (i < nvec) out[i / V] = word[u];
   }
 }
 
 // The compare key of the code rule for gamma: the fp32 threshold's bit
-// pattern, or for bf16 the two-halves subtraction bias of codes8_bf16.
+// pattern, or for bf16 the threshold truncated to bf16 in both halves.
 template <bool kF32>
 __device__ __forceinline__ uint32_t code_key(float gamma) {
   const float thr = __double2float_rd(__dmul_rn(static_cast<double>(gamma), 0.5 + 0x1p-25));
   if constexpr (kF32) return __float_as_uint(thr);
   const uint32_t tb = __float_as_uint(thr) >> 16;
-  return (tb | (tb << 16)) + 0x80008000u;
+  return tb | (tb << 16);
+}
+
+// Waits (bounded) until `mode` is set; -1 after the wait limit.
+__device__ __forceinline__ int wait_mode(const volatile int* mode, int* err) {
+  int m = *mode;
+  if (m) return m;
+  const unsigned long long t0 = globaltimer_ns();
+  for (uint32_t i = 1;; ++i) {
+    m = *mode;
+    if (m) return m;
+    if ((i & 255) == 0 && globaltimer_ns() - t0 > kWaitLimitNs) {
+      record_error(err, kDevTimeout);
+      return -1;
+    }
+  }
 }
 
 // Code launch, kCodeThreads threads per CTA, all CTAs resident together (the
-// exact-sum path meets at a grid-wide barrier). Warp g of the grid codes
-// rounds g, g + (warps of the grid), ...; its first round is loaded before
-// gamma is known, every later one while the previous is coded. Warp 0 of
-// every CTA adds the partial sums (lane l: partial sums l, l + 32, ... in
-// order, then a butterfly), so every CTA forms the same gamma. If the
+// exact-sum path meets at a grid-wide barrier). CTA b codes the rounds
+// [b R / G, (b + 1) R / G) of the R rounds of 128 vectors: warp w first takes
+// round w of the range, then claims the next unclaimed one from a counter of
+// the CTA, loading each round while it codes the one before. Warps 1..r of
+// the CTA also quantise the CTA's r token rows (S2 rows the sum launch left),
+// their loads issued first, while warp 0 adds the partial sums (lane l:
+// partial sums l, l + 32, ... in order, then a butterfly, so every CTA forms
+// the same gamma) and the other warps load their first round. If the
 // enclosure of S straddles a rounding boundary of gamma (rare), every warp
-// bins the vectors of its rounds for the exact sum, the CTAs add their bins
-// to the grid's and meet at the barrier, and every CTA forms the exact gamma.
-template <bool kF32>
-__global__ void __launch_bounds__(kCodeThreads) quant_code_kernel(const __grid_constant__ CodeArgs a) {
+// bins rounds w, w + 16, ... of the CTA's range for the exact sum, the CTAs
+// add their bins to the grid's and meet at the barrier, and every CTA forms
+// the exact gamma.
+template <bool kF32, int VPL>
+__global__ void __launch_bounds__(kCodeThreads, 2) quant_code_kernel(const __grid_constant__ CodeArgs a) {
   __shared__ unsigned long long s_bins[256];
-  __shared__ double s_parts[kMaxQuantCtas];
   __shared__ float s_gamma;
-  __shared__ int s_mode;  // 1: gamma known, 2: exact sum needed, -1: gave up
-  pdl_wait_primary();     // the sum launch has completed
+  __shared__ int s_mode;        // 0: not known yet, 1: gamma known, 2: exact sum needed, -1: gave up
+  __shared__ uint32_t s_next;   // next round of the CTA's range to claim (offset from its first)
+  pdl_wait_primary();           // the sum launch has completed
   pdl_launch_dependents();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t nw = static_cast<int64_t>(gridDim.x) * kCodeWarps;
+  const int64_t b = blockIdx.x, G = gridDim.x;
   const int64_t nrounds = (a.nvec + 127) / 128;
-  int64_t r = static_cast<int64_t>(blockIdx.x) * kCodeWarps + warp;
-  uint4 v[4];
-  load_round(a.W, r, nrounds, a.nvec, lane, v);
-  // the partial sums into shared memory, all loads of the CTA at once
-  for (int p = threadIdx.x; p < a.nparts; p += kCodeThreads) s_parts[p] = __ldcg(a.parts + p);
+  const int64_t q0 = b * nrounds / G, q1 = (b + 1) * nrounds / G;
+  const int64_t q_full = a.nvec / 128 < q1 ? a.nvec / 128 : q1;  // rounds wholly inside W
+  const int64_t row = a.m_begin + b * a.M2 / G + warp - 1;
+  const bool has_row = warp >= 1 && row < a.m_begin + (b + 1) * a.M2 / G;
+  int64_t r = q0 + warp;
+  // Warp 0's first loads of partial sums go out before any load of W or x
+  // (which would queue ahead of them); lane l adds partial sums l, l + 32,
+  // ... in order, 8 loads at a time.
+  constexpr int kPartBatch = 8;
+  double pv[kPartBatch];
+  if (warp == 0) {
+#pragma unroll
+    for (int u = 0; u < kPartBatch; ++u) {
+      const int p = 32 * u + lane;
+      pv[u] = p < a.nparts ? __ldcg(a.parts + p) : 0.0;
+    }
+  }
+  if (threadIdx.x == 0) s_mode = 0;
   __syncthreads();
+  // one register array serves the token row (VPL vectors) and then the round
+  // being coded (the first 4)
+  uint4 buf[VPL > 4 ? VPL : 4];
+  uint4(&v)[4] = *reinterpret_cast<uint4(*)[4]>(buf);
+  if (has_row) {
+    if constexpr (VPL > 0) load_row<VPL>(a.x + row * a.nv, a.nv, lane, *reinterpret_cast<uint4(*)[VPL > 0 ? VPL : 1]>(buf));
+  } else {
+    load_round(a.W, r, q1, q_full, a.nvec, lane, v);
+  }
   if (warp == 0) {
     double s = 0.0;
-    for (int p = lane; p < a.nparts; p += 32) s = __dadd_rn(s, s_parts[p]);
+    for (int k0 = 0; k0 < a.nparts; k0 += 32 * kPartBatch) {
+      if (k0 > 0) {
+#pragma unroll
+        for (int u = 0; u < kPartBatch; ++u) {
+          const int p = k0 + 32 * u + lane;
+          pv[u] = p < a.nparts ? __ldcg(a.parts + p) : 0.0;
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kPartBatch; ++u)
+        if (k0 + 32 * u + lane < a.nparts) s = __dadd_rn(s, pv[u]);
+    }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) s = __dadd_rn(s, __shfl_xor_sync(0xffffffffu, s, off));
+    for (int e = lane; e < 256; e += 32) s_bins[e] = 0ull;
+    __syncwarp();
     if (lane == 0) {
       const float glo = gamma_of_sum(__dmul_rd(s, a.enc_lo), a.numel);
       const float ghi = gamma_of_sum(__dmul_ru(s, a.enc_hi), a.numel);
       s_gamma = glo;
-      s_mode = __float_as_uint(glo) == __float_as_uint(ghi) ? 1 : 2;
+      s_next = kCodeWarps;
+      __threadfence_block();
+      *reinterpret_cast<volatile int*>(&s_mode) = __float_as_uint(glo) == __float_as_uint(ghi) ? 1 : 2;
     }
-    for (int e = lane; e < 256; e += 32) s_bins[e] = 0ull;
   }
-  __syncthreads();
-  if (s_mode == 2) {
-    for (int64_t q = r; q < nrounds; q += nw) {
+  if (has_row) {
+    if constexpr (VPL > 0) quant_row<VPL>(*reinterpret_cast<uint4(*)[VPL > 0 ? VPL : 1]>(buf), a.nv, lane, row, a.xq, a.sx);
+    else act_rows_two_pass(a.x, row + 1, a.nv, a.xq, a.sx, row, 1);
+  }
+  int mode = wait_mode(&s_mode, a.err);
+  if (mode == 2) {
+    for (int64_t q = q0 + warp; q < q1; q += kCodeWarps) {
       uint4 w[4];
-      load_round(a.W, q, nrounds, a.nvec, lane, w);
+      load_round(a.W, q, q1, q_full, a.nvec, lane, w);
 #pragma unroll
       for (int u = 0; u < 4; ++u) bin_abs<kF32>(s_bins, w[u]);
     }
@@ -609,17 +711,23 @@ __global__ void __launch_bounds__(kCodeThreads) quant_code_kernel(const __grid_c
       }
     }
     __syncthreads();
-    if (s_mode < 0) return;
+    mode = s_mode;
   }
-  const float gamma = s_gamma;
-  if (blockIdx.x == 0 && threadIdx.x == 0) *a.gamma_out = gamma;
+  if (mode < 0) return;
+  const float gamma = *reinterpret_cast<const volatile float*>(&s_gamma);
+  if (b == 0 && threadIdx.x == 0) *a.gamma_out = gamma;
   const uint32_t key = code_key<kF32>(gamma);
-  for (; r < nrounds; r += nw) {
+  if (has_row) load_round(a.W, r, q1, q_full, a.nvec, lane, v);
+  while (r < q1) {
+    uint32_t c = 0;
+    if (lane == 0) c = atomicAdd(&s_next, 1u);
+    const int64_t rn = q0 + __shfl_sync(0xffffffffu, c, 0);
     uint4 nx[4];
-    load_round(a.W, r + nw, nrounds, a.nvec, lane, nx);
-    store_codes<kF32>(v, 128 * r, a.nvec, a.packed, key, lane);
+    load_round(a.W, rn, q1, q_full, a.nvec, lane, nx);
+    store_round<kF32>(v, r, q_full, a.nvec, a.packed, key, lane);
 #pragma unroll
     for (int u = 0; u < 4; ++u) v[u] = nx[u];
+    r = rn;
   }
 }
 
@@ -656,29 +764,38 @@ cudaError_t launch_s1(const void* W, int64_t N, int64_t K, const void* x, int64_
   constexpr int kElems = kF32 ? 4 : 8;  // elements per 16-byte vector
   static int occ_sum[64] = {}, occ_code[64] = {};
   const int64_t sms = device_sm_count();
+  const int64_t nvec = N * K / kElems;
+  // code launch: no more CTAs than can be resident at once (the exact-sum
+  // barrier), and no more warps than rounds of 128 vectors; it takes up to
+  // kCodeRowsPerCta token rows per CTA (the rest go to the sum launch)
+  const int64_t nrounds = (nvec + 127) / 128;
+  const int64_t cap2 = sms * blocks_per_sm(quant_code_kernel<kF32, VPL>, kCodeThreads, occ_code);
+  const int64_t G2 = std::max<int64_t>(1, std::min<int64_t>(cap2, (nrounds + kCodeWarps - 1) / kCodeWarps));
+  const int64_t M2 = std::min<int64_t>(M, G2 * kCodeRowsPerCta), M1 = M - M2;
+
   SumArgs sa{};
   sa.W = static_cast<const uint4*>(W);
-  sa.nvec = N * K / kElems;
+  sa.nvec = nvec;
   sa.ws = ws;
   sa.parts = reinterpret_cast<double*>(ws + kWsParts);
   sa.x = static_cast<const uint4*>(x);
-  sa.M = M;
+  sa.M = M1;
   sa.nv = static_cast<int>(K / 8);
   sa.xq = xq;
   sa.sx = sx;
   // sum launch: every SM filled (at most kMaxQuantCtas partial sums), fewer
-  // CTAs only when W has fewer than 2048 vectors per CTA and the tokens fewer
+  // CTAs only when W has fewer than 2048 vectors per CTA and its tokens fewer
   // than one row per warp
   const int64_t cap1 =
       std::min<int64_t>(sms * blocks_per_sm(quant_sum_kernel<kF32, VPL>, kSumThreads, occ_sum), kMaxQuantCtas);
-  const int64_t want1 = std::max<int64_t>((sa.nvec + kSumThreads * kSumUnroll - 1) / (kSumThreads * kSumUnroll),
-                                          (M + kSumWarps - 1) / kSumWarps);
+  const int64_t want1 = std::max<int64_t>((nvec + kSumThreads * kSumUnroll - 1) / (kSumThreads * kSumUnroll),
+                                          (M1 + kSumWarps - 1) / kSumWarps);
   const int64_t G1 = std::max<int64_t>(1, std::min(want1, cap1));
-  sa.per = (sa.nvec + G1 - 1) / G1;
+  sa.per = (nvec + G1 - 1) / G1;
 
   CodeArgs ca{};
   ca.W = sa.W;
-  ca.nvec = sa.nvec;
+  ca.nvec = nvec;
   ca.parts = sa.parts;
   ca.nparts = static_cast<int>(G1);
   ca.numel = static_cast<double>(N * K);
@@ -686,11 +803,12 @@ cudaError_t launch_s1(const void* W, int64_t N, int64_t K, const void* x, int64_
   ca.gamma_out = gamma;
   ca.ws = ws;
   ca.err = err;
-  // code launch: no more CTAs than can be resident at once (the exact-sum
-  // barrier), and no more warps than rounds of 128 vectors
-  const int64_t nrounds = (sa.nvec + 127) / 128;
-  const int64_t cap2 = sms * blocks_per_sm(quant_code_kernel<kF32>, kCodeThreads, occ_code);
-  const int64_t G2 = std::max<int64_t>(1, std::min<int64_t>(cap2, (nrounds + kCodeWarps - 1) / kCodeWarps));
+  ca.x = sa.x;
+  ca.m_begin = M1;
+  ca.M2 = M2;
+  ca.nv = sa.nv;
+  ca.xq = xq;
+  ca.sx = sx;
   // Enclosure of S around the fp64 sum. Every |w| passes through at most d
   // roundings: its accumulator's sequential adds (kElems per vector, at most
   // ceil(nj / 4) vectors of the thread's nj), the two levels joining the four
@@ -700,7 +818,8 @@ cudaError_t launch_s1(const void* W, int64_t N, int64_t K, const void* x, int64_
   // partial sum, and with all terms >= 0 every partial sum is at most
   // S (1 + 2^-30), so |fp64 sum - S| <= d 2^-53 (1 + 2^-30) S; e = d 2^-52
   // (8 roundings to spare) covers S on both sides.
-  const int64_t nj = (sa.per + kSumThreads - 1) / kSumThreads;
+  const int64_t nj = kSumInterleave ? ((nvec + kSumThreads - 1) / kSumThreads + G1 - 1) / G1
+                                    : (sa.per + kSumThreads - 1) / kSumThreads;  // vectors per thread
   const double d = static_cast<double>(kElems) * static_cast<double>((nj + 3) / 4) + 2 + 5 + kSumWarps +
                    static_cast<double>((G1 + 31) / 32) + 5 + 8;
   const double e = std::ldexp(d, -52);
@@ -709,7 +828,7 @@ cudaError_t launch_s1(const void* W, int64_t N, int64_t K, const void* x, int64_
 
   cudaError_t st = launch_pdl(quant_sum_kernel<kF32, VPL>, dim3(static_cast<unsigned>(G1)), dim3(kSumThreads), 0, s, sa);
   if (st != cudaSuccess) return st;
-  return launch_pdl(quant_code_kernel<kF32>, dim3(static_cast<unsigned>(G2)), dim3(kCodeThreads), 0, s, ca);
+  return launch_pdl(quant_code_kernel<kF32, VPL>, dim3(static_cast<unsigned>(G2)), dim3(kCodeThreads), 0, s, ca);
 }
 
 template <int VPL>
