@@ -932,129 +932,357 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 }
 
 // ---------------------------------------------------------------- forward for few tokens
-// With a handful of tokens the forward is bound by reading the packed codes
-// once (N K / 4 bytes), not by arithmetic, and the tensor-core tiles would
-// leave most SMs idle. Used for M <= 8, where it measured faster than the
-// tile kernel (at the up-projection weight: 10.2 us at M = 1 and 16.4 us at
-// M = 8 against 19.5 us; beyond M = 8 the tile kernel wins). A CTA takes 32 output features (lane = feature n) and all M
-// tokens; its 8 warps split K into contiguous runs of 32-code groups. The tokens'
-// INT8 rows sit in shared memory (read with broadcast loads), the codes are
-// expanded to int8 with the same bit arithmetic as the GEMM rebuild, and
-// __dp4a keeps the sums exact in INT32. The warps' partial sums are added in
-// a fixed order, and y = bf16_rn(fp32(acc) * fp32(s_x[m] * gamma)) as in the
-// GEMM epilogue.
-constexpr int kDecodeWarps = 8;
-constexpr int kDecodeMaxM = 8;
+// With up to 16 tokens the forward is bound by reading the packed codes once
+// (N K / 4 bytes), not by arithmetic, and the tensor-core tiles would leave
+// most SMs idle. Warp w takes rows_per_warp consecutive output features n
+// (rows of the packed codes); for each row its lanes read consecutive
+// chunks of the row (16 bytes = 64 codes, or 8 bytes when K % 64 != 0), so
+// every load instruction of the warp covers contiguous bytes, and each lane
+// forms the INT32 partial dot products of its chunks with all kM tokens
+// (codes expanded to int8 as in the GEMM rebuild, __dp4a). The tokens' INT8
+// rows sit in shared memory with a 16-byte pad after every chunk's bytes, so
+// the lanes' 16-byte loads fall in distinct banks. A row's kM sums are then
+// reduced over the warp by recursive halving (each step exchanges half of
+// the remaining sums, so every lane ends with the total of one token) -- all
+// integer adds, exact in any order -- and y = bf16_rn(fp32(acc) *
+// fp32(s_x[m] * gamma)) as in the GEMM epilogue. Before its dependency wait
+// every warp asks L2 to prefetch its rows' bytes: a prefetch only warms L2,
+// which stays coherent with whatever the kernel before writes, so it is safe
+// before the wait and lets the code fetch overlap the previous launch.
+constexpr int kFewWarps = 8;
+constexpr int kFewMaxM = 16;
+constexpr int kFewWarpsPerSm = 16;  // target resident warps per SM when N allows
 
-template <int kMaxM>
-__global__ void __launch_bounds__(32 * kDecodeWarps) decode_forward_kernel(
+__device__ __forceinline__ void prefetch_l2_bulk(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
+// Sums v[0..kM) over the warp: on return lane l holds the total of token
+// few_token_of<kM>(l) (every lane of a group of 32 / kM lanes the same).
+template <int kM>
+__device__ __forceinline__ int32_t few_reduce(int32_t (&v)[kM], int lane) {
+  int off = 16;
+#pragma unroll
+  for (int w = kM / 2; w >= 1; w /= 2, off /= 2) {
+    const bool up = (lane & off) != 0;
+#pragma unroll
+    for (int i = 0; i < w; ++i) {
+      const int32_t send = up ? v[i] : v[i + w];
+      const int32_t keep = up ? v[i + w] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+    }
+  }
+  int32_t s = v[0];
+#pragma unroll
+  for (int o = off; o >= 1; o /= 2) s += __shfl_xor_sync(0xffffffffu, s, o);
+  return s;
+}
+
+template <int kM>
+__device__ __forceinline__ int few_token_of(int lane) {
+  int m = 0, off = 16;
+#pragma unroll
+  for (int w = kM / 2; w >= 1; w /= 2, off /= 2) m += (lane & off) ? w : 0;
+  return m;
+}
+
+// Lanes whose bits below the last halving step are zero write the results.
+template <int kM>
+__device__ __forceinline__ bool few_writer(int lane) {
+  constexpr int kLow = 32 / kM;  // lanes holding one token's total
+  return (lane & (kLow - 1)) == 0;
+}
+
+template <int kM, int kChunk>
+__global__ void __launch_bounds__(32 * kFewWarps) few_forward_kernel(
     const int8_t* __restrict__ xq, const float* __restrict__ sx, const uint8_t* __restrict__ packed,
-    const float* __restrict__ gamma_ptr, int M, int N, int K, __nv_bfloat16* __restrict__ y,
+    const float* __restrict__ gamma_ptr, int M, int N, int K, int rows_per_warp, __nv_bfloat16* __restrict__ y,
     int32_t* __restrict__ debug_acc) {
-  extern __shared__ __align__(16) uint8_t s_q[];  // [kMaxM][K] int8, then the warps' partial sums
+  extern __shared__ __align__(16) uint8_t s_x[];  // [kM][cpr] chunks of 4 kChunk bytes, each + 16 pad
+  constexpr int kPitch = 4 * kChunk + 16;
+  constexpr int kWords = kChunk / 4;  // 32-bit code words per chunk (16 codes each)
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int row_bytes = K / 4, cpr = row_bytes / kChunk;
+  const int64_t n0 = (static_cast<int64_t>(blockIdx.x) * kFewWarps + warp) * rows_per_warp;
+  const int nrows = n0 < N ? static_cast<int>(N - n0 < rows_per_warp ? N - n0 : rows_per_warp) : 0;
+  if (kChunk == 16 && lane == 0 && nrows > 0)
+    prefetch_l2_bulk(packed + n0 * row_bytes, static_cast<uint32_t>(nrows) * row_bytes);
   pdl_wait_primary();
   pdl_launch_dependents();
-  const int lane = threadIdx.x & 31;
-  const int warp = threadIdx.x >> 5;
-  // tokens' codes into shared memory (rows of K bytes, K % 32 == 0); rows
-  // M .. kMaxM-1 are zero, so every token slot is summed without a branch
-  const int qvec = M * K / 16, qall = kMaxM * K / 16;
-  for (int i = threadIdx.x; i < qall; i += blockDim.x)
-    reinterpret_cast<uint4*>(s_q)[i] =
-        i < qvec ? __ldg(reinterpret_cast<const uint4*>(xq) + i) : make_uint4(0u, 0u, 0u, 0u);
+  // the tokens' rows into shared memory (rows M .. kM-1 zero)
+  const int pieces = K / 16;  // 16-byte pieces per token row
+  for (int i = threadIdx.x; i < kM * pieces; i += blockDim.x) {
+    const int m = i / pieces, q = i - m * pieces;
+    const int c = q / kWords, t = q - c * kWords;
+    const uint4 v = m < M ? __ldg(reinterpret_cast<const uint4*>(xq + static_cast<int64_t>(m) * K) + q)
+                          : make_uint4(0u, 0u, 0u, 0u);
+    *reinterpret_cast<uint4*>(s_x + (m * cpr + c) * kPitch + 16 * t) = v;
+  }
   __syncthreads();
-
-  const int n = blockIdx.x * 32 + lane;
-  const bool row_ok = n < N;
-  const uint2* row = reinterpret_cast<const uint2*>(packed + static_cast<int64_t>(row_ok ? n : 0) * (K / 4));
-  int32_t acc[kMaxM];
+  if (nrows == 0) return;
+  const float gamma = __ldg(gamma_ptr);
+  const uint32_t sbase = smem_u32(s_x);
+  const int me = few_token_of<kM>(lane);
+  const bool writer = few_writer<kM>(lane) && me < M;
+  const float scale = writer ? __fmul_rn(__ldg(sx + me), gamma) : 0.0f;
+  // kRows rows at a time, so that every token chunk read from shared memory
+  // serves kRows rows; kSlots chunks per row and lane in flight
+  constexpr int kRows = kM >= 16 ? 2 : 4;
+  constexpr int kSlots = 8 / kRows;
+  for (int g = 0; g < nrows; g += kRows) {
+    int32_t acc[kRows][kM];
 #pragma unroll
-  for (int m = 0; m < kMaxM; ++m) acc[m] = 0;
-  // each warp takes a contiguous run of 32-code groups (8 bytes each) and
-  // each lane loads its row's groups kBatch at a time, the next batch while
-  // the current one is summed
-  constexpr int kBatch = 8;
-  const int groups = K / 32;
-  const int gpw = (groups + kDecodeWarps - 1) / kDecodeWarps;
-  const int g_begin = warp * gpw;
-  const int g_end = min(g_begin + gpw, groups);
-  uint2 cur[kBatch];
+    for (int r = 0; r < kRows; ++r)
 #pragma unroll
-  for (int b = 0; b < kBatch; ++b)
-    cur[b] = (row_ok && g_begin + b < g_end) ? __ldg(row + g_begin + b) : make_uint2(0u, 0u);
-  for (int g = g_begin; g < g_end; g += kBatch) {
-    uint2 nxt[kBatch];
+      for (int m = 0; m < kM; ++m) acc[r][m] = 0;
+    for (int c0 = 0; c0 < cpr; c0 += 32 * kSlots) {
+      uint32_t words[kRows][kSlots][kWords];
 #pragma unroll
-    for (int b = 0; b < kBatch; ++b)
-      nxt[b] = (row_ok && g + kBatch + b < g_end) ? __ldg(row + g + kBatch + b) : make_uint2(0u, 0u);
+      for (int r = 0; r < kRows; ++r) {
+        const uint8_t* row = packed + (n0 + g + r) * row_bytes;
 #pragma unroll
-    for (int b = 0; b < kBatch; ++b) {
-      if (g + b >= g_end) break;
-      const uint4 c0 = codes16_to_s8(cur[b].x), c1 = codes16_to_s8(cur[b].y);
-      const int32_t c[8] = {static_cast<int32_t>(c0.x), static_cast<int32_t>(c0.y), static_cast<int32_t>(c0.z),
-                            static_cast<int32_t>(c0.w), static_cast<int32_t>(c1.x), static_cast<int32_t>(c1.y),
-                            static_cast<int32_t>(c1.z), static_cast<int32_t>(c1.w)};
-      const uint32_t qbase = smem_u32(s_q) + (g + b) * 32;
+        for (int u = 0; u < kSlots; ++u) {
+          const int c = c0 + 32 * u + lane;
+          const bool ok = g + r < nrows && c < cpr;
+          if constexpr (kChunk == 16) {
+            const uint4 w = ok ? __ldg(reinterpret_cast<const uint4*>(row) + c) : make_uint4(0u, 0u, 0u, 0u);
+            words[r][u][0] = w.x; words[r][u][1] = w.y; words[r][u][2] = w.z; words[r][u][3] = w.w;
+          } else {
+            const uint2 w = ok ? __ldg(reinterpret_cast<const uint2*>(row) + c) : make_uint2(0u, 0u);
+            words[r][u][0] = w.x; words[r][u][1] = w.y;
+          }
+        }
+      }
 #pragma unroll
-      for (int m = 0; m < kMaxM; ++m) {
-        const uint4 qa = ld_shared_v4(qbase + m * K);
-        const uint4 qb = ld_shared_v4(qbase + m * K + 16);
-        // two independent chains, added at the end (integer sums are exact)
-        int32_t a = __dp4a(c[0], static_cast<int32_t>(qa.x), 0);
-        int32_t b = __dp4a(c[4], static_cast<int32_t>(qb.x), 0);
-        a = __dp4a(c[1], static_cast<int32_t>(qa.y), a);
-        b = __dp4a(c[5], static_cast<int32_t>(qb.y), b);
-        a = __dp4a(c[2], static_cast<int32_t>(qa.z), a);
-        b = __dp4a(c[6], static_cast<int32_t>(qb.z), b);
-        a = __dp4a(c[3], static_cast<int32_t>(qa.w), a);
-        b = __dp4a(c[7], static_cast<int32_t>(qb.w), b);
-        acc[m] += a + b;
+      for (int u = 0; u < kSlots; ++u) {
+        if (c0 + 32 * u >= cpr) break;  // no lane of the warp has chunk slot u
+        const int c = c0 + 32 * u + lane;
+        if (c < cpr) {
+#pragma unroll
+          for (int t = 0; t < kWords; ++t) {
+            uint4 q[kRows];
+#pragma unroll
+            for (int r = 0; r < kRows; ++r) q[r] = codes16_to_s8(words[r][u][t]);
+            const uint32_t xa = sbase + c * kPitch + 16 * t;
+#pragma unroll
+            for (int m = 0; m < kM; ++m) {
+              const uint4 xv = ld_shared_v4(xa + m * cpr * kPitch);
+#pragma unroll
+              for (int r = 0; r < kRows; ++r) {
+                int32_t a = __dp4a(static_cast<int32_t>(q[r].x), static_cast<int32_t>(xv.x), acc[r][m]);
+                a = __dp4a(static_cast<int32_t>(q[r].y), static_cast<int32_t>(xv.y), a);
+                a = __dp4a(static_cast<int32_t>(q[r].z), static_cast<int32_t>(xv.z), a);
+                acc[r][m] = __dp4a(static_cast<int32_t>(q[r].w), static_cast<int32_t>(xv.w), a);
+              }
+            }
+          }
+        }
       }
     }
 #pragma unroll
-    for (int b = 0; b < kBatch; ++b) cur[b] = nxt[b];
-  }
-  // fixed-order sum over the warps: warps 1.. park their sums, warp 0 adds
-  int32_t* red = reinterpret_cast<int32_t*>(s_q + kMaxM * K);  // [warp-1][m][32]
-  if (warp > 0) {
-#pragma unroll
-    for (int m = 0; m < kMaxM; ++m)
-      if (m < M) red[((warp - 1) * kMaxM + m) * 32 + lane] = acc[m];
-  }
-  __syncthreads();
-  if (warp != 0) return;
-  const float gamma = __ldg(gamma_ptr);
-#pragma unroll
-  for (int m = 0; m < kMaxM; ++m) {
-    if (m < M) {
-      int32_t a = acc[m];
-      for (int w = 1; w < kDecodeWarps; ++w) a += red[((w - 1) * kMaxM + m) * 32 + lane];
-      if (row_ok) {
-        const int64_t off = static_cast<int64_t>(m) * N + n;
-        y[off] = __float2bfloat16_rn(__fmul_rn(static_cast<float>(a), __fmul_rn(__ldg(sx + m), gamma)));
-        if (debug_acc) debug_acc[off] = a;
+    for (int r = 0; r < kRows; ++r) {
+      const int32_t total = few_reduce<kM>(acc[r], lane);
+      if (writer && g + r < nrows) {
+        const int64_t off = static_cast<int64_t>(me) * N + n0 + g + r;
+        y[off] = __float2bfloat16_rn(__fmul_rn(static_cast<float>(total), scale));
+        if (debug_acc) debug_acc[off] = total;
       }
     }
   }
 }
 
-template <int kMaxM>
-cudaError_t launch_decode(const int8_t* xq, const float* sx, const uint8_t* packed, const float* gamma, int M, int N,
-                          int K, void* y, int32_t* debug_acc, cudaStream_t s) {
-  const size_t smem = static_cast<size_t>(kMaxM) * K + static_cast<size_t>(kDecodeWarps - 1) * kMaxM * 32 * 4;
+template <int kM, int kChunk>
+cudaError_t launch_few(const int8_t* xq, const float* sx, const uint8_t* packed, const float* gamma, int M, int N,
+                       int K, void* y, int32_t* debug_acc, cudaStream_t s) {
+  const int cpr = K / 4 / kChunk;
+  const size_t smem = static_cast<size_t>(kM) * cpr * (4 * kChunk + 16);
   static int configured[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
-  const int max_smem = kSmemLimit;
   if (dev >= 0 && dev < 64 && !configured[dev]) {
-    cudaError_t e =
-        cudaFuncSetAttribute(decode_forward_kernel<kMaxM>, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem);
+    cudaError_t e = cudaFuncSetAttribute(few_forward_kernel<kM, kChunk>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         kSmemLimit);
     if (e != cudaSuccess) return e;
     configured[dev] = 1;
   }
-  const unsigned grid = static_cast<unsigned>((N + 31) / 32);
-  cudaError_t e = launch_pdl(decode_forward_kernel<kMaxM>, dim3(grid), dim3(32 * kDecodeWarps), smem, s, xq, sx,
-                             packed, gamma, M, N, K, static_cast<__nv_bfloat16*>(y), debug_acc);
+  // enough warps to fill every SM when N allows, each with whole rows
+  constexpr int kRows = kM >= 16 ? 2 : 4;  // rows a warp takes at a time
+  const int64_t target = static_cast<int64_t>(device_sm_count()) * kFewWarpsPerSm;
+  int rpw = static_cast<int>(std::max<int64_t>(1, (N + target - 1) / target));
+  rpw = (rpw + kRows - 1) / kRows * kRows;
+  const int64_t warps = (N + rpw - 1) / rpw;
+  const unsigned grid = static_cast<unsigned>((warps + kFewWarps - 1) / kFewWarps);
+  cudaError_t e = launch_pdl(few_forward_kernel<kM, kChunk>, dim3(grid), dim3(32 * kFewWarps), smem, s, xq, sx,
+                             packed, gamma, M, N, K, rpw, static_cast<__nv_bfloat16*>(y), debug_acc);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+// Smallest power-of-two token count >= M that the few-token kernel takes at
+// this K (its shared memory holds kM token rows), else 0.
+int few_slots(int64_t M, int64_t K) {
+  if (M > kFewMaxM) return 0;
+  int slots = 1;
+  while (slots < M) slots *= 2;
+  const int chunk = (K % 64) == 0 ? 16 : 8;
+  const size_t smem = static_cast<size_t>(slots) * (K / 4 / chunk) * (4 * chunk + 16);
+  return smem <= static_cast<size_t>(kSmemLimit) ? slots : 0;
+}
+
+template <int kChunk>
+cudaError_t launch_few_chunk(int slots, const int8_t* xq, const float* sx, const uint8_t* packed, const float* gamma,
+                             int M, int N, int K, void* y, int32_t* debug_acc, cudaStream_t s) {
+  switch (slots) {
+    case 1: return launch_few<1, kChunk>(xq, sx, packed, gamma, M, N, K, y, debug_acc, s);
+    case 2: return launch_few<2, kChunk>(xq, sx, packed, gamma, M, N, K, y, debug_acc, s);
+    case 4: return launch_few<4, kChunk>(xq, sx, packed, gamma, M, N, K, y, debug_acc, s);
+    case 8: return launch_few<8, kChunk>(xq, sx, packed, gamma, M, N, K, y, debug_acc, s);
+    default: return launch_few<16, kChunk>(xq, sx, packed, gamma, M, N, K, y, debug_acc, s);
+  }
+}
+
+// Few tokens with K % 64 == 0: the same products on the tensor cores' warp
+// MMA (m16n8k32, s8 x s8 -> s32), so that a code is expanded to int8 once
+// for all the tokens instead of once per token and lane. A warp takes a tile
+// of 16 output features (rows of the packed codes) and a slice of K in blocks
+// of 256 codes; lane (g, t) (g = lane / 4, t = lane % 4) reads the 16 bytes
+// [16 t, 16 t + 16) of a block of rows g and g + 8 and the 64 matching INT8
+// values of tokens g (and g + 8). The MMA's k index 4 t + j (16 + 4 t + j)
+// stands for the block's code 64 t + 16 w + j (64 t + 16 w + 4 + j) in its
+// step 2 w and 64 t + 16 w + 8 + j (... + 12 + j) in step 2 w + 1: the
+// mapping depends on t and j only, so A and B agree on it and the sum over k
+// is the dot product (INT32 sums are exact in any order). The CTA's warps
+// take consecutive K slices of one tile and their sums are added in shared
+// memory. Tensor cores of this form (not tcgen05) suit a launch this small:
+// no tensor memory to allocate, and the work per SM is a few hundred MMAs.
+constexpr int kFewMmaMaxWarps = 8;
+
+__device__ __forceinline__ void mma_s8_16832(int32_t (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                             uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+template <int kNT>  // tiles of 8 tokens: 1 (M <= 8) or 2 (M <= 16)
+__global__ void __launch_bounds__(32 * kFewMmaMaxWarps) few_mma_forward_kernel(
+    const int8_t* __restrict__ xq, const float* __restrict__ sx, const uint8_t* __restrict__ packed,
+    const float* __restrict__ gamma_ptr, int M, int N, int K, __nv_bfloat16* __restrict__ y,
+    int32_t* __restrict__ debug_acc) {
+  __shared__ int32_t s_red[kFewMmaMaxWarps - 1][4 * kNT][32];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, S = blockDim.x >> 5;
+  const int g = lane >> 2, t = lane & 3;
+  const int row_bytes = K / 4;
+  const int nblocks = (K + 255) / 256;
+  const int b0 = warp * nblocks / S, b1 = (warp + 1) * nblocks / S;  // this warp's blocks
+  const int64_t n_base = static_cast<int64_t>(blockIdx.x) * 16;
+  // L2 prefetch of the slice of the tile's rows (safe before the wait)
+  if (lane < 16 && n_base + lane < N && b1 > b0) {
+    const int lo = b0 * 64, hi = b1 * 64 < row_bytes ? b1 * 64 : row_bytes;
+    prefetch_l2_bulk(packed + (n_base + lane) * row_bytes + lo, static_cast<uint32_t>(hi - lo));
+  }
+  pdl_wait_primary();
+  pdl_launch_dependents();
+  const bool r0ok = n_base + g < N, r1ok = n_base + g + 8 < N;
+  const uint8_t* row0 = packed + (n_base + g) * row_bytes;
+  const uint8_t* row1 = packed + (n_base + g + 8) * row_bytes;
+  // the epilogue's scales, fetched now (warp 0 writes: tokens 8 j + 2 t + {0, 1})
+  float scale[kNT][2];
+  if (warp == 0) {
+    const float gamma = __ldg(gamma_ptr);
+#pragma unroll
+    for (int j = 0; j < kNT; ++j)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int m = 8 * j + 2 * t + h;
+        scale[j][h] = m < M ? __fmul_rn(__ldg(sx + m), gamma) : 0.0f;
+      }
+  }
+  int32_t acc[kNT][4];
+#pragma unroll
+  for (int j = 0; j < kNT; ++j)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) acc[j][i] = 0;
+  // block b's operands of this lane: codes of rows g and g + 8, tokens' INT8
+  struct Operands {
+    uint4 c0, c1, x[kNT][4];
+  };
+  auto load_block = [&](int b, Operands& o) {
+    const int off = b * 64 + 16 * t;  // this lane's 16 bytes of the block (64 codes)
+    const bool in = b < b1 && off < row_bytes;
+    o.c0 = (in && r0ok) ? __ldg(reinterpret_cast<const uint4*>(row0 + off)) : make_uint4(0u, 0u, 0u, 0u);
+    o.c1 = (in && r1ok) ? __ldg(reinterpret_cast<const uint4*>(row1 + off)) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+    for (int j = 0; j < kNT; ++j) {
+      const int m = 8 * j + g;
+      const uint4* xr = reinterpret_cast<const uint4*>(xq + static_cast<int64_t>(m) * K + 4 * off);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) o.x[j][u] = (in && m < M) ? __ldg(xr + u) : make_uint4(0u, 0u, 0u, 0u);
+    }
+  };
+  // one token tile: the next block's loads are in flight while this one is
+  // multiplied; two tiles: loaded one block at a time (registers)
+  Operands cur, nxt;
+  load_block(b0, cur);
+  for (int b = b0; b < b1; ++b) {
+    if constexpr (kNT == 1) load_block(b + 1, nxt);
+    const uint32_t w0[4] = {cur.c0.x, cur.c0.y, cur.c0.z, cur.c0.w}, w1[4] = {cur.c1.x, cur.c1.y, cur.c1.z, cur.c1.w};
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      const uint4 qa = codes16_to_s8(w0[w]), qb = codes16_to_s8(w1[w]);
+#pragma unroll
+      for (int j = 0; j < kNT; ++j) {
+        mma_s8_16832(acc[j], qa.x, qb.x, qa.y, qb.y, cur.x[j][w].x, cur.x[j][w].y);
+        mma_s8_16832(acc[j], qa.z, qb.z, qa.w, qb.w, cur.x[j][w].z, cur.x[j][w].w);
+      }
+    }
+    if constexpr (kNT == 1) cur = nxt;
+    else load_block(b + 1, cur);
+  }
+  // the warps' sums, added by warp 0
+  if (warp > 0) {
+#pragma unroll
+    for (int j = 0; j < kNT; ++j)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) s_red[warp - 1][4 * j + i][lane] = acc[j][i];
+  }
+  __syncthreads();
+  if (warp != 0) return;
+  for (int w = 1; w < S; ++w)
+#pragma unroll
+    for (int j = 0; j < kNT; ++j)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) acc[j][i] += s_red[w - 1][4 * j + i][lane];
+  // acc[j][i]: feature n_base + g (+8 for i >= 2), token 8 j + 2 t + (i & 1)
+#pragma unroll
+  for (int j = 0; j < kNT; ++j)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int m = 8 * j + 2 * t + (i & 1);
+      const int64_t n = n_base + g + (i >= 2 ? 8 : 0);
+      if (m < M && n < N) {
+        const int64_t o = static_cast<int64_t>(m) * N + n;
+        y[o] = __float2bfloat16_rn(__fmul_rn(static_cast<float>(acc[j][i]), scale[j][i & 1]));
+        if (debug_acc) debug_acc[o] = acc[j][i];
+      }
+    }
+}
+
+template <int kNT>
+cudaError_t launch_few_mma(const int8_t* xq, const float* sx, const uint8_t* packed, const float* gamma, int M,
+                           int N, int K, void* y, int32_t* debug_acc, cudaStream_t s) {
+  // warps per tile (a power of two, at most one per block of 256 codes):
+  // enough warps to fill every SM, while leaving room for the next launch's
+  // CTAs (whose L2 prefetch then overlaps this launch)
+  const int64_t tiles = (N + 15) / 16;
+  const int nblocks = (K + 255) / 256;
+  const int64_t target = static_cast<int64_t>(device_sm_count()) * kFewWarpsPerSm;
+  int S = 1;
+  while (S < kFewMmaMaxWarps && S < nblocks && tiles * S < target) S *= 2;
+  cudaError_t e = launch_pdl(few_mma_forward_kernel<kNT>, dim3(static_cast<unsigned>(tiles)), dim3(32 * S), 0, s, xq,
+                             sx, packed, gamma, M, N, K, static_cast<__nv_bfloat16*>(y), debug_acc);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
@@ -1274,18 +1502,14 @@ cudaError_t launch_forward(const int8_t* xq, const float* sx, const uint8_t* w_p
   if (M == 0 || N == 0) return cudaSuccess;
   // few tokens: the packed codes' bandwidth, not the tensor cores, bounds the
   // forward (the tokens' codes must fit in shared memory)
-  if (M <= kDecodeMaxM) {
-    int slots = 1;
-    while (slots < M) slots *= 2;
-    if (static_cast<size_t>(slots) * K + static_cast<size_t>(kDecodeWarps - 1) * slots * 32 * 4 <= kSmemLimit) {
-      const int m = static_cast<int>(M), nn = static_cast<int>(N), kk = static_cast<int>(K);
-      switch (slots) {
-        case 1: return launch_decode<1>(xq, sx, w_packed, gamma, m, nn, kk, y, debug_acc, s);
-        case 2: return launch_decode<2>(xq, sx, w_packed, gamma, m, nn, kk, y, debug_acc, s);
-        case 4: return launch_decode<4>(xq, sx, w_packed, gamma, m, nn, kk, y, debug_acc, s);
-        default: return launch_decode<8>(xq, sx, w_packed, gamma, m, nn, kk, y, debug_acc, s);
-      }
-    }
+  if (M <= kFewMaxM && (K % 64) == 0) {
+    const int m = static_cast<int>(M), nn = static_cast<int>(N), kk = static_cast<int>(K);
+    return M <= 8 ? launch_few_mma<1>(xq, sx, w_packed, gamma, m, nn, kk, y, debug_acc, s)
+                  : launch_few_mma<2>(xq, sx, w_packed, gamma, m, nn, kk, y, debug_acc, s);
+  }
+  if (const int slots = few_slots(M, K)) {
+    const int m = static_cast<int>(M), nn = static_cast<int>(N), kk = static_cast<int>(K);
+    return launch_few_chunk<8>(slots, xq, sx, w_packed, gamma, m, nn, kk, y, debug_acc, s);
   }
   static const int kCands[3] = {256, 192, 128};
   const int npairs = resident_pairs<Family::Fwd, 256>();

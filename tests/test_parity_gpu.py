@@ -418,7 +418,7 @@ def test_quantize_fused_matches_separate(M, N, K, w_dtype):
 
 @pytest.mark.parametrize("M", [1, 2, 3, 5, 8, 9, 16])
 def test_forward_few_tokens(M):
-    """Forward with few tokens on the up-projection weight (M <= 8: the
+    """Forward with few tokens on the up-projection weight (M <= 16: the
     code-bandwidth kernel, every token-slot count; above: the tile kernel):
     INT32 sums and y bit-exact."""
     bl = _bl()
@@ -441,3 +441,26 @@ def test_forward_few_tokens(M):
     y_o = ref.round_to_bf16_bits(ref.forward_output(acc_o, sx, gamma))
     np.testing.assert_array_equal(bits(bufs.y), y_o)
     np.testing.assert_array_equal(bits(y2), y_o)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("M,N,K", [(3, 2560, 6912), (16, 2560, 6912), (5, 1000, 96), (16, 333, 160),
+                                   (1, 7, 32), (9, 2049, 4096)])
+def test_forward_few_tokens_shapes(M, N, K):
+    """Few-token forward at other shapes: the down-projection weight (long
+    rows), K % 64 != 0 (8-byte code chunks), N not a multiple of the rows a
+    warp takes, a single short row: INT32 sums and y bit-exact."""
+    bl = _bl()
+    x, w, _ = make_inputs(M, K, N, seed=60 + M + K)
+    bufs = bl.StepBuffers.allocate(M, N, K)
+    acc = torch.empty((M, N), dtype=torch.int32, device="cuda")
+    bl.bl_quantize_weight(w.cuda(), bufs.w_packed, bufs.gamma, bufs.workspace)
+    bl.bl_quantize_act(x.cuda(), bufs.xq, bufs.sx)
+    bl.bl_forward(bufs.xq, bufs.sx, bufs.w_packed, bufs.gamma, bufs.y, acc)
+    torch.cuda.synchronize()
+    assert bl.bl_get_last_error() == 0
+    codes, gamma = ref.ternarize(ref.bf16_bits_to_f32(bits(w)))
+    q, sx = ref.quantize_activations(ref.bf16_bits_to_f32(bits(x)))
+    acc_o = ref.forward_accumulate(q, codes)
+    np.testing.assert_array_equal(acc.cpu().numpy(), acc_o)
+    np.testing.assert_array_equal(bits(bufs.y), ref.round_to_bf16_bits(ref.forward_output(acc_o, sx, gamma)))
