@@ -934,21 +934,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 // ---------------------------------------------------------------- forward for few tokens
 // With up to 16 tokens the forward is bound by reading the packed codes once
 // (N K / 4 bytes), not by arithmetic, and the tensor-core tiles would leave
-// most SMs idle. Warp w takes rows_per_warp consecutive output features n
-// (rows of the packed codes); for each row its lanes read consecutive
-// chunks of the row (16 bytes = 64 codes, or 8 bytes when K % 64 != 0), so
-// every load instruction of the warp covers contiguous bytes, and each lane
-// forms the INT32 partial dot products of its chunks with all kM tokens
-// (codes expanded to int8 as in the GEMM rebuild, __dp4a). The tokens' INT8
-// rows sit in shared memory with a 16-byte pad after every chunk's bytes, so
-// the lanes' 16-byte loads fall in distinct banks. A row's kM sums are then
-// reduced over the warp by recursive halving (each step exchanges half of
-// the remaining sums, so every lane ends with the total of one token) -- all
-// integer adds, exact in any order -- and y = bf16_rn(fp32(acc) *
-// fp32(s_x[m] * gamma)) as in the GEMM epilogue. Before its dependency wait
-// every warp asks L2 to prefetch its rows' bytes: a prefetch only warms L2,
-// which stays coherent with whatever the kernel before writes, so it is safe
-// before the wait and lets the code fetch overlap the previous launch.
+// most SMs idle. K % 64 == 0 takes the warp-MMA kernel further down; the
+// kernel here covers K % 64 != 0, where rows of packed codes are 8-byte but
+// not 16-byte aligned. Warp w takes rows_per_warp consecutive output features
+// n (rows of the packed codes); for each row its lanes read consecutive
+// 8-byte chunks (32 codes), so every load instruction of the warp covers
+// contiguous bytes, and each lane forms the INT32 partial dot products of its
+// chunks with all kM tokens (codes expanded to int8 as in the GEMM rebuild,
+// __dp4a). The tokens' INT8 rows sit in shared memory with a 16-byte pad
+// after every chunk's 32 bytes, so the lanes' 16-byte loads fall in distinct
+// banks; kRows rows are taken at a time so that each token chunk read from
+// shared memory serves several rows. A row's kM sums are reduced over the
+// warp by recursive halving (each step exchanges half of the remaining sums,
+// so every lane ends with the total of one token) -- integer adds, exact in
+// any order -- and y = bf16_rn(fp32(acc) * fp32(s_x[m] * gamma)) as in the
+// GEMM epilogue.
 constexpr int kFewWarps = 8;
 constexpr int kFewMaxM = 16;
 constexpr int kFewWarpsPerSm = 16;  // target resident warps per SM when N allows
@@ -993,20 +993,19 @@ __device__ __forceinline__ bool few_writer(int lane) {
   return (lane & (kLow - 1)) == 0;
 }
 
-template <int kM, int kChunk>
+template <int kM>
 __global__ void __launch_bounds__(32 * kFewWarps) few_forward_kernel(
     const int8_t* __restrict__ xq, const float* __restrict__ sx, const uint8_t* __restrict__ packed,
     const float* __restrict__ gamma_ptr, int M, int N, int K, int rows_per_warp, __nv_bfloat16* __restrict__ y,
     int32_t* __restrict__ debug_acc) {
-  extern __shared__ __align__(16) uint8_t s_x[];  // [kM][cpr] chunks of 4 kChunk bytes, each + 16 pad
+  constexpr int kChunk = 8;           // bytes of packed codes per lane chunk (32 codes)
+  extern __shared__ __align__(16) uint8_t s_x[];  // [kM][cpr] chunks of 32 token bytes, each + 16 pad
   constexpr int kPitch = 4 * kChunk + 16;
   constexpr int kWords = kChunk / 4;  // 32-bit code words per chunk (16 codes each)
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int row_bytes = K / 4, cpr = row_bytes / kChunk;
   const int64_t n0 = (static_cast<int64_t>(blockIdx.x) * kFewWarps + warp) * rows_per_warp;
   const int nrows = n0 < N ? static_cast<int>(N - n0 < rows_per_warp ? N - n0 : rows_per_warp) : 0;
-  if (kChunk == 16 && lane == 0 && nrows > 0)
-    prefetch_l2_bulk(packed + n0 * row_bytes, static_cast<uint32_t>(nrows) * row_bytes);
   pdl_wait_primary();
   pdl_launch_dependents();
   // the tokens' rows into shared memory (rows M .. kM-1 zero)
@@ -1044,13 +1043,9 @@ __global__ void __launch_bounds__(32 * kFewWarps) few_forward_kernel(
         for (int u = 0; u < kSlots; ++u) {
           const int c = c0 + 32 * u + lane;
           const bool ok = g + r < nrows && c < cpr;
-          if constexpr (kChunk == 16) {
-            const uint4 w = ok ? __ldg(reinterpret_cast<const uint4*>(row) + c) : make_uint4(0u, 0u, 0u, 0u);
-            words[r][u][0] = w.x; words[r][u][1] = w.y; words[r][u][2] = w.z; words[r][u][3] = w.w;
-          } else {
-            const uint2 w = ok ? __ldg(reinterpret_cast<const uint2*>(row) + c) : make_uint2(0u, 0u);
-            words[r][u][0] = w.x; words[r][u][1] = w.y;
-          }
+          const uint2 w = ok ? __ldg(reinterpret_cast<const uint2*>(row) + c) : make_uint2(0u, 0u);
+          words[r][u][0] = w.x;
+          words[r][u][1] = w.y;
         }
       }
 #pragma unroll
@@ -1091,17 +1086,17 @@ __global__ void __launch_bounds__(32 * kFewWarps) few_forward_kernel(
   }
 }
 
-template <int kM, int kChunk>
+template <int kM>
 cudaError_t launch_few(const int8_t* xq, const float* sx, const uint8_t* packed, const float* gamma, int M, int N,
                        int K, void* y, int32_t* debug_acc, cudaStream_t s) {
-  const int cpr = K / 4 / kChunk;
-  const size_t smem = static_cast<size_t>(kM) * cpr * (4 * kChunk + 16);
+  const int cpr = K / 4 / 8;
+  const size_t smem = static_cast<size_t>(kM) * cpr * (4 * 8 + 16);
   static int configured[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !configured[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(few_forward_kernel<kM, kChunk>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         kSmemLimit);
+    cudaError_t e =
+        cudaFuncSetAttribute(few_forward_kernel<kM>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit);
     if (e != cudaSuccess) return e;
     configured[dev] = 1;
   }
@@ -1112,32 +1107,30 @@ cudaError_t launch_few(const int8_t* xq, const float* sx, const uint8_t* packed,
   rpw = (rpw + kRows - 1) / kRows * kRows;
   const int64_t warps = (N + rpw - 1) / rpw;
   const unsigned grid = static_cast<unsigned>((warps + kFewWarps - 1) / kFewWarps);
-  cudaError_t e = launch_pdl(few_forward_kernel<kM, kChunk>, dim3(grid), dim3(32 * kFewWarps), smem, s, xq, sx,
-                             packed, gamma, M, N, K, rpw, static_cast<__nv_bfloat16*>(y), debug_acc);
+  cudaError_t e = launch_pdl(few_forward_kernel<kM>, dim3(grid), dim3(32 * kFewWarps), smem, s, xq, sx, packed, gamma,
+                             M, N, K, rpw, static_cast<__nv_bfloat16*>(y), debug_acc);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
-// Smallest power-of-two token count >= M that the few-token kernel takes at
-// this K (its shared memory holds kM token rows), else 0.
+// Smallest power-of-two token count >= M whose token rows fit the SIMT
+// few-token kernel's shared memory at this K, else 0.
 int few_slots(int64_t M, int64_t K) {
   if (M > kFewMaxM) return 0;
   int slots = 1;
   while (slots < M) slots *= 2;
-  const int chunk = (K % 64) == 0 ? 16 : 8;
-  const size_t smem = static_cast<size_t>(slots) * (K / 4 / chunk) * (4 * chunk + 16);
+  const size_t smem = static_cast<size_t>(slots) * (K / 4 / 8) * (4 * 8 + 16);
   return smem <= static_cast<size_t>(kSmemLimit) ? slots : 0;
 }
 
-template <int kChunk>
-cudaError_t launch_few_chunk(int slots, const int8_t* xq, const float* sx, const uint8_t* packed, const float* gamma,
+cudaError_t launch_few_slots(int slots, const int8_t* xq, const float* sx, const uint8_t* packed, const float* gamma,
                              int M, int N, int K, void* y, int32_t* debug_acc, cudaStream_t s) {
   switch (slots) {
-    case 1: return launch_few<1, kChunk>(xq, sx, packed, gamma, M, N, K, y, debug_acc, s);
-    case 2: return launch_few<2, kChunk>(xq, sx, packed, gamma, M, N, K, y, debug_acc, s);
-    case 4: return launch_few<4, kChunk>(xq, sx, packed, gamma, M, N, K, y, debug_acc, s);
-    case 8: return launch_few<8, kChunk>(xq, sx, packed, gamma, M, N, K, y, debug_acc, s);
-    default: return launch_few<16, kChunk>(xq, sx, packed, gamma, M, N, K, y, debug_acc, s);
+    case 1: return launch_few<1>(xq, sx, packed, gamma, M, N, K, y, debug_acc, s);
+    case 2: return launch_few<2>(xq, sx, packed, gamma, M, N, K, y, debug_acc, s);
+    case 4: return launch_few<4>(xq, sx, packed, gamma, M, N, K, y, debug_acc, s);
+    case 8: return launch_few<8>(xq, sx, packed, gamma, M, N, K, y, debug_acc, s);
+    default: return launch_few<16>(xq, sx, packed, gamma, M, N, K, y, debug_acc, s);
   }
 }
 
@@ -1509,7 +1502,7 @@ cudaError_t launch_forward(const int8_t* xq, const float* sx, const uint8_t* w_p
   }
   if (const int slots = few_slots(M, K)) {
     const int m = static_cast<int>(M), nn = static_cast<int>(N), kk = static_cast<int>(K);
-    return launch_few_chunk<8>(slots, xq, sx, w_packed, gamma, m, nn, kk, y, debug_acc, s);
+    return launch_few_slots(slots, xq, sx, w_packed, gamma, m, nn, kk, y, debug_acc, s);
   }
   static const int kCands[3] = {256, 192, 128};
   const int npairs = resident_pairs<Family::Fwd, 256>();
