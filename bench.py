@@ -714,12 +714,14 @@ def run_few_tokens(args, rank, world, local_rank):
 
 def run_signsgd(args, rank, world, local_rank):
     """Sign-gradient data-parallel mode at up_proj: every rank quantises its
-    tokens, runs forward and backward with the 2-bit codes it holds, packs the
-    signs of its dW and sends them to rank 0, which alone holds the master W,
-    votes, updates W, re-ternarises and broadcasts the new codes. The line
-    reports the whole step (6 M N K per rank over the max-over-ranks time) and,
-    per sign-gradient kernel, achieved HBM GB/s against the measured copy
-    bandwidth."""
+    tokens, runs forward and backward with the 2-bit codes it holds -- the
+    backward writing dX and the sign words of dW, not dW
+    (bl_backward_signs) -- and sends the words to rank 0, which alone holds
+    the master W, votes, updates W, re-ternarises and broadcasts the new
+    codes. The line reports the whole step (6 M N K per rank over the
+    max-over-ranks time), the same step with dW written and packed by
+    bl_sign_pack (`unfused_ms_per_step`) and, per sign-gradient kernel,
+    achieved HBM GB/s against the copy bandwidth."""
     import ternary_weight_quantization_b200 as bl
     from ternary_weight_quantization_b200.signsgd import SignBuffers, signsgd_dp_step
     from workloads import workload_inputs
@@ -751,34 +753,44 @@ def run_signsgd(args, rank, world, local_rank):
         torch.distributed.broadcast(gamma, src=0)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
 
+    words = torch.empty((N, K // 32), dtype=torch.int32, device=dev)
+
     def step():
+        bl.bl_quantize_act(x, xq, sx)
+        bl.bl_forward(xq, sx, packed, gamma, y)
+        bl.bl_backward_signs(dy, xq, sx, packed, gamma, dX, words)
+        signsgd_dp_step(None, packed, gamma, lr, master_W=master, workspace=ws if holder else None, buffers=buf,
+                        words=words)
+
+    def step_unfused():
         bl.bl_quantize_act(x, xq, sx)
         bl.bl_forward(xq, sx, packed, gamma, y)
         bl.bl_backward(dy, xq, sx, packed, gamma, dX, dW)
         signsgd_dp_step(dW, packed, gamma, lr, master_W=master, workspace=ws if holder else None, buffers=buf)
 
-    times = []
+    # the two forms of the step alternate, so that both see the same clocks
+    times = {step: [], step_unfused: []}
     for i in range(args.warmup + args.steps):
-        flush.fill_(i & 0xFF)
-        flush.view(torch.int64).max()
-        if world > 1:
-            torch.distributed.barrier()
-        torch.cuda.synchronize(dev)
-        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        s.record(stream)
-        step()
-        e.record(stream)
-        torch.cuda.synchronize(dev)
-        if i >= args.warmup:
-            times.append(s.elapsed_time(e))
-    local_ms = sum(times) / len(times)
-    job_ms = job_time_ms(local_ms, world, dev)
+        for fn in (step, step_unfused):
+            flush.fill_(i & 0xFF)
+            flush.view(torch.int64).max()
+            if world > 1:
+                torch.distributed.barrier()
+            torch.cuda.synchronize(dev)
+            s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s.record(stream)
+            fn()
+            e.record(stream)
+            torch.cuda.synchronize(dev)
+            if i >= args.warmup:
+                times[fn].append(s.elapsed_time(e))
+    job_ms = job_time_ms(sum(times[step]) / len(times[step]), world, dev)
+    unfused_ms = job_time_ms(sum(times[step_unfused]) / len(times[step_unfused]), world, dev)
 
     # breakdown of the holder's sign-gradient kernels (events between the calls)
     peaks, peak_src = load_peaks()
     kern = {}
     if holder:
-        words = buf.gathered[0] if world == 1 else buf.words
         calls = {
             "sign_pack": (lambda: bl.bl_sign_pack(dW, words), N * K * 2 + N * K // 8),
             "sign_vote": (lambda: bl.bl_sign_vote(buf.gathered, buf.direction), world * N * K // 8 + N * K // 4),
@@ -809,6 +821,7 @@ def run_signsgd(args, rank, world, local_rank):
     ops = 6.0 * M * N * K
     return {"metric": "bitlinear_signsgd_dp_step_tops", "value": round(job_tops(ops, world, 1, job_ms), 2),
             "unit": "TOPS", "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(job_ms, 5),
+            "unfused_ms_per_step": round(unfused_ms, 5),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8/bf16",
             "data": "synthetic",
             "config": {"workload": "up_proj, sign-gradient data-parallel step", "M": M, "K": K, "N": N,
@@ -881,7 +894,7 @@ def run_extras(args, local_rank):
     line = run_few_tokens(ft, 0, 1, local_rank)
     extras["few_tokens"] = keep(line, ["by_tokens", "peak_gbs", "config"])
     line = run_signsgd(copy.copy(short), 0, 1, local_rank)
-    extras["signsgd"] = keep(line, ["value", "unit", "ms_per_step", "kernels"])
+    extras["signsgd"] = keep(line, ["value", "unit", "ms_per_step", "unfused_ms_per_step", "kernels"])
     line = run_lm(copy.copy(short), 0, 1, local_rank)
     extras["lm"] = keep(line, ["value", "unit", "ms_per_step", "loss_first", "loss_last", "max_abs_dloss_vs_oracle",
                                "dtype"])

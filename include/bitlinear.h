@@ -234,7 +234,8 @@ bl_status bl_export_weights(const uint8_t* w_packed, const float* gamma,
  * sign-based optimiser needs only the 2-bit weights on each device and one
  * bit of gradient per weight, sent to one place that accumulates them).
  * One step over R data-parallel ranks:
- *   every rank   bl_backward -> dW, bl_sign_pack -> its sign words
+ *   every rank   bl_backward_signs -> dX and the sign words of dW (or
+ *                bl_backward -> dW, then bl_sign_pack -> its sign words)
  *   exchange     the R ranks' sign words are gathered (N*K/8 bytes a rank)
  *   holder of W  bl_sign_vote -> direction, bl_signsgd_update on W, then
  *                bl_quantize_weight -> the next codes and gamma, which go
@@ -251,6 +252,21 @@ bl_status bl_export_weights(const uint8_t* w_packed, const float* gamma,
  */
 bl_status bl_sign_pack(const void* dW, bl_dtype dw_dtype, int64_t N, int64_t K,
                        uint32_t* sign_words, void* stream);
+
+/*
+ * S4 with G1 fused: bl_backward's dX (may be NULL) and, instead of dW, its
+ * sign words -- dw_sign_words [N*K/32] uint32 in bl_sign_pack's layout,
+ * written by the epilogue of the dW tiles straight from the fp32 sums (the
+ * rounding of dW to bf16 or fp32 keeps the sign, -0 included, so the words
+ * equal bl_sign_pack of bl_backward's dW bit for bit). dW is never written:
+ * N*K/8 bytes leave the kernel instead of N*K*2, and no second pass reads dW
+ * back. M == 0 writes all-zero words (dW = +0).
+ * Arguments and errors: as bl_backward (no accumulation, no dtype).
+ */
+bl_status bl_backward_signs(const void* dY, const int8_t* xq, const float* sx,
+                            const uint8_t* w_packed, const float* gamma,
+                            int64_t M, int64_t N, int64_t K,
+                            void* dX, uint32_t* dw_sign_words, void* stream);
 
 /*
  * G2: the accumulation. sign_words holds `ranks` arrays of N*K/32 words back

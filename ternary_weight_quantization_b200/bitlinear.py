@@ -40,6 +40,7 @@ SIGNATURES = {
     "bl_quantize": (_I32, [_VP, _I32, _I64, _I64, _VP, _I64, _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
     "bl_forward": (_I32, [_VP, _VP, _VP, _VP, _I64, _I64, _I64, _VP, _VP, _VP]),
     "bl_backward": (_I32, [_VP, _VP, _VP, _VP, _VP, _I64, _I64, _I64, _VP, _VP, _I32, _I32, _VP]),
+    "bl_backward_signs": (_I32, [_VP, _VP, _VP, _VP, _VP, _I64, _I64, _I64, _VP, _VP, _VP]),
     "bl_export_weights": (_I32, [_VP, _VP, _I64, _I64, _VP, _VP, _VP]),
     "bl_get_last_error": (_I32, []),
     "bl_reset_error": (_I32, []),
@@ -208,6 +209,25 @@ def bl_backward(dY, xq, sx, w_packed, gamma, dX=None, dW=None, accumulate_dW=Fal
     _check(load_library().bl_backward(_ptr(dY), _ptr(xq), _ptr(sx), _ptr(w_packed), _ptr(gamma), M, N, K,
                                       _ptr(dX), _ptr(dW), dwdt, int(bool(accumulate_dW)), _stream(stream)),
            "bl_backward")
+
+
+def bl_backward_signs(dY, xq, sx, w_packed, gamma, dX, dw_sign_words, stream=None):
+    """S4 with G1 fused: dX [M,K] bf16 (or None) as bl_backward, and the sign
+    words of dW, dw_sign_words [N, K/32] int32 (bit patterns), instead of dW."""
+    M, N = dY.shape
+    K = xq.shape[1]
+    _need(dY, torch.bfloat16, (M, N), "dY")
+    _need(xq, torch.int8, (M, K), "xq")
+    _need(sx, torch.float32, (M,), "sx")
+    _need(w_packed, torch.uint8, (N, K // 4), "w_packed")
+    _need(gamma, torch.float32, (1,), "gamma")
+    if dX is not None:
+        _need(dX, torch.bfloat16, (M, K), "dX")
+    _need(dw_sign_words, torch.int32, (N, K // 32), "dw_sign_words")
+    _on_current_device(dY, xq, sx, w_packed, gamma, dX, dw_sign_words)
+    _check(load_library().bl_backward_signs(_ptr(dY), _ptr(xq), _ptr(sx), _ptr(w_packed), _ptr(gamma), M, N, K,
+                                            _ptr(dX), _ptr(dw_sign_words), _stream(stream)),
+           "bl_backward_signs")
 
 
 def bl_sign_pack(dW, sign_words, stream=None):

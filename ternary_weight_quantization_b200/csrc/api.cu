@@ -206,8 +206,31 @@ bl_status bl_backward(const void* dY, const int8_t* xq, const float* sx, const u
   int* err = nullptr;
   if (bl_status s = current_device(&err)) return s;
   return cuda_status(bl::launch_backward(dY, xq, sx, w_packed, gamma, M, N, K, dX, dW, dw_dtype == BL_F32,
-                                         accumulate_dW != 0, err, static_cast<cudaStream_t>(stream)),
+                                         accumulate_dW != 0, 0, err, static_cast<cudaStream_t>(stream)),
                      "bl_backward launch");
+}
+
+bl_status bl_backward_signs(const void* dY, const int8_t* xq, const float* sx, const uint8_t* w_packed,
+                            const float* gamma, int64_t M, int64_t N, int64_t K, void* dX, uint32_t* dw_sign_words,
+                            void* stream) {
+  g_msg[0] = 0;
+  if (M < 0 || N < 1) return fail(BL_ERR_INVALID_ARG, "M=%lld, N=%lld", (long long)M, (long long)N);
+  if (bl_status s = check_k(K)) return s;
+  if (N % 8 != 0) return fail(BL_ERR_UNSUPPORTED_SHAPE, "N=%lld must be a multiple of 8", (long long)N);
+  if (M > (int64_t(1) << 30) || N > (int64_t(1) << 30)) return fail(BL_ERR_UNSUPPORTED_SHAPE, "M or N too large");
+  if (!dw_sign_words) return fail(BL_ERR_INVALID_ARG, "null dw_sign_words");
+  if (M > 0 && !dY) return fail(BL_ERR_INVALID_ARG, "null dY");
+  if (dX && (!w_packed || !gamma)) return fail(BL_ERR_INVALID_ARG, "dX needs w_packed and gamma");
+  if (M > 0 && (!xq || !sx)) return fail(BL_ERR_INVALID_ARG, "the sign words need xq and sx");
+  if ((dY && !aligned16(dY)) || (xq && !aligned16(xq)) || (sx && !aligned16(sx)) ||
+      (w_packed && !aligned16(w_packed)) || (gamma && !aligned16(gamma)) || (dX && !aligned16(dX)) ||
+      !aligned16(dw_sign_words))
+    return fail(BL_ERR_ALIGNMENT, "tensors must be 16-byte aligned");
+  int* err = nullptr;
+  if (bl_status s = current_device(&err)) return s;
+  return cuda_status(bl::launch_backward(dY, xq, sx, w_packed, gamma, M, N, K, dX, dw_sign_words, 0, 0, 1, err,
+                                         static_cast<cudaStream_t>(stream)),
+                     "bl_backward_signs launch");
 }
 
 bl_status bl_export_weights(const uint8_t* w_packed, const float* gamma, int64_t N, int64_t K,

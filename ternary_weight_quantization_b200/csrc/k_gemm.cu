@@ -188,6 +188,7 @@ struct OpParams {
   int accumulate; // Dw
   int src_tma;    // Fwd/Dx: packed codes by TMA (K % 64 == 0) instead of cp.async
   int tma_store;  // output through the TMA store map of this op
+  int sign_words; // Dw: out receives the sign bits of dW (32 per word along K) instead of dW
 };
 
 struct GemmParams {
@@ -542,6 +543,24 @@ __device__ __noinline__ void epilogue_chunk_direct(const GemmParams& p, const Op
   }
 }
 
+// Sign bits of dW instead of dW: lane = k (i0 + lane), r[jj] = the fp32 sum
+// of dW[j0 + jj][k]. Rounding to bf16 or fp32 keeps the sign (-0 included),
+// so the sign bit of the sum is the sign bit of dW; one ballot per row gives
+// the row's 32 bits for k = i0 .. i0 + 31 (bit l = k i0 + l), which is word
+// (j K + i0) / 32 of the flattened [N, K] sign words. Lane jj writes row
+// j0 + jj's word.
+__device__ __forceinline__ void epilogue_chunk_signs(const OpParams& P, const uint32_t (&r)[32], int lane, int i0,
+                                                     int j0) {
+  uint32_t mine = 0;
+#pragma unroll
+  for (int jj = 0; jj < 32; ++jj) {
+    const uint32_t w = __ballot_sync(0xffffffffu, (r[jj] >> 31) != 0u);
+    mine = lane == jj ? w : mine;
+  }
+  const int j = j0 + lane;
+  if (j < P.rows_b) static_cast<uint32_t*>(P.out)[static_cast<int64_t>(j) * (P.ldo / 32) + i0 / 32] = mine;
+}
+
 // Epilogue, one 32 x 32 chunk in registers: lane = output column i (A row),
 // r[jj] = output row j0 + jj. The common case is a bf16 box converted into
 // one of the warp's kSlots 2 KB staging slots (used in turn) and written by
@@ -551,6 +570,12 @@ __device__ __forceinline__ void epilogue_chunk(const GemmParams& p, const OpPara
                                                uint32_t (&r)[32], uint32_t stg, uint32_t scales, int lane, int i0,
                                                int j0, int c, float col_scale, float gamma, uint32_t& seq) {
   if (i0 >= P.rows_a || j0 >= P.rows_b) return;
+  if constexpr (op == Op::Dw) {
+    if (P.sign_words) {
+      epilogue_chunk_signs(P, r, lane, i0, j0);
+      return;
+    }
+  }
   if (!P.tma_store || P.out_f32) {
     // the out-of-line paths take a copy, so that r itself stays in registers
     uint32_t t[32];
@@ -1540,10 +1565,12 @@ cudaError_t launch_forward(const int8_t* xq, const float* sx, const uint8_t* w_p
 // dX and/or dW in one launch (either output may be null).
 cudaError_t launch_backward(const void* dY, const int8_t* xq, const float* sx, const uint8_t* w_packed,
                             const float* gamma, int64_t M, int64_t N, int64_t K, void* dX, void* dW, int dw_is_f32,
-                            int accumulate, int* err, cudaStream_t s) {
+                            int accumulate, int dw_signs, int* err, cudaStream_t s) {
   if (dW && M == 0) {
-    const int64_t n = N * K;
-    zero_dw_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, s>>>(dW, n, dw_is_f32, accumulate);
+    // dW = 0: zeros, or sign words of +0 (all bits clear, 4-byte words)
+    const int64_t n = dw_signs ? N * K / 32 : N * K;
+    zero_dw_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, s>>>(dW, n, dw_signs ? 1 : dw_is_f32,
+                                                                           dw_signs ? 0 : accumulate);
     if (cudaError_t e = cudaGetLastError(); e != cudaSuccess) return e;
   }
   if (M == 0) return cudaSuccess;
@@ -1570,7 +1597,8 @@ cudaError_t launch_backward(const void* dY, const int8_t* xq, const float* sx, c
         !make_map_2d(&maps[6], sx, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, M, 1, sx_pitch, 64, 1, CU_TENSOR_MAP_SWIZZLE_NONE,
                      "sx (dW)"))
       return cudaErrorInvalidValue;
-    if (!accumulate && !make_out_map(&maps[5], dW, dw_is_f32 != 0, N, K, "dW")) return cudaErrorInvalidValue;
+    if (!accumulate && !dw_signs && !make_out_map(&maps[5], dW, dw_is_f32 != 0, N, K, "dW"))
+      return cudaErrorInvalidValue;
   }
   static thread_local GemmParams p;
   std::memset(&p, 0, offsetof(GemmParams, sched_start));
@@ -1585,9 +1613,10 @@ cudaError_t launch_backward(const void* dY, const int8_t* xq, const float* sx, c
     fill_op(p.op[1], static_cast<int>(K), static_cast<int>(N), static_cast<int>(M), 64, BN);
     p.op[1].out = dW;
     p.op[1].ldo = K;
-    p.op[1].out_f32 = dw_is_f32;
-    p.op[1].accumulate = accumulate;
-    p.op[1].tma_store = !accumulate;
+    p.op[1].out_f32 = dw_signs ? 0 : dw_is_f32;
+    p.op[1].accumulate = dw_signs ? 0 : accumulate;
+    p.op[1].tma_store = !accumulate && !dw_signs;
+    p.op[1].sign_words = dw_signs;
   }
   p.K = K;
   p.packed = w_packed;

@@ -7,7 +7,8 @@ and one bit of gradient per weight, streamed to one place that accumulates
 them. Here that place is the holder rank, which alone keeps the master W.
 
 One step, entered by every rank in the same order:
-  1. every rank: the sign words of its dW (``bl_sign_pack``, N*K/8 bytes)
+  1. every rank: the sign words of its dW (``bl_sign_pack`` on dW, or made
+     by the backward itself with ``bl_backward_signs``; N*K/8 bytes)
   2. gather of the R ranks' words on the holder (torch.distributed; NCCL on
      GPUs, each rank sends N*K/8 bytes)
   3. holder: majority vote (``bl_sign_vote``), the update of W
@@ -63,29 +64,39 @@ def _world():
 
 
 def signsgd_dp_step(dW, w_packed, gamma, lr, *, master_W=None, workspace=None, holder: int = 0,
-                    buffers: SignBuffers | None = None, ops: SignOps | None = None):
+                    buffers: SignBuffers | None = None, ops: SignOps | None = None, words=None):
     """One sign-gradient step of one layer over the default process group.
 
-    dW [N, K]: this rank's gradient (bf16 or f32). w_packed [N, K/4] uint8 and
-    gamma [1] f32: this rank's codes, replaced by the step's new ones.
-    master_W [N, K] and workspace (``bl_quantize_weight``'s scratch): needed on
-    the holder rank only. Returns (w_packed, gamma).
+    dW [N, K]: this rank's gradient (bf16 or f32) -- or dW None and words
+    [N, K/32] int32: its sign words, already made (``bl_backward_signs``).
+    w_packed [N, K/4] uint8 and gamma [1] f32: this rank's codes, replaced by
+    the step's new ones. master_W [N, K] and workspace
+    (``bl_quantize_weight``'s scratch): needed on the holder rank only.
+    Returns (w_packed, gamma).
     """
     ops = ops or SignOps()
     world, rank = _world()
-    N, K = dW.shape
+    if (dW is None) == (words is None):
+        raise ValueError("pass exactly one of dW and words")
+    N, K = w_packed.shape[0], w_packed.shape[1] * 4
     is_holder = rank == holder
     if is_holder and (master_W is None or workspace is None):
         raise ValueError("the holder rank needs master_W and workspace")
-    buf = buffers or SignBuffers.allocate(N, K, world, is_holder, dW.device)
+    buf = buffers or SignBuffers.allocate(N, K, world, is_holder, w_packed.device)
 
     if world > 1:
-        ops.sign_pack(dW, buf.words)
-        dist.gather(buf.words, list(buf.gathered.unbind(0)) if is_holder else None, dst=holder)
-    else:
+        if words is None:
+            ops.sign_pack(dW, buf.words)
+            words = buf.words
+        dist.gather(words, list(buf.gathered.unbind(0)) if is_holder else None, dst=holder)
+        votes = buf.gathered
+    elif words is None:
         ops.sign_pack(dW, buf.gathered[0])  # a single rank votes on its own words
+        votes = buf.gathered
+    else:
+        votes = words.unsqueeze(0)
     if is_holder:
-        ops.sign_vote(buf.gathered, buf.direction)
+        ops.sign_vote(votes, buf.direction)
         ops.update(master_W, buf.direction, lr)
         ops.quantize_weight(master_W, w_packed, gamma, workspace)
     if world > 1:

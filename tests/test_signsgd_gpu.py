@@ -134,3 +134,93 @@ def test_single_rank_step_matches_oracle_chain(shape, w_dtype):
     codes, gm = ref.ternarize(w_new)
     assert float(gamma.item()) == float(gm)
     assert np.array_equal(w_packed.cpu().numpy(), ref.pack_ternary(codes))
+
+
+@pytest.mark.parametrize("M,N,K", [(17, 136, 96), (300, 520, 320), (64, 1000, 160), (257, 392, 544),
+                                   (4096, 6912, 2560)])
+def test_backward_signs_match_sign_pack_of_dw(M, N, K):
+    """bl_backward_signs: dX as bl_backward's and the sign words equal to
+    bl_sign_pack of bl_backward's dW (bf16 and f32), bit for bit; against the
+    oracle, every element whose dW is clearly away from zero has its sign."""
+    bl = _bl()
+    from workloads import make_inputs
+    x, w, dy = make_inputs(M, K, N, seed=M + N + K)
+    packed = torch.empty((N, K // 4), dtype=torch.uint8, device="cuda")
+    gamma = torch.empty(1, dtype=torch.float32, device="cuda")
+    ws = torch.empty(max(bl.bl_quantize_weight_workspace_size(N, K), 16), dtype=torch.uint8, device="cuda")
+    xq = torch.empty((M, K), dtype=torch.int8, device="cuda")
+    sx = torch.empty(M, dtype=torch.float32, device="cuda")
+    bl.bl_quantize(w.cuda(), x.cuda(), packed, gamma, xq, sx, ws)
+    dyd = dy.cuda()
+    dx_ref = torch.empty((M, K), dtype=torch.bfloat16, device="cuda")
+    dx = torch.empty_like(dx_ref)
+    words_ref = {}
+    for dt in (torch.bfloat16, torch.float32):
+        dw = torch.empty((N, K), dtype=dt, device="cuda")
+        bl.bl_backward(dyd, xq, sx, packed, gamma, dx_ref, dw)
+        wr = torch.empty((N, K // 32), dtype=torch.int32, device="cuda")
+        bl.bl_sign_pack(dw, wr)
+        words_ref[dt] = wr
+    words = torch.full((N, K // 32), -1, dtype=torch.int32, device="cuda")
+    bl.bl_backward_signs(dyd, xq, sx, packed, gamma, dx, words)
+    torch.cuda.synchronize()
+    assert bl.bl_get_last_error() == 0
+    assert torch.equal(words, words_ref[torch.bfloat16])
+    assert torch.equal(words, words_ref[torch.float32])
+    assert torch.equal(dx.view(torch.int16), dx_ref.view(torch.int16))
+    if M * N * K > 10 ** 9:
+        return  # full size: the bit-exact equality above; the oracle's fp64 dW would take minutes
+    # signs against the oracle's fp64 dW where |dW| > 1e-2 rms (far above any rounding)
+    q, s_x = ref.quantize_activations(ref.bf16_bits_to_f32(_u16(x)))
+    x_hat = ref.bf16_bits_to_f32(ref.round_to_bf16_bits(ref.dequantize_activations(q, s_x)))
+    dw_o = ref.backward_dw(ref.bf16_bits_to_f32(_u16(dy)), x_hat)
+    bits = sg.unpack_sign_bits(words.cpu().numpy().view(np.uint32)).reshape(N, K)
+    clear = np.abs(dw_o) > 1e-2 * np.sqrt(np.mean(dw_o ** 2))
+    assert np.array_equal(bits[clear], (dw_o[clear] < 0).astype(bits.dtype))
+
+
+def test_backward_signs_without_tokens():
+    """M = 0: dW = +0, so every sign word is zero; dX may be omitted."""
+    bl = _bl()
+    N, K = 64, 128
+    packed = torch.zeros((N, K // 4), dtype=torch.uint8, device="cuda")
+    gamma = torch.ones(1, dtype=torch.float32, device="cuda")
+    words = torch.full((N, K // 32), -1, dtype=torch.int32, device="cuda")
+    bl.bl_backward_signs(torch.empty((0, N), dtype=torch.bfloat16, device="cuda"),
+                         torch.empty((0, K), dtype=torch.int8, device="cuda"),
+                         torch.empty(0, dtype=torch.float32, device="cuda"), packed, gamma, None, words)
+    torch.cuda.synchronize()
+    assert int(words.abs().sum()) == 0
+
+
+def test_single_rank_step_from_fused_sign_words():
+    """The whole sign-gradient step fed by bl_backward_signs ends with the same
+    master, codes and gamma as the step fed by bl_backward's dW."""
+    bl = _bl()
+    from ternary_weight_quantization_b200.signsgd import signsgd_dp_step
+    from workloads import make_inputs
+    M, N, K = 512, 1024, 640
+    x, w, dy = make_inputs(M, K, N, seed=5)
+    results = []
+    for fused in (False, True):
+        wd = w.cuda()
+        packed = torch.empty((N, K // 4), dtype=torch.uint8, device="cuda")
+        gamma = torch.empty(1, dtype=torch.float32, device="cuda")
+        ws = torch.empty(max(bl.bl_quantize_weight_workspace_size(N, K), 16), dtype=torch.uint8, device="cuda")
+        xq = torch.empty((M, K), dtype=torch.int8, device="cuda")
+        sx = torch.empty(M, dtype=torch.float32, device="cuda")
+        dx = torch.empty((M, K), dtype=torch.bfloat16, device="cuda")
+        bl.bl_quantize(wd, x.cuda(), packed, gamma, xq, sx, ws)
+        if fused:
+            words = torch.empty((N, K // 32), dtype=torch.int32, device="cuda")
+            bl.bl_backward_signs(dy.cuda(), xq, sx, packed, gamma, dx, words)
+            signsgd_dp_step(None, packed, gamma, 2.0 ** -8, master_W=wd, workspace=ws, words=words)
+        else:
+            dw = torch.empty((N, K), dtype=torch.bfloat16, device="cuda")
+            bl.bl_backward(dy.cuda(), xq, sx, packed, gamma, dx, dw)
+            signsgd_dp_step(dw, packed, gamma, 2.0 ** -8, master_W=wd, workspace=ws)
+        torch.cuda.synchronize()
+        results.append((_u16(wd), packed.cpu().numpy(), float(gamma.item())))
+    assert np.array_equal(results[0][0], results[1][0])
+    assert np.array_equal(results[0][1], results[1][1])
+    assert results[0][2] == results[1][2]

@@ -66,7 +66,12 @@ def _expected(world):
     return ref.pack_ternary(codes), float(g)
 
 
-def _worker(rank, world, port, holder, out):
+def _words(rank):
+    """The rank's sign words as a fused backward would hand them over."""
+    return torch.from_numpy(sg.sign_bits(_grad(rank).float().numpy()).view(np.int32).copy())
+
+
+def _worker(rank, world, port, holder, out, with_words=False):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     torch.distributed.init_process_group("gloo", rank=rank, world_size=world,
                                          timeout=datetime.timedelta(seconds=60))
@@ -75,18 +80,23 @@ def _worker(rank, world, port, holder, out):
         w_packed = torch.zeros((N, K // 4), dtype=torch.uint8)
         gamma = torch.zeros(1, dtype=torch.float32)
         kw = dict(master_W=_master(), workspace=torch.empty(64, dtype=torch.uint8)) if rank == holder else {}
-        signsgd_dp_step(_grad(rank), w_packed, gamma, LR, holder=holder, ops=_oracle_ops(), **kw)
+        if with_words:
+            signsgd_dp_step(None, w_packed, gamma, LR, holder=holder, ops=_oracle_ops(), words=_words(rank), **kw)
+        else:
+            signsgd_dp_step(_grad(rank), w_packed, gamma, LR, holder=holder, ops=_oracle_ops(), **kw)
         out[rank] = (w_packed.numpy().tobytes(), float(gamma[0]))
     finally:
         torch.distributed.destroy_process_group()
 
 
-@pytest.mark.parametrize("world,holder", [(2, 0), (3, 1)])
-def test_ranks_end_with_the_holders_codes(world, holder):
+@pytest.mark.parametrize("world,holder,with_words", [(2, 0, False), (3, 1, False), (2, 1, True)])
+def test_ranks_end_with_the_holders_codes(world, holder, with_words):
+    """Every rank ends with the oracle chain's codes and gamma, whether it
+    hands over dW (packed here) or the sign words a fused backward made."""
     ctx = mp.get_context("spawn")
     out = ctx.Manager().dict()
     port = _free_port()
-    procs = [ctx.Process(target=_worker, args=(r, world, port, holder, out)) for r in range(world)]
+    procs = [ctx.Process(target=_worker, args=(r, world, port, holder, out, with_words)) for r in range(world)]
     for p in procs:
         p.start()
     for p in procs:
@@ -112,3 +122,23 @@ def test_holder_needs_the_master():
     from ternary_weight_quantization_b200.signsgd import signsgd_dp_step
     with pytest.raises(ValueError):
         signsgd_dp_step(_grad(0), torch.zeros((N, K // 4), dtype=torch.uint8), torch.zeros(1), LR, ops=_oracle_ops())
+
+
+def test_single_rank_from_sign_words():
+    from ternary_weight_quantization_b200.signsgd import signsgd_dp_step
+    w_packed = torch.zeros((N, K // 4), dtype=torch.uint8)
+    gamma = torch.zeros(1, dtype=torch.float32)
+    signsgd_dp_step(None, w_packed, gamma, LR, master_W=_master(), workspace=torch.empty(64, dtype=torch.uint8),
+                    ops=_oracle_ops(), words=_words(0))
+    packed, g = _expected(1)
+    assert w_packed.numpy().tobytes() == packed.tobytes() and float(gamma[0]) == g
+
+
+def test_exactly_one_gradient_form():
+    from ternary_weight_quantization_b200.signsgd import signsgd_dp_step
+    kw = dict(master_W=_master(), workspace=torch.empty(64, dtype=torch.uint8), ops=_oracle_ops())
+    with pytest.raises(ValueError):
+        signsgd_dp_step(_grad(0), torch.zeros((N, K // 4), dtype=torch.uint8), torch.zeros(1), LR, words=_words(0),
+                        **kw)
+    with pytest.raises(ValueError):
+        signsgd_dp_step(None, torch.zeros((N, K // 4), dtype=torch.uint8), torch.zeros(1), LR, **kw)
