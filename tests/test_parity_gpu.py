@@ -201,7 +201,8 @@ def test_gamma_at_an_fp32_midpoint(case, expected, w_dtype):
     """Mean |W| on, 2^-44 above or 2^-44 below the fp32 midpoint 1 + 2^-24
     (the fp64 tree sum's error bound straddles it, so gamma comes from the
     exact integer sum): gamma and the codes bit-exact to the oracle through
-    bl_quantize_weight, bl_quantize and bl_quantize_weight_noalloc, twice."""
+    bl_quantize_weight, bl_quantize (with its token rows, also bit-exact) and
+    bl_quantize_weight_noalloc, twice."""
     from workloads import gamma_midpoint_weights
     bl = _bl()
     w = gamma_midpoint_weights(case, w_dtype)
@@ -210,20 +211,25 @@ def test_gamma_at_an_fp32_midpoint(case, expected, w_dtype):
     assert g == np.float32(expected)
     expect = ref.pack_ternary(codes)
     wd = w.cuda()
-    x, _, _ = make_inputs(64, K, 8, seed=3)
-    xd = x.cuda()
+    # 64 tokens all go to the coding launch; 4000 are split between the two launches
+    xs = {m: make_inputs(m, K, 8, seed=3 + m)[0] for m in (64, 4000)}
     ws = torch.empty(bl.bl_quantize_weight_workspace_size(N, K), dtype=torch.uint8, device="cuda")
     lib = bl.load_library()
     for rep in range(2):
-        for how in ("weight", "fused", "noalloc"):
+        for how in ("weight", "fused64", "fused4000", "noalloc"):
             packed = torch.full((N, K // 4), 0xAA, dtype=torch.uint8, device="cuda")
             gamma = torch.full((1,), -1.0, dtype=torch.float32, device="cuda")
             if how == "weight":
                 bl.bl_quantize_weight(wd, packed, gamma, ws)
-            elif how == "fused":
-                xq = torch.empty((64, K), dtype=torch.int8, device="cuda")
-                sx = torch.empty(64, dtype=torch.float32, device="cuda")
-                bl.bl_quantize(wd, xd, packed, gamma, xq, sx, ws)
+            elif how.startswith("fused"):
+                m = int(how[5:])
+                xq = torch.empty((m, K), dtype=torch.int8, device="cuda")
+                sx = torch.empty(m, dtype=torch.float32, device="cuda")
+                bl.bl_quantize(wd, xs[m].cuda(), packed, gamma, xq, sx, ws)
+                torch.cuda.synchronize()
+                q_o, s_o = ref.quantize_activations(ref.bf16_bits_to_f32(bits(xs[m])))
+                np.testing.assert_array_equal(xq.cpu().numpy(), q_o, err_msg=how)
+                np.testing.assert_array_equal(sx.cpu().numpy().view(np.uint32), s_o.view(np.uint32), err_msg=how)
             else:
                 wdt = bl.BL_F32 if w_dtype == torch.float32 else bl.BL_BF16
                 import ctypes
