@@ -53,7 +53,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 INT8_OVER_BF16 = 2.0  # nominal dense ratio (4.5 / 2.25 PFLOP/s)
 KERNEL_SOURCES = ["ternary_weight_quantization_b200/csrc/k_quant.cu",
                   "ternary_weight_quantization_b200/csrc/k_gemm.cu",
-                  "ternary_weight_quantization_b200/csrc/bl_device.cuh"]
+                  "ternary_weight_quantization_b200/csrc/bl_device.cuh",
+                  "ternary_weight_quantization_b200/csrc/bl_abs_sum.cuh"]
 
 
 def load_peaks():
@@ -717,13 +718,15 @@ def run_signsgd(args, rank, world, local_rank):
     tokens, runs forward and backward with the 2-bit codes it holds -- the
     backward writing dX and the sign words of dW, not dW
     (bl_backward_signs) -- and sends the words to rank 0, which alone holds
-    the master W, votes, updates W, re-ternarises and broadcasts the new
-    codes. The line reports the whole step (6 M N K per rank over the
-    max-over-ranks time), the same step with dW written and packed by
-    bl_sign_pack (`unfused_ms_per_step`) and, per sign-gradient kernel,
-    achieved HBM GB/s against the copy bandwidth."""
+    the master W, votes, updates W and re-ternarises (bl_signsgd_apply: the
+    vote, the update and the |W| sums in one sweep, then the code launch) and
+    broadcasts the new codes. The line reports the whole step (6 M N K per
+    rank over the max-over-ranks time), the same step unfused
+    (`unfused_ms_per_step`: dW written and packed by bl_sign_pack, then
+    bl_sign_vote, bl_signsgd_update and bl_quantize_weight) and, per
+    sign-gradient call, achieved HBM GB/s against the copy bandwidth."""
     import ternary_weight_quantization_b200 as bl
-    from ternary_weight_quantization_b200.signsgd import SignBuffers, signsgd_dp_step
+    from ternary_weight_quantization_b200.signsgd import SignBuffers, SignOps, signsgd_dp_step
     from workloads import workload_inputs
 
     bl.load_library()
@@ -762,11 +765,14 @@ def run_signsgd(args, rank, world, local_rank):
         signsgd_dp_step(None, packed, gamma, lr, master_W=master, workspace=ws if holder else None, buffers=buf,
                         words=words)
 
+    three_calls = SignOps(apply=None)
+
     def step_unfused():
         bl.bl_quantize_act(x, xq, sx)
         bl.bl_forward(xq, sx, packed, gamma, y)
         bl.bl_backward(dy, xq, sx, packed, gamma, dX, dW)
-        signsgd_dp_step(dW, packed, gamma, lr, master_W=master, workspace=ws if holder else None, buffers=buf)
+        signsgd_dp_step(dW, packed, gamma, lr, master_W=master, workspace=ws if holder else None, buffers=buf,
+                        ops=three_calls)
 
     # the two forms of the step alternate, so that both see the same clocks
     times = {step: [], step_unfused: []}
@@ -797,6 +803,9 @@ def run_signsgd(args, rank, world, local_rank):
             "signsgd_update": (lambda: bl.bl_signsgd_update(master, buf.direction, 0.0),
                                2 * N * K * 2 + N * K // 4),
             "quantize_weight": (lambda: bl.bl_quantize_weight(master, packed, gamma, ws), N * K * 2 + N * K // 4),
+            # vote + update + new codes: words read, W read and written once, codes written
+            "signsgd_apply": (lambda: bl.bl_signsgd_apply(buf.gathered, master, 0.0, packed, gamma, ws),
+                              world * N * K // 8 + 2 * N * K * 2 + N * K // 4),
         }
         for name, (fn, nbytes) in calls.items():
             ts = []

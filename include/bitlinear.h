@@ -237,9 +237,10 @@ bl_status bl_export_weights(const uint8_t* w_packed, const float* gamma,
  *   every rank   bl_backward_signs -> dX and the sign words of dW (or
  *                bl_backward -> dW, then bl_sign_pack -> its sign words)
  *   exchange     the R ranks' sign words are gathered (N*K/8 bytes a rank)
- *   holder of W  bl_sign_vote -> direction, bl_signsgd_update on W, then
- *                bl_quantize_weight -> the next codes and gamma, which go
- *                back to the ranks.
+ *   holder of W  bl_signsgd_apply: vote, update of W and the next codes and
+ *                gamma in two launches (or the three calls bl_sign_vote,
+ *                bl_signsgd_update, bl_quantize_weight), which go back to
+ *                the ranks.
  */
 
 /*
@@ -289,6 +290,25 @@ bl_status bl_sign_vote(const uint32_t* sign_words, int ranks, int64_t N, int64_t
  */
 bl_status bl_signsgd_update(void* W, bl_dtype w_dtype, int64_t N, int64_t K,
                             const uint8_t* direction, float lr, void* stream);
+
+/*
+ * G2 + G3 + S1 on the holder, fused: the same W, w_packed and gamma as
+ * bl_sign_vote, bl_signsgd_update and bl_quantize_weight called in turn, bit
+ * for bit, in two launches. The first votes the `ranks` sign-word arrays
+ * (layout of bl_sign_vote), updates W in place (bl_signsgd_update's rule) and
+ * sums |W| of the updated weights in fp64 in the same sweep; the second is
+ * bl_quantize_weight's code launch (gamma exactly as there, then the codes,
+ * re-reading W from L2). Saves the direction array (N*K/4 bytes written and
+ * read back), the vote launch and the re-read of W from HBM for its sum.
+ * workspace: as bl_quantize_weight (bl_quantize_weight_workspace_size bytes,
+ * 16-byte aligned, no initialisation; one call at a time per workspace).
+ * Errors: as bl_signsgd_update and bl_quantize_weight (BL_ERR_INVALID_ARG
+ * also for ranks out of 1..127, BL_ERR_WORKSPACE); a device wait that gave up
+ * records BL_ERR_TIMEOUT (bl_get_last_error).
+ */
+bl_status bl_signsgd_apply(const uint32_t* sign_words, int ranks, void* W, bl_dtype w_dtype,
+                           int64_t N, int64_t K, float lr, uint8_t* w_packed, float* gamma,
+                           void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * Synchronises the current device, then returns BL_OK or the first device

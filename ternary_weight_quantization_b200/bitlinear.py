@@ -48,6 +48,7 @@ SIGNATURES = {
     "bl_sign_pack": (_I32, [_VP, _I32, _I64, _I64, _VP, _VP]),
     "bl_sign_vote": (_I32, [_VP, _I32, _I64, _I64, _VP, _VP]),
     "bl_signsgd_update": (_I32, [_VP, _I32, _I64, _I64, _VP, ctypes.c_float, _VP]),
+    "bl_signsgd_apply": (_I32, [_VP, _I32, _VP, _I32, _I64, _I64, ctypes.c_float, _VP, _VP, _VP, _SZ, _VP]),
 }
 
 
@@ -263,6 +264,26 @@ def bl_signsgd_update(W, direction, lr, stream=None):
     dt = BL_F32 if W.dtype == torch.float32 else BL_BF16
     _check(load_library().bl_signsgd_update(_ptr(W), dt, N, K, _ptr(direction), float(lr), _stream(stream)),
            "bl_signsgd_update")
+
+
+def bl_signsgd_apply(sign_words, W, lr, w_packed, gamma, workspace, stream=None):
+    """G2 + G3 + S1 fused on the holder: the majority direction of sign_words
+    [R, N, K/32] int32 applied to W [N, K] (bf16|f32) in place, then W's new
+    w_packed [N, K/4] uint8 and gamma [1] f32 (two launches)."""
+    R, N, KW = sign_words.shape
+    K = KW * 32
+    if W.dtype not in (torch.bfloat16, torch.float32):
+        raise ValueError("W must be bf16 or f32")
+    _need(sign_words, torch.int32, (R, N, KW), "sign_words")
+    _need(W, W.dtype, (N, K), "W")
+    _need(w_packed, torch.uint8, (N, K // 4), "w_packed")
+    _need(gamma, torch.float32, (1,), "gamma")
+    _on_current_device(sign_words, W, w_packed, gamma, workspace)
+    dt = BL_F32 if W.dtype == torch.float32 else BL_BF16
+    _check(load_library().bl_signsgd_apply(_ptr(sign_words), R, _ptr(W), dt, N, K, float(lr), _ptr(w_packed),
+                                           _ptr(gamma), _ptr(workspace),
+                                           workspace.numel() * workspace.element_size(), _stream(stream)),
+           "bl_signsgd_apply")
 
 
 def bl_export_weights(w_packed, gamma, stream=None):

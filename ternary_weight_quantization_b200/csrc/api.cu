@@ -294,6 +294,28 @@ bl_status bl_signsgd_update(void* W, bl_dtype w_dtype, int64_t N, int64_t K, con
                      "bl_signsgd_update");
 }
 
+bl_status bl_signsgd_apply(const uint32_t* sign_words, int ranks, void* W, bl_dtype w_dtype, int64_t N, int64_t K,
+                           float lr, uint8_t* w_packed, float* gamma, void* workspace, size_t workspace_bytes,
+                           void* stream) {
+  g_msg[0] = 0;
+  if (N < 1) return fail(BL_ERR_INVALID_ARG, "N=%lld must be >= 1", (long long)N);
+  if (bl_status s = check_k(K)) return s;
+  if (ranks < 1 || ranks > 127) return fail(BL_ERR_INVALID_ARG, "ranks=%d must be in 1..127", ranks);
+  if (w_dtype != BL_BF16 && w_dtype != BL_F32) return fail(BL_ERR_DTYPE, "w_dtype %d", (int)w_dtype);
+  if (!(lr - lr == 0.0f)) return fail(BL_ERR_INVALID_ARG, "lr must be finite");
+  if (!sign_words || !W || !w_packed || !gamma) return fail(BL_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(sign_words) || !aligned16(W) || !aligned16(w_packed) || !aligned16(gamma))
+    return fail(BL_ERR_ALIGNMENT, "sign_words, W, w_packed and gamma must be 16-byte aligned");
+  const size_t need = bl_quantize_weight_workspace_size(N, K);
+  if (!workspace || workspace_bytes < need || !aligned16(workspace))
+    return fail(BL_ERR_WORKSPACE, "workspace needs %zu bytes, 16-byte aligned", need);
+  int* err = nullptr;
+  if (bl_status s = current_device(&err)) return s;
+  return cuda_status(bl::launch_signsgd_apply(sign_words, ranks, W, w_dtype == BL_F32, N, K, lr, w_packed, gamma,
+                                              workspace, err, static_cast<cudaStream_t>(stream)),
+                     "bl_signsgd_apply");
+}
+
 bl_status bl_selftest_timeout(void* stream) {
   g_msg[0] = 0;
   int* err = nullptr;

@@ -30,6 +30,17 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 // Most CTAs of the sum launch of S1 (one fp64 partial sum each).
 constexpr int kMaxQuantCtas = 1024;
 
+// Workspace (each part on its own 128-byte lines): at 0 the arrivals at the
+// exact-sum barrier (u32); at 128 256 uint64 exact-sum bins (one per exponent
+// field); at 2304 one fp64 partial sum per CTA of the sum launch. The launch
+// that makes the partial sums (the sum launch, or the sign-gradient apply
+// pass) clears the first two parts and fills the third on every call, so the
+// caller's workspace needs no initialisation.
+constexpr size_t kWsArrive = 0;
+constexpr size_t kWsBins = 128;
+constexpr size_t kWsParts = kWsBins + 8 * 256 + 128;
+constexpr size_t kWsBytes = kWsParts + 8 * static_cast<size_t>(kMaxQuantCtas);
+
 // Bytes of the S1 workspace (exact-sum arrival counter and bins, one fp64
 // partial sum per CTA of the sum launch); the same for every tensor size.
 // Needs no initialisation.
@@ -50,6 +61,15 @@ cudaError_t launch_quantize_weight(const void* W, int w_is_f32, int64_t N, int64
 // S1 with the workspace in a fixed device array (g_noalloc_ws in k_quant.cu).
 cudaError_t launch_quantize_weight_noalloc(const void* W, int w_is_f32, int64_t N, int64_t K, uint8_t* packed,
                                            float* gamma, int* err, cudaStream_t s);
+
+// The code launch of S1 alone, for a W whose |W| partial sums another kernel
+// of the stream has just left in the workspace (nparts fp64 values at
+// kWsParts, bins and arrival counter cleared). part_roundings bounds the
+// roundings any term went through inside its partial sum (it sets the
+// enclosure of S that gamma is formed from).
+cudaError_t launch_quantize_codes(const void* W, int w_is_f32, int64_t N, int64_t K, int nparts,
+                                  double part_roundings, uint8_t* packed, float* gamma, void* workspace, int* err,
+                                  cudaStream_t s);
 
 // ---- S2 alone: per-token absmax INT8
 cudaError_t launch_quantize_act(const void* x, int64_t M, int64_t K, int8_t* xq, float* sx, cudaStream_t s);
@@ -76,6 +96,12 @@ cudaError_t launch_sign_vote(const uint32_t* words, int ranks, int64_t N, int64_
 // W [N,K] (bf16 or f32) <- dtype_rn(fp32(W) - lr * direction), in place.
 cudaError_t launch_signsgd_update(void* W, int w_is_f32, int64_t N, int64_t K, const uint8_t* direction, float lr,
                                   cudaStream_t s);
+
+// The holder's whole step in two launches: vote of `ranks` sign-word arrays,
+// the update of W in place, |W'| partial sums in the same sweep, then the
+// code launch of S1 (new packed codes and gamma of W').
+cudaError_t launch_signsgd_apply(const uint32_t* words, int ranks, void* W, int w_is_f32, int64_t N, int64_t K,
+                                 float lr, uint8_t* packed, float* gamma, void* workspace, int* err, cudaStream_t s);
 
 // One warp waiting on an mbarrier that is never completed (bounded wait test).
 cudaError_t launch_selftest_timeout(int* err, cudaStream_t s);

@@ -31,14 +31,12 @@
 #include <cmath>
 #include <cstdint>
 
+#include "bl_abs_sum.cuh"
 #include "bl_device.cuh"
 #include "bl_internal.h"
 
 namespace bl {
 namespace {
-
-__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
-__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
 // ---------------------------------------------------------------- S1 geometry
 constexpr int kSumThreads = 1024; // sum launch: 32 warps per CTA
@@ -49,64 +47,6 @@ constexpr int kCodeThreads = 512; // code launch: 16 warps per CTA
 constexpr int kCodeWarps = kCodeThreads / 32;
 constexpr int kCodeRowsPerCta = 10;// token rows a code-launch CTA quantises (< kCodeWarps)
 
-// Workspace (each part on its own 128-byte lines): at 0 the arrivals at the
-// exact-sum barrier (u32); at 128 256 uint64 exact-sum bins (one per exponent
-// field); at 2304 one fp64 partial sum per CTA of the sum launch. The sum
-// launch clears the first two parts and fills the third on every call, so the
-// caller's workspace needs no initialisation.
-constexpr size_t kWsArrive = 0;
-constexpr size_t kWsBins = 128;
-constexpr size_t kWsParts = kWsBins + 8 * 256 + 128;
-constexpr size_t kWsBytes = kWsParts + 8 * static_cast<size_t>(kMaxQuantCtas);
-
-// ---------------------------------------------------------------- |W| in fp64
-// |w| widened to fp64 exactly from its bit pattern with the sign cleared.
-// Normal values take integer arithmetic only (a bf16's fp64 high word is
-// b * 2^13 + 0x38000000: exponent re-bias 127 -> 1023; an fp32's is
-// (b >> 3) + 0x38000000 with low word b << 29); zeros and subnormals (zero
-// exponent field) take a separate, rarely taken path. Inputs are finite.
-//
-// 8 bf16 magnitudes of one 16-byte vector, added to acc in element order.
-__device__ __forceinline__ double add_abs8_bf16(double acc, const uint4& v) {
-  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-  uint32_t mn = 0xFFFFFFFFu;  // per half: smallest 15-bit magnitude
-#pragma unroll
-  for (int j = 0; j < 4; ++j) asm("min.u16x2 %0, %0, %1;" : "+r"(mn) : "r"(w[j] & 0x7FFF7FFFu));
-  if (min(mn << 16, mn & 0xFFFF0000u) >= 0x00800000u) {
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      acc = __dadd_rn(acc, __hiloint2double(static_cast<int>(((w[j] & 0x7FFFu) << 13) + 0x38000000u), 0));
-      acc = __dadd_rn(acc, __hiloint2double(static_cast<int>(((w[j] & 0x7FFF0000u) >> 3) + 0x38000000u), 0));
-    }
-    return acc;
-  }
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    acc = __dadd_rn(acc, static_cast<double>(fabsf(bf16_lo(w[j]))));
-    acc = __dadd_rn(acc, static_cast<double>(fabsf(bf16_hi(w[j]))));
-  }
-  return acc;
-}
-
-// 4 fp32 magnitudes of one 16-byte vector, added to acc in element order.
-__device__ __forceinline__ double add_abs4_f32(double acc, const uint4& v) {
-  const uint32_t w[4] = {v.x & 0x7FFFFFFFu, v.y & 0x7FFFFFFFu, v.z & 0x7FFFFFFFu, v.w & 0x7FFFFFFFu};
-  if (min(min(w[0], w[1]), min(w[2], w[3])) >= 0x00800000u) {
-#pragma unroll
-    for (int j = 0; j < 4; ++j)
-      acc = __dadd_rn(acc, __hiloint2double(static_cast<int>((w[j] >> 3) + 0x38000000u), static_cast<int>(w[j] << 29)));
-    return acc;
-  }
-#pragma unroll
-  for (int j = 0; j < 4; ++j) acc = __dadd_rn(acc, static_cast<double>(__uint_as_float(w[j])));
-  return acc;
-}
-
-template <bool kF32>
-__device__ __forceinline__ double add_abs(double acc, const uint4& v) {
-  if constexpr (kF32) return add_abs4_f32(acc, v);
-  else return add_abs8_bf16(acc, v);
-}
 
 // Exact-sum bins: bin e collects the integer significands (hidden bit
 // included; none for e = 0) of the elements whose exponent field is e, so
@@ -757,20 +697,58 @@ int blocks_per_sm(Kernel kernel, int threads, int (&cache)[64]) {
   return occ;
 }
 
+// Blocks of the code launch for W of `nvec` vectors: no more CTAs than can
+// be resident at once (the exact-sum barrier), and no more warps than rounds
+// of 128 vectors.
+template <bool kF32, int VPL>
+int64_t code_grid(int64_t nvec) {
+  static int occ_code[64] = {};
+  const int64_t nrounds = (nvec + 127) / 128;
+  const int64_t cap = device_sm_count() * blocks_per_sm(quant_code_kernel<kF32, VPL>, kCodeThreads, occ_code);
+  return std::max<int64_t>(1, std::min<int64_t>(cap, (nrounds + kCodeWarps - 1) / kCodeWarps));
+}
+
+// The code launch's arguments for W (`nvec` vectors, `numel` elements) whose
+// `nparts` partial sums are in the workspace, every term having passed
+// through at most `part_roundings` roundings inside its partial sum. No
+// token rows (the caller sets them).
+//
+// Enclosure of S around the fp64 sum: on top of those roundings the code
+// launch adds the ceil(nparts / 32) sequential partial sums of a lane and 5
+// butterfly levels. Each rounding is off by at most 2^-53 of a partial sum,
+// and with all terms >= 0 every partial sum is at most S (1 + 2^-30), so
+// |fp64 sum - S| <= d 2^-53 (1 + 2^-30) S; e = d 2^-52 (8 roundings to
+// spare) covers S on both sides.
+CodeArgs code_args(const void* W, int64_t nvec, int64_t numel, int nparts, double part_roundings, uint8_t* packed,
+                   float* gamma, uint8_t* ws, int* err) {
+  CodeArgs ca{};
+  ca.W = static_cast<const uint4*>(W);
+  ca.nvec = nvec;
+  ca.parts = reinterpret_cast<const double*>(ws + kWsParts);
+  ca.nparts = nparts;
+  ca.numel = static_cast<double>(numel);
+  ca.packed = reinterpret_cast<uint32_t*>(packed);
+  ca.gamma_out = gamma;
+  ca.ws = ws;
+  ca.err = err;
+  const double d = part_roundings + static_cast<double>((nparts + 31) / 32) + 5 + 8;
+  const double e = std::ldexp(d, -52);
+  ca.enc_lo = 1.0 - e;
+  ca.enc_hi = 1.0 + e;
+  return ca;
+}
+
 // The two launches of S1 (+ S2 when M > 0).
 template <bool kF32, int VPL>
 cudaError_t launch_s1(const void* W, int64_t N, int64_t K, const void* x, int64_t M, uint8_t* packed, float* gamma,
                       uint8_t* ws, int8_t* xq, float* sx, int* err, cudaStream_t s) {
   constexpr int kElems = kF32 ? 4 : 8;  // elements per 16-byte vector
-  static int occ_sum[64] = {}, occ_code[64] = {};
+  static int occ_sum[64] = {};
   const int64_t sms = device_sm_count();
   const int64_t nvec = N * K / kElems;
-  // code launch: no more CTAs than can be resident at once (the exact-sum
-  // barrier), and no more warps than rounds of 128 vectors; it takes up to
-  // kCodeRowsPerCta token rows per CTA (the rest go to the sum launch)
-  const int64_t nrounds = (nvec + 127) / 128;
-  const int64_t cap2 = sms * blocks_per_sm(quant_code_kernel<kF32, VPL>, kCodeThreads, occ_code);
-  const int64_t G2 = std::max<int64_t>(1, std::min<int64_t>(cap2, (nrounds + kCodeWarps - 1) / kCodeWarps));
+  // the code launch takes up to kCodeRowsPerCta token rows per CTA (the rest
+  // go to the sum launch)
+  const int64_t G2 = code_grid<kF32, VPL>(nvec);
   const int64_t M2 = std::min<int64_t>(M, G2 * kCodeRowsPerCta), M1 = M - M2;
 
   SumArgs sa{};
@@ -793,38 +771,20 @@ cudaError_t launch_s1(const void* W, int64_t N, int64_t K, const void* x, int64_
   const int64_t G1 = std::max<int64_t>(1, std::min(want1, cap1));
   sa.per = (nvec + G1 - 1) / G1;
 
-  CodeArgs ca{};
-  ca.W = sa.W;
-  ca.nvec = nvec;
-  ca.parts = sa.parts;
-  ca.nparts = static_cast<int>(G1);
-  ca.numel = static_cast<double>(N * K);
-  ca.packed = reinterpret_cast<uint32_t*>(packed);
-  ca.gamma_out = gamma;
-  ca.ws = ws;
-  ca.err = err;
+  // Roundings of a term inside its partial sum: its accumulator's sequential
+  // adds (kElems per vector, at most ceil(nj / 4) vectors of the thread's nj),
+  // the two levels joining the four accumulators, the 5 butterfly levels and
+  // the kSumWarps sequential warp sums.
+  const int64_t nj = kSumInterleave ? ((nvec + kSumThreads - 1) / kSumThreads + G1 - 1) / G1
+                                    : (sa.per + kSumThreads - 1) / kSumThreads;  // vectors per thread
+  const double part_roundings = static_cast<double>(kElems) * static_cast<double>((nj + 3) / 4) + 2 + 5 + kSumWarps;
+  CodeArgs ca = code_args(W, nvec, N * K, static_cast<int>(G1), part_roundings, packed, gamma, ws, err);
   ca.x = sa.x;
   ca.m_begin = M1;
   ca.M2 = M2;
   ca.nv = sa.nv;
   ca.xq = xq;
   ca.sx = sx;
-  // Enclosure of S around the fp64 sum. Every |w| passes through at most d
-  // roundings: its accumulator's sequential adds (kElems per vector, at most
-  // ceil(nj / 4) vectors of the thread's nj), the two levels joining the four
-  // accumulators, the 5 butterfly levels, the kSumWarps sequential warp sums,
-  // the ceil(G1 / 32) sequential partial sums of a lane and the 5 butterfly
-  // levels of the code launch. Each rounding is off by at most 2^-53 of a
-  // partial sum, and with all terms >= 0 every partial sum is at most
-  // S (1 + 2^-30), so |fp64 sum - S| <= d 2^-53 (1 + 2^-30) S; e = d 2^-52
-  // (8 roundings to spare) covers S on both sides.
-  const int64_t nj = kSumInterleave ? ((nvec + kSumThreads - 1) / kSumThreads + G1 - 1) / G1
-                                    : (sa.per + kSumThreads - 1) / kSumThreads;  // vectors per thread
-  const double d = static_cast<double>(kElems) * static_cast<double>((nj + 3) / 4) + 2 + 5 + kSumWarps +
-                   static_cast<double>((G1 + 31) / 32) + 5 + 8;
-  const double e = std::ldexp(d, -52);
-  ca.enc_lo = 1.0 - e;
-  ca.enc_hi = 1.0 + e;
 
   cudaError_t st = launch_pdl(quant_sum_kernel<kF32, VPL>, dim3(static_cast<unsigned>(G1)), dim3(kSumThreads), 0, s, sa);
   if (st != cudaSuccess) return st;
@@ -870,6 +830,22 @@ cudaError_t launch_quantize(const void* W, int w_is_f32, int64_t N, int64_t K, c
 cudaError_t launch_quantize_weight(const void* W, int w_is_f32, int64_t N, int64_t K, uint8_t* packed,
                                    float* gamma, void* workspace, int* err, cudaStream_t s) {
   return launch_quantize(W, w_is_f32, N, K, nullptr, 0, packed, gamma, workspace, nullptr, nullptr, err, s);
+}
+
+cudaError_t launch_quantize_codes(const void* W, int w_is_f32, int64_t N, int64_t K, int nparts,
+                                  double part_roundings, uint8_t* packed, float* gamma, void* workspace, int* err,
+                                  cudaStream_t s) {
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const int64_t nvec = N * K / (w_is_f32 ? 4 : 8);
+  const CodeArgs ca = code_args(W, nvec, N * K, nparts, part_roundings, packed, gamma, ws, err);
+  const dim3 block(kCodeThreads);
+  cudaError_t e = w_is_f32
+                      ? launch_pdl(quant_code_kernel<true, 0>, dim3(static_cast<unsigned>(code_grid<true, 0>(nvec))),
+                                   block, 0, s, ca)
+                      : launch_pdl(quant_code_kernel<false, 0>, dim3(static_cast<unsigned>(code_grid<false, 0>(nvec))),
+                                   block, 0, s, ca);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
 }
 
 // Device address of g_noalloc_ws on the current device. Host code only holds

@@ -11,9 +11,11 @@ One step, entered by every rank in the same order:
      by the backward itself with ``bl_backward_signs``; N*K/8 bytes)
   2. gather of the R ranks' words on the holder (torch.distributed; NCCL on
      GPUs, each rank sends N*K/8 bytes)
-  3. holder: majority vote (``bl_sign_vote``), the update of W
-     (``bl_signsgd_update``) and its new codes and gamma
-     (``bl_quantize_weight``)
+  3. holder: majority vote, the update of W and its new codes and gamma
+     (``bl_signsgd_apply``: two launches, the vote, update and |W| sums in
+     one sweep over W; or the three calls ``bl_sign_vote``,
+     ``bl_signsgd_update``, ``bl_quantize_weight`` when ``SignOps.apply`` is
+     None)
   4. broadcast of the new w_packed and gamma from the holder (N*K/4 + 4 bytes)
 
 Only argument marshalling and the order of the collectives live here; every
@@ -39,12 +41,16 @@ class SignOps:
     sign_vote: Callable = field(default=b.bl_sign_vote)
     update: Callable = field(default=b.bl_signsgd_update)
     quantize_weight: Callable = field(default=b.bl_quantize_weight)
+    # the holder's vote + update + new codes in one call (None: the three
+    # separate calls above)
+    apply: Callable | None = field(default=b.bl_signsgd_apply)
 
 
 @dataclass
 class SignBuffers:
     """Scratch of one layer's step: this rank's words, and on the holder the
-    gathered words of every rank and the vote's direction."""
+    gathered words of every rank and the vote's direction (used only by the
+    three-call form of the holder's step)."""
     words: torch.Tensor
     gathered: torch.Tensor | None
     direction: torch.Tensor | None
@@ -96,9 +102,12 @@ def signsgd_dp_step(dW, w_packed, gamma, lr, *, master_W=None, workspace=None, h
     else:
         votes = words.unsqueeze(0)
     if is_holder:
-        ops.sign_vote(votes, buf.direction)
-        ops.update(master_W, buf.direction, lr)
-        ops.quantize_weight(master_W, w_packed, gamma, workspace)
+        if ops.apply is not None:
+            ops.apply(votes, master_W, lr, w_packed, gamma, workspace)
+        else:
+            ops.sign_vote(votes, buf.direction)
+            ops.update(master_W, buf.direction, lr)
+            ops.quantize_weight(master_W, w_packed, gamma, workspace)
     if world > 1:
         dist.broadcast(w_packed, src=holder)
         dist.broadcast(gamma, src=holder)

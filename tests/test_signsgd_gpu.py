@@ -224,3 +224,83 @@ def test_single_rank_step_from_fused_sign_words():
     assert np.array_equal(results[0][0], results[1][0])
     assert np.array_equal(results[0][1], results[1][1])
     assert results[0][2] == results[1][2]
+
+
+def _rank_words(ranks, shape, seed):
+    """ranks sign-word arrays [R, N, K/32] int32 of random bits."""
+    g = torch.Generator().manual_seed(seed)
+    n, k = shape
+    return torch.randint(-2 ** 31, 2 ** 31, (ranks, n, k // 32), generator=g, dtype=torch.int64).to(torch.int32)
+
+
+@pytest.mark.parametrize("ranks,shape,w_dtype", [(1, (3, 96), torch.bfloat16), (3, (33, 2560), torch.bfloat16),
+                                                 (8, (1000, 160), torch.bfloat16), (2, (6912, 2560), torch.bfloat16),
+                                                 (1, (6912, 2560), torch.bfloat16), (127, (5, 64), torch.float32),
+                                                 (3, (96, 320), torch.float32), (4, (2560, 1024), torch.float32)])
+def test_apply_matches_the_three_calls_and_the_oracle(ranks, shape, w_dtype):
+    """bl_signsgd_apply (vote, update and |W| sums in one sweep, then the code
+    launch) leaves W, w_packed and gamma bit for bit as bl_sign_vote,
+    bl_signsgd_update and bl_quantize_weight in turn do, and as the oracle
+    chain; twice in a row on the same workspace."""
+    bl = _bl()
+    n, k = shape
+    g = torch.Generator().manual_seed(21 + ranks)
+    master = (torch.randn(shape, generator=g) * 0.02).to(w_dtype)
+    lr = 2.0 ** -9
+    ws = torch.empty(bl.bl_quantize_weight_workspace_size(n, k), dtype=torch.uint8, device="cuda")
+    ws.fill_(0x5C)
+    w_a, w_b = master.cuda(), master.cuda()
+    direction = torch.empty((n, k // 4), dtype=torch.uint8, device="cuda")
+    outs = []
+    for step in range(2):
+        words = _rank_words(ranks, shape, seed=100 * step + ranks).cuda()
+        pa = torch.full((n, k // 4), 0xAA, dtype=torch.uint8, device="cuda")
+        ga = torch.full((1,), -1.0, dtype=torch.float32, device="cuda")
+        pb, gb = pa.clone(), ga.clone()
+        bl.bl_signsgd_apply(words, w_a, lr, pa, ga, ws)
+        bl.bl_sign_vote(words, direction)
+        bl.bl_signsgd_update(w_b, direction, lr)
+        bl.bl_quantize_weight(w_b, pb, gb, ws)
+        torch.cuda.synchronize()
+        assert bl.bl_get_last_error() == 0
+        assert torch.equal(w_a.view(torch.int16 if w_dtype == torch.bfloat16 else torch.int32),
+                           w_b.view(torch.int16 if w_dtype == torch.bfloat16 else torch.int32)), step
+        assert torch.equal(pa, pb) and ga.cpu().numpy().tobytes() == gb.cpu().numpy().tobytes(), step
+        outs.append((words.cpu(), pa.cpu(), ga.cpu()))
+    if n * k > 1 << 22:
+        return  # the oracle chain runs on the smaller shapes
+    w = _as_f32(master)
+    for words, pa, ga in outs:
+        d = sg.majority_direction([x.numpy().view(np.uint32) for x in words])
+        w = sg.signsgd_update(w, d, lr, w_is_bf16=w_dtype == torch.bfloat16)
+        if w_dtype == torch.bfloat16:
+            w = ref.bf16_bits_to_f32(ref.round_to_bf16_bits(w))
+        codes, gm = ref.ternarize(w)
+        assert float(ga[0]) == float(gm)
+        assert np.array_equal(pa.numpy(), ref.pack_ternary(codes))
+
+
+@pytest.mark.parametrize("case,expected", [("tie", 1.0), ("above", 1.0 + 2.0 ** -23), ("below", 1.0)])
+@pytest.mark.parametrize("w_dtype", [torch.bfloat16, torch.float32])
+def test_apply_exact_gamma_at_an_fp32_midpoint(case, expected, w_dtype):
+    """Two ranks voting opposite signs everywhere leave W unchanged (a tie
+    moves nothing), so on a W whose mean |W| sits on or 2^-44 off the fp32
+    midpoint 1 + 2^-24 the code launch must take the exact integer sum after
+    the fused sweep's partial sums too: gamma and codes bit-exact."""
+    from workloads import gamma_midpoint_weights
+    bl = _bl()
+    w = gamma_midpoint_weights(case, w_dtype)
+    n, k = w.shape
+    codes, gm = ref.ternarize(w.float().numpy())
+    assert gm == np.float32(expected)
+    words = torch.stack([torch.full((n, k // 32), -1, dtype=torch.int32), torch.zeros((n, k // 32), dtype=torch.int32)])
+    wd = w.cuda()
+    packed = torch.full((n, k // 4), 0xAA, dtype=torch.uint8, device="cuda")
+    gamma = torch.full((1,), -1.0, dtype=torch.float32, device="cuda")
+    ws = torch.empty(bl.bl_quantize_weight_workspace_size(n, k), dtype=torch.uint8, device="cuda")
+    bl.bl_signsgd_apply(words.cuda(), wd, 2.0 ** -4, packed, gamma, ws)
+    torch.cuda.synchronize()
+    assert bl.bl_get_last_error() == 0
+    assert torch.equal(wd.cpu(), w)
+    assert gamma.cpu().numpy()[0].tobytes() == np.float32(expected).tobytes()
+    np.testing.assert_array_equal(packed.cpu().numpy(), ref.pack_ternary(codes))

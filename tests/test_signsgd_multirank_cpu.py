@@ -37,7 +37,9 @@ def _master():
     return (torch.randn((N, K), generator=g) * 0.05).to(torch.float32)
 
 
-def _oracle_ops():
+def _oracle_ops(fused=False):
+    """The oracle in place of the device calls; fused: the holder's vote,
+    update and new codes as one call (the form ``bl_signsgd_apply`` takes)."""
     from ternary_weight_quantization_b200.signsgd import SignOps
 
     def sign_pack(dW, words):
@@ -56,7 +58,13 @@ def _oracle_ops():
         w_packed.copy_(torch.from_numpy(ref.pack_ternary(codes)))
         gamma[0] = float(g)
 
-    return SignOps(sign_pack=sign_pack, sign_vote=sign_vote, update=update, quantize_weight=quantize_weight)
+    def apply(gathered, W, lr, w_packed, gamma, workspace):
+        d = sg.majority_direction([w.numpy().view(np.uint32) for w in gathered])
+        W.copy_(torch.from_numpy(sg.signsgd_update(W.numpy(), d, lr, w_is_bf16=False)))
+        quantize_weight(W, w_packed, gamma, workspace)
+
+    return SignOps(sign_pack=sign_pack, sign_vote=sign_vote, update=update, quantize_weight=quantize_weight,
+                   apply=apply if fused else None)
 
 
 def _expected(world):
@@ -71,7 +79,7 @@ def _words(rank):
     return torch.from_numpy(sg.sign_bits(_grad(rank).float().numpy()).view(np.int32).copy())
 
 
-def _worker(rank, world, port, holder, out, with_words=False):
+def _worker(rank, world, port, holder, out, with_words=False, fused=False):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     torch.distributed.init_process_group("gloo", rank=rank, world_size=world,
                                          timeout=datetime.timedelta(seconds=60))
@@ -81,22 +89,25 @@ def _worker(rank, world, port, holder, out, with_words=False):
         gamma = torch.zeros(1, dtype=torch.float32)
         kw = dict(master_W=_master(), workspace=torch.empty(64, dtype=torch.uint8)) if rank == holder else {}
         if with_words:
-            signsgd_dp_step(None, w_packed, gamma, LR, holder=holder, ops=_oracle_ops(), words=_words(rank), **kw)
+            signsgd_dp_step(None, w_packed, gamma, LR, holder=holder, ops=_oracle_ops(fused), words=_words(rank), **kw)
         else:
-            signsgd_dp_step(_grad(rank), w_packed, gamma, LR, holder=holder, ops=_oracle_ops(), **kw)
+            signsgd_dp_step(_grad(rank), w_packed, gamma, LR, holder=holder, ops=_oracle_ops(fused), **kw)
         out[rank] = (w_packed.numpy().tobytes(), float(gamma[0]))
     finally:
         torch.distributed.destroy_process_group()
 
 
-@pytest.mark.parametrize("world,holder,with_words", [(2, 0, False), (3, 1, False), (2, 1, True)])
-def test_ranks_end_with_the_holders_codes(world, holder, with_words):
+@pytest.mark.parametrize("world,holder,with_words,fused",
+                         [(2, 0, False, False), (3, 1, False, True), (2, 1, True, False), (3, 2, True, True)])
+def test_ranks_end_with_the_holders_codes(world, holder, with_words, fused):
     """Every rank ends with the oracle chain's codes and gamma, whether it
-    hands over dW (packed here) or the sign words a fused backward made."""
+    hands over dW (packed here) or the sign words a fused backward made, and
+    whether the holder takes the three calls or the fused one."""
     ctx = mp.get_context("spawn")
     out = ctx.Manager().dict()
     port = _free_port()
-    procs = [ctx.Process(target=_worker, args=(r, world, port, holder, out, with_words)) for r in range(world)]
+    procs = [ctx.Process(target=_worker, args=(r, world, port, holder, out, with_words, fused))
+             for r in range(world)]
     for p in procs:
         p.start()
     for p in procs:
