@@ -18,7 +18,10 @@
 // 128 A rows from the staged 2-bit / INT8 source (never written to HBM) and
 // TMA-loads its own BN/2 B rows; the leader CTA issues one M=256 MMA that
 // reads both CTAs' shared memory and accumulates 128 rows into each CTA's
-// TMEM. No TMA multicast is used.
+// TMEM. No TMA multicast is used. Forward tiles wider than one MMA (BN = 320,
+// for shapes with a few more tiles than pairs) issue two MMAs per step on the
+// same A -- columns 0..255 and 256..BN-1 -- into one accumulator of BN
+// columns (the two-buffer overlap of epilogue and MMAs needs BN <= 256).
 //
 // The forward family runs one GEMM per launch. The backward family runs dX
 // and dW in ONE launch: the two GEMMs' tiles (different lengths: N/64 and M/64
@@ -30,7 +33,7 @@
 //   warp 0      loads: TMA for B, for Dw's q / s_x and for the packed codes
 //               (cp.async for the codes when K % 64 != 0: their rows are then
 //               not 16-byte aligned, which a tensor map requires)
-//   warp 1      TMEM allocation (2 x 256 columns, pair-wide); in the leader
+//   warp 1      TMEM allocation (512 columns, pair-wide); in the leader
 //               CTA one lane issues the tcgen05.mma
 //   warps 2-4, 6-8, 10-11  rebuild A from the staged source, in two groups
 //               of four taking alternate stages
@@ -86,13 +89,24 @@ __device__ __forceinline__ int rebuild_slot(int w) {
 }
 
 constexpr int BM = 128;              // A rows per CTA; a pair covers 2 * BM
-constexpr uint32_t kTmemCols = 512;  // two accumulators at columns 0 and 256
+constexpr uint32_t kTmemCols = 512;  // two accumulators at columns 0 and 256 (one of BN for BN > 256)
 constexpr int kSmemLimit = 232448;           // per-CTA dynamic shared memory on sm_100
 constexpr int kMaxPairs = 128;
 constexpr int kMaxSchedTiles = 2048;
 
 enum class Op { Fwd, Dx, Dw };
 enum class Family { Fwd, Bwd };
+
+// TMEM accumulators a pair cycles through: two of 256 columns, or one of BN
+// columns for the wide forward tiles.
+template <int BN>
+constexpr int kAccBufs = BN > 256 ? 1 : 2;
+// Wide forward tiles: this CTA's B rows 0..127 hold tokens bp + 128 r + (0..127)
+// (the first MMA's half for rank r) and rows 128..BN/2-1 hold tokens
+// bp + 256 + (BN/2 - 128) r + ..., so accumulator column c is token bp + c;
+// they arrive in boxes of BN/2 - 128 rows.
+template <int BN>
+constexpr int kWideBox = BN > 256 ? BN / 2 - 128 : BN / 2;
 
 // Stage geometry of a family. Every op issues four MMAs per stage.
 template <Family F, int BN>
@@ -104,7 +118,7 @@ struct Geo;
 template <int BN>
 struct Geo<Family::Fwd, BN> {
   static constexpr int kEpiSlots = 4;
-  static constexpr int kEpiScaleBytes = 256 * 4;  // s_x[m] * gamma of the tile's columns
+  static constexpr int kEpiScaleBytes = (BN > 256 ? BN : 256) * 4;  // s_x[m] * gamma of the tile's columns
   static constexpr int kBlockR = 128;
   static constexpr int kABytes = BM * 128;         // 128 rows x 128 int8
   static constexpr int kBBytes = (BN / 2) * 128;   // BN/2 rows x 128 int8
@@ -134,7 +148,10 @@ template <Op op, int BN>
 struct MmaCfg;
 template <int BN>
 struct MmaCfg<Op::Fwd, BN> {
-  static constexpr uint32_t kIdesc = make_idesc(2 /*s32*/, 1 /*s8*/, 0, 0, 2 * BM, BN);
+  // BN > 256: one MMA of N = 256, then one of N = BN - 256 on B rows 128.. of
+  // each CTA (columns 256.. of the accumulator)
+  static constexpr uint32_t kIdesc = make_idesc(2 /*s32*/, 1 /*s8*/, 0, 0, 2 * BM, BN > 256 ? 256 : BN);
+  static constexpr uint32_t kIdesc2 = make_idesc(2, 1, 0, 0, 2 * BM, BN > 256 ? BN - 256 : 16);
   static constexpr uint32_t kLboA = 16, kLboB = 16;
   static constexpr uint64_t kStepA = 2, kStepB = 2;  // 32 bytes of K (K-major)
 };
@@ -346,7 +363,7 @@ struct Maps {
 // which expects one arrival).
 template <Op op, Family F, int BN>
 __device__ __forceinline__ void load_stage(const GemmParams& p, const OpParams& P, const Maps& m, bool leader,
-                                           int lane, int a0, int bh, int kb, uint64_t* full, uint32_t full_lead,
+                                           int lane, int a0, int bp, int bh, int kb, uint64_t* full, uint32_t full_lead,
                                            uint64_t* src_full, uint8_t* sB, uint8_t* sSrc, uint8_t* sSx) {
   using G = Geo<F, BN>;
   const int r0 = kb * G::kBlockR;
@@ -360,7 +377,16 @@ __device__ __forceinline__ void load_stage(const GemmParams& p, const OpParams& 
       tma_load_2d(m.src, src_full, sSrc, a0, r0);
       tma_load_2d(m.sx, src_full, sSx, r0, 0);
     } else {
-      tma_load_2d_pair(m.b, full_lead, sB, r0, bh);
+      if constexpr (op == Op::Fwd && BN > 256) {
+        static_assert(128 % kWideBox<BN> == 0, "the first MMA's rows come in whole boxes");
+        const int r = (bh - bp) / (BN / 2);  // rank of this CTA
+#pragma unroll
+        for (int t = 0; t < 128 / kWideBox<BN>; ++t)
+          tma_load_2d_pair(m.b, full_lead, sB + t * kWideBox<BN> * 128, r0, bp + 128 * r + t * kWideBox<BN>);
+        tma_load_2d_pair(m.b, full_lead, sB + 128 * 128, r0, bp + 256 + kWideBox<BN> * r);
+      } else {
+        tma_load_2d_pair(m.b, full_lead, sB, r0, bh);
+      }
       if (P.src_tma) {
         // packed codes as one TMA box: Fwd rows a0..a0+127 x bytes [kb*32, +32);
         // Dx rows (n) r0..r0+63 x bytes [a0/4, +32)
@@ -449,7 +475,7 @@ __device__ __forceinline__ void rebuild_stage(int rt, uint32_t sA, uint32_t sSrc
   }
 }
 
-// MMA lane, one stage: four pair MMAs.
+// MMA lane, one stage: four pair MMAs (eight for the wide forward tiles).
 template <Op op, int BN>
 __device__ __forceinline__ void mma_stage(uint32_t d_tmem, uint32_t sa, uint32_t sb, int kb) {
   using M = MmaCfg<op, BN>;
@@ -458,9 +484,13 @@ __device__ __forceinline__ void mma_stage(uint32_t d_tmem, uint32_t sa, uint32_t
 #pragma unroll
   for (int kk = 0; kk < 4; ++kk) {
     const uint32_t acc = (kb | kk) != 0;
-    if constexpr (op == Op::Fwd)
+    if constexpr (op == Op::Fwd) {
       mma_i8_pair(d_tmem, ad + kk * M::kStepA, bd + kk * M::kStepB, M::kIdesc, acc);
-    else
+      if constexpr (BN > 256) {
+        const uint64_t bd2 = smem_desc_sw128(sb + 128 * 128, M::kLboB, 1024);
+        mma_i8_pair(d_tmem + 256, ad + kk * M::kStepA, bd2 + kk * M::kStepB, M::kIdesc2, acc);
+      }
+    } else
       mma_f16_pair(d_tmem, ad + kk * M::kStepA, bd + kk * M::kStepB, M::kIdesc, acc);
   }
 }
@@ -793,10 +823,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         uint8_t* sSrc = smem + L::kOffSrc + stage * G::kSrcBytes;
         uint8_t* sSx = smem + L::kOffSx + stage * G::kSxBytes;
         if (t.opi == 0)
-          load_stage<kOp0, F, BN>(p, P, maps0, leader, lane, t.a0, bh, kb, &full[stage], lead(&full[stage]),
+          load_stage<kOp0, F, BN>(p, P, maps0, leader, lane, t.a0, t.bp, bh, kb, &full[stage], lead(&full[stage]),
                                   &src_full[stage], sB, sSrc, sSx);
         else if constexpr (F == Family::Bwd)
-          load_stage<Op::Dw, F, BN>(p, P, maps1, leader, lane, t.a0, bh, kb, &full[stage], lead(&full[stage]),
+          load_stage<Op::Dw, F, BN>(p, P, maps1, leader, lane, t.a0, t.bp, bh, kb, &full[stage], lead(&full[stage]),
                                     &src_full[stage], sB, sSrc, sSx);
         if (++stage == S) {
           stage = 0;
@@ -850,7 +880,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             phase ^= 1;
           }
         }
-        if (++buf == 2) {
+        if (++buf == kAccBufs<BN>) {
           buf = 0;
           buf_phase ^= 1;
         }
@@ -939,7 +969,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           epilogue_tile<Op::Dw, BN, G::kEpiSlots>(p, P, &map_out1, tmem_base, buf, stg, lane, q, t.a0, t.bp, gamma,
                                                   pb, ps, !last, lead(&tmem_empty[buf]), seq);
       }
-      if (++buf == 2) {
+      if (++buf == kAccBufs<BN>) {
         buf = 0;
         buf_phase ^= 1;
       }
@@ -1477,19 +1507,29 @@ bool make_out_map(CUtensorMap* m, void* base, bool f32, int64_t rows, int64_t co
                      cols * (f32 ? 4 : 2), 32, 32, CU_TENSOR_MAP_SWIZZLE_NONE, what);
 }
 
-// B rows per pair tile for the forward: the candidate with the fewest
-// tile-rows of work per pair after wave quantisation (waves x BN), ties to
-// the larger tile.
-int choose_bn(int rows_a, int rows_b, int npairs, const int* cands, int ncands) {
-  const int tiles_a = (rows_a + 2 * BM - 1) / (2 * BM);
-  int best = cands[0];
+// B rows per pair tile for the forward: the candidate with the least
+// estimated time, rounds x (k-blocks x stage time + tile overhead), where a
+// round is one tile on every pair. The stage and tile times are per-BN
+// weights measured on B200 (ns, CUDA graphs of the up- and down-projection
+// forwards): up to 256 columns a stage takes ~0.42-0.45 us and the
+// epilogue overlaps the next tile; the 320-column tile's second MMA and
+// single accumulator cost more per stage and expose its epilogue, so it wins
+// only where it saves a round (the down-projection: 70 tiles in one round
+// against 80 in two).
+struct BnCost {
+  int bn, stage_ns, tile_ns;
+};
+int choose_bn(int rows_a, int rows_b, int red, int npairs, const BnCost* cands, int ncands) {
+  const long long tiles_a = (rows_a + 2 * BM - 1) / (2 * BM);
+  const long long kb = (red + 127) / 128;
+  int best = cands[0].bn;
   long long best_cost = -1;
   for (int i = 0; i < ncands; ++i) {
-    const int bn = cands[i];
-    const long long tiles = static_cast<long long>(tiles_a) * ((rows_b + bn - 1) / bn);
-    const long long cost = ((tiles + npairs - 1) / npairs) * bn;
+    const long long tiles = tiles_a * ((rows_b + cands[i].bn - 1) / cands[i].bn);
+    const long long rounds = (tiles + npairs - 1) / npairs;
+    const long long cost = rounds * (kb * cands[i].stage_ns + cands[i].tile_ns);
     if (best_cost < 0 || cost < best_cost) {
-      best = bn;
+      best = cands[i].bn;
       best_cost = cost;
     }
   }
@@ -1532,11 +1572,12 @@ cudaError_t launch_forward(const int8_t* xq, const float* sx, const uint8_t* w_p
     const int m = static_cast<int>(M), nn = static_cast<int>(N), kk = static_cast<int>(K);
     return launch_few_slots(slots, xq, sx, w_packed, gamma, m, nn, kk, y, debug_acc, s);
   }
-  static const int kCands[3] = {256, 192, 128};
+  static const BnCost kCands[4] = {{256, 450, 500}, {320, 680, 2800}, {192, 445, 500}, {128, 420, 500}};
   const int npairs = resident_pairs<Family::Fwd, 256>();
-  const int bn = choose_bn(static_cast<int>(N), static_cast<int>(M), npairs, kCands, 3);
+  const int bn = choose_bn(static_cast<int>(N), static_cast<int>(M), static_cast<int>(K), npairs, kCands, 4);
   CUtensorMap maps[7] = {};  // b0, src0, out0, b1, src1, out1, sx
-  if (!make_map_2d(&maps[0], xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, K, M, K, 128, bn / 2, CU_TENSOR_MAP_SWIZZLE_128B,
+  const int box_rows = bn > 256 ? bn / 2 - 128 : bn / 2;  // wide tiles load B in several boxes
+  if (!make_map_2d(&maps[0], xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, K, M, K, 128, box_rows, CU_TENSOR_MAP_SWIZZLE_128B,
                    "xq"))
     return cudaErrorInvalidValue;
   // y [M][N] bf16 by TMA stores when its rows are 16-byte multiples
@@ -1560,6 +1601,7 @@ cudaError_t launch_forward(const int8_t* xq, const float* sx, const uint8_t* w_p
   p.gamma = gamma;
   p.debug_acc = debug_acc;
   p.err = err;
+  if (bn == 320) return launch_pair<Family::Fwd, 320>(maps, p, npairs, s);
   if (bn == 256) return launch_pair<Family::Fwd, 256>(maps, p, npairs, s);
   if (bn == 192) return launch_pair<Family::Fwd, 192>(maps, p, npairs, s);
   return launch_pair<Family::Fwd, 128>(maps, p, npairs, s);

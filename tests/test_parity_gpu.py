@@ -470,3 +470,33 @@ def test_forward_few_tokens_shapes(M, N, K):
     acc_o = ref.forward_accumulate(q, codes)
     np.testing.assert_array_equal(acc.cpu().numpy(), acc_o)
     np.testing.assert_array_equal(bits(bufs.y), ref.round_to_bf16_bits(ref.forward_output(acc_o, sx, gamma)))
+
+
+@pytest.mark.parametrize("M,N,K", [(2000, 2500, 2560), (2048, 2560, 6912), (2400, 2200, 4096)])
+def test_forward_wide_tiles(M, N, K):
+    """Shapes with a few more 256-column tiles than CTA pairs take the
+    320-column forward tiles (two MMAs per step into one accumulator, tokens
+    in five boxes per CTA): INT32 sums and y (through the debug path and
+    through the TMA-store path) bit-exact on sampled token rows, ragged
+    tokens and features included."""
+    bl = _bl()
+    x, w, _ = make_inputs(M, K, N, seed=70 + M)
+    bufs = bl.StepBuffers.allocate(M, N, K)
+    acc = torch.empty((M, N), dtype=torch.int32, device="cuda")
+    y2 = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    bl.bl_quantize_weight(w.cuda(), bufs.w_packed, bufs.gamma, bufs.workspace)
+    bl.bl_quantize_act(x.cuda(), bufs.xq, bufs.sx)
+    bl.bl_forward(bufs.xq, bufs.sx, bufs.w_packed, bufs.gamma, bufs.y, acc)
+    bl.bl_forward(bufs.xq, bufs.sx, bufs.w_packed, bufs.gamma, y2)
+    torch.cuda.synchronize()
+    assert bl.bl_get_last_error() == 0
+    codes, gamma = ref.ternarize(ref.bf16_bits_to_f32(bits(w)))
+    q, sx = ref.quantize_activations(ref.bf16_bits_to_f32(bits(x)))
+    # every 320-token tile's first and last rows, and a random sample
+    rows = np.unique(np.concatenate([np.arange(0, M, 320), np.minimum(np.arange(319, M + 319, 320), M - 1),
+                                     _sample(M, 64, 3)]))
+    acc_o = ref.forward_accumulate(q[rows], codes)
+    np.testing.assert_array_equal(acc.cpu().numpy()[rows], acc_o)
+    y_o = ref.round_to_bf16_bits(ref.forward_output(acc_o, sx[rows], gamma))
+    np.testing.assert_array_equal(bits(bufs.y)[rows], y_o)
+    np.testing.assert_array_equal(bits(y2)[rows], y_o)
