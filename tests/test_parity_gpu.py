@@ -472,13 +472,14 @@ def test_forward_few_tokens_shapes(M, N, K):
     np.testing.assert_array_equal(bits(bufs.y), ref.round_to_bf16_bits(ref.forward_output(acc_o, sx, gamma)))
 
 
-@pytest.mark.parametrize("M,N,K", [(2000, 2500, 2560), (2048, 2560, 6912), (2400, 2200, 4096)])
+@pytest.mark.parametrize("M,N,K", [(2000, 2500, 2560), (2048, 2560, 6912), (2400, 2200, 4096), (2000, 2500, 2592)])
 def test_forward_wide_tiles(M, N, K):
     """Shapes with a few more 256-column tiles than CTA pairs take the
     320-column forward tiles (two MMAs per step into one accumulator, tokens
     in five boxes per CTA): INT32 sums and y (through the debug path and
     through the TMA-store path) bit-exact on sampled token rows, ragged
-    tokens and features included."""
+    tokens and features included; K = 2592 (K % 64 != 0) stages the packed
+    codes by cp.async and ends on a partial k-block."""
     bl = _bl()
     x, w, _ = make_inputs(M, K, N, seed=70 + M)
     bufs = bl.StepBuffers.allocate(M, N, K)
