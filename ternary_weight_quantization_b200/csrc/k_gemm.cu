@@ -11,7 +11,7 @@
 //
 //   op   A (REBUILT in smem)                    B (TMA)                       r
 //   Fwd  codes[n][k] int8, K-major              xq[m][k] int8, K-major        k
-//   Dx   codes^T[k][n] bf16 {-1,0,1}, MN-major  dY[m][n] bf16, K-major        n
+//   Dx   2 codes^T[k][n] bf16 {-2,0,2}, MN-major dY[m][n] bf16, K-major        n
 //   Dw   x_hat^T[k][m] bf16, MN-major           dY^T[n][m] bf16, MN-major     m
 //
 // A pair tile is 256 A rows x BN B rows. Each CTA of the pair rebuilds its own
@@ -279,21 +279,20 @@ __device__ __forceinline__ uint4 codes16_to_s8(uint32_t w) {
   return r;
 }
 
-// 8 packed codes (16 bits) -> 8 bf16 values in {-1, 0, +1}.
-// Field bit 0 marks a nonzero code and bit 1 a negative one, so each bf16 is
-// b0 * 0x3F80 + b1 * 0x8000; two codes are handled per 32-bit word.
-__device__ __forceinline__ uint4 codes8_to_bf16(uint32_t h) {
+// 8 packed codes (16 bits) -> 8 bf16 values 2 * code in {-2, 0, +2}. With
+// the factor 2 the map is linear in the 2-bit field: bf16 2.0 is 0x4000 and
+// -2.0 is 0xC000, i.e. field f in {0, 1, 3} -> f * 0x4000, so each field only
+// moves to bits 14-15 of its half (one shift and one mask per two codes). The
+// dX epilogue scales by gamma / 2 (exact), and (2 acc) * (gamma / 2) is
+// acc * gamma exactly, so dX is unchanged: every product and partial sum of
+// the doubled operand is exactly twice the plain one.
+__device__ __forceinline__ uint4 codes8_to_bf16x2(uint32_t h) {
   h &= 0xFFFFu;
-  const uint32_t s = h | (h << 14);  // field 2w at bits 4w.., field 2w+1 at bits 4w+16..
-  uint32_t r[4];
-#pragma unroll
-  for (int w = 0; w < 4; ++w) {
-    const uint32_t g = s >> (4 * w);
-    const uint32_t nz = g & 0x00010001u;
-    const uint32_t neg = (g << 14) & 0x80008000u;
-    r[w] = nz * 0x3F80u + neg;
-  }
-  return make_uint4(r[0], r[1], r[2], r[3]);
+  // field 2w at bits 4w, 4w+1; field 2w+1 at bits 4w+16, 4w+17 (bits 14-15
+  // hold two fields at once but are never selected)
+  const uint32_t s = h | (h << 14);
+  return make_uint4((s << 14) & 0xC000C000u, (s << 10) & 0xC000C000u, (s << 6) & 0xC000C000u,
+                    (s << 2) & 0xC000C000u);
 }
 
 // 16 int8 (x_hat source) * s -> 16 bf16, each bf16_rn(fp32(q) * s).
@@ -455,7 +454,7 @@ __device__ __forceinline__ void rebuild_stage(int rt, uint32_t sA, uint32_t sSrc
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       const uint32_t hw = words[j >> 1] >> ((j & 1) * 16);
-      st_shared_v4(base + ((j ^ (n & 7)) << 4), codes8_to_bf16(hw));
+      st_shared_v4(base + ((j ^ (n & 7)) << 4), codes8_to_bf16x2(hw));
     }
   } else {
     // token m = rt % 64, k half = rt / 64; q staging is 128-byte swizzled
@@ -496,7 +495,8 @@ __device__ __forceinline__ void mma_stage(uint32_t d_tmem, uint32_t sa, uint32_t
 }
 
 // Epilogue value of accumulator word `a`: the forward scales the exact INT32
-// sum by s_x[m] * gamma, dX by gamma; dW is the fp32 sum.
+// sum by s_x[m] * gamma, dX by gamma / 2 (its sum is over 2 * code); dW is
+// the fp32 sum.
 template <Op op>
 __device__ __forceinline__ float epi_value(uint32_t a, float scale) {
   if constexpr (op == Op::Fwd) return __fmul_rn(static_cast<float>(static_cast<int32_t>(a)), scale);
@@ -943,7 +943,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const int q = warp & 3;  // TMEM lane quadrant this warp may access
     const uint32_t stg = epi_warp ? smem_u32(smem + L::kOffEpi + (warp - kWarpEpi0) * L::kEpiStageBytes)
                                   : smem_u32(smem + L::kOffA + warp * L::kEpiStageBytes);
-    const float gamma = p.gamma ? __ldg(p.gamma) : 1.0f;
+    // dX's operand holds 2 * code (codes8_to_bf16x2): its epilogue takes gamma / 2
+    const float gamma = p.gamma ? (F == Family::Bwd ? 0.5f : 1.0f) * __ldg(p.gamma) : 1.0f;
     int n = 0, tile = 0;
     while (next_tile(p, pair, npairs, n, tile)) ++n;
     bool ready = epi_warp || (n > 0 && wait(done_bar, 0));
