@@ -3,7 +3,8 @@
 One step = one pass of the whole hot path over one batch:
   S1 + S2 bl_quantize (2 launches: |W| partial sums with part of the token
   rows, then gamma and the codes with the other rows) -> S3 bl_forward
-  -> S4 bl_backward (dX and dW in one launch)                  (4 launches)
+  -> S4 bl_backward with its x_hat workspace (for N >= 3072 one launch makes
+  x_hat, then dX and dW in one launch)                   (4 or 5 launches)
 
 Default workload: the up-projection BitLinear 2560 -> 6912 at 8 x 512 tokens
 (M=4096, K=2560, N=6912; x, dY bf16 ~ N(0,1), W bf16 kaiming-uniform).
@@ -180,7 +181,13 @@ def job_tops(ops_per_rank_step: float, world: int, steps: int, job_ms: float) ->
 # ----------------------------------------------------------------- our arm
 
 STAGES = ["quantize", "forward", "backward"]
-LAUNCHES_PER_STEP = 4  # S1 sums (+ S2 rows); S1 codes (+ S2 rows); S3; S4 (dX and dW in one launch)
+
+
+def launches_per_step(N):
+    """S1 sums (+ S2 rows); S1 codes (+ S2 rows); S3; S4: dX and dW in one
+    launch, after one that makes x_hat in the backward's workspace where dW
+    has N >= 3072 features (below that the library rebuilds x_hat instead)."""
+    return 5 if N >= 3072 else 4
 
 
 def stage_work(M, N, K, w_bytes):
@@ -211,7 +218,7 @@ def stage_graph_ms(bl, x, w, dy, M, N, K, dev, n_sets=4, calls=16, reps=5):
         "quantize": lambda t: bl.bl_quantize(t[1], t[0], t[3].w_packed, t[3].gamma, t[3].xq, t[3].sx, t[3].workspace),
         "forward": lambda t: bl.bl_forward(t[3].xq, t[3].sx, t[3].w_packed, t[3].gamma, t[3].y, None),
         "backward": lambda t: bl.bl_backward(t[2], t[3].xq, t[3].sx, t[3].w_packed, t[3].gamma, t[3].dX, t[3].dW,
-                                             False),
+                                             False, workspace=t[3].bwd_workspace),
     }
     out = {}
     for name, call in calls_of.items():
@@ -280,7 +287,8 @@ def run_ours(args, rank, world, local_rank):
         evs[1].record(stream)
         bl.bl_forward(bufs.xq, bufs.sx, bufs.w_packed, bufs.gamma, bufs.y, None, stream)
         evs[2].record(stream)
-        bl.bl_backward(dy, bufs.xq, bufs.sx, bufs.w_packed, bufs.gamma, bufs.dX, bufs.dW, False, stream)
+        bl.bl_backward(dy, bufs.xq, bufs.sx, bufs.w_packed, bufs.gamma, bufs.dX, bufs.dW, False, stream,
+                       workspace=bufs.bwd_workspace)
         evs[3].record(stream)
         if world > 1:
             with torch.cuda.stream(stream):
@@ -397,7 +405,7 @@ def run_ours(args, rank, world, local_rank):
         **({"allreduce_ms_per_step": round(per_stage["allreduce"] / args.steps, 5),
             "allreduce_bytes": bufs.dW.numel() * bufs.dW.element_size()} if world > 1 else {}),
         "e2e": e2e,
-        "gpu_launches": LAUNCHES_PER_STEP * args.steps,
+        "gpu_launches": launches_per_step(N) * args.steps,
         "clocks": clocks,
     }
     if world == 1 and not args.no_cpu_baseline:
@@ -623,7 +631,7 @@ def run_stack(args, rank, world, local_rank):
                    "parallelism": f"dp{world} independent replicas" if world > 1 else "single GPU"},
         "peak_device_memory_mb": round(peak_mb, 1),
         "saved_state_mb": round(saved / 1e6, 2),
-        "gpu_launches": 4 * (len(dims) - 1) * args.steps,
+        "gpu_launches": sum(launches_per_step(n) for n in dims[1:]) * args.steps,
         "clocks": clocks,
     }
 
@@ -757,11 +765,12 @@ def run_signsgd(args, rank, world, local_rank):
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
 
     words = torch.empty((N, K // 32), dtype=torch.int32, device=dev)
+    bws = torch.empty(max(bl.bl_backward_workspace_size(M, K), 16), dtype=torch.uint8, device=dev)
 
     def step():
         bl.bl_quantize_act(x, xq, sx)
         bl.bl_forward(xq, sx, packed, gamma, y)
-        bl.bl_backward_signs(dy, xq, sx, packed, gamma, dX, words)
+        bl.bl_backward_signs(dy, xq, sx, packed, gamma, dX, words, workspace=bws)
         signsgd_dp_step(None, packed, gamma, lr, master_W=master, workspace=ws if holder else None, buffers=buf,
                         words=words)
 
@@ -770,7 +779,7 @@ def run_signsgd(args, rank, world, local_rank):
     def step_unfused():
         bl.bl_quantize_act(x, xq, sx)
         bl.bl_forward(xq, sx, packed, gamma, y)
-        bl.bl_backward(dy, xq, sx, packed, gamma, dX, dW)
+        bl.bl_backward(dy, xq, sx, packed, gamma, dX, dW, workspace=bws)
         signsgd_dp_step(dW, packed, gamma, lr, master_W=master, workspace=ws if holder else None, buffers=buf,
                         ops=three_calls)
 

@@ -204,7 +204,8 @@ bl_status bl_forward(const int8_t* xq, const float* sx, const uint8_t* w_packed,
  *   x_hat[m,k] = bf16_rn(fp32(xq[m,k]) * sx[m])
  *
  * Both operands are rebuilt in shared memory from the saved 2-bit / INT8
- * state; no bf16 copy of W_hat or x_hat is written to device memory.
+ * state; no bf16 copy of W_hat or x_hat is written to device memory (see
+ * bl_backward_ws for the form that makes x_hat once in a workspace).
  * dY [M,N] bf16. dX [M,K] bf16 output or NULL (skipped). dW [N,K] output or
  * NULL (skipped), of dw_dtype (BL_BF16 or BL_F32); accumulate_dW != 0 adds to
  * the existing contents instead of overwriting them.
@@ -216,6 +217,27 @@ bl_status bl_backward(const void* dY, const int8_t* xq, const float* sx,
                       int64_t M, int64_t N, int64_t K,
                       void* dX, void* dW, bl_dtype dw_dtype, int accumulate_dW,
                       void* stream);
+
+/*
+ * bl_backward with a workspace for x_hat: the same dX and dW, bit for bit.
+ * A first launch writes x_hat (bf16 [M][K], M*K*2 bytes) into the
+ * workspace from xq and sx, converted exactly as above; dW's tiles then load
+ * their x_hat operand by TMA instead of rebuilding it from xq and sx in every
+ * tile (each element would be rebuilt once per 256-feature block of dW).
+ * The workspace is transient scratch of this call (no saved state; it holds
+ * nothing the caller needs afterwards), owned by the caller, 16-byte
+ * aligned, of at least bl_backward_workspace_size(M, K) bytes, and needs no
+ * initialisation; one call at a time per workspace. workspace == NULL: as
+ * bl_backward. Where dW has fewer than 3072 features (12 blocks of 256, each
+ * of which rebuilds x_hat once) the extra launch costs more than it saves and
+ * the workspace is left unused. Errors: as bl_backward, plus BL_ERR_WORKSPACE.
+ */
+size_t bl_backward_workspace_size(int64_t M, int64_t K);
+bl_status bl_backward_ws(const void* dY, const int8_t* xq, const float* sx,
+                         const uint8_t* w_packed, const float* gamma,
+                         int64_t M, int64_t N, int64_t K,
+                         void* dX, void* dW, bl_dtype dw_dtype, int accumulate_dW,
+                         void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * Export of the packed weights and their scale for inference
@@ -268,6 +290,14 @@ bl_status bl_backward_signs(const void* dY, const int8_t* xq, const float* sx,
                             const uint8_t* w_packed, const float* gamma,
                             int64_t M, int64_t N, int64_t K,
                             void* dX, uint32_t* dw_sign_words, void* stream);
+
+/* bl_backward_signs with bl_backward_ws's x_hat workspace (same words, same
+ * dX). Arguments and errors: as those two. */
+bl_status bl_backward_signs_ws(const void* dY, const int8_t* xq, const float* sx,
+                               const uint8_t* w_packed, const float* gamma,
+                               int64_t M, int64_t N, int64_t K,
+                               void* dX, uint32_t* dw_sign_words,
+                               void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * G2: the accumulation. sign_words holds `ranks` arrays of N*K/32 words back

@@ -41,6 +41,9 @@ SIGNATURES = {
     "bl_forward": (_I32, [_VP, _VP, _VP, _VP, _I64, _I64, _I64, _VP, _VP, _VP]),
     "bl_backward": (_I32, [_VP, _VP, _VP, _VP, _VP, _I64, _I64, _I64, _VP, _VP, _I32, _I32, _VP]),
     "bl_backward_signs": (_I32, [_VP, _VP, _VP, _VP, _VP, _I64, _I64, _I64, _VP, _VP, _VP]),
+    "bl_backward_workspace_size": (_SZ, [_I64, _I64]),
+    "bl_backward_ws": (_I32, [_VP, _VP, _VP, _VP, _VP, _I64, _I64, _I64, _VP, _VP, _I32, _I32, _VP, _SZ, _VP]),
+    "bl_backward_signs_ws": (_I32, [_VP, _VP, _VP, _VP, _VP, _I64, _I64, _I64, _VP, _VP, _VP, _SZ, _VP]),
     "bl_export_weights": (_I32, [_VP, _VP, _I64, _I64, _VP, _VP, _VP]),
     "bl_get_last_error": (_I32, []),
     "bl_reset_error": (_I32, []),
@@ -189,8 +192,14 @@ def bl_forward(xq, sx, w_packed, gamma, y, debug_acc=None, stream=None):
                                      _ptr(debug_acc), _stream(stream)), "bl_forward")
 
 
-def bl_backward(dY, xq, sx, w_packed, gamma, dX=None, dW=None, accumulate_dW=False, stream=None):
-    """S4: dX [M,K] bf16 = gamma * dY . codes; dW [N,K] (bf16|f32) = dY^T . x_hat."""
+def bl_backward_workspace_size(M: int, K: int) -> int:
+    return load_library().bl_backward_workspace_size(M, K)
+
+
+def bl_backward(dY, xq, sx, w_packed, gamma, dX=None, dW=None, accumulate_dW=False, stream=None, workspace=None):
+    """S4: dX [M,K] bf16 = gamma * dY . codes; dW [N,K] (bf16|f32) = dY^T . x_hat.
+    workspace (bl_backward_workspace_size bytes): x_hat is made once there
+    (bl_backward_ws) instead of rebuilt in every dW tile; same results."""
     M, N = dY.shape
     K = xq.shape[1]
     _need(dY, torch.bfloat16, (M, N), "dY")
@@ -206,15 +215,23 @@ def bl_backward(dY, xq, sx, w_packed, gamma, dX=None, dW=None, accumulate_dW=Fal
             raise ValueError("dW must be bf16 or f32")
         _need(dW, dW.dtype, (N, K), "dW")
         dwdt = BL_F32 if dW.dtype == torch.float32 else BL_BF16
-    _on_current_device(dY, xq, sx, w_packed, gamma, dX, dW)
-    _check(load_library().bl_backward(_ptr(dY), _ptr(xq), _ptr(sx), _ptr(w_packed), _ptr(gamma), M, N, K,
-                                      _ptr(dX), _ptr(dW), dwdt, int(bool(accumulate_dW)), _stream(stream)),
-           "bl_backward")
+    _on_current_device(dY, xq, sx, w_packed, gamma, dX, dW, workspace)
+    lib = load_library()
+    if workspace is None:
+        _check(lib.bl_backward(_ptr(dY), _ptr(xq), _ptr(sx), _ptr(w_packed), _ptr(gamma), M, N, K,
+                               _ptr(dX), _ptr(dW), dwdt, int(bool(accumulate_dW)), _stream(stream)),
+               "bl_backward")
+    else:
+        _check(lib.bl_backward_ws(_ptr(dY), _ptr(xq), _ptr(sx), _ptr(w_packed), _ptr(gamma), M, N, K,
+                                  _ptr(dX), _ptr(dW), dwdt, int(bool(accumulate_dW)), _ptr(workspace),
+                                  workspace.numel() * workspace.element_size(), _stream(stream)),
+               "bl_backward_ws")
 
 
-def bl_backward_signs(dY, xq, sx, w_packed, gamma, dX, dw_sign_words, stream=None):
+def bl_backward_signs(dY, xq, sx, w_packed, gamma, dX, dw_sign_words, stream=None, workspace=None):
     """S4 with G1 fused: dX [M,K] bf16 (or None) as bl_backward, and the sign
-    words of dW, dw_sign_words [N, K/32] int32 (bit patterns), instead of dW."""
+    words of dW, dw_sign_words [N, K/32] int32 (bit patterns), instead of dW.
+    workspace: as bl_backward's."""
     M, N = dY.shape
     K = xq.shape[1]
     _need(dY, torch.bfloat16, (M, N), "dY")
@@ -225,10 +242,17 @@ def bl_backward_signs(dY, xq, sx, w_packed, gamma, dX, dw_sign_words, stream=Non
     if dX is not None:
         _need(dX, torch.bfloat16, (M, K), "dX")
     _need(dw_sign_words, torch.int32, (N, K // 32), "dw_sign_words")
-    _on_current_device(dY, xq, sx, w_packed, gamma, dX, dw_sign_words)
-    _check(load_library().bl_backward_signs(_ptr(dY), _ptr(xq), _ptr(sx), _ptr(w_packed), _ptr(gamma), M, N, K,
-                                            _ptr(dX), _ptr(dw_sign_words), _stream(stream)),
-           "bl_backward_signs")
+    _on_current_device(dY, xq, sx, w_packed, gamma, dX, dw_sign_words, workspace)
+    lib = load_library()
+    if workspace is None:
+        _check(lib.bl_backward_signs(_ptr(dY), _ptr(xq), _ptr(sx), _ptr(w_packed), _ptr(gamma), M, N, K,
+                                     _ptr(dX), _ptr(dw_sign_words), _stream(stream)),
+               "bl_backward_signs")
+    else:
+        _check(lib.bl_backward_signs_ws(_ptr(dY), _ptr(xq), _ptr(sx), _ptr(w_packed), _ptr(gamma), M, N, K,
+                                        _ptr(dX), _ptr(dw_sign_words), _ptr(workspace),
+                                        workspace.numel() * workspace.element_size(), _stream(stream)),
+               "bl_backward_signs_ws")
 
 
 def bl_sign_pack(dW, sign_words, stream=None):
@@ -317,6 +341,7 @@ class StepBuffers:
     y: torch.Tensor
     dX: torch.Tensor
     dW: torch.Tensor
+    bwd_workspace: torch.Tensor | None = None  # x_hat scratch of the backward (bl_backward_ws)
 
     @staticmethod
     def allocate(M, N, K, dw_dtype=torch.bfloat16, device="cuda"):
@@ -330,6 +355,7 @@ class StepBuffers:
             y=torch.empty((M, N), dtype=torch.bfloat16, device=device),
             dX=torch.empty((M, K), dtype=torch.bfloat16, device=device),
             dW=torch.empty((N, K), dtype=dw_dtype, device=device),
+            bwd_workspace=torch.empty(max(bl_backward_workspace_size(M, K), 16), dtype=torch.uint8, device=device),
         )
 
 
@@ -337,4 +363,5 @@ def bitlinear_step(x, W, dY, bufs: StepBuffers, stream=None):
     """One BitLinear forward + backward: S1 + S2 (bl_quantize) -> S3 -> S4 (four kernel launches)."""
     bl_quantize(W, x, bufs.w_packed, bufs.gamma, bufs.xq, bufs.sx, bufs.workspace, stream)
     bl_forward(bufs.xq, bufs.sx, bufs.w_packed, bufs.gamma, bufs.y, None, stream)
-    bl_backward(dY, bufs.xq, bufs.sx, bufs.w_packed, bufs.gamma, bufs.dX, bufs.dW, False, stream)
+    bl_backward(dY, bufs.xq, bufs.sx, bufs.w_packed, bufs.gamma, bufs.dX, bufs.dW, False, stream,
+                workspace=bufs.bwd_workspace)

@@ -186,16 +186,23 @@ bl_status bl_forward(const int8_t* xq, const float* sx, const uint8_t* w_packed,
                      "bl_forward launch");
 }
 
-bl_status bl_backward(const void* dY, const int8_t* xq, const float* sx, const uint8_t* w_packed,
-                      const float* gamma, int64_t M, int64_t N, int64_t K, void* dX, void* dW, bl_dtype dw_dtype,
-                      int accumulate_dW, void* stream) {
+// The checks and the launch shared by bl_backward, bl_backward_signs and
+// their workspace forms. dw_signs: dW receives sign words.
+static bl_status backward_common(const void* dY, const int8_t* xq, const float* sx, const uint8_t* w_packed,
+                                 const float* gamma, int64_t M, int64_t N, int64_t K, void* dX, void* dW,
+                                 bl_dtype dw_dtype, int accumulate_dW, int dw_signs, void* workspace,
+                                 size_t workspace_bytes, void* stream, const char* what) {
   g_msg[0] = 0;
   if (M < 0 || N < 1) return fail(BL_ERR_INVALID_ARG, "M=%lld, N=%lld", (long long)M, (long long)N);
   if (bl_status s = check_k(K)) return s;
   if (N % 8 != 0) return fail(BL_ERR_UNSUPPORTED_SHAPE, "N=%lld must be a multiple of 8", (long long)N);
   if (M > (int64_t(1) << 30) || N > (int64_t(1) << 30)) return fail(BL_ERR_UNSUPPORTED_SHAPE, "M or N too large");
-  if (dW && dw_dtype != BL_BF16 && dw_dtype != BL_F32) return fail(BL_ERR_DTYPE, "dw_dtype %d", (int)dw_dtype);
-  if (!dX && !dW) return BL_OK;
+  if (dw_signs) {
+    if (!dW) return fail(BL_ERR_INVALID_ARG, "null dw_sign_words");
+  } else {
+    if (dW && dw_dtype != BL_BF16 && dw_dtype != BL_F32) return fail(BL_ERR_DTYPE, "dw_dtype %d", (int)dw_dtype);
+    if (!dX && !dW) return BL_OK;
+  }
   if (M > 0 && !dY) return fail(BL_ERR_INVALID_ARG, "null dY");
   if (dX && (!w_packed || !gamma)) return fail(BL_ERR_INVALID_ARG, "dX needs w_packed and gamma");
   if (dW && M > 0 && (!xq || !sx)) return fail(BL_ERR_INVALID_ARG, "dW needs xq and sx");
@@ -203,34 +210,51 @@ bl_status bl_backward(const void* dY, const int8_t* xq, const float* sx, const u
       (w_packed && !aligned16(w_packed)) || (gamma && !aligned16(gamma)) || (dX && !aligned16(dX)) ||
       (dW && !aligned16(dW)))
     return fail(BL_ERR_ALIGNMENT, "tensors must be 16-byte aligned");
+  if (workspace) {
+    const size_t need = bl_backward_workspace_size(M, K);
+    if (workspace_bytes < need || !aligned16(workspace))
+      return fail(BL_ERR_WORKSPACE, "workspace needs %zu bytes, 16-byte aligned", need);
+  }
+  // x_hat is only worth making when dW is computed from tokens
+  void* xhat = (workspace && dW && M > 0) ? workspace : nullptr;
   int* err = nullptr;
   if (bl_status s = current_device(&err)) return s;
-  return cuda_status(bl::launch_backward(dY, xq, sx, w_packed, gamma, M, N, K, dX, dW, dw_dtype == BL_F32,
-                                         accumulate_dW != 0, 0, err, static_cast<cudaStream_t>(stream)),
-                     "bl_backward launch");
+  return cuda_status(bl::launch_backward(dY, xq, sx, w_packed, gamma, M, N, K, dX, dW,
+                                         dw_signs ? 0 : dw_dtype == BL_F32, dw_signs ? 0 : accumulate_dW != 0,
+                                         dw_signs, xhat, err, static_cast<cudaStream_t>(stream)),
+                     what);
+}
+
+size_t bl_backward_workspace_size(int64_t M, int64_t K) {
+  return (M > 0 && K > 0) ? static_cast<size_t>(M) * static_cast<size_t>(K) * 2 : 0;
+}
+
+bl_status bl_backward(const void* dY, const int8_t* xq, const float* sx, const uint8_t* w_packed,
+                      const float* gamma, int64_t M, int64_t N, int64_t K, void* dX, void* dW, bl_dtype dw_dtype,
+                      int accumulate_dW, void* stream) {
+  return backward_common(dY, xq, sx, w_packed, gamma, M, N, K, dX, dW, dw_dtype, accumulate_dW, 0, nullptr, 0,
+                         stream, "bl_backward launch");
+}
+
+bl_status bl_backward_ws(const void* dY, const int8_t* xq, const float* sx, const uint8_t* w_packed,
+                         const float* gamma, int64_t M, int64_t N, int64_t K, void* dX, void* dW, bl_dtype dw_dtype,
+                         int accumulate_dW, void* workspace, size_t workspace_bytes, void* stream) {
+  return backward_common(dY, xq, sx, w_packed, gamma, M, N, K, dX, dW, dw_dtype, accumulate_dW, 0, workspace,
+                         workspace_bytes, stream, "bl_backward_ws launch");
 }
 
 bl_status bl_backward_signs(const void* dY, const int8_t* xq, const float* sx, const uint8_t* w_packed,
                             const float* gamma, int64_t M, int64_t N, int64_t K, void* dX, uint32_t* dw_sign_words,
                             void* stream) {
-  g_msg[0] = 0;
-  if (M < 0 || N < 1) return fail(BL_ERR_INVALID_ARG, "M=%lld, N=%lld", (long long)M, (long long)N);
-  if (bl_status s = check_k(K)) return s;
-  if (N % 8 != 0) return fail(BL_ERR_UNSUPPORTED_SHAPE, "N=%lld must be a multiple of 8", (long long)N);
-  if (M > (int64_t(1) << 30) || N > (int64_t(1) << 30)) return fail(BL_ERR_UNSUPPORTED_SHAPE, "M or N too large");
-  if (!dw_sign_words) return fail(BL_ERR_INVALID_ARG, "null dw_sign_words");
-  if (M > 0 && !dY) return fail(BL_ERR_INVALID_ARG, "null dY");
-  if (dX && (!w_packed || !gamma)) return fail(BL_ERR_INVALID_ARG, "dX needs w_packed and gamma");
-  if (M > 0 && (!xq || !sx)) return fail(BL_ERR_INVALID_ARG, "the sign words need xq and sx");
-  if ((dY && !aligned16(dY)) || (xq && !aligned16(xq)) || (sx && !aligned16(sx)) ||
-      (w_packed && !aligned16(w_packed)) || (gamma && !aligned16(gamma)) || (dX && !aligned16(dX)) ||
-      !aligned16(dw_sign_words))
-    return fail(BL_ERR_ALIGNMENT, "tensors must be 16-byte aligned");
-  int* err = nullptr;
-  if (bl_status s = current_device(&err)) return s;
-  return cuda_status(bl::launch_backward(dY, xq, sx, w_packed, gamma, M, N, K, dX, dw_sign_words, 0, 0, 1, err,
-                                         static_cast<cudaStream_t>(stream)),
-                     "bl_backward_signs launch");
+  return backward_common(dY, xq, sx, w_packed, gamma, M, N, K, dX, dw_sign_words, BL_BF16, 0, 1, nullptr, 0, stream,
+                         "bl_backward_signs launch");
+}
+
+bl_status bl_backward_signs_ws(const void* dY, const int8_t* xq, const float* sx, const uint8_t* w_packed,
+                               const float* gamma, int64_t M, int64_t N, int64_t K, void* dX,
+                               uint32_t* dw_sign_words, void* workspace, size_t workspace_bytes, void* stream) {
+  return backward_common(dY, xq, sx, w_packed, gamma, M, N, K, dX, dw_sign_words, BL_BF16, 0, 1, workspace,
+                         workspace_bytes, stream, "bl_backward_signs_ws launch");
 }
 
 bl_status bl_export_weights(const uint8_t* w_packed, const float* gamma, int64_t N, int64_t K,

@@ -81,10 +81,12 @@ cudaError_t launch_forward(const int8_t* xq, const float* sx, const uint8_t* w_p
 
 // dX and/or dW (either output may be null) in one launch. With dw_signs, dW
 // receives the sign words of dW ([N*K/32] uint32, element 32w + j at bit j of
-// word w) instead of dW itself.
+// word w) instead of dW itself. With xhat_ws (bf16 [M][K], 16-byte aligned), a
+// launch before the GEMMs writes x_hat there and dW's tiles load it instead of
+// rebuilding it.
 cudaError_t launch_backward(const void* dY, const int8_t* xq, const float* sx, const uint8_t* w_packed,
                             const float* gamma, int64_t M, int64_t N, int64_t K, void* dX, void* dW, int dw_is_f32,
-                            int accumulate, int dw_signs, int* err, cudaStream_t s);
+                            int accumulate, int dw_signs, void* xhat_ws, int* err, cudaStream_t s);
 
 // ---- Master-free sign-gradient update (k_signsgd.cu)
 // Sign bits of dW [N,K] (bf16 or f32): out [N*K/32] words, element 32w+j -> bit j.

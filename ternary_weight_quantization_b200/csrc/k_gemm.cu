@@ -206,6 +206,8 @@ struct OpParams {
   int src_tma;    // Fwd/Dx: packed codes by TMA (K % 64 == 0) instead of cp.async
   int tma_store;  // output through the TMA store map of this op
   int sign_words; // Dw: out receives the sign bits of dW (32 per word along K) instead of dW
+  int xhat_tma;   // Dw: A = x_hat^T loaded by TMA from a bf16 [M][K] copy made before the launch
+                  // (the source map), instead of rebuilt from q and s_x in every tile
 };
 
 struct GemmParams {
@@ -363,7 +365,7 @@ struct Maps {
 template <Op op, Family F, int BN>
 __device__ __forceinline__ void load_stage(const GemmParams& p, const OpParams& P, const Maps& m, bool leader,
                                            int lane, int a0, int bp, int bh, int kb, uint64_t* full, uint32_t full_lead,
-                                           uint64_t* src_full, uint8_t* sB, uint8_t* sSrc, uint8_t* sSx) {
+                                           uint64_t* src_full, uint8_t* sA, uint8_t* sB, uint8_t* sSrc, uint8_t* sSx) {
   using G = Geo<F, BN>;
   const int r0 = kb * G::kBlockR;
   const int kq = static_cast<int>(p.K / 4);
@@ -372,9 +374,17 @@ __device__ __forceinline__ void load_stage(const GemmParams& p, const OpParams& 
     if constexpr (op == Op::Dw) {
 #pragma unroll
       for (int j = 0; j < (BN / 2) / 64; ++j) tma_load_2d_pair(m.b, full_lead, sB + j * 8192, bh + 64 * j, r0);
-      mbar_arrive_expect_tx(src_full, 64 * 128 + 64 * 4);
-      tma_load_2d(m.src, src_full, sSrc, a0, r0);
-      tma_load_2d(m.sx, src_full, sSx, r0, 0);
+      if (P.xhat_tma) {
+        // A itself: two 64 (k) x 64 (m) bf16 boxes of x_hat, 128-byte
+        // swizzled exactly as the rebuild writes them
+        mbar_arrive_expect_tx(src_full, 2 * 64 * 128);
+        tma_load_2d(m.src, src_full, sA, a0, r0);
+        tma_load_2d(m.src, src_full, sA + 8192, a0 + 64, r0);
+      } else {
+        mbar_arrive_expect_tx(src_full, 64 * 128 + 64 * 4);
+        tma_load_2d(m.src, src_full, sSrc, a0, r0);
+        tma_load_2d(m.sx, src_full, sSx, r0, 0);
+      }
     } else {
       if constexpr (op == Op::Fwd && BN > 256) {
         static_assert(128 % kWideBox<BN> == 0, "the first MMA's rows come in whole boxes");
@@ -802,7 +812,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       if (F == Family::Bwd && p.op[1].ntiles) {
         prefetch_tensormap(&map_b1);
         prefetch_tensormap(&map_src1);
-        prefetch_tensormap(&map_sx);
+        if (!p.op[1].xhat_tma) prefetch_tensormap(&map_sx);
       }
     }
     int stage = 0;
@@ -819,15 +829,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           break;
         }
         if (lane == 0) issued_parity[stage] = static_cast<int>(phase);
+        uint8_t* sA = smem + L::kOffA + stage * G::kABytes;
         uint8_t* sB = smem + L::kOffB + stage * G::kBBytes;
         uint8_t* sSrc = smem + L::kOffSrc + stage * G::kSrcBytes;
         uint8_t* sSx = smem + L::kOffSx + stage * G::kSxBytes;
         if (t.opi == 0)
           load_stage<kOp0, F, BN>(p, P, maps0, leader, lane, t.a0, t.bp, bh, kb, &full[stage], lead(&full[stage]),
-                                  &src_full[stage], sB, sSrc, sSx);
+                                  &src_full[stage], sA, sB, sSrc, sSx);
         else if constexpr (F == Family::Bwd)
           load_stage<Op::Dw, F, BN>(p, P, maps1, leader, lane, t.a0, t.bp, bh, kb, &full[stage], lead(&full[stage]),
-                                    &src_full[stage], sB, sSrc, sSx);
+                                    &src_full[stage], sA, sB, sSrc, sSx);
         if (++stage == S) {
           stage = 0;
           phase ^= 1;
@@ -915,8 +926,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           const float* sSx = reinterpret_cast<const float*>(smem + L::kOffSx + stage * G::kSxBytes);
           if (opi == 0)
             rebuild_stage<kOp0, F, BN>(rt, sA, sSrc, sSx);
-          else if constexpr (F == Family::Bwd)
-            rebuild_stage<Op::Dw, F, BN>(rt, sA, sSrc, sSx);
+          else if constexpr (F == Family::Bwd) {
+            if (!p.op[1].xhat_tma) rebuild_stage<Op::Dw, F, BN>(rt, sA, sSrc, sSx);
+          }
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) mbar_arrive_cluster(lead(&full[stage]));
@@ -1350,6 +1362,44 @@ __global__ void zero_dw_kernel(void* out, int64_t n, int out_f32, int accumulate
     static_cast<uint16_t*>(out)[i] = 0;
 }
 
+// x_hat = bf16_rn(fp32(q) * s_x[m]) for all of xq [M][K] into a bf16 [M][K]
+// workspace, converted exactly as the dW rebuild does (s8x16_to_bf16), so
+// that dW tiles can load their A operand by TMA instead of rebuilding it in
+// every tile (each x_hat element would otherwise be rebuilt once per
+// 256-feature block of dW). Thread t takes kXhatU 16-element chunks spaced
+// one grid apart, all loads issued first (16-byte loads, two 16-byte stores
+// per chunk); the grid is sized so that one pass covers xq.
+constexpr int kXhatU = 4;
+
+__global__ void __launch_bounds__(256) xhat_kernel(const uint4* __restrict__ xq, const float* __restrict__ sx,
+                                                   int64_t chunks, int chunks_per_row, uint4* __restrict__ out) {
+  pdl_wait_primary();
+  pdl_launch_dependents();
+  const int64_t T = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t c0 = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; c0 < chunks; c0 += kXhatU * T) {
+    uint4 v[kXhatU];
+    float s[kXhatU];
+#pragma unroll
+    for (int u = 0; u < kXhatU; ++u) {
+      const int64_t c = c0 + u * T;
+      if (c < chunks) {
+        v[u] = __ldg(xq + c);
+        s[u] = __ldg(sx + c / chunks_per_row);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kXhatU; ++u) {
+      const int64_t c = c0 + u * T;
+      if (c < chunks) {
+        uint4 o0, o1;
+        s8x16_to_bf16(v[u], s[u], o0, o1);
+        out[2 * c] = o0;
+        out[2 * c + 1] = o1;
+      }
+    }
+  }
+}
+
 // ---------------------------------------------------------------- host side
 
 thread_local char g_launch_detail[160] = "";
@@ -1611,7 +1661,7 @@ cudaError_t launch_forward(const int8_t* xq, const float* sx, const uint8_t* w_p
 // dX and/or dW in one launch (either output may be null).
 cudaError_t launch_backward(const void* dY, const int8_t* xq, const float* sx, const uint8_t* w_packed,
                             const float* gamma, int64_t M, int64_t N, int64_t K, void* dX, void* dW, int dw_is_f32,
-                            int accumulate, int dw_signs, int* err, cudaStream_t s) {
+                            int accumulate, int dw_signs, void* xhat_ws, int* err, cudaStream_t s) {
   if (dW && M == 0) {
     // dW = 0: zeros, or sign words of +0 (all bits clear, 4-byte words)
     const int64_t n = dw_signs ? N * K / 32 : N * K;
@@ -1621,6 +1671,14 @@ cudaError_t launch_backward(const void* dY, const int8_t* xq, const float* sx, c
   }
   if (M == 0) return cudaSuccess;
   constexpr int BN = 256;
+  // x_hat is made in the workspace only where its rebuilds would cost more
+  // than the extra launch: every dW tile column block (256 features) rebuilds
+  // all of x_hat once, and the launch moves 3 bytes per element. Measured on
+  // B200 (CUDA graphs, rebuild against workspace, interleaved): 27 blocks
+  // (N 6912) 220.7 -> 213.5 us, 10 blocks (N 2560) 116.2 -> 117.4 us; the
+  // break-even is near 12 blocks.
+  constexpr int64_t kXhatMinN = 12 * 256;
+  if (N < kXhatMinN) xhat_ws = nullptr;
   const int npairs = resident_pairs<Family::Bwd, BN>();
   CUtensorMap maps[7] = {};  // b0, src0, out0, b1, src1, out1, sx
   const bool src_tma = (K % 64) == 0;
@@ -1637,12 +1695,19 @@ cudaError_t launch_backward(const void* dY, const int8_t* xq, const float* sx, c
     // s_x as a one-row 2D tensor: [1][M] floats, row pitch rounded up to 16 bytes
     const uint64_t sx_pitch = ((static_cast<uint64_t>(M) * 4 + 15) / 16) * 16;
     if (!make_map_2d(&maps[3], dY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, N, M, N * 2, 64, 64,
-                     CU_TENSOR_MAP_SWIZZLE_128B, "dY (dW)") ||
-        !make_map_2d(&maps[4], xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, K, M, K, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B,
-                     "xq (dW)") ||
-        !make_map_2d(&maps[6], sx, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, M, 1, sx_pitch, 64, 1, CU_TENSOR_MAP_SWIZZLE_NONE,
-                     "sx (dW)"))
+                     CU_TENSOR_MAP_SWIZZLE_128B, "dY (dW)"))
       return cudaErrorInvalidValue;
+    if (xhat_ws) {
+      // x_hat [M][K] bf16 in the workspace, loaded as dW's A in 64 x 64 boxes
+      if (!make_map_2d(&maps[4], xhat_ws, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, K, M, K * 2, 64, 64,
+                       CU_TENSOR_MAP_SWIZZLE_128B, "x_hat (dW)"))
+        return cudaErrorInvalidValue;
+    } else if (!make_map_2d(&maps[4], xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, K, M, K, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B,
+                            "xq (dW)") ||
+               !make_map_2d(&maps[6], sx, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, M, 1, sx_pitch, 64, 1,
+                            CU_TENSOR_MAP_SWIZZLE_NONE, "sx (dW)")) {
+      return cudaErrorInvalidValue;
+    }
     if (!accumulate && !dw_signs && !make_out_map(&maps[5], dW, dw_is_f32 != 0, N, K, "dW"))
       return cudaErrorInvalidValue;
   }
@@ -1663,12 +1728,22 @@ cudaError_t launch_backward(const void* dY, const int8_t* xq, const float* sx, c
     p.op[1].accumulate = dw_signs ? 0 : accumulate;
     p.op[1].tma_store = !accumulate && !dw_signs;
     p.op[1].sign_words = dw_signs;
+    p.op[1].xhat_tma = xhat_ws != nullptr;
   }
   p.K = K;
   p.packed = w_packed;
   p.sx = sx;
   p.gamma = dX ? gamma : nullptr;
   p.err = err;
+  if (dW && xhat_ws) {
+    const int64_t chunks = M * K / 16;
+    const int64_t want = (chunks + 256 * kXhatU - 1) / (256 * kXhatU);
+    const int64_t cap = static_cast<int64_t>(8) * device_sm_count();
+    cudaError_t e = launch_pdl(xhat_kernel, dim3(static_cast<unsigned>(want < cap ? want : cap)), dim3(256), 0, s,
+                               reinterpret_cast<const uint4*>(xq), sx, chunks, static_cast<int>(K / 16),
+                               static_cast<uint4*>(xhat_ws));
+    if (e != cudaSuccess) return e;
+  }
   return launch_pair<Family::Bwd, BN>(maps, p, npairs, s);
 }
 

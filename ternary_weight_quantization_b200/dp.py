@@ -54,7 +54,8 @@ def dp_step(x, W, dY, bufs: b.StepBuffers, *, group=None, stream=None, ops: DPOp
     ops = ops or DPOps()
     ops.quantize(W, x, bufs.w_packed, bufs.gamma, bufs.xq, bufs.sx, bufs.workspace, stream)
     ops.forward(bufs.xq, bufs.sx, bufs.w_packed, bufs.gamma, bufs.y, None, stream)
-    ops.backward(dY, bufs.xq, bufs.sx, bufs.w_packed, bufs.gamma, bufs.dX, bufs.dW, False, stream)
+    ws = {} if bufs.bwd_workspace is None else {"workspace": bufs.bwd_workspace}  # x_hat scratch
+    ops.backward(dY, bufs.xq, bufs.sx, bufs.w_packed, bufs.gamma, bufs.dX, bufs.dW, False, stream, **ws)
     if dist.is_available() and dist.is_initialized() and dist.get_world_size(group) > 1:
         if stream is not None and bufs.dW.is_cuda:
             with torch.cuda.stream(stream):

@@ -39,6 +39,7 @@ class BitLinearStack:
     layers: list = field(default_factory=list)
     act: list = field(default_factory=list)   # two [M, max_dim] bf16 buffers (forward outputs)
     grad: list = field(default_factory=list)  # two [M, max_dim] bf16 buffers (backward dX)
+    bwd_workspace: torch.Tensor | None = None  # x_hat scratch of the backward, shared by the layers
 
     @staticmethod
     def allocate(M, dims, dw_dtype=torch.bfloat16, device="cuda"):
@@ -57,6 +58,10 @@ class BitLinearStack:
         big = M * max(dims)
         s.act = [torch.empty(big, dtype=torch.bfloat16, device=device) for _ in range(2)]
         s.grad = [torch.empty(big, dtype=torch.bfloat16, device=device) for _ in range(2)]
+        # the library makes x_hat in the workspace only for layers with at
+        # least 3072 output features (bl_backward_ws)
+        need = max([b.bl_backward_workspace_size(M, K) for K, N in zip(dims[:-1], dims[1:]) if N >= 3072] or [0])
+        s.bwd_workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=device)
         return s
 
     def forward(self, x, weights, stream=None, on_layer=None):
@@ -85,7 +90,7 @@ class BitLinearStack:
             L = self.layers[i]
             want_dx = input_grad or i > 0
             dX = self.grad[i % 2][: self.M * L.K].view(self.M, L.K) if want_dx else None
-            b.bl_backward(g, L.xq, L.sx, L.w_packed, L.gamma, dX, L.dW, False, stream)
+            b.bl_backward(g, L.xq, L.sx, L.w_packed, L.gamma, dX, L.dW, False, stream, workspace=self.bwd_workspace)
             if on_layer is not None:
                 on_layer(i, g, dX)
             g = dX

@@ -501,3 +501,40 @@ def test_forward_wide_tiles(M, N, K):
     y_o = ref.round_to_bf16_bits(ref.forward_output(acc_o, sx[rows], gamma))
     np.testing.assert_array_equal(bits(bufs.y)[rows], y_o)
     np.testing.assert_array_equal(bits(y2)[rows], y_o)
+
+
+@pytest.mark.parametrize("M,N,K,dw_dtype,accumulate", [
+    (4096, 6912, 2560, torch.bfloat16, False),   # the up-projection
+    (2048, 2560, 6912, torch.bfloat16, False),   # the down-projection: workspace left unused (N < 3072)
+    (300, 3072, 320, torch.float32, False),
+    (257, 3200, 544, torch.bfloat16, True),      # ragged tokens and features, accumulation
+    (17, 4096, 96, torch.float32, True),         # K % 64 != 0: a partial x_hat box
+    (64, 3080, 1024, torch.bfloat16, False),
+])
+def test_backward_workspace_matches_rebuild(M, N, K, dw_dtype, accumulate):
+    """bl_backward_ws (x_hat made once in the workspace, dW's operand loaded
+    by TMA, for N >= 3072) gives dX and dW bit for bit as bl_backward (x_hat
+    rebuilt in every dW tile), and the sign-word form the same words; the
+    workspace starts as garbage."""
+    bl = _bl()
+    x, w, dy = make_inputs(M, K, N, seed=80 + M)
+    bufs = bl.StepBuffers.allocate(M, N, K, dw_dtype)
+    xd, wd, dyd = x.cuda(), w.cuda(), dy.cuda()
+    bl.bl_quantize_weight(wd, bufs.w_packed, bufs.gamma, bufs.workspace)
+    bl.bl_quantize_act(xd, bufs.xq, bufs.sx)
+    ws = torch.full((bl.bl_backward_workspace_size(M, K),), 0xAB, dtype=torch.uint8, device="cuda")
+    prev = (torch.randn(N, K, generator=torch.Generator().manual_seed(5)) * 3).to(dw_dtype).cuda()
+    outs = []
+    for workspace in (None, ws):
+        dX = torch.empty((M, K), dtype=torch.bfloat16, device="cuda")
+        dW = prev.clone() if accumulate else torch.full((N, K), 7.0, dtype=dw_dtype, device="cuda")
+        words = torch.zeros((N, K // 32), dtype=torch.int32, device="cuda")
+        dX2 = torch.empty((M, K), dtype=torch.bfloat16, device="cuda")
+        bl.bl_backward(dyd, bufs.xq, bufs.sx, bufs.w_packed, bufs.gamma, dX, dW, accumulate, workspace=workspace)
+        bl.bl_backward_signs(dyd, bufs.xq, bufs.sx, bufs.w_packed, bufs.gamma, dX2, words, workspace=workspace)
+        torch.cuda.synchronize()
+        assert bl.bl_get_last_error() == 0
+        outs.append([t.cpu() for t in (dX, dW, words, dX2)])
+    for a, b in zip(*outs):
+        assert torch.equal(a.view(torch.uint8), b.view(torch.uint8))
+    assert torch.equal(outs[1][0].view(torch.int16), outs[1][3].view(torch.int16))
