@@ -765,7 +765,7 @@ def run_signsgd(args, rank, world, local_rank):
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
 
     words = torch.empty((N, K // 32), dtype=torch.int32, device=dev)
-    bws = torch.empty(max(bl.bl_backward_workspace_size(M, K), 16), dtype=torch.uint8, device=dev)
+    bws = torch.empty(max(bl.bl_backward_workspace_size(M, N, K), 16), dtype=torch.uint8, device=dev)
 
     def step():
         bl.bl_quantize_act(x, xq, sx)

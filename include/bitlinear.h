@@ -226,13 +226,14 @@ bl_status bl_backward(const void* dY, const int8_t* xq, const float* sx,
  * tile (each element would be rebuilt once per 256-feature block of dW).
  * The workspace is transient scratch of this call (no saved state; it holds
  * nothing the caller needs afterwards), owned by the caller, 16-byte
- * aligned, of at least bl_backward_workspace_size(M, K) bytes, and needs no
- * initialisation; one call at a time per workspace. workspace == NULL: as
+ * aligned, of at least bl_backward_workspace_size(M, N, K) bytes, and needs
+ * no initialisation; one call at a time per workspace. workspace == NULL: as
  * bl_backward. Where dW has fewer than 3072 features (12 blocks of 256, each
- * of which rebuilds x_hat once) the extra launch costs more than it saves and
- * the workspace is left unused. Errors: as bl_backward, plus BL_ERR_WORKSPACE.
+ * of which rebuilds x_hat once) the extra launch costs more than it saves:
+ * the size is then 0 and the workspace is not used (any pointer, or NULL).
+ * Errors: as bl_backward, plus BL_ERR_WORKSPACE.
  */
-size_t bl_backward_workspace_size(int64_t M, int64_t K);
+size_t bl_backward_workspace_size(int64_t M, int64_t N, int64_t K);
 bl_status bl_backward_ws(const void* dY, const int8_t* xq, const float* sx,
                          const uint8_t* w_packed, const float* gamma,
                          int64_t M, int64_t N, int64_t K,

@@ -41,7 +41,7 @@ SIGNATURES = {
     "bl_forward": (_I32, [_VP, _VP, _VP, _VP, _I64, _I64, _I64, _VP, _VP, _VP]),
     "bl_backward": (_I32, [_VP, _VP, _VP, _VP, _VP, _I64, _I64, _I64, _VP, _VP, _I32, _I32, _VP]),
     "bl_backward_signs": (_I32, [_VP, _VP, _VP, _VP, _VP, _I64, _I64, _I64, _VP, _VP, _VP]),
-    "bl_backward_workspace_size": (_SZ, [_I64, _I64]),
+    "bl_backward_workspace_size": (_SZ, [_I64, _I64, _I64]),
     "bl_backward_ws": (_I32, [_VP, _VP, _VP, _VP, _VP, _I64, _I64, _I64, _VP, _VP, _I32, _I32, _VP, _SZ, _VP]),
     "bl_backward_signs_ws": (_I32, [_VP, _VP, _VP, _VP, _VP, _I64, _I64, _I64, _VP, _VP, _VP, _SZ, _VP]),
     "bl_export_weights": (_I32, [_VP, _VP, _I64, _I64, _VP, _VP, _VP]),
@@ -192,8 +192,8 @@ def bl_forward(xq, sx, w_packed, gamma, y, debug_acc=None, stream=None):
                                      _ptr(debug_acc), _stream(stream)), "bl_forward")
 
 
-def bl_backward_workspace_size(M: int, K: int) -> int:
-    return load_library().bl_backward_workspace_size(M, K)
+def bl_backward_workspace_size(M: int, N: int, K: int) -> int:
+    return load_library().bl_backward_workspace_size(M, N, K)
 
 
 def bl_backward(dY, xq, sx, w_packed, gamma, dX=None, dW=None, accumulate_dW=False, stream=None, workspace=None):
@@ -355,7 +355,7 @@ class StepBuffers:
             y=torch.empty((M, N), dtype=torch.bfloat16, device=device),
             dX=torch.empty((M, K), dtype=torch.bfloat16, device=device),
             dW=torch.empty((N, K), dtype=dw_dtype, device=device),
-            bwd_workspace=torch.empty(max(bl_backward_workspace_size(M, K), 16), dtype=torch.uint8, device=device),
+            bwd_workspace=torch.empty(max(bl_backward_workspace_size(M, N, K), 16), dtype=torch.uint8, device=device),
         )
 
 

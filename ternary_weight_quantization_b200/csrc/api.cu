@@ -210,13 +210,13 @@ static bl_status backward_common(const void* dY, const int8_t* xq, const float* 
       (w_packed && !aligned16(w_packed)) || (gamma && !aligned16(gamma)) || (dX && !aligned16(dX)) ||
       (dW && !aligned16(dW)))
     return fail(BL_ERR_ALIGNMENT, "tensors must be 16-byte aligned");
-  if (workspace) {
-    const size_t need = bl_backward_workspace_size(M, K);
+  if (workspace && bl::backward_uses_xhat(N)) {
+    const size_t need = bl_backward_workspace_size(M, N, K);
     if (workspace_bytes < need || !aligned16(workspace))
       return fail(BL_ERR_WORKSPACE, "workspace needs %zu bytes, 16-byte aligned", need);
   }
-  // x_hat is only worth making when dW is computed from tokens
-  void* xhat = (workspace && dW && M > 0) ? workspace : nullptr;
+  // x_hat is only made when dW is computed from tokens and worth it
+  void* xhat = (workspace && dW && M > 0 && bl::backward_uses_xhat(N)) ? workspace : nullptr;
   int* err = nullptr;
   if (bl_status s = current_device(&err)) return s;
   return cuda_status(bl::launch_backward(dY, xq, sx, w_packed, gamma, M, N, K, dX, dW,
@@ -225,8 +225,8 @@ static bl_status backward_common(const void* dY, const int8_t* xq, const float* 
                      what);
 }
 
-size_t bl_backward_workspace_size(int64_t M, int64_t K) {
-  return (M > 0 && K > 0) ? static_cast<size_t>(M) * static_cast<size_t>(K) * 2 : 0;
+size_t bl_backward_workspace_size(int64_t M, int64_t N, int64_t K) {
+  return (M > 0 && K > 0 && bl::backward_uses_xhat(N)) ? static_cast<size_t>(M) * static_cast<size_t>(K) * 2 : 0;
 }
 
 bl_status bl_backward(const void* dY, const int8_t* xq, const float* sx, const uint8_t* w_packed,

@@ -79,6 +79,10 @@ cudaError_t launch_forward(const int8_t* xq, const float* sx, const uint8_t* w_p
                            int64_t M, int64_t N, int64_t K, void* y, int32_t* debug_acc, int* err,
                            cudaStream_t s);
 
+// Whether the backward makes x_hat in a workspace for dW with N features
+// (else it rebuilds x_hat in every dW tile).
+bool backward_uses_xhat(int64_t N);
+
 // dX and/or dW (either output may be null) in one launch. With dw_signs, dW
 // receives the sign words of dW ([N*K/32] uint32, element 32w + j at bit j of
 // word w) instead of dW itself. With xhat_ws (bf16 [M][K], 16-byte aligned), a

@@ -1658,6 +1658,14 @@ cudaError_t launch_forward(const int8_t* xq, const float* sx, const uint8_t* w_p
   return launch_pair<Family::Fwd, 128>(maps, p, npairs, s);
 }
 
+// x_hat is made in the workspace only where its rebuilds would cost more
+// than the extra launch: every dW tile column block (256 features) rebuilds
+// all of x_hat once, and the launch moves 3 bytes per element. Measured on
+// B200 (CUDA graphs, rebuild against workspace, interleaved): 27 blocks
+// (N 6912) 213.8 -> 205.8 us, 10 blocks (N 2560) 116.2 -> 117.4 us; the
+// break-even is near 12 blocks.
+bool backward_uses_xhat(int64_t N) { return N >= 12 * 256; }
+
 // dX and/or dW in one launch (either output may be null).
 cudaError_t launch_backward(const void* dY, const int8_t* xq, const float* sx, const uint8_t* w_packed,
                             const float* gamma, int64_t M, int64_t N, int64_t K, void* dX, void* dW, int dw_is_f32,
@@ -1671,14 +1679,7 @@ cudaError_t launch_backward(const void* dY, const int8_t* xq, const float* sx, c
   }
   if (M == 0) return cudaSuccess;
   constexpr int BN = 256;
-  // x_hat is made in the workspace only where its rebuilds would cost more
-  // than the extra launch: every dW tile column block (256 features) rebuilds
-  // all of x_hat once, and the launch moves 3 bytes per element. Measured on
-  // B200 (CUDA graphs, rebuild against workspace, interleaved): 27 blocks
-  // (N 6912) 220.7 -> 213.5 us, 10 blocks (N 2560) 116.2 -> 117.4 us; the
-  // break-even is near 12 blocks.
-  constexpr int64_t kXhatMinN = 12 * 256;
-  if (N < kXhatMinN) xhat_ws = nullptr;
+  if (!backward_uses_xhat(N)) xhat_ws = nullptr;
   const int npairs = resident_pairs<Family::Bwd, BN>();
   CUtensorMap maps[7] = {};  // b0, src0, out0, b1, src1, out1, sx
   const bool src_tma = (K % 64) == 0;

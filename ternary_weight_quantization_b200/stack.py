@@ -58,9 +58,7 @@ class BitLinearStack:
         big = M * max(dims)
         s.act = [torch.empty(big, dtype=torch.bfloat16, device=device) for _ in range(2)]
         s.grad = [torch.empty(big, dtype=torch.bfloat16, device=device) for _ in range(2)]
-        # the library makes x_hat in the workspace only for layers with at
-        # least 3072 output features (bl_backward_ws)
-        need = max([b.bl_backward_workspace_size(M, K) for K, N in zip(dims[:-1], dims[1:]) if N >= 3072] or [0])
+        need = max(b.bl_backward_workspace_size(M, N, K) for K, N in zip(dims[:-1], dims[1:]))
         s.bwd_workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=device)
         return s
 

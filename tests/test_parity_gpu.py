@@ -522,7 +522,7 @@ def test_backward_workspace_matches_rebuild(M, N, K, dw_dtype, accumulate):
     xd, wd, dyd = x.cuda(), w.cuda(), dy.cuda()
     bl.bl_quantize_weight(wd, bufs.w_packed, bufs.gamma, bufs.workspace)
     bl.bl_quantize_act(xd, bufs.xq, bufs.sx)
-    ws = torch.full((bl.bl_backward_workspace_size(M, K),), 0xAB, dtype=torch.uint8, device="cuda")
+    ws = torch.full((max(bl.bl_backward_workspace_size(M, N, K), 16),), 0xAB, dtype=torch.uint8, device="cuda")
     prev = (torch.randn(N, K, generator=torch.Generator().manual_seed(5)) * 3).to(dw_dtype).cuda()
     outs = []
     for workspace in (None, ws):
