@@ -28,6 +28,9 @@
 // k-blocks) are spread over the CTA pairs by a longest-processing-time
 // schedule computed on the host and passed in the kernel parameters, so the
 // pairs finish together instead of idling through a partly filled last wave.
+// Given a workspace and N >= 3072, a launch before it writes x_hat once
+// (xhat_kernel) and dW's stages load their A operand from there by TMA
+// instead of rebuilding it (every dW tile would rebuild its x_hat slab).
 //
 // Warp w runs on SM sub-partition w % 4. Roles (512 threads per CTA):
 //   warp 0      loads: TMA for B, for Dw's q / s_x and for the packed codes

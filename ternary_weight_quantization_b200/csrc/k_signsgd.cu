@@ -7,12 +7,15 @@
 //   G1 sign words   dW -> one sign bit per weight, 32 to a word
 //   G2 vote         R ranks' sign words -> majority direction, 2-bit packed
 //   G3 update       W <- dtype_rn(fp32(W) - lr * direction) where W is held
+//   G2 + G3 + S1    the holder's vote and update in one sweep that also forms
+//                   S1's |W| partial sums, followed by S1's code launch
 //
-// All three are HBM-bound streaming passes with 16-byte vector loads. Each
-// thread takes U items spaced one grid apart (so every load instruction of a
-// warp stays contiguous) and issues all of their loads before it computes:
-// with the grid sized to the work, the whole tensor is in flight in about one
-// round trip instead of several dependent ones.
+// The three separate passes are HBM-bound streams with 16-byte vector loads.
+// Each thread takes U items spaced one grid apart (so every load instruction
+// of a warp stays contiguous) and issues all of their loads before it
+// computes: with the grid sized to the work, the whole tensor is in flight in
+// about one round trip instead of several dependent ones. The fused sweep
+// works in warp rounds of 32 word positions (see signsgd_apply_kernel).
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
