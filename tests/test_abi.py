@@ -44,6 +44,15 @@ def test_workspace_size():
     assert b.bl_quantize_weight_workspace_size(6912, 2560) == 128 + 8 * 256 + 128 + 8 * 1024
 
 
+def test_backward_workspace_size():
+    # x_hat as bf16 [M][K] where dW has at least 3072 features; nothing below
+    assert b.bl_backward_workspace_size(4096, 6912, 2560) == 4096 * 2560 * 2
+    assert b.bl_backward_workspace_size(7, 3072, 96) == 7 * 96 * 2
+    assert b.bl_backward_workspace_size(2048, 2560, 6912) == 0
+    assert b.bl_backward_workspace_size(4096, 3064, 2560) == 0
+    assert b.bl_backward_workspace_size(0, 6912, 2560) == 0
+
+
 FAKE = ctypes.c_void_p(0x10000)        # never dereferenced: validation fails first
 MISALIGNED = ctypes.c_void_p(0x10008)
 
@@ -63,6 +72,12 @@ MISALIGNED = ctypes.c_void_p(0x10008)
     (lambda L: L.bl_backward(FAKE, FAKE, FAKE, FAKE, FAKE, 4, 12, 64, FAKE, FAKE, 0, 0, None), 2),  # N % 8
     (lambda L: L.bl_backward(FAKE, FAKE, FAKE, FAKE, FAKE, 4, 16, 64, FAKE, FAKE, 9, 0, None), 3),
     (lambda L: L.bl_backward(FAKE, FAKE, FAKE, None, FAKE, 4, 16, 64, FAKE, None, 0, 0, None), 1),
+    (lambda L: L.bl_backward_ws(FAKE, FAKE, FAKE, FAKE, FAKE, 4, 3072, 64, FAKE, FAKE, 0, 0, FAKE, 64, None),
+     8),                                                                       # workspace too small
+    (lambda L: L.bl_backward_ws(FAKE, FAKE, FAKE, FAKE, FAKE, 4, 3072, 64, FAKE, FAKE, 0, 0, MISALIGNED, 1 << 20,
+                                None), 8),                                     # workspace misaligned
+    (lambda L: L.bl_backward_signs_ws(FAKE, FAKE, FAKE, FAKE, FAKE, 4, 3072, 64, FAKE, None, FAKE, 1 << 20, None),
+     1),                                                                       # no sign words
     (lambda L: L.bl_export_weights(FAKE, FAKE, 4, 64, None, FAKE, None), 1),
     (lambda L: L.bl_sign_pack(FAKE, 0, 4, 48, FAKE, None), 2),               # K % 32
     (lambda L: L.bl_sign_pack(FAKE, 5, 4, 64, FAKE, None), 3),
@@ -74,6 +89,10 @@ MISALIGNED = ctypes.c_void_p(0x10008)
     (lambda L: L.bl_signsgd_update(FAKE, 0, 4, 64, FAKE, float("nan"), None), 1),
     (lambda L: L.bl_signsgd_update(FAKE, 2, 4, 64, FAKE, 0.1, None), 3),
     (lambda L: L.bl_signsgd_update(FAKE, 0, 0, 64, FAKE, 0.1, None), 1),
+    (lambda L: L.bl_signsgd_apply(FAKE, 0, FAKE, 0, 4, 64, 0.1, FAKE, FAKE, FAKE, 1 << 20, None), 1),  # ranks
+    (lambda L: L.bl_signsgd_apply(FAKE, 2, FAKE, 0, 4, 64, float("nan"), FAKE, FAKE, FAKE, 1 << 20, None), 1),
+    (lambda L: L.bl_signsgd_apply(FAKE, 2, FAKE, 0, 4, 64, 0.1, FAKE, FAKE, FAKE, 64, None), 8),  # workspace
+    (lambda L: L.bl_signsgd_apply(FAKE, 2, FAKE, 0, 4, 48, 0.1, FAKE, FAKE, FAKE, 1 << 20, None), 2),  # K % 32
 ])
 def test_host_validation_without_gpu(call, expect):
     lib = b.load_library()
