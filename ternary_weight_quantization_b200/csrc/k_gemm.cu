@@ -539,6 +539,14 @@ __device__ __forceinline__ void st_shared_b32(uint32_t addr, uint32_t v) {
   asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
 }
 
+__device__ __forceinline__ void st_shared_b16(uint32_t addr, uint32_t v) {
+  asm volatile("st.shared.b16 [%0], %1;" ::"r"(addr), "h"(static_cast<unsigned short>(v)) : "memory");
+}
+
+__device__ __forceinline__ uint64_t pair_u64(uint32_t lo, uint32_t hi) {
+  return (static_cast<uint64_t>(hi) << 32) | lo;
+}
+
 // Epilogue paths taken for f32 output, accumulation, the debug output and
 // row pitches a tensor map cannot take: kept out of line so that the common
 // bf16 path stays small in the instruction caches.
@@ -633,40 +641,50 @@ __device__ __forceinline__ void epilogue_chunk(const GemmParams& p, const OpPara
   const uint32_t slot = stg + (seq % kSlots) * 2048u;
   if (lane == 0) bulk_wait_group_read<kSlots - 1>();  // the box last stored from this slot has been read
   __syncwarp();
-  // values of this lane's column for the chunk's 32 rows
-  float v[32];
+  // This lane's column for the chunk's 32 rows: rows 2 pr and 2 pr + 1 are
+  // converted together (packed fp32x2 arithmetic, each half rounded like the
+  // scalar instruction, then one bf16x2 conversion) and written to their two
+  // rows of the staging box by two 16-bit stores.
+  const uint32_t col = slot + static_cast<uint32_t>(lane) * 2;
   if constexpr (op == Op::Fwd) {
     // exact int32 -> fp32 through the 1.5 * 2^23 shifter (|acc| <= 127 K < 2^22)
     // when K allows, else the conversion instruction; then one rounding by
     // the row's scale, read from the warp's table (broadcast loads)
     const bool shifter = P.red <= kShifterMaxK;
+    constexpr uint64_t kMagic2 = 0x4B4000004B400000ull;  // {1.5 * 2^23, 1.5 * 2^23}
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
       const float4 sc = ld_shared_f4(scales + (c * 32 + 4 * u) * 4);
       const float sv[4] = {sc.x, sc.y, sc.z, sc.w};
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const uint32_t a = r[4 * u + e];
-        const float f = shifter ? __fsub_rn(__int_as_float(static_cast<int>(a) + 0x4B400000), 12582912.0f)
-                                : static_cast<float>(static_cast<int32_t>(a));
-        v[4 * u + e] = __fmul_rn(f, sv[e]);
+      for (int h = 0; h < 2; ++h) {
+        const int j = 4 * u + 2 * h;
+        uint64_t f2;
+        if (shifter) {
+          f2 = f32x2_sub(pair_u64(r[j] + 0x4B400000u, r[j + 1] + 0x4B400000u), kMagic2);
+        } else {
+          f2 = pair_u64(__float_as_uint(static_cast<float>(static_cast<int32_t>(r[j]))),
+                        __float_as_uint(static_cast<float>(static_cast<int32_t>(r[j + 1]))));
+        }
+        const uint32_t b2 =
+            f32x2_to_bf16x2(f32x2_mul(f2, pair_u64(__float_as_uint(sv[2 * h]), __float_as_uint(sv[2 * h + 1]))));
+        st_shared_b16(col + j * 64, b2);
+        st_shared_b16(col + (j + 1) * 64, b2 >> 16);
       }
     }
   } else {
 #pragma unroll
-    for (int jj = 0; jj < 32; ++jj) v[jj] = epi_value<op>(r[jj], gamma);
-  }
-  // lanes 2k and 2k+1 swap one value per pair of rows, so that each holds two
-  // adjacent columns of one row: one bf16x2 conversion and one 32-bit store
-  const bool odd = lane & 1;
-  const uint32_t col_bytes = static_cast<uint32_t>(lane & ~1) * 2;
-#pragma unroll
-  for (int pr = 0; pr < 16; ++pr) {
-    const float send = odd ? v[2 * pr] : v[2 * pr + 1];
-    const float recv = __shfl_xor_sync(0xffffffffu, send, 1);
-    const float lo = odd ? recv : v[2 * pr];
-    const float hi = odd ? v[2 * pr + 1] : recv;
-    st_shared_b32(slot + (2 * pr + (odd ? 1 : 0)) * 64 + col_bytes, cvt_bf16x2(hi, lo));
+    for (int pr = 0; pr < 16; ++pr) {
+      const int j = 2 * pr;
+      uint32_t b2;
+      if constexpr (op == Op::Dx)
+        b2 = f32x2_to_bf16x2(f32x2_mul(pair_u64(r[j], r[j + 1]),
+                                       pair_u64(__float_as_uint(gamma), __float_as_uint(gamma))));
+      else
+        b2 = f32x2_to_bf16x2(pair_u64(r[j], r[j + 1]));
+      st_shared_b16(col + j * 64, b2);
+      st_shared_b16(col + (j + 1) * 64, b2 >> 16);
+    }
   }
   fence_proxy_async_smem();
   __syncwarp();
