@@ -3,7 +3,7 @@
 One step = one pass of the whole hot path over one batch:
   S1 + S2 bl_quantize (2 launches: |W| partial sums with part of the token
   rows, then gamma and the codes with the other rows) -> S3 bl_forward
-  -> S4 bl_backward with its x_hat workspace (for N >= 3072 one launch makes
+  -> S4 bl_backward with its x_hat workspace (for N >= 2048 one launch makes
   x_hat, then dX and dW in one launch)                   (4 or 5 launches)
 
 Default workload: the up-projection BitLinear 2560 -> 6912 at 8 x 512 tokens
@@ -186,8 +186,8 @@ STAGES = ["quantize", "forward", "backward"]
 def launches_per_step(N):
     """S1 sums (+ S2 rows); S1 codes (+ S2 rows); S3; S4: dX and dW in one
     launch, after one that makes x_hat in the backward's workspace where dW
-    has N >= 3072 features (below that the library rebuilds x_hat instead)."""
-    return 5 if N >= 3072 else 4
+    has N >= 2048 features (below that the library rebuilds x_hat instead)."""
+    return 5 if N >= 2048 else 4
 
 
 def stage_work(M, N, K, w_bytes):

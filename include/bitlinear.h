@@ -228,7 +228,7 @@ bl_status bl_backward(const void* dY, const int8_t* xq, const float* sx,
  * nothing the caller needs afterwards), owned by the caller, 16-byte
  * aligned, of at least bl_backward_workspace_size(M, N, K) bytes, and needs
  * no initialisation; one call at a time per workspace. workspace == NULL: as
- * bl_backward. Where dW has fewer than 3072 features (12 blocks of 256, each
+ * bl_backward. Where dW has fewer than 2048 features (8 blocks of 256, each
  * of which rebuilds x_hat once) the extra launch costs more than it saves:
  * the size is then 0 and the workspace is not used (any pointer, or NULL).
  * Errors: as bl_backward, plus BL_ERR_WORKSPACE.

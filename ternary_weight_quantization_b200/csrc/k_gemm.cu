@@ -28,7 +28,7 @@
 // k-blocks) are spread over the CTA pairs by a longest-processing-time
 // schedule computed on the host and passed in the kernel parameters, so the
 // pairs finish together instead of idling through a partly filled last wave.
-// Given a workspace and N >= 3072, a launch before it writes x_hat once
+// Given a workspace and N >= 2048, a launch before it writes x_hat once
 // (xhat_kernel) and dW's stages load their A operand from there by TMA
 // instead of rebuilding it (every dW tile would rebuild its x_hat slab).
 //
@@ -1387,35 +1387,41 @@ __global__ void zero_dw_kernel(void* out, int64_t n, int out_f32, int accumulate
 // workspace, converted exactly as the dW rebuild does (s8x16_to_bf16), so
 // that dW tiles can load their A operand by TMA instead of rebuilding it in
 // every tile (each x_hat element would otherwise be rebuilt once per
-// 256-feature block of dW). Thread t takes kXhatU 16-element chunks spaced
-// one grid apart, all loads issued first (16-byte loads, two 16-byte stores
-// per chunk); the grid is sized so that one pass covers xq.
-constexpr int kXhatU = 4;
+// 256-feature block of dW). A chunk is 8 values: an 8-byte load and one
+// 16-byte store, so consecutive lanes read 256 and write 512 contiguous bytes
+// per warp access (whole 32-byte sectors). Thread t takes kXhatU chunks
+// spaced one grid apart, all loads issued first, in a grid of up to 16 CTAs
+// per SM. Measured on B200 at 4096 x 2560 (CUDA graphs, one box): 6.5 us
+// with 2 chunks per thread, 6.8 with 4, 7.4 with 8, 10.1 with 16; 9.2 us
+// for 16-value chunks (16-byte loads, two 16-byte stores 32 bytes apart).
+constexpr int kXhatU = 2;
 
-__global__ void __launch_bounds__(256) xhat_kernel(const uint4* __restrict__ xq, const float* __restrict__ sx,
+__global__ void __launch_bounds__(256) xhat_kernel(const uint2* __restrict__ xq, const float* __restrict__ sx,
                                                    int64_t chunks, int chunks_per_row, uint4* __restrict__ out) {
   pdl_wait_primary();
   pdl_launch_dependents();
   const int64_t T = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  const bool narrow = chunks <= 0xFFFFFFFFll;  // the row index by 32-bit division
   for (int64_t c0 = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; c0 < chunks; c0 += kXhatU * T) {
-    uint4 v[kXhatU];
+    uint2 v[kXhatU];
     float s[kXhatU];
 #pragma unroll
     for (int u = 0; u < kXhatU; ++u) {
       const int64_t c = c0 + u * T;
       if (c < chunks) {
         v[u] = __ldg(xq + c);
-        s[u] = __ldg(sx + c / chunks_per_row);
+        const int64_t row = narrow ? static_cast<int64_t>(static_cast<uint32_t>(c) / static_cast<uint32_t>(chunks_per_row))
+                                   : c / chunks_per_row;
+        s[u] = __ldg(sx + row);
       }
     }
 #pragma unroll
     for (int u = 0; u < kXhatU; ++u) {
       const int64_t c = c0 + u * T;
       if (c < chunks) {
-        uint4 o0, o1;
-        s8x16_to_bf16(v[u], s[u], o0, o1);
-        out[2 * c] = o0;
-        out[2 * c + 1] = o1;
+        uint4 o0, o1;  // o1 (values 8..15 of a 16-value chunk) is not needed
+        s8x16_to_bf16(make_uint4(v[u].x, v[u].y, 0u, 0u), s[u], o0, o1);
+        out[c] = o0;
       }
     }
   }
@@ -1683,9 +1689,10 @@ cudaError_t launch_forward(const int8_t* xq, const float* sx, const uint8_t* w_p
 // than the extra launch: every dW tile column block (256 features) rebuilds
 // all of x_hat once, and the launch moves 3 bytes per element. Measured on
 // B200 (CUDA graphs, rebuild against workspace, interleaved): 27 blocks
-// (N 6912) 213.8 -> 205.8 us, 10 blocks (N 2560) 116.2 -> 117.4 us; the
-// break-even is near 12 blocks.
-bool backward_uses_xhat(int64_t N) { return N >= 12 * 256; }
+// (N 6912, K 2560) 213.8 -> 205.8 us with the first form of the launch;
+// with the current one (6.5 us at 4096 x 2560) 10 blocks (N 2560, K 6912)
+// 117.3 -> 115.0 us. The break-even is near 7 blocks.
+bool backward_uses_xhat(int64_t N) { return N >= 8 * 256; }
 
 // dX and/or dW in one launch (either output may be null).
 cudaError_t launch_backward(const void* dY, const int8_t* xq, const float* sx, const uint8_t* w_packed,
@@ -1758,11 +1765,11 @@ cudaError_t launch_backward(const void* dY, const int8_t* xq, const float* sx, c
   p.gamma = dX ? gamma : nullptr;
   p.err = err;
   if (dW && xhat_ws) {
-    const int64_t chunks = M * K / 16;
+    const int64_t chunks = M * K / 8;
     const int64_t want = (chunks + 256 * kXhatU - 1) / (256 * kXhatU);
-    const int64_t cap = static_cast<int64_t>(8) * device_sm_count();
+    const int64_t cap = static_cast<int64_t>(16) * device_sm_count();
     cudaError_t e = launch_pdl(xhat_kernel, dim3(static_cast<unsigned>(want < cap ? want : cap)), dim3(256), 0, s,
-                               reinterpret_cast<const uint4*>(xq), sx, chunks, static_cast<int>(K / 16),
+                               reinterpret_cast<const uint2*>(xq), sx, chunks, static_cast<int>(K / 8),
                                static_cast<uint4*>(xhat_ws));
     if (e != cudaSuccess) return e;
   }

@@ -45,11 +45,11 @@ def test_workspace_size():
 
 
 def test_backward_workspace_size():
-    # x_hat as bf16 [M][K] where dW has at least 3072 features; nothing below
+    # x_hat as bf16 [M][K] where dW has at least 2048 features; nothing below
     assert b.bl_backward_workspace_size(4096, 6912, 2560) == 4096 * 2560 * 2
-    assert b.bl_backward_workspace_size(7, 3072, 96) == 7 * 96 * 2
-    assert b.bl_backward_workspace_size(2048, 2560, 6912) == 0
-    assert b.bl_backward_workspace_size(4096, 3064, 2560) == 0
+    assert b.bl_backward_workspace_size(7, 2048, 96) == 7 * 96 * 2
+    assert b.bl_backward_workspace_size(2048, 2560, 6912) == 2048 * 6912 * 2
+    assert b.bl_backward_workspace_size(4096, 2040, 2560) == 0
     assert b.bl_backward_workspace_size(0, 6912, 2560) == 0
 
 
@@ -72,11 +72,11 @@ MISALIGNED = ctypes.c_void_p(0x10008)
     (lambda L: L.bl_backward(FAKE, FAKE, FAKE, FAKE, FAKE, 4, 12, 64, FAKE, FAKE, 0, 0, None), 2),  # N % 8
     (lambda L: L.bl_backward(FAKE, FAKE, FAKE, FAKE, FAKE, 4, 16, 64, FAKE, FAKE, 9, 0, None), 3),
     (lambda L: L.bl_backward(FAKE, FAKE, FAKE, None, FAKE, 4, 16, 64, FAKE, None, 0, 0, None), 1),
-    (lambda L: L.bl_backward_ws(FAKE, FAKE, FAKE, FAKE, FAKE, 4, 3072, 64, FAKE, FAKE, 0, 0, FAKE, 64, None),
+    (lambda L: L.bl_backward_ws(FAKE, FAKE, FAKE, FAKE, FAKE, 4, 2048, 64, FAKE, FAKE, 0, 0, FAKE, 64, None),
      8),                                                                       # workspace too small
-    (lambda L: L.bl_backward_ws(FAKE, FAKE, FAKE, FAKE, FAKE, 4, 3072, 64, FAKE, FAKE, 0, 0, MISALIGNED, 1 << 20,
+    (lambda L: L.bl_backward_ws(FAKE, FAKE, FAKE, FAKE, FAKE, 4, 2048, 64, FAKE, FAKE, 0, 0, MISALIGNED, 1 << 20,
                                 None), 8),                                     # workspace misaligned
-    (lambda L: L.bl_backward_signs_ws(FAKE, FAKE, FAKE, FAKE, FAKE, 4, 3072, 64, FAKE, None, FAKE, 1 << 20, None),
+    (lambda L: L.bl_backward_signs_ws(FAKE, FAKE, FAKE, FAKE, FAKE, 4, 2048, 64, FAKE, None, FAKE, 1 << 20, None),
      1),                                                                       # no sign words
     (lambda L: L.bl_export_weights(FAKE, FAKE, 4, 64, None, FAKE, None), 1),
     (lambda L: L.bl_sign_pack(FAKE, 0, 4, 48, FAKE, None), 2),               # K % 32
