@@ -302,10 +302,40 @@ def run_ours(args, rank, world, local_rank):
     if bl.bl_get_last_error() != 0:
         raise RuntimeError("device error during warm-up")
 
-    def timed(per_stage):
+    # The step's C-ABI calls captured once into a CUDA graph (their tensor maps
+    # and launch shapes are fixed by the buffers), then replayed: one host
+    # launch per step instead of the Python-side issue of every call, which
+    # on a slow host leaves gaps between the step's kernels. Every kernel of
+    # the step runs on every replay. The all-reduce of N > 1 is issued after
+    # each replay, outside the graph.
+    def compute(st):
+        bl.bl_quantize(w, x, bufs.w_packed, bufs.gamma, bufs.xq, bufs.sx, bufs.workspace, st)
+        bl.bl_forward(bufs.xq, bufs.sx, bufs.w_packed, bufs.gamma, bufs.y, None, st)
+        bl.bl_backward(dy, bufs.xq, bufs.sx, bufs.w_packed, bufs.gamma, bufs.dX, bufs.dW, False, st,
+                       workspace=bufs.bwd_workspace)
+
+    graph = None
+    if not args.eager:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            compute(torch.cuda.current_stream(dev))
+        torch.cuda.synchronize(dev)
+
+    def graph_step():
+        graph.replay()
+        if world > 1:
+            torch.distributed.all_reduce(bufs.dW)
+
+    for i in range(args.warmup if graph is not None else 0):
+        flush_l2(i)
+        graph_step()
+    torch.cuda.synchronize(dev)
+
+    def timed(per_stage, replay=False):
         """K steps, L2 flushed before each. per_stage: events between the C-ABI
         calls (kernel breakdown); otherwise events only around each step, so
-        consecutive kernels keep their programmatic-launch overlap."""
+        consecutive kernels keep their programmatic-launch overlap. replay:
+        the step as the captured graph (plus the all-reduce for N > 1)."""
         n_ev = len(STAGES) + 1 + (world > 1) if per_stage else 2
         evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
         if world > 1:
@@ -317,7 +347,7 @@ def run_ours(args, rank, world, local_rank):
                 step(evs[i])
             else:
                 evs[i][0].record(stream)
-                step()
+                graph_step() if replay else step()
                 evs[i][1].record(stream)
         torch.cuda.synchronize(dev)
         if world > 1:
@@ -334,15 +364,17 @@ def run_ours(args, rank, world, local_rank):
 
     sampler = ClockSampler(dev.index if dev.index is not None else 0)
     sampler.start()
-    total_ms, _ = timed(False)
+    total_ms, _ = timed(False, graph is not None)
     clocks = sampler.stop()
     remeasured = False
     if sampler.rejected(clocks):
         sampler = ClockSampler(dev.index if dev.index is not None else 0)
         sampler.start()
-        total_ms, _ = timed(False)
+        total_ms, _ = timed(False, graph is not None)
         clocks = sampler.stop()
         remeasured = True
+    eager_ms = timed(False)[0] if graph is not None else total_ms
+    del graph
     breakdown_ms, per_stage = timed(True)
     clocks["remeasured"] = remeasured
     graph_ms = stage_graph_ms(bl, x, w, dy, M, N, K, dev)
@@ -350,6 +382,7 @@ def run_ours(args, rank, world, local_rank):
         raise RuntimeError("device error during the timed region")
 
     job_ms = job_time_ms(total_ms, world, dev)
+    eager_job_ms = job_time_ms(eager_ms, world, dev)
 
     e2e = measure_e2e(bl, args, dev, stream, bufs, x_cpu, w_cpu, dy_cpu, world)
     if rank != 0:
@@ -400,6 +433,9 @@ def run_ours(args, rank, world, local_rank):
                    if world > 1 else "single GPU"},
         "roofline": roofline,
         "step_roofline_frac": round(roof_ms / ms_per_step, 4),
+        "launch": "one CUDA graph replay per step (the step's C-ABI calls captured once)"
+        if not args.eager else "the step's C-ABI calls issued from Python every step",
+        "ms_per_step_eager": round(eager_job_ms / args.steps, 5),
         "kernel_breakdown_ms_per_step": round(breakdown_ms / args.steps, 5),
         "kernels": kernels,
         **({"allreduce_ms_per_step": round(per_stage["allreduce"] / args.steps, 5),
@@ -584,9 +620,9 @@ def run_stack(args, rank, world, local_rank):
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
-    def step():
-        st.forward(x, ws, stream)
-        st.backward(dy, True, stream)
+    def step(s=stream):
+        st.forward(x, ws, s)
+        st.backward(dy, True, s)
 
     for i in range(args.warmup):
         flush.fill_(i & 0xFF)
@@ -596,26 +632,43 @@ def run_stack(args, rank, world, local_rank):
     if bl.bl_get_last_error() != 0:
         raise RuntimeError("device error during warm-up")
     peak_mb = (torch.cuda.max_memory_allocated(dev) - base - flush.numel()) / 1e6
+    # the step's calls captured once into a CUDA graph and replayed (every
+    # kernel of the step on every replay), as in the single-layer mode
+    graph = None
+    if not args.eager:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            step(torch.cuda.current_stream(dev))
+        torch.cuda.synchronize(dev)
+
+    def timed(replay):
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize(dev)
+        for i in range(args.steps):
+            flush.fill_(i & 0xFF)
+            flush.view(torch.int64).max()
+            evs[i][0].record(stream)
+            graph.replay() if replay else step()
+            evs[i][1].record(stream)
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            torch.distributed.barrier()
+        return sum(e[0].elapsed_time(e[1]) for e in evs)
+
+    if graph is not None:
+        timed(True)  # warm-up replays
     sampler = ClockSampler(dev.index if dev.index is not None else 0)
     sampler.start()
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
-    if world > 1:
-        torch.distributed.barrier()
-    torch.cuda.synchronize(dev)
-    for i in range(args.steps):
-        flush.fill_(i & 0xFF)
-        flush.view(torch.int64).max()
-        evs[i][0].record(stream)
-        step()
-        evs[i][1].record(stream)
-    torch.cuda.synchronize(dev)
-    if world > 1:
-        torch.distributed.barrier()
+    total = timed(graph is not None)
     clocks = sampler.stop()
+    eager_total = timed(False) if graph is not None else total
+    del graph
     if bl.bl_get_last_error() != 0:
         raise RuntimeError("device error during the timed region")
-    total = sum(e[0].elapsed_time(e[1]) for e in evs)
     job_ms = job_time_ms(total, world, dev)
+    eager_job_ms = job_time_ms(eager_total, world, dev)
     if rank != 0:
         return None
     ops_step = 6.0 * M * sum(k * n for k, n in zip(dims[:-1], dims[1:]))
@@ -629,6 +682,9 @@ def run_stack(args, rank, world, local_rank):
         "config": {"workload": args.stack, "M": M, "dims": dims, "layers": len(dims) - 1,
                    "l2": "flushed before every step (256 MiB written, then read back)",
                    "parallelism": f"dp{world} independent replicas" if world > 1 else "single GPU"},
+        "launch": "one CUDA graph replay per step (the step's C-ABI calls captured once)"
+        if not args.eager else "the step's C-ABI calls issued from Python every step",
+        "ms_per_step_eager": round(eager_job_ms / args.steps, 5),
         "peak_device_memory_mb": round(peak_mb, 1),
         "saved_state_mb": round(saved / 1e6, 2),
         "gpu_launches": sum(launches_per_step(n) for n in dims[1:]) * args.steps,
@@ -901,11 +957,13 @@ def run_extras(args, local_rank):
     down = copy.copy(short)
     down.workload, down.no_cpu_baseline = "down_proj", True
     line = run_ours(down, 0, 1, local_rank)
-    extras["down_proj"] = keep(line, ["value", "unit", "ms_per_step", "roofline", "kernels", "clocks"])
+    extras["down_proj"] = keep(line, ["value", "unit", "ms_per_step", "ms_per_step_eager", "roofline", "kernels",
+                                      "clocks"])
     st = copy.copy(short)
     st.stack = "stack8"
     line = run_stack(st, 0, 1, local_rank)
-    extras["stack8"] = keep(line, ["value", "unit", "ms_per_step", "peak_device_memory_mb", "saved_state_mb",
+    extras["stack8"] = keep(line, ["value", "unit", "ms_per_step", "ms_per_step_eager", "peak_device_memory_mb",
+                                   "saved_state_mb",
                                    "config", "clocks"])
     ft = copy.copy(short)
     ft.few_tokens = "1,2,4,8,16"
@@ -928,6 +986,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=["up_proj", "down_proj", "tiny"], default="up_proj")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--eager", action="store_true",
+                    help="issue the step's calls from Python every step instead of replaying a CUDA graph of them")
     ap.add_argument("--cpu-tokens", type=int, default=4096)
     ap.add_argument("--stack", choices=["stack8"], default=None,
                     help="layer-stack mode (prints its own line instead of the single-layer one)")
