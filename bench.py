@@ -230,7 +230,7 @@ def stage_graph_ms(bl, x, w, dy, M, N, K, dev, n_sets=4, calls=16, reps=5):
         torch.cuda.current_stream(dev).wait_stream(side)
         torch.cuda.synchronize(dev)
         g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
+        with torch.cuda.graph(g, capture_error_mode="thread_local"):
             for i in range(calls):
                 call(sets[i % n_sets])
         ts = []
@@ -317,7 +317,9 @@ def run_ours(args, rank, world, local_rank):
     graph = None
     if not args.eager:
         graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph):
+        # thread-local capture: CUDA calls of other threads (the process
+        # group's watchdog under torchrun) do not invalidate the capture
+        with torch.cuda.graph(graph, capture_error_mode="thread_local"):
             compute(torch.cuda.current_stream(dev))
         torch.cuda.synchronize(dev)
 
@@ -637,7 +639,7 @@ def run_stack(args, rank, world, local_rank):
     graph = None
     if not args.eager:
         graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph):
+        with torch.cuda.graph(graph, capture_error_mode="thread_local"):
             step(torch.cuda.current_stream(dev))
         torch.cuda.synchronize(dev)
 
@@ -744,7 +746,7 @@ def run_few_tokens(args, rank, world, local_rank):
         torch.cuda.current_stream(dev).wait_stream(side)
         torch.cuda.synchronize(dev)
         g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
+        with torch.cuda.graph(g, capture_error_mode="thread_local"):
             for c in copies:
                 bl.bl_forward(xq, sx, c, gamma, y)
         gt = []
