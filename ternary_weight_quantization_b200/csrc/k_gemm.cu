@@ -648,9 +648,10 @@ __device__ __forceinline__ void epilogue_chunk(const GemmParams& p, const OpPara
   const uint32_t col = slot + static_cast<uint32_t>(lane) * 2;
   if constexpr (op == Op::Fwd) {
     // exact int32 -> fp32 through the 1.5 * 2^23 shifter (|acc| <= 127 K < 2^22)
-    // when K allows, else the conversion instruction; then one rounding by
-    // the row's scale, read from the warp's table (broadcast loads)
-    const bool shifter = P.red <= kShifterMaxK;
+    // when K allows (always in the lean instance), else the conversion
+    // instruction; then one rounding by the row's scale, read from the warp's
+    // table (broadcast loads)
+    const bool shifter = kLean || P.red <= kShifterMaxK;
     constexpr uint64_t kMagic2 = 0x4B4000004B400000ull;  // {1.5 * 2^23, 1.5 * 2^23}
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
@@ -1552,15 +1553,18 @@ void build_schedule(GemmParams& p, int npairs) {
 }
 
 // Whether every op with tiles takes the common paths: operands and packed
-// codes by TMA (x_hat from the workspace for dW) and bf16 outputs by TMA
-// store (no sign words, no accumulation, no debug output). Such launches run
-// the kernel instance compiled without the other paths (measured on B200:
-// forward 59.1 -> 58.1 us, backward 205.2 -> 204.9 us at up_proj, the
-// outputs unchanged).
-bool lean_params(const GemmParams& p) {
+// codes by TMA (x_hat from the workspace for dW), bf16 outputs by TMA store
+// (no sign words, no accumulation, no debug output) and, for the forward,
+// sums small enough for the shifter conversion. Such launches run the kernel
+// instance compiled without the other paths (measured on B200: forward
+// 59.1 -> 58.1 us, backward 205.2 -> 204.9 us at up_proj; the forward's
+// conversion then fixed to the shifter: 58.7 -> 57.4 us; the outputs
+// unchanged).
+bool lean_params(const GemmParams& p, bool fwd) {
   const OpParams& a = p.op[0];
   const OpParams& b = p.op[1];
-  const bool a_ok = a.ntiles == 0 || (a.src_tma && a.tma_store && !a.out_f32);
+  const bool a_ok =
+      a.ntiles == 0 || (a.src_tma && a.tma_store && !a.out_f32 && (!fwd || a.red <= kShifterMaxK));
   const bool b_ok = b.ntiles == 0 || (b.xhat_tma && b.tma_store && !b.out_f32 && !b.sign_words && !b.accumulate);
   return a_ok && b_ok && p.debug_acc == nullptr;
 }
@@ -1587,7 +1591,8 @@ cudaError_t launch_pair(const CUtensorMap* maps, GemmParams& p, int npairs, cuda
     std::fprintf(stderr, "[bitlinear] gemm family=%d BN=%d stages=%d smem=%d tiles=%d+%d kb=%d/%d pairs=%d sched=%d\n",
                  static_cast<int>(F), BN, L::kS, L::kDynBytes, p.op[0].ntiles, p.op[1].ntiles, p.op[0].num_kb,
                  p.op[1].num_kb, pairs, p.use_sched);
-  cudaError_t e = launch_pdl(lean_params(p) ? gemm_pair_kernel<F, BN, true> : gemm_pair_kernel<F, BN, false>,
+  cudaError_t e = launch_pdl(lean_params(p, F == Family::Fwd) ? gemm_pair_kernel<F, BN, true>
+                                                              : gemm_pair_kernel<F, BN, false>,
                              dim3(2 * pairs), dim3(kThreads), L::kDynBytes, s, maps[0], maps[1], maps[2], maps[3],
                              maps[4], maps[5], maps[6], p);
   if (e != cudaSuccess) return e;

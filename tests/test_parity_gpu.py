@@ -124,6 +124,27 @@ def test_forward_ragged_n(M, N, K):
     check_all(run_step(x, w, dy), oracle_step(x, w, dy), N)
 
 
+@pytest.mark.parametrize("M,N,K", [(40, 64, 33088), (300, 136, 33024)])
+def test_forward_tile_path_shifter_range(M, N, K):
+    """The tensor-core forward (more than 16 tokens) at K past the int32 ->
+    fp32 shifter's range (33088: conversion instruction, the general kernel
+    instance even without the debug output) and at its edge (33024: shifter,
+    the lean instance without the debug output): y with and without the
+    INT32 output bit for bit equal, and equal to the oracle."""
+    bl = _bl()
+    x, w, dy = make_inputs(M, K, N, seed=11)
+    g = run_step(x, w, dy)
+    check_all(g, oracle_step(x, w, dy), N)
+    bufs = bl.StepBuffers.allocate(M, N, K)
+    bl.bl_quantize_weight(w.cuda(), bufs.w_packed, bufs.gamma, bufs.workspace)
+    bl.bl_quantize_act(x.cuda(), bufs.xq, bufs.sx)
+    y2 = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    bl.bl_forward(bufs.xq, bufs.sx, bufs.w_packed, bufs.gamma, y2)
+    torch.cuda.synchronize()
+    assert bl.bl_get_last_error() == 0
+    np.testing.assert_array_equal(bits(y2), g["y_bits"])
+
+
 def _threshold_probe_weights(N=64, K=128, f32=True, seed=0):
     """Weights whose magnitudes crowd around gamma / 2.
 
