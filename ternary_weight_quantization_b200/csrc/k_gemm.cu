@@ -121,7 +121,10 @@ struct Geo;
 // Forward: reduction over k in blocks of 128 bytes; kind::i8 consumes 32 k per MMA.
 template <int BN>
 struct Geo<Family::Fwd, BN> {
-  static constexpr int kEpiSlots = 4;
+  // 320-column tiles: two staging slots per epilogue warp leave room for a
+  // fifth pipeline stage (four with four slots); measured on B200 at the
+  // down-projection 35.5 -> 33.7 us
+  static constexpr int kEpiSlots = BN > 256 ? 2 : 4;
   static constexpr int kEpiScaleBytes = (BN > 256 ? BN : 256) * 4;  // s_x[m] * gamma of the tile's columns
   static constexpr int kBlockR = 128;
   static constexpr int kABytes = BM * 128;         // 128 rows x 128 int8
